@@ -1,0 +1,236 @@
+"""Python access to the SharQ CPU oracle (oracle/sharq_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's
+CPU-baseline leg use it. The CUDA path never imports this package.
+
+Every function takes and returns numpy arrays in the oracle's canonical
+layouts (one code per byte, row-major scales, ascending kept indices).
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import build as _build
+
+NVFP4, MXFP4 = 0, 1
+BLOCK = {NVFP4: 16, MXFP4: 32}
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = C.CDLL(_build.build())
+        _declare(_lib)
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def _declare(L):
+    vp, i64, f32, i32 = C.c_void_p, C.c_int64, C.c_float, C.c_int
+    L.oracle_half_to_double.argtypes = [C.c_uint16]
+    L.oracle_half_to_double.restype = C.c_double
+    L.oracle_u128_to_double.argtypes = [C.c_uint64, C.c_uint64]
+    L.oracle_u128_to_double.restype = C.c_double
+    L.oracle_ln_stats.argtypes = [vp, i64, i64, f32, vp, vp]
+    L.oracle_ln_apply.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
+    L.oracle_e2m1_value.argtypes = [i32]
+    L.oracle_e2m1_value.restype = C.c_double
+    L.oracle_e2m1_encode.argtypes = [f32]
+    L.oracle_e2m1_encode.restype = i32
+    L.oracle_ue4m3_value.argtypes = [i32]
+    L.oracle_ue4m3_value.restype = C.c_double
+    L.oracle_ue4m3_encode.argtypes = [f32]
+    L.oracle_ue4m3_encode.restype = i32
+    L.oracle_mx_exponent.argtypes = [f32]
+    L.oracle_mx_exponent.restype = i32
+    L.oracle_quantize.argtypes = [vp, i64, i64, i32, f32, vp, vp]
+    L.oracle_tensor_scale.argtypes = [vp, i64, i32]
+    L.oracle_tensor_scale.restype = f32
+    L.oracle_mask.argtypes = [vp, i64, i64, i32, i32, vp, vp]
+    L.oracle_prepare.argtypes = [vp, i64, i64, vp, vp, f32, i32, i32, i32] + [vp] * 13
+    L.oracle_quantize_weight.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp]
+    L.oracle_linear.argtypes = [vp, vp, vp, vp, f32, vp, vp, f32, i64, i64, i64, i32, vp, vp]
+
+
+def _u16(a):
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float16:
+        a = a.view(np.uint16)
+    assert a.dtype == np.uint16
+    return a
+
+
+# ---------------------------------------------------------------------------
+# Scalar codecs
+
+
+def e2m1_encode(y: float) -> int:
+    return lib().oracle_e2m1_encode(float(y))
+
+
+def e2m1_value(code: int) -> float:
+    return lib().oracle_e2m1_value(int(code))
+
+
+def ue4m3_encode(u: float) -> int:
+    return lib().oracle_ue4m3_encode(float(u))
+
+
+def ue4m3_value(code: int) -> float:
+    return lib().oracle_ue4m3_value(int(code))
+
+
+def mx_exponent(a: float) -> int:
+    return lib().oracle_mx_exponent(float(a))
+
+
+def u128_to_double(v: int) -> float:
+    return lib().oracle_u128_to_double((v >> 64) & ((1 << 64) - 1), v & ((1 << 64) - 1))
+
+
+def half_to_double(h: int) -> float:
+    return lib().oracle_half_to_double(int(h))
+
+
+# ---------------------------------------------------------------------------
+# Array steps
+
+
+def ln_stats(x: np.ndarray, eps: float):
+    x = _u16(x)
+    rows, k = x.shape
+    mu = np.empty(rows, np.float32)
+    rstd = np.empty(rows, np.float32)
+    lib().oracle_ln_stats(_p(x), rows, k, eps, _p(mu), _p(rstd))
+    return mu, rstd
+
+
+def ln_apply(x, gamma, beta, mu, rstd):
+    x = _u16(x)
+    rows, k = x.shape
+    g = None if gamma is None else _u16(gamma)
+    b = None if beta is None else _u16(beta)
+    out = np.empty((rows, k), np.float32)
+    lib().oracle_ln_apply(_p(x), rows, k, _p(g), _p(b), _p(np.ascontiguousarray(mu, np.float32)),
+                          _p(np.ascontiguousarray(rstd, np.float32)), _p(out))
+    return out
+
+
+def tensor_scale(v: np.ndarray, fmt: int) -> np.float32:
+    v = np.ascontiguousarray(v, np.float32)
+    return np.float32(lib().oracle_tensor_scale(_p(v), v.size, fmt))
+
+
+def mask(x_ln: np.ndarray, n: int, m: int):
+    x_ln = np.ascontiguousarray(x_ln, np.float32)
+    rows, k = x_ln.shape
+    idx = np.empty((rows, k // m, n), np.uint8)
+    keep = np.empty((rows, k), np.uint8)
+    lib().oracle_mask(_p(x_ln), rows, k, n, m, _p(idx), _p(keep))
+    return idx, keep
+
+
+def quantize(v: np.ndarray, fmt: int, s_t: float):
+    v = np.ascontiguousarray(v, np.float32)
+    rows, k = v.shape
+    codes = np.empty((rows, k), np.uint8)
+    scales = np.empty((rows, k // BLOCK[fmt]), np.uint8)
+    lib().oracle_quantize(_p(v), rows, k, fmt, float(s_t), _p(codes), _p(scales))
+    return codes, scales
+
+
+@dataclass
+class Prepared:
+    mu: np.ndarray
+    rstd: np.ndarray
+    x_ln: np.ndarray
+    s: np.ndarray
+    deq_s: np.ndarray
+    r: np.ndarray
+    idx: np.ndarray
+    keep: np.ndarray
+    s_codes: np.ndarray
+    s_scales: np.ndarray
+    r_codes: np.ndarray
+    r_scales: np.ndarray
+    s_t: np.float32
+    fmt: int
+    n: int
+    m: int
+
+
+def prepare(x, gamma, beta, eps: float, n: int, m: int, fmt: int) -> Prepared:
+    x = _u16(x)
+    rows, k = x.shape
+    blk = BLOCK[fmt]
+    g = None if gamma is None else _u16(gamma)
+    b = None if beta is None else _u16(beta)
+    f = lambda: np.empty((rows, k), np.float32)
+    mu, rstd = np.empty(rows, np.float32), np.empty(rows, np.float32)
+    x_ln, s, deq_s, r = f(), f(), f(), f()
+    idx = np.empty((rows, k // m, n), np.uint8)
+    keep = np.empty((rows, k), np.uint8)
+    s_codes, r_codes = np.empty((rows, k), np.uint8), np.empty((rows, k), np.uint8)
+    s_scales = np.empty((rows, k // blk), np.uint8)
+    r_scales = np.empty((rows, k // blk), np.uint8)
+    s_t = np.empty(1, np.float32)
+    lib().oracle_prepare(_p(x), rows, k, _p(g), _p(b), eps, n, m, fmt,
+                         _p(mu), _p(rstd), _p(x_ln), _p(s), _p(deq_s), _p(r),
+                         _p(idx), _p(keep), _p(s_codes), _p(s_scales),
+                         _p(r_codes), _p(r_scales), _p(s_t))
+    return Prepared(mu, rstd, x_ln, s, deq_s, r, idx, keep, s_codes, s_scales,
+                    r_codes, r_scales, s_t[0], fmt, n, m)
+
+
+@dataclass
+class QWeight:
+    w_f32: np.ndarray
+    codes: np.ndarray
+    scales: np.ndarray
+    s_tw: np.float32
+    fmt: int
+
+
+def quantize_weight(w, fmt: int) -> QWeight:
+    w = _u16(w)
+    n_out, k = w.shape
+    w_f32 = np.empty((n_out, k), np.float32)
+    codes = np.empty((n_out, k), np.uint8)
+    scales = np.empty((n_out, k // BLOCK[fmt]), np.uint8)
+    s_tw = np.empty(1, np.float32)
+    lib().oracle_quantize_weight(_p(w), n_out, k, fmt, _p(w_f32), _p(codes), _p(scales), _p(s_tw))
+    return QWeight(w_f32, codes, scales, s_tw[0], fmt)
+
+
+def linear(s_codes, s_scales, r_codes, r_scales, s_t, w_codes, w_scales, s_tw, fmt,
+           want_bound: bool = True):
+    """fp64 dual-path output and its tolerance scale, for the given rows."""
+    s_codes = np.ascontiguousarray(s_codes, np.uint8)
+    r_codes = np.ascontiguousarray(r_codes, np.uint8)
+    s_scales = np.ascontiguousarray(s_scales, np.uint8)
+    r_scales = np.ascontiguousarray(r_scales, np.uint8)
+    w_codes = np.ascontiguousarray(w_codes, np.uint8)
+    w_scales = np.ascontiguousarray(w_scales, np.uint8)
+    rows, k = s_codes.shape
+    n_out = w_codes.shape[0]
+    out = np.empty((rows, n_out), np.float64)
+    bound = np.empty((rows, n_out), np.float64) if want_bound else None
+    lib().oracle_linear(_p(s_codes), _p(s_scales), _p(r_codes), _p(r_scales), float(s_t),
+                        _p(w_codes), _p(w_scales), float(s_tw), rows, n_out, k, fmt,
+                        _p(out), _p(bound))
+    return out, bound
+
+
+def linear_prepared(p: Prepared, qw: QWeight, rows=None):
+    """Dual-path output for a Prepared activation (optionally a row subset)."""
+    sel = slice(None) if rows is None else rows
+    return linear(p.s_codes[sel], p.s_scales[sel], p.r_codes[sel], p.r_scales[sel], p.s_t,
+                  qw.codes, qw.scales, qw.s_tw, p.fmt)

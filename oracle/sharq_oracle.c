@@ -1,0 +1,408 @@
+/*
+ * SharQ CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this file's library. The CUDA path
+ * never calls it, and it shares no code, header, table or helper with the
+ * CUDA path.
+ *
+ * What it computes comes from the SharQ abstract ("SharQ: Bridging Activation
+ * Sparsity and FP4 Quantization for LLM Inference", arXiv 2606.26587,
+ * Abstract): LayerNorm, an input-adaptive N:M mask that extracts an
+ * outlier-dominated sparse backbone S, FP4 quantization of S, a dense
+ * residual R = X_ln - deq(Q(S)) taken against the quantized backbone, FP4
+ * quantization of R, and two FP4 GEMMs against one shared FP4 weight payload
+ * whose outputs are summed. The abstract leaves the arithmetic open; each
+ * function below states the reading it implements.
+ *
+ * Formats: NVFP4 = E2M1 codes, one UE4M3 scale per 16 elements and one fp32
+ * tensor scale (NVIDIA's NVFP4 description); MXFP4 = E2M1 codes and one E8M0
+ * scale per 32 elements (OCP Microscaling Formats v1.0).
+ *
+ * Arithmetic: every float operation is one IEEE-754 binary32 (or binary64
+ * where stated) operation rounded to nearest even. Build with
+ * -ffp-contract=off so that no multiply-add is fused. Codecs are brute-force
+ * nearest-value searches over the format's value table, the plainest
+ * correct definition.
+ *
+ * Canonical layouts (row-major, one value per byte):
+ *   codes   [rows][k]        E2M1 code, bit 3 = sign, bits 0-2 = magnitude
+ *   scales  [rows][k / blk]  UE4M3 code (NVFP4) or E8M0 code (MXFP4)
+ *   idx     [rows][k / m][n] kept positions inside each M-group, ascending
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+typedef unsigned __int128 u128;
+typedef __int128 i128;
+
+#define FMT_NVFP4 0
+#define FMT_MXFP4 1
+
+/* ------------------------------------------------------------------ */
+/* fp16 decode (IEEE-754 binary16), exact in binary64.                 */
+
+double oracle_half_to_double(uint16_t h)
+{
+    int s = h >> 15, e = (h >> 10) & 31, f = h & 1023;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -24);
+    else if (e == 31)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(f + 1024), e - 25);
+    return s ? -v : v;
+}
+
+/* ------------------------------------------------------------------ */
+/* Correctly rounded (nearest, ties to even) binary64 value of a       */
+/* non-negative 128-bit integer, written as an integer routine.        */
+
+static double u128_to_double_rn(u128 v)
+{
+    if (v == 0)
+        return 0.0;
+    int p = 127;
+    while (!((v >> p) & 1))
+        --p;
+    if (p < 53)
+        return (double)(uint64_t)v;
+    int drop = p - 52; /* keep the top 53 bits */
+    u128 q = v >> drop;
+    u128 rem = v - (q << drop);
+    u128 half = (u128)1 << (drop - 1);
+    if (rem > half || (rem == half && (q & 1)))
+        q += 1; /* q <= 2^53: still exact */
+    return ldexp((double)(uint64_t)q, drop);
+}
+
+double oracle_u128_to_double(uint64_t hi, uint64_t lo)
+{
+    return u128_to_double_rn(((u128)hi << 64) | lo);
+}
+
+/* ------------------------------------------------------------------ */
+/* LayerNorm statistics, exactly (reading: the abstract names "layer   */
+/* normalization" inside the fused preparation operator; it does not   */
+/* say how the statistics round, so they are defined from exact        */
+/* integer sums, which makes them independent of summation order).     */
+/*                                                                      */
+/*   a_i  = x_i * 2^24                  integer, |a_i| < 2^40          */
+/*   S1   = sum a_i,  S2 = sum a_i^2     exact                          */
+/*   D    = K*S2 - S1^2                  exact, >= 0                    */
+/*   mu   = RN32( RN64(S1) / (K*2^24) )                                 */
+/*   var  = RN64(D) / (K^2 * 2^48)        (binary64 division)           */
+/*   rstd = RN32( 1 / sqrt(var + eps) )   (binary64 sqrt and division)  */
+
+void oracle_ln_stats(const uint16_t *x, int64_t rows, int64_t k, float eps,
+                     float *mu, float *rstd)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t s1 = 0;
+        u128 s2 = 0;
+        for (int64_t i = 0; i < k; ++i) {
+            int64_t a = (int64_t)ldexp(oracle_half_to_double(x[r * k + i]), 24);
+            s1 += a;
+            s2 += (u128)((i128)a * (i128)a);
+        }
+        i128 d = (i128)k * (i128)s2 - (i128)s1 * (i128)s1;
+        double mean64 = (double)s1 / ((double)k * 16777216.0);
+        double var64 = u128_to_double_rn((u128)d) /
+                       ((double)k * (double)k * 281474976710656.0);
+        mu[r] = (float)mean64;
+        rstd[r] = (float)(1.0 / sqrt(var64 + (double)eps));
+    }
+}
+
+/* LayerNorm apply, left to right, each step rounded to binary32:       */
+/*   X_ln = RN32( RN32( RN32(x - mu) * rstd ) * gamma ) + beta           */
+/* gamma == NULL skips the multiply, beta == NULL skips the add.        */
+void oracle_ln_apply(const uint16_t *x, int64_t rows, int64_t k,
+                     const uint16_t *gamma, const uint16_t *beta,
+                     const float *mu, const float *rstd, float *x_ln)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t i = 0; i < k; ++i) {
+            float t = (float)oracle_half_to_double(x[r * k + i]) - mu[r];
+            t = t * rstd[r];
+            if (gamma)
+                t = t * (float)oracle_half_to_double(gamma[i]);
+            if (beta)
+                t = t + (float)oracle_half_to_double(beta[i]);
+            x_ln[r * k + i] = t;
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* Codecs.                                                              */
+
+static const double E2M1_GRID[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+/* E2M1 value of a code (bit 3 = sign). */
+double oracle_e2m1_value(int code)
+{
+    double v = E2M1_GRID[code & 7];
+    return (code & 8) ? -v : v;
+}
+
+/* E2M1 code of y: nearest magnitude on the grid, equal distances go to the
+ * even code, |y| beyond 6 gives 6 (saturating); the sign bit is y's sign, so
+ * a small negative y gives -0 (code 8). */
+int oracle_e2m1_encode(float y)
+{
+    double a = fabs((double)y);
+    int best = 0;
+    double bd = a;
+    for (int c = 1; c < 8; ++c) {
+        double dd = fabs(a - E2M1_GRID[c]);
+        if (dd < bd || (dd == bd && (c & 1) == 0)) {
+            best = c;
+            bd = dd;
+        }
+    }
+    return best | (signbit(y) ? 8 : 0);
+}
+
+/* UE4M3 value: e = code>>3 (bias 7), m = code&7; e == 0 is subnormal.
+ * Code 127 is NaN in E4M3 and is never produced. */
+double oracle_ue4m3_value(int code)
+{
+    int e = (code >> 3) & 15, m = code & 7;
+    return e == 0 ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10);
+}
+
+/* UE4M3 code of u >= 0: nearest finite value (0 .. 448), equal distances go
+ * to the even code; values above 448 give 448 (saturating). */
+int oracle_ue4m3_encode(float u)
+{
+    double a = (double)u;
+    int best = 0;
+    double bd = fabs(a);
+    for (int c = 1; c < 127; ++c) {
+        double dd = fabs(a - oracle_ue4m3_value(c));
+        if (dd < bd || (dd == bd && (c & 1) == 0)) {
+            best = c;
+            bd = dd;
+        }
+    }
+    return best;
+}
+
+/* E8M0 block exponent of OCP MX v1.0: for a block amax a > 0,
+ * e = floor(log2 a) - emax(E2M1), emax(E2M1) = 2, clamped to [-127, 127]. */
+int oracle_mx_exponent(float a)
+{
+    int ex;
+    frexp((double)a, &ex); /* a = f * 2^ex, f in [0.5, 1): floor(log2 a) = ex-1 */
+    int e = ex - 1 - 2;
+    if (e < -127)
+        e = -127;
+    if (e > 127)
+        e = 127;
+    return e;
+}
+
+/* ------------------------------------------------------------------ */
+/* Block quantization of one row of values (used for S, R and W).       */
+/*                                                                      */
+/* NVFP4, blocks of 16:  a = max|v|;  u = a / RN32(6 * s_t);             */
+/*   sb = UE4M3(u);  d = RN32(value(sb) * s_t);                          */
+/*   code = d == 0 ? +0 : E2M1(RN32(v / d)).                             */
+/* MXFP4, blocks of 32:  a == 0 gives scale code 0 and +0 codes;         */
+/*   else e = mx_exponent(a), scale code e + 127, d = 2^e,               */
+/*   code = E2M1(RN32(v / d)).                                           */
+/* The per-value division (not a multiply by a reciprocal) is the reading */
+/* of "quantizes it to FP4"; d doubles as the dequantization step.        */
+
+static void quantize_row(const float *v, int64_t k, int fmt, float s_t,
+                         uint8_t *codes, uint8_t *scales)
+{
+    int blk = fmt == FMT_NVFP4 ? 16 : 32;
+    for (int64_t b = 0; b < k / blk; ++b) {
+        const float *vb = v + b * blk;
+        float a = 0.0f;
+        for (int i = 0; i < blk; ++i)
+            if (fabsf(vb[i]) > a)
+                a = fabsf(vb[i]);
+        float d;
+        if (fmt == FMT_NVFP4) {
+            float six_st = 6.0f * s_t;
+            float u = a / six_st;
+            int sb = oracle_ue4m3_encode(u);
+            scales[b] = (uint8_t)sb;
+            d = (float)oracle_ue4m3_value(sb) * s_t;
+        } else {
+            if (a == 0.0f) {
+                scales[b] = 0;
+                d = 0.0f;
+            } else {
+                int e = oracle_mx_exponent(a);
+                scales[b] = (uint8_t)(e + 127);
+                d = (float)ldexp(1.0, e);
+            }
+        }
+        for (int i = 0; i < blk; ++i)
+            codes[b * blk + i] = d == 0.0f ? 0 : (uint8_t)oracle_e2m1_encode(vb[i] / d);
+    }
+}
+
+/* Dequantized value of one code with step d (RN32 product). */
+static float deq(int code, float d)
+{
+    return (float)oracle_e2m1_value(code) * d;
+}
+
+/* Step d of a block from its scale code. */
+static float block_step(int fmt, int scale_code, float s_t)
+{
+    if (fmt == FMT_NVFP4)
+        return (float)oracle_ue4m3_value(scale_code) * s_t;
+    return (float)ldexp(1.0, scale_code - 127);
+}
+
+void oracle_quantize(const float *v, int64_t rows, int64_t k, int fmt, float s_t,
+                     uint8_t *codes, uint8_t *scales)
+{
+    int blk = fmt == FMT_NVFP4 ? 16 : 32;
+    for (int64_t r = 0; r < rows; ++r)
+        quantize_row(v + r * k, k, fmt, s_t, codes + r * k, scales + r * (k / blk));
+}
+
+/* ------------------------------------------------------------------ */
+/* Tensor scale (reading: north-star "fp32 tensor scale" for NVFP4 is    */
+/* one dynamic scale per tensor from amax over the whole tensor:          */
+/* s_t = RN32(amax / 2688), 2688 = 448 * 6; s_t = 1 if amax == 0; MXFP4   */
+/* has no tensor scale, s_t = 1).                                         */
+
+float oracle_tensor_scale(const float *v, int64_t count, int fmt)
+{
+    if (fmt != FMT_NVFP4)
+        return 1.0f;
+    float a = 0.0f;
+    for (int64_t i = 0; i < count; ++i)
+        if (fabsf(v[i]) > a)
+            a = fabsf(v[i]);
+    return a == 0.0f ? 1.0f : a / 2688.0f;
+}
+
+/* ------------------------------------------------------------------ */
+/* N:M mask: in every row, in every aligned group of m consecutive       */
+/* values along K, keep the n largest |X_ln|; equal magnitudes go to the  */
+/* lower index (so -0 and +0 tie). Exactly n survivors per group.         */
+/* Writes the kept positions ascending, and a 0/1 keep map.               */
+
+void oracle_mask(const float *x_ln, int64_t rows, int64_t k, int n, int m,
+                 uint8_t *idx, uint8_t *keep)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t g = 0; g < k / m; ++g) {
+            const float *v = x_ln + r * k + g * m;
+            uint8_t taken[16] = {0};
+            for (int j = 0; j < n; ++j) { /* pick the j-th largest */
+                int best = -1;
+                for (int i = 0; i < m; ++i)
+                    if (!taken[i] && (best < 0 || fabsf(v[i]) > fabsf(v[best])))
+                        best = i;
+                taken[best] = 1;
+            }
+            int w = 0;
+            for (int i = 0; i < m; ++i) {
+                if (taken[i])
+                    idx[(r * (k / m) + g) * n + w++] = (uint8_t)i;
+                if (keep)
+                    keep[r * k + g * m + i] = taken[i];
+            }
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* The preparation operator, step by step in the abstract's order:       */
+/* LayerNorm -> N:M mask -> Q(S) -> R = X_ln - deq(Q(S)) -> Q(R).         */
+/* S is X_ln on survivors and +0 elsewhere; deq(Q(S)) is 0 off the mask;  */
+/* R = RN32(X_ln - deqS); Q(R) uses the same tensor scale as Q(S).        */
+/* Every output pointer may be NULL except the ones the caller needs;     */
+/* work buffers (x_ln, s, deq_s, r) must be rows*k floats when non-NULL,   */
+/* and are required.                                                      */
+
+void oracle_prepare(const uint16_t *x, int64_t rows, int64_t k,
+                    const uint16_t *gamma, const uint16_t *beta, float eps,
+                    int n, int m, int fmt,
+                    float *mu, float *rstd, float *x_ln, float *s, float *deq_s, float *r,
+                    uint8_t *idx, uint8_t *keep,
+                    uint8_t *s_codes, uint8_t *s_scales,
+                    uint8_t *r_codes, uint8_t *r_scales, float *s_t_out)
+{
+    int blk = fmt == FMT_NVFP4 ? 16 : 32;
+    oracle_ln_stats(x, rows, k, eps, mu, rstd);
+    oracle_ln_apply(x, rows, k, gamma, beta, mu, rstd, x_ln);
+    float s_t = oracle_tensor_scale(x_ln, rows * k, fmt);
+    *s_t_out = s_t;
+    oracle_mask(x_ln, rows, k, n, m, idx, keep);
+    for (int64_t i = 0; i < rows * k; ++i)
+        s[i] = keep[i] ? x_ln[i] : 0.0f;
+    oracle_quantize(s, rows, k, fmt, s_t, s_codes, s_scales);
+    for (int64_t row = 0; row < rows; ++row)
+        for (int64_t i = 0; i < k; ++i) {
+            int64_t e = row * k + i;
+            float d = block_step(fmt, s_scales[row * (k / blk) + i / blk], s_t);
+            deq_s[e] = keep[e] ? deq(s_codes[e], d) : 0.0f;
+            r[e] = x_ln[e] - deq_s[e];
+        }
+    oracle_quantize(r, rows, k, fmt, s_t, r_codes, r_scales);
+}
+
+/* Weight quantization: the same block quantizer along K on every row of  */
+/* W [n_out][k], with s_tW = RN32(amax(W) / 2688) (NVFP4) or 1 (MXFP4).   */
+/* One code payload serves both GEMM paths.                               */
+void oracle_quantize_weight(const uint16_t *w, int64_t n_out, int64_t k, int fmt,
+                            float *w_f32, uint8_t *codes, uint8_t *scales, float *s_tw)
+{
+    for (int64_t i = 0; i < n_out * k; ++i)
+        w_f32[i] = (float)oracle_half_to_double(w[i]);
+    *s_tw = oracle_tensor_scale(w_f32, n_out * k, fmt);
+    oracle_quantize(w_f32, n_out, k, fmt, *s_tw, codes, scales);
+}
+
+/* Dequantized value of element (row, i) in the factored form the GEMM uses:
+ * value(code) * value(scale), without the tensor scale. Exact in binary64. */
+static double block_value(int fmt, const uint8_t *codes, const uint8_t *scales,
+                          int64_t k, int64_t row, int64_t i)
+{
+    int blk = fmt == FMT_NVFP4 ? 16 : 32;
+    int sc = scales[row * (k / blk) + i / blk];
+    double sv = fmt == FMT_NVFP4 ? oracle_ue4m3_value(sc) : ldexp(1.0, sc - 127);
+    return oracle_e2m1_value(codes[row * k + i]) * sv;
+}
+
+/* Dual-path linear: the backbone GEMM on Q(S) and the residual GEMM on    */
+/* Q(R) against the same Q(W), summed (abstract: "A sparse FP4 GEMM        */
+/* processes the backbone while a dense FP4 GEMM compensates"):             */
+/*   out[i][j] = s_t * s_tW * sum_k (aS[i][k] + aR[i][k]) * w[j][k]         */
+/* with a, w the block-scaled code values, in binary64 (every product is    */
+/* exact; only the sum rounds). bound[i][j] is the same sum over absolute   */
+/* values, the scale of the acceptance tolerance. Either may be NULL.       */
+void oracle_linear(const uint8_t *s_codes, const uint8_t *s_scales,
+                   const uint8_t *r_codes, const uint8_t *r_scales, float s_t,
+                   const uint8_t *w_codes, const uint8_t *w_scales, float s_tw,
+                   int64_t rows, int64_t n_out, int64_t k, int fmt,
+                   double *out, double *bound)
+{
+    double ts = (double)s_t * (double)s_tw;
+    for (int64_t i = 0; i < rows; ++i)
+        for (int64_t j = 0; j < n_out; ++j) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t q = 0; q < k; ++q) {
+                double a_s = block_value(fmt, s_codes, s_scales, k, i, q);
+                double a_r = block_value(fmt, r_codes, r_scales, k, i, q);
+                double w = block_value(fmt, w_codes, w_scales, k, j, q);
+                acc += a_s * w + a_r * w;
+                mag += fabs(a_s) * fabs(w) + fabs(a_r) * fabs(w);
+            }
+            if (out)
+                out[i * n_out + j] = ts * acc;
+            if (bound)
+                bound[i * n_out + j] = ts * mag;
+        }
+}

@@ -1,0 +1,50 @@
+"""The seeded generators are deterministic and draw the stated distributions."""
+import numpy as np
+
+import synth
+
+
+def test_splitmix64_reference_values():
+    # splitmix64 with state 0: the first outputs of the published generator
+    # (state += golden; mix) are these constants.
+    z = synth._mix64(np.array([0x9E3779B97F4A7C15, 0x3C6EF372FE94F82A], dtype=np.uint64))
+    assert int(z[0]) == 0xE220A8397B1DCDAF
+    assert int(z[1]) == 0x6E789E6AA1B965F4
+
+
+def test_deterministic_and_seed_sensitive():
+    a = synth.activations_student(3, 4, 256)
+    b = synth.activations_student(3, 4, 256)
+    c = synth.activations_student(4, 4, 256)
+    assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+    assert not np.array_equal(a, c)
+
+
+def test_normal_moments():
+    z = synth.normal(0, synth.S_BODY, 200000)
+    assert abs(z.mean()) < 0.01 and abs(z.std() - 1) < 0.01
+
+
+def test_outlier_channels():
+    x = synth.activations_gaussian(0, 64, 256, 4, 50.0).astype(np.float64)
+    std = x.std(0)
+    big = np.sort(np.argsort(-std)[:4])
+    assert np.all(std[big] > 20) and np.median(std) < 2
+    assert np.array_equal(big, np.sort(synth.permutation(0, synth.S_OUTLIER_PICK, 256)[:4]))
+
+
+def test_student_outliers_fraction():
+    x = synth.activations_student(1, 32, 4096)
+    n_out = int(np.ceil(0.01 * 4096))
+    med = np.median(np.abs(x.astype(np.float64)), axis=0)
+    assert (med > 10).sum() == n_out
+
+
+def test_moe_routing_shapes():
+    row_idx, off = synth.moe_routing(2, 64, 16, 4)
+    assert off[-1] == 64 * 4 and len(row_idx) == 64 * 4
+    for e in range(16):
+        seg = row_idx[off[e]:off[e + 1]]
+        assert np.all(np.diff(seg) > 0)
+    counts = np.bincount(row_idx, minlength=64)
+    assert np.all(counts == 4)
