@@ -1,0 +1,448 @@
+#!/usr/bin/env python
+"""Benchmark of the SharQ per-linear-layer hot path on B200.
+
+One step = the whole hot path over one batch: the 4 preparation operators and
+the 7 dual-path FP4 linears of a Llama-3.1-8B-shaped layer set
+(q/k/v share one prep, gate/up share one prep) on M tokens, NVFP4, 2:4.
+Inputs are seeded synthetic Student-t(3) activations with 1% outlier channels
+scaled x20..100 and N(0, 0.02^2) weights (quantized offline, outside the
+timed region), resident in HBM. L2 is flushed (256 MB write) before every
+timed step; each step is timed with CUDA events on the launching stream.
+
+Prints ONE JSON line (rank 0). Multi-GPU: one process per GPU (torchrun),
+each rank runs its own replica of the workload (the path has no exchange
+step), value = all ranks' tokens / the max over ranks of the timed region.
+
+--impl reference times the CPU oracle (oracle/) on a bounded sample of the
+same workload, as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "SharQ linear tokens/s & FP4 TFLOPS (% tensor peak), prep GB/s (% HBM)"
+UNIT = "tokens/s"
+EPS = 1e-5
+N_KEEP, M_GROUP = 2, 4
+FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
+PREP_BYTES_PER_ELEM = 3.25  # x 2 + S codes 0.5 + mask metadata 0.125 + S scales 0.0625 + R codes 0.5 + R scales 0.0625
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["sharq", "reference"], default="sharq")
+    ap.add_argument("--tokens", type=int, default=8192, help="M: tokens per step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-sample-tokens", type=int, default=1)
+    ap.add_argument("--cpu-sample-cols", type=int, default=512,
+                    help="output columns of each linear in the CPU sample (cost is linear in columns)")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(tokens):
+    return (f"Llama-3.1-8B layer set (q/k/v 4096->4096/1024/1024, o 4096->4096, gate/up 4096->14336, "
+            f"down 14336->4096): 4 preps + 7 dual-path linears, M={tokens} tokens, NVFP4, 2:4")
+
+
+def layer_set():
+    ls = synth.LLAMA31_8B
+    preps = list(ls.preps)
+    return ls, preps
+
+
+def flops_algorithmic(tokens):
+    ls, _ = layer_set()
+    return sum(2.0 * tokens * l.n_out * l.k * (1.0 + N_KEEP / M_GROUP) for l in ls.linears)
+
+
+def flops_executed(tokens):
+    ls, _ = layer_set()
+    return sum(4.0 * tokens * l.n_out * l.k for l in ls.linears)  # both paths run dense FP4 MMAs
+
+
+def prep_bytes_algorithmic(tokens):
+    _, preps = layer_set()
+    return sum(PREP_BYTES_PER_ELEM * tokens * k for _, k in preps)
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu_index = gpu_index
+        self.path = os.path.join(ROOT, "gpurun_out" if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ".",
+                                 f".clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-lms", "50", "-i", str(self.gpu_index)], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self, t_start: float, t_end: float):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].isdigit():
+                    rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [int(r[1]) for r in rows]
+        loaded = [r for r in rows if r[3] not in ("[N/A]",) and _float(r[3]) > 200.0] or rows
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in loaded:
+            for name, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": float(statistics.median(int(r[1]) for r in loaded)), "sm_max_mhz": float(max(int(r[2]) for r in rows)),
+                "reasons": sorted(reasons), "samples": len(loaded), "sm_mhz_min": min(sm)}
+
+
+def _float(s):
+    try:
+        return float(s)
+    except ValueError:
+        return 0.0
+
+
+# ---------------------------------------------------------------------------
+# Distributed plumbing
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "sharq" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# The CUDA path
+
+
+def run_sharq(args, world, rank, local):
+    import sparsity_gemm_b200 as sq
+    from sparsity_gemm_b200 import build as lib_build
+    if not os.path.exists(sq.LIB_PATH):
+        lib_build.build()
+    sq.lib()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    M = args.tokens
+    ls, preps = layer_set()
+    prep_index = {name: i for i, (name, _) in enumerate(preps)}
+
+    # Inputs: seeded synthetic activations and weights, resident in HBM.
+    xs_host = [torch.from_numpy(synth.activations_student(i, M, k).view(np.float16)) for i, (_, k) in enumerate(preps)]
+    xs = [t.to(dev) for t in xs_host]
+    qws = []
+    for j, lin in enumerate(ls.linears):
+        w = torch.from_numpy(synth.weights(1000 + j, lin.n_out, lin.k).view(np.float16)).to(dev)
+        qws.append(sq.quantize_weight(w, sq.NVFP4))
+        del w
+    prep_bufs = [sq.prepare(xs[i], None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4) for i in range(len(preps))]
+    outs = [torch.empty((M, lin.n_out), dtype=torch.float16, device=dev) for lin in ls.linears]
+    torch.cuda.synchronize()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    launches = [0]
+
+    def step(x_list, ev=None):
+        for i in range(len(preps)):
+            prep_bufs[i] = sq.prepare(x_list[i], None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4, out=prep_bufs[i])
+            launches[0] += sq.last_launch_count()
+            if ev is not None:
+                ev[1 + i].record(stream)
+        for j, lin in enumerate(ls.linears):
+            sq.linear(prep_bufs[prep_index[lin.prep]], qws[j], out=outs[j])
+            launches[0] += sq.last_launch_count()
+            if ev is not None:
+                ev[1 + len(preps) + j].record(stream)
+
+    n_ev = 1 + len(preps) + len(ls.linears)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(xs)
+    torch.cuda.synchronize()
+    status = sq.get_last_error()
+    if status != sq.OK:
+        raise RuntimeError(f"device status after warm-up: {sq.status_name(status)}")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    launches[0] = 0
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        t0 = time.time()
+        for s in range(args.steps):
+            flush.zero_()
+            events[s][0].record(stream)
+            step(xs, events[s])
+        torch.cuda.synchronize()
+        t1 = time.time()
+    barrier(world)
+    status = sq.get_last_error()
+    if status != sq.OK:
+        raise RuntimeError(f"device status after timing: {sq.status_name(status)}")
+
+    prep_ms = gemm_ms = 0.0
+    gemm_each = np.zeros(len(ls.linears))
+    for ev in events:
+        for i in range(len(preps)):
+            prep_ms += ev[i].elapsed_time(ev[i + 1])
+        for j in range(len(ls.linears)):
+            d = ev[len(preps) + j].elapsed_time(ev[len(preps) + j + 1])
+            gemm_ms += d
+            gemm_each[j] += d
+    total_ms = prep_ms + gemm_ms
+    total_ms_max = max_over_ranks(total_ms, world, dev)
+    steps = args.steps
+    value = world * M * steps / (total_ms_max / 1e3)
+    gpu_launches = launches[0]
+
+    peaks, peak_src = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    gemm_alg_tflops = flops_algorithmic(M) * steps / (gemm_ms / 1e3) / 1e12
+    gemm_exec_tflops = flops_executed(M) * steps / (gemm_ms / 1e3) / 1e12
+    prep_gbs = prep_bytes_algorithmic(M) * steps / (prep_ms / 1e3) / 1e9
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": total_ms_max / steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 + ue4m3/16 + fp32 tensor scale), fp32 accumulate",
+        "data": "synthetic (seeded Student-t(3) activations, 1% outlier channels x20-100; N(0,0.02^2) weights)",
+        "config": {"workload": workload_desc(M), "tokens": M, "fmt": "nvfp4", "nm": f"{N_KEEP}:{M_GROUP}",
+                   "layernorm": "gamma/beta NULL", "l2": "flushed (256 MB write) before every timed step",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "tensor", "kernel": "dual_gemm_kernel (7 linears)",
+                     "achieved": gemm_alg_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": gemm_alg_tflops / fp4_peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 {peaks['bf16_tflops']} TF/s x {FP4_OVER_BF16} (FP4/BF16 nominal)",
+                     "flops_per_step": flops_algorithmic(M), "flop_count": "2*M*N*K*(1+n/m)",
+                     "executed_tflops": gemm_exec_tflops, "executed_frac": gemm_exec_tflops / fp4_peak},
+        "prep_roofline": {"bound": "hbm", "kernel": "ln_stats_kernel + prep_encode_kernel (4 preps)",
+                          "achieved": prep_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": prep_gbs / peaks["hbm_gbs"], "bytes_per_elem": PREP_BYTES_PER_ELEM},
+        "split_ms_per_step": {"prep": prep_ms / steps, "gemm": gemm_ms / steps,
+                              "gemm_each": {lin.name: float(gemm_each[j] / steps) for j, lin in enumerate(ls.linears)}},
+        "gpu_launches": gpu_launches,
+        "wall_s_timed": t1 - t0,
+    }
+    cs = clocks.summary(t0, t1)
+    result["clocks"] = {"sm_mhz": cs.get("sm_mhz"), "sm_max_mhz": cs.get("sm_max_mhz"), "reasons": cs.get("reasons"),
+                        "samples": cs.get("samples")}
+
+    if not args.no_e2e:
+        result["e2e"] = e2e_sharq(args, sq, dev, stream, xs_host, preps, prep_bufs, qws, outs, ls, prep_index, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args)
+    return result
+
+
+def e2e_sharq(args, sq, dev, stream, xs_host, preps, prep_bufs, qws, outs, ls, prep_index, world):
+    """Same metric through the public API with host buffers: every step copies
+    its activations from pinned host memory and reads every output back."""
+    M = args.tokens
+    pinned_in = [t.pin_memory() for t in xs_host]
+    pinned_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
+    dev_in = [torch.empty_like(t, device=dev) for t in xs_host]
+    steps = max(3, min(args.steps, 20))
+
+    def one():
+        for i in range(len(preps)):
+            dev_in[i].copy_(pinned_in[i], non_blocking=True)
+        for i in range(len(preps)):
+            prep_bufs[i] = sq.prepare(dev_in[i], None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4, out=prep_bufs[i])
+        for j, lin in enumerate(ls.linears):
+            sq.linear(prep_bufs[prep_index[lin.prep]], qws[j], out=outs[j])
+        for j in range(len(outs)):
+            pinned_out[j].copy_(outs[j], non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    return {"value": world * M * steps / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": int(sum(t.numel() * 2 for t in xs_host)),
+            "d2h_bytes_per_step": int(sum(o.numel() * 2 for o in outs)), "steps": steps}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+
+
+def oracle_sample(tokens: int, cols: int):
+    """Builds the bounded CPU sample: `tokens` rows of each activation and the
+    first `cols` output columns of each linear (weights quantized up front)."""
+    import oracle
+    ls, preps = layer_set()
+    xs = [synth.activations_student(i, tokens, k) for i, (_, k) in enumerate(preps)]
+    ws = []
+    for j, lin in enumerate(ls.linears):
+        c = min(cols, lin.n_out)
+        ws.append(oracle.quantize_weight(synth.weights(1000 + j, c, lin.k), oracle.NVFP4))
+    return ls, preps, xs, ws
+
+
+def oracle_step(sample):
+    import oracle
+    ls, preps, xs, ws = sample
+    prepared = [oracle.prepare(x, None, None, EPS, N_KEEP, M_GROUP, oracle.NVFP4) for x in xs]
+    pidx = {name: i for i, (name, _) in enumerate(preps)}
+    for j, lin in enumerate(ls.linears):
+        oracle.linear_prepared(prepared[pidx[lin.prep]], ws[j])
+
+
+def token_fraction(sample, tokens):
+    """Token-equivalents of one sample step: the sample runs the full prep of
+    `tokens` rows but only a fraction of each linear's columns; the linears
+    dominate the oracle's cost, so weight them by their share of the MACs."""
+    ls, preps, xs, ws = sample
+    macs_full = sum(l.n_out * l.k for l in ls.linears)
+    macs_sample = sum(w.codes.shape[0] * l.k for w, l in zip(ws, ls.linears))
+    return tokens * macs_sample / macs_full
+
+
+def cpu_baseline(args):
+    sample = oracle_sample(args.cpu_sample_tokens, args.cpu_sample_cols)
+    t0 = time.perf_counter()
+    oracle_step(sample)
+    dt = time.perf_counter() - t0
+    tok = token_fraction(sample, args.cpu_sample_tokens)
+    return {"value": tok / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{args.cpu_sample_tokens} token(s): full prep of each activation row, and the first "
+                      f"{args.cpu_sample_cols} output columns of each linear (cost linear in columns; value = "
+                      f"{tok:.4f} token-equivalents / {dt:.2f} s), single-threaded C oracle"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    sample = oracle_sample(args.cpu_sample_tokens, args.cpu_sample_cols)
+    for _ in range(args.warmup):
+        oracle_step(sample)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(sample)
+        times.append(time.perf_counter() - t0)
+    tok = token_fraction(sample, args.cpu_sample_tokens)
+    total = sum(times)
+    value = tok * len(times) / total
+    desc = (f"{args.cpu_sample_tokens} token(s) per step: full prep of each activation row and the first "
+            f"{args.cpu_sample_cols} output columns of each linear ({tok:.4f} token-equivalents per step)")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 prep, f64 GEMM",
+            "data": "synthetic (same seeded generator)",
+            "config": {"workload": workload_desc(args.tokens), "tokens": args.tokens, "fmt": "nvfp4",
+                       "nm": f"{N_KEEP}:{M_GROUP}"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main():
+    args = parse_args()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, world, rank)
+        else:
+            res = run_sharq(args, world, rank, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

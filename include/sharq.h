@@ -1,0 +1,245 @@
+/*
+ * sharq.h - C ABI of the SharQ per-linear-layer hot path for NVIDIA B200
+ * (sm_100a).
+ *
+ * Method: "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM
+ * Inference" (arXiv 2606.26587), Abstract. For each activation tensor a
+ * fused preparation operator applies layer normalization, generates an
+ * input-adaptive N:M mask that extracts an outlier-dominated sparse backbone
+ * S, quantizes S to FP4, defines a dense residual R relative to the
+ * quantized backbone (R = X_ln - deq(Q(S))) and quantizes R to FP4. A sparse
+ * FP4 GEMM on the backbone and a dense FP4 GEMM on the residual read one
+ * shared FP4 weight payload through path-specific scale views, and their
+ * results are summed.
+ *
+ * Formats: SHARQ_NVFP4 = E2M1 codes, one UE4M3 scale per 16 elements and one
+ * fp32 tensor scale; SHARQ_MXFP4 = E2M1 codes and one E8M0 scale per 32
+ * elements (OCP Microscaling Formats v1.0).
+ *
+ * Conventions for every entry point:
+ *  - Pointers named *_dev are device pointers (cudaMalloc / torch CUDA
+ *    memory) of the current device; pointers named *_host are host memory.
+ *  - The caller owns all memory. The library never allocates device memory:
+ *    size queries say how many bytes a buffer needs, and handles
+ *    (sharq_wq, sharq_prep) are plain descriptors that point into the
+ *    caller's buffers. They stay valid as long as those buffers do.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream). All work is
+ *    enqueued asynchronously on it; only the *_export calls and
+ *    sharq_get_last_error synchronize it.
+ *  - Arguments are validated on the host before anything is enqueued; a
+ *    violation returns SHARQ_ERR_INVALID_ARG (or SHARQ_ERR_UNSUPPORTED) and
+ *    enqueues nothing. Device buffers must be 256-byte aligned.
+ *  - Inputs must be finite. Non-finite inputs are not detected and give
+ *    unspecified (but memory-safe) results.
+ *  - Kernels that wait on the hardware bound every wait; a wait that runs
+ *    out records a status that sharq_get_last_error reports as
+ *    SHARQ_ERR_TIMEOUT.
+ */
+#ifndef SHARQ_H
+#define SHARQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sharq_fmt {
+    SHARQ_NVFP4 = 0, /* E2M1 + UE4M3 scale per 16 + fp32 tensor scale */
+    SHARQ_MXFP4 = 1  /* E2M1 + E8M0 scale per 32 */
+} sharq_fmt;
+
+typedef enum sharq_status {
+    SHARQ_OK = 0,
+    SHARQ_ERR_INVALID_ARG = 1, /* a precondition below does not hold */
+    SHARQ_ERR_UNSUPPORTED = 2, /* valid request this build does not serve */
+    SHARQ_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+    SHARQ_ERR_TIMEOUT = 4      /* a bounded device-side wait ran out */
+} sharq_status;
+
+/* Shape limits. k must be a multiple of SHARQ_K_ALIGN (the GEMM's K tile)
+ * and at most SHARQ_K_MAX; n_out must be a multiple of SHARQ_N_ALIGN. */
+#define SHARQ_K_ALIGN 256
+#define SHARQ_K_MAX 65536
+#define SHARQ_N_ALIGN 32
+
+/*
+ * Block-scale layout ("MMA scale view"). Scales of a [rows][k/blk] matrix
+ * (blk = 16 for NVFP4, 32 for MXFP4) are stored in 512-byte atoms, each
+ * holding 4 consecutive scales of 128 consecutive rows. The scale of row r,
+ * block j is at byte
+ *     ((r / 128) * (k / blk / 4) + j / 4) * 512
+ *       + (r % 32) * 16 + ((r % 128) / 32) * 4 + (j % 4).
+ * This is the order in which a 32-lane x 128-bit tensor-memory copy
+ * delivers per-row scales to the block-scaled tcgen05 MMA. Rows are padded
+ * to a multiple of 128 (activations) or 256 (weights) with zero scales.
+ *
+ * Code layout: E2M1 codes packed two per byte, row-major [rows][k/2];
+ * element 2i in the low nibble, 2i+1 in the high nibble. Bit 3 of a code is
+ * its sign, so -0 (code 8) is kept distinct from +0 (code 0).
+ *
+ * Mask metadata layout: per row, for each aligned group of m elements along
+ * k, the n kept positions in ascending order, each ceil(log2 m) bits wide
+ * (m = 2: 1 bit), concatenated LSB-first into a bit stream of
+ * (k/m)*n*ceil(log2 m) bits; each row starts at a multiple of
+ * meta_row_bytes = ceil(that / 8) bytes.
+ */
+
+/* Quantized weight: one E2M1 code payload that both GEMM paths read. The
+ * backbone and the residual GEMM each see the scales through their own
+ * scale view (scales + tensor_scale); both views hold the same values, as
+ * the dequantized weight must be identical on both paths. */
+typedef struct sharq_wq {
+    int64_t n_out;       /* output features (rows of W) */
+    int64_t k;           /* input features */
+    int32_t fmt;         /* sharq_fmt */
+    int32_t reserved;
+    int64_t sf_rows;     /* rows of the scale layout: n_out rounded up to 256 */
+    void *codes;         /* device, [n_out][k/2] bytes */
+    void *scales_backbone; /* device, MMA scale view for the backbone path */
+    void *scales_residual; /* device, MMA scale view for the residual path */
+    float *tensor_scale; /* device, 1 float: s_tW = amax(W)/2688 (NVFP4) or 1 */
+    void *scratch;       /* device, library-internal words */
+} sharq_wq;
+
+/* Prepared activation: outputs of the preparation operator. */
+typedef struct sharq_prep {
+    int64_t m_tok;       /* rows (tokens) */
+    int64_t k;           /* input features */
+    int32_t n, m;        /* N:M ratio of the mask */
+    int32_t fmt;         /* sharq_fmt */
+    int32_t reserved;
+    int64_t sf_rows;     /* rows of the scale layouts: m_tok rounded up to 128 */
+    int64_t meta_row_bytes;
+    void *s_codes;       /* device, backbone Q(S) codes [m_tok][k/2] (zeros off the mask) */
+    void *r_codes;       /* device, residual Q(R) codes [m_tok][k/2] */
+    void *s_scales;      /* device, MMA scale view of Q(S) */
+    void *r_scales;      /* device, MMA scale view of Q(R) */
+    void *meta;          /* device, mask metadata [m_tok][meta_row_bytes] */
+    float *tensor_scale; /* device, 1 float: s_t = amax(X_ln)/2688 (NVFP4) or 1 */
+    void *scratch;       /* device, per-row statistics and reduction words */
+} sharq_prep;
+
+/* Bytes of the device buffer sharq_quantize_weight needs. 0 if the shape or
+ * format is invalid. */
+size_t sharq_weight_bytes(int64_t n_out, int64_t k, int fmt);
+
+/* Bytes of the device buffer sharq_prepare needs. 0 if invalid. */
+size_t sharq_prep_bytes(int64_t m_tok, int64_t k, int n, int m, int fmt);
+
+/*
+ * Weight quantization (offline). Abstract: "The two paths share a single FP4
+ * weight payload with path-specific scale views."
+ *   w_dev    fp16 [n_out][k] row-major (K-major), so the layer computes X W^T.
+ *   wq_dev   device buffer of at least sharq_weight_bytes(n_out, k, fmt).
+ *   wq_out   host struct, filled with pointers into wq_dev.
+ * NVFP4: s_tW = RN32(amax|W| / 2688) (1 if W == 0); each 16-element block
+ * gets UE4M3 scale RN-satfinite(amax_blk / RN32(6 s_tW)) and codes
+ * E2M1(RN32(w / RN32(scale * s_tW))). MXFP4: E8M0 exponent
+ * floor(log2 amax_blk) - 2 per 32-element block and codes E2M1(w / 2^e).
+ * Preconditions: n_out >= 1, n_out % SHARQ_N_ALIGN == 0, k % SHARQ_K_ALIGN
+ * == 0, 0 < k <= SHARQ_K_MAX, fmt valid, pointers non-NULL and aligned.
+ */
+sharq_status sharq_quantize_weight(const void *w_dev, int64_t n_out, int64_t k, int fmt,
+                                   void *wq_dev, size_t wq_bytes, sharq_wq *wq_out,
+                                   void *stream);
+
+/*
+ * Fused preparation operator (per activation). Abstract: "a fused
+ * preparation kernel absorbs mask generation, residual construction, and
+ * layer normalization into one operator."
+ *   x_dev     fp16 [m_tok][k] row-major activations.
+ *   ln_w_dev  fp16 [k] LayerNorm gamma, or NULL (no multiply).
+ *   ln_b_dev  fp16 [k] LayerNorm beta, or NULL (no add; -0 is preserved).
+ *   eps       LayerNorm epsilon, finite and > 0.
+ *   n, m      keep the n largest |X_ln| of every aligned group of m along k
+ *             (equal magnitudes: lower index first); m in {2,4,8,16},
+ *             1 <= n <= m.
+ *   prep_dev  device buffer of at least sharq_prep_bytes(...).
+ *   prep_out  host struct, filled with pointers into prep_dev.
+ * Steps, each an IEEE binary32 operation rounded to nearest even:
+ *   LayerNorm with statistics from exact integer sums: mu = RN32(S1/K),
+ *   rstd = RN32(1/sqrt(var + eps)) in binary64 from D = K*S2 - S1^2;
+ *   X_ln = RN32(RN32(RN32(x - mu) * rstd) * gamma) + beta;
+ *   s_t = RN32(amax|X_ln| / 2688) (1 if zero; MXFP4: 1);
+ *   S = X_ln on the mask, +0 elsewhere; Q(S) block-quantized as for weights;
+ *   R = RN32(X_ln - deq(Q(S))), deq = RN32(E2M1 value * RN32(scale * s_t));
+ *   Q(R) block-quantized with the same s_t.
+ * m_tok == 0 is valid and enqueues nothing but the tensor scale (1).
+ */
+sharq_status sharq_prepare(const void *x_dev, int64_t m_tok, int64_t k,
+                           const void *ln_w_dev, const void *ln_b_dev, float eps,
+                           int n, int m, int fmt,
+                           void *prep_dev, size_t prep_bytes, sharq_prep *prep_out,
+                           void *stream);
+
+/*
+ * Dual-path FP4 linear layer. Abstract: "A sparse FP4 GEMM processes the
+ * backbone while a dense FP4 GEMM compensates for both mask-induced
+ * activation loss and sparse-path quantization error."
+ *   out_dev  fp16 [m_tok][n_out] row-major:
+ *     out = RN16( s_t * s_tW * sum_k (Q(S) + Q(R))[i,k] * Q(W)[j,k] )
+ *   with the block-scaled code values; products are exact, accumulation is
+ *   fp32 in tensor memory (both paths into one accumulator).
+ * Preconditions: prep and wq from this library, prep->fmt == wq->fmt,
+ * prep->k == wq->k, out_dev non-NULL (may be NULL only if m_tok == 0).
+ */
+sharq_status sharq_linear(const sharq_prep *prep, const sharq_wq *wq, void *out_dev,
+                          void *stream);
+
+/*
+ * Canonical host copies of a prepared activation, for inspection and tests.
+ * Synchronizes `stream`. Every output may be NULL. One value per byte:
+ *   idx_host      [m_tok][k/m][n] kept positions, ascending
+ *   s_codes_host  [m_tok][k]      Q(S) codes (0..15)
+ *   s_scales_host [m_tok][k/blk]  Q(S) scale codes
+ *   r_codes_host, r_scales_host   same for Q(R)
+ *   mu_host, rstd_host [m_tok]    LayerNorm statistics (float)
+ *   s_t_host      1 float
+ */
+sharq_status sharq_prep_export(const sharq_prep *prep, uint8_t *idx_host,
+                               uint8_t *s_codes_host, uint8_t *s_scales_host,
+                               uint8_t *r_codes_host, uint8_t *r_scales_host,
+                               float *mu_host, float *rstd_host, float *s_t_host,
+                               void *stream);
+
+/* Canonical host copies of a quantized weight. Synchronizes `stream`.
+ *   codes_host [n_out][k], scales_host [n_out][k/blk] (backbone view),
+ *   scales_residual_host [n_out][k/blk] (residual view), s_tw_host 1 float. */
+sharq_status sharq_weight_export(const sharq_wq *wq, uint8_t *codes_host,
+                                 uint8_t *scales_host, uint8_t *scales_residual_host,
+                                 float *s_tw_host, void *stream);
+
+/* Synchronizes `stream`, then reports (and clears) the device status word:
+ * SHARQ_ERR_TIMEOUT if a bounded wait ran out since the last call,
+ * SHARQ_ERR_CUDA if the stream holds a CUDA error, else SHARQ_OK. */
+sharq_status sharq_get_last_error(void *stream);
+
+/* Where the last SHARQ_ERR_TIMEOUT came from (an internal site code), 0 if
+ * none. Valid after sharq_get_last_error returned SHARQ_ERR_TIMEOUT. */
+uint32_t sharq_last_timeout_site(void);
+
+/* Test hook: the wait limit of the GEMM's bounded waits, in nanoseconds
+ * (default 2e9). 0 restores the default. Returns the previous value. */
+uint64_t sharq_set_wait_limit_ns(uint64_t ns);
+
+/* Failure-detection self-test: enqueues one CTA whose single thread waits,
+ * with the library's bounded wait, on a barrier that nothing ever arrives
+ * at. After limit_ns (1 .. 1e10) the wait gives up and records site 0x1FF;
+ * the kernel returns normally and the context stays usable. A following
+ * sharq_get_last_error must report SHARQ_ERR_TIMEOUT. */
+sharq_status sharq_selftest_wait(uint64_t limit_ns, void *stream);
+
+/* Human-readable status name (static string). */
+const char *sharq_status_string(sharq_status s);
+
+/* Number of kernel launches the last entry point enqueued (for launch
+ * accounting in benchmarks). */
+int sharq_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SHARQ_H */

@@ -55,7 +55,7 @@ def _declare(L):
     L.oracle_tensor_scale.argtypes = [vp, i64, i32]
     L.oracle_tensor_scale.restype = f32
     L.oracle_mask.argtypes = [vp, i64, i64, i32, i32, vp, vp]
-    L.oracle_prepare.argtypes = [vp, i64, i64, vp, vp, f32, i32, i32, i32] + [vp] * 13
+    L.oracle_prepare.argtypes = [vp, i64, i64, vp, vp, f32, i32, i32, i32] + [vp] * 14
     L.oracle_quantize_weight.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp]
     L.oracle_linear.argtypes = [vp, vp, vp, vp, f32, vp, vp, f32, i64, i64, i64, i32, vp, vp]
 
@@ -167,7 +167,10 @@ class Prepared:
     m: int
 
 
-def prepare(x, gamma, beta, eps: float, n: int, m: int, fmt: int) -> Prepared:
+def prepare(x, gamma, beta, eps: float, n: int, m: int, fmt: int, s_t=None) -> Prepared:
+    """The preparation operator on the rows of x. s_t=None derives the
+    tensor scale from these rows; a given s_t (the scale of a larger tensor
+    these rows were sampled from) is used as is."""
     x = _u16(x)
     rows, k = x.shape
     blk = BLOCK[fmt]
@@ -181,11 +184,13 @@ def prepare(x, gamma, beta, eps: float, n: int, m: int, fmt: int) -> Prepared:
     s_codes, r_codes = np.empty((rows, k), np.uint8), np.empty((rows, k), np.uint8)
     s_scales = np.empty((rows, k // blk), np.uint8)
     r_scales = np.empty((rows, k // blk), np.uint8)
-    s_t = np.empty(1, np.float32)
+    s_t_arr = np.empty(1, np.float32)
+    s_t_in = None if s_t is None else np.array([s_t], np.float32)
     lib().oracle_prepare(_p(x), rows, k, _p(g), _p(b), eps, n, m, fmt,
                          _p(mu), _p(rstd), _p(x_ln), _p(s), _p(deq_s), _p(r),
                          _p(idx), _p(keep), _p(s_codes), _p(s_scales),
-                         _p(r_codes), _p(r_scales), _p(s_t))
+                         _p(r_codes), _p(r_scales), _p(s_t_arr), _p(s_t_in))
+    s_t = s_t_arr
     return Prepared(mu, rstd, x_ln, s, deq_s, r, idx, keep, s_codes, s_scales,
                     r_codes, r_scales, s_t[0], fmt, n, m)
 
@@ -197,6 +202,23 @@ class QWeight:
     scales: np.ndarray
     s_tw: np.float32
     fmt: int
+
+
+def tensor_scale_of(x, gamma, beta, eps: float, fmt: int) -> np.float32:
+    """The activation tensor scale over all rows of x (LayerNorm, then
+    amax), computed in row chunks to bound memory."""
+    x = _u16(x)
+    rows = x.shape[0]
+    amax = np.float32(0.0)
+    step = max(1, (1 << 24) // max(1, x.shape[1]))
+    for r0 in range(0, rows, step):
+        xs = x[r0:r0 + step]
+        mu, rstd = ln_stats(xs, eps)
+        xl = ln_apply(xs, gamma, beta, mu, rstd)
+        amax = max(amax, np.abs(xl).max() if xl.size else np.float32(0))
+    if fmt != NVFP4:
+        return np.float32(1.0)
+    return tensor_scale(np.array([amax], np.float32), fmt)
 
 
 def quantize_weight(w, fmt: int) -> QWeight:

@@ -322,9 +322,11 @@ void oracle_mask(const float *x_ln, int64_t rows, int64_t k, int n, int m,
 /* LayerNorm -> N:M mask -> Q(S) -> R = X_ln - deq(Q(S)) -> Q(R).         */
 /* S is X_ln on survivors and +0 elsewhere; deq(Q(S)) is 0 off the mask;  */
 /* R = RN32(X_ln - deqS); Q(R) uses the same tensor scale as Q(S).        */
-/* Every output pointer may be NULL except the ones the caller needs;     */
-/* work buffers (x_ln, s, deq_s, r) must be rows*k floats when non-NULL,   */
-/* and are required.                                                      */
+/* All arrays are required (rows*k floats / bytes as named).               */
+/* s_t_in: NULL computes the tensor scale from these rows; otherwise the   */
+/* given value is used, so that a sample of rows of a larger tensor can be */
+/* prepared with that tensor's scale (the per-row steps do not depend on   */
+/* other rows).                                                            */
 
 void oracle_prepare(const uint16_t *x, int64_t rows, int64_t k,
                     const uint16_t *gamma, const uint16_t *beta, float eps,
@@ -332,12 +334,12 @@ void oracle_prepare(const uint16_t *x, int64_t rows, int64_t k,
                     float *mu, float *rstd, float *x_ln, float *s, float *deq_s, float *r,
                     uint8_t *idx, uint8_t *keep,
                     uint8_t *s_codes, uint8_t *s_scales,
-                    uint8_t *r_codes, uint8_t *r_scales, float *s_t_out)
+                    uint8_t *r_codes, uint8_t *r_scales, float *s_t_out, const float *s_t_in)
 {
     int blk = fmt == FMT_NVFP4 ? 16 : 32;
     oracle_ln_stats(x, rows, k, eps, mu, rstd);
     oracle_ln_apply(x, rows, k, gamma, beta, mu, rstd, x_ln);
-    float s_t = oracle_tensor_scale(x_ln, rows * k, fmt);
+    float s_t = s_t_in ? *s_t_in : oracle_tensor_scale(x_ln, rows * k, fmt);
     *s_t_out = s_t;
     oracle_mask(x_ln, rows, k, n, m, idx, keep);
     for (int64_t i = 0; i < rows * k; ++i)

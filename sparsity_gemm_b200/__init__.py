@@ -1,0 +1,235 @@
+"""SharQ per-linear-layer hot path on NVIDIA B200 (sm_100a).
+
+A thin binding over the C ABI of libsharq.so (include/sharq.h): it allocates
+caller-owned buffers with torch, passes raw device pointers and the current
+CUDA stream, and checks status codes. Every step of the path runs in the
+library's CUDA kernels; there is no CPU or PyTorch fallback, and importing
+the package fails loudly when the library is missing.
+
+Method: "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM
+Inference" (arXiv 2606.26587), Abstract.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsharq.so")
+
+NVFP4, MXFP4 = 0, 1
+BLOCK = {NVFP4: 16, MXFP4: 32}
+K_ALIGN, K_MAX, N_ALIGN = 256, 65536, 32
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+
+
+class SharqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_name(status)}")
+        self.status = status
+
+
+class SharqWQ(C.Structure):
+    _fields_ = [("n_out", C.c_int64), ("k", C.c_int64), ("fmt", C.c_int32), ("reserved", C.c_int32),
+                ("sf_rows", C.c_int64), ("codes", C.c_void_p), ("scales_backbone", C.c_void_p),
+                ("scales_residual", C.c_void_p), ("tensor_scale", C.c_void_p), ("scratch", C.c_void_p)]
+
+
+class SharqPrep(C.Structure):
+    _fields_ = [("m_tok", C.c_int64), ("k", C.c_int64), ("n", C.c_int32), ("m", C.c_int32),
+                ("fmt", C.c_int32), ("reserved", C.c_int32), ("sf_rows", C.c_int64),
+                ("meta_row_bytes", C.c_int64), ("s_codes", C.c_void_p), ("r_codes", C.c_void_p),
+                ("s_scales", C.c_void_p), ("r_scales", C.c_void_p), ("meta", C.c_void_p),
+                ("tensor_scale", C.c_void_p), ("scratch", C.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded libsharq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m sparsity_gemm_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        vp, i64, i32, f32, sz = C.c_void_p, C.c_int64, C.c_int, C.c_float, C.c_size_t
+        L.sharq_weight_bytes.argtypes = [i64, i64, i32]
+        L.sharq_weight_bytes.restype = sz
+        L.sharq_prep_bytes.argtypes = [i64, i64, i32, i32, i32]
+        L.sharq_prep_bytes.restype = sz
+        L.sharq_quantize_weight.argtypes = [vp, i64, i64, i32, vp, sz, C.POINTER(SharqWQ), vp]
+        L.sharq_prepare.argtypes = [vp, i64, i64, vp, vp, f32, i32, i32, i32, vp, sz, C.POINTER(SharqPrep), vp]
+        L.sharq_linear.argtypes = [C.POINTER(SharqPrep), C.POINTER(SharqWQ), vp, vp]
+        L.sharq_prep_export.argtypes = [C.POINTER(SharqPrep)] + [vp] * 8 + [vp]
+        L.sharq_weight_export.argtypes = [C.POINTER(SharqWQ), vp, vp, vp, vp, vp]
+        L.sharq_get_last_error.argtypes = [vp]
+        L.sharq_last_timeout_site.restype = C.c_uint32
+        L.sharq_set_wait_limit_ns.argtypes = [C.c_uint64]
+        L.sharq_set_wait_limit_ns.restype = C.c_uint64
+        L.sharq_selftest_wait.argtypes = [C.c_uint64, vp]
+        L.sharq_selftest_wait.restype = i32
+        L.sharq_status_string.argtypes = [i32]
+        L.sharq_status_string.restype = C.c_char_p
+        L.sharq_last_launch_count.restype = i32
+        for name in ("sharq_quantize_weight", "sharq_prepare", "sharq_linear", "sharq_prep_export",
+                     "sharq_weight_export", "sharq_get_last_error"):
+            getattr(L, name).restype = i32
+        _lib = L
+    return _lib
+
+
+def status_name(status: int) -> str:
+    return lib().sharq_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise SharqError(status, what)
+
+
+def _stream(stream) -> C.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return C.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def weight_bytes(n_out: int, k: int, fmt: int) -> int:
+    return int(lib().sharq_weight_bytes(n_out, k, fmt))
+
+
+def prep_bytes(m_tok: int, k: int, n: int, m: int, fmt: int) -> int:
+    return int(lib().sharq_prep_bytes(m_tok, k, n, m, fmt))
+
+
+class QuantizedWeight:
+    """One FP4 weight payload (codes + MMA scale view + tensor scale)."""
+
+    def __init__(self, buf: torch.Tensor, desc: SharqWQ):
+        self.buf, self.desc = buf, desc
+
+    @property
+    def n_out(self):
+        return self.desc.n_out
+
+    @property
+    def k(self):
+        return self.desc.k
+
+
+class Prepared:
+    """Outputs of the preparation operator for one activation tensor."""
+
+    def __init__(self, buf: torch.Tensor, desc: SharqPrep):
+        self.buf, self.desc = buf, desc
+
+    @property
+    def m_tok(self):
+        return self.desc.m_tok
+
+
+def _device_buffer(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
+
+
+def quantize_weight(w: torch.Tensor, fmt: int = NVFP4, stream=None) -> QuantizedWeight:
+    """Offline FP4 quantization of W [n_out, k] (fp16, CUDA)."""
+    assert w.dtype == torch.float16 and w.is_cuda and w.dim() == 2 and w.is_contiguous()
+    n_out, k = w.shape
+    nbytes = weight_bytes(n_out, k, fmt)
+    if nbytes == 0:
+        raise SharqError(ERR_INVALID_ARG, f"weight shape {tuple(w.shape)} fmt {fmt}")
+    buf = _device_buffer(nbytes, w.device)
+    desc = SharqWQ()
+    _check(lib().sharq_quantize_weight(_ptr(w), n_out, k, fmt, _ptr(buf), nbytes, C.byref(desc), _stream(stream)),
+           "sharq_quantize_weight")
+    return QuantizedWeight(buf, desc)
+
+
+def prepare(x: torch.Tensor, ln_w=None, ln_b=None, eps: float = 1e-5, n: int = 2, m: int = 4,
+            fmt: int = NVFP4, out: Prepared | None = None, stream=None) -> Prepared:
+    """Fused preparation operator on x [m_tok, k] (fp16, CUDA)."""
+    assert x.dtype == torch.float16 and x.is_cuda and x.dim() == 2 and x.is_contiguous()
+    for t in (ln_w, ln_b):
+        assert t is None or (t.dtype == torch.float16 and t.is_cuda and t.numel() == x.shape[1] and t.is_contiguous())
+    m_tok, k = x.shape
+    nbytes = prep_bytes(m_tok, k, n, m, fmt)
+    if nbytes == 0:
+        raise SharqError(ERR_INVALID_ARG, f"prep shape {tuple(x.shape)} {n}:{m} fmt {fmt}")
+    if out is None or out.buf.numel() < nbytes:
+        buf = _device_buffer(nbytes, x.device)
+    else:
+        buf = out.buf
+    desc = SharqPrep()
+    xp = _ptr(x) if m_tok > 0 else None
+    _check(lib().sharq_prepare(xp, m_tok, k, _ptr(ln_w), _ptr(ln_b), float(eps), n, m, fmt, _ptr(buf),
+                               buf.numel(), C.byref(desc), _stream(stream)), "sharq_prepare")
+    return Prepared(buf, desc)
+
+
+def linear(prep: Prepared, qw: QuantizedWeight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Dual-path FP4 linear: fp16 [m_tok, n_out] = (Q(S) + Q(R)) Q(W)^T, scaled."""
+    if out is None:
+        out = torch.empty((prep.m_tok, qw.n_out), dtype=torch.float16, device=prep.buf.device)
+    assert out.dtype == torch.float16 and out.is_contiguous() and tuple(out.shape) == (prep.m_tok, qw.n_out)
+    optr = _ptr(out) if out.numel() else None
+    _check(lib().sharq_linear(C.byref(prep.desc), C.byref(qw.desc), optr, _stream(stream)), "sharq_linear")
+    return out
+
+
+def prep_export(prep: Prepared, stream=None) -> dict:
+    """Canonical host copies (numpy) of a prepared activation."""
+    d = prep.desc
+    m_tok, k, blk = d.m_tok, d.k, BLOCK[d.fmt]
+    out = dict(
+        idx=np.zeros((m_tok, k // d.m, d.n), np.uint8),
+        s_codes=np.zeros((m_tok, k), np.uint8), s_scales=np.zeros((m_tok, k // blk), np.uint8),
+        r_codes=np.zeros((m_tok, k), np.uint8), r_scales=np.zeros((m_tok, k // blk), np.uint8),
+        mu=np.zeros(m_tok, np.float32), rstd=np.zeros(m_tok, np.float32), s_t=np.zeros(1, np.float32))
+    p = lambda a: a.ctypes.data_as(C.c_void_p)
+    _check(lib().sharq_prep_export(C.byref(d), p(out["idx"]), p(out["s_codes"]), p(out["s_scales"]),
+                                   p(out["r_codes"]), p(out["r_scales"]), p(out["mu"]), p(out["rstd"]),
+                                   p(out["s_t"]), _stream(stream)), "sharq_prep_export")
+    out["s_t"] = out["s_t"][0]
+    return out
+
+
+def weight_export(qw: QuantizedWeight, stream=None) -> dict:
+    d = qw.desc
+    blk = BLOCK[d.fmt]
+    out = dict(codes=np.zeros((d.n_out, d.k), np.uint8), scales=np.zeros((d.n_out, d.k // blk), np.uint8),
+               scales_residual=np.zeros((d.n_out, d.k // blk), np.uint8), s_tw=np.zeros(1, np.float32))
+    p = lambda a: a.ctypes.data_as(C.c_void_p)
+    _check(lib().sharq_weight_export(C.byref(d), p(out["codes"]), p(out["scales"]), p(out["scales_residual"]),
+                                     p(out["s_tw"]), _stream(stream)), "sharq_weight_export")
+    out["s_tw"] = out["s_tw"][0]
+    return out
+
+
+def get_last_error(stream=None) -> int:
+    """Synchronizes the stream; returns (and clears) the device status."""
+    return int(lib().sharq_get_last_error(_stream(stream)))
+
+
+def selftest_wait(limit_ns: int, stream=None) -> None:
+    """Enqueues the bounded-wait probe (see sharq_selftest_wait)."""
+    _check(lib().sharq_selftest_wait(int(limit_ns), _stream(stream)), "sharq_selftest_wait")
+
+
+def last_timeout_site() -> int:
+    return int(lib().sharq_last_timeout_site())
+
+
+def set_wait_limit_ns(ns: int) -> int:
+    return int(lib().sharq_set_wait_limit_ns(ns))
+
+
+def last_launch_count() -> int:
+    return int(lib().sharq_last_launch_count())

@@ -1,0 +1,289 @@
+// C ABI of the SharQ library: argument validation, buffer layout, the device
+// status word and the canonical exports. All compute runs in the kernels of
+// prep.cu, wquant.cu and gemm.cu.
+#include <cuda_runtime.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <vector>
+
+#include "layout.h"
+#include "sq_internal.h"
+
+namespace {
+
+__device__ unsigned g_status;  // first timeout site since the last sharq_get_last_error
+
+uint64_t g_wait_ns = 2000000000ull;
+uint32_t g_last_site = 0;
+int g_last_launches = 0;
+
+bool fmt_ok(int fmt) { return fmt == sq::kFmtNV || fmt == sq::kFmtMX; }
+bool nm_ok(int n, int m) { return (m == 2 || m == 4 || m == 8 || m == 16) && n >= 1 && n <= m; }
+bool k_ok(int64_t k) { return k > 0 && k <= SHARQ_K_MAX && k % SHARQ_K_ALIGN == 0; }
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+sharq_status make_ctx(void *stream, sq::LaunchCtx &ctx) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SHARQ_ERR_CUDA;
+    static int sms[64] = {0};
+    if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
+    if (!sms[dev] && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return SHARQ_ERR_CUDA;
+    static unsigned *status_ptr[64] = {nullptr};
+    if (!status_ptr[dev] && cudaGetSymbolAddress((void **)&status_ptr[dev], g_status) != cudaSuccess)
+        return SHARQ_ERR_CUDA;
+    ctx.stream = reinterpret_cast<cudaStream_t>(stream);
+    ctx.status = status_ptr[dev];
+    ctx.wait_ns = g_wait_ns;
+    ctx.num_sms = sms[dev];
+    ctx.launches = 0;
+    return SHARQ_OK;
+}
+
+void fill_prep(sharq_prep *P, void *buf, int64_t m_tok, int64_t k, int n, int m, int fmt) {
+    sq::PrepLayout L = sq::prep_layout(m_tok, k, n, m, fmt);
+    uint8_t *b = static_cast<uint8_t *>(buf);
+    memset(P, 0, sizeof(*P));
+    P->m_tok = m_tok;
+    P->k = k;
+    P->n = n;
+    P->m = m;
+    P->fmt = fmt;
+    P->sf_rows = L.sf_rows;
+    P->meta_row_bytes = L.meta_row;
+    P->s_codes = b + L.s_codes;
+    P->r_codes = b + L.r_codes;
+    P->s_scales = b + L.s_scales;
+    P->r_scales = b + L.r_scales;
+    P->meta = b + L.meta;
+    P->scratch = b + L.stats;
+    P->tensor_scale = reinterpret_cast<float *>(b + L.words) + 1;
+}
+
+void fill_wq(sharq_wq *W, void *buf, int64_t n_out, int64_t k, int fmt) {
+    sq::WLayout L = sq::w_layout(n_out, k, fmt);
+    uint8_t *b = static_cast<uint8_t *>(buf);
+    memset(W, 0, sizeof(*W));
+    W->n_out = n_out;
+    W->k = k;
+    W->fmt = fmt;
+    W->sf_rows = L.sf_rows;
+    W->codes = b + L.codes;
+    W->scales_backbone = b + L.scales;
+    W->scales_residual = b + L.scales;  // same values in the same MMA layout
+    W->scratch = b + L.words;
+    W->tensor_scale = reinterpret_cast<float *>(b + L.words) + 1;
+}
+
+void unpack_codes(const std::vector<uint8_t> &packed, int64_t count, uint8_t *dst) {
+    for (int64_t i = 0; i < count / 2; ++i) {
+        dst[2 * i] = packed[i] & 0xF;
+        dst[2 * i + 1] = packed[i] >> 4;
+    }
+}
+
+void unpack_scales(const std::vector<uint8_t> &sf, int64_t rows, int64_t nblk, uint8_t *dst) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < nblk; ++j) dst[r * nblk + j] = sf[sq::sf_offset(r, j, nblk)];
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sharq_status_string(sharq_status s) {
+    switch (s) {
+        case SHARQ_OK: return "SHARQ_OK";
+        case SHARQ_ERR_INVALID_ARG: return "SHARQ_ERR_INVALID_ARG";
+        case SHARQ_ERR_UNSUPPORTED: return "SHARQ_ERR_UNSUPPORTED";
+        case SHARQ_ERR_CUDA: return "SHARQ_ERR_CUDA";
+        case SHARQ_ERR_TIMEOUT: return "SHARQ_ERR_TIMEOUT";
+    }
+    return "SHARQ_ERR_UNKNOWN";
+}
+
+int sharq_last_launch_count(void) { return g_last_launches; }
+
+uint64_t sharq_set_wait_limit_ns(uint64_t ns) {
+    uint64_t old = g_wait_ns;
+    g_wait_ns = ns ? ns : 2000000000ull;
+    return old;
+}
+
+uint32_t sharq_last_timeout_site(void) { return g_last_site; }
+
+size_t sharq_weight_bytes(int64_t n_out, int64_t k, int fmt) {
+    if (n_out < 1 || n_out % SHARQ_N_ALIGN != 0 || n_out > (1ll << 30) || !k_ok(k) || !fmt_ok(fmt)) return 0;
+    return (size_t)sq::w_layout(n_out, k, fmt).total;
+}
+
+size_t sharq_prep_bytes(int64_t m_tok, int64_t k, int n, int m, int fmt) {
+    if (m_tok < 0 || m_tok > (1ll << 30) || !k_ok(k) || !nm_ok(n, m) || !fmt_ok(fmt)) return 0;
+    return (size_t)sq::prep_layout(m_tok, k, n, m, fmt).total;
+}
+
+sharq_status sharq_quantize_weight(const void *w_dev, int64_t n_out, int64_t k, int fmt, void *wq_dev,
+                                   size_t wq_bytes, sharq_wq *wq_out, void *stream) {
+    g_last_launches = 0;
+    size_t need = sharq_weight_bytes(n_out, k, fmt);
+    if (!need || !w_dev || !wq_dev || !wq_out || wq_bytes < need) return SHARQ_ERR_INVALID_ARG;
+    if (!aligned(w_dev, 16) || !aligned(wq_dev, sq::kAlign)) return SHARQ_ERR_INVALID_ARG;
+    sq::LaunchCtx ctx;
+    sharq_status st = make_ctx(stream, ctx);
+    if (st != SHARQ_OK) return st;
+    fill_wq(wq_out, wq_dev, n_out, k, fmt);
+    st = sq::launch_quantize_weight(ctx, *wq_out, w_dev);
+    g_last_launches = ctx.launches;
+    return st;
+}
+
+sharq_status sharq_prepare(const void *x_dev, int64_t m_tok, int64_t k, const void *ln_w_dev, const void *ln_b_dev,
+                           float eps, int n, int m, int fmt, void *prep_dev, size_t prep_bytes, sharq_prep *prep_out,
+                           void *stream) {
+    g_last_launches = 0;
+    size_t need = sharq_prep_bytes(m_tok, k, n, m, fmt);
+    if (!need || !prep_dev || !prep_out || prep_bytes < need) return SHARQ_ERR_INVALID_ARG;
+    if (m_tok > 0 && !x_dev) return SHARQ_ERR_INVALID_ARG;
+    if (!(eps > 0.0f) || eps != eps || eps > 3.0e38f) return SHARQ_ERR_INVALID_ARG;
+    if ((x_dev && !aligned(x_dev, 16)) || !aligned(prep_dev, sq::kAlign) || (ln_w_dev && !aligned(ln_w_dev, 16)) ||
+        (ln_b_dev && !aligned(ln_b_dev, 16)))
+        return SHARQ_ERR_INVALID_ARG;
+    sq::LaunchCtx ctx;
+    sharq_status st = make_ctx(stream, ctx);
+    if (st != SHARQ_OK) return st;
+    fill_prep(prep_out, prep_dev, m_tok, k, n, m, fmt);
+    st = sq::launch_prepare(ctx, *prep_out, x_dev, ln_w_dev, ln_b_dev, eps);
+    if (st == SHARQ_OK && cudaGetLastError() != cudaSuccess) st = SHARQ_ERR_CUDA;
+    g_last_launches = ctx.launches;
+    return st;
+}
+
+sharq_status sharq_linear(const sharq_prep *prep, const sharq_wq *wq, void *out_dev, void *stream) {
+    g_last_launches = 0;
+    if (!prep || !wq) return SHARQ_ERR_INVALID_ARG;
+    if (!fmt_ok(prep->fmt) || prep->fmt != wq->fmt || prep->k != wq->k || !k_ok(prep->k)) return SHARQ_ERR_INVALID_ARG;
+    if (wq->n_out < 1 || wq->n_out % SHARQ_N_ALIGN != 0 || prep->m_tok < 0) return SHARQ_ERR_INVALID_ARG;
+    if (prep->sf_rows < prep->m_tok || wq->sf_rows < wq->n_out || wq->sf_rows % sq::kWRowPad != 0 ||
+        prep->sf_rows % sq::kActRowPad != 0)
+        return SHARQ_ERR_INVALID_ARG;
+    if (prep->m_tok == 0) return SHARQ_OK;
+    if (!out_dev || !aligned(out_dev, 16) || !prep->s_codes || !prep->r_codes || !wq->codes ||
+        wq->scales_backbone != wq->scales_residual)
+        return SHARQ_ERR_INVALID_ARG;
+    if (prep->m_tok > (1ll << 31) - 256) return SHARQ_ERR_UNSUPPORTED;
+    sq::LaunchCtx ctx;
+    sharq_status st = make_ctx(stream, ctx);
+    if (st != SHARQ_OK) return st;
+    st = sq::launch_linear(ctx, *prep, *wq, out_dev);
+    g_last_launches = ctx.launches;
+    return st;
+}
+
+sharq_status sharq_prep_export(const sharq_prep *prep, uint8_t *idx_host, uint8_t *s_codes_host,
+                               uint8_t *s_scales_host, uint8_t *r_codes_host, uint8_t *r_scales_host,
+                               float *mu_host, float *rstd_host, float *s_t_host, void *stream) {
+    if (!prep || !fmt_ok(prep->fmt) || !nm_ok(prep->n, prep->m) || prep->m_tok < 0) return SHARQ_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SHARQ_ERR_CUDA;
+    const int64_t m_tok = prep->m_tok, k = prep->k, nblk = k / sq::blk_of(prep->fmt);
+    const int64_t codes = m_tok * (k / 2), sf = prep->sf_rows * nblk;
+    std::vector<uint8_t> buf;
+    auto fetch = [&](const void *src, int64_t bytes) -> bool {
+        buf.resize((size_t)(bytes > 0 ? bytes : 1));
+        return bytes == 0 || cudaMemcpy(buf.data(), src, (size_t)bytes, cudaMemcpyDeviceToHost) == cudaSuccess;
+    };
+    if (s_codes_host) {
+        if (!fetch(prep->s_codes, codes)) return SHARQ_ERR_CUDA;
+        unpack_codes(buf, m_tok * k, s_codes_host);
+    }
+    if (r_codes_host) {
+        if (!fetch(prep->r_codes, codes)) return SHARQ_ERR_CUDA;
+        unpack_codes(buf, m_tok * k, r_codes_host);
+    }
+    if (s_scales_host) {
+        if (!fetch(prep->s_scales, sf)) return SHARQ_ERR_CUDA;
+        unpack_scales(buf, m_tok, nblk, s_scales_host);
+    }
+    if (r_scales_host) {
+        if (!fetch(prep->r_scales, sf)) return SHARQ_ERR_CUDA;
+        unpack_scales(buf, m_tok, nblk, r_scales_host);
+    }
+    if (idx_host) {
+        if (!fetch(prep->meta, m_tok * prep->meta_row_bytes)) return SHARQ_ERR_CUDA;
+        const int ib = sq::idx_bits(prep->m), n = prep->n, groups = (int)(k / prep->m);
+        for (int64_t r = 0; r < m_tok; ++r) {
+            const uint8_t *row = buf.data() + r * prep->meta_row_bytes;
+            for (int64_t f = 0; f < (int64_t)groups * n; ++f) {
+                uint32_t v = 0;
+                for (int b = 0; b < ib; ++b) {
+                    int64_t bit = f * ib + b;
+                    v |= (uint32_t)((row[bit >> 3] >> (bit & 7)) & 1u) << b;
+                }
+                idx_host[r * groups * n + f] = (uint8_t)v;
+            }
+        }
+    }
+    if (mu_host || rstd_host) {
+        if (!fetch(prep->scratch, m_tok * 8)) return SHARQ_ERR_CUDA;
+        const float *st = reinterpret_cast<const float *>(buf.data());
+        for (int64_t r = 0; r < m_tok; ++r) {
+            if (mu_host) mu_host[r] = st[2 * r];
+            if (rstd_host) rstd_host[r] = st[2 * r + 1];
+        }
+    }
+    if (s_t_host && cudaMemcpy(s_t_host, prep->tensor_scale, sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SHARQ_ERR_CUDA;
+    return SHARQ_OK;
+}
+
+sharq_status sharq_weight_export(const sharq_wq *wq, uint8_t *codes_host, uint8_t *scales_host,
+                                 uint8_t *scales_residual_host, float *s_tw_host, void *stream) {
+    if (!wq || !fmt_ok(wq->fmt)) return SHARQ_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SHARQ_ERR_CUDA;
+    const int64_t nblk = wq->k / sq::blk_of(wq->fmt);
+    std::vector<uint8_t> buf;
+    if (codes_host) {
+        buf.resize((size_t)(wq->n_out * (wq->k / 2)));
+        if (cudaMemcpy(buf.data(), wq->codes, buf.size(), cudaMemcpyDeviceToHost) != cudaSuccess) return SHARQ_ERR_CUDA;
+        unpack_codes(buf, wq->n_out * wq->k, codes_host);
+    }
+    const void *views[2] = {wq->scales_backbone, wq->scales_residual};
+    uint8_t *dsts[2] = {scales_host, scales_residual_host};
+    for (int v = 0; v < 2; ++v) {
+        if (!dsts[v]) continue;
+        buf.resize((size_t)(wq->sf_rows * nblk));
+        if (cudaMemcpy(buf.data(), views[v], buf.size(), cudaMemcpyDeviceToHost) != cudaSuccess) return SHARQ_ERR_CUDA;
+        unpack_scales(buf, wq->n_out, nblk, dsts[v]);
+    }
+    if (s_tw_host && cudaMemcpy(s_tw_host, wq->tensor_scale, sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SHARQ_ERR_CUDA;
+    return SHARQ_OK;
+}
+
+sharq_status sharq_selftest_wait(uint64_t limit_ns, void *stream) {
+    g_last_launches = 0;
+    if (limit_ns == 0 || limit_ns > 10000000000ull) return SHARQ_ERR_INVALID_ARG;
+    sq::LaunchCtx ctx;
+    sharq_status st = make_ctx(stream, ctx);
+    if (st != SHARQ_OK) return st;
+    st = sq::launch_wait_probe(ctx, limit_ns);
+    g_last_launches = ctx.launches;
+    return st;
+}
+
+sharq_status sharq_get_last_error(void *stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SHARQ_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return SHARQ_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return SHARQ_ERR_CUDA;
+    if (v != 0) {
+        g_last_site = v;
+        unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return SHARQ_ERR_CUDA;
+        return SHARQ_ERR_TIMEOUT;
+    }
+    return SHARQ_OK;
+}
+
+}  // extern "C"

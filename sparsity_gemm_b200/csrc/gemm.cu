@@ -1,0 +1,362 @@
+// Dual-path FP4 GEMM of SharQ on sm_100a (tcgen05 block-scaled MMA).
+//
+// "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM
+// Inference", Abstract: a sparse FP4 GEMM processes the backbone while a
+// dense FP4 GEMM compensates; the two paths share a single FP4 weight payload
+// with path-specific scale views. Here both paths issue into ONE tensor-memory
+// accumulator, and every W tile (codes and scale view) is loaded once per
+// K step and read by both paths' MMAs:
+//     acc = sum_k Q(S)[i,k] W[j,k] + Q(R)[i,k] W[j,k]      (block-scaled)
+//     out = RN16(acc * s_t * s_tW)
+//
+// The backbone runs as a dense FP4 MMA over the full K with zeros off the
+// mask: the block-scaled FP4 sparse MMA kinds take pair-wise 4:8 metadata,
+// which an element-wise top-n-of-m mask does not satisfy in general.
+//
+// Structure: persistent CTAs (one per SM), tile 128 x 256 x 256 (M x N x K),
+// 3-stage TMA pipeline, 6 warps:
+//   warp 0      TMA producer (A_S, A_R, W tiles; scale atoms by bulk copy)
+//   warp 1      tensor-memory allocation and the single-thread MMA issuer
+//               (scale atoms -> tensor memory by tcgen05.cp, then MMAs)
+//   warps 2..5  epilogue: tensor memory -> registers -> fp16 -> global
+// Every mbarrier wait is bounded (global-timer limit); a wait that runs out
+// records a site code in the status word and the CTA winds down cleanly.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+
+#include "sharq_dev.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+
+constexpr int kBM = 128, kBN = 256, kBKBytes = 128, kStages = 3;  // K tile: 256 FP4 = 128 bytes
+constexpr int kABytes = kBM * kBKBytes;                            // 16 KB
+constexpr int kBBytes = kBN * kBKBytes;                            // 32 KB
+constexpr int kSfaMax = 2048, kSfbMax = 4096;                      // NVFP4 sizes (MXFP4 uses half)
+constexpr int kOffAS = 0, kOffAR = kABytes, kOffB = 2 * kABytes;
+constexpr int kOffSFAS = kOffB + kBBytes, kOffSFAR = kOffSFAS + kSfaMax, kOffSFB = kOffSFAR + kSfaMax;
+constexpr int kStageBytes = kOffSFB + kSfbMax;                     // 72 KB, a multiple of 1024
+constexpr int kBarOff = kStages * kStageBytes;
+constexpr int kSmemBytes = kBarOff + 256 + 1024;                   // barriers + alignment slack
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColSfaS = 256, kColSfaR = 272, kColSfb = 288;  // scale columns after the accumulator
+constexpr int kGemmThreads = 192;
+
+enum : unsigned {
+    kSiteProducer = 0x101,
+    kSiteMmaAcc = 0x102,
+    kSiteMmaFull = 0x103,
+    kSiteEpilogue = 0x104,
+    kSiteProbe = 0x1FF,
+};
+
+// Exit drains (in-flight copies, outstanding MMAs) always get this long,
+// whatever the configurable wait limit is.
+constexpr uint64_t kDrainNs = 2000000000ull;
+
+struct GemmParams {
+    const uint8_t *sfa_s, *sfa_r, *sfb;
+    const float *s_t, *s_tw;
+    __half *out;
+    int32_t m_tok, n_out, k;
+    unsigned *status;
+    uint64_t wait_ns;
+};
+
+// Instruction descriptor of the block-scaled MMA (M = 128, N = 256, E2M1 x
+// E2M1, K-major A and B): A/B format E2M1 at bits 7-9 / 10-12, N >> 3 at
+// bits 17-22, scale format (0 = UE4M3, 1 = E8M0) at bit 23, M >> 4 at bits
+// 24-28; scale-factor byte selectors at bits 29-30 (A) and 4-5 (B).
+template <int FMT>
+__device__ __forceinline__ uint32_t idesc_of(uint32_t sf_id) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((FMT == kFmtMX ? 1u : 0u) << 23) |
+           ((uint32_t)(kBM >> 4) << 24) | (sf_id << 29) | (sf_id << 4);
+}
+
+// K-major operand tile, rows of 128 bytes, 128-byte swizzle; 8-row groups
+// are 1024 bytes apart.
+__device__ __forceinline__ uint64_t desc_operand(uint32_t addr) { return smem_desc(addr, 16, 1024, 2); }
+
+// One 512-byte scale atom: 32 rows of 16 bytes, no swizzle, 8-row groups
+// 128 bytes apart.
+__device__ __forceinline__ uint64_t desc_scales(uint32_t addr) { return smem_desc(addr, 0, 128, 0); }
+
+// Wait bounded only by time (used to drain in-flight copies on exit).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+    uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer_ns() - t0 > limit_ns) break;
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constant__ CUtensorMap tm_ar,
+                 const __grid_constant__ CUtensorMap tm_b, const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + kBarOff;  // full[s], empty[s], acc_full, acc_empty, drain
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+    const uint32_t acc_full = bar0 + 8u * (2 * kStages);
+    const uint32_t acc_empty = acc_full + 8u;
+    const uint32_t drain_bar = acc_full + 16u;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOff + 128);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int m_tiles = (p.m_tok + kBM - 1) / kBM, n_tiles = (p.n_out + kBN - 1) / kBN;
+    const int num_tiles = m_tiles * n_tiles, kt_count = p.k / 256;
+    const int64_t atoms_per_row_blk = (int64_t)(p.k / (FMT == kFmtNV ? 16 : 32)) / 4;
+    constexpr int kAtomsPerTile = FMT == kFmtNV ? 4 : 2;  // 512-byte atoms per 128 rows per K tile
+    constexpr uint32_t kSfBytes = 512u * kAtomsPerTile;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 128);
+        mbar_init(drain_bar, 1);
+        mbar_fence_init();
+        prefetch_tmap(&tm_as);
+        prefetch_tmap(&tm_ar);
+        prefetch_tmap(&tm_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int32_t last[kStages];
+            for (int s = 0; s < kStages; ++s) last[s] = -1;
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                const int nb = tile % n_tiles, mb = tile / n_tiles;
+                for (int kt = 0; kt < kt_count; ++kt, ++it) {
+                    const int s = (int)(it % kStages);
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!mbar_wait(empty_bar(s), ph ^ 1u, p.status, kSiteProducer, p.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = full_bar(s);
+                    const uint32_t st = sbase + (uint32_t)(s * kStageBytes);
+                    mbar_arrive_expect_tx(fb, 2 * kABytes + kBBytes + 4 * kSfBytes);
+                    tma_load_2d(st + kOffAS, &tm_as, kt * kBKBytes, mb * kBM, fb);
+                    tma_load_2d(st + kOffAR, &tm_ar, kt * kBKBytes, mb * kBM, fb);
+                    tma_load_2d(st + kOffB, &tm_b, kt * kBKBytes, nb * kBN, fb);
+                    const int64_t a_off = ((int64_t)mb * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
+                    const int64_t b0 = ((int64_t)(2 * nb) * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
+                    const int64_t b1 = b0 + atoms_per_row_blk * 512;
+                    bulk_load(st + kOffSFAS, p.sfa_s + a_off, kSfBytes, fb);
+                    bulk_load(st + kOffSFAR, p.sfa_r + a_off, kSfBytes, fb);
+                    bulk_load(st + kOffSFB, p.sfb + b0, kSfBytes, fb);
+                    bulk_load(st + kOffSFB + kSfBytes, p.sfb + b1, kSfBytes, fb);
+                    last[s] = (int32_t)it;
+                }
+            }
+            // Never leave the CTA with copies in flight.
+            for (int s = 0; s < kStages; ++s)
+                if (last[s] >= 0) drain_wait(full_bar(s), ((uint32_t)last[s] / kStages) & 1u, kDrainNs);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            uint32_t it = 0, tile_iter = 0;
+            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tile_iter) {
+                if (!mbar_wait(acc_empty, (tile_iter & 1u) ^ 1u, p.status, kSiteMmaAcc, p.wait_ns)) break;
+                tc_fence_after();
+                bool ok = true;
+                for (int kt = 0; kt < kt_count; ++kt, ++it) {
+                    const int s = (int)(it % kStages);
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!mbar_wait(full_bar(s), ph, p.status, kSiteMmaFull, p.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = sbase + (uint32_t)(s * kStageBytes);
+                    // Scale atoms -> tensor memory. One atom (128 rows x 4
+                    // scales) fills 4 columns; the W tile's 256 rows take two.
+#pragma unroll
+                    for (int a = 0; a < kAtomsPerTile; ++a) {
+                        tc_copy_scales(tmem + kColSfaS + 4 * a, desc_scales(st + kOffSFAS + 512 * a));
+                        tc_copy_scales(tmem + kColSfaR + 4 * a, desc_scales(st + kOffSFAR + 512 * a));
+                        tc_copy_scales(tmem + kColSfb + 8 * a, desc_scales(st + kOffSFB + 512 * a));
+                        tc_copy_scales(tmem + kColSfb + 8 * a + 4, desc_scales(st + kOffSFB + kSfBytes + 512 * a));
+                    }
+                    const uint64_t da_s = desc_operand(st + kOffAS);
+                    const uint64_t da_r = desc_operand(st + kOffAR);
+                    const uint64_t db = desc_operand(st + kOffB);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {  // 4 MMAs of K = 64 (32 bytes) per K tile
+                        const uint32_t acc = (kt | j) != 0;
+                        if (FMT == kFmtNV) {
+                            const uint32_t idesc = idesc_of<FMT>(0);
+                            tc_mma_nvf4(tmem, da_s + 2 * j, db + 2 * j, idesc, tmem + kColSfaS + 4 * j,
+                                        tmem + kColSfb + 8 * j, acc);
+                            tc_mma_nvf4(tmem, da_r + 2 * j, db + 2 * j, idesc, tmem + kColSfaR + 4 * j,
+                                        tmem + kColSfb + 8 * j, 1u);
+                        } else {
+                            const uint32_t sf_id = (uint32_t)(j & 1) * 2u;  // 2 scales per row per MMA
+                            const uint32_t idesc = idesc_of<FMT>(sf_id);
+                            const uint32_t a_col = 4 * (j >> 1), b_col = 8 * (j >> 1);
+                            tc_mma_mxf4(tmem, da_s + 2 * j, db + 2 * j, idesc, (tmem + kColSfaS + a_col) | (sf_id << 30),
+                                        (tmem + kColSfb + b_col) | (sf_id << 30), acc);
+                            tc_mma_mxf4(tmem, da_r + 2 * j, db + 2 * j, idesc, (tmem + kColSfaR + a_col) | (sf_id << 30),
+                                        (tmem + kColSfb + b_col) | (sf_id << 30), 1u);
+                        }
+                    }
+                    tc_commit(empty_bar(s));  // frees the stage once these MMAs complete
+                }
+                if (!ok) break;
+                tc_commit(acc_full);
+            }
+            tc_commit(drain_bar);  // every MMA and copy of this thread done before exit
+            drain_wait(drain_bar, 0, kDrainNs);
+        }
+        __syncwarp();
+    } else {
+        const int q = warp & 3;  // tensor-memory lane quadrant this warp may access
+        const float alpha = __fmul_rn(*p.s_t, *p.s_tw);
+        uint32_t tile_iter = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tile_iter) {
+            if (!mbar_wait(acc_full, tile_iter & 1u, p.status, kSiteEpilogue, p.wait_ns)) break;
+            tc_fence_after();
+            const int nb = tile % n_tiles, mb = tile / n_tiles;
+            const int row = mb * kBM + q * 32 + lane;
+#pragma unroll 1
+            for (int cc = 0; cc < kBN / 32; ++cc) {
+                uint32_t r[32];
+                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cc * 32), r);
+                tmem_ld_wait();
+                const int col0 = nb * kBN + cc * 32;
+                if (row < p.m_tok && col0 < p.n_out) {
+                    uint32_t h[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        __half2 v = __floats2half2_rn(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
+                                                      __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
+                        h[i] = *reinterpret_cast<uint32_t *>(&v);
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + (int64_t)row * p.n_out + col0);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(acc_empty);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Failure-detection probe: one thread waits, with the bounded wait the GEMM
+// uses, on an mbarrier that nothing ever arrives at. The wait runs out and
+// records kSiteProbe; the kernel then returns normally.
+__global__ void wait_probe_kernel(unsigned *status, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(b, 0, status, kSiteProbe, limit_ns);
+}
+
+sharq_status launch_wait_probe(LaunchCtx &ctx, uint64_t limit_ns) {
+    wait_probe_kernel<<<1, 32, 0, ctx.stream>>>(ctx.status, limit_ns);
+    ctx.launches++;
+    SQ_CUDA_TRY(cudaGetLastError());
+    return SHARQ_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D byte tensor [rows][row_bytes], box = 128 bytes x box_rows, 128-byte swizzle.
+static bool make_code_map(CUtensorMap *tm, const void *base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {row_bytes, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)kBKBytes, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, void *out) {
+    if (P.m_tok == 0) return SHARQ_OK;
+    static bool attr_done[64][2] = {};
+    int dev = 0;
+    SQ_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
+    const int f = P.fmt == kFmtNV ? 0 : 1;
+    if (!attr_done[dev][f]) {
+        if (f == 0)
+            SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<kFmtNV>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes));
+        else
+            SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<kFmtMX>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes));
+        attr_done[dev][f] = true;
+    }
+    CUtensorMap tm_as, tm_ar, tm_b;
+    if (!make_code_map(&tm_as, P.s_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
+        !make_code_map(&tm_ar, P.r_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
+        !make_code_map(&tm_b, W.codes, (uint64_t)(W.k / 2), (uint64_t)W.n_out, kBN))
+        return SHARQ_ERR_CUDA;
+    GemmParams gp;
+    gp.sfa_s = (const uint8_t *)P.s_scales;
+    gp.sfa_r = (const uint8_t *)P.r_scales;
+    gp.sfb = (const uint8_t *)W.scales_backbone;  // the residual view holds the same bytes
+    gp.s_t = P.tensor_scale;
+    gp.s_tw = W.tensor_scale;
+    gp.out = (__half *)out;
+    gp.m_tok = (int32_t)P.m_tok;
+    gp.n_out = (int32_t)W.n_out;
+    gp.k = (int32_t)P.k;
+    gp.status = ctx.status;
+    gp.wait_ns = ctx.wait_ns;
+    const int64_t tiles = ((P.m_tok + kBM - 1) / kBM) * ((W.n_out + kBN - 1) / kBN);
+    const unsigned grid = (unsigned)(tiles < ctx.num_sms ? tiles : ctx.num_sms);
+    if (f == 0)
+        dual_gemm_kernel<kFmtNV><<<grid, kGemmThreads, kSmemBytes, ctx.stream>>>(tm_as, tm_ar, tm_b, gp);
+    else
+        dual_gemm_kernel<kFmtMX><<<grid, kGemmThreads, kSmemBytes, ctx.stream>>>(tm_as, tm_ar, tm_b, gp);
+    ctx.launches++;
+    SQ_CUDA_TRY(cudaGetLastError());
+    return SHARQ_OK;
+}
+
+}  // namespace sq

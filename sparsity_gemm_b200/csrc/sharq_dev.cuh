@@ -1,0 +1,280 @@
+// Device helpers of the SharQ library: numeric steps shared by the
+// preparation and weight kernels, and thin wrappers over the sm_100a PTX the
+// GEMM uses (mbarrier, TMA, tcgen05). Every floating-point step is an
+// explicit round-to-nearest intrinsic, so the compiler cannot contract a
+// multiply and an add into one FMA.
+#pragma once
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "layout.h"
+
+namespace sq {
+
+// ---------------------------------------------------------------------------
+// Status word: the first non-zero site code wins.
+__device__ __forceinline__ void record_status(unsigned *status, unsigned site) {
+    if (status) atomicCAS(status, 0u, site);
+}
+
+__device__ __forceinline__ unsigned read_status(const unsigned *status) {
+    return status ? *(volatile const unsigned *)status : 0u;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------------------------
+// Numeric steps
+
+// fp16 -> fp32 (exact).
+__device__ __forceinline__ float h2f(uint16_t h) { return __half2float(__ushort_as_half(h)); }
+
+// LayerNorm apply: RN32(RN32(RN32(x - mu) * rstd) * gamma) + beta.
+__device__ __forceinline__ float ln_apply(float x, float mu, float rstd, bool has_g, float g, bool has_b,
+                                          float b) {
+    float t = __fsub_rn(x, mu);
+    t = __fmul_rn(t, rstd);
+    if (has_g) t = __fmul_rn(t, g);
+    if (has_b) t = __fadd_rn(t, b);
+    return t;
+}
+
+// E2M1 codes of (lo, hi) packed into one byte, lo in bits 0-3. The hardware
+// conversion rounds to nearest even and saturates to 6; the sign bit is then
+// forced from the operand so that values rounding to zero keep their sign.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+    uint32_t b;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(b) : "f"(hi), "f"(lo));
+    b |= (__float_as_uint(lo) >> 31) << 3;
+    b |= (__float_as_uint(hi) >> 31) << 7;
+    return b;
+}
+
+// Values of two E2M1 codes in one byte (lo nibble first), as floats.
+__device__ __forceinline__ float2 e2m1x2_value(uint32_t byte) {
+    uint32_t h2;
+    asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(h2) : "r"(byte));
+    __half2 h = *reinterpret_cast<__half2 *>(&h2);
+    return __half22float2(h);
+}
+
+// UE4M3 code of u >= 0: round to nearest even, saturate to 448.
+__device__ __forceinline__ uint32_t ue4m3_code(float u) {
+    uint16_t e;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(e) : "f"(0.0f), "f"(u));
+    return e & 0xFFu;
+}
+
+// Value of a UE4M3 code (exact: every E4M3 value is an fp16 value).
+__device__ __forceinline__ float ue4m3_value(uint32_t code) {
+    uint32_t h2;
+    uint16_t c = (uint16_t)code;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+    return __half2float(__ushort_as_half((uint16_t)(h2 & 0xFFFF)));
+}
+
+// OCP MX block exponent: floor(log2 a) - 2 for a > 0, clamped to [-127, 127].
+__device__ __forceinline__ int mx_exponent(float a) {
+    uint32_t bits = __float_as_uint(a);
+    int ex = (int)(bits >> 23);
+    int fl = ex ? ex - 127 : (31 - __clz((int)(bits & 0x7FFFFF))) - 149;
+    int e = fl - 2;
+    return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// 2^e as a float, e in [-127, 127] (2^-127 is subnormal).
+__device__ __forceinline__ float pow2f(int e) {
+    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// Step d and scale code of one block with amax a (tensor scale s_t; c6 =
+// RN32(6 s_t)). NVFP4: code = UE4M3(a / c6), d = RN32(value * s_t). MXFP4:
+// code = e + 127, d = 2^e; a == 0 gives code 0 and d = 0.
+template <int FMT>
+__device__ __forceinline__ float block_step(float a, float s_t, float c6, uint32_t &code) {
+    if (FMT == kFmtNV) {
+        float u = __fdiv_rn(a, c6);
+        code = ue4m3_code(u);
+        return __fmul_rn(ue4m3_value(code), s_t);
+    } else {
+        if (a == 0.0f) {
+            code = 0;
+            return 0.0f;
+        }
+        int e = mx_exponent(a);
+        code = (uint32_t)(e + 127);
+        return pow2f(e);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Shared-memory and barrier primitives
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait on a phase of an mbarrier. Gives up after `limit_ns` of
+// global time, or as soon as another thread has recorded a status, and then
+// records `site` (first writer wins) and returns false.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned *status, unsigned site,
+                                          uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (read_status(status) != 0u) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                record_status(status, site);
+                return false;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// TMA and bulk copies (no multicast anywhere in this library).
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int32_t c0, int32_t c1, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const void *tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05 (5th-generation tensor core) wrappers, cta_group::1.
+
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Arrive on `bar` once every tcgen05 operation this thread issued so far
+// has completed.
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05 format, version 1).
+//   start: byte address >> 4 (bits 0-13); lbo: bits 16-29; sbo: bits 32-45;
+//   version 1 at bits 46-47; layout type at bits 61-63 (2 = 128-byte swizzle,
+//   0 = no swizzle).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                                              uint32_t layout) {
+    uint64_t d = (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= 1ull << 46;
+    d |= (uint64_t)layout << 61;
+    return d;
+}
+
+// Copy one 512-byte scale atom (32 rows x 128 bits, replicated to the four
+// 32-lane sub-partitions) from shared memory into tensor memory.
+__device__ __forceinline__ void tc_copy_scales(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T with per-16 UE4M3 block scales (NVFP4).
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Same with per-32 E8M0 block scales (MXFP4).
+__device__ __forceinline__ void tc_mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// 32 consecutive fp32 columns of this warp's 32 tensor-memory lanes.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+}  // namespace sq

@@ -1,0 +1,30 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sharq.h"
+
+namespace sq {
+
+struct LaunchCtx {
+    cudaStream_t stream;
+    unsigned *status;      // device status word
+    uint64_t wait_ns;      // bound of every device-side wait
+    int num_sms;
+    int launches;          // kernels enqueued by the current entry point
+};
+
+sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, const void *gamma,
+                            const void *beta, float eps);
+sharq_status launch_quantize_weight(LaunchCtx &ctx, const sharq_wq &W, const void *w);
+sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, void *out);
+sharq_status launch_wait_probe(LaunchCtx &ctx, uint64_t limit_ns);
+
+}  // namespace sq
+
+#define SQ_CUDA_TRY(expr)                                         \
+    do {                                                          \
+        cudaError_t _e = (expr);                                  \
+        if (_e != cudaSuccess) return SHARQ_ERR_CUDA;             \
+    } while (0)

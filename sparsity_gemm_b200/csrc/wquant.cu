@@ -1,0 +1,121 @@
+// Weight quantization (offline) of SharQ on sm_100a.
+//
+// "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM
+// Inference", Abstract: the two GEMM paths share a single FP4 weight payload
+// with path-specific scale views. This kernel pair writes that payload: one
+// E2M1 code matrix and one block-scale matrix in the tcgen05 MMA scale layout,
+// which both paths' scale views point at (the same values, as the
+// dequantized weight must be identical on both paths).
+//   1. absmax_kernel: amax|W| over the whole matrix (NVFP4 tensor scale).
+//   2. wq_encode_kernel: per 32-element chunk, block scales and E2M1 codes.
+#include <cuda_fp16.h>
+
+#include "sharq_dev.cuh"
+#include "sq_internal.h"
+
+namespace sq {
+
+constexpr int kWThreads = 256;
+
+// amax of |fp16| over `count` halves (count a multiple of 8): the absolute
+// value of a finite fp16 orders like its low 15 bits.
+__global__ void __launch_bounds__(kWThreads) absmax_kernel(const uint16_t *__restrict__ w, int64_t count,
+                                                          unsigned *__restrict__ amax_word) {
+    __shared__ unsigned red[kWThreads / 32];
+    const uint4 *p = reinterpret_cast<const uint4 *>(w);
+    const int64_t nvec = count / 8;
+    unsigned m = 0;
+    for (int64_t i = (int64_t)blockIdx.x * kWThreads + threadIdx.x; i < nvec; i += (int64_t)gridDim.x * kWThreads) {
+        uint4 v = __ldg(p + i);
+        const uint32_t ws[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            m = max(m, ws[q] & 0x7FFFu);
+            m = max(m, (ws[q] >> 16) & 0x7FFFu);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (threadIdx.x % 32 == 0) red[threadIdx.x / 32] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned a = 0;
+        for (int i = 0; i < kWThreads / 32; ++i) a = max(a, red[i]);
+        atomicMax(amax_word, __float_as_uint(h2f((uint16_t)a)));
+    }
+}
+
+template <int FMT>
+__global__ void __launch_bounds__(kWThreads)
+wq_encode_kernel(const uint16_t *__restrict__ w, int64_t n_out, int64_t sf_rows, int64_t k,
+                 const unsigned *__restrict__ amax_word, float *__restrict__ s_tw_out, uint8_t *__restrict__ codes,
+                 uint8_t *__restrict__ sf) {
+    constexpr int BLK = FMT == kFmtNV ? 16 : 32;
+    constexpr int NB = 32 / BLK;
+    const float amax = __uint_as_float(*amax_word);
+    const float s_t = (FMT == kFmtNV && amax != 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+    const float c6 = __fmul_rn(6.0f, s_t);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *s_tw_out = s_t;
+    const int64_t cpr = k / 32, nblk = k / BLK, total = sf_rows * cpr;
+    for (int64_t t = (int64_t)blockIdx.x * kWThreads + threadIdx.x; t < total; t += (int64_t)gridDim.x * kWThreads) {
+        const int64_t row = t / cpr, c = t - row * cpr;
+        if (row >= n_out) {  // scale-layout padding rows
+            if (FMT == kFmtNV) *reinterpret_cast<uint16_t *>(sf + sf_offset(row, 2 * c, nblk)) = 0;
+            else sf[sf_offset(row, c, nblk)] = 0;
+            continue;
+        }
+        const uint4 *wp = reinterpret_cast<const uint4 *>(w + row * k + c * 32);
+        float v[32];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint4 u = __ldcs(wp + q);
+            const uint32_t ws[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[8 * q + i] = h2f((uint16_t)(ws[i / 2] >> (16 * (i % 2))));
+        }
+        uint32_t pk[4] = {0, 0, 0, 0}, sc[NB];
+#pragma unroll
+        for (int bk = 0; bk < NB; ++bk) {
+            float a = 0.0f;
+#pragma unroll
+            for (int i = bk * BLK; i < (bk + 1) * BLK; ++i) a = fmaxf(a, fabsf(v[i]));
+            uint32_t code;
+            const float d = block_step<FMT>(a, s_t, c6, code);
+            sc[bk] = code;
+            if (d != 0.0f) {
+#pragma unroll
+                for (int i = bk * BLK; i < (bk + 1) * BLK; i += 2)
+                    pk[i / 8] |= e2m1x2(__fdiv_rn(v[i], d), __fdiv_rn(v[i + 1], d)) << (4 * (i % 8));
+            }
+        }
+        *reinterpret_cast<uint4 *>(codes + row * (k / 2) + c * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        if (FMT == kFmtNV) *reinterpret_cast<uint16_t *>(sf + sf_offset(row, 2 * c, nblk)) = (uint16_t)(sc[0] | (sc[NB - 1] << 8));
+        else sf[sf_offset(row, c, nblk)] = (uint8_t)sc[0];
+    }
+}
+
+sharq_status launch_quantize_weight(LaunchCtx &ctx, const sharq_wq &W, const void *w) {
+    unsigned *words = reinterpret_cast<unsigned *>(W.tensor_scale) - 1;  // [0] amax bits, [1] s_tW
+    SQ_CUDA_TRY(cudaMemsetAsync(words, 0, sizeof(unsigned), ctx.stream));
+    const int64_t count = W.n_out * W.k;
+    int64_t blocks = (count / 8 + kWThreads - 1) / kWThreads;
+    if (blocks > (int64_t)ctx.num_sms * 4) blocks = (int64_t)ctx.num_sms * 4;
+    absmax_kernel<<<(unsigned)blocks, kWThreads, 0, ctx.stream>>>((const uint16_t *)w, count, words);
+    ctx.launches++;
+    const int64_t total = W.sf_rows * (W.k / 32);
+    int64_t eb = (total + kWThreads - 1) / kWThreads;
+    if (eb > (int64_t)ctx.num_sms * 8) eb = (int64_t)ctx.num_sms * 8;
+    if (W.fmt == kFmtNV)
+        wq_encode_kernel<kFmtNV><<<(unsigned)eb, kWThreads, 0, ctx.stream>>>(
+            (const uint16_t *)w, W.n_out, W.sf_rows, W.k, words, W.tensor_scale, (uint8_t *)W.codes,
+            (uint8_t *)W.scales_backbone);
+    else
+        wq_encode_kernel<kFmtMX><<<(unsigned)eb, kWThreads, 0, ctx.stream>>>(
+            (const uint16_t *)w, W.n_out, W.sf_rows, W.k, words, W.tensor_scale, (uint8_t *)W.codes,
+            (uint8_t *)W.scales_backbone);
+    ctx.launches++;
+    SQ_CUDA_TRY(cudaGetLastError());
+    return SHARQ_OK;
+}
+
+}  // namespace sq

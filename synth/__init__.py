@@ -9,8 +9,9 @@ Generator: counter-based splitmix64 (Steele, Lea & Flood, "Fast splittable
 pseudorandom number generators", OOPSLA 2014). Draw i of stream (seed, stream)
 is mix64(key + (i + 1) * GOLDEN) with key = mix64(seed * GOLDEN ^ stream).
 Uniforms take the top 53 bits. Normals come from the Box-Muller transform in
-fp64. All of it is plain numpy uint64/float64 arithmetic, so the bytes are
-identical on every host.
+fp64. The bulk generators run in synth.c (OpenMP over independent elements,
+so the bytes do not depend on the thread count); the *_np functions state the
+same definition in numpy and the tests hold the two equal.
 
 Workloads follow the SharQ abstract ("SharQ: Bridging Activation Sparsity and
 FP4 Quantization for LLM Inference", arXiv 2606.26587, abstract): the paper
@@ -19,10 +20,43 @@ used; only the layer shapes are, with outlier-heavy synthetic activations.
 """
 from __future__ import annotations
 
+import ctypes as C
 import math
+import os
+import subprocess
 from dataclasses import dataclass
 
 import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "synth.c")
+_LIB = os.path.join(_HERE, "libsynth.so")
+_clib = None
+
+
+def build(force: bool = False) -> str:
+    """Compiles synth.c (the hot loops below) into synth/libsynth.so."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.run(["gcc", "-O2", "-std=gnu11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+                        _SRC, "-o", _LIB + ".tmp", "-lm"], check=True)
+        os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+def _c():
+    global _clib
+    if _clib is None:
+        L = C.CDLL(build())
+        u64, i64, vp = C.c_uint64, C.c_int64, C.c_void_p
+        L.synth_normal.argtypes = [u64, u64, i64, i64, vp]
+        L.synth_student_fp16.argtypes = [u64, u64, i64, i64, i64, vp, vp]
+        L.synth_normal_fp16.argtypes = [u64, u64, i64, i64, i64, vp, vp]
+        _clib = L
+    return _clib
+
+
+def _vp(a):
+    return a.ctypes.data_as(C.c_void_p)
 
 GOLDEN = np.uint64(0x9E3779B97F4A7C15)
 _M1 = np.uint64(0xBF58476D1CE4E5B9)
@@ -60,6 +94,13 @@ def uniform(seed: int, stream: int, count: int) -> np.ndarray:
 
 def normal(seed: int, stream: int, count: int) -> np.ndarray:
     """N(0, 1) doubles by Box-Muller on pairs of uniforms (u1 in (0, 1])."""
+    out = np.empty(count, np.float64)
+    _c().synth_normal(seed, stream, 0, count, _vp(out))
+    return out
+
+
+def normal_np(seed: int, stream: int, count: int) -> np.ndarray:
+    """Pure-numpy statement of normal(), kept as the reference of synth.c."""
     pairs = (count + 1) // 2
     u = uniform(seed, stream, 2 * pairs)
     u1 = 1.0 - u[0::2]
@@ -72,9 +113,10 @@ def normal(seed: int, stream: int, count: int) -> np.ndarray:
     return out[:count]
 
 
-def student_t3(seed: int, stream: int, count: int) -> np.ndarray:
-    """Student-t with 3 degrees of freedom: Z / sqrt((Z1^2 + Z2^2 + Z3^2) / 3)."""
-    z = normal(seed, stream, 4 * count).reshape(count, 4)
+def student_t3_np(seed: int, stream: int, count: int) -> np.ndarray:
+    """Student-t with 3 degrees of freedom: Z / sqrt((Z1^2 + Z2^2 + Z3^2) / 3)
+    (pure-numpy reference of synth.c)."""
+    z = normal_np(seed, stream, 4 * count).reshape(count, 4)
     chi = (z[:, 1] ** 2 + z[:, 2] ** 2 + z[:, 3] ** 2) / 3.0
     return z[:, 0] / np.sqrt(chi)
 
@@ -93,29 +135,52 @@ def to_fp16(v: np.ndarray) -> np.ndarray:
 S_BODY, S_OUTLIER_PICK, S_OUTLIER_GAIN, S_WEIGHT, S_GATE, S_LN = 1, 2, 3, 4, 5, 6
 
 
-def activations_gaussian(seed: int, rows: int, k: int, n_outlier: int, gain: float) -> np.ndarray:
-    """X ~ N(0, 1) with n_outlier channels (seeded choice) multiplied by gain."""
-    x = normal(seed, S_BODY, rows * k).reshape(rows, k)
-    ch = permutation(seed, S_OUTLIER_PICK, k)[:n_outlier]
-    x[:, ch] *= gain
-    return to_fp16(x)
+def gaussian_gains(seed: int, k: int, n_outlier: int, gain: float) -> np.ndarray:
+    g = np.ones(k, np.float64)
+    g[permutation(seed, S_OUTLIER_PICK, k)[:n_outlier]] = gain
+    return g
+
+
+def student_gains(seed: int, k: int, outlier_frac: float = 0.01, gain_lo: float = 20.0,
+                  gain_hi: float = 100.0) -> np.ndarray:
+    n_out = int(math.ceil(outlier_frac * k))
+    g = np.ones(k, np.float64)
+    g[permutation(seed, S_OUTLIER_PICK, k)[:n_out]] = gain_lo + (gain_hi - gain_lo) * uniform(seed, S_OUTLIER_GAIN, n_out)
+    return g
+
+
+def activations_gaussian(seed: int, rows: int, k: int, n_outlier: int, gain: float, row0: int = 0) -> np.ndarray:
+    """X ~ N(0, 1) with n_outlier channels (seeded choice) multiplied by gain.
+    Rows row0 .. row0+rows-1 of the tensor of that seed."""
+    out = np.empty((rows, k), np.uint16)
+    _c().synth_normal_fp16(seed, S_BODY, row0, rows, k, _vp(gaussian_gains(seed, k, n_outlier, gain)), _vp(out))
+    return out.view(np.float16)
 
 
 def activations_student(seed: int, rows: int, k: int, outlier_frac: float = 0.01,
-                        gain_lo: float = 20.0, gain_hi: float = 100.0) -> np.ndarray:
+                        gain_lo: float = 20.0, gain_hi: float = 100.0, row0: int = 0) -> np.ndarray:
     """Student-t(3) body; ceil(outlier_frac * k) channels, fixed across tokens,
-    scaled by a per-channel gain drawn from U[gain_lo, gain_hi]."""
-    x = student_t3(seed, S_BODY, rows * k).reshape(rows, k)
-    n_out = int(math.ceil(outlier_frac * k))
-    ch = permutation(seed, S_OUTLIER_PICK, k)[:n_out]
-    gain = gain_lo + (gain_hi - gain_lo) * uniform(seed, S_OUTLIER_GAIN, n_out)
-    x[:, ch] *= gain[None, :]
+    scaled by a per-channel gain drawn from U[gain_lo, gain_hi]. Rows row0 ..
+    row0+rows-1 of the tensor of that seed."""
+    out = np.empty((rows, k), np.uint16)
+    g = student_gains(seed, k, outlier_frac, gain_lo, gain_hi)
+    _c().synth_student_fp16(seed, S_BODY, row0, rows, k, _vp(g), _vp(out))
+    return out.view(np.float16)
+
+
+def activations_student_np(seed: int, rows: int, k: int, outlier_frac: float = 0.01,
+                           gain_lo: float = 20.0, gain_hi: float = 100.0) -> np.ndarray:
+    """Pure-numpy statement of activations_student (reference of synth.c)."""
+    x = student_t3_np(seed, S_BODY, rows * k).reshape(rows, k)
+    x *= student_gains(seed, k, outlier_frac, gain_lo, gain_hi)[None, :]
     return to_fp16(x)
 
 
-def weights(seed: int, n_out: int, k: int, std: float = 0.02) -> np.ndarray:
+def weights(seed: int, n_out: int, k: int, std: float = 0.02, row0: int = 0) -> np.ndarray:
     """W ~ N(0, std^2), fp16, [n_out, k] row-major (K-major)."""
-    return to_fp16(std * normal(seed, S_WEIGHT, n_out * k).reshape(n_out, k))
+    out = np.empty((n_out, k), np.uint16)
+    _c().synth_normal_fp16(seed, S_WEIGHT, row0, n_out, k, _vp(np.full(k, std)), _vp(out))
+    return out.view(np.float16)
 
 
 def ln_params(seed: int, k: int) -> tuple[np.ndarray, np.ndarray]:

@@ -1,0 +1,186 @@
+"""Parity of the CUDA path with the CPU oracle at sizes the oracle finishes in
+seconds: several tiles plus ragged tails in M, N and K-chunks, every format,
+several N:M ratios, LayerNorm with and without affine parameters, and the
+degenerate inputs. Prep outputs must be bit-exact; the GEMM within
+1e-3 * sum|a||w| per element."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_common import (assert_linear_close, assert_prep_matches, assert_weight_matches, cuda16,
+                        gpu_prepare)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    import sparsity_gemm_b200 as sq
+    assert torch.cuda.is_available()
+    sq.lib()
+    yield
+
+
+def test_single_linear_16x256x256_nvfp4_2of4():
+    """The single-linear workload: X ~ N(0,1) with 4 of 256 channels x50,
+    W ~ N(0, 0.02^2), LayerNorm gamma=1 beta=0, NVFP4, 2:4."""
+    import sparsity_gemm_b200 as sq
+    x = synth.activations_gaussian(0, 16, 256, 4, 50.0)
+    w = synth.weights(1, 256, 256)
+    ones, zeros = np.ones(256, np.float16), np.zeros(256, np.float16)
+    op = oracle.prepare(x, ones, zeros, 1e-5, 2, 4, oracle.NVFP4)
+    p, ex = gpu_prepare(x, ones, zeros, 1e-5, 2, 4, sq.NVFP4)
+    assert_prep_matches(ex, op)
+    ow = oracle.quantize_weight(w, oracle.NVFP4)
+    qw = sq.quantize_weight(cuda16(w), sq.NVFP4)
+    assert_weight_matches(sq.weight_export(qw), ow)
+    out = sq.linear(p, qw).cpu().numpy()
+    want, bound = oracle.linear_prepared(op, ow)
+    assert_linear_close(out, want, bound)
+    assert sq.get_last_error() == sq.OK
+
+
+PREP_CASES = [
+    # (m_tok, k, fmt, n, m, affine)
+    (37, 256, 0, 2, 4, False),
+    (300, 512, 0, 2, 4, True),
+    (300, 512, 1, 2, 4, False),
+    (129, 768, 1, 4, 8, True),
+    (64, 512, 0, 4, 8, False),
+    (33, 256, 0, 1, 2, False),
+    (33, 256, 1, 3, 8, True),   # m = 8 with odd n: metadata chunks share bytes
+    (17, 512, 0, 5, 8, False),
+    (40, 512, 0, 8, 16, True),
+    (40, 512, 1, 4, 4, False),  # n = m: plain quantization
+    (24, 256, 0, 1, 4, False),
+    (9, 1024, 1, 16, 16, True),
+]
+
+
+@pytest.mark.parametrize("m_tok,k,fmt,n,m,affine", PREP_CASES)
+def test_prepare_bit_exact(m_tok, k, fmt, n, m, affine):
+    x = synth.activations_student(100 + m_tok + k + n * 7 + m, m_tok, k)
+    g, b = synth.ln_params(5, k) if affine else (None, None)
+    op = oracle.prepare(x, g, b, 1e-5, n, m, fmt)
+    _, ex = gpu_prepare(x, g, b, 1e-5, n, m, fmt)
+    assert_prep_matches(ex, op)
+
+
+@pytest.mark.parametrize("n_out,k,fmt", [(32, 256, 0), (544, 512, 0), (544, 512, 1), (256, 1024, 1)])
+def test_weight_quantization_bit_exact(n_out, k, fmt):
+    import sparsity_gemm_b200 as sq
+    w = synth.weights(7 + n_out, n_out, k)
+    ow = oracle.quantize_weight(w, fmt)
+    qw = sq.quantize_weight(cuda16(w), fmt)
+    assert_weight_matches(sq.weight_export(qw), ow)
+
+
+LINEAR_CASES = [
+    # (m_tok, n_out, k, fmt, n, m)
+    (16, 256, 256, 0, 2, 4),
+    (300, 544, 512, 0, 2, 4),   # ragged M (3 tiles) and N (2 tiles + 32)
+    (300, 544, 512, 1, 2, 4),
+    (1, 256, 256, 0, 2, 4),
+    (129, 512, 1024, 0, 4, 8),
+    (129, 512, 1024, 1, 4, 8),
+    (256, 288, 768, 0, 1, 2),
+    (45, 1024, 2048, 0, 2, 4),  # 8 K tiles, more than the pipeline depth
+]
+
+
+@pytest.mark.parametrize("m_tok,n_out,k,fmt,n,m", LINEAR_CASES)
+def test_linear_within_tolerance(m_tok, n_out, k, fmt, n, m):
+    import sparsity_gemm_b200 as sq
+    x = synth.activations_student(200 + m_tok, m_tok, k)
+    w = synth.weights(300 + n_out, n_out, k)
+    op = oracle.prepare(x, None, None, 1e-5, n, m, fmt)
+    ow = oracle.quantize_weight(w, fmt)
+    p, ex = gpu_prepare(x, None, None, 1e-5, n, m, fmt)
+    assert_prep_matches(ex, op)
+    qw = sq.quantize_weight(cuda16(w), fmt)
+    out = sq.linear(p, qw).cpu().numpy()
+    want, bound = oracle.linear_prepared(op, ow)
+    assert_linear_close(out, want, bound)
+    assert sq.get_last_error() == sq.OK
+
+
+def test_empty_activation():
+    import sparsity_gemm_b200 as sq
+    x = np.zeros((0, 256), np.float16)
+    p = sq.prepare(torch.zeros((0, 256), dtype=torch.float16, device="cuda"), None, None, 1e-5, 2, 4, sq.NVFP4)
+    assert sq.prep_export(p)["s_t"] == 1.0
+    qw = sq.quantize_weight(cuda16(synth.weights(1, 256, 256)), sq.NVFP4)
+    out = sq.linear(p, qw)
+    assert out.shape == (0, 256)
+    assert sq.get_last_error() == sq.OK
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_degenerate_rows(fmt):
+    """All-zero tensor (tensor scale 1), constant rows (variance 0), -0
+    entries, fp16 extremes (65504 and subnormals)."""
+    import sparsity_gemm_b200 as sq
+    zero = np.zeros((5, 256), np.float16)
+    op = oracle.prepare(zero, None, None, 1e-5, 2, 4, fmt)
+    _, ex = gpu_prepare(zero, None, None, 1e-5, 2, 4, fmt)
+    assert_prep_matches(ex, op)
+    assert ex["s_t"] == 1.0
+
+    x = synth.activations_student(9, 6, 512)
+    x[0] = np.float16(3.5)                       # constant row
+    x[1, ::2] = np.float16(65504.0)              # extremes
+    x[1, 1::2] = np.float16(-65504.0)
+    x[2] = 0
+    x[2].view(np.uint16)[::3] = 0x8000            # -0 entries
+    x[3].view(np.uint16)[:] = np.arange(512, dtype=np.uint16) % 64 + 1  # fp16 subnormals
+    x[4].view(np.uint16)[::2] |= 0x8000
+    op = oracle.prepare(x, None, None, 1e-5, 2, 4, fmt)
+    _, ex = gpu_prepare(x, None, None, 1e-5, 2, 4, fmt)
+    assert_prep_matches(ex, op)
+
+
+def test_all_zero_weight():
+    import sparsity_gemm_b200 as sq
+    w = np.zeros((64, 256), np.float16)
+    ow = oracle.quantize_weight(w, 0)
+    qw = sq.quantize_weight(cuda16(w), 0)
+    assert_weight_matches(sq.weight_export(qw), ow)
+    assert ow.s_tw == 1.0
+
+
+def test_launch_counts_and_no_host_sync():
+    import sparsity_gemm_b200 as sq
+    x = cuda16(synth.activations_student(1, 64, 512))
+    p = sq.prepare(x, None, None, 1e-5, 2, 4, sq.NVFP4)
+    assert sq.last_launch_count() == 2
+    qw = sq.quantize_weight(cuda16(synth.weights(2, 256, 512)), sq.NVFP4)
+    assert sq.last_launch_count() == 2
+    sq.linear(p, qw)
+    assert sq.last_launch_count() == 1
+    assert sq.get_last_error() == sq.OK
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait on a barrier nothing arrives at runs out after its limit; the
+    status comes back as SHARQ_ERR_TIMEOUT and the context stays usable."""
+    import sparsity_gemm_b200 as sq
+    assert sq.get_last_error() == sq.OK
+    sq.selftest_wait(50_000_000)  # 50 ms
+    assert sq.get_last_error() == sq.ERR_TIMEOUT
+    assert sq.last_timeout_site() == 0x1FF
+    assert sq.get_last_error() == sq.OK  # cleared
+    test_single_linear_16x256x256_nvfp4_2of4()
+
+
+def test_results_do_not_depend_on_stream_or_buffer_reuse():
+    import sparsity_gemm_b200 as sq
+    x = synth.activations_student(77, 200, 512)
+    p1, ex1 = gpu_prepare(x, None, None, 1e-5, 2, 4, 0)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        p2 = sq.prepare(cuda16(x), None, None, 1e-5, 2, 4, 0, out=p1, stream=s)
+        ex2 = sq.prep_export(p2, stream=s)
+    for key in ex1:
+        np.testing.assert_array_equal(np.asarray(ex1[key]), np.asarray(ex2[key]))

@@ -48,3 +48,19 @@ def test_moe_routing_shapes():
         assert np.all(np.diff(seg) > 0)
     counts = np.bincount(row_idx, minlength=64)
     assert np.all(counts == 4)
+
+
+def test_c_generator_matches_numpy_statement():
+    a = synth.activations_student(3, 16, 512)
+    b = synth.activations_student_np(3, 16, 512)
+    assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+    z = synth.normal(5, 1, 10001)
+    assert np.allclose(z, synth.normal_np(5, 1, 10001), rtol=0, atol=1e-12)
+
+
+def test_row_slices_are_independent():
+    full = synth.activations_student(8, 40, 256)
+    part = synth.activations_student(8, 7, 256, row0=20)
+    assert np.array_equal(full[20:27].view(np.uint16), part.view(np.uint16))
+    w = synth.weights(9, 64, 256)
+    assert np.array_equal(w[32:].view(np.uint16), synth.weights(9, 32, 256, row0=32).view(np.uint16))
