@@ -55,6 +55,10 @@ def parse_args():
     ap.add_argument("--cpu-sample-tokens", type=int, default=1)
     ap.add_argument("--cpu-sample-cols", type=int, default=512,
                     help="output columns of each linear in the CPU sample (cost is linear in columns)")
+    ap.add_argument("--case", default=None,
+                    help="time one op instead of the layer set: prep:M:K[:fmt:n:m] or linear:M:N:K[:fmt:n:m] "
+                         "(fmt 0 = NVFP4, 1 = MXFP4); used for profiling and shape sweeps")
+    ap.add_argument("--outlier-frac", type=float, default=0.01)
     return ap.parse_args()
 
 
@@ -427,11 +431,73 @@ def run_reference(args, world, rank):
             "gpu_launches": 0}
 
 
+def run_case(args, world, rank, local):
+    """One op on one shape: W warm-up and K timed launches, L2 flushed before
+    each, CUDA events on the launching stream. Prints a JSON line with the
+    op's time and its roofline figure."""
+    import sparsity_gemm_b200 as sq
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    parts = args.case.split(":")
+    kind = parts[0]
+    nums = [int(v) for v in parts[1:]]
+    peaks, peak_src = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    if kind == "prep":
+        M, K = nums[:2]
+        fmt, n, m = (nums[2:5] + [0, N_KEEP, M_GROUP][len(nums[2:5]):])
+        x = torch.from_numpy(synth.activations_student(0, M, K, outlier_frac=args.outlier_frac).view(np.float16)).to(dev)
+        buf = sq.prepare(x, None, None, EPS, n, m, fmt)
+        op = lambda: sq.prepare(x, None, None, EPS, n, m, fmt, out=buf)
+        meta = (K // m) * n * max(1, (m - 1).bit_length()) / 8.0 / K
+        per_elem = 2 + 0.5 + meta + 2.0 / (16 if fmt == 0 else 32) + 0.5
+        work, unit, peak, bound = per_elem * M * K, "GB/s", peaks["hbm_gbs"], "hbm"
+    elif kind == "linear":
+        M, N, K = nums[:3]
+        fmt, n, m = (nums[3:6] + [0, N_KEEP, M_GROUP][len(nums[3:6]):])
+        x = torch.from_numpy(synth.activations_student(0, M, K, outlier_frac=args.outlier_frac).view(np.float16)).to(dev)
+        w = torch.from_numpy(synth.weights(1000, N, K).view(np.float16)).to(dev)
+        qw = sq.quantize_weight(w, fmt)
+        prep = sq.prepare(x, None, None, EPS, n, m, fmt)
+        out = torch.empty((M, N), dtype=torch.float16, device=dev)
+        op = lambda: sq.linear(prep, qw, out=out)
+        work, unit, bound = 2.0 * M * N * K * (1.0 + n / m), "TFLOP/s", "tensor"
+        peak = peaks["bf16_tflops"] * FP4_OVER_BF16 * 1e3  # in GFLOP/s, scaled below
+    else:
+        raise SystemExit(f"unknown case {args.case}")
+    for _ in range(args.warmup):
+        flush.zero_()
+        op()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        op()
+        b.record(stream)
+    torch.cuda.synchronize()
+    st = sq.get_last_error()
+    if st != sq.OK:
+        raise RuntimeError(sq.status_name(st))
+    ms = [a.elapsed_time(b) for a, b in evs]
+    t = statistics.median(ms) / 1e3
+    achieved = work / t / 1e9  # GB/s or GFLOP/s
+    if unit == "TFLOP/s":
+        achieved /= 1e3
+        peak /= 1e3
+    return {"case": args.case, "ms_median": t * 1e3, "ms_min": min(ms), "achieved": achieved, "unit": unit,
+            "peak": peak, "frac": achieved / peak, "bound": bound, "steps": args.steps,
+            "outlier_frac": args.outlier_frac, "peak_source": peak_src}
+
+
 def main():
     args = parse_args()
     world, rank, local = dist_setup(args)
     try:
-        if args.impl == "reference":
+        if args.case:
+            res = run_case(args, world, rank, local)
+        elif args.impl == "reference":
             res = run_reference(args, world, rank)
         else:
             res = run_sharq(args, world, rank, local)

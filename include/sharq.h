@@ -231,6 +231,20 @@ uint64_t sharq_set_wait_limit_ns(uint64_t ns);
  * sharq_get_last_error must report SHARQ_ERR_TIMEOUT. */
 sharq_status sharq_selftest_wait(uint64_t limit_ns, void *stream);
 
+/* Self-test of the quantizer's division: the encode kernels divide by a
+ * block step d with a reciprocal and two fused multiply-add corrections
+ * (Markstein's method), which must equal the correctly rounded quotient.
+ * Runs `count` operand pairs drawn from `seed` (divisors in [2^-90, 2^90],
+ * quotients of exponent -30 .. 30, many near the E2M1 rounding boundaries)
+ * on the GPU and writes to *mismatches_host how many quotients of magnitude
+ * >= 2^-4 differ from the hardware's correctly rounded division, plus how
+ * many quotients of any size encode to a different E2M1 code (expected: 0). If examples_host is not NULL
+ * it receives 16 x 4 floats: the first mismatching (dividend, divisor,
+ * quotient, correctly rounded quotient) rows, zeros past the count.
+ * Synchronizes `stream`. */
+sharq_status sharq_selftest_division(uint64_t count, uint64_t seed, uint64_t *mismatches_host,
+                                     float *examples_host, void *stream);
+
 /* Human-readable status name (static string). */
 const char *sharq_status_string(sharq_status s);
 

@@ -73,6 +73,8 @@ def lib():
         L.sharq_set_wait_limit_ns.restype = C.c_uint64
         L.sharq_selftest_wait.argtypes = [C.c_uint64, vp]
         L.sharq_selftest_wait.restype = i32
+        L.sharq_selftest_division.argtypes = [C.c_uint64, C.c_uint64, C.POINTER(C.c_uint64), vp, vp]
+        L.sharq_selftest_division.restype = i32
         L.sharq_status_string.argtypes = [i32]
         L.sharq_status_string.restype = C.c_char_p
         L.sharq_last_launch_count.restype = i32
@@ -221,6 +223,16 @@ def get_last_error(stream=None) -> int:
 def selftest_wait(limit_ns: int, stream=None) -> None:
     """Enqueues the bounded-wait probe (see sharq_selftest_wait)."""
     _check(lib().sharq_selftest_wait(int(limit_ns), _stream(stream)), "sharq_selftest_wait")
+
+
+def selftest_division(count: int, seed: int = 1, stream=None, examples: bool = False):
+    """Mismatches of the encode kernels' division against div.rn (expected 0);
+    with examples=True also the first mismatching rows (v, d, q, reference)."""
+    out = C.c_uint64(0)
+    ex = np.zeros((16, 4), np.float32)
+    _check(lib().sharq_selftest_division(int(count), int(seed), C.byref(out), ex.ctypes.data_as(C.c_void_p),
+                                         _stream(stream)), "sharq_selftest_division")
+    return (int(out.value), ex) if examples else int(out.value)
 
 
 def last_timeout_site() -> int:

@@ -18,7 +18,7 @@ HEADERS = ["layout.h", "sharq_dev.cuh", "sq_internal.h", os.path.join("..", ".."
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
-    "-lineinfo", "-O3", "-std=c++17",
+    "-lineinfo", "-O3", "-std=c++17", "-fmad=false",
     "-Xcompiler", "-fPIC", "-shared",
     "-cudart", "shared",
     "-Xlinker", "-rpath=/usr/local/cuda/lib64",

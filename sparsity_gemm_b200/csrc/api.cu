@@ -272,6 +272,18 @@ sharq_status sharq_selftest_wait(uint64_t limit_ns, void *stream) {
     return st;
 }
 
+sharq_status sharq_selftest_division(uint64_t count, uint64_t seed, uint64_t *mismatches_host, float *examples_host,
+                                     void *stream) {
+    g_last_launches = 0;
+    if (!mismatches_host || count == 0) return SHARQ_ERR_INVALID_ARG;
+    sq::LaunchCtx ctx;
+    sharq_status st = make_ctx(stream, ctx);
+    if (st != SHARQ_OK) return st;
+    st = sq::launch_div_check(ctx, count, seed, mismatches_host, examples_host);
+    g_last_launches = ctx.launches;
+    return st;
+}
+
 sharq_status sharq_get_last_error(void *stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SHARQ_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return SHARQ_ERR_CUDA;

@@ -8,11 +8,14 @@
 // Two passes over the activations, because the NVFP4 tensor scale depends on
 // amax(X_ln) over the whole tensor:
 //   1. ln_stats_kernel (one CTA per row): exact LayerNorm statistics from
-//      integer sums, then amax|X_ln| of the row (row cached in shared memory),
-//      folded into one global word by an atomic max.
-//   2. prep_encode_kernel (one thread per 32-element chunk): LayerNorm apply,
-//      top-n-of-m selection, Q(S), R = X_ln - deq(Q(S)), Q(R), and packed
-//      code / scale / metadata stores. The second read of x mostly hits L2.
+//      integer sums and the row's amax|X_ln|, folded into one global word by
+//      an atomic max. Without gamma/beta, X_ln is a non-decreasing function of
+//      x within a row, so amax|X_ln| comes from the row's min and max of x;
+//      with gamma/beta the row is kept in shared memory and swept again.
+//   2. prep_encode_kernel (one thread per 16 consecutive elements; an MXFP4
+//      block of 32 spans a lane pair): LayerNorm apply, top-n-of-m selection,
+//      Q(S), R = X_ln - deq(Q(S)), Q(R), and packed code / scale / metadata
+//      stores. The second read of x mostly hits L2.
 #include <cuda_fp16.h>
 
 #include "sharq_dev.cuh"
@@ -22,32 +25,38 @@ namespace sq {
 
 constexpr int kStatsThreads = 256;
 constexpr int kEncodeThreads = 256;
+constexpr int kUnit = 16;  // elements per encode thread
 
 // ---------------------------------------------------------------------------
-// Exact statistics. With a = x * 2^24 (an integer, |a| < 2^40), split
-// |a| = hi * 2^20 + lo (hi, lo < 2^20). Then
-//   S1 = sum(+-a),   S2 = sum a^2 = 2^40 sum hi^2 + 2^21 sum hi*lo + sum lo^2,
-// where every partial sum fits a 64-bit integer for k <= 2^16.
+// Exact statistics. With a = x * 2^24 (an integer, |a| < 2^40), write
+// t = x * 2^4 = hi + lo * 2^-20 with hi = floor(t) (|hi| <= 2^20, signed) and
+// 0 <= lo < 2^20, so that a = hi * 2^20 + lo and
+//   S1 = 2^20 sum hi + sum lo,
+//   S2 = 2^40 sum hi^2 + 2^21 sum hi*lo + sum lo^2.
+// hi and lo come out of the binary32 pipeline exactly: t + 1.5*2^23 rounded
+// toward -inf holds floor(t) in its low mantissa bits, and (t - floor(t)) *
+// 2^20 + 2^23 holds lo in its low mantissa bits (every step is exact).
 struct ExactSums {
-    int64_t s1;
-    uint64_t hh, hl, ll;
+    int64_t hi, lo;  // sum hi, sum lo
+    int64_t hh, hl;  // sum hi^2, sum hi*lo
+    uint64_t ll;     // sum lo^2
 };
 
-__device__ __forceinline__ void accum_half(uint32_t h, ExactSums &e) {
-    float t = __fmul_rn(fabsf(h2f((uint16_t)h)), 16.0f);                        // |x| * 2^4, exact
-    float hf = floorf(t);
-    uint32_t hi = (uint32_t)hf;                                                // < 2^20
-    uint32_t lo = (uint32_t)__fmul_rn(__fsub_rn(t, hf), 1048576.0f);           // < 2^20, exact
-    int64_t a = (int64_t)(((uint64_t)hi << 20) | lo);
-    e.s1 += (h & 0x8000u) ? -a : a;
-    e.hh += (uint64_t)hi * hi;
-    e.hl += (uint64_t)hi * lo;
-    e.ll += (uint64_t)lo * lo;
-}
-
-__device__ __forceinline__ void accum_word(uint32_t w, ExactSums &e) {
-    accum_half(w & 0xFFFFu, e);
-    accum_half(w >> 16, e);
+__device__ __forceinline__ void accum_pair(uint32_t w, ExactSums &e) {
+    // The product x * 2^4 is exact, so fusing it into the following add is harmless.
+    const uint64_t t = mul2(h2_to_f2(w), pk2(16.0f, 16.0f));             // x * 2^4, exact
+    const uint64_t hm = add2_rm(t, pk2(12582912.0f, 12582912.0f));      // 1.5*2^23 + floor(t)
+    const uint64_t hf = sub2(hm, pk2(12582912.0f, 12582912.0f));        // floor(t), exact
+    const uint64_t lm = fma2(sub2(t, hf), pk2(1048576.0f, 1048576.0f),  // frac * 2^20 + 2^23, exact
+                             pk2(8388608.0f, 8388608.0f));
+    const float2 hmf = up2(hm), lmf = up2(lm);
+    const int32_t h0 = (int32_t)__float_as_uint(hmf.x) - 0x4B400000, h1 = (int32_t)__float_as_uint(hmf.y) - 0x4B400000;
+    const int32_t l0 = (int32_t)(__float_as_uint(lmf.x) & 0x7FFFFFu), l1 = (int32_t)(__float_as_uint(lmf.y) & 0x7FFFFFu);
+    e.hi += h0 + h1;
+    e.lo += l0 + l1;
+    e.hh += (int64_t)h0 * h0 + (int64_t)h1 * h1;
+    e.hl += (int64_t)h0 * l0 + (int64_t)h1 * l1;
+    e.ll += (uint64_t)(uint32_t)l0 * (uint32_t)l0 + (uint64_t)(uint32_t)l1 * (uint32_t)l1;
 }
 
 // Round-to-nearest-even binary64 value of a non-negative 128-bit integer.
@@ -64,13 +73,26 @@ __device__ double u128_to_f64(unsigned __int128 v) {
     return __dmul_rn(__ull2double_rn((uint64_t)q), scale);
 }
 
+// mu = RN32(RN64(S1) / (K 2^24)); rstd = RN32(1 / sqrt(RN64(D) / (K^2 2^48) + eps)).
+__device__ float2 finish_stats(const ExactSums &e, int64_t k, float eps) {
+    const __int128 s1 = (__int128)e.hi * 1048576 + e.lo;
+    const __int128 s2 = ((__int128)e.hh << 40) + ((__int128)e.hl << 21) + (__int128)e.ll;
+    const __int128 d = (__int128)k * s2 - s1 * s1;
+    const double kd = (double)k;
+    const double mean64 = __ddiv_rn(__ll2double_rn((long long)s1), __dmul_rn(kd, 16777216.0));
+    const double var64 = __ddiv_rn(u128_to_f64((unsigned __int128)d), __dmul_rn(__dmul_rn(kd, kd), 281474976710656.0));
+    return make_float2(__double2float_rn(mean64),
+                       __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(var64, (double)eps)))));
+}
+
+template <bool AFFINE>
 __global__ void __launch_bounds__(kStatsThreads)
 ln_stats_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gamma,
                 const uint16_t *__restrict__ beta, float eps, int64_t k, float2 *__restrict__ stats,
                 unsigned *__restrict__ amax_word) {
-    extern __shared__ uint4 row_cache[];  // k / 8 vectors of 8 halves
-    __shared__ int64_t red_s1[kStatsThreads / 32];
-    __shared__ uint64_t red_hh[kStatsThreads / 32], red_hl[kStatsThreads / 32], red_ll[kStatsThreads / 32];
+    extern __shared__ uint4 row_cache[];  // AFFINE only: k / 8 vectors of 8 halves
+    __shared__ ExactSums red[kStatsThreads / 32];
+    __shared__ uint32_t red_mx[kStatsThreads / 32], red_mn[kStatsThreads / 32];
     __shared__ float red_max[kStatsThreads / 32];
     __shared__ float2 row_stat;
 
@@ -79,66 +101,88 @@ ln_stats_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gam
     const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * k);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-    ExactSums e = {0, 0, 0, 0};
+    ExactSums e = {0, 0, 0, 0, 0};
+    uint32_t mx = 0xFC00FC00u, mn = 0x7C007C00u;  // (-inf, -inf), (+inf, +inf) as half2
     for (int c = threadIdx.x; c < nvec; c += kStatsThreads) {
-        uint4 v = xr[c];  // default caching: the encode pass re-reads x from L2
-        row_cache[c] = v;
-        accum_word(v.x, e);
-        accum_word(v.y, e);
-        accum_word(v.z, e);
-        accum_word(v.w, e);
+        const uint4 v = xr[c];  // default caching: the encode pass re-reads x from L2
+        if (AFFINE) row_cache[c] = v;
+        accum_pair(v.x, e);
+        accum_pair(v.y, e);
+        accum_pair(v.z, e);
+        accum_pair(v.w, e);
+        if (!AFFINE) {
+            asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(v.x));
+            asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(v.y));
+            asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(v.z));
+            asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(v.w));
+            asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(v.x));
+            asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(v.y));
+            asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(v.z));
+            asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(v.w));
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-        e.s1 += __shfl_xor_sync(0xFFFFFFFFu, e.s1, o);
+        e.hi += __shfl_xor_sync(0xFFFFFFFFu, e.hi, o);
+        e.lo += __shfl_xor_sync(0xFFFFFFFFu, e.lo, o);
         e.hh += __shfl_xor_sync(0xFFFFFFFFu, e.hh, o);
         e.hl += __shfl_xor_sync(0xFFFFFFFFu, e.hl, o);
         e.ll += __shfl_xor_sync(0xFFFFFFFFu, e.ll, o);
+        if (!AFFINE) {
+            const uint32_t omx = __shfl_xor_sync(0xFFFFFFFFu, mx, o), omn = __shfl_xor_sync(0xFFFFFFFFu, mn, o);
+            asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(omx));
+            asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(omn));
+        }
     }
     if (lane == 0) {
-        red_s1[warp] = e.s1;
-        red_hh[warp] = e.hh;
-        red_hl[warp] = e.hl;
-        red_ll[warp] = e.ll;
+        red[warp] = e;
+        red_mx[warp] = mx;
+        red_mn[warp] = mn;
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        int64_t s1 = 0;
-        uint64_t hh = 0, hl = 0, ll = 0;
-        for (int w = 0; w < kStatsThreads / 32; ++w) {
-            s1 += red_s1[w];
-            hh += red_hh[w];
-            hl += red_hl[w];
-            ll += red_ll[w];
+        ExactSums t = red[0];
+        uint32_t tmx = red_mx[0], tmn = red_mn[0];
+        for (int w = 1; w < kStatsThreads / 32; ++w) {
+            t.hi += red[w].hi;
+            t.lo += red[w].lo;
+            t.hh += red[w].hh;
+            t.hl += red[w].hl;
+            t.ll += red[w].ll;
+            asm("max.f16x2 %0, %0, %1;" : "+r"(tmx) : "r"(red_mx[w]));
+            asm("min.f16x2 %0, %0, %1;" : "+r"(tmn) : "r"(red_mn[w]));
         }
-        unsigned __int128 s2 = ((unsigned __int128)hh << 40) + ((unsigned __int128)hl << 21) + ll;
-        __int128 d = (__int128)k * (__int128)s2 - (__int128)s1 * (__int128)s1;
-        double kd = (double)k;
-        double mean64 = __ddiv_rn(__ll2double_rn(s1), __dmul_rn(kd, 16777216.0));
-        double var64 = __ddiv_rn(u128_to_f64((unsigned __int128)d), __dmul_rn(__dmul_rn(kd, kd), 281474976710656.0));
-        float mu = __double2float_rn(mean64);
-        float rstd = __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(var64, (double)eps))));
-        row_stat = make_float2(mu, rstd);
-        stats[row] = row_stat;
+        const float2 st = finish_stats(t, k, eps);
+        stats[row] = st;
+        row_stat = st;
+        if (!AFFINE) {
+            // X_ln = RN(RN(x - mu) * rstd) is non-decreasing in x: the row's
+            // amax|X_ln| is reached at its smallest or largest x.
+            const float xmax = fmaxf(h2f((uint16_t)tmx), h2f((uint16_t)(tmx >> 16)));
+            const float xmin = fminf(h2f((uint16_t)tmn), h2f((uint16_t)(tmn >> 16)));
+            const float a = fmaxf(fabsf(__fmul_rn(__fsub_rn(xmax, st.x), st.y)),
+                                  fabsf(__fmul_rn(__fsub_rn(xmin, st.x), st.y)));
+            atomicMax(amax_word, __float_as_uint(a));  // non-negative floats order like their bits
+        }
     }
+    if (!AFFINE) return;
     __syncthreads();
     const float mu = row_stat.x, rstd = row_stat.y;
     const bool has_g = gamma != nullptr, has_b = beta != nullptr;
     float amax = 0.0f;
     for (int c = threadIdx.x; c < nvec; c += kStatsThreads) {
-        uint4 v = row_cache[c];
-        uint4 g = has_g ? __ldg(reinterpret_cast<const uint4 *>(gamma) + c) : make_uint4(0, 0, 0, 0);
-        uint4 b = has_b ? __ldg(reinterpret_cast<const uint4 *>(beta) + c) : make_uint4(0, 0, 0, 0);
+        const uint4 v = row_cache[c];
+        const uint4 g = has_g ? __ldg(reinterpret_cast<const uint4 *>(gamma) + c) : make_uint4(0, 0, 0, 0);
+        const uint4 b = has_b ? __ldg(reinterpret_cast<const uint4 *>(beta) + c) : make_uint4(0, 0, 0, 0);
         const uint32_t xv[4] = {v.x, v.y, v.z, v.w}, gv[4] = {g.x, g.y, g.z, g.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 4; ++q)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                float xl = ln_apply(h2f((uint16_t)(xv[q] >> (16 * h))), mu, rstd, has_g,
-                                    h2f((uint16_t)(gv[q] >> (16 * h))), has_b, h2f((uint16_t)(bv[q] >> (16 * h))));
+                const float xl = ln_apply(h2f((uint16_t)(xv[q] >> (16 * h))), mu, rstd, has_g,
+                                          h2f((uint16_t)(gv[q] >> (16 * h))), has_b, h2f((uint16_t)(bv[q] >> (16 * h))));
                 amax = fmaxf(amax, fabsf(xl));
             }
-        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
@@ -147,20 +191,20 @@ ln_stats_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gam
     if (threadIdx.x == 0) {
         float a = 0.0f;
         for (int w = 0; w < kStatsThreads / 32; ++w) a = fmaxf(a, red_max[w]);
-        atomicMax(amax_word, __float_as_uint(a));  // non-negative floats order like their bits
+        atomicMax(amax_word, __float_as_uint(a));
     }
 }
 
 // ---------------------------------------------------------------------------
 // Encode pass.
 
-// Store `nbytes` (<= 16) little-endian bytes of (hi:lo) at p, using the widest
+// Store `nbytes` (<= 8) little-endian bytes of v at p, using the widest
 // aligned stores the address allows.
-__device__ __forceinline__ void store_bits(uint8_t *p, uint64_t lo, uint64_t hi, int nbytes) {
+__device__ __forceinline__ void store_bytes(uint8_t *p, uint64_t v, int nbytes) {
     int i = 0;
     while (i < nbytes) {
-        uint64_t w = i < 8 ? (lo >> (8 * i)) | (i ? (hi << (64 - 8 * i)) : 0) : hi >> (8 * (i - 8));
-        uintptr_t a = reinterpret_cast<uintptr_t>(p + i);
+        const uintptr_t a = reinterpret_cast<uintptr_t>(p + i);
+        const uint64_t w = v >> (8 * i);
         if (nbytes - i >= 4 && (a & 3) == 0) {
             *reinterpret_cast<uint32_t *>(p + i) = (uint32_t)w;
             i += 4;
@@ -174,14 +218,92 @@ __device__ __forceinline__ void store_bits(uint8_t *p, uint64_t lo, uint64_t hi,
     }
 }
 
-// Append a `bits`-wide field at bit position pos of a 128-bit stream.
-__device__ __forceinline__ void put_bits(uint64_t &lo, uint64_t &hi, uint32_t val, int bits, int pos) {
-    if (pos < 64) {
-        lo |= (uint64_t)val << pos;
-        if (pos + bits > 64) hi |= (uint64_t)val >> (64 - pos);
-    } else {
-        hi |= (uint64_t)val << (pos - 64);
+// OR `bits` (<= 64) bits of v into the bit stream at bit position `pos` from
+// a 4-byte-aligned base, with word atomics (neighbouring units share words).
+__device__ __forceinline__ void or_bits(uint32_t *base, uint64_t pos, uint64_t v, int bits) {
+    uint64_t w = pos >> 5;
+    int sh = (int)(pos & 31);
+    int done = 0;
+    while (done < bits) {
+        const uint32_t piece = (uint32_t)((v >> done) << sh);
+        const int take = 32 - sh < bits - done ? 32 - sh : bits - done;
+        const uint32_t mask = take >= 32 ? 0xFFFFFFFFu : (((1u << take) - 1u) << sh);
+        if (piece & mask) atomicOr(base + w, piece & mask);
+        done += take;
+        sh = 0;
+        ++w;
     }
+}
+
+// Keep mask of the 16 values of a unit: in every aligned group of M, the n
+// largest magnitudes, equal magnitudes to the lower index. The rank of value
+// i counts the values that beat it: larger, or equal at a lower index.
+template <int M>
+__device__ __forceinline__ uint32_t keep_mask(const float (&v)[kUnit], int n) {
+    uint32_t keep = 0;
+#pragma unroll
+    for (int g = 0; g < kUnit / M; ++g) {
+        uint32_t a[M];
+        int rank[M];
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+            a[i] = __float_as_uint(v[g * M + i]) & 0x7FFFFFFFu;
+            rank[i] = 0;
+        }
+#pragma unroll
+        for (int i = 0; i < M; ++i)
+#pragma unroll
+            for (int j = i + 1; j < M; ++j) {
+                const int c = a[i] >= a[j];  // i beats j
+                rank[j] += c;
+                rank[i] += 1 - c;
+            }
+#pragma unroll
+        for (int i = 0; i < M; ++i) keep |= (uint32_t)(rank[i] < n) << (g * M + i);
+    }
+    return keep;
+}
+
+// Block quantization of one thread's 16 values (an NVFP4 block, or half of an
+// MXFP4 block whose other half sits in the neighbouring lane). Produces the
+// scale code, the step d and the 16 E2M1 codes (8 bytes).
+template <int FMT>
+__device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, float c6, uint32_t &scale_code,
+                                            uint32_t &codes_lo, uint32_t &codes_hi) {
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kUnit; ++i) a = fmaxf(a, fabsf(v[i]));
+    if (FMT == kFmtMX) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
+    const float d = block_step<FMT>(a, s_t, c6, scale_code);
+    uint32_t c[2] = {0u, 0u};
+    if (d != 0.0f) {
+        if (FMT == kFmtMX) {
+            const float inv = pow2f(-mx_exponent(a));  // division by 2^e is this exact product
+            const uint64_t y2 = pk2(inv, inv);
+#pragma unroll
+            for (int i = 0; i < kUnit; i += 2) {
+                const uint64_t q = mul2(pk2(v[i], v[i + 1]), y2);
+                c[i / 8] |= e2m1_pair(q, __float_as_uint(v[i]), __float_as_uint(v[i + 1])) << (4 * (i % 8));
+            }
+        } else if (d >= 0x1p-90f && d <= 0x1p90f) {
+            const float y = __frcp_rn(d);
+            const uint64_t y2 = pk2(y, y), nd2 = pk2(-d, -d), d2 = pk2(d, d);
+#pragma unroll
+            for (int i = 0; i < kUnit; i += 2) {
+                const uint64_t q = div2(pk2(v[i], v[i + 1]), d2, nd2, y2);
+                c[i / 8] |= e2m1_pair(q, __float_as_uint(v[i]), __float_as_uint(v[i + 1])) << (4 * (i % 8));
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < kUnit; i += 2) {
+                const uint64_t q = pk2(__fdiv_rn(v[i], d), __fdiv_rn(v[i + 1], d));
+                c[i / 8] |= e2m1_pair(q, __float_as_uint(v[i]), __float_as_uint(v[i + 1])) << (4 * (i % 8));
+            }
+        }
+    }
+    codes_lo = c[0];
+    codes_hi = c[1];
+    return d;
 }
 
 template <int FMT, int M>
@@ -192,174 +314,223 @@ prep_encode_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ 
                    int64_t sf_rows, int64_t k, int n, uint8_t *__restrict__ s_codes, uint8_t *__restrict__ r_codes,
                    uint8_t *__restrict__ s_sf, uint8_t *__restrict__ r_sf, uint8_t *__restrict__ meta,
                    int64_t meta_row) {
-    constexpr int BLK = FMT == kFmtNV ? 16 : 32;
-    constexpr int NB = 32 / BLK;  // blocks per chunk
     constexpr int IB = M <= 2 ? 1 : M <= 4 ? 2 : M <= 8 ? 3 : 4;
+    constexpr int G = kUnit / M;  // mask groups per unit
+    __shared__ uint32_t lut[M <= 8 ? (1 << M) : 1];  // keep bits of a group -> kept positions, ascending
+    if (M <= 8) {
+        for (int msk = threadIdx.x; msk < (1 << M); msk += kEncodeThreads) {
+            uint32_t packed = 0;
+            int pos = 0;
+            for (int i = 0; i < M; ++i)
+                if ((msk >> i) & 1) {
+                    packed |= (uint32_t)i << pos;
+                    pos += IB;
+                }
+            lut[msk] = packed;
+        }
+        __syncthreads();
+    }
 
     const float amax = __uint_as_float(*amax_word);
     const float s_t = (FMT == kFmtNV && amax != 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
     const float c6 = __fmul_rn(6.0f, s_t);
     if (blockIdx.x == 0 && threadIdx.x == 0) *s_t_out = s_t;
 
-    const int64_t cpr = k / 32;
-    const int64_t nblk = k / BLK;
-    const int B = (32 / M) * n * IB;  // metadata bits per chunk
-    const int64_t total = sf_rows * cpr;
+    const int64_t upr = k / kUnit;                 // units per row
+    const int64_t nblk = k / (FMT == kFmtNV ? 16 : 32);
+    const int gbits = n * IB;                      // metadata bits per group
+    const int B = G * gbits;                       // metadata bits per unit
+    const bool byte_aligned = (B & 7) == 0;
+    const int64_t total = sf_rows * upr;
     const int64_t stride = (int64_t)gridDim.x * kEncodeThreads;
     const bool has_g = gamma != nullptr, has_b = beta != nullptr;
 
     for (int64_t base = (int64_t)blockIdx.x * kEncodeThreads; base < total; base += stride) {
         const int64_t t = base + threadIdx.x;
         const bool active = t < total;
-        const int64_t row = active ? t / cpr : 0;
-        const int64_t c = active ? t - row * cpr : 0;
+        const int64_t row = active ? t / upr : 0;
+        const int64_t u = active ? t - row * upr : 0;
         const bool real = active && row < m_tok;
-        uint64_t mlo = 0, mhi = 0;
 
-        if (active && !real) {  // scale-layout padding rows: zero scales
-            if (FMT == kFmtNV) {
-                *reinterpret_cast<uint16_t *>(s_sf + sf_offset(row, 2 * c, nblk)) = 0;
-                *reinterpret_cast<uint16_t *>(r_sf + sf_offset(row, 2 * c, nblk)) = 0;
-            } else {
-                s_sf[sf_offset(row, c, nblk)] = 0;
-                r_sf[sf_offset(row, c, nblk)] = 0;
+        // LayerNorm apply on the unit's 16 values (zeros on idle lanes, which
+        // still take part in the MXFP4 lane-pair exchanges).
+        float v[kUnit];
+        {
+            uint4 xa = make_uint4(0, 0, 0, 0), xb = xa, ga = xa, gb = xa, ba = xa, bb = xa;
+            float2 st = make_float2(0.0f, 1.0f);
+            if (real) {
+                const uint4 *xp = reinterpret_cast<const uint4 *>(x + row * k + u * kUnit);
+                xa = __ldcs(xp);
+                xb = __ldcs(xp + 1);
+                st = stats[row];
+                if (has_g) {
+                    ga = __ldg(reinterpret_cast<const uint4 *>(gamma + u * kUnit));
+                    gb = __ldg(reinterpret_cast<const uint4 *>(gamma + u * kUnit) + 1);
+                }
+                if (has_b) {
+                    ba = __ldg(reinterpret_cast<const uint4 *>(beta + u * kUnit));
+                    bb = __ldg(reinterpret_cast<const uint4 *>(beta + u * kUnit) + 1);
+                }
+            }
+            const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+            const uint32_t gw[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            const uint32_t bw[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+            // (x - mu) * rstd in packed pairs (no multiply feeds an add here);
+            // gamma and beta with scalar intrinsics, which the compiler never
+            // fuses into a multiply-add (a packed multiply followed by a packed
+            // add may be fused, which would skip the rounding of the product).
+            const uint64_t mu2 = pk2(st.x, st.x), rs2 = pk2(st.y, st.y);
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                float2 f = up2(mul2(sub2(h2_to_f2(xw[p]), mu2), rs2));
+                if (has_g) {
+                    f.x = __fmul_rn(f.x, h2f((uint16_t)gw[p]));
+                    f.y = __fmul_rn(f.y, h2f((uint16_t)(gw[p] >> 16)));
+                }
+                if (has_b) {
+                    f.x = __fadd_rn(f.x, h2f((uint16_t)bw[p]));
+                    f.y = __fadd_rn(f.y, h2f((uint16_t)(bw[p] >> 16)));
+                }
+                v[2 * p] = f.x;
+                v[2 * p + 1] = f.y;
             }
         }
-        if (real) {
-            const uint4 *xp = reinterpret_cast<const uint4 *>(x + row * k + c * 32);
-            const float2 st = stats[row];
-            float v[32];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint4 xv = __ldcs(xp + q);
-                uint4 gv = has_g ? __ldg(reinterpret_cast<const uint4 *>(gamma + c * 32) + q) : make_uint4(0, 0, 0, 0);
-                uint4 bv = has_b ? __ldg(reinterpret_cast<const uint4 *>(beta + c * 32) + q) : make_uint4(0, 0, 0, 0);
-                const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-                const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-                const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int wsel = i / 2, sh = 16 * (i % 2);
-                    v[8 * q + i] = ln_apply(h2f((uint16_t)(xw[wsel] >> sh)), st.x, st.y, has_g,
-                                            h2f((uint16_t)(gw[wsel] >> sh)), has_b, h2f((uint16_t)(bw[wsel] >> sh)));
-                }
-            }
 
-            // Top-n of every group of M by magnitude; equal magnitudes go to
-            // the lower index. rank_i = #{j < i: |v_j| >= |v_i|} + #{j > i: |v_j| > |v_i|}.
-            uint32_t keep = 0;
+        const uint32_t keep = keep_mask<M>(v, n);
+
+        // Backbone S = X_ln on the mask, +0 elsewhere.
+        float s[kUnit];
 #pragma unroll
-            for (int g = 0; g < 32 / M; ++g) {
-                uint32_t a[M];
-                int rank[M];
+        for (int i = 0; i < kUnit; ++i) s[i] = ((keep >> i) & 1u) ? v[i] : 0.0f;
+        uint32_t s_scale, s_lo, s_hi;
+        const float ds = quantize16<FMT>(s, s_t, c6, s_scale, s_lo, s_hi);
+
+        // Residual against the quantized backbone: R = RN32(X_ln - RN32(value * d)).
+        // Scalar intrinsics: the product must be rounded before the subtraction.
+        float r[kUnit];
 #pragma unroll
-                for (int i = 0; i < M; ++i) {
-                    a[i] = __float_as_uint(v[g * M + i]) & 0x7FFFFFFFu;
-                    rank[i] = 0;
-                }
+        for (int i = 0; i < kUnit; i += 2) {
+            const uint32_t byte = ((i < 8 ? s_lo : s_hi) >> (4 * (i % 8))) & 0xFFu;
+            const float2 cv = e2m1x2_value(byte);
+            r[i] = __fsub_rn(v[i], __fmul_rn(cv.x, ds));
+            r[i + 1] = __fsub_rn(v[i + 1], __fmul_rn(cv.y, ds));
+        }
+        uint32_t r_scale, r_lo, r_hi;
+        quantize16<FMT>(r, s_t, c6, r_scale, r_lo, r_hi);
+
+        // Mask metadata: each group holds exactly n kept positions, so its
+        // field sits at a fixed offset of the unit's bit range.
+        uint64_t mbits = 0;
+        if (M <= 8) {
 #pragma unroll
-                for (int i = 0; i < M; ++i)
-#pragma unroll
-                    for (int j = i + 1; j < M; ++j) {
-                        if (a[i] >= a[j]) ++rank[j];
-                        else ++rank[i];
-                    }
-#pragma unroll
-                for (int i = 0; i < M; ++i)
-                    if (rank[i] < n) keep |= 1u << (g * M + i);
-            }
-            // Metadata: kept positions of every group, ascending, IB bits each.
+            for (int g = 0; g < G; ++g)
+                mbits |= (uint64_t)lut[(keep >> (g * M)) & ((1u << M) - 1u)] << (g * gbits);
+        } else {
             int pos = 0;
 #pragma unroll
-            for (int g = 0; g < 32 / M; ++g)
-#pragma unroll
-                for (int i = 0; i < M; ++i)
-                    if ((keep >> (g * M + i)) & 1u) {
-                        put_bits(mlo, mhi, (uint32_t)i, IB, pos);
-                        pos += IB;
-                    }
-
-            // Backbone S = X_ln on the mask: block scales, codes, residual.
-            float rr[32];
-            uint32_t spk[4] = {0, 0, 0, 0}, rpk[4] = {0, 0, 0, 0};
-            uint32_t s_sc[NB], r_sc[NB];
-#pragma unroll
-            for (int bk = 0; bk < NB; ++bk) {
-                float a = 0.0f;
-#pragma unroll
-                for (int i = bk * BLK; i < (bk + 1) * BLK; ++i)
-                    if ((keep >> i) & 1u) a = fmaxf(a, fabsf(v[i]));
-                uint32_t code;
-                const float d = block_step<FMT>(a, s_t, c6, code);
-                s_sc[bk] = code;
-#pragma unroll
-                for (int i = bk * BLK; i < (bk + 1) * BLK; i += 2) {
-                    const bool k0 = (keep >> i) & 1u, k1 = (keep >> (i + 1)) & 1u;
-                    uint32_t byte = 0;
-                    if (d != 0.0f) {
-                        const float q0 = k0 ? __fdiv_rn(v[i], d) : 0.0f;
-                        const float q1 = k1 ? __fdiv_rn(v[i + 1], d) : 0.0f;
-                        byte = e2m1x2(q0, q1);
-                    }
-                    const float2 cv = e2m1x2_value(byte);
-                    rr[i] = k0 ? __fsub_rn(v[i], __fmul_rn(cv.x, d)) : v[i];
-                    rr[i + 1] = k1 ? __fsub_rn(v[i + 1], __fmul_rn(cv.y, d)) : v[i + 1];
-                    spk[i / 8] |= byte << (4 * (i % 8));
+            for (int i = 0; i < M; ++i)
+                if ((keep >> i) & 1u) {
+                    mbits |= (uint64_t)i << pos;
+                    pos += IB;
                 }
-            }
-            // Residual R: dense block quantization with the same tensor scale.
-#pragma unroll
-            for (int bk = 0; bk < NB; ++bk) {
-                float a = 0.0f;
-#pragma unroll
-                for (int i = bk * BLK; i < (bk + 1) * BLK; ++i) a = fmaxf(a, fabsf(rr[i]));
-                uint32_t code;
-                const float d = block_step<FMT>(a, s_t, c6, code);
-                r_sc[bk] = code;
-                if (d != 0.0f) {
-#pragma unroll
-                    for (int i = bk * BLK; i < (bk + 1) * BLK; i += 2) {
-                        const uint32_t byte = e2m1x2(__fdiv_rn(rr[i], d), __fdiv_rn(rr[i + 1], d));
-                        rpk[i / 8] |= byte << (4 * (i % 8));
-                    }
-                }
-            }
-            *reinterpret_cast<uint4 *>(s_codes + row * (k / 2) + c * 16) = make_uint4(spk[0], spk[1], spk[2], spk[3]);
-            *reinterpret_cast<uint4 *>(r_codes + row * (k / 2) + c * 16) = make_uint4(rpk[0], rpk[1], rpk[2], rpk[3]);
-            if (FMT == kFmtNV) {
-                *reinterpret_cast<uint16_t *>(s_sf + sf_offset(row, 2 * c, nblk)) = (uint16_t)(s_sc[0] | (s_sc[NB - 1] << 8));
-                *reinterpret_cast<uint16_t *>(r_sf + sf_offset(row, 2 * c, nblk)) = (uint16_t)(r_sc[0] | (r_sc[NB - 1] << 8));
-            } else {
-                s_sf[sf_offset(row, c, nblk)] = (uint8_t)s_sc[0];
-                r_sf[sf_offset(row, c, nblk)] = (uint8_t)r_sc[0];
-            }
         }
 
-        // Metadata store. B bits per chunk; when B is not a whole number of
-        // bytes (m = 8 with odd n: B = 4 mod 8) the chunk pair (2i, 2i+1),
-        // which sits in lanes (2i, 2i+1), shares one byte: the even lane
-        // writes it with the odd lane's first nibble.
-        if ((B & 7) == 0) {
-            if (real) store_bits(meta + row * meta_row + c * (B / 8), mlo, mhi, B / 8);
-        } else {
-            const uint32_t first_nib = (uint32_t)(mlo & 0xF);
-            const uint32_t partner = __shfl_down_sync(0xFFFFFFFFu, first_nib, 1);
-            if (real) {
-                const int full = B / 8;  // whole bytes before the shared nibble
-                if ((c & 1) == 0) {
-                    uint8_t *p = meta + row * meta_row + (c / 2) * (2 * B / 8);
-                    store_bits(p, mlo, mhi, full);
-                    const uint64_t last = full < 8 ? (mlo >> (8 * full)) | (full ? (mhi << (64 - 8 * full)) : 0)
-                                                   : mhi >> (8 * (full - 8));
-                    p[full] = (uint8_t)((last & 0xF) | (partner << 4));
-                } else {
-                    uint8_t *p = meta + row * meta_row + (c / 2) * (2 * B / 8) + full + 1;
-                    const uint64_t lo4 = (mlo >> 4) | (mhi << 60), hi4 = mhi >> 4;
-                    store_bits(p, lo4, hi4, (B - 4) / 8);
-                }
+        if (real) {
+            *reinterpret_cast<uint2 *>(s_codes + row * (k / 2) + u * 8) = make_uint2(s_lo, s_hi);
+            *reinterpret_cast<uint2 *>(r_codes + row * (k / 2) + u * 8) = make_uint2(r_lo, r_hi);
+            if (FMT == kFmtNV) {
+                s_sf[sf_offset(row, u, nblk)] = (uint8_t)s_scale;
+                r_sf[sf_offset(row, u, nblk)] = (uint8_t)r_scale;
+            } else if ((u & 1) == 0) {
+                s_sf[sf_offset(row, u >> 1, nblk)] = (uint8_t)s_scale;
+                r_sf[sf_offset(row, u >> 1, nblk)] = (uint8_t)r_scale;
+            }
+            if (byte_aligned)
+                store_bytes(meta + row * meta_row + u * (B / 8), mbits, B / 8);
+            else
+                or_bits(reinterpret_cast<uint32_t *>(meta), (uint64_t)row * meta_row * 8 + (uint64_t)u * B, mbits, B);
+        } else if (active) {  // scale-layout padding rows: zero scales
+            if (FMT == kFmtNV) {
+                s_sf[sf_offset(row, u, nblk)] = 0;
+                r_sf[sf_offset(row, u, nblk)] = 0;
+            } else if ((u & 1) == 0) {
+                s_sf[sf_offset(row, u >> 1, nblk)] = 0;
+                r_sf[sf_offset(row, u >> 1, nblk)] = 0;
             }
         }
     }
+}
+
+// ---------------------------------------------------------------------------
+// Division self-test: the packed correction division against the correctly
+// rounded hardware division, on operands drawn from a counter-based hash:
+// random quotients in [2^-4, 2^4], quotients within a few ulps of the E2M1
+// rounding boundaries, and quotients of exponent -30 .. 30; divisors span
+// [2^-90, 2^90]. A mismatch is a quotient of magnitude >= 2^-4 whose bits
+// differ, or any quotient whose E2M1 code differs. (Below 2^-4 the remainder
+// of the method can leave the normal range; such quotients only ever give a
+// zero code, whose sign comes from the dividend.)
+__device__ unsigned long long g_div_mismatch;
+__device__ float g_div_examples[16][4];  // first mismatches: v, d, quotient, reference
+
+__device__ __forceinline__ uint64_t hash64(uint64_t z) {
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+__global__ void div_check_kernel(uint64_t count, uint64_t seed) {
+    const float ties[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
+    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (uint64_t)gridDim.x * blockDim.x) {
+        const uint64_t h = hash64(seed + 0x9E3779B97F4A7C15ull * (i + 1)), g = hash64(h);
+        const int de = (int)(h % 181) - 90;                       // divisor exponent in [-90, 90]
+        const float d = __uint_as_float((uint32_t)(de + 127) << 23 | (uint32_t)(g & 0x7FFFFF));
+        float v;
+        const int kind = (int)((h >> 40) & 3);
+        if (kind == 0) {  // near an E2M1 rounding boundary
+            const float t = ties[(g >> 23) % 7];
+            const int ulps = (int)((g >> 30) % 9) - 4;
+            v = __fmul_rn(__uint_as_float(__float_as_uint(t) + ulps), d);
+        } else if (kind == 1) {  // quotient exponent in [-30, 30]
+            const int qe = (int)((g >> 24) % 61) - 30;
+            v = __fmul_rn(__uint_as_float((uint32_t)(qe + 127) << 23 | (uint32_t)(h & 0x7FFFFF)), d);
+        } else {  // quotient in [2^-4, 2^4]
+            const int qe = (int)((g >> 24) % 9) - 4;
+            v = __fmul_rn(__uint_as_float((uint32_t)(qe + 127) << 23 | (uint32_t)(h & 0x7FFFFF)), d);
+        }
+        if ((g >> 63) & 1) v = -v;
+        const float y = __frcp_rn(d);
+        const float2 q = up2(div2(pk2(v, v), pk2(d, d), pk2(-d, -d), pk2(y, y)));
+        const float ref = __fdiv_rn(v, d);
+        const uint32_t sv = __float_as_uint(v);
+        const bool bits_differ = (__float_as_uint(q.x) & 0x7FFFFFFFu) != (__float_as_uint(ref) & 0x7FFFFFFFu);
+        const bool code_differs = (e2m1_pair(pk2(q.x, q.x), sv, sv) & 0xFu) != (e2m1_pair(pk2(ref, ref), sv, sv) & 0xFu);
+        if (ref == ref && ((bits_differ && fabsf(ref) >= 0x1p-4f) || code_differs)) {
+            const unsigned long long slot = atomicAdd(&g_div_mismatch, 1ull);
+            if (slot < 16) {
+                g_div_examples[slot][0] = v;
+                g_div_examples[slot][1] = d;
+                g_div_examples[slot][2] = q.x;
+                g_div_examples[slot][3] = ref;
+            }
+        }
+    }
+}
+
+sharq_status launch_div_check(LaunchCtx &ctx, uint64_t count, uint64_t seed, uint64_t *mismatches, float *examples) {
+    unsigned long long zero = 0;
+    SQ_CUDA_TRY(cudaMemcpyToSymbolAsync(g_div_mismatch, &zero, sizeof(zero), 0, cudaMemcpyHostToDevice, ctx.stream));
+    div_check_kernel<<<ctx.num_sms * 8, 256, 0, ctx.stream>>>(count, seed);
+    ctx.launches++;
+    SQ_CUDA_TRY(cudaGetLastError());
+    unsigned long long host = 0;
+    SQ_CUDA_TRY(cudaMemcpyFromSymbolAsync(&host, g_div_mismatch, sizeof(host), 0, cudaMemcpyDeviceToHost, ctx.stream));
+    if (examples)
+        SQ_CUDA_TRY(cudaMemcpyFromSymbolAsync(examples, g_div_examples, sizeof(g_div_examples), 0,
+                                              cudaMemcpyDeviceToHost, ctx.stream));
+    SQ_CUDA_TRY(cudaStreamSynchronize(ctx.stream));
+    *mismatches = host;
+    return SHARQ_OK;
 }
 
 template <int FMT>
@@ -379,21 +550,29 @@ sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, 
     SQ_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
     if (!attr_done[dev]) {
-        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)(2 * SHARQ_K_MAX)));
         attr_done[dev] = true;
     }
     unsigned *words = reinterpret_cast<unsigned *>(P.tensor_scale) - 1;  // [0] amax bits, [1] s_t
     SQ_CUDA_TRY(cudaMemsetAsync(words, 0, sizeof(unsigned), ctx.stream));
+    const int ib = idx_bits(P.m);
+    const bool meta_atomic = ((kUnit / P.m) * P.n * ib) % 8 != 0;
+    if (meta_atomic && P.m_tok > 0)  // unaligned metadata fields are OR-ed into a zeroed stream
+        SQ_CUDA_TRY(cudaMemsetAsync(P.meta, 0, (size_t)(P.m_tok * P.meta_row_bytes), ctx.stream));
     float2 *stats = reinterpret_cast<float2 *>(P.scratch);
     if (P.m_tok > 0) {
-        ln_stats_kernel<<<(unsigned)P.m_tok, kStatsThreads, (size_t)(2 * P.k), ctx.stream>>>(
-            (const uint16_t *)x, (const uint16_t *)gamma, (const uint16_t *)beta, eps, P.k, stats, words);
+        if (gamma || beta)
+            ln_stats_kernel<true><<<(unsigned)P.m_tok, kStatsThreads, (size_t)(2 * P.k), ctx.stream>>>(
+                (const uint16_t *)x, (const uint16_t *)gamma, (const uint16_t *)beta, eps, P.k, stats, words);
+        else
+            ln_stats_kernel<false><<<(unsigned)P.m_tok, kStatsThreads, 0, ctx.stream>>>(
+                (const uint16_t *)x, nullptr, nullptr, eps, P.k, stats, words);
         ctx.launches++;
     }
-    const int64_t total = P.sf_rows * (P.k / 32);
+    const int64_t total = P.sf_rows * (P.k / kUnit);
     int64_t blocks = (total + kEncodeThreads - 1) / kEncodeThreads;
-    const int64_t cap = (int64_t)ctx.num_sms * 8;
+    const int64_t cap = (int64_t)ctx.num_sms * 16;
     if (blocks > cap) blocks = cap;
     void *fn = P.fmt == kFmtNV ? encode_fn<kFmtNV>(P.m) : encode_fn<kFmtMX>(P.m);
     const uint16_t *xx = (const uint16_t *)x, *gg = (const uint16_t *)gamma, *bb = (const uint16_t *)beta;

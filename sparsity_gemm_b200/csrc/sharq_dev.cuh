@@ -113,6 +113,84 @@ __device__ __forceinline__ float block_step(float a, float s_t, float c6, uint32
 }
 
 // ---------------------------------------------------------------------------
+// Packed pairs of binary32 (sm_100 f32x2 instructions): one instruction for
+// two independent IEEE operations, each rounded to nearest even. Code
+// generation may fuse a packed multiply that feeds a packed add or subtract
+// into one fused multiply-add (the product then goes unrounded), so callers
+// use these only where no product feeds an add, or where the FMA is meant;
+// rounded products that feed an add use the scalar __fmul_rn / __fadd_rn.
+
+__device__ __forceinline__ uint64_t pk2(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ float2 up2(uint64_t r) {
+    float2 f;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(r));
+    return f;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t add2_rm(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// Two fp16 values (one 32-bit word, low half first) as a packed float pair.
+__device__ __forceinline__ uint64_t h2_to_f2(uint32_t w) {
+    float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w));
+    return pk2(f.x, f.y);
+}
+
+// Correctly rounded quotients v / d of a packed pair, for d in [2^-90, 2^90]
+// with y = RN(1/d) and |v / d| >= 2^-4 (smaller quotients come out within an
+// ulp, which is all E2M1 encoding needs there). Markstein's correction (P. Markstein, "Computation of
+// elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990): q0 = RN(v y); one FMA residual step makes the quotient
+// faithful; with the remainder r = v - d q1 then exact, RN(q1 + r y) is the
+// correctly rounded quotient. Zero quotients may lose their sign; callers
+// take the sign from v.
+__device__ __forceinline__ uint64_t div2(uint64_t v, uint64_t d2, uint64_t nd2, uint64_t y2) {
+    uint64_t q = mul2(v, y2);
+    uint64_t r = fma2(q, nd2, v);
+    q = fma2(r, y2, q);
+    r = fma2(q, nd2, v);
+    return fma2(r, y2, q);
+}
+
+// E2M1 byte of two quotients (lo nibble = q.x), rounded to nearest even with
+// saturation to 6 by the hardware conversion; the sign bits are taken from the
+// dividends (sign_lo, sign_hi: their bit patterns), which carry the sign of
+// the exact quotient also where the quotient is zero.
+__device__ __forceinline__ uint32_t e2m1_pair(uint64_t q, uint32_t sign_lo, uint32_t sign_hi) {
+    float2 f = up2(q);
+    uint32_t b;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(b) : "f"(f.y), "f"(f.x));
+    return (b & 0x77u) | ((sign_lo >> 31) << 3) | ((sign_hi >> 31) << 7);
+}
+
+// ---------------------------------------------------------------------------
 // Shared-memory and barrier primitives
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {

@@ -20,6 +20,7 @@ sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, 
 sharq_status launch_quantize_weight(LaunchCtx &ctx, const sharq_wq &W, const void *w);
 sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, void *out);
 sharq_status launch_wait_probe(LaunchCtx &ctx, uint64_t limit_ns);
+sharq_status launch_div_check(LaunchCtx &ctx, uint64_t count, uint64_t seed, uint64_t *mismatches, float *examples);
 
 }  // namespace sq
 

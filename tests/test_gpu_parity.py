@@ -184,3 +184,25 @@ def test_results_do_not_depend_on_stream_or_buffer_reuse():
         ex2 = sq.prep_export(p2, stream=s)
     for key in ex1:
         np.testing.assert_array_equal(np.asarray(ex1[key]), np.asarray(ex2[key]))
+
+
+def test_quantizer_division_is_correctly_rounded():
+    """The encode kernels' reciprocal-and-correction division equals the
+    correctly rounded quotient on 2^26 operand pairs."""
+    import sparsity_gemm_b200 as sq
+    assert sq.selftest_division(1 << 26, seed=12345) == 0
+
+
+def test_tiny_and_huge_scales_bit_exact():
+    """Activation tensors far from unit scale (large eps shrinks X_ln) and
+    weights with tiny magnitudes still match the oracle bit for bit."""
+    import sparsity_gemm_b200 as sq
+    x = synth.activations_student(31, 40, 512)
+    for eps in [1e-5, 1e20, 3e38]:
+        op = oracle.prepare(x, None, None, eps, 2, 4, 0)
+        _, ex = gpu_prepare(x, None, None, eps, 2, 4, 0)
+        assert_prep_matches(ex, op)
+    w = (synth.weights(32, 64, 256).astype(np.float32) * 1e-3).astype(np.float16)
+    ow = oracle.quantize_weight(w, 0)
+    qw = sq.quantize_weight(cuda16(w), 0)
+    assert_weight_matches(sq.weight_export(qw), ow)
