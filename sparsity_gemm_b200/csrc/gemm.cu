@@ -13,12 +13,14 @@
 // mask: the block-scaled FP4 sparse MMA kinds take pair-wise 4:8 metadata,
 // which an element-wise top-n-of-m mask does not satisfy in general.
 //
-// Structure: persistent CTAs (one per SM), tile 128 x 256 x 256 (M x N x K),
-// 3-stage TMA pipeline, 6 warps:
+// Structure: persistent CTAs (one per SM), tile 128 x 256 (M x N) with a
+// K step of 2 * SQ_GEMM_BKB FP4 values, a TMA pipeline as deep as shared
+// memory allows, 6 warps:
 //   warp 0      TMA producer (A_S, A_R, W tiles; scale atoms by bulk copy)
 //   warp 1      tensor-memory allocation and the single-thread MMA issuer
-//               (scale atoms -> tensor memory by tcgen05.cp, then MMAs)
 //   warps 2..5  epilogue: tensor memory -> registers -> fp16 -> global
+//   warp 6      scale copies: the stage's scale atoms -> one of two scale
+//               buffers in tensor memory (tcgen05.cp), ahead of the MMAs
 // Every mbarrier wait is bounded (global-timer limit); a wait that runs out
 // records a site code in the status word and the CTA winds down cleanly.
 #include <cuda.h>
@@ -30,24 +32,44 @@
 
 namespace sq {
 
-constexpr int kBM = 128, kBN = 256, kBKBytes = 128, kStages = 3;  // K tile: 256 FP4 = 128 bytes
-constexpr int kABytes = kBM * kBKBytes;                            // 16 KB
-constexpr int kBBytes = kBN * kBKBytes;                            // 32 KB
-constexpr int kSfaMax = 2048, kSfbMax = 4096;                      // NVFP4 sizes (MXFP4 uses half)
+// K tile width in bytes per operand row (two FP4 values per byte). Measured
+// on B200: 128-byte rows (3 stages) beat 64-byte rows (6 stages) by ~5%. 64 bytes
+// (128 elements, 64-byte swizzle) gives 36 KB stages and a 6-deep pipeline;
+// 128 bytes (256 elements, 128-byte swizzle) gives 72 KB stages, 3 deep.
+#ifndef SQ_GEMM_BKB
+#define SQ_GEMM_BKB 128
+#endif
+constexpr int kBM = 128, kBN = 256, kBKBytes = SQ_GEMM_BKB;
+constexpr int kABytes = kBM * kBKBytes;
+constexpr int kBBytes = kBN * kBKBytes;
+constexpr int kSfaMax = 512 * (kBKBytes / 32), kSfbMax = 2 * kSfaMax;  // NVFP4 sizes (MXFP4 uses half)
 constexpr int kOffAS = 0, kOffAR = kABytes, kOffB = 2 * kABytes;
 constexpr int kOffSFAS = kOffB + kBBytes, kOffSFAR = kOffSFAS + kSfaMax, kOffSFB = kOffSFAR + kSfaMax;
-constexpr int kStageBytes = kOffSFB + kSfbMax;                     // 72 KB, a multiple of 1024
+constexpr int kStageBytes = kOffSFB + kSfbMax;                     // a multiple of 1024
+constexpr int kStages = (232448 - 2048) / kStageBytes;
 constexpr int kBarOff = kStages * kStageBytes;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;                   // barriers + alignment slack
+constexpr int kMmaPerStage = kBKBytes / 32;                        // MMAs of K = 64 per path per stage
+constexpr uint32_t kSwizzleLayout = kBKBytes == 128 ? 2u : 4u;     // descriptor layout: 128B / 64B swizzle
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColSfaS = 256, kColSfaR = 272, kColSfb = 288;  // scale columns after the accumulator
-constexpr int kGemmThreads = 192;
+// Scale buffers after the accumulator (columns 0..255): two of 64 columns,
+// filled alternately by the scale-copy warp; within a buffer, the backbone
+// A scales at +0, the residual A scales at +16, the W scales at +32.
+constexpr uint32_t kColSf0 = 256, kSfBufCols = 64;
+constexpr uint32_t kSfaS = 0, kSfaR = 16, kSfb = 32;
+constexpr int kGemmThreads = 224;
+static_assert(kStageBytes % 1024 == 0, "stage buffers must stay 1024-byte aligned");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(8 * (2 * kStages + 8) + 4 <= 256, "barrier area");
 
 enum : unsigned {
     kSiteProducer = 0x101,
     kSiteMmaAcc = 0x102,
     kSiteMmaFull = 0x103,
     kSiteEpilogue = 0x104,
+    kSiteMmaScales = 0x105,
+    kSiteScaleFull = 0x106,
+    kSiteScaleEmpty = 0x107,
     kSiteProbe = 0x1FF,
 };
 
@@ -74,9 +96,11 @@ __device__ __forceinline__ uint32_t idesc_of(uint32_t sf_id) {
            ((uint32_t)(kBM >> 4) << 24) | (sf_id << 29) | (sf_id << 4);
 }
 
-// K-major operand tile, rows of 128 bytes, 128-byte swizzle; 8-row groups
-// are 1024 bytes apart.
-__device__ __forceinline__ uint64_t desc_operand(uint32_t addr) { return smem_desc(addr, 16, 1024, 2); }
+// K-major operand tile, rows of kBKBytes bytes swizzled in kBKBytes-wide
+// atoms; 8-row groups are 8 * kBKBytes bytes apart.
+__device__ __forceinline__ uint64_t desc_operand(uint32_t addr) {
+    return smem_desc(addr, 16, 8 * kBKBytes, kSwizzleLayout);
+}
 
 // One 512-byte scale atom: 32 rows of 16 bytes, no swizzle, 8-row groups
 // 128 bytes apart.
@@ -97,19 +121,23 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     const uint32_t raw_s = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t bar0 = sbase + kBarOff;  // full[s], empty[s], acc_full, acc_empty, drain
+    const uint32_t bar0 = sbase + kBarOff;  // full[s], empty[s], acc_full, acc_empty, drain x2, sf_full[2], sf_empty[2]
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
     const uint32_t acc_full = bar0 + 8u * (2 * kStages);
     const uint32_t acc_empty = acc_full + 8u;
     const uint32_t drain_bar = acc_full + 16u;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOff + 128);
+    const uint32_t drain_sf_bar = acc_full + 24u;
+    auto sf_full_bar = [&](int b) { return acc_full + 32u + 8u * b; };
+    auto sf_empty_bar = [&](int b) { return acc_full + 48u + 8u * b; };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOff + 8 * (2 * kStages + 8));
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int m_tiles = (p.m_tok + kBM - 1) / kBM, n_tiles = (p.n_out + kBN - 1) / kBN;
-    const int num_tiles = m_tiles * n_tiles, kt_count = p.k / 256;
+    const int num_tiles = m_tiles * n_tiles, kt_count = p.k / (2 * kBKBytes);
     const int64_t atoms_per_row_blk = (int64_t)(p.k / (FMT == kFmtNV ? 16 : 32)) / 4;
-    constexpr int kAtomsPerTile = FMT == kFmtNV ? 4 : 2;  // 512-byte atoms per 128 rows per K tile
+    // 512-byte scale atoms (128 rows x 4 scales) per 128 rows per K tile
+    constexpr int kAtomsPerTile = FMT == kFmtNV ? kBKBytes / 32 : kBKBytes / 64;
     constexpr uint32_t kSfBytes = 512u * kAtomsPerTile;
 
     if (threadIdx.x == 0) {
@@ -120,6 +148,11 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 128);
         mbar_init(drain_bar, 1);
+        mbar_init(drain_sf_bar, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(sf_full_bar(b), 1);
+            mbar_init(sf_empty_bar(b), 1);
+        }
         mbar_fence_init();
         prefetch_tmap(&tm_as);
         prefetch_tmap(&tm_ar);
@@ -184,40 +217,36 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                         ok = false;
                         break;
                     }
+                    const int sb = (int)(it & 1u);  // scale buffer of this stage
+                    if (!mbar_wait(sf_full_bar(sb), (it >> 1) & 1u, p.status, kSiteMmaScales, p.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t st = sbase + (uint32_t)(s * kStageBytes);
-                    // Scale atoms -> tensor memory. One atom (128 rows x 4
-                    // scales) fills 4 columns; the W tile's 256 rows take two.
-#pragma unroll
-                    for (int a = 0; a < kAtomsPerTile; ++a) {
-                        tc_copy_scales(tmem + kColSfaS + 4 * a, desc_scales(st + kOffSFAS + 512 * a));
-                        tc_copy_scales(tmem + kColSfaR + 4 * a, desc_scales(st + kOffSFAR + 512 * a));
-                        tc_copy_scales(tmem + kColSfb + 8 * a, desc_scales(st + kOffSFB + 512 * a));
-                        tc_copy_scales(tmem + kColSfb + 8 * a + 4, desc_scales(st + kOffSFB + kSfBytes + 512 * a));
-                    }
+                    const uint32_t sf = tmem + kColSf0 + kSfBufCols * (uint32_t)sb;
                     const uint64_t da_s = desc_operand(st + kOffAS);
                     const uint64_t da_r = desc_operand(st + kOffAR);
                     const uint64_t db = desc_operand(st + kOffB);
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {  // 4 MMAs of K = 64 (32 bytes) per K tile
+                    for (int j = 0; j < kMmaPerStage; ++j) {  // MMAs of K = 64 (32 bytes) per K tile
                         const uint32_t acc = (kt | j) != 0;
                         if (FMT == kFmtNV) {
                             const uint32_t idesc = idesc_of<FMT>(0);
-                            tc_mma_nvf4(tmem, da_s + 2 * j, db + 2 * j, idesc, tmem + kColSfaS + 4 * j,
-                                        tmem + kColSfb + 8 * j, acc);
-                            tc_mma_nvf4(tmem, da_r + 2 * j, db + 2 * j, idesc, tmem + kColSfaR + 4 * j,
-                                        tmem + kColSfb + 8 * j, 1u);
+                            tc_mma_nvf4(tmem, da_s + 2 * j, db + 2 * j, idesc, sf + kSfaS + 4 * j, sf + kSfb + 8 * j, acc);
+                            tc_mma_nvf4(tmem, da_r + 2 * j, db + 2 * j, idesc, sf + kSfaR + 4 * j, sf + kSfb + 8 * j, 1u);
                         } else {
                             const uint32_t sf_id = (uint32_t)(j & 1) * 2u;  // 2 scales per row per MMA
                             const uint32_t idesc = idesc_of<FMT>(sf_id);
                             const uint32_t a_col = 4 * (j >> 1), b_col = 8 * (j >> 1);
-                            tc_mma_mxf4(tmem, da_s + 2 * j, db + 2 * j, idesc, (tmem + kColSfaS + a_col) | (sf_id << 30),
-                                        (tmem + kColSfb + b_col) | (sf_id << 30), acc);
-                            tc_mma_mxf4(tmem, da_r + 2 * j, db + 2 * j, idesc, (tmem + kColSfaR + a_col) | (sf_id << 30),
-                                        (tmem + kColSfb + b_col) | (sf_id << 30), 1u);
+                            tc_mma_mxf4(tmem, da_s + 2 * j, db + 2 * j, idesc, (sf + kSfaS + a_col) | (sf_id << 30),
+                                        (sf + kSfb + b_col) | (sf_id << 30), acc);
+                            tc_mma_mxf4(tmem, da_r + 2 * j, db + 2 * j, idesc, (sf + kSfaR + a_col) | (sf_id << 30),
+                                        (sf + kSfb + b_col) | (sf_id << 30), 1u);
                         }
                     }
-                    tc_commit(empty_bar(s));  // frees the stage once these MMAs complete
+                    tc_commit(empty_bar(s));       // frees the stage once these MMAs complete
+                    tc_commit(sf_empty_bar(sb));   // and the scale buffer
                 }
                 if (!ok) break;
                 tc_commit(acc_full);
@@ -226,36 +255,78 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             drain_wait(drain_bar, 0, kDrainNs);
         }
         __syncwarp();
+    } else if (warp == 6) {
+        // Scale copies, one stage ahead of the MMAs where the pipeline allows:
+        // the stage's atoms (128 rows x 4 scales, 512 bytes) fill 4 columns
+        // each; the W tile's 256 rows take two atoms per K step.
+        if (lane == 0) {
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                for (int kt = 0; kt < kt_count; ++kt, ++it) {
+                    const int s = (int)(it % kStages);
+                    const int sb = (int)(it & 1u);
+                    if (!mbar_wait(full_bar(s), (it / kStages) & 1u, p.status, kSiteScaleFull, p.wait_ns) ||
+                        !mbar_wait(sf_empty_bar(sb), ((it >> 1) & 1u) ^ 1u, p.status, kSiteScaleEmpty, p.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t st = sbase + (uint32_t)(s * kStageBytes);
+                    const uint32_t sf = tmem + kColSf0 + kSfBufCols * (uint32_t)sb;
+#pragma unroll
+                    for (int a = 0; a < kAtomsPerTile; ++a) {
+                        tc_copy_scales(sf + kSfaS + 4 * a, desc_scales(st + kOffSFAS + 512 * a));
+                        tc_copy_scales(sf + kSfaR + 4 * a, desc_scales(st + kOffSFAR + 512 * a));
+                        tc_copy_scales(sf + kSfb + 8 * a, desc_scales(st + kOffSFB + 512 * a));
+                        tc_copy_scales(sf + kSfb + 8 * a + 4, desc_scales(st + kOffSFB + kSfBytes + 512 * a));
+                    }
+                    tc_commit(sf_full_bar(sb));  // the MMAs may read this buffer once the copies land
+                }
+            }
+            tc_commit(drain_sf_bar);
+            drain_wait(drain_sf_bar, 0, kDrainNs);
+        }
+        __syncwarp();
     } else {
+        // Epilogue. The accumulator is first drained from tensor memory into
+        // registers (as packed fp16) and handed back to the MMA warp, so that
+        // the next tile's MMAs overlap with this tile's global stores.
         const int q = warp & 3;  // tensor-memory lane quadrant this warp may access
         const float alpha = __fmul_rn(*p.s_t, *p.s_tw);
         uint32_t tile_iter = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tile_iter) {
             if (!mbar_wait(acc_full, tile_iter & 1u, p.status, kSiteEpilogue, p.wait_ns)) break;
             tc_fence_after();
-            const int nb = tile % n_tiles, mb = tile / n_tiles;
-            const int row = mb * kBM + q * 32 + lane;
-#pragma unroll 1
+            uint32_t h[kBN / 32][16];
+#pragma unroll
             for (int cc = 0; cc < kBN / 32; ++cc) {
                 uint32_t r[32];
                 tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cc * 32), r);
                 tmem_ld_wait();
-                const int col0 = nb * kBN + cc * 32;
-                if (row < p.m_tok && col0 < p.n_out) {
-                    uint32_t h[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        __half2 v = __floats2half2_rn(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
-                                                      __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
-                        h[i] = *reinterpret_cast<uint32_t *>(&v);
-                    }
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + (int64_t)row * p.n_out + col0);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+                for (int i = 0; i < 16; ++i) {
+                    __half2 v = __floats2half2_rn(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
+                                                  __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
+                    h[cc][i] = *reinterpret_cast<uint32_t *>(&v);
                 }
             }
             tc_fence_before();
             mbar_arrive(acc_empty);
+            const int nb = tile % n_tiles, mb = tile / n_tiles;
+            const int row = mb * kBM + q * 32 + lane;
+            if (row < p.m_tok) {
+#pragma unroll
+                for (int cc = 0; cc < kBN / 32; ++cc) {
+                    const int col0 = nb * kBN + cc * 32;
+                    if (col0 < p.n_out) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + (int64_t)row * p.n_out + col0);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(h[cc][4 * i], h[cc][4 * i + 1], h[cc][4 * i + 2], h[cc][4 * i + 3]);
+                    }
+                }
+            }
         }
     }
 
@@ -303,7 +374,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 2-D byte tensor [rows][row_bytes], box = 128 bytes x box_rows, 128-byte swizzle.
+// 2-D byte tensor [rows][row_bytes], box = kBKBytes x box_rows, swizzled in
+// kBKBytes-wide atoms.
 static bool make_code_map(CUtensorMap *tm, const void *base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
@@ -312,7 +384,9 @@ static bool make_code_map(CUtensorMap *tm, const void *base, uint64_t row_bytes,
     cuuint32_t box[2] = {(cuuint32_t)kBKBytes, box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     kBKBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }

@@ -103,8 +103,7 @@ ln_stats_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gam
 
     ExactSums e = {0, 0, 0, 0, 0};
     uint32_t mx = 0xFC00FC00u, mn = 0x7C007C00u;  // (-inf, -inf), (+inf, +inf) as half2
-    for (int c = threadIdx.x; c < nvec; c += kStatsThreads) {
-        const uint4 v = xr[c];  // default caching: the encode pass re-reads x from L2
+    auto consume = [&](const uint4 &v, int c) {
         if (AFFINE) row_cache[c] = v;
         accum_pair(v.x, e);
         accum_pair(v.y, e);
@@ -120,7 +119,16 @@ ln_stats_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gam
             asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(v.z));
             asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(v.w));
         }
+    };
+    // Two loads in flight per thread (default caching: the encode pass
+    // re-reads x from L2).
+    int c = threadIdx.x;
+    for (; c + kStatsThreads < nvec; c += 2 * kStatsThreads) {
+        const uint4 v0 = xr[c], v1 = xr[c + kStatsThreads];
+        consume(v0, c);
+        consume(v1, c + kStatsThreads);
     }
+    if (c < nvec) consume(xr[c], c);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         e.hi += __shfl_xor_sync(0xFFFFFFFFu, e.hi, o);
@@ -267,6 +275,42 @@ __device__ __forceinline__ uint32_t keep_mask(const float (&v)[kUnit], int n) {
 // Block quantization of one thread's 16 values (an NVFP4 block, or half of an
 // MXFP4 block whose other half sits in the neighbouring lane). Produces the
 // scale code, the step d and the 16 E2M1 codes (8 bytes).
+// m = 4: the four ranks as the bytes of one word; each of the six pairs adds
+// 1 to the byte of the element that loses the comparison. A rank byte r
+// survives iff r < n: (0x80 + r - n) has bit 7 clear exactly then (no
+// borrows cross bytes since r, n <= 4); a multiply gathers the four bits.
+template <>
+__device__ __forceinline__ uint32_t keep_mask<4>(const float (&v)[kUnit], int n) {
+    const uint32_t nn = (uint32_t)n * 0x01010101u;
+    uint32_t keep = 0;
+#pragma unroll
+    for (int g = 0; g < kUnit / 4; ++g) {
+        const uint32_t a0 = __float_as_uint(v[4 * g]) & 0x7FFFFFFFu, a1 = __float_as_uint(v[4 * g + 1]) & 0x7FFFFFFFu;
+        const uint32_t a2 = __float_as_uint(v[4 * g + 2]) & 0x7FFFFFFFu, a3 = __float_as_uint(v[4 * g + 3]) & 0x7FFFFFFFu;
+        uint32_t r = (a0 >= a1 ? 0x00000100u : 0x00000001u) + (a0 >= a2 ? 0x00010000u : 0x00000001u) +
+                     (a0 >= a3 ? 0x01000000u : 0x00000001u);
+        r += (a1 >= a2 ? 0x00010000u : 0x00000100u) + (a1 >= a3 ? 0x01000000u : 0x00000100u) +
+             (a2 >= a3 ? 0x01000000u : 0x00010000u);
+        const uint32_t lost = ((r | 0x80808080u) - nn) & 0x80808080u;  // bit 7 of byte i: rank_i >= n
+        const uint32_t kept = (~lost & 0x80808080u) >> 7;               // bits 0, 8, 16, 24
+        keep |= ((kept * 0x00204081u) >> 21 & 0xFu) << (4 * g);
+    }
+    return keep;
+}
+
+// m = 2: keep both (n = 2) or the larger, the first on ties (n = 1).
+template <>
+__device__ __forceinline__ uint32_t keep_mask<2>(const float (&v)[kUnit], int n) {
+    if (n >= 2) return 0xFFFFu;
+    uint32_t keep = 0;
+#pragma unroll
+    for (int g = 0; g < kUnit / 2; ++g) {
+        const uint32_t a0 = __float_as_uint(v[2 * g]) & 0x7FFFFFFFu, a1 = __float_as_uint(v[2 * g + 1]) & 0x7FFFFFFFu;
+        keep |= (a0 >= a1 ? 1u : 2u) << (2 * g);
+    }
+    return keep;
+}
+
 template <int FMT>
 __device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, float c6, uint32_t &scale_code,
                                             uint32_t &codes_lo, uint32_t &codes_hi) {
@@ -345,11 +389,21 @@ prep_encode_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ 
     const int64_t stride = (int64_t)gridDim.x * kEncodeThreads;
     const bool has_g = gamma != nullptr, has_b = beta != nullptr;
 
+    // (row, unit) of this thread's first unit, then stepped by the grid
+    // stride without dividing again.
+    const int64_t t0 = (int64_t)blockIdx.x * kEncodeThreads + threadIdx.x;
+    int64_t row_i = t0 / upr, u_i = t0 - (t0 / upr) * upr;
+    const int64_t step_rows = stride / upr, step_units = stride - (stride / upr) * upr;
     for (int64_t base = (int64_t)blockIdx.x * kEncodeThreads; base < total; base += stride) {
         const int64_t t = base + threadIdx.x;
         const bool active = t < total;
-        const int64_t row = active ? t / upr : 0;
-        const int64_t u = active ? t - row * upr : 0;
+        const int64_t row = row_i, u = u_i;
+        row_i += step_rows;
+        u_i += step_units;
+        if (u_i >= upr) {
+            u_i -= upr;
+            ++row_i;
+        }
         const bool real = active && row < m_tok;
 
         // LayerNorm apply on the unit's 16 values (zeros on idle lanes, which

@@ -179,15 +179,18 @@ __device__ __forceinline__ uint64_t div2(uint64_t v, uint64_t d2, uint64_t nd2, 
 }
 
 // E2M1 byte of two quotients (lo nibble = q.x), rounded to nearest even with
-// saturation to 6 by the hardware conversion; the sign bits are taken from the
-// dividends (sign_lo, sign_hi: their bit patterns), which carry the sign of
-// the exact quotient also where the quotient is zero.
+// saturation to 6 by the hardware conversion, which keeps the sign of zeros.
+// The quotients first take the sign bits of their dividends (sign_lo,
+// sign_hi: bit patterns): that is the sign of the exact quotient, also where
+// a zero dividend's quotient came out of the division as +0.
 __device__ __forceinline__ uint32_t e2m1_pair(uint64_t q, uint32_t sign_lo, uint32_t sign_hi) {
-    float2 f = up2(q);
+    const float2 f = up2(q);
+    const float lo = __uint_as_float(__float_as_uint(f.x) | (sign_lo & 0x80000000u));
+    const float hi = __uint_as_float(__float_as_uint(f.y) | (sign_hi & 0x80000000u));
     uint32_t b;
     asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
-        : "=r"(b) : "f"(f.y), "f"(f.x));
-    return (b & 0x77u) | ((sign_lo >> 31) << 3) | ((sign_hi >> 31) << 7);
+        : "=r"(b) : "f"(hi), "f"(lo));
+    return b;
 }
 
 // ---------------------------------------------------------------------------
