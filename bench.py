@@ -41,6 +41,11 @@ N_KEEP, M_GROUP = 2, 4
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
 PREP_BYTES_PER_ELEM = 3.25  # x 2 + S codes 0.5 + mask metadata 0.125 + S scales 0.0625 + R codes 0.5 + R scales 0.0625
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of the 7 GEMM launches of one M = 8192 step, from
+# one ncu capture of the current dual_gemm_kernel (dram__bytes_read.sum +
+# dram__bytes_write.sum; profiles/dual_gemm_kernel_m8192_n4096_k14336.md).
+# Set to None whenever the kernel changes until it is captured again.
+GEMM_TRAFFIC_BYTES_PER_STEP_M8192 = 981.1e6
 
 
 def parse_args():
@@ -299,7 +304,9 @@ def run_sharq(args, world, rank, local):
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "tensor", "kernel": "dual_gemm_kernel (7 linears)",
                      "achieved": gemm_alg_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
-                     "frac": gemm_alg_tflops / fp4_peak, "traffic": None,
+                     "frac": gemm_alg_tflops / fp4_peak,
+                     "traffic": GEMM_TRAFFIC_BYTES_PER_STEP_M8192 if M == 8192 else None,
+                     "traffic_scope": "DRAM bytes of the 7 GEMM launches of one step (ncu capture)",
                      "peak_source": f"{peak_src} bf16 {peaks['bf16_tflops']} TF/s x {FP4_OVER_BF16} (FP4/BF16 nominal)",
                      "flops_per_step": flops_algorithmic(M), "flop_count": "2*M*N*K*(1+n/m)",
                      "executed_tflops": gemm_exec_tflops, "executed_frac": gemm_exec_tflops / fp4_peak},

@@ -271,10 +271,11 @@ void oracle_quantize(const float *v, int64_t rows, int64_t k, int fmt, float s_t
 }
 
 /* ------------------------------------------------------------------ */
-/* Tensor scale (reading: north-star "fp32 tensor scale" for NVFP4 is    */
-/* one dynamic scale per tensor from amax over the whole tensor:          */
-/* s_t = RN32(amax / 2688), 2688 = 448 * 6; s_t = 1 if amax == 0; MXFP4   */
-/* has no tensor scale, s_t = 1).                                         */
+/* Tensor scale (reading: NVFP4 carries one fp32 scale per tensor; the    */
+/* abstract does not say how it is chosen, so it is one dynamic scale per  */
+/* activation tensor from amax over the whole tensor:                      */
+/* s_t = RN32(amax / 2688), 2688 = 448 * 6; s_t = 1 if amax == 0; MXFP4    */
+/* has no tensor scale, s_t = 1).                                          */
 
 float oracle_tensor_scale(const float *v, int64_t count, int fmt)
 {
