@@ -175,6 +175,51 @@ sharq_status sharq_prepare(const void *x_dev, int64_t m_tok, int64_t k,
                            void *stream);
 
 /*
+ * Preparation operator for callers that cannot allocate device memory.
+ * (An interface addition: the SharQ paper has no counterpart.)
+ *
+ * sharq_prepare keeps its working memory (per-row LayerNorm statistics and
+ * the word that collects the tensor's amax) inside the caller's prep buffer.
+ * Some callers cannot provide that: a plugin or custom operator inside
+ * another framework is handed its input and output tensors and owns no
+ * allocator; code on a latency-critical path must not call cudaMalloc,
+ * which waits for the device to go idle; and deployments that plan all
+ * device memory ahead of time have no room for a per-call scratch region.
+ * This entry point computes exactly what sharq_prepare computes (same
+ * kernels, same results bit for bit) but keeps that working memory in one
+ * fixed array compiled into the library: 256 + 8 * SHARQ_NOALLOC_MAX_ROWS
+ * bytes (about 128 KB) on every GPU that loads the library, held until the
+ * process exits. It calls no allocator.
+ *
+ *   x_dev, m_tok, k, ln_w_dev, ln_b_dev, eps, n, m, fmt: as sharq_prepare.
+ *   Outputs (device, 256-byte aligned, sizes in bytes; blk = 16 for NVFP4,
+ *   32 for MXFP4; sf_rows = m_tok rounded up to 128, at least 128):
+ *     s_codes_dev, r_codes_dev   m_tok * k / 2 each (code layout above)
+ *     s_scales_dev, r_scales_dev sf_rows * k / blk each (MMA scale view)
+ *     meta_dev                   m_tok * ceil((k/m) * n * ceil(log2 m) / 8)
+ *     s_t_dev                    1 float (4-byte aligned)
+ *   prep_out  host struct for sharq_linear / sharq_prep_export; its scratch
+ *             pointer refers to the library's array.
+ * Limits and sharing: m_tok <= SHARQ_NOALLOC_MAX_ROWS, else
+ * SHARQ_ERR_UNSUPPORTED and nothing is enqueued. All calls share the one
+ * array, which keeps the last call's contents (the statistics that
+ * sharq_prep_export returns for prep_out are those of the latest call on the
+ * device); the amax word is cleared at the start of every call. Calls whose
+ * work overlaps on the GPU (different streams, no ordering between them)
+ * race on the array and give wrong results. The first call on a device looks
+ * up the array's device address with the device current; make that first
+ * call before any stream capture.
+ */
+#define SHARQ_NOALLOC_MAX_ROWS 16384
+sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, int64_t k,
+                                   const void *ln_w_dev, const void *ln_b_dev, float eps,
+                                   int n, int m, int fmt,
+                                   void *s_codes_dev, void *r_codes_dev,
+                                   void *s_scales_dev, void *r_scales_dev,
+                                   void *meta_dev, float *s_t_dev,
+                                   sharq_prep *prep_out, void *stream);
+
+/*
  * Dual-path FP4 linear layer. Abstract: "A sparse FP4 GEMM processes the
  * backbone while a dense FP4 GEMM compensates for both mask-induced
  * activation loss and sparse-path quantization error."

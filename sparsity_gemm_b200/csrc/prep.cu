@@ -18,6 +18,8 @@
 //      stores. The second read of x mostly hits L2.
 #include <cuda_fp16.h>
 
+#include <string.h>
+
 #include "sharq_dev.cuh"
 #include "sq_internal.h"
 
@@ -596,6 +598,130 @@ static void *encode_fn(int m) {
         default: return (void *)prep_encode_kernel<FMT, 16>;
     }
 }
+
+// ---------------------------------------------------------------------------
+// Preparation whose scratch lives in the library instead of the caller's
+// buffer (sharq_prepare_noalloc). The statistics kernel's per-row (mu, rstd)
+// and the tensor-amax word go into one fixed device array; every GPU that
+// loads the library holds it until the process exits.
+
+constexpr int64_t kStaticScratchRows = SHARQ_NOALLOC_MAX_ROWS;
+constexpr size_t kStaticScratchBytes = 256 + 8 * (size_t)kStaticScratchRows;  // [0,4) amax word, [256,...) stats
+static __device__ __align__(256) unsigned char g_prep_scratch[kStaticScratchBytes];
+
+// Device address of g_prep_scratch on the current device, looked up once per
+// device (in host code the array's name is only a stand-in for the symbol).
+static sharq_status static_scratch(int dev, unsigned char **out) {
+    static unsigned char *addr[64] = {nullptr};
+    if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
+    if (!addr[dev]) {
+        unsigned char *p = nullptr;
+        if (cudaGetSymbolAddress((void **)&p, g_prep_scratch) != cudaSuccess || !p) return SHARQ_ERR_CUDA;
+        addr[dev] = p;
+    }
+    *out = addr[dev];
+    return SHARQ_OK;
+}
+
+static bool noalloc_aligned(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+}  // namespace sq
+
+extern "C" sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, int64_t k, const void *ln_w_dev,
+                                              const void *ln_b_dev, float eps, int n, int m, int fmt,
+                                              void *s_codes_dev, void *r_codes_dev, void *s_scales_dev,
+                                              void *r_scales_dev, void *meta_dev, float *s_t_dev,
+                                              sharq_prep *prep_out, void *stream) {
+    using namespace sq;
+    const bool fmt_ok = fmt == kFmtNV || fmt == kFmtMX;
+    const bool nm_ok = (m == 2 || m == 4 || m == 8 || m == 16) && n >= 1 && n <= m;
+    if (!fmt_ok || !nm_ok || k <= 0 || k > SHARQ_K_MAX || k % SHARQ_K_ALIGN != 0 || m_tok < 0 || !prep_out ||
+        !s_t_dev)
+        return SHARQ_ERR_INVALID_ARG;
+    if (!(eps > 0.0f) || eps > 3.0e38f) return SHARQ_ERR_INVALID_ARG;
+    if (m_tok > kStaticScratchRows) return SHARQ_ERR_UNSUPPORTED;  // beyond the fixed scratch array
+    if (!s_scales_dev || !r_scales_dev || !noalloc_aligned(s_scales_dev) || !noalloc_aligned(r_scales_dev) ||
+        (reinterpret_cast<uintptr_t>(s_t_dev) & 3u))
+        return SHARQ_ERR_INVALID_ARG;
+    if (m_tok > 0 && (!x_dev || !s_codes_dev || !r_codes_dev || !meta_dev || !noalloc_aligned(s_codes_dev) ||
+                      !noalloc_aligned(r_codes_dev) || !noalloc_aligned(meta_dev) ||
+                      (reinterpret_cast<uintptr_t>(x_dev) & 15u)))
+        return SHARQ_ERR_INVALID_ARG;
+    if ((ln_w_dev && (reinterpret_cast<uintptr_t>(ln_w_dev) & 15u)) ||
+        (ln_b_dev && (reinterpret_cast<uintptr_t>(ln_b_dev) & 15u)))
+        return SHARQ_ERR_INVALID_ARG;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SHARQ_ERR_CUDA;
+    unsigned char *scratch = nullptr;
+    sharq_status st = static_scratch(dev, &scratch);
+    if (st != SHARQ_OK) return st;
+    static int sms[64] = {0};
+    if (!sms[dev] && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return SHARQ_ERR_CUDA;
+    static bool attr_done[64] = {false};
+    if (!attr_done[dev]) {
+        if (cudaFuncSetAttribute(ln_stats_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)(2 * SHARQ_K_MAX)) != cudaSuccess)
+            return SHARQ_ERR_CUDA;
+        attr_done[dev] = true;
+    }
+
+    const PrepLayout L = prep_layout(m_tok, k, n, m, fmt);
+    sharq_prep P;
+    memset(&P, 0, sizeof(P));
+    P.m_tok = m_tok;
+    P.k = k;
+    P.n = n;
+    P.m = m;
+    P.fmt = fmt;
+    P.sf_rows = L.sf_rows;
+    P.meta_row_bytes = L.meta_row;
+    P.s_codes = s_codes_dev;
+    P.r_codes = r_codes_dev;
+    P.s_scales = s_scales_dev;
+    P.r_scales = r_scales_dev;
+    P.meta = meta_dev;
+    P.tensor_scale = s_t_dev;
+    P.scratch = scratch + 256;  // per-row (mu, rstd)
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned *amax_word = reinterpret_cast<unsigned *>(scratch);
+    float2 *stats = reinterpret_cast<float2 *>(scratch + 256);
+    if (cudaMemsetAsync(amax_word, 0, sizeof(unsigned), s) != cudaSuccess) return SHARQ_ERR_CUDA;
+    const bool meta_atomic = ((kUnit / m) * n * idx_bits(m)) % 8 != 0;
+    if (meta_atomic && m_tok > 0 && cudaMemsetAsync(meta_dev, 0, (size_t)(m_tok * L.meta_row), s) != cudaSuccess)
+        return SHARQ_ERR_CUDA;
+    if (m_tok > 0) {
+        if (ln_w_dev || ln_b_dev)
+            ln_stats_kernel<true><<<(unsigned)m_tok, kStatsThreads, (size_t)(2 * k), s>>>(
+                (const uint16_t *)x_dev, (const uint16_t *)ln_w_dev, (const uint16_t *)ln_b_dev, eps, k, stats,
+                amax_word);
+        else
+            ln_stats_kernel<false><<<(unsigned)m_tok, kStatsThreads, 0, s>>>((const uint16_t *)x_dev, nullptr, nullptr,
+                                                                           eps, k, stats, amax_word);
+    }
+    const int64_t total = P.sf_rows * (k / kUnit);
+    int64_t blocks = (total + kEncodeThreads - 1) / kEncodeThreads;
+    if (blocks > (int64_t)sms[dev] * 16) blocks = (int64_t)sms[dev] * 16;
+    void *fn = fmt == kFmtNV ? encode_fn<kFmtNV>(m) : encode_fn<kFmtMX>(m);
+    const uint16_t *xx = (const uint16_t *)x_dev, *gg = (const uint16_t *)ln_w_dev, *bb = (const uint16_t *)ln_b_dev;
+    const float2 *cst = stats;
+    const unsigned *aw = amax_word;
+    float *sto = s_t_dev;
+    int64_t mt = m_tok, sfr = P.sf_rows, kk = k, mrow = L.meta_row;
+    int nn = n;
+    uint8_t *sc = (uint8_t *)s_codes_dev, *rc = (uint8_t *)r_codes_dev, *ss = (uint8_t *)s_scales_dev,
+            *rs = (uint8_t *)r_scales_dev, *mt8 = (uint8_t *)meta_dev;
+    void *args[] = {&xx, &gg, &bb, &cst, &aw, &sto, &mt, &sfr, &kk, &nn, &sc, &rc, &ss, &rs, &mt8, &mrow};
+    if (cudaLaunchKernel(fn, dim3((unsigned)blocks), dim3(kEncodeThreads), args, 0, s) != cudaSuccess)
+        return SHARQ_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return SHARQ_ERR_CUDA;
+    *prep_out = P;
+    return SHARQ_OK;
+}
+
+namespace sq {
 
 sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, const void *gamma, const void *beta,
                             float eps) {
