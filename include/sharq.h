@@ -3,14 +3,14 @@
  * (sm_100a).
  *
  * Method: "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM
- * Inference" (arXiv 2606.26587), Abstract. For each activation tensor a
- * fused preparation operator applies layer normalization, generates an
- * input-adaptive N:M mask that extracts an outlier-dominated sparse backbone
- * S, quantizes S to FP4, defines a dense residual R relative to the
- * quantized backbone (R = X_ln - deq(Q(S))) and quantizes R to FP4. A sparse
- * FP4 GEMM on the backbone and a dense FP4 GEMM on the residual read one
- * shared FP4 weight payload through path-specific scale views, and their
- * results are summed.
+ * Inference" (arXiv 2606.26587), Abstract. Each activation tensor goes
+ * through one fused preparation operator: LayerNorm; a per-row N:M mask,
+ * chosen from the data, that keeps a sparse backbone S of the large
+ * (outlier) values; FP4 quantization of S; the dense residual
+ * R = X_ln - deq(Q(S)), measured from the quantized backbone; and FP4
+ * quantization of R. A sparse FP4 GEMM on Q(S) and a dense FP4 GEMM on Q(R)
+ * use the same FP4 weight codes, each with a scale view of its own, and
+ * their results are added.
  *
  * Formats: SHARQ_NVFP4 = E2M1 codes, one UE4M3 scale per 16 elements and one
  * fp32 tensor scale; SHARQ_MXFP4 = E2M1 codes and one E8M0 scale per 32
@@ -94,7 +94,11 @@ typedef struct sharq_wq {
     int64_t n_out;       /* output features (rows of W) */
     int64_t k;           /* input features */
     int32_t fmt;         /* sharq_fmt */
-    int32_t reserved;
+    int32_t groups;      /* stacked weights (experts): 1 (0 reads as 1), or
+                            n_groups from sharq_quantize_weight_grouped;
+                            group g's payload is g * sharq_weight_bytes(n_out,
+                            k, fmt) bytes after group 0's, which every pointer
+                            refers to */
     int64_t sf_rows;     /* rows of the scale layout: n_out rounded up to 256 */
     void *codes;         /* device, [n_out][k/2] bytes */
     void *scales_backbone; /* device, MMA scale view for the backbone path */
@@ -109,7 +113,8 @@ typedef struct sharq_prep {
     int64_t k;           /* input features */
     int32_t n, m;        /* N:M ratio of the mask */
     int32_t fmt;         /* sharq_fmt */
-    int32_t reserved;
+    int32_t groups;      /* 1 (0 reads as 1), or n_groups for the output of
+                            sharq_gather_rows */
     int64_t sf_rows;     /* rows of the scale layouts: m_tok rounded up to 128 */
     int64_t meta_row_bytes;
     void *s_codes;       /* device, backbone Q(S) codes [m_tok][k/2] (zeros off the mask) */
@@ -129,8 +134,8 @@ size_t sharq_weight_bytes(int64_t n_out, int64_t k, int fmt);
 size_t sharq_prep_bytes(int64_t m_tok, int64_t k, int n, int m, int fmt);
 
 /*
- * Weight quantization (offline). Abstract: "The two paths share a single FP4
- * weight payload with path-specific scale views."
+ * Weight quantization (offline). SharQ, Abstract: both GEMM paths read one
+ * FP4 weight payload, each through a scale view of its own.
  *   w_dev    fp16 [n_out][k] row-major (K-major), so the layer computes X W^T.
  *   wq_dev   device buffer of at least sharq_weight_bytes(n_out, k, fmt).
  *   wq_out   host struct, filled with pointers into wq_dev.
@@ -146,9 +151,8 @@ sharq_status sharq_quantize_weight(const void *w_dev, int64_t n_out, int64_t k, 
                                    void *stream);
 
 /*
- * Fused preparation operator (per activation). Abstract: "a fused
- * preparation kernel absorbs mask generation, residual construction, and
- * layer normalization into one operator."
+ * Fused preparation operator (per activation). SharQ, Abstract: LayerNorm,
+ * mask generation and residual construction are done by one fused operator.
  *   x_dev     fp16 [m_tok][k] row-major activations.
  *   ln_w_dev  fp16 [k] LayerNorm gamma, or NULL (no multiply).
  *   ln_b_dev  fp16 [k] LayerNorm beta, or NULL (no add; -0 is preserved).
@@ -220,9 +224,9 @@ sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, int64_t k,
                                    sharq_prep *prep_out, void *stream);
 
 /*
- * Dual-path FP4 linear layer. Abstract: "A sparse FP4 GEMM processes the
- * backbone while a dense FP4 GEMM compensates for both mask-induced
- * activation loss and sparse-path quantization error."
+ * Dual-path FP4 linear layer. SharQ, Abstract: the backbone goes through a
+ * sparse FP4 GEMM, and a dense FP4 GEMM on the residual makes up both for
+ * what the mask dropped and for the backbone's quantization error.
  *   out_dev  fp16 [m_tok][n_out] row-major:
  *     out = RN16( s_t * s_tW * sum_k (Q(S) + Q(R))[i,k] * Q(W)[j,k] )
  *   with the block-scaled code values; products are exact, accumulation is
@@ -258,11 +262,14 @@ sharq_status sharq_weight_export(const sharq_wq *wq, uint8_t *codes_host,
 
 /* Synchronizes `stream`, then reports (and clears) the device status word:
  * SHARQ_ERR_TIMEOUT if a bounded wait ran out since the last call,
- * SHARQ_ERR_CUDA if the stream holds a CUDA error, else SHARQ_OK. */
+ * SHARQ_ERR_INVALID_ARG if a device-side argument check failed (grouped
+ * routing arrays), SHARQ_ERR_CUDA if the stream holds a CUDA error, else
+ * SHARQ_OK. The first such event since the last call is the one reported. */
 sharq_status sharq_get_last_error(void *stream);
 
-/* Where the last SHARQ_ERR_TIMEOUT came from (an internal site code), 0 if
- * none. Valid after sharq_get_last_error returned SHARQ_ERR_TIMEOUT. */
+/* Where the last SHARQ_ERR_TIMEOUT or device-side SHARQ_ERR_INVALID_ARG
+ * came from (an internal site code; 0x2xx = argument checks), 0 if none.
+ * Valid after sharq_get_last_error returned one of them. */
 uint32_t sharq_last_timeout_site(void);
 
 /* Test hook: the wait limit of the GEMM's bounded waits, in nanoseconds

@@ -8,11 +8,11 @@
  *
  * What it computes comes from the SharQ abstract ("SharQ: Bridging Activation
  * Sparsity and FP4 Quantization for LLM Inference", arXiv 2606.26587,
- * Abstract): LayerNorm, an input-adaptive N:M mask that extracts an
- * outlier-dominated sparse backbone S, FP4 quantization of S, a dense
- * residual R = X_ln - deq(Q(S)) taken against the quantized backbone, FP4
- * quantization of R, and two FP4 GEMMs against one shared FP4 weight payload
- * whose outputs are summed. The abstract leaves the arithmetic open; each
+ * Abstract): LayerNorm; per row, an N:M mask chosen from the data that keeps
+ * a sparse backbone S holding the large (outlier) values; FP4 quantization
+ * of S; a dense residual R = X_ln - deq(Q(S)), measured from the quantized
+ * backbone; FP4 quantization of R; and two FP4 GEMMs that use the same FP4
+ * weight codes and whose outputs are added. The abstract leaves the arithmetic open; each
  * function below states the reading it implements.
  *
  * Formats: NVFP4 = E2M1 codes, one UE4M3 scale per 16 elements and one fp32
@@ -380,8 +380,8 @@ static double block_value(int fmt, const uint8_t *codes, const uint8_t *scales,
 }
 
 /* Dual-path linear: the backbone GEMM on Q(S) and the residual GEMM on    */
-/* Q(R) against the same Q(W), summed (abstract: "A sparse FP4 GEMM        */
-/* processes the backbone while a dense FP4 GEMM compensates"):             */
+/* Q(R) against the same Q(W), summed (SharQ, Abstract: a sparse GEMM for  */
+/* the backbone, a dense one for the residual):                             */
 /*   out[i][j] = s_t * s_tW * sum_k (aS[i][k] + aR[i][k]) * w[j][k]         */
 /* with a, w the block-scaled code values, in binary64 (every product is    */
 /* exact; only the sum rounds). bound[i][j] is the same sum over absolute   */

@@ -34,14 +34,14 @@ class SharqError(RuntimeError):
 
 
 class SharqWQ(C.Structure):
-    _fields_ = [("n_out", C.c_int64), ("k", C.c_int64), ("fmt", C.c_int32), ("reserved", C.c_int32),
+    _fields_ = [("n_out", C.c_int64), ("k", C.c_int64), ("fmt", C.c_int32), ("groups", C.c_int32),
                 ("sf_rows", C.c_int64), ("codes", C.c_void_p), ("scales_backbone", C.c_void_p),
                 ("scales_residual", C.c_void_p), ("tensor_scale", C.c_void_p), ("scratch", C.c_void_p)]
 
 
 class SharqPrep(C.Structure):
     _fields_ = [("m_tok", C.c_int64), ("k", C.c_int64), ("n", C.c_int32), ("m", C.c_int32),
-                ("fmt", C.c_int32), ("reserved", C.c_int32), ("sf_rows", C.c_int64),
+                ("fmt", C.c_int32), ("groups", C.c_int32), ("sf_rows", C.c_int64),
                 ("meta_row_bytes", C.c_int64), ("s_codes", C.c_void_p), ("r_codes", C.c_void_p),
                 ("s_scales", C.c_void_p), ("r_scales", C.c_void_p), ("meta", C.c_void_p),
                 ("tensor_scale", C.c_void_p), ("scratch", C.c_void_p)]

@@ -46,6 +46,7 @@ void fill_prep(sharq_prep *P, void *buf, int64_t m_tok, int64_t k, int n, int m,
     uint8_t *b = static_cast<uint8_t *>(buf);
     memset(P, 0, sizeof(*P));
     P->m_tok = m_tok;
+    P->groups = 1;
     P->k = k;
     P->n = n;
     P->m = m;
@@ -66,6 +67,7 @@ void fill_wq(sharq_wq *W, void *buf, int64_t n_out, int64_t k, int fmt) {
     uint8_t *b = static_cast<uint8_t *>(buf);
     memset(W, 0, sizeof(*W));
     W->n_out = n_out;
+    W->groups = 1;
     W->k = k;
     W->fmt = fmt;
     W->sf_rows = L.sf_rows;

@@ -1,9 +1,9 @@
 // Dual-path FP4 GEMM of SharQ on sm_100a (tcgen05 block-scaled MMA).
 //
 // "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM
-// Inference", Abstract: a sparse FP4 GEMM processes the backbone while a
-// dense FP4 GEMM compensates; the two paths share a single FP4 weight payload
-// with path-specific scale views. Here both paths issue into ONE tensor-memory
+// Inference", Abstract: a sparse FP4 GEMM on the backbone and a dense FP4
+// GEMM on the residual, both on the same FP4 weight codes (each path with a
+// scale view of its own), added together. Here both paths issue into ONE tensor-memory
 // accumulator, and every W tile (codes and scale view) is loaded once per
 // K step and read by both paths' MMAs:
 //     acc = sum_k Q(S)[i,k] W[j,k] + Q(R)[i,k] W[j,k]      (block-scaled)

@@ -1,9 +1,9 @@
 // Fused preparation operator of SharQ on sm_100a.
 //
 // "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM
-// Inference", Abstract: a fused preparation kernel absorbs mask generation,
-// residual construction and layer normalization into one operator; the
-// residual is defined relative to the quantized sparse backbone.
+// Inference", Abstract: one fused operator does the LayerNorm, builds the
+// mask and forms the residual, which is taken from the quantized backbone
+// (not from the unquantized sparse values).
 //
 // Two passes over the activations, because the NVFP4 tensor scale depends on
 // amax(X_ln) over the whole tensor:

@@ -1,8 +1,8 @@
 // Weight quantization (offline) of SharQ on sm_100a.
 //
 // "SharQ: Bridging Activation Sparsity and FP4 Quantization for LLM
-// Inference", Abstract: the two GEMM paths share a single FP4 weight payload
-// with path-specific scale views. This kernel pair writes that payload: one
+// Inference", Abstract: both GEMM paths read the same FP4 weight codes, each
+// through a scale view of its own. This kernel pair writes that payload: one
 // E2M1 code matrix and one block-scale matrix in the tcgen05 MMA scale layout,
 // which both paths' scale views point at (the same values, as the
 // dequantized weight must be identical on both paths).
