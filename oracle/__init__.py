@@ -256,3 +256,46 @@ def linear_prepared(p: Prepared, qw: QWeight, rows=None):
     sel = slice(None) if rows is None else rows
     return linear(p.s_codes[sel], p.s_scales[sel], p.r_codes[sel], p.r_scales[sel], p.s_t,
                   qw.codes, qw.scales, qw.s_tw, p.fmt)
+
+
+# --------------------------------------------------------------------------
+# Mixture-of-experts grouped variant. The SharQ abstract names Qwen3-30B-A3B
+# (a mixture-of-experts model) among its models without describing the
+# expert layers. Reading: each expert's linear is the dual-path linear over
+# the rows routed to it; the activation is prepared once over all rows (one
+# tensor scale); each expert's weight is quantized on its own.
+
+
+def expert_of(offsets, i):
+    """Group of grouped row i: the g with offsets[g] <= i < offsets[g+1]."""
+    offsets = np.asarray(offsets)
+    g = int(np.searchsorted(offsets, i, side="right")) - 1
+    assert 0 <= g < len(offsets) - 1 and offsets[g] <= i < offsets[g + 1]
+    return g
+
+
+def quantize_weight_grouped(w, fmt: int) -> list:
+    """One QWeight per expert; w is [groups][n_out][k]."""
+    return [quantize_weight(w[g], fmt) for g in range(w.shape[0])]
+
+
+def linear_grouped(p: Prepared, row_idx, offsets, qws: list, sel=None, cols=None):
+    """out[i] = the dual-path linear of expert g's weight on prepared row
+    row_idx[i], for grouped rows i of expert g (offsets[g] <= i <
+    offsets[g+1]). sel: grouped rows to compute (default all); cols: output
+    columns (default all). Returns (out, bound) like linear()."""
+    offsets = np.asarray(offsets)
+    row_idx = np.asarray(row_idx)
+    sel = np.arange(int(offsets[-1])) if sel is None else np.asarray(sel)
+    cols = slice(None) if cols is None else np.asarray(cols)
+    n_out = qws[0].codes[cols].shape[0]
+    out = np.zeros((len(sel), n_out), np.float64)
+    bound = np.zeros((len(sel), n_out), np.float64)
+    for j, i in enumerate(sel):
+        g = expert_of(offsets, int(i))
+        t = int(row_idx[int(i)])
+        qw = qws[g]
+        o, b = linear(p.s_codes[t:t + 1], p.s_scales[t:t + 1], p.r_codes[t:t + 1], p.r_scales[t:t + 1],
+                      p.s_t, qw.codes[cols], qw.scales[cols], qw.s_tw, p.fmt)
+        out[j], bound[j] = o[0], b[0]
+    return out, bound
