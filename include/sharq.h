@@ -238,6 +238,91 @@ sharq_status sharq_linear(const sharq_prep *prep, const sharq_wq *wq, void *out_
                           void *stream);
 
 /*
+ * Mixture-of-experts grouped variant.
+ *
+ * The SharQ Abstract lists Qwen3-30B-A3B, a mixture-of-experts model, among
+ * the evaluated models but does not say how expert layers are computed. The
+ * reading taken here: each expert's linear is the dual-path linear above,
+ * applied to the rows (tokens) routed to that expert; an activation tensor
+ * is prepared ONCE over all its rows, so one tensor scale s_t covers every
+ * row of every expert; each expert's weight is quantized on its own (its
+ * own s_tW). Three calls:
+ *   sharq_quantize_weight_grouped  the experts' weights, stacked
+ *   sharq_gather_rows              prepared rows -> expert-grouped order
+ *   sharq_linear_grouped           one launch over all experts' tiles
+ *
+ * Routing is given by device arrays, so that it can come from a router
+ * kernel without a host round trip:
+ *   offsets_dev  int32 [n_groups + 1]: offsets[0] = 0, nondecreasing,
+ *                offsets[n_groups] = rows. Grouped rows offsets[g] ..
+ *                offsets[g+1]-1 belong to group (expert) g.
+ *   row_idx_dev  int32 [rows]: grouped row i is prepared row row_idx[i].
+ * The kernels check these on the device. On a violation they write no
+ * output, and sharq_get_last_error then reports SHARQ_ERR_INVALID_ARG.
+ */
+#define SHARQ_GROUPS_MAX 1024
+
+/* Bytes of the buffer sharq_quantize_weight_grouped needs:
+ * n_groups * sharq_weight_bytes(n_out, k, fmt). 0 if invalid. */
+size_t sharq_weight_bytes_grouped(int64_t n_groups, int64_t n_out, int64_t k, int fmt);
+
+/* Quantizes n_groups weights in one call, each exactly as
+ * sharq_quantize_weight would (its own tensor scale and block scales).
+ *   w_dev   fp16 [n_groups][n_out][k] row-major.
+ *   wq_out  host struct describing group 0, with groups = n_groups.
+ * Preconditions: 1 <= n_groups <= SHARQ_GROUPS_MAX, plus those of
+ * sharq_quantize_weight. */
+sharq_status sharq_quantize_weight_grouped(const void *w_dev, int64_t n_groups, int64_t n_out, int64_t k,
+                                           int fmt, void *wq_dev, size_t wq_bytes, sharq_wq *wq_out,
+                                           void *stream);
+
+/* Rows of a grouped prep. Each group starts at a multiple of 128 rows, so
+ * that no 128-row GEMM tile spans two groups: rows + 127 * n_groups, rounded
+ * up to 128. -1 if invalid. */
+int64_t sharq_grouped_rows(int64_t rows, int64_t n_groups);
+
+/* Bytes of the buffer sharq_gather_rows needs:
+ * sharq_prep_bytes(sharq_grouped_rows(rows, n_groups), k, n, m, fmt). */
+size_t sharq_gather_bytes(int64_t rows, int64_t n_groups, int64_t k, int n, int m, int fmt);
+
+/*
+ * Copies prepared rows into expert-grouped order. No arithmetic: the codes,
+ * block scales, mask metadata and LayerNorm statistics of each row move bit
+ * for bit, and the tensor scale is copied.
+ *   src          a prep from sharq_prepare.
+ *   row_idx_dev  as above; NULL means row_idx[i] = i (src already in
+ *                grouped order, as a down projection's input is).
+ *   offsets_dev, n_groups, rows: as above; 1 <= n_groups <=
+ *                SHARQ_GROUPS_MAX, 0 <= rows <= 2^30.
+ *   dst_dev      buffer of at least sharq_gather_bytes(...) bytes.
+ *   dst_out      host struct: m_tok = sharq_grouped_rows(rows, n_groups),
+ *                groups = n_groups. Grouped row i of group g is stored at
+ *                row 128 * T_g + (i - offsets[g]), where T_g counts the
+ *                128-row tiles of groups 0 .. g-1 (ceil(size / 128) each).
+ *                Every other row is zero (codes, scales, metadata and
+ *                statistics).
+ * Device-side checks: the offsets as above, and 0 <= row_idx[i] < src->m_tok.
+ */
+sharq_status sharq_gather_rows(const sharq_prep *src, const int32_t *row_idx_dev, const int32_t *offsets_dev,
+                               int64_t n_groups, int64_t rows, void *dst_dev, size_t dst_bytes,
+                               sharq_prep *dst_out, void *stream);
+
+/*
+ * Grouped dual-path FP4 linear: for every group g and grouped row i of g,
+ *   out[i][j] = RN16( s_t * s_tW[g] * sum_k (Q(S) + Q(R))[i,k] * Q(W_g)[j,k] )
+ * with the terms of sharq_linear. One persistent launch walks the 128 x 256
+ * output tiles of all groups.
+ *   prep     from sharq_gather_rows with the same offsets and n_groups.
+ *   wq       from sharq_quantize_weight_grouped with groups == n_groups.
+ *   out_dev  fp16 [rows][n_out] row-major, grouped order.
+ * Preconditions: those of sharq_linear, plus prep->groups == wq->groups ==
+ * n_groups and rows <= prep->m_tok. Device-side checks: the offsets, and
+ * that the rows they pad to fit in prep->m_tok.
+ */
+sharq_status sharq_linear_grouped(const sharq_prep *prep, const int32_t *offsets_dev, int64_t n_groups,
+                                  int64_t rows, const sharq_wq *wq, void *out_dev, void *stream);
+
+/*
  * Canonical host copies of a prepared activation, for inspection and tests.
  * Synchronizes `stream`. Every output may be NULL. One value per byte:
  *   idx_host      [m_tok][k/m][n] kept positions, ascending

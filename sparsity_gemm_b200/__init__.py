@@ -75,11 +75,21 @@ def lib():
         L.sharq_selftest_wait.restype = i32
         L.sharq_selftest_division.argtypes = [C.c_uint64, C.c_uint64, C.POINTER(C.c_uint64), vp, vp]
         L.sharq_selftest_division.restype = i32
+        L.sharq_weight_bytes_grouped.argtypes = [i64, i64, i64, i32]
+        L.sharq_weight_bytes_grouped.restype = sz
+        L.sharq_quantize_weight_grouped.argtypes = [vp, i64, i64, i64, i32, vp, sz, C.POINTER(SharqWQ), vp]
+        L.sharq_grouped_rows.argtypes = [i64, i64]
+        L.sharq_grouped_rows.restype = i64
+        L.sharq_gather_bytes.argtypes = [i64, i64, i64, i32, i32, i32]
+        L.sharq_gather_bytes.restype = sz
+        L.sharq_gather_rows.argtypes = [C.POINTER(SharqPrep), vp, vp, i64, i64, vp, sz, C.POINTER(SharqPrep), vp]
+        L.sharq_linear_grouped.argtypes = [C.POINTER(SharqPrep), vp, i64, i64, C.POINTER(SharqWQ), vp, vp]
         L.sharq_status_string.argtypes = [i32]
         L.sharq_status_string.restype = C.c_char_p
         L.sharq_last_launch_count.restype = i32
         for name in ("sharq_quantize_weight", "sharq_prepare", "sharq_linear", "sharq_prep_export",
-                     "sharq_weight_export", "sharq_get_last_error"):
+                     "sharq_weight_export", "sharq_get_last_error", "sharq_quantize_weight_grouped",
+                     "sharq_gather_rows", "sharq_linear_grouped"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -212,6 +222,76 @@ def weight_export(qw: QuantizedWeight, stream=None) -> dict:
     _check(lib().sharq_weight_export(C.byref(d), p(out["codes"]), p(out["scales"]), p(out["scales_residual"]),
                                      p(out["s_tw"]), _stream(stream)), "sharq_weight_export")
     out["s_tw"] = out["s_tw"][0]
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Mixture-of-experts grouped variant
+
+
+def quantize_weight_grouped(w: torch.Tensor, fmt: int = NVFP4, stream=None) -> QuantizedWeight:
+    """Offline FP4 quantization of a stack of weights w [groups, n_out, k]
+    (fp16, CUDA), each with its own tensor scale."""
+    assert w.dtype == torch.float16 and w.is_cuda and w.dim() == 3 and w.is_contiguous()
+    groups, n_out, k = w.shape
+    nbytes = int(lib().sharq_weight_bytes_grouped(groups, n_out, k, fmt))
+    if nbytes == 0:
+        raise SharqError(ERR_INVALID_ARG, f"grouped weight shape {tuple(w.shape)} fmt {fmt}")
+    buf = _device_buffer(nbytes, w.device)
+    desc = SharqWQ()
+    _check(lib().sharq_quantize_weight_grouped(_ptr(w), groups, n_out, k, fmt, _ptr(buf), nbytes, C.byref(desc),
+                                               _stream(stream)), "sharq_quantize_weight_grouped")
+    return QuantizedWeight(buf, desc)
+
+
+def group_view(qw: QuantizedWeight, g: int) -> QuantizedWeight:
+    """A plain (one-group) descriptor of group g of a stacked weight; it
+    shares qw's buffer."""
+    d = qw.desc
+    assert 0 <= g < max(1, d.groups)
+    stride = weight_bytes(d.n_out, d.k, d.fmt) * g
+    v = SharqWQ()
+    C.pointer(v)[0] = d
+    v.groups = 1
+    for f in ("codes", "scales_backbone", "scales_residual", "tensor_scale", "scratch"):
+        setattr(v, f, getattr(d, f) + stride)
+    return QuantizedWeight(qw.buf, v)
+
+
+def grouped_rows(rows: int, groups: int) -> int:
+    return int(lib().sharq_grouped_rows(rows, groups))
+
+
+def gather_rows(prep: Prepared, row_idx, offsets: torch.Tensor, rows: int, out: Prepared | None = None,
+                stream=None) -> Prepared:
+    """Expert-grouped copy of prepared rows: grouped row i of group g (offsets
+    [g] <= i < offsets[g+1]) is prepared row row_idx[i] (row_idx None: i).
+    row_idx and offsets are int32 CUDA tensors."""
+    for t in (row_idx, offsets):
+        assert t is None or (t.dtype == torch.int32 and t.is_cuda and t.is_contiguous())
+    groups = offsets.numel() - 1
+    d = prep.desc
+    nbytes = int(lib().sharq_gather_bytes(rows, groups, d.k, d.n, d.m, d.fmt))
+    if nbytes == 0:
+        raise SharqError(ERR_INVALID_ARG, f"gather rows {rows} groups {groups}")
+    buf = out.buf if out is not None and out.buf.numel() >= nbytes else _device_buffer(nbytes, prep.buf.device)
+    desc = SharqPrep()
+    _check(lib().sharq_gather_rows(C.byref(d), _ptr(row_idx), _ptr(offsets), groups, rows, _ptr(buf), buf.numel(),
+                                   C.byref(desc), _stream(stream)), "sharq_gather_rows")
+    return Prepared(buf, desc)
+
+
+def linear_grouped(prep: Prepared, offsets: torch.Tensor, qw: QuantizedWeight, rows: int,
+                   out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Grouped dual-path FP4 linear: fp16 [rows, n_out] in grouped order,
+    group g's rows through group g's weight."""
+    assert offsets.dtype == torch.int32 and offsets.is_cuda and offsets.is_contiguous()
+    if out is None:
+        out = torch.empty((rows, qw.n_out), dtype=torch.float16, device=prep.buf.device)
+    assert out.dtype == torch.float16 and out.is_contiguous() and tuple(out.shape) == (rows, qw.n_out)
+    optr = _ptr(out) if out.numel() else None
+    _check(lib().sharq_linear_grouped(C.byref(prep.desc), _ptr(offsets), offsets.numel() - 1, rows, C.byref(qw.desc),
+                                      optr, _stream(stream)), "sharq_linear_grouped")
     return out
 
 

@@ -13,7 +13,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libsharq.so")
-SOURCES = ["api.cu", "prep.cu", "wquant.cu", "gemm.cu"]
+SOURCES = ["api.cu", "prep.cu", "wquant.cu", "gemm.cu", "group.cu"]
 HEADERS = ["layout.h", "sharq_dev.cuh", "sq_internal.h", os.path.join("..", "..", "include", "sharq.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

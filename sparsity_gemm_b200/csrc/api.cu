@@ -135,7 +135,7 @@ sharq_status sharq_quantize_weight(const void *w_dev, int64_t n_out, int64_t k, 
     sharq_status st = make_ctx(stream, ctx);
     if (st != SHARQ_OK) return st;
     fill_wq(wq_out, wq_dev, n_out, k, fmt);
-    st = sq::launch_quantize_weight(ctx, *wq_out, w_dev);
+    st = sq::launch_quantize_weight(ctx, *wq_out, w_dev, 1, (int64_t)need);
     g_last_launches = ctx.launches;
     return st;
 }
@@ -166,6 +166,7 @@ sharq_status sharq_linear(const sharq_prep *prep, const sharq_wq *wq, void *out_
     if (!prep || !wq) return SHARQ_ERR_INVALID_ARG;
     if (!fmt_ok(prep->fmt) || prep->fmt != wq->fmt || prep->k != wq->k || !k_ok(prep->k)) return SHARQ_ERR_INVALID_ARG;
     if (wq->n_out < 1 || wq->n_out % SHARQ_N_ALIGN != 0 || prep->m_tok < 0) return SHARQ_ERR_INVALID_ARG;
+    if (wq->groups > 1) return SHARQ_ERR_INVALID_ARG;  // stacked weights: sharq_linear_grouped
     if (prep->sf_rows < prep->m_tok || wq->sf_rows < wq->n_out || wq->sf_rows % sq::kWRowPad != 0 ||
         prep->sf_rows % sq::kActRowPad != 0)
         return SHARQ_ERR_INVALID_ARG;
@@ -178,6 +179,92 @@ sharq_status sharq_linear(const sharq_prep *prep, const sharq_wq *wq, void *out_
     sharq_status st = make_ctx(stream, ctx);
     if (st != SHARQ_OK) return st;
     st = sq::launch_linear(ctx, *prep, *wq, out_dev);
+    g_last_launches = ctx.launches;
+    return st;
+}
+
+size_t sharq_weight_bytes_grouped(int64_t n_groups, int64_t n_out, int64_t k, int fmt) {
+    const size_t one = sharq_weight_bytes(n_out, k, fmt);
+    if (!one || n_groups < 1 || n_groups > sq::kGroupsMax) return 0;
+    return one * (size_t)n_groups;
+}
+
+sharq_status sharq_quantize_weight_grouped(const void *w_dev, int64_t n_groups, int64_t n_out, int64_t k, int fmt,
+                                           void *wq_dev, size_t wq_bytes, sharq_wq *wq_out, void *stream) {
+    g_last_launches = 0;
+    const size_t need = sharq_weight_bytes_grouped(n_groups, n_out, k, fmt);
+    if (!need || !w_dev || !wq_dev || !wq_out || wq_bytes < need) return SHARQ_ERR_INVALID_ARG;
+    if (!aligned(w_dev, 16) || !aligned(wq_dev, sq::kAlign)) return SHARQ_ERR_INVALID_ARG;
+    sq::LaunchCtx ctx;
+    sharq_status st = make_ctx(stream, ctx);
+    if (st != SHARQ_OK) return st;
+    fill_wq(wq_out, wq_dev, n_out, k, fmt);
+    wq_out->groups = (int32_t)n_groups;
+    st = sq::launch_quantize_weight(ctx, *wq_out, w_dev, n_groups, (int64_t)(need / (size_t)n_groups));
+    g_last_launches = ctx.launches;
+    return st;
+}
+
+int64_t sharq_grouped_rows(int64_t rows, int64_t n_groups) {
+    if (rows < 0 || rows > (1ll << 30) || n_groups < 1 || n_groups > sq::kGroupsMax) return -1;
+    return sq::grouped_rows(rows, n_groups);
+}
+
+size_t sharq_gather_bytes(int64_t rows, int64_t n_groups, int64_t k, int n, int m, int fmt) {
+    const int64_t cap = sharq_grouped_rows(rows, n_groups);
+    return cap < 0 ? 0 : sharq_prep_bytes(cap, k, n, m, fmt);
+}
+
+sharq_status sharq_gather_rows(const sharq_prep *src, const int32_t *row_idx_dev, const int32_t *offsets_dev,
+                               int64_t n_groups, int64_t rows, void *dst_dev, size_t dst_bytes, sharq_prep *dst_out,
+                               void *stream) {
+    g_last_launches = 0;
+    if (!src || !offsets_dev || !dst_dev || !dst_out) return SHARQ_ERR_INVALID_ARG;
+    if (!fmt_ok(src->fmt) || !nm_ok(src->n, src->m) || !k_ok(src->k) || src->m_tok < 0 || src->m_tok > (1ll << 30))
+        return SHARQ_ERR_INVALID_ARG;
+    if (src->meta_row_bytes != sq::meta_row_bytes(src->k, src->n, src->m) || src->sf_rows < src->m_tok ||
+        src->sf_rows % sq::kActRowPad != 0)
+        return SHARQ_ERR_INVALID_ARG;
+    if (src->m_tok > 0 && (!src->s_codes || !src->r_codes || !src->s_scales || !src->r_scales || !src->meta ||
+                           !src->scratch || !src->tensor_scale))
+        return SHARQ_ERR_INVALID_ARG;
+    if (!src->tensor_scale) return SHARQ_ERR_INVALID_ARG;
+    const size_t need = sharq_gather_bytes(rows, n_groups, src->k, src->n, src->m, src->fmt);
+    if (!need || dst_bytes < need || !aligned(dst_dev, sq::kAlign) || !aligned(offsets_dev, 4) ||
+        (row_idx_dev && !aligned(row_idx_dev, 4)))
+        return SHARQ_ERR_INVALID_ARG;
+    if (rows > 0 && !row_idx_dev && rows > src->m_tok) return SHARQ_ERR_INVALID_ARG;
+    sq::LaunchCtx ctx;
+    sharq_status st = make_ctx(stream, ctx);
+    if (st != SHARQ_OK) return st;
+    fill_prep(dst_out, dst_dev, sq::grouped_rows(rows, n_groups), src->k, src->n, src->m, src->fmt);
+    dst_out->groups = (int32_t)n_groups;
+    st = sq::launch_gather(ctx, *src, row_idx_dev, offsets_dev, (int32_t)n_groups, rows, *dst_out);
+    g_last_launches = ctx.launches;
+    return st;
+}
+
+sharq_status sharq_linear_grouped(const sharq_prep *prep, const int32_t *offsets_dev, int64_t n_groups, int64_t rows,
+                                  const sharq_wq *wq, void *out_dev, void *stream) {
+    g_last_launches = 0;
+    if (!prep || !wq || !offsets_dev || !aligned(offsets_dev, 4)) return SHARQ_ERR_INVALID_ARG;
+    if (!fmt_ok(prep->fmt) || prep->fmt != wq->fmt || prep->k != wq->k || !k_ok(prep->k)) return SHARQ_ERR_INVALID_ARG;
+    if (n_groups < 1 || n_groups > sq::kGroupsMax || prep->groups != n_groups || wq->groups != n_groups)
+        return SHARQ_ERR_INVALID_ARG;
+    if (wq->n_out < 1 || wq->n_out % SHARQ_N_ALIGN != 0 || rows < 0 || rows > prep->m_tok)
+        return SHARQ_ERR_INVALID_ARG;
+    if (prep->m_tok % sq::kActRowPad != 0 || prep->sf_rows != prep->m_tok || wq->sf_rows < wq->n_out ||
+        wq->sf_rows % sq::kWRowPad != 0)
+        return SHARQ_ERR_INVALID_ARG;
+    if (!prep->s_codes || !prep->r_codes || !wq->codes || wq->scales_backbone != wq->scales_residual)
+        return SHARQ_ERR_INVALID_ARG;
+    if (rows > 0 && (!out_dev || !aligned(out_dev, 16))) return SHARQ_ERR_INVALID_ARG;
+    if (prep->m_tok > (1ll << 31) - 256) return SHARQ_ERR_UNSUPPORTED;
+    sq::LaunchCtx ctx;
+    sharq_status st = make_ctx(stream, ctx);
+    if (st != SHARQ_OK) return st;
+    const int64_t gstride = (int64_t)sharq_weight_bytes(wq->n_out, wq->k, wq->fmt);
+    st = sq::launch_linear_grouped(ctx, *prep, *wq, offsets_dev, (int32_t)n_groups, rows, gstride, out_dev);
     g_last_launches = ctx.launches;
     return st;
 }
@@ -295,7 +382,7 @@ sharq_status sharq_get_last_error(void *stream) {
         g_last_site = v;
         unsigned zero = 0;
         if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return SHARQ_ERR_CUDA;
-        return SHARQ_ERR_TIMEOUT;
+        return (v & 0xF00u) == 0x200u ? SHARQ_ERR_INVALID_ARG : SHARQ_ERR_TIMEOUT;
     }
     return SHARQ_OK;
 }

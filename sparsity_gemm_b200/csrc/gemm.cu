@@ -26,6 +26,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
+#include <string.h>
 
 #include "sharq_dev.cuh"
 #include "sq_internal.h"
@@ -48,7 +49,9 @@ constexpr int kOffSFAS = kOffB + kBBytes, kOffSFAR = kOffSFAS + kSfaMax, kOffSFB
 constexpr int kStageBytes = kOffSFB + kSfbMax;                     // a multiple of 1024
 constexpr int kStages = (232448 - 2048) / kStageBytes;
 constexpr int kBarOff = kStages * kStageBytes;
-constexpr int kSmemBytes = kBarOff + 256 + 1024;                   // barriers + alignment slack
+// Grouped launches: the tile table (kGroupsMax + 1 ints) and its valid flag.
+constexpr int kTableOff = kBarOff + 256, kTableBytes = 4 * (int)(kGroupsMax + 1) + 12;
+constexpr int kSmemBytes = kTableOff + kTableBytes + 1024;        // barriers, table, alignment slack
 constexpr int kMmaPerStage = kBKBytes / 32;                        // MMAs of K = 64 per path per stage
 constexpr uint32_t kSwizzleLayout = kBKBytes == 128 ? 2u : 4u;     // descriptor layout: 128B / 64B swizzle
 constexpr uint32_t kTmemCols = 512;
@@ -61,6 +64,7 @@ constexpr int kGemmThreads = 224;
 static_assert(kStageBytes % 1024 == 0, "stage buffers must stay 1024-byte aligned");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(8 * (2 * kStages + 8) + 4 <= 256, "barrier area");
+static_assert(kTableBytes % 4 == 0, "table alignment");
 
 enum : unsigned {
     kSiteProducer = 0x101,
@@ -84,6 +88,11 @@ struct GemmParams {
     int32_t m_tok, n_out, k;
     unsigned *status;
     uint64_t wait_ns;
+    // grouped launches only
+    const int32_t *offsets;  // [groups + 1], device
+    int32_t groups;
+    int64_t rows;            // grouped rows (= offsets[groups])
+    int64_t w_gstride;       // bytes between two groups' weight payloads
 };
 
 // Instruction descriptor of the block-scaled MMA (M = 128, N = 256, E2M1 x
@@ -113,7 +122,11 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
         if (globaltimer_ns() - t0 > limit_ns) break;
 }
 
-template <int FMT>
+// GROUPED: the A rows are a grouped prep (groups start at multiples of 128
+// rows; tile table in shared memory), W is a stack of `groups` weights read
+// through a 3-D tensor map (K bytes, n_out, group), each group with its own
+// tensor scale, and output rows are remapped to grouped-row order.
+template <int FMT, bool GROUPED>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constant__ CUtensorMap tm_ar,
                  const __grid_constant__ CUtensorMap tm_b, const GemmParams p) {
@@ -131,10 +144,17 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     auto sf_full_bar = [&](int b) { return acc_full + 32u + 8u * b; };
     auto sf_empty_bar = [&](int b) { return acc_full + 48u + 8u * b; };
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOff + 8 * (2 * kStages + 8));
+    int32_t *tiles = reinterpret_cast<int32_t *>(smem + kTableOff);
+    int32_t *table_ok = tiles + (kGroupsMax + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int m_tiles = (p.m_tok + kBM - 1) / kBM, n_tiles = (p.n_out + kBN - 1) / kBN;
-    const int num_tiles = m_tiles * n_tiles, kt_count = p.k / (2 * kBKBytes);
+    if (GROUPED && warp == 2) {
+        const bool ok = build_tile_table(p.offsets, p.groups, p.rows, p.m_tok, tiles);
+        if (lane == 0) {
+            *table_ok = ok ? 1 : 0;
+            if (!ok && blockIdx.x == 0) record_status(p.status, kSiteBadOffsets);
+        }
+    }
     const int64_t atoms_per_row_blk = (int64_t)(p.k / (FMT == kFmtNV ? 16 : 32)) / 4;
     // 512-byte scale atoms (128 rows x 4 scales) per 128 rows per K tile
     constexpr int kAtomsPerTile = FMT == kFmtNV ? kBKBytes / 32 : kBKBytes / 64;
@@ -166,6 +186,11 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // m tiles: 128-row tiles of the prep (grouped: of all groups; none if the
+    // offsets are invalid)
+    const int m_tiles = GROUPED ? (*table_ok ? tiles[p.groups] : 0) : (p.m_tok + kBM - 1) / kBM;
+    const int n_tiles = (p.n_out + kBN - 1) / kBN;
+    const int num_tiles = m_tiles * n_tiles, kt_count = p.k / (2 * kBKBytes);
 
     if (warp == 0) {
         if (lane == 0) {
@@ -175,6 +200,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
                 const int nb = tile % n_tiles, mb = tile / n_tiles;
+                const int grp = GROUPED ? group_of_tile(tiles, p.groups, mb) : 0;
+                const uint8_t *sfb = p.sfb + (GROUPED ? (int64_t)grp * p.w_gstride : 0);
                 for (int kt = 0; kt < kt_count; ++kt, ++it) {
                     const int s = (int)(it % kStages);
                     const uint32_t ph = (it / kStages) & 1u;
@@ -187,14 +214,15 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                     mbar_arrive_expect_tx(fb, 2 * kABytes + kBBytes + 4 * kSfBytes);
                     tma_load_2d(st + kOffAS, &tm_as, kt * kBKBytes, mb * kBM, fb);
                     tma_load_2d(st + kOffAR, &tm_ar, kt * kBKBytes, mb * kBM, fb);
-                    tma_load_2d(st + kOffB, &tm_b, kt * kBKBytes, nb * kBN, fb);
+                    if (GROUPED) tma_load_3d(st + kOffB, &tm_b, kt * kBKBytes, nb * kBN, grp, fb);
+                    else tma_load_2d(st + kOffB, &tm_b, kt * kBKBytes, nb * kBN, fb);
                     const int64_t a_off = ((int64_t)mb * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
                     const int64_t b0 = ((int64_t)(2 * nb) * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
                     const int64_t b1 = b0 + atoms_per_row_blk * 512;
                     bulk_load(st + kOffSFAS, p.sfa_s + a_off, kSfBytes, fb);
                     bulk_load(st + kOffSFAR, p.sfa_r + a_off, kSfBytes, fb);
-                    bulk_load(st + kOffSFB, p.sfb + b0, kSfBytes, fb);
-                    bulk_load(st + kOffSFB + kSfBytes, p.sfb + b1, kSfBytes, fb);
+                    bulk_load(st + kOffSFB, sfb + b0, kSfBytes, fb);
+                    bulk_load(st + kOffSFB + kSfBytes, sfb + b1, kSfBytes, fb);
                     last[s] = (int32_t)it;
                 }
             }
@@ -293,9 +321,17 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         // registers (as packed fp16) and handed back to the MMA warp, so that
         // the next tile's MMAs overlap with this tile's global stores.
         const int q = warp & 3;  // tensor-memory lane quadrant this warp may access
-        const float alpha = __fmul_rn(*p.s_t, *p.s_tw);
+        const float s_t = *p.s_t;
+        float alpha = __fmul_rn(s_t, *p.s_tw);
         uint32_t tile_iter = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tile_iter) {
+            const int nb = tile % n_tiles, mb = tile / n_tiles;
+            int grp = 0;
+            if constexpr (GROUPED) {
+                grp = group_of_tile(tiles, p.groups, mb);
+                alpha = __fmul_rn(s_t, *reinterpret_cast<const float *>(
+                                           reinterpret_cast<const uint8_t *>(p.s_tw) + (int64_t)grp * p.w_gstride));
+            }
             if (!mbar_wait(acc_full, tile_iter & 1u, p.status, kSiteEpilogue, p.wait_ns)) break;
             tc_fence_after();
             uint32_t h[kBN / 32][16];
@@ -313,14 +349,21 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             }
             tc_fence_before();
             mbar_arrive(acc_empty);
-            const int nb = tile % n_tiles, mb = tile / n_tiles;
-            const int row = mb * kBM + q * 32 + lane;
-            if (row < p.m_tok) {
+            int64_t row, row_end;  // output row of this lane; end of the tile's valid rows
+            if constexpr (GROUPED) {
+                const int32_t first = p.offsets[grp], last = p.offsets[grp + 1];
+                row = (int64_t)first + (int64_t)(mb - tiles[grp]) * kBM + q * 32 + lane;
+                row_end = last;
+            } else {
+                row = mb * kBM + q * 32 + lane;
+                row_end = p.m_tok;
+            }
+            if (row < row_end) {
 #pragma unroll
                 for (int cc = 0; cc < kBN / 32; ++cc) {
                     const int col0 = nb * kBN + cc * 32;
                     if (col0 < p.n_out) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + (int64_t)row * p.n_out + col0);
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + row * p.n_out + col0);
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
                             dst[i] = make_uint4(h[cc][4 * i], h[cc][4 * i + 1], h[cc][4 * i + 2], h[cc][4 * i + 3]);
@@ -391,26 +434,46 @@ static bool make_code_map(CUtensorMap *tm, const void *base, uint64_t row_bytes,
     return r == CUDA_SUCCESS;
 }
 
-sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, void *out) {
-    if (P.m_tok == 0) return SHARQ_OK;
-    static bool attr_done[64][2] = {};
+// 3-D byte tensor [groups][rows][row_bytes] with `group_stride` bytes
+// between groups; box = kBKBytes x box_rows x 1, swizzled like make_code_map.
+static bool make_grouped_code_map(CUtensorMap *tm, const void *base, uint64_t row_bytes, uint64_t rows,
+                                  uint64_t groups, uint64_t group_stride, uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {row_bytes, rows, groups};
+    cuuint64_t strides[2] = {row_bytes, group_stride};
+    cuuint32_t box[3] = {(cuuint32_t)kBKBytes, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     kBKBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int FMT, bool GROUPED>
+static sharq_status launch_gemm(LaunchCtx &ctx, const CUtensorMap &tm_as, const CUtensorMap &tm_ar,
+                                const CUtensorMap &tm_b, const GemmParams &gp, int64_t max_tiles) {
+    static bool attr_done[64] = {};
     int dev = 0;
     SQ_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
-    const int f = P.fmt == kFmtNV ? 0 : 1;
-    if (!attr_done[dev][f]) {
-        if (f == 0)
-            SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<kFmtNV>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes));
-        else
-            SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<kFmtMX>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes));
-        attr_done[dev][f] = true;
+    if (!attr_done[dev]) {
+        SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<FMT, GROUPED>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes));
+        attr_done[dev] = true;
     }
-    CUtensorMap tm_as, tm_ar, tm_b;
-    if (!make_code_map(&tm_as, P.s_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
-        !make_code_map(&tm_ar, P.r_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
-        !make_code_map(&tm_b, W.codes, (uint64_t)(W.k / 2), (uint64_t)W.n_out, kBN))
-        return SHARQ_ERR_CUDA;
+    const unsigned grid = (unsigned)(max_tiles < ctx.num_sms ? max_tiles : ctx.num_sms);
+    dual_gemm_kernel<FMT, GROUPED><<<grid, kGemmThreads, kSmemBytes, ctx.stream>>>(tm_as, tm_ar, tm_b, gp);
+    ctx.launches++;
+    SQ_CUDA_TRY(cudaGetLastError());
+    return SHARQ_OK;
+}
+
+static GemmParams gemm_params(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, void *out) {
     GemmParams gp;
+    memset(&gp, 0, sizeof(gp));
     gp.sfa_s = (const uint8_t *)P.s_scales;
     gp.sfa_r = (const uint8_t *)P.r_scales;
     gp.sfb = (const uint8_t *)W.scales_backbone;  // the residual view holds the same bytes
@@ -422,15 +485,40 @@ sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &
     gp.k = (int32_t)P.k;
     gp.status = ctx.status;
     gp.wait_ns = ctx.wait_ns;
+    return gp;
+}
+
+sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, void *out) {
+    if (P.m_tok == 0) return SHARQ_OK;
+    CUtensorMap tm_as, tm_ar, tm_b;
+    if (!make_code_map(&tm_as, P.s_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
+        !make_code_map(&tm_ar, P.r_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
+        !make_code_map(&tm_b, W.codes, (uint64_t)(W.k / 2), (uint64_t)W.n_out, kBN))
+        return SHARQ_ERR_CUDA;
+    const GemmParams gp = gemm_params(ctx, P, W, out);
     const int64_t tiles = ((P.m_tok + kBM - 1) / kBM) * ((W.n_out + kBN - 1) / kBN);
-    const unsigned grid = (unsigned)(tiles < ctx.num_sms ? tiles : ctx.num_sms);
-    if (f == 0)
-        dual_gemm_kernel<kFmtNV><<<grid, kGemmThreads, kSmemBytes, ctx.stream>>>(tm_as, tm_ar, tm_b, gp);
-    else
-        dual_gemm_kernel<kFmtMX><<<grid, kGemmThreads, kSmemBytes, ctx.stream>>>(tm_as, tm_ar, tm_b, gp);
-    ctx.launches++;
-    SQ_CUDA_TRY(cudaGetLastError());
-    return SHARQ_OK;
+    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
+                           : launch_gemm<kFmtMX, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
+}
+
+sharq_status launch_linear_grouped(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, const int32_t *offsets,
+                                   int32_t groups, int64_t rows, int64_t w_gstride, void *out) {
+    CUtensorMap tm_as, tm_ar, tm_b;
+    if (!make_code_map(&tm_as, P.s_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
+        !make_code_map(&tm_ar, P.r_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
+        !make_grouped_code_map(&tm_b, W.codes, (uint64_t)(W.k / 2), (uint64_t)W.n_out, (uint64_t)groups,
+                               (uint64_t)w_gstride, kBN))
+        return SHARQ_ERR_CUDA;
+    GemmParams gp = gemm_params(ctx, P, W, out);
+    gp.offsets = offsets;
+    gp.groups = groups;
+    gp.rows = rows;
+    gp.w_gstride = w_gstride;
+    // at most P.m_tok / 128 m tiles (the device checks the offsets against it)
+    const int64_t tiles = (P.m_tok / kBM) * ((W.n_out + kBN - 1) / kBN);
+    if (tiles == 0) return SHARQ_OK;
+    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, true>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
+                           : launch_gemm<kFmtMX, true>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
 }
 
 }  // namespace sq

@@ -33,6 +33,10 @@ SQ_HD int64_t meta_row_bytes(int64_t k, int n, int m) {
     return ((k / m) * n * idx_bits(m) + 7) / 8;
 }
 
+// Rows of a grouped prep: every group starts at a multiple of 128 rows.
+constexpr int64_t kGroupsMax = 1024;
+SQ_HD int64_t grouped_rows(int64_t rows, int64_t groups) { return round_up(rows + 127 * groups, kActRowPad); }
+
 // Sections of a prep buffer.
 struct PrepLayout {
     int64_t s_codes, r_codes, s_scales, r_scales, meta, stats, words, total;

@@ -249,6 +249,59 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
 }
 
 // ---------------------------------------------------------------------------
+// Grouped (mixture-of-experts) launches. Group g owns grouped rows
+// offsets[g] .. offsets[g+1]-1 and, in a grouped prep, the 128-row tiles
+// tiles[g] .. tiles[g+1]-1, where tiles[g] counts ceil(size / 128) over the
+// groups before g.
+
+// Device-side argument codes (status word values 0x2xx).
+enum : unsigned { kSiteBadOffsets = 0x201, kSiteBadRowIndex = 0x202 };
+
+// Builds tiles[0 .. groups] in shared memory with the calling warp (all 32
+// lanes must call). Returns, in every lane, whether the offsets are valid:
+// offsets[0] == 0, nondecreasing, offsets[groups] == rows, and the padded
+// rows 128 * tiles[groups] fit in cap_rows. Counts are clamped while
+// scanning, so nothing overflows on invalid input; the table is then unused.
+__device__ __forceinline__ bool build_tile_table(const int32_t *offsets, int groups, int64_t rows, int64_t cap_rows,
+                                                 int32_t *tiles) {
+    const int lane = threadIdx.x & 31;
+    bool ok = offsets[0] == 0 && (int64_t)offsets[groups] == rows;
+    int64_t carry = 0;
+    if (lane == 0) tiles[0] = 0;
+    for (int base = 0; base < groups; base += 32) {
+        const int g = base + lane;
+        int32_t t = 0;
+        if (g < groups) {
+            const int32_t a = offsets[g], b = offsets[g + 1];
+            if (b < a) ok = false;
+            const int64_t c = b >= a ? min((int64_t)b - a, rows) : 0;
+            t = (int32_t)((c + 127) >> 7);
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t v = __shfl_up_sync(0xFFFFFFFFu, t, o);
+            if (lane >= o) t += v;
+        }
+        if (g < groups) tiles[g + 1] = (int32_t)min(carry + t, (int64_t)0x7FFFFFFF);
+        carry += __shfl_sync(0xFFFFFFFFu, t, 31);
+    }
+    if (carry * 128 > cap_rows) ok = false;
+    return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// The group whose tiles hold 128-row tile `tile` (< tiles[groups]): the
+// largest g with tiles[g] <= tile (empty groups own no tile).
+__device__ __forceinline__ int group_of_tile(const int32_t *tiles, int groups, int32_t tile) {
+    int lo = 0, hi = groups;  // tiles[lo] <= tile < tiles[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tiles[mid] <= tile) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
+// ---------------------------------------------------------------------------
 // TMA and bulk copies (no multicast anywhere in this library).
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int32_t c0, int32_t c1, uint32_t bar) {
@@ -256,6 +309,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int3
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
         "l"(tmap), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+
+// 3-D tile load: coordinates (c0 innermost, c1, c2).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int32_t c0, int32_t c1, int32_t c2,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
         : "memory");
 }
 

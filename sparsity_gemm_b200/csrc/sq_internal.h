@@ -17,8 +17,13 @@ struct LaunchCtx {
 
 sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, const void *gamma,
                             const void *beta, float eps);
-sharq_status launch_quantize_weight(LaunchCtx &ctx, const sharq_wq &W, const void *w);
+sharq_status launch_quantize_weight(LaunchCtx &ctx, const sharq_wq &W, const void *w, int64_t groups,
+                                   int64_t gstride);
 sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, void *out);
+sharq_status launch_linear_grouped(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, const int32_t *offsets,
+                                   int32_t groups, int64_t rows, int64_t w_gstride, void *out);
+sharq_status launch_gather(LaunchCtx &ctx, const sharq_prep &S, const int32_t *row_idx, const int32_t *offsets,
+                           int32_t groups, int64_t rows, const sharq_prep &D);
 sharq_status launch_wait_probe(LaunchCtx &ctx, uint64_t limit_ns);
 sharq_status launch_div_check(LaunchCtx &ctx, uint64_t count, uint64_t seed, uint64_t *mismatches, float *examples);
 

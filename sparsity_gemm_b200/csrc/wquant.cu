@@ -8,6 +8,10 @@
 // dequantized weight must be identical on both paths).
 //   1. absmax_kernel: amax|W| over the whole matrix (NVFP4 tensor scale).
 //   2. wq_encode_kernel: per 32-element chunk, block scales and E2M1 codes.
+// A stack of weights (the experts of a mixture-of-experts layer) is
+// quantized in the same two launches: blockIdx.y is the group, each group
+// with its own tensor scale, its payload `gstride` bytes after the previous
+// group's.
 #include <cuda_fp16.h>
 
 #include "sharq_dev.cuh"
@@ -20,8 +24,10 @@ constexpr int kWThreads = 256;
 // amax of |fp16| over `count` halves (count a multiple of 8): the absolute
 // value of a finite fp16 orders like its low 15 bits.
 __global__ void __launch_bounds__(kWThreads) absmax_kernel(const uint16_t *__restrict__ w, int64_t count,
-                                                          unsigned *__restrict__ amax_word) {
+                                                          unsigned *__restrict__ amax_word, int64_t gstride) {
     __shared__ unsigned red[kWThreads / 32];
+    w += (int64_t)blockIdx.y * count;
+    amax_word = reinterpret_cast<unsigned *>(reinterpret_cast<uint8_t *>(amax_word) + (int64_t)blockIdx.y * gstride);
     const uint4 *p = reinterpret_cast<const uint4 *>(w);
     const int64_t nvec = count / 8;
     unsigned m = 0;
@@ -49,8 +55,16 @@ template <int FMT>
 __global__ void __launch_bounds__(kWThreads)
 wq_encode_kernel(const uint16_t *__restrict__ w, int64_t n_out, int64_t sf_rows, int64_t k,
                  const unsigned *__restrict__ amax_word, float *__restrict__ s_tw_out, uint8_t *__restrict__ codes,
-                 uint8_t *__restrict__ sf) {
+                 uint8_t *__restrict__ sf, int64_t gstride) {
     constexpr int BLK = FMT == kFmtNV ? 16 : 32;
+    {
+        const int64_t gofs = (int64_t)blockIdx.y * gstride;
+        w += (int64_t)blockIdx.y * n_out * k;
+        amax_word = reinterpret_cast<const unsigned *>(reinterpret_cast<const uint8_t *>(amax_word) + gofs);
+        s_tw_out = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(s_tw_out) + gofs);
+        codes += gofs;
+        sf += gofs;
+    }
     constexpr int NB = 32 / BLK;
     const float amax = __uint_as_float(*amax_word);
     const float s_t = (FMT == kFmtNV && amax != 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
@@ -94,25 +108,31 @@ wq_encode_kernel(const uint16_t *__restrict__ w, int64_t n_out, int64_t sf_rows,
     }
 }
 
-sharq_status launch_quantize_weight(LaunchCtx &ctx, const sharq_wq &W, const void *w) {
+sharq_status launch_quantize_weight(LaunchCtx &ctx, const sharq_wq &W, const void *w, int64_t groups,
+                                   int64_t gstride) {
     unsigned *words = reinterpret_cast<unsigned *>(W.tensor_scale) - 1;  // [0] amax bits, [1] s_tW
-    SQ_CUDA_TRY(cudaMemsetAsync(words, 0, sizeof(unsigned), ctx.stream));
+    if (groups == 1) SQ_CUDA_TRY(cudaMemsetAsync(words, 0, sizeof(unsigned), ctx.stream));
+    else SQ_CUDA_TRY(cudaMemset2DAsync(words, (size_t)gstride, 0, sizeof(unsigned), (size_t)groups, ctx.stream));
+    // grid-stride loops: about 4 (absmax) and 8 (encode) CTAs per SM over all groups
+    const int64_t per_group_cap = (int64_t)ctx.num_sms * 4 / groups > 0 ? (int64_t)ctx.num_sms * 4 / groups : 1;
     const int64_t count = W.n_out * W.k;
     int64_t blocks = (count / 8 + kWThreads - 1) / kWThreads;
-    if (blocks > (int64_t)ctx.num_sms * 4) blocks = (int64_t)ctx.num_sms * 4;
-    absmax_kernel<<<(unsigned)blocks, kWThreads, 0, ctx.stream>>>((const uint16_t *)w, count, words);
+    if (blocks > per_group_cap) blocks = per_group_cap;
+    const dim3 ga((unsigned)blocks, (unsigned)groups);
+    absmax_kernel<<<ga, kWThreads, 0, ctx.stream>>>((const uint16_t *)w, count, words, gstride);
     ctx.launches++;
     const int64_t total = W.sf_rows * (W.k / 32);
     int64_t eb = (total + kWThreads - 1) / kWThreads;
-    if (eb > (int64_t)ctx.num_sms * 8) eb = (int64_t)ctx.num_sms * 8;
+    if (eb > 2 * per_group_cap) eb = 2 * per_group_cap;
+    const dim3 ge((unsigned)eb, (unsigned)groups);
     if (W.fmt == kFmtNV)
-        wq_encode_kernel<kFmtNV><<<(unsigned)eb, kWThreads, 0, ctx.stream>>>(
+        wq_encode_kernel<kFmtNV><<<ge, kWThreads, 0, ctx.stream>>>(
             (const uint16_t *)w, W.n_out, W.sf_rows, W.k, words, W.tensor_scale, (uint8_t *)W.codes,
-            (uint8_t *)W.scales_backbone);
+            (uint8_t *)W.scales_backbone, gstride);
     else
-        wq_encode_kernel<kFmtMX><<<(unsigned)eb, kWThreads, 0, ctx.stream>>>(
+        wq_encode_kernel<kFmtMX><<<ge, kWThreads, 0, ctx.stream>>>(
             (const uint16_t *)w, W.n_out, W.sf_rows, W.k, words, W.tensor_scale, (uint8_t *)W.codes,
-            (uint8_t *)W.scales_backbone);
+            (uint8_t *)W.scales_backbone, gstride);
     ctx.launches++;
     SQ_CUDA_TRY(cudaGetLastError());
     return SHARQ_OK;
