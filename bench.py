@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # one ncu capture of the current dual_gemm_kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum; profiles/dual_gemm_kernel_m8192_n4096_k14336.md).
 # Set to None whenever the kernel changes until it is captured again.
-GEMM_TRAFFIC_BYTES_PER_STEP_M8192 = 981.1e6
+GEMM_TRAFFIC_BYTES_PER_STEP_M8192 = None
 
 
 def parse_args():
@@ -451,6 +451,8 @@ def run_case(args, world, rank, local):
     peaks, peak_src = load_peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+    if kind == "moe":
+        return run_moe(args, nums[0] if nums else 4096)
     if kind == "prep":
         M, K = nums[:2]
         fmt, n, m = (nums[2:5] + [0, N_KEEP, M_GROUP][len(nums[2:5]):])
@@ -496,6 +498,87 @@ def run_case(args, world, rank, local):
     return {"case": args.case, "ms_median": t * 1e3, "ms_min": min(ms), "achieved": achieved, "unit": unit,
             "peak": peak, "frac": achieved / peak, "bound": bound, "steps": args.steps,
             "outlier_frac": args.outlier_frac, "peak_source": peak_src}
+
+
+def run_moe(args, tokens):
+    """The Qwen3-30B-A3B-shaped MoE FFN (hidden 2048, 128 experts of
+    intermediate 768, top-8 routing from N(0,1) gate logits) as one step:
+    prep of the token activation, expert-grouped gather, gate and up
+    grouped linears, prep of the down projection's grouped-order input,
+    its gather (identity rows), down grouped linear. L2 flushed before every
+    step; every launch timed with CUDA events on the launching stream."""
+    import sparsity_gemm_b200 as sq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    cfg = synth.QWEN3_MOE
+    hidden, inter, groups, top_k = cfg["hidden"], cfg["inter"], cfg["n_experts"], cfg["top_k"]
+    fmt, n, m = 0, N_KEEP, M_GROUP
+    peaks, peak_src = load_peaks()
+    row_idx, offsets = synth.moe_routing(0, tokens, groups, top_k)
+    rows = len(row_idx)
+    h16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.float16)).to(dev)
+    x = h16(synth.activations_student(0, tokens, hidden, outlier_frac=args.outlier_frac))
+    xd = h16(synth.activations_student(1, rows, inter, outlier_frac=args.outlier_frac))
+    ri = torch.from_numpy(row_idx).to(dev)
+    off = torch.from_numpy(offsets).to(dev)
+    qws = {}
+    for j, (name, n_out, k) in enumerate([("gate", inter, hidden), ("up", inter, hidden), ("down", hidden, inter)]):
+        w = h16(np.stack([synth.weights(2000 + 1000 * j + g, n_out, k) for g in range(groups)]))
+        qws[name] = sq.quantize_weight_grouped(w, fmt)
+        del w
+    p_tok = sq.prepare(x, None, None, EPS, n, m, fmt)
+    g_tok = sq.gather_rows(p_tok, ri, off, rows)
+    p_d = sq.prepare(xd, None, None, EPS, n, m, fmt)
+    g_d = sq.gather_rows(p_d, None, off, rows)
+    o_gate = torch.empty((rows, inter), dtype=torch.float16, device=dev)
+    o_up = torch.empty_like(o_gate)
+    o_down = torch.empty((rows, hidden), dtype=torch.float16, device=dev)
+    ops = [
+        ("prep", lambda: sq.prepare(x, None, None, EPS, n, m, fmt, out=p_tok)),
+        ("gather", lambda: sq.gather_rows(p_tok, ri, off, rows, out=g_tok)),
+        ("gate", lambda: sq.linear_grouped(g_tok, off, qws["gate"], rows, out=o_gate)),
+        ("up", lambda: sq.linear_grouped(g_tok, off, qws["up"], rows, out=o_up)),
+        ("prep_down", lambda: sq.prepare(xd, None, None, EPS, n, m, fmt, out=p_d)),
+        ("gather_down", lambda: sq.gather_rows(p_d, None, off, rows, out=g_d)),
+        ("down", lambda: sq.linear_grouped(g_d, off, qws["down"], rows, out=o_down)),
+    ]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    launches = 0
+    for i in range(args.warmup):
+        flush.zero_()
+        for _, f in ops:
+            f()
+            launches += sq.last_launch_count() if i == 0 else 0
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(ops) + 1)] for _ in range(args.steps)]
+    for e in ev:
+        flush.zero_()
+        e[0].record(stream)
+        for i, (_, f) in enumerate(ops):
+            f()
+            e[i + 1].record(stream)
+    torch.cuda.synchronize()
+    st = sq.get_last_error()
+    if st != sq.OK:
+        raise RuntimeError(sq.status_name(st))
+    per = {name: statistics.median([e[i].elapsed_time(e[i + 1]) for e in ev]) for i, (name, _) in enumerate(ops)}
+    step_ms = statistics.median([e[0].elapsed_time(e[-1]) for e in ev])
+    lin = {"gate": (inter, hidden), "up": (inter, hidden), "down": (hidden, inter)}
+    flops = {k: 2.0 * rows * no * kk * (1.0 + n / m) for k, (no, kk) in lin.items()}
+    counts = np.diff(offsets)
+    padded = int(128 * ((counts + 127) // 128).sum())
+    gemm_ms = sum(per[k] for k in lin)
+    peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    achieved = sum(flops.values()) / (gemm_ms / 1e3) / 1e12
+    return {"case": f"moe:{tokens}", "workload": "Qwen3-30B-A3B MoE FFN: hidden 2048, 128 experts x "
+            "intermediate 768, top-8 of N(0,1) gate logits; gate/up/down grouped SharQ linears, NVFP4 2:4",
+            "tokens": tokens, "rows": rows, "padded_rows": padded, "ms_per_step": step_ms,
+            "tokens_per_s": tokens / (step_ms / 1e3), "ms": per,
+            "gemm_roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                              "frac": achieved / peak, "flops_algorithmic": sum(flops.values()),
+                              "peak_source": peak_src + " (bf16 burst x 4)"},
+            "gpu_launches_per_step": launches, "steps": args.steps,
+            "warmup": args.warmup, "l2": "flushed (256 MB write) before every step"}
 
 
 def main():

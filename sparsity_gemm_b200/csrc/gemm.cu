@@ -18,9 +18,9 @@
 // memory allows, 6 warps:
 //   warp 0      TMA producer (A_S, A_R, W tiles; scale atoms by bulk copy)
 //   warp 1      tensor-memory allocation and the single-thread MMA issuer
-//   warps 2..5  epilogue: tensor memory -> registers -> fp16 -> global
-//   warp 6      scale copies: the stage's scale atoms -> one of two scale
-//               buffers in tensor memory (tcgen05.cp), ahead of the MMAs
+//   warps 2..5  scale writes (shared memory -> registers -> one of four
+//               scale buffers in tensor memory, ahead of the MMAs) and the
+//               epilogue (tensor memory -> registers -> fp16 -> global)
 // Every mbarrier wait is bounded (global-timer limit); a wait that runs out
 // records a site code in the status word and the CTA winds down cleanly.
 #include <cuda.h>
@@ -49,21 +49,25 @@ constexpr int kOffSFAS = kOffB + kBBytes, kOffSFAR = kOffSFAS + kSfaMax, kOffSFB
 constexpr int kStageBytes = kOffSFB + kSfbMax;                     // a multiple of 1024
 constexpr int kStages = (232448 - 2048) / kStageBytes;
 constexpr int kBarOff = kStages * kStageBytes;
+constexpr int kSfBufs = 4;                                          // scale buffers in tensor memory
+constexpr int kLookahead = kSfBufs < kStages ? kSfBufs : kStages;  // scale writes ahead of a tile's drain
+constexpr int kBarBytes = 8 * (2 * kStages + 3 + 2 * kSfBufs);     // mbarriers; the TMEM slot follows
 // Grouped launches: the tile table (kGroupsMax + 1 ints) and its valid flag.
 constexpr int kTableOff = kBarOff + 256, kTableBytes = 4 * (int)(kGroupsMax + 1) + 12;
 constexpr int kSmemBytes = kTableOff + kTableBytes + 1024;        // barriers, table, alignment slack
 constexpr int kMmaPerStage = kBKBytes / 32;                        // MMAs of K = 64 per path per stage
 constexpr uint32_t kSwizzleLayout = kBKBytes == 128 ? 2u : 4u;     // descriptor layout: 128B / 64B swizzle
 constexpr uint32_t kTmemCols = 512;
-// Scale buffers after the accumulator (columns 0..255): two of 64 columns,
-// filled alternately by the scale-copy warp; within a buffer, the backbone
-// A scales at +0, the residual A scales at +16, the W scales at +32.
+// Scale buffers after the accumulator (columns 0..255): four of 64 columns,
+// filled in turn by the scale writers; within a buffer, the backbone A
+// scales at +0, the residual A scales at +16, the W scales at +32.
 constexpr uint32_t kColSf0 = 256, kSfBufCols = 64;
 constexpr uint32_t kSfaS = 0, kSfaR = 16, kSfb = 32;
-constexpr int kGemmThreads = 224;
+constexpr int kGemmThreads = 192;
 static_assert(kStageBytes % 1024 == 0, "stage buffers must stay 1024-byte aligned");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(8 * (2 * kStages + 8) + 4 <= 256, "barrier area");
+static_assert(kBarBytes + 4 <= 256, "barrier area");
+static_assert(kColSf0 + kSfBufs * kSfBufCols <= kTmemCols, "tensor memory columns");
 static_assert(kTableBytes % 4 == 0, "table alignment");
 
 enum : unsigned {
@@ -111,9 +115,6 @@ __device__ __forceinline__ uint64_t desc_operand(uint32_t addr) {
     return smem_desc(addr, 16, 8 * kBKBytes, kSwizzleLayout);
 }
 
-// One 512-byte scale atom: 32 rows of 16 bytes, no swizzle, 8-row groups
-// 128 bytes apart.
-__device__ __forceinline__ uint64_t desc_scales(uint32_t addr) { return smem_desc(addr, 0, 128, 0); }
 
 // Wait bounded only by time (used to drain in-flight copies on exit).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
@@ -134,16 +135,16 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     const uint32_t raw_s = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t bar0 = sbase + kBarOff;  // full[s], empty[s], acc_full, acc_empty, drain x2, sf_full[2], sf_empty[2]
+    // barriers: full[s], empty[s], acc_full, acc_empty, drain, sf_full[b], sf_empty[b]
+    const uint32_t bar0 = sbase + kBarOff;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
     const uint32_t acc_full = bar0 + 8u * (2 * kStages);
     const uint32_t acc_empty = acc_full + 8u;
     const uint32_t drain_bar = acc_full + 16u;
-    const uint32_t drain_sf_bar = acc_full + 24u;
-    auto sf_full_bar = [&](int b) { return acc_full + 32u + 8u * b; };
-    auto sf_empty_bar = [&](int b) { return acc_full + 48u + 8u * b; };
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOff + 8 * (2 * kStages + 8));
+    auto sf_full_bar = [&](int b) { return acc_full + 24u + 8u * b; };
+    auto sf_empty_bar = [&](int b) { return acc_full + 24u + 8u * (kSfBufs + b); };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOff + kBarBytes);
     int32_t *tiles = reinterpret_cast<int32_t *>(smem + kTableOff);
     int32_t *table_ok = tiles + (kGroupsMax + 1);
 
@@ -155,7 +156,6 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             if (!ok && blockIdx.x == 0) record_status(p.status, kSiteBadOffsets);
         }
     }
-    const int64_t atoms_per_row_blk = (int64_t)(p.k / (FMT == kFmtNV ? 16 : 32)) / 4;
     // 512-byte scale atoms (128 rows x 4 scales) per 128 rows per K tile
     constexpr int kAtomsPerTile = FMT == kFmtNV ? kBKBytes / 32 : kBKBytes / 64;
     constexpr uint32_t kSfBytes = 512u * kAtomsPerTile;
@@ -168,9 +168,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 128);
         mbar_init(drain_bar, 1);
-        mbar_init(drain_sf_bar, 1);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(sf_full_bar(b), 1);
+        for (int b = 0; b < kSfBufs; ++b) {
+            mbar_init(sf_full_bar(b), 128);
             mbar_init(sf_empty_bar(b), 1);
         }
         mbar_fence_init();
@@ -191,6 +190,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     const int m_tiles = GROUPED ? (*table_ok ? tiles[p.groups] : 0) : (p.m_tok + kBM - 1) / kBM;
     const int n_tiles = (p.n_out + kBN - 1) / kBN;
     const int num_tiles = m_tiles * n_tiles, kt_count = p.k / (2 * kBKBytes);
+    const int64_t atoms_per_row_blk = (int64_t)(p.k / (FMT == kFmtNV ? 16 : 32)) / 4;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -245,8 +245,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                         ok = false;
                         break;
                     }
-                    const int sb = (int)(it & 1u);  // scale buffer of this stage
-                    if (!mbar_wait(sf_full_bar(sb), (it >> 1) & 1u, p.status, kSiteMmaScales, p.wait_ns)) {
+                    const int sb = (int)(it % kSfBufs);  // scale buffer of this stage
+                    if (!mbar_wait(sf_full_bar(sb), (it / kSfBufs) & 1u, p.status, kSiteMmaScales, p.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -273,58 +273,86 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                                         (sf + kSfb + b_col) | (sf_id << 30), 1u);
                         }
                     }
-                    tc_commit(empty_bar(s));       // frees the stage once these MMAs complete
-                    tc_commit(sf_empty_bar(sb));   // and the scale buffer
+                    tc_commit(empty_bar(s));      // frees the stage once these MMAs complete
+                    tc_commit(sf_empty_bar(sb));  // and the scale buffer
                 }
                 if (!ok) break;
                 tc_commit(acc_full);
             }
-            tc_commit(drain_bar);  // every MMA and copy of this thread done before exit
+            tc_commit(drain_bar);  // every MMA of this thread done before exit
             drain_wait(drain_bar, 0, kDrainNs);
         }
         __syncwarp();
-    } else if (warp == 6) {
-        // Scale copies, one stage ahead of the MMAs where the pipeline allows:
-        // the stage's atoms (128 rows x 4 scales, 512 bytes) fill 4 columns
-        // each; the W tile's 256 rows take two atoms per K step.
-        if (lane == 0) {
-            uint32_t it = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-                for (int kt = 0; kt < kt_count; ++kt, ++it) {
-                    const int s = (int)(it % kStages);
-                    const int sb = (int)(it & 1u);
-                    if (!mbar_wait(full_bar(s), (it / kStages) & 1u, p.status, kSiteScaleFull, p.wait_ns) ||
-                        !mbar_wait(sf_empty_bar(sb), ((it >> 1) & 1u) ^ 1u, p.status, kSiteScaleEmpty, p.wait_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t st = sbase + (uint32_t)(s * kStageBytes);
-                    const uint32_t sf = tmem + kColSf0 + kSfBufCols * (uint32_t)sb;
-#pragma unroll
-                    for (int a = 0; a < kAtomsPerTile; ++a) {
-                        tc_copy_scales(sf + kSfaS + 4 * a, desc_scales(st + kOffSFAS + 512 * a));
-                        tc_copy_scales(sf + kSfaR + 4 * a, desc_scales(st + kOffSFAR + 512 * a));
-                        tc_copy_scales(sf + kSfb + 8 * a, desc_scales(st + kOffSFB + 512 * a));
-                        tc_copy_scales(sf + kSfb + 8 * a + 4, desc_scales(st + kOffSFB + kSfBytes + 512 * a));
-                    }
-                    tc_commit(sf_full_bar(sb));  // the MMAs may read this buffer once the copies land
-                }
-            }
-            tc_commit(drain_sf_bar);
-            drain_wait(drain_sf_bar, 0, kDrainNs);
-        }
-        __syncwarp();
     } else {
-        // Epilogue. The accumulator is first drained from tensor memory into
-        // registers (as packed fp16) and handed back to the MMA warp, so that
-        // the next tile's MMAs overlap with this tile's global stores.
-        const int q = warp & 3;  // tensor-memory lane quadrant this warp may access
+        // Warps 2..5, one per tensor-memory lane quadrant q. Two duties:
+        //  - scale writes: each stage's scale atoms go from shared memory into
+        //    one of kSfBufs scale buffers in tensor memory through registers
+        //    (tcgen05.st, which does not occupy the MMA pipe as tcgen05.cp
+        //    does). Every lane of quadrant q receives row (lane) of each
+        //    atom, the same columns a 32x128b.warpx4 copy fills. Writes run
+        //    up to kLookahead stages into the next tile (only stages already
+        //    loaded, before this tile's drain); those stages depend only on
+        //    MMAs of this tile, so the lookahead cannot deadlock.
+        //  - epilogue: the accumulator is drained from tensor memory into
+        //    registers (as packed fp16) and handed back to the MMA warp, so
+        //    that the next tile's MMAs overlap with this tile's global stores.
+        const int q = warp & 3;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const float s_t = *p.s_t;
         float alpha = __fmul_rn(s_t, *p.s_tw);
+        const int my_tiles = (int)blockIdx.x < num_tiles ? (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+        const uint32_t total_stages = (uint32_t)my_tiles * (uint32_t)kt_count;
+        uint32_t it_sc = 0;  // next stage whose scales this warp writes
+        // Scale atoms of stage it_sc -> scale buffer it_sc % kSfBufs.
+        auto write_stage = [&]() {
+            const int s = (int)(it_sc % kStages);
+            const int b = (int)(it_sc % kSfBufs);
+            tc_fence_after();
+            const uint32_t st = sbase + (uint32_t)(s * kStageBytes) + (uint32_t)lane * 16u;
+            const uint32_t sf = tmem + lane_base + kColSf0 + kSfBufCols * (uint32_t)b;
+#pragma unroll
+            for (int a = 0; a < kAtomsPerTile; ++a) {
+                tmem_st4(sf + kSfaS + 4 * a, lds128(st + kOffSFAS + 512 * a));
+                tmem_st4(sf + kSfaR + 4 * a, lds128(st + kOffSFAR + 512 * a));
+                tmem_st4(sf + kSfb + 8 * a, lds128(st + kOffSFB + 512 * a));
+                tmem_st4(sf + kSfb + 8 * a + 4, lds128(st + kOffSFB + kSfBytes + 512 * a));
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(sf_full_bar(b));
+        };
+        // Stages up to `limit`, waiting for each (bounded); false on a timeout.
+        auto write_blocking = [&](uint32_t limit) -> bool {
+            for (; it_sc < limit; ++it_sc) {
+                const int s = (int)(it_sc % kStages);
+                const int b = (int)(it_sc % kSfBufs);
+                const bool w1 = mbar_wait(full_bar(s), (it_sc / kStages) & 1u, p.status, kSiteScaleFull, p.wait_ns);
+                const bool w2 = w1 && mbar_wait(sf_empty_bar(b), ((it_sc / kSfBufs) & 1u) ^ 1u, p.status,
+                                                kSiteScaleEmpty, p.wait_ns);
+                if (!__all_sync(0xFFFFFFFFu, w2)) return false;  // warp-uniform: tcgen05.st is .aligned
+                write_stage();
+            }
+            return true;
+        };
+        // Stages up to `limit` whose data and buffer are ready now; stops at
+        // the first that is not.
+        auto write_ready = [&](uint32_t limit) {
+            for (; it_sc < limit; ++it_sc) {
+                const bool r = mbar_try_wait(full_bar((int)(it_sc % kStages)), (it_sc / kStages) & 1u) &&
+                               mbar_try_wait(sf_empty_bar((int)(it_sc % kSfBufs)), ((it_sc / kSfBufs) & 1u) ^ 1u);
+                if (!__all_sync(0xFFFFFFFFu, r)) return;
+                write_stage();
+            }
+        };
         uint32_t tile_iter = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tile_iter) {
+            // This tile's stages (its MMAs need them), then those of the next
+            // tile that are already in shared memory: the drain below must
+            // not wait for loads that are still in flight.
+            const uint32_t tile_end = (tile_iter + 1) * (uint32_t)kt_count;
+            const uint32_t ahead = tile_end + kLookahead < total_stages ? tile_end + kLookahead : total_stages;
+            if (!write_blocking(tile_end)) break;
+            write_ready(ahead);
             const int nb = tile % n_tiles, mb = tile / n_tiles;
             int grp = 0;
             if constexpr (GROUPED) {
@@ -332,23 +360,34 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                 alpha = __fmul_rn(s_t, *reinterpret_cast<const float *>(
                                            reinterpret_cast<const uint8_t *>(p.s_tw) + (int64_t)grp * p.w_gstride));
             }
-            if (!mbar_wait(acc_full, tile_iter & 1u, p.status, kSiteEpilogue, p.wait_ns)) break;
+            const bool got = mbar_wait(acc_full, tile_iter & 1u, p.status, kSiteEpilogue, p.wait_ns);
+            if (!__all_sync(0xFFFFFFFFu, got)) break;  // warp-uniform: tcgen05.ld is .aligned
             tc_fence_after();
+            // Two 32-column loads in flight per wait; out = RN16(RN32(acc * alpha))
+            // (packed multiplies round each product to fp32 before the
+            // conversion).
             uint32_t h[kBN / 32][16];
+            const uint64_t alpha2 = pk2(alpha, alpha);
 #pragma unroll
-            for (int cc = 0; cc < kBN / 32; ++cc) {
-                uint32_t r[32];
-                tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cc * 32), r);
+            for (int cc = 0; cc < kBN / 32; cc += 2) {
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tmem + lane_base + (uint32_t)(cc * 32), r0);
+                tmem_ld32(tmem + lane_base + (uint32_t)(cc * 32 + 32), r1);
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    __half2 v = __floats2half2_rn(__fmul_rn(__uint_as_float(r[2 * i]), alpha),
-                                                  __fmul_rn(__uint_as_float(r[2 * i + 1]), alpha));
-                    h[cc][i] = *reinterpret_cast<uint32_t *>(&v);
+                    const float2 f0 = up2(mul2(pk2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1])), alpha2));
+                    const float2 f1 = up2(mul2(pk2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1])), alpha2));
+                    __half2 v0 = __floats2half2_rn(f0.x, f0.y), v1 = __floats2half2_rn(f1.x, f1.y);
+                    h[cc][i] = *reinterpret_cast<uint32_t *>(&v0);
+                    h[cc + 1][i] = *reinterpret_cast<uint32_t *>(&v1);
                 }
             }
             tc_fence_before();
             mbar_arrive(acc_empty);
+            // The next tile's MMAs start now: the scales of its first stages
+            // before this tile's stores.
+            if (!write_blocking(ahead)) break;
             int64_t row, row_end;  // output row of this lane; end of the tile's valid rows
             if constexpr (GROUPED) {
                 const int32_t first = p.offsets[grp], last = p.offsets[grp + 1];
