@@ -15,12 +15,12 @@
 //
 // Structure: persistent CTAs (one per SM), tile 128 x 256 (M x N) with a
 // K step of 2 * SQ_GEMM_BKB FP4 values, a TMA pipeline as deep as shared
-// memory allows, 6 warps:
+// memory allows, 10 warps:
 //   warp 0      TMA producer (A_S, A_R, W tiles; scale atoms by bulk copy)
 //   warp 1      tensor-memory allocation and the single-thread MMA issuer
-//   warps 2..5  scale writes (shared memory -> registers -> one of four
-//               scale buffers in tensor memory, ahead of the MMAs) and the
-//               epilogue (tensor memory -> registers -> fp16 -> global)
+//   warps 2..5  epilogue: tensor memory -> registers -> fp16 -> global
+//   warps 6..9  scale writes: shared memory -> registers -> one of four
+//               scale buffers in tensor memory, ahead of the MMAs
 // Every mbarrier wait is bounded (global-timer limit); a wait that runs out
 // records a site code in the status word and the CTA winds down cleanly.
 #include <cuda.h>
@@ -49,24 +49,27 @@ constexpr int kOffSFAS = kOffB + kBBytes, kOffSFAR = kOffSFAS + kSfaMax, kOffSFB
 constexpr int kStageBytes = kOffSFB + kSfbMax;                     // a multiple of 1024
 constexpr int kStages = (232448 - 2048) / kStageBytes;
 constexpr int kBarOff = kStages * kStageBytes;
-constexpr int kSfBufs = 4;                                          // scale buffers in tensor memory
-constexpr int kLookahead = kSfBufs < kStages ? kSfBufs : kStages;  // scale writes ahead of a tile's drain
-constexpr int kBarBytes = 8 * (2 * kStages + 3 + 2 * kSfBufs);     // mbarriers; the TMEM slot follows
+// Scale buffers in tensor memory after the accumulator (columns 0..255):
+// per buffer, the backbone A scales, the residual A scales and the W scales
+// of one stage (NVFP4: kBKBytes / 32 atoms per 128 rows; MXFP4 uses half).
+constexpr uint32_t kNvAtoms = kBKBytes / 32;
+constexpr uint32_t kColSf0 = 256, kSfBufCols = 16 * kNvAtoms;
+constexpr uint32_t kSfaS = 0, kSfaR = 4 * kNvAtoms, kSfb = 8 * kNvAtoms;
+constexpr int kSfBufs = (int)(256 / kSfBufCols);
+// mbarriers: full[s], empty[s], sf_loaded[s], acc_full, acc_empty, drain,
+// sf_full[b], sf_empty[b]; the tensor-memory slot follows.
+constexpr int kBarBytes = 8 * (3 * kStages + 3 + 2 * kSfBufs);
+constexpr int kBarArea = (kBarBytes + 4 + 127) / 128 * 128;
 // Grouped launches: the tile table (kGroupsMax + 1 ints) and its valid flag.
-constexpr int kTableOff = kBarOff + 256, kTableBytes = 4 * (int)(kGroupsMax + 1) + 12;
+constexpr int kTableOff = kBarOff + kBarArea, kTableBytes = 4 * (int)(kGroupsMax + 1) + 12;
 constexpr int kSmemBytes = kTableOff + kTableBytes + 1024;        // barriers, table, alignment slack
 constexpr int kMmaPerStage = kBKBytes / 32;                        // MMAs of K = 64 per path per stage
 constexpr uint32_t kSwizzleLayout = kBKBytes == 128 ? 2u : 4u;     // descriptor layout: 128B / 64B swizzle
 constexpr uint32_t kTmemCols = 512;
-// Scale buffers after the accumulator (columns 0..255): four of 64 columns,
-// filled in turn by the scale writers; within a buffer, the backbone A
-// scales at +0, the residual A scales at +16, the W scales at +32.
-constexpr uint32_t kColSf0 = 256, kSfBufCols = 64;
-constexpr uint32_t kSfaS = 0, kSfaR = 16, kSfb = 32;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;
 static_assert(kStageBytes % 1024 == 0, "stage buffers must stay 1024-byte aligned");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kBarBytes + 4 <= 256, "barrier area");
+static_assert(kBarBytes + 4 <= kBarArea, "barrier area");
 static_assert(kColSf0 + kSfBufs * kSfBufCols <= kTmemCols, "tensor memory columns");
 static_assert(kTableBytes % 4 == 0, "table alignment");
 
@@ -135,11 +138,13 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     const uint32_t raw_s = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
     const uint32_t sbase = smem_u32(smem);
-    // barriers: full[s], empty[s], acc_full, acc_empty, drain, sf_full[b], sf_empty[b]
+    // barriers: full[s] (operands), empty[s], sf_loaded[s] (scale atoms),
+    // acc_full, acc_empty, drain, sf_full[b], sf_empty[b]
     const uint32_t bar0 = sbase + kBarOff;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-    const uint32_t acc_full = bar0 + 8u * (2 * kStages);
+    auto sf_loaded_bar = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
+    const uint32_t acc_full = bar0 + 8u * (3 * kStages);
     const uint32_t acc_empty = acc_full + 8u;
     const uint32_t drain_bar = acc_full + 16u;
     auto sf_full_bar = [&](int b) { return acc_full + 24u + 8u * b; };
@@ -164,6 +169,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         for (int s = 0; s < kStages; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
+            mbar_init(sf_loaded_bar(s), 1);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 128);
@@ -209,26 +215,33 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                         ok = false;
                         break;
                     }
-                    const uint32_t fb = full_bar(s);
+                    const uint32_t fb = full_bar(s), lb = sf_loaded_bar(s);
                     const uint32_t st = sbase + (uint32_t)(s * kStageBytes);
-                    mbar_arrive_expect_tx(fb, 2 * kABytes + kBBytes + 4 * kSfBytes);
+                    // Scale atoms first, on their own barrier: the scale
+                    // writers move them to tensor memory while the operand
+                    // tiles are still in flight.
+                    const int64_t a_off = ((int64_t)mb * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
+                    const int64_t b0 = ((int64_t)(2 * nb) * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
+                    const int64_t b1 = b0 + atoms_per_row_blk * 512;
+                    mbar_arrive_expect_tx(lb, 4 * kSfBytes);
+                    bulk_load(st + kOffSFAS, p.sfa_s + a_off, kSfBytes, lb);
+                    bulk_load(st + kOffSFAR, p.sfa_r + a_off, kSfBytes, lb);
+                    bulk_load(st + kOffSFB, sfb + b0, kSfBytes, lb);
+                    bulk_load(st + kOffSFB + kSfBytes, sfb + b1, kSfBytes, lb);
+                    mbar_arrive_expect_tx(fb, 2 * kABytes + kBBytes);
                     tma_load_2d(st + kOffAS, &tm_as, kt * kBKBytes, mb * kBM, fb);
                     tma_load_2d(st + kOffAR, &tm_ar, kt * kBKBytes, mb * kBM, fb);
                     if (GROUPED) tma_load_3d(st + kOffB, &tm_b, kt * kBKBytes, nb * kBN, grp, fb);
                     else tma_load_2d(st + kOffB, &tm_b, kt * kBKBytes, nb * kBN, fb);
-                    const int64_t a_off = ((int64_t)mb * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
-                    const int64_t b0 = ((int64_t)(2 * nb) * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
-                    const int64_t b1 = b0 + atoms_per_row_blk * 512;
-                    bulk_load(st + kOffSFAS, p.sfa_s + a_off, kSfBytes, fb);
-                    bulk_load(st + kOffSFAR, p.sfa_r + a_off, kSfBytes, fb);
-                    bulk_load(st + kOffSFB, sfb + b0, kSfBytes, fb);
-                    bulk_load(st + kOffSFB + kSfBytes, sfb + b1, kSfBytes, fb);
                     last[s] = (int32_t)it;
                 }
             }
             // Never leave the CTA with copies in flight.
             for (int s = 0; s < kStages; ++s)
-                if (last[s] >= 0) drain_wait(full_bar(s), ((uint32_t)last[s] / kStages) & 1u, kDrainNs);
+                if (last[s] >= 0) {
+                    drain_wait(full_bar(s), ((uint32_t)last[s] / kStages) & 1u, kDrainNs);
+                    drain_wait(sf_loaded_bar(s), ((uint32_t)last[s] / kStages) & 1u, kDrainNs);
+                }
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -283,30 +296,28 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             drain_wait(drain_bar, 0, kDrainNs);
         }
         __syncwarp();
-    } else {
-        // Warps 2..5, one per tensor-memory lane quadrant q. Two duties:
-        //  - scale writes: each stage's scale atoms go from shared memory into
-        //    one of kSfBufs scale buffers in tensor memory through registers
-        //    (tcgen05.st, which does not occupy the MMA pipe as tcgen05.cp
-        //    does). Every lane of quadrant q receives row (lane) of each
-        //    atom, the same columns a 32x128b.warpx4 copy fills. Writes run
-        //    up to kLookahead stages into the next tile (only stages already
-        //    loaded, before this tile's drain); those stages depend only on
-        //    MMAs of this tile, so the lookahead cannot deadlock.
-        //  - epilogue: the accumulator is drained from tensor memory into
-        //    registers (as packed fp16) and handed back to the MMA warp, so
-        //    that the next tile's MMAs overlap with this tile's global stores.
+    } else if (warp >= 6) {
+        // Warps 6..9, one per tensor-memory lane quadrant q: scale writes.
+        // Each stage's scale atoms go from shared memory into one of
+        // kSfBufs scale buffers in tensor memory through registers
+        // (tcgen05.st, which does not occupy the MMA pipe as tcgen05.cp
+        // does). Every lane of quadrant q receives row (lane) of each atom:
+        // the columns a 32x128b.warpx4 copy fills, with the same bytes.
+        // Stage i waits for its scale atoms and for the MMAs of stage
+        // i - kSfBufs to release its buffer, so these warps run up to
+        // kSfBufs stages ahead of the MMAs, across tile boundaries; they
+        // depend on nothing the epilogue does.
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const float s_t = *p.s_t;
-        float alpha = __fmul_rn(s_t, *p.s_tw);
         const int my_tiles = (int)blockIdx.x < num_tiles ? (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
         const uint32_t total_stages = (uint32_t)my_tiles * (uint32_t)kt_count;
-        uint32_t it_sc = 0;  // next stage whose scales this warp writes
-        // Scale atoms of stage it_sc -> scale buffer it_sc % kSfBufs.
-        auto write_stage = [&]() {
-            const int s = (int)(it_sc % kStages);
-            const int b = (int)(it_sc % kSfBufs);
+        for (uint32_t it = 0; it < total_stages; ++it) {
+            const int s = (int)(it % kStages);
+            const int b = (int)(it % kSfBufs);
+            const bool w1 = mbar_wait(sf_loaded_bar(s), (it / kStages) & 1u, p.status, kSiteScaleFull, p.wait_ns);
+            const bool w2 = w1 && mbar_wait(sf_empty_bar(b), ((it / kSfBufs) & 1u) ^ 1u, p.status, kSiteScaleEmpty,
+                                            p.wait_ns);
+            if (!__all_sync(0xFFFFFFFFu, w2)) break;  // warp-uniform: tcgen05.st is .aligned
             tc_fence_after();
             const uint32_t st = sbase + (uint32_t)(s * kStageBytes) + (uint32_t)lane * 16u;
             const uint32_t sf = tmem + lane_base + kColSf0 + kSfBufCols * (uint32_t)b;
@@ -320,39 +331,19 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(sf_full_bar(b));
-        };
-        // Stages up to `limit`, waiting for each (bounded); false on a timeout.
-        auto write_blocking = [&](uint32_t limit) -> bool {
-            for (; it_sc < limit; ++it_sc) {
-                const int s = (int)(it_sc % kStages);
-                const int b = (int)(it_sc % kSfBufs);
-                const bool w1 = mbar_wait(full_bar(s), (it_sc / kStages) & 1u, p.status, kSiteScaleFull, p.wait_ns);
-                const bool w2 = w1 && mbar_wait(sf_empty_bar(b), ((it_sc / kSfBufs) & 1u) ^ 1u, p.status,
-                                                kSiteScaleEmpty, p.wait_ns);
-                if (!__all_sync(0xFFFFFFFFu, w2)) return false;  // warp-uniform: tcgen05.st is .aligned
-                write_stage();
-            }
-            return true;
-        };
-        // Stages up to `limit` whose data and buffer are ready now; stops at
-        // the first that is not.
-        auto write_ready = [&](uint32_t limit) {
-            for (; it_sc < limit; ++it_sc) {
-                const bool r = mbar_try_wait(full_bar((int)(it_sc % kStages)), (it_sc / kStages) & 1u) &&
-                               mbar_try_wait(sf_empty_bar((int)(it_sc % kSfBufs)), ((it_sc / kSfBufs) & 1u) ^ 1u);
-                if (!__all_sync(0xFFFFFFFFu, r)) return;
-                write_stage();
-            }
-        };
+        }
+    } else {
+        // Warps 2..5, one per tensor-memory lane quadrant q: epilogue. The
+        // accumulator is drained from tensor memory into registers (as
+        // packed fp16) and handed back to the MMA warp, so that the next
+        // tile's MMAs overlap with this tile's global stores.
+        const int q = warp & 3;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        const float s_t = *p.s_t;
+        float alpha = __fmul_rn(s_t, *p.s_tw);
+        const unsigned store_pause_ns = (unsigned)min(60 * kt_count, 1000);
         uint32_t tile_iter = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tile_iter) {
-            // This tile's stages (its MMAs need them), then those of the next
-            // tile that are already in shared memory: the drain below must
-            // not wait for loads that are still in flight.
-            const uint32_t tile_end = (tile_iter + 1) * (uint32_t)kt_count;
-            const uint32_t ahead = tile_end + kLookahead < total_stages ? tile_end + kLookahead : total_stages;
-            if (!write_blocking(tile_end)) break;
-            write_ready(ahead);
             const int nb = tile % n_tiles, mb = tile / n_tiles;
             int grp = 0;
             if constexpr (GROUPED) {
@@ -363,31 +354,24 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             const bool got = mbar_wait(acc_full, tile_iter & 1u, p.status, kSiteEpilogue, p.wait_ns);
             if (!__all_sync(0xFFFFFFFFu, got)) break;  // warp-uniform: tcgen05.ld is .aligned
             tc_fence_after();
-            // Two 32-column loads in flight per wait; out = RN16(RN32(acc * alpha))
-            // (packed multiplies round each product to fp32 before the
-            // conversion).
+            // out = RN16(RN32(acc * alpha)) (packed multiplies round each
+            // product to fp32 before the conversion).
             uint32_t h[kBN / 32][16];
             const uint64_t alpha2 = pk2(alpha, alpha);
 #pragma unroll
-            for (int cc = 0; cc < kBN / 32; cc += 2) {
-                uint32_t r0[32], r1[32];
-                tmem_ld32(tmem + lane_base + (uint32_t)(cc * 32), r0);
-                tmem_ld32(tmem + lane_base + (uint32_t)(cc * 32 + 32), r1);
+            for (int cc = 0; cc < kBN / 32; ++cc) {
+                uint32_t r[32];
+                tmem_ld32(tmem + lane_base + (uint32_t)(cc * 32), r);
                 tmem_ld_wait();
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float2 f0 = up2(mul2(pk2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1])), alpha2));
-                    const float2 f1 = up2(mul2(pk2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1])), alpha2));
-                    __half2 v0 = __floats2half2_rn(f0.x, f0.y), v1 = __floats2half2_rn(f1.x, f1.y);
-                    h[cc][i] = *reinterpret_cast<uint32_t *>(&v0);
-                    h[cc + 1][i] = *reinterpret_cast<uint32_t *>(&v1);
+                    const float2 f = up2(mul2(pk2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), alpha2));
+                    __half2 v = __floats2half2_rn(f.x, f.y);
+                    h[cc][i] = *reinterpret_cast<uint32_t *>(&v);
                 }
             }
             tc_fence_before();
             mbar_arrive(acc_empty);
-            // The next tile's MMAs start now: the scales of its first stages
-            // before this tile's stores.
-            if (!write_blocking(ahead)) break;
             int64_t row, row_end;  // output row of this lane; end of the tile's valid rows
             if constexpr (GROUPED) {
                 const int32_t first = p.offsets[grp], last = p.offsets[grp + 1];
@@ -397,17 +381,23 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                 row = mb * kBM + q * 32 + lane;
                 row_end = p.m_tok;
             }
-            if (row < row_end) {
+            const unsigned pause_ns = tile + (int)gridDim.x < num_tiles ? store_pause_ns : 0u;
+            // The stores are spread over the next tile's main loop: every SM
+            // reaches its tile boundary at about the same time, and a burst
+            // of all their stores delays the operand loads the next tile
+            // starts with. The pause per 32-column chunk scales with the
+            // main loop's length (about 60 ns per K step, at most 1 us); the
+            // CTA's last tile stores at once.
 #pragma unroll
-                for (int cc = 0; cc < kBN / 32; ++cc) {
-                    const int col0 = nb * kBN + cc * 32;
-                    if (col0 < p.n_out) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(p.out + row * p.n_out + col0);
+            for (int cc = 0; cc < kBN / 32; ++cc) {
+                const int col0 = nb * kBN + cc * 32;
+                if (row < row_end && col0 < p.n_out) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + row * p.n_out + col0);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(h[cc][4 * i], h[cc][4 * i + 1], h[cc][4 * i + 2], h[cc][4 * i + 3]);
-                    }
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(h[cc][4 * i], h[cc][4 * i + 1], h[cc][4 * i + 2], h[cc][4 * i + 3]);
                 }
+                if (cc + 1 < kBN / 32 && pause_ns) __nanosleep(pause_ns);
             }
         }
     }
