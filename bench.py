@@ -43,9 +43,9 @@ PREP_BYTES_PER_ELEM = 3.25  # x 2 + S codes 0.5 + mask metadata 0.125 + S scales
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of the 7 GEMM launches of one M = 8192 step, from
 # one ncu capture of the current dual_gemm_kernel (dram__bytes_read.sum +
-# dram__bytes_write.sum; profiles/dual_gemm_kernel_m8192_n4096_k14336.md).
-# Set to None whenever the kernel changes until it is captured again.
-GEMM_TRAFFIC_BYTES_PER_STEP_M8192 = None
+# dram__bytes_write.sum of the layer-set launch list). Set to None whenever
+# the kernel changes until it is captured again.
+GEMM_TRAFFIC_BYTES_PER_STEP_M8192 = 997.8e6
 
 
 def parse_args():
@@ -57,6 +57,7 @@ def parse_args():
     ap.add_argument("--tokens", type=int, default=8192, help="M: tokens per step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-quality", action="store_true", help="skip the output-error report")
     ap.add_argument("--cpu-sample-tokens", type=int, default=1)
     ap.add_argument("--cpu-sample-cols", type=int, default=512,
                     help="output columns of each linear in the CPU sample (cost is linear in columns)")
@@ -322,11 +323,80 @@ def run_sharq(args, world, rank, local):
     result["clocks"] = {"sm_mhz": cs.get("sm_mhz"), "sm_max_mhz": cs.get("sm_max_mhz"), "reasons": cs.get("reasons"),
                         "samples": cs.get("samples")}
 
+    if not args.no_quality and rank == 0:
+        result["quality"] = quality_report(sq, dev, xs, preps, prep_bufs, outs, ls, prep_index)
     if not args.no_e2e:
         result["e2e"] = e2e_sharq(args, sq, dev, stream, xs_host, preps, prep_bufs, qws, outs, ls, prep_index, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args)
     return result
+
+
+E2M1_VALUES = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0, -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0]
+
+
+def dequantized_weight(sq, qw, dev):
+    """deq(Q(W)) in fp32 from the library's exported codes and scales (for
+    the quality report only): E2M1 value x block scale x tensor scale."""
+    wx = sq.weight_export(qw)
+    blk = sq.BLOCK[qw.desc.fmt]
+    codes = torch.from_numpy(wx["codes"]).to(dev).long()
+    sc = torch.from_numpy(wx["scales"]).to(dev)
+    sv = (sc.view(torch.float8_e4m3fn).float() if qw.desc.fmt == sq.NVFP4
+          else torch.exp2(sc.float() - 127.0))
+    table = torch.tensor(E2M1_VALUES, device=dev)
+    return table[codes] * sv.repeat_interleave(blk, dim=1) * float(wx["s_tw"])
+
+
+def quality_report(sq, dev, xs, preps, prep_bufs, outs, ls, prep_index):
+    """Output error of every linear against an fp16 GEMM, next to plain NVFP4
+    (reported, not gated). Reference: RN16(LayerNorm(x)) times the fp16
+    weight, in fp32 (torch, outside the timed region: a measuring stick, not
+    part of the path). Plain NVFP4: this library with n = m (the mask keeps
+    everything) and the residual codes zeroed, so that only deq(Q(X_ln))
+    times deq(Q(W)) remains. Metric: relative Frobenius error; "recovered"
+    is the share of plain NVFP4's error that SharQ removes. Both paths use
+    the same Q(W), whose error dominates against the fp16 weight, so the
+    report adds the activation-side error: against RN16(LayerNorm(x)) times
+    deq(Q(W))."""
+    torch.backends.cuda.matmul.allow_tf32 = False
+    per = {}
+    plain = {}
+    for i, (name, k) in enumerate(preps):
+        p = sq.prepare(xs[i], None, None, EPS, M_GROUP, M_GROUP, sq.NVFP4)
+        off = p.desc.r_codes - p.buf.data_ptr()
+        p.buf[off:off + xs[i].shape[0] * k // 2].zero_()
+        plain[name] = p
+    for j, lin in enumerate(ls.linears):
+        i = prep_index[lin.prep]
+        w = torch.from_numpy(synth.weights(1000 + j, lin.n_out, lin.k).view(np.float16)).to(dev)
+        x_ln = torch.nn.functional.layer_norm(xs[i].float(), (lin.k,), eps=EPS).half().float()
+        qw = sq.quantize_weight(w, sq.NVFP4)
+        out_plain = sq.linear(plain[lin.prep], qw)
+        rec = {}
+        for tag, wref in (("", w.float()), ("act_", None)):
+            ref = x_ln @ (wref if wref is not None else dequantized_weight(sq, qw, dev)).t()
+            nref = torch.linalg.vector_norm(ref).item()
+            e_sharq = torch.linalg.vector_norm(outs[j].float() - ref).item() / nref
+            e_plain = torch.linalg.vector_norm(out_plain.float() - ref).item() / nref
+            rec.update({tag + "sharq": e_sharq, tag + "nvfp4": e_plain, tag + "recovered": (e_plain - e_sharq) / e_plain})
+            del ref
+        per[lin.name] = rec
+        del x_ln, out_plain, qw, w
+    torch.cuda.synchronize()
+    st = sq.get_last_error()
+    if st != sq.OK:
+        raise RuntimeError(f"device status after quality report: {sq.status_name(st)}")
+    return {"metric": "relative Frobenius error vs fp16 GEMM of RN16(LayerNorm(x)) W^T",
+            "plain": "NVFP4 (n = m, no residual path)",
+            "mean_sharq": float(np.mean([v["sharq"] for v in per.values()])),
+            "mean_nvfp4": float(np.mean([v["nvfp4"] for v in per.values()])),
+            "mean_recovered": float(np.mean([v["recovered"] for v in per.values()])),
+            "act_reference": "RN16(LayerNorm(x)) deq(Q(W))^T: activation-side error only",
+            "mean_act_sharq": float(np.mean([v["act_sharq"] for v in per.values()])),
+            "mean_act_nvfp4": float(np.mean([v["act_nvfp4"] for v in per.values()])),
+            "mean_act_recovered": float(np.mean([v["act_recovered"] for v in per.values()])),
+            "per_linear": per}
 
 
 def e2e_sharq(args, sq, dev, stream, xs_host, preps, prep_bufs, qws, outs, ls, prep_index, world):
