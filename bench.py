@@ -523,6 +523,8 @@ def run_case(args, world, rank, local):
     stream = torch.cuda.current_stream()
     if kind == "moe":
         return run_moe(args, nums[0] if nums else 4096)
+    if kind == "sweep":
+        return run_sweep(args)
     if kind == "prep":
         M, K = nums[:2]
         fmt, n, m = (nums[2:5] + [0, N_KEEP, M_GROUP][len(nums[2:5]):])
@@ -568,6 +570,67 @@ def run_case(args, world, rank, local):
     return {"case": args.case, "ms_median": t * 1e3, "ms_min": min(ms), "achieved": achieved, "unit": unit,
             "peak": peak, "frac": achieved / peak, "bound": bound, "steps": args.steps,
             "outlier_frac": args.outlier_frac, "peak_source": peak_src}
+
+
+def run_sweep(args):
+    """Decode-vs-prefill sweep on the Llama-3.1-8B down projection (14336 ->
+    4096), NVFP4 2:4: for M = 1, 2, 4, ..., 16384 the prep and the dual GEMM
+    are timed separately (CUDA events, L2 flushed before every call, median
+    of the steps). Reported per M: prep GB/s (algorithmic bytes), GEMM
+    TFLOP/s (algorithmic), GEMM GB/s over the weight and activation bytes it
+    must read, and which roofline bounds it (t_ideal = max(flops / FP4 peak,
+    bytes / HBM peak))."""
+    import sparsity_gemm_b200 as sq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    K, N = 14336, 4096
+    peaks, peak_src = load_peaks()
+    fp4 = peaks["bf16_tflops"] * FP4_OVER_BF16 * 1e12
+    hbm = peaks["hbm_gbs"] * 1e9
+    w = torch.from_numpy(synth.weights(1006, N, K).view(np.float16)).to(dev)
+    qw = sq.quantize_weight(w, sq.NVFP4)
+    del w
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    w_bytes = N * K * (0.5 + 1.0 / 16)
+    rows = []
+    for lg in range(15):
+        M = 1 << lg
+        x = torch.from_numpy(synth.activations_student(6, M, K, outlier_frac=args.outlier_frac).view(np.float16)).to(dev)
+        p = sq.prepare(x, None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4)
+        out = torch.empty((M, N), dtype=torch.float16, device=dev)
+        ops = (lambda: sq.prepare(x, None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4, out=p),
+               lambda: sq.linear(p, qw, out=out))
+        t = []
+        for op in ops:
+            for _ in range(args.warmup):
+                flush.zero_()
+                op()
+            ms = []
+            for _ in range(args.steps):
+                flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                op()
+                b.record(stream)
+                b.synchronize()
+                ms.append(a.elapsed_time(b))
+            t.append(statistics.median(ms) / 1e3)
+        st = sq.get_last_error()
+        if st != sq.OK:
+            raise RuntimeError(sq.status_name(st))
+        flops = 2.0 * M * N * K * (1 + N_KEEP / M_GROUP)
+        g_bytes = w_bytes + M * K * (1.0 + 2.0 / 16) + 2.0 * M * N
+        t_ideal = max(flops / fp4, g_bytes / hbm)
+        rows.append({"M": M, "prep_us": t[0] * 1e6, "prep_gbs": PREP_BYTES_PER_ELEM * M * K / t[0] / 1e9,
+                     "gemm_us": t[1] * 1e6, "gemm_tflops": flops / t[1] / 1e12, "gemm_gbs": g_bytes / t[1] / 1e9,
+                     "gemm_bound": "tensor" if flops / fp4 > g_bytes / hbm else "hbm",
+                     "gemm_roofline_frac": t_ideal / t[1]})
+        del x, p, out
+    cross = next((r["M"] for r in rows if r["gemm_bound"] == "tensor"), None)
+    return {"case": "sweep", "workload": "Llama-3.1-8B down projection 14336 -> 4096, NVFP4 2:4, M = 1 .. 16384",
+            "outlier_frac": args.outlier_frac, "crossover_M": cross,
+            "peaks": {"fp4_tflops": fp4 / 1e12, "hbm_gbs": hbm / 1e9, "source": peak_src},
+            "l2": "flushed (256 MB write) before every call", "steps": args.steps, "rows": rows}
 
 
 def run_moe(args, tokens):

@@ -72,6 +72,11 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kBarBytes + 4 <= kBarArea, "barrier area");
 static_assert(kColSf0 + kSfBufs * kSfBufCols <= kTmemCols, "tensor memory columns");
 static_assert(kTableBytes % 4 == 0, "table alignment");
+// Split-K partial tile in the stage memory: 128 rows of 256 fp32, rows
+// padded by 16 bytes so that a warp's 32 rows hit different banks.
+constexpr uint32_t kPartStride = kBN * 4 + 16;
+constexpr int kMaxSplit = 8;
+static_assert(kBM * kPartStride <= (uint32_t)(kStages * kStageBytes), "split-K partial fits the stages");
 
 enum : unsigned {
     kSiteProducer = 0x101,
@@ -100,6 +105,10 @@ struct GemmParams {
     int32_t groups;
     int64_t rows;            // grouped rows (= offsets[groups])
     int64_t w_gstride;       // bytes between two groups' weight payloads
+    // split-K (dense launches only): `split` CTAs of one cluster share a
+    // tile, each over a K range, and reduce through distributed shared
+    // memory; 1 = no split.
+    int32_t split;
 };
 
 // Instruction descriptor of the block-scaled MMA (M = 128, N = 256, E2M1 x
@@ -196,6 +205,19 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     const int m_tiles = GROUPED ? (*table_ok ? tiles[p.groups] : 0) : (p.m_tok + kBM - 1) / kBM;
     const int n_tiles = (p.n_out + kBN - 1) / kBN;
     const int num_tiles = m_tiles * n_tiles, kt_count = p.k / (2 * kBKBytes);
+    // Tiles of this CTA: tile_begin, tile_begin + tile_step, ...; K steps
+    // kt_begin .. kt_end - 1 of each. Split-K: one tile per cluster, one K
+    // range per CTA of the cluster.
+    const bool split = !GROUPED && p.split > 1;
+    int tile_begin = blockIdx.x, tile_step = gridDim.x, kt_begin = 0, kt_end = kt_count, rank = 0;
+    if (split) {
+        rank = (int)cluster_ctarank();
+        tile_begin = blockIdx.x / p.split;
+        tile_step = num_tiles;
+        kt_begin = rank * kt_count / p.split;
+        kt_end = (rank + 1) * kt_count / p.split;
+    }
+    const int kt_n = kt_end - kt_begin;
     const int64_t atoms_per_row_blk = (int64_t)(p.k / (FMT == kFmtNV ? 16 : 32)) / 4;
 
     if (warp == 0) {
@@ -204,11 +226,11 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             for (int s = 0; s < kStages; ++s) last[s] = -1;
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+            for (int tile = tile_begin; ok && tile < num_tiles; tile += tile_step) {
                 const int nb = tile % n_tiles, mb = tile / n_tiles;
                 const int grp = GROUPED ? group_of_tile(tiles, p.groups, mb) : 0;
                 const uint8_t *sfb = p.sfb + (GROUPED ? (int64_t)grp * p.w_gstride : 0);
-                for (int kt = 0; kt < kt_count; ++kt, ++it) {
+                for (int kt = kt_begin; kt < kt_end; ++kt, ++it) {
                     const int s = (int)(it % kStages);
                     const uint32_t ph = (it / kStages) & 1u;
                     if (!mbar_wait(empty_bar(s), ph ^ 1u, p.status, kSiteProducer, p.wait_ns)) {
@@ -247,11 +269,11 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     } else if (warp == 1) {
         if (lane == 0) {
             uint32_t it = 0, tile_iter = 0;
-            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tile_iter) {
+            for (int tile = tile_begin; tile < num_tiles; tile += tile_step, ++tile_iter) {
                 if (!mbar_wait(acc_empty, (tile_iter & 1u) ^ 1u, p.status, kSiteMmaAcc, p.wait_ns)) break;
                 tc_fence_after();
                 bool ok = true;
-                for (int kt = 0; kt < kt_count; ++kt, ++it) {
+                for (int kt = kt_begin; kt < kt_end; ++kt, ++it) {
                     const int s = (int)(it % kStages);
                     const uint32_t ph = (it / kStages) & 1u;
                     if (!mbar_wait(full_bar(s), ph, p.status, kSiteMmaFull, p.wait_ns)) {
@@ -271,7 +293,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                     const uint64_t db = desc_operand(st + kOffB);
 #pragma unroll
                     for (int j = 0; j < kMmaPerStage; ++j) {  // MMAs of K = 64 (32 bytes) per K tile
-                        const uint32_t acc = (kt | j) != 0;
+                        const uint32_t acc = (kt != kt_begin || j != 0) ? 1u : 0u;
                         if (FMT == kFmtNV) {
                             const uint32_t idesc = idesc_of<FMT>(0);
                             tc_mma_nvf4(tmem, da_s + 2 * j, db + 2 * j, idesc, sf + kSfaS + 4 * j, sf + kSfb + 8 * j, acc);
@@ -309,8 +331,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         // depend on nothing the epilogue does.
         const int q = warp & 3;
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-        const int my_tiles = (int)blockIdx.x < num_tiles ? (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-        const uint32_t total_stages = (uint32_t)my_tiles * (uint32_t)kt_count;
+        const int my_tiles = tile_begin < num_tiles ? (num_tiles - 1 - tile_begin) / tile_step + 1 : 0;
+        const uint32_t total_stages = (uint32_t)my_tiles * (uint32_t)kt_n;
         for (uint32_t it = 0; it < total_stages; ++it) {
             const int s = (int)(it % kStages);
             const int b = (int)(it % kSfBufs);
@@ -341,9 +363,9 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const float s_t = *p.s_t;
         float alpha = __fmul_rn(s_t, *p.s_tw);
-        const unsigned store_pause_ns = (unsigned)min(60 * kt_count, 1000);
+        const unsigned store_pause_ns = (unsigned)min(60 * kt_n, 1000);
         uint32_t tile_iter = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tile_iter) {
+        for (int tile = tile_begin; tile < num_tiles; tile += tile_step, ++tile_iter) {
             const int nb = tile % n_tiles, mb = tile / n_tiles;
             int grp = 0;
             if constexpr (GROUPED) {
@@ -354,6 +376,26 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             const bool got = mbar_wait(acc_full, tile_iter & 1u, p.status, kSiteEpilogue, p.wait_ns);
             if (!__all_sync(0xFFFFFFFFu, got)) break;  // warp-uniform: tcgen05.ld is .aligned
             tc_fence_after();
+            if (split) {
+                // Split-K: the fp32 partial tile (rows below m_tok) goes to
+                // this CTA's stage memory, which no copy or MMA uses any
+                // more; the cluster reduces it at the end of the kernel.
+                const int row_local = q * 32 + lane;
+                const bool keep = (int64_t)mb * kBM + row_local < p.m_tok;
+                const uint32_t dst = sbase + (uint32_t)row_local * kPartStride;
+#pragma unroll
+                for (int cc = 0; cc < kBN / 32; ++cc) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + lane_base + (uint32_t)(cc * 32), r);
+                    tmem_ld_wait();
+                    if (keep) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            sts128(dst + (uint32_t)(cc * 128 + 16 * i), r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+                    }
+                }
+                break;  // one tile per CTA
+            }
             // out = RN16(RN32(acc * alpha)) (packed multiplies round each
             // product to fp32 before the conversion).
             uint32_t h[kBN / 32][16];
@@ -381,7 +423,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                 row = mb * kBM + q * 32 + lane;
                 row_end = p.m_tok;
             }
-            const unsigned pause_ns = tile + (int)gridDim.x < num_tiles ? store_pause_ns : 0u;
+            const unsigned pause_ns = tile + tile_step < num_tiles ? store_pause_ns : 0u;
             // The stores are spread over the next tile's main loop: every SM
             // reaches its tile boundary at about the same time, and a burst
             // of all their stores delays the operand loads the next tile
@@ -400,6 +442,39 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                 if (cc + 1 < kBN / 32 && pause_ns) __nanosleep(pause_ns);
             }
         }
+    }
+
+    if (split) {
+        // Split-K reduction: CTA `rank` of the cluster sums column slice
+        // rank of the tile over every CTA's partial, in rank order (a fixed
+        // order, so results do not depend on timing), reading the peers'
+        // shared memory; then scales, rounds to fp16 and stores. All
+        // threads of all CTAs pass both cluster barriers.
+        cluster_sync();  // every partial is in its CTA's shared memory
+        if (warp >= 2 && warp <= 5 && tile_begin < num_tiles) {
+            const int mb = tile_begin / n_tiles, nb = tile_begin % n_tiles;
+            const int S = p.split, cols = kBN / S, groups4 = cols / 4;
+            const int valid = (int)min((int64_t)kBM, (int64_t)p.m_tok - (int64_t)mb * kBM);
+            const float alpha = __fmul_rn(*p.s_t, *p.s_tw);
+            for (int item = (warp - 2) * 32 + lane; item < valid * groups4; item += 128) {
+                const int r = item / groups4, col = rank * cols + (item % groups4) * 4;
+                if (nb * kBN + col >= p.n_out) continue;
+                const uint32_t off = sbase + (uint32_t)r * kPartStride + (uint32_t)col * 4u;
+                float4 acc = ld_cluster_f4(mapa_shared(off, 0));
+                for (int c = 1; c < S; ++c) {
+                    const float4 v = ld_cluster_f4(mapa_shared(off, (uint32_t)c));
+                    acc.x = __fadd_rn(acc.x, v.x);
+                    acc.y = __fadd_rn(acc.y, v.y);
+                    acc.z = __fadd_rn(acc.z, v.z);
+                    acc.w = __fadd_rn(acc.w, v.w);
+                }
+                __half2 h0 = __floats2half2_rn(__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha));
+                __half2 h1 = __floats2half2_rn(__fmul_rn(acc.z, alpha), __fmul_rn(acc.w, alpha));
+                *reinterpret_cast<uint2 *>(p.out + ((int64_t)mb * kBM + r) * p.n_out + nb * kBN + col) =
+                    make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
+            }
+        }
+        cluster_sync();  // no CTA leaves while its partial is being read
     }
 
     tc_fence_before();
@@ -482,8 +557,7 @@ static bool make_grouped_code_map(CUtensorMap *tm, const void *base, uint64_t ro
 }
 
 template <int FMT, bool GROUPED>
-static sharq_status launch_gemm(LaunchCtx &ctx, const CUtensorMap &tm_as, const CUtensorMap &tm_ar,
-                                const CUtensorMap &tm_b, const GemmParams &gp, int64_t max_tiles) {
+static sharq_status set_gemm_attrs() {
     static bool attr_done[64] = {};
     int dev = 0;
     SQ_CUDA_TRY(cudaGetDevice(&dev));
@@ -493,11 +567,88 @@ static sharq_status launch_gemm(LaunchCtx &ctx, const CUtensorMap &tm_as, const 
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes));
         attr_done[dev] = true;
     }
+    return SHARQ_OK;
+}
+
+template <int FMT, bool GROUPED>
+static sharq_status launch_gemm(LaunchCtx &ctx, const CUtensorMap &tm_as, const CUtensorMap &tm_ar,
+                                const CUtensorMap &tm_b, const GemmParams &gp, int64_t max_tiles) {
+    sharq_status st = set_gemm_attrs<FMT, GROUPED>();
+    if (st != SHARQ_OK) return st;
     const unsigned grid = (unsigned)(max_tiles < ctx.num_sms ? max_tiles : ctx.num_sms);
     dual_gemm_kernel<FMT, GROUPED><<<grid, kGemmThreads, kSmemBytes, ctx.stream>>>(tm_as, tm_ar, tm_b, gp);
     ctx.launches++;
     SQ_CUDA_TRY(cudaGetLastError());
     return SHARQ_OK;
+}
+
+// Split-K launch: `tiles` clusters of gp.split CTAs, one tile per cluster.
+template <int FMT>
+static sharq_status launch_gemm_split(LaunchCtx &ctx, const CUtensorMap &tm_as, const CUtensorMap &tm_ar,
+                                      const CUtensorMap &tm_b, const GemmParams &gp, int64_t tiles) {
+    sharq_status st = set_gemm_attrs<FMT, false>();
+    if (st != SHARQ_OK) return st;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(tiles * gp.split), 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = ctx.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)gp.split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    SQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, dual_gemm_kernel<FMT, false>, tm_as, tm_ar, tm_b, gp));
+    ctx.launches++;
+    SQ_CUDA_TRY(cudaGetLastError());
+    return SHARQ_OK;
+}
+
+// Clusters of `split` CTAs of this kernel that can be resident at once (0 if
+// such a cluster does not fit), cached per device, format and size.
+template <int FMT>
+static int active_clusters(int split) {
+    static int cache[64][kMaxSplit + 1];
+    static bool known[64][kMaxSplit + 1] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || split > kMaxSplit) return 0;
+    if (!known[dev][split]) {
+        if (set_gemm_attrs<FMT, false>() != SHARQ_OK) return 0;
+        cudaLaunchConfig_t cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3((unsigned)split, 1, 1);
+        cfg.blockDim = dim3(kGemmThreads, 1, 1);
+        cfg.dynamicSmemBytes = kSmemBytes;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)split;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, dual_gemm_kernel<FMT, false>, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        cache[dev][split] = n;
+        known[dev][split] = true;
+    }
+    return cache[dev][split];
+}
+
+// Split-K factor for a dense launch: when the tiles fill less than half the
+// SMs, the largest power of two <= 8 with tiles x split <= SMs, split <= K
+// steps, and all the clusters resident at once; 1 otherwise.
+template <int FMT>
+static int choose_split(LaunchCtx &ctx, int64_t tiles, int kt_count) {
+    if (tiles * 2 > ctx.num_sms) return 1;
+    int s = kMaxSplit;
+    while (s > 1 && (tiles * s > ctx.num_sms || s > kt_count || active_clusters<FMT>(s) < tiles)) s >>= 1;
+    return s;
 }
 
 static GemmParams gemm_params(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, void *out) {
@@ -514,6 +665,7 @@ static GemmParams gemm_params(LaunchCtx &ctx, const sharq_prep &P, const sharq_w
     gp.k = (int32_t)P.k;
     gp.status = ctx.status;
     gp.wait_ns = ctx.wait_ns;
+    gp.split = 1;
     return gp;
 }
 
@@ -524,8 +676,13 @@ sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &
         !make_code_map(&tm_ar, P.r_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
         !make_code_map(&tm_b, W.codes, (uint64_t)(W.k / 2), (uint64_t)W.n_out, kBN))
         return SHARQ_ERR_CUDA;
-    const GemmParams gp = gemm_params(ctx, P, W, out);
+    GemmParams gp = gemm_params(ctx, P, W, out);
     const int64_t tiles = ((P.m_tok + kBM - 1) / kBM) * ((W.n_out + kBN - 1) / kBN);
+    const int kt_count = (int)(P.k / (2 * kBKBytes));
+    gp.split = P.fmt == kFmtNV ? choose_split<kFmtNV>(ctx, tiles, kt_count) : choose_split<kFmtMX>(ctx, tiles, kt_count);
+    if (gp.split > 1)
+        return P.fmt == kFmtNV ? launch_gemm_split<kFmtNV>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
+                               : launch_gemm_split<kFmtMX>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
     return P.fmt == kFmtNV ? launch_gemm<kFmtNV, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
                            : launch_gemm<kFmtMX, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
 }

@@ -121,8 +121,9 @@ def test_linear_grouped_matches_oracle(sq, fmt, n_out):
 
 def test_one_group_identity_equals_dense_linear(sq):
     """One expert over all rows in order: the grouped path runs the dense
-    path's arithmetic, so the outputs are identical."""
-    tokens, k, n_out = 257, 768, 320
+    path's arithmetic, so the outputs are identical (a shape with enough
+    tiles that the dense launch does not split K)."""
+    tokens, k, n_out = 1217, 768, 2048
     x = synth.activations_student(240, tokens, k)
     w = synth.weights(241, n_out, k)
     p = sq.prepare(cuda16(x), None, None, EPS, 2, 4, 0)

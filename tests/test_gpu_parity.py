@@ -87,6 +87,11 @@ LINEAR_CASES = [
     (129, 512, 1024, 1, 4, 8),
     (256, 288, 768, 0, 1, 2),
     (45, 1024, 2048, 0, 2, 4),  # 8 K tiles, more than the pipeline depth
+    # Few tiles: K is split across a cluster (300 x 544: 2 CTAs per tile,
+    # 129 x 512: 4, 45 x 1024: 8) and reduced through distributed shared
+    # memory; the rows below end the MXFP4 and 16-tile variants.
+    (3, 512, 2048, 1, 2, 4),
+    (130, 2048, 2048, 0, 2, 4),
 ]
 
 
