@@ -7,7 +7,8 @@
 //
 // Two passes over the activations, because the NVFP4 tensor scale depends on
 // amax(X_ln) over the whole tensor:
-//   1. ln_stats_kernel (one CTA per row): exact LayerNorm statistics from
+//   1. ln_stats_kernel (one CTA per row; ln_stats_warp_kernel, one warp per
+//      row, for short rows or many rows): exact LayerNorm statistics from
 //      integer sums and the row's amax|X_ln|, folded into one global word by
 //      an atomic max. Without gamma/beta, X_ln is a non-decreasing function of
 //      x within a row, so amax|X_ln| comes from the row's min and max of x;
@@ -202,6 +203,107 @@ ln_stats_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gam
         float a = 0.0f;
         for (int w = 0; w < kStatsThreads / 32; ++w) a = fmaxf(a, red_max[w]);
         atomicMax(amax_word, __float_as_uint(a));
+    }
+}
+
+// Warp per row (rows of at most kWarpRowMaxK elements, or any row length
+// when the rows fill the GPU): eight rows per CTA, the statistics reduced with shuffles only, and one atomic per CTA for
+// the tensor's amax (one CTA per row leaves most threads idle on short rows
+// and puts one atomic per row on a single word). Same exact sums, so the
+// results equal those of ln_stats_kernel bit for bit. With gamma/beta the
+// row is read a second time (from L2) for amax|X_ln|.
+constexpr int64_t kWarpRowMaxK = 8192;
+
+template <bool AFFINE>
+__global__ void __launch_bounds__(kStatsThreads)
+ln_stats_warp_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gamma,
+                     const uint16_t *__restrict__ beta, float eps, int64_t k, int64_t m_tok,
+                     float2 *__restrict__ stats, unsigned *__restrict__ amax_word) {
+    __shared__ float red_max[kStatsThreads / 32];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t row = (int64_t)blockIdx.x * (kStatsThreads / 32) + warp;
+    float amax = 0.0f;
+    if (row < m_tok) {
+        const int nvec = (int)(k / 8);
+        const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * k);
+        ExactSums e = {0, 0, 0, 0, 0};
+        uint32_t mx = 0xFC00FC00u, mn = 0x7C007C00u;  // (-inf, -inf), (+inf, +inf) as half2
+        auto consume = [&](const uint4 &v) {
+            accum_pair(v.x, e);
+            accum_pair(v.y, e);
+            accum_pair(v.z, e);
+            accum_pair(v.w, e);
+            if (!AFFINE) {
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(w4[q]));
+                    asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(w4[q]));
+                }
+            }
+        };
+        int c = lane;
+        for (; c + 96 < nvec; c += 128) {  // four loads in flight per lane
+            const uint4 v0 = xr[c], v1 = xr[c + 32], v2 = xr[c + 64], v3 = xr[c + 96];
+            consume(v0);
+            consume(v1);
+            consume(v2);
+            consume(v3);
+        }
+        for (; c < nvec; c += 32) consume(xr[c]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            e.hi += __shfl_xor_sync(0xFFFFFFFFu, e.hi, o);
+            e.lo += __shfl_xor_sync(0xFFFFFFFFu, e.lo, o);
+            e.hh += __shfl_xor_sync(0xFFFFFFFFu, e.hh, o);
+            e.hl += __shfl_xor_sync(0xFFFFFFFFu, e.hl, o);
+            e.ll += __shfl_xor_sync(0xFFFFFFFFu, e.ll, o);
+            if (!AFFINE) {
+                const uint32_t omx = __shfl_xor_sync(0xFFFFFFFFu, mx, o), omn = __shfl_xor_sync(0xFFFFFFFFu, mn, o);
+                asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(omx));
+                asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(omn));
+            }
+        }
+        float2 st = make_float2(0.0f, 0.0f);
+        if (lane == 0) {
+            st = finish_stats(e, k, eps);
+            stats[row] = st;
+        }
+        st.x = __shfl_sync(0xFFFFFFFFu, st.x, 0);
+        st.y = __shfl_sync(0xFFFFFFFFu, st.y, 0);
+        if (!AFFINE) {
+            // X_ln = RN(RN(x - mu) * rstd) is non-decreasing in x: the row's
+            // amax|X_ln| is reached at its smallest or largest x.
+            const float xmax = fmaxf(h2f((uint16_t)mx), h2f((uint16_t)(mx >> 16)));
+            const float xmin = fminf(h2f((uint16_t)mn), h2f((uint16_t)(mn >> 16)));
+            amax = fmaxf(fabsf(__fmul_rn(__fsub_rn(xmax, st.x), st.y)), fabsf(__fmul_rn(__fsub_rn(xmin, st.x), st.y)));
+        } else {
+            const bool has_g = gamma != nullptr, has_b = beta != nullptr;
+            for (int cc = lane; cc < nvec; cc += 32) {
+                const uint4 v = xr[cc];
+                const uint4 g = has_g ? __ldg(reinterpret_cast<const uint4 *>(gamma) + cc) : make_uint4(0, 0, 0, 0);
+                const uint4 bb = has_b ? __ldg(reinterpret_cast<const uint4 *>(beta) + cc) : make_uint4(0, 0, 0, 0);
+                const uint32_t xv[4] = {v.x, v.y, v.z, v.w}, gv[4] = {g.x, g.y, g.z, g.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float xl = ln_apply(h2f((uint16_t)(xv[q] >> (16 * h))), st.x, st.y, has_g,
+                                                  h2f((uint16_t)(gv[q] >> (16 * h))), has_b,
+                                                  h2f((uint16_t)(bv[q] >> (16 * h))));
+                        amax = fmaxf(amax, fabsf(xl));
+                    }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+        }
+    }
+    if (lane == 0) red_max[warp] = amax;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float a = 0.0f;
+        for (int w = 0; w < kStatsThreads / 32; ++w) a = fmaxf(a, red_max[w]);
+        atomicMax(amax_word, __float_as_uint(a));  // non-negative floats order like their bits
     }
 }
 
@@ -741,7 +843,20 @@ sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, 
     if (meta_atomic && P.m_tok > 0)  // unaligned metadata fields are OR-ed into a zeroed stream
         SQ_CUDA_TRY(cudaMemsetAsync(P.meta, 0, (size_t)(P.m_tok * P.meta_row_bytes), ctx.stream));
     float2 *stats = reinterpret_cast<float2 *>(P.scratch);
-    if (P.m_tok > 0) {
+    // Warp per row when there are rows enough for a CTA of eight per SM (or
+    // the rows are short); one CTA per row keeps few-row (decode) launches
+    // short.
+    const bool warp_rows = P.m_tok >= (int64_t)ctx.num_sms * (kStatsThreads / 32) || P.k <= kWarpRowMaxK;
+    if (P.m_tok > 0 && warp_rows) {
+        const unsigned grid = (unsigned)((P.m_tok + kStatsThreads / 32 - 1) / (kStatsThreads / 32));
+        if (gamma || beta)
+            ln_stats_warp_kernel<true><<<grid, kStatsThreads, 0, ctx.stream>>>(
+                (const uint16_t *)x, (const uint16_t *)gamma, (const uint16_t *)beta, eps, P.k, P.m_tok, stats, words);
+        else
+            ln_stats_warp_kernel<false><<<grid, kStatsThreads, 0, ctx.stream>>>(
+                (const uint16_t *)x, nullptr, nullptr, eps, P.k, P.m_tok, stats, words);
+        ctx.launches++;
+    } else if (P.m_tok > 0) {
         if (gamma || beta)
             ln_stats_kernel<true><<<(unsigned)P.m_tok, kStatsThreads, (size_t)(2 * P.k), ctx.stream>>>(
                 (const uint16_t *)x, (const uint16_t *)gamma, (const uint16_t *)beta, eps, P.k, stats, words);
