@@ -40,6 +40,7 @@ def _declare(L):
     L.oracle_u128_to_double.argtypes = [C.c_uint64, C.c_uint64]
     L.oracle_u128_to_double.restype = C.c_double
     L.oracle_ln_stats.argtypes = [vp, i64, i64, f32, vp, vp]
+    L.oracle_rms_stats.argtypes = [vp, i64, i64, f32, vp, vp]
     L.oracle_ln_apply.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp]
     L.oracle_e2m1_value.argtypes = [i32]
     L.oracle_e2m1_value.restype = C.c_double
@@ -56,6 +57,7 @@ def _declare(L):
     L.oracle_tensor_scale.restype = f32
     L.oracle_mask.argtypes = [vp, i64, i64, i32, i32, vp, vp]
     L.oracle_prepare.argtypes = [vp, i64, i64, vp, vp, f32, i32, i32, i32] + [vp] * 14
+    L.oracle_prepare_norm.argtypes = [vp, i64, i64, vp, vp, f32, i32, i32, i32, i32] + [vp] * 14
     L.oracle_quantize_weight.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp]
     L.oracle_linear.argtypes = [vp, vp, vp, vp, f32, vp, vp, f32, i64, i64, i64, i32, vp, vp]
 
@@ -113,6 +115,19 @@ def ln_stats(x: np.ndarray, eps: float):
     return mu, rstd
 
 
+def rms_stats(x: np.ndarray, eps: float):
+    """RMSNorm statistics: (mu = 0, rstd) per row."""
+    x = _u16(x)
+    rows, k = x.shape
+    mu = np.empty(rows, np.float32)
+    rstd = np.empty(rows, np.float32)
+    lib().oracle_rms_stats(_p(x), rows, k, eps, _p(mu), _p(rstd))
+    return mu, rstd
+
+
+NORMS = {"layer": 0, "rms": 1}
+
+
 def ln_apply(x, gamma, beta, mu, rstd):
     x = _u16(x)
     rows, k = x.shape
@@ -167,10 +182,12 @@ class Prepared:
     m: int
 
 
-def prepare(x, gamma, beta, eps: float, n: int, m: int, fmt: int, s_t=None) -> Prepared:
+def prepare(x, gamma, beta, eps: float, n: int, m: int, fmt: int, s_t=None, norm: str = "layer") -> Prepared:
     """The preparation operator on the rows of x. s_t=None derives the
     tensor scale from these rows; a given s_t (the scale of a larger tensor
-    these rows were sampled from) is used as is."""
+    these rows were sampled from) is used as is. norm: "layer" (LayerNorm)
+    or "rms" (RMSNorm: no centring, beta must be None)."""
+    assert norm in NORMS and (norm == "layer" or beta is None)
     x = _u16(x)
     rows, k = x.shape
     blk = BLOCK[fmt]
@@ -186,10 +203,10 @@ def prepare(x, gamma, beta, eps: float, n: int, m: int, fmt: int, s_t=None) -> P
     r_scales = np.empty((rows, k // blk), np.uint8)
     s_t_arr = np.empty(1, np.float32)
     s_t_in = None if s_t is None else np.array([s_t], np.float32)
-    lib().oracle_prepare(_p(x), rows, k, _p(g), _p(b), eps, n, m, fmt,
-                         _p(mu), _p(rstd), _p(x_ln), _p(s), _p(deq_s), _p(r),
-                         _p(idx), _p(keep), _p(s_codes), _p(s_scales),
-                         _p(r_codes), _p(r_scales), _p(s_t_arr), _p(s_t_in))
+    lib().oracle_prepare_norm(_p(x), rows, k, _p(g), _p(b), eps, n, m, fmt, NORMS[norm],
+                              _p(mu), _p(rstd), _p(x_ln), _p(s), _p(deq_s), _p(r),
+                              _p(idx), _p(keep), _p(s_codes), _p(s_scales),
+                              _p(r_codes), _p(r_scales), _p(s_t_arr), _p(s_t_in))
     s_t = s_t_arr
     return Prepared(mu, rstd, x_ln, s, deq_s, r, idx, keep, s_codes, s_scales,
                     r_codes, r_scales, s_t[0], fmt, n, m)
@@ -204,16 +221,16 @@ class QWeight:
     fmt: int
 
 
-def tensor_scale_of(x, gamma, beta, eps: float, fmt: int) -> np.float32:
-    """The activation tensor scale over all rows of x (LayerNorm, then
-    amax), computed in row chunks to bound memory."""
+def tensor_scale_of(x, gamma, beta, eps: float, fmt: int, norm: str = "layer") -> np.float32:
+    """The activation tensor scale over all rows of x (the normalization,
+    then amax), computed in row chunks to bound memory."""
     x = _u16(x)
     rows = x.shape[0]
     amax = np.float32(0.0)
     step = max(1, (1 << 24) // max(1, x.shape[1]))
     for r0 in range(0, rows, step):
         xs = x[r0:r0 + step]
-        mu, rstd = ln_stats(xs, eps)
+        mu, rstd = (ln_stats if norm == "layer" else rms_stats)(xs, eps)
         xl = ln_apply(xs, gamma, beta, mu, rstd)
         amax = max(amax, np.abs(xl).max() if xl.size else np.float32(0))
     if fmt != NVFP4:

@@ -116,6 +116,30 @@ void oracle_ln_stats(const uint16_t *x, int64_t rows, int64_t k, float eps,
     }
 }
 
+/* RMSNorm statistics, exactly (reading: models that normalize by the    */
+/* root mean square, without centring, use this form of the preparation */
+/* operator's normalization; same exact sums as above):                 */
+/*                                                                      */
+/*   S2   = sum a_i^2                     exact                          */
+/*   ms   = RN64(S2) / (K * 2^48)          (binary64 division)           */
+/*   rstd = RN32( 1 / sqrt(ms + eps) )    (binary64 sqrt and division)  */
+/*   mu   = 0, so the apply step below gives RN32(RN32(x * rstd) * g).   */
+
+void oracle_rms_stats(const uint16_t *x, int64_t rows, int64_t k, float eps,
+                      float *mu, float *rstd)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        u128 s2 = 0;
+        for (int64_t i = 0; i < k; ++i) {
+            int64_t a = (int64_t)ldexp(oracle_half_to_double(x[r * k + i]), 24);
+            s2 += (u128)((i128)a * (i128)a);
+        }
+        double ms64 = u128_to_double_rn(s2) / ((double)k * 281474976710656.0);
+        mu[r] = 0.0f;
+        rstd[r] = (float)(1.0 / sqrt(ms64 + (double)eps));
+    }
+}
+
 /* LayerNorm apply, left to right, each step rounded to binary32:       */
 /*   X_ln = RN32( RN32( RN32(x - mu) * rstd ) * gamma ) + beta           */
 /* gamma == NULL skips the multiply, beta == NULL skips the add.        */
@@ -329,16 +353,21 @@ void oracle_mask(const float *x_ln, int64_t rows, int64_t k, int n, int m,
 /* prepared with that tensor's scale (the per-row steps do not depend on   */
 /* other rows).                                                            */
 
-void oracle_prepare(const uint16_t *x, int64_t rows, int64_t k,
-                    const uint16_t *gamma, const uint16_t *beta, float eps,
-                    int n, int m, int fmt,
-                    float *mu, float *rstd, float *x_ln, float *s, float *deq_s, float *r,
-                    uint8_t *idx, uint8_t *keep,
-                    uint8_t *s_codes, uint8_t *s_scales,
-                    uint8_t *r_codes, uint8_t *r_scales, float *s_t_out, const float *s_t_in)
+/* norm: 0 = LayerNorm (oracle_ln_stats), 1 = RMSNorm (oracle_rms_stats,  */
+/* no beta). The steps after the normalization are the same.               */
+void oracle_prepare_norm(const uint16_t *x, int64_t rows, int64_t k,
+                         const uint16_t *gamma, const uint16_t *beta, float eps,
+                         int n, int m, int fmt, int norm,
+                         float *mu, float *rstd, float *x_ln, float *s, float *deq_s, float *r,
+                         uint8_t *idx, uint8_t *keep,
+                         uint8_t *s_codes, uint8_t *s_scales,
+                         uint8_t *r_codes, uint8_t *r_scales, float *s_t_out, const float *s_t_in)
 {
     int blk = fmt == FMT_NVFP4 ? 16 : 32;
-    oracle_ln_stats(x, rows, k, eps, mu, rstd);
+    if (norm)
+        oracle_rms_stats(x, rows, k, eps, mu, rstd);
+    else
+        oracle_ln_stats(x, rows, k, eps, mu, rstd);
     oracle_ln_apply(x, rows, k, gamma, beta, mu, rstd, x_ln);
     float s_t = s_t_in ? *s_t_in : oracle_tensor_scale(x_ln, rows * k, fmt);
     *s_t_out = s_t;
@@ -354,6 +383,18 @@ void oracle_prepare(const uint16_t *x, int64_t rows, int64_t k,
             r[e] = x_ln[e] - deq_s[e];
         }
     oracle_quantize(r, rows, k, fmt, s_t, r_codes, r_scales);
+}
+
+void oracle_prepare(const uint16_t *x, int64_t rows, int64_t k,
+                    const uint16_t *gamma, const uint16_t *beta, float eps,
+                    int n, int m, int fmt,
+                    float *mu, float *rstd, float *x_ln, float *s, float *deq_s, float *r,
+                    uint8_t *idx, uint8_t *keep,
+                    uint8_t *s_codes, uint8_t *s_scales,
+                    uint8_t *r_codes, uint8_t *r_scales, float *s_t_out, const float *s_t_in)
+{
+    oracle_prepare_norm(x, rows, k, gamma, beta, eps, n, m, fmt, 0, mu, rstd, x_ln, s, deq_s, r, idx, keep,
+                        s_codes, s_scales, r_codes, r_scales, s_t_out, s_t_in);
 }
 
 /* Weight quantization: the same block quantizer along K on every row of  */
