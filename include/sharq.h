@@ -179,6 +179,22 @@ sharq_status sharq_prepare(const void *x_dev, int64_t m_tok, int64_t k,
                            void *stream);
 
 /*
+ * The preparation operator with RMSNorm in place of LayerNorm: the form the
+ * evaluated model families (Llama, Qwen) normalize with. An interface
+ * addition: the SharQ abstract names layer normalization only. Statistics
+ * from the same exact integer sums, without centring:
+ *   ms = RN64(S2) / (K 2^48), rstd = RN32(1/sqrt(ms + eps)) in binary64,
+ *   X_n = RN32(RN32(x * rstd) * w)
+ * then the mask, Q(S), R and Q(R) exactly as sharq_prepare. The exported
+ * mu is 0.
+ *   w_dev  fp16 [k] RMSNorm weight, or NULL (no multiply).
+ * Everything else (arguments, buffer, preconditions) as sharq_prepare.
+ */
+sharq_status sharq_prepare_rms(const void *x_dev, int64_t m_tok, int64_t k, const void *w_dev, float eps,
+                               int n, int m, int fmt, void *prep_dev, size_t prep_bytes, sharq_prep *prep_out,
+                               void *stream);
+
+/*
  * Preparation operator for callers that cannot allocate device memory.
  * (An interface addition: the SharQ paper has no counterpart.)
  *

@@ -64,6 +64,7 @@ def lib():
         L.sharq_prep_bytes.restype = sz
         L.sharq_quantize_weight.argtypes = [vp, i64, i64, i32, vp, sz, C.POINTER(SharqWQ), vp]
         L.sharq_prepare.argtypes = [vp, i64, i64, vp, vp, f32, i32, i32, i32, vp, sz, C.POINTER(SharqPrep), vp]
+        L.sharq_prepare_rms.argtypes = [vp, i64, i64, vp, f32, i32, i32, i32, vp, sz, C.POINTER(SharqPrep), vp]
         L.sharq_linear.argtypes = [C.POINTER(SharqPrep), C.POINTER(SharqWQ), vp, vp]
         L.sharq_prep_export.argtypes = [C.POINTER(SharqPrep)] + [vp] * 8 + [vp]
         L.sharq_weight_export.argtypes = [C.POINTER(SharqWQ), vp, vp, vp, vp, vp]
@@ -89,7 +90,7 @@ def lib():
         L.sharq_last_launch_count.restype = i32
         for name in ("sharq_quantize_weight", "sharq_prepare", "sharq_linear", "sharq_prep_export",
                      "sharq_weight_export", "sharq_get_last_error", "sharq_quantize_weight_grouped",
-                     "sharq_gather_rows", "sharq_linear_grouped"):
+                     "sharq_gather_rows", "sharq_linear_grouped", "sharq_prepare_rms"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -166,8 +167,11 @@ def quantize_weight(w: torch.Tensor, fmt: int = NVFP4, stream=None) -> Quantized
 
 
 def prepare(x: torch.Tensor, ln_w=None, ln_b=None, eps: float = 1e-5, n: int = 2, m: int = 4,
-            fmt: int = NVFP4, out: Prepared | None = None, stream=None) -> Prepared:
-    """Fused preparation operator on x [m_tok, k] (fp16, CUDA)."""
+            fmt: int = NVFP4, out: Prepared | None = None, stream=None, norm: str = "layer") -> Prepared:
+    """Fused preparation operator on x [m_tok, k] (fp16, CUDA). norm:
+    "layer" (LayerNorm with ln_w, ln_b) or "rms" (RMSNorm with weight ln_w;
+    ln_b must be None)."""
+    assert norm in ("layer", "rms") and (norm == "layer" or ln_b is None)
     assert x.dtype == torch.float16 and x.is_cuda and x.dim() == 2 and x.is_contiguous()
     for t in (ln_w, ln_b):
         assert t is None or (t.dtype == torch.float16 and t.is_cuda and t.numel() == x.shape[1] and t.is_contiguous())
@@ -181,8 +185,12 @@ def prepare(x: torch.Tensor, ln_w=None, ln_b=None, eps: float = 1e-5, n: int = 2
         buf = out.buf
     desc = SharqPrep()
     xp = _ptr(x) if m_tok > 0 else None
-    _check(lib().sharq_prepare(xp, m_tok, k, _ptr(ln_w), _ptr(ln_b), float(eps), n, m, fmt, _ptr(buf),
-                               buf.numel(), C.byref(desc), _stream(stream)), "sharq_prepare")
+    if norm == "rms":
+        _check(lib().sharq_prepare_rms(xp, m_tok, k, _ptr(ln_w), float(eps), n, m, fmt, _ptr(buf), buf.numel(),
+                                       C.byref(desc), _stream(stream)), "sharq_prepare_rms")
+    else:
+        _check(lib().sharq_prepare(xp, m_tok, k, _ptr(ln_w), _ptr(ln_b), float(eps), n, m, fmt, _ptr(buf),
+                                   buf.numel(), C.byref(desc), _stream(stream)), "sharq_prepare")
     return Prepared(buf, desc)
 
 

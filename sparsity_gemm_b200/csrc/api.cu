@@ -140,9 +140,9 @@ sharq_status sharq_quantize_weight(const void *w_dev, int64_t n_out, int64_t k, 
     return st;
 }
 
-sharq_status sharq_prepare(const void *x_dev, int64_t m_tok, int64_t k, const void *ln_w_dev, const void *ln_b_dev,
-                           float eps, int n, int m, int fmt, void *prep_dev, size_t prep_bytes, sharq_prep *prep_out,
-                           void *stream) {
+static sharq_status prepare_norm(const void *x_dev, int64_t m_tok, int64_t k, const void *ln_w_dev,
+                                 const void *ln_b_dev, float eps, int n, int m, int fmt, void *prep_dev,
+                                 size_t prep_bytes, sharq_prep *prep_out, void *stream, int norm) {
     g_last_launches = 0;
     size_t need = sharq_prep_bytes(m_tok, k, n, m, fmt);
     if (!need || !prep_dev || !prep_out || prep_bytes < need) return SHARQ_ERR_INVALID_ARG;
@@ -155,10 +155,21 @@ sharq_status sharq_prepare(const void *x_dev, int64_t m_tok, int64_t k, const vo
     sharq_status st = make_ctx(stream, ctx);
     if (st != SHARQ_OK) return st;
     fill_prep(prep_out, prep_dev, m_tok, k, n, m, fmt);
-    st = sq::launch_prepare(ctx, *prep_out, x_dev, ln_w_dev, ln_b_dev, eps);
+    st = sq::launch_prepare(ctx, *prep_out, x_dev, ln_w_dev, ln_b_dev, eps, norm);
     if (st == SHARQ_OK && cudaGetLastError() != cudaSuccess) st = SHARQ_ERR_CUDA;
     g_last_launches = ctx.launches;
     return st;
+}
+
+sharq_status sharq_prepare(const void *x_dev, int64_t m_tok, int64_t k, const void *ln_w_dev, const void *ln_b_dev,
+                           float eps, int n, int m, int fmt, void *prep_dev, size_t prep_bytes, sharq_prep *prep_out,
+                           void *stream) {
+    return prepare_norm(x_dev, m_tok, k, ln_w_dev, ln_b_dev, eps, n, m, fmt, prep_dev, prep_bytes, prep_out, stream, 0);
+}
+
+sharq_status sharq_prepare_rms(const void *x_dev, int64_t m_tok, int64_t k, const void *w_dev, float eps, int n,
+                               int m, int fmt, void *prep_dev, size_t prep_bytes, sharq_prep *prep_out, void *stream) {
+    return prepare_norm(x_dev, m_tok, k, w_dev, nullptr, eps, n, m, fmt, prep_dev, prep_bytes, prep_out, stream, 1);
 }
 
 sharq_status sharq_linear(const sharq_prep *prep, const sharq_wq *wq, void *out_dev, void *stream) {

@@ -88,7 +88,15 @@ __device__ float2 finish_stats(const ExactSums &e, int64_t k, float eps) {
                        __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(var64, (double)eps)))));
 }
 
-template <bool AFFINE>
+// RMSNorm: ms = RN64(S2) / (K 2^48); rstd = RN32(1 / sqrt(ms + eps)); mu = 0.
+__device__ float2 finish_stats_rms(const ExactSums &e, int64_t k, float eps) {
+    const __int128 s2 = ((__int128)e.hh << 40) + ((__int128)e.hl << 21) + (__int128)e.ll;
+    const double ms64 = __ddiv_rn(u128_to_f64((unsigned __int128)s2), __dmul_rn((double)k, 281474976710656.0));
+    return make_float2(0.0f, __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms64, (double)eps)))));
+}
+
+// RMS: RMSNorm statistics (no centring) instead of LayerNorm's.
+template <bool AFFINE, bool RMS>
 __global__ void __launch_bounds__(kStatsThreads)
 ln_stats_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gamma,
                 const uint16_t *__restrict__ beta, float eps, int64_t k, float2 *__restrict__ stats,
@@ -163,7 +171,7 @@ ln_stats_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gam
             asm("max.f16x2 %0, %0, %1;" : "+r"(tmx) : "r"(red_mx[w]));
             asm("min.f16x2 %0, %0, %1;" : "+r"(tmn) : "r"(red_mn[w]));
         }
-        const float2 st = finish_stats(t, k, eps);
+        const float2 st = RMS ? finish_stats_rms(t, k, eps) : finish_stats(t, k, eps);
         stats[row] = st;
         row_stat = st;
         if (!AFFINE) {
@@ -214,7 +222,7 @@ ln_stats_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gam
 // row is read a second time (from L2) for amax|X_ln|.
 constexpr int64_t kWarpRowMaxK = 8192;
 
-template <bool AFFINE>
+template <bool AFFINE, bool RMS>
 __global__ void __launch_bounds__(kStatsThreads)
 ln_stats_warp_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gamma,
                      const uint16_t *__restrict__ beta, float eps, int64_t k, int64_t m_tok,
@@ -266,7 +274,7 @@ ln_stats_warp_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
         }
         float2 st = make_float2(0.0f, 0.0f);
         if (lane == 0) {
-            st = finish_stats(e, k, eps);
+            st = RMS ? finish_stats_rms(e, k, eps) : finish_stats(e, k, eps);
             stats[row] = st;
         }
         st.x = __shfl_sync(0xFFFFFFFFu, st.x, 0);
@@ -763,7 +771,7 @@ extern "C" sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, 
         return SHARQ_ERR_CUDA;
     static bool attr_done[64] = {false};
     if (!attr_done[dev]) {
-        if (cudaFuncSetAttribute(ln_stats_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(ln_stats_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)(2 * SHARQ_K_MAX)) != cudaSuccess)
             return SHARQ_ERR_CUDA;
         attr_done[dev] = true;
@@ -796,11 +804,11 @@ extern "C" sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, 
         return SHARQ_ERR_CUDA;
     if (m_tok > 0) {
         if (ln_w_dev || ln_b_dev)
-            ln_stats_kernel<true><<<(unsigned)m_tok, kStatsThreads, (size_t)(2 * k), s>>>(
+            ln_stats_kernel<true, false><<<(unsigned)m_tok, kStatsThreads, (size_t)(2 * k), s>>>(
                 (const uint16_t *)x_dev, (const uint16_t *)ln_w_dev, (const uint16_t *)ln_b_dev, eps, k, stats,
                 amax_word);
         else
-            ln_stats_kernel<false><<<(unsigned)m_tok, kStatsThreads, 0, s>>>((const uint16_t *)x_dev, nullptr, nullptr,
+            ln_stats_kernel<false, false><<<(unsigned)m_tok, kStatsThreads, 0, s>>>((const uint16_t *)x_dev, nullptr, nullptr,
                                                                            eps, k, stats, amax_word);
     }
     const int64_t total = P.sf_rows * (k / kUnit);
@@ -825,17 +833,47 @@ extern "C" sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, 
 
 namespace sq {
 
-sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, const void *gamma, const void *beta,
-                            float eps) {
+// Statistics pass: one warp per row when there are rows enough for a CTA of
+// eight per SM (or the rows are short); one CTA per row keeps few-row
+// (decode) launches short.
+template <bool RMS>
+static sharq_status launch_stats(LaunchCtx &ctx, const sharq_prep &P, const void *x, const void *gamma,
+                                 const void *beta, float eps, float2 *stats, unsigned *words) {
     static bool attr_done[64] = {false};
     int dev = 0;
     SQ_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
     if (!attr_done[dev]) {
-        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_kernel<true, RMS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)(2 * SHARQ_K_MAX)));
         attr_done[dev] = true;
     }
+    if (P.m_tok == 0) return SHARQ_OK;
+    const bool warp_rows = P.m_tok >= (int64_t)ctx.num_sms * (kStatsThreads / 32) || P.k <= kWarpRowMaxK;
+    const uint16_t *xx = (const uint16_t *)x, *gg = (const uint16_t *)gamma, *bb = (const uint16_t *)beta;
+    if (warp_rows) {
+        const unsigned grid = (unsigned)((P.m_tok + kStatsThreads / 32 - 1) / (kStatsThreads / 32));
+        if (gamma || beta)
+            ln_stats_warp_kernel<true, RMS><<<grid, kStatsThreads, 0, ctx.stream>>>(xx, gg, bb, eps, P.k, P.m_tok,
+                                                                                   stats, words);
+        else
+            ln_stats_warp_kernel<false, RMS><<<grid, kStatsThreads, 0, ctx.stream>>>(xx, nullptr, nullptr, eps, P.k,
+                                                                                    P.m_tok, stats, words);
+    } else {
+        if (gamma || beta)
+            ln_stats_kernel<true, RMS><<<(unsigned)P.m_tok, kStatsThreads, (size_t)(2 * P.k), ctx.stream>>>(
+                xx, gg, bb, eps, P.k, stats, words);
+        else
+            ln_stats_kernel<false, RMS><<<(unsigned)P.m_tok, kStatsThreads, 0, ctx.stream>>>(xx, nullptr, nullptr,
+                                                                                           eps, P.k, stats, words);
+    }
+    ctx.launches++;
+    SQ_CUDA_TRY(cudaGetLastError());
+    return SHARQ_OK;
+}
+
+sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, const void *gamma, const void *beta,
+                            float eps, int norm) {
     unsigned *words = reinterpret_cast<unsigned *>(P.tensor_scale) - 1;  // [0] amax bits, [1] s_t
     SQ_CUDA_TRY(cudaMemsetAsync(words, 0, sizeof(unsigned), ctx.stream));
     const int ib = idx_bits(P.m);
@@ -843,28 +881,9 @@ sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, 
     if (meta_atomic && P.m_tok > 0)  // unaligned metadata fields are OR-ed into a zeroed stream
         SQ_CUDA_TRY(cudaMemsetAsync(P.meta, 0, (size_t)(P.m_tok * P.meta_row_bytes), ctx.stream));
     float2 *stats = reinterpret_cast<float2 *>(P.scratch);
-    // Warp per row when there are rows enough for a CTA of eight per SM (or
-    // the rows are short); one CTA per row keeps few-row (decode) launches
-    // short.
-    const bool warp_rows = P.m_tok >= (int64_t)ctx.num_sms * (kStatsThreads / 32) || P.k <= kWarpRowMaxK;
-    if (P.m_tok > 0 && warp_rows) {
-        const unsigned grid = (unsigned)((P.m_tok + kStatsThreads / 32 - 1) / (kStatsThreads / 32));
-        if (gamma || beta)
-            ln_stats_warp_kernel<true><<<grid, kStatsThreads, 0, ctx.stream>>>(
-                (const uint16_t *)x, (const uint16_t *)gamma, (const uint16_t *)beta, eps, P.k, P.m_tok, stats, words);
-        else
-            ln_stats_warp_kernel<false><<<grid, kStatsThreads, 0, ctx.stream>>>(
-                (const uint16_t *)x, nullptr, nullptr, eps, P.k, P.m_tok, stats, words);
-        ctx.launches++;
-    } else if (P.m_tok > 0) {
-        if (gamma || beta)
-            ln_stats_kernel<true><<<(unsigned)P.m_tok, kStatsThreads, (size_t)(2 * P.k), ctx.stream>>>(
-                (const uint16_t *)x, (const uint16_t *)gamma, (const uint16_t *)beta, eps, P.k, stats, words);
-        else
-            ln_stats_kernel<false><<<(unsigned)P.m_tok, kStatsThreads, 0, ctx.stream>>>(
-                (const uint16_t *)x, nullptr, nullptr, eps, P.k, stats, words);
-        ctx.launches++;
-    }
+    const sharq_status sst = norm ? launch_stats<true>(ctx, P, x, gamma, beta, eps, stats, words)
+                                  : launch_stats<false>(ctx, P, x, gamma, beta, eps, stats, words);
+    if (sst != SHARQ_OK) return sst;
     const int64_t total = P.sf_rows * (P.k / kUnit);
     int64_t blocks = (total + kEncodeThreads - 1) / kEncodeThreads;
     const int64_t cap = (int64_t)ctx.num_sms * 16;

@@ -15,8 +15,9 @@ struct LaunchCtx {
     int launches;          // kernels enqueued by the current entry point
 };
 
+// norm: 0 = LayerNorm, 1 = RMSNorm (beta must be NULL).
 sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, const void *gamma,
-                            const void *beta, float eps);
+                            const void *beta, float eps, int norm);
 sharq_status launch_quantize_weight(LaunchCtx &ctx, const sharq_wq &W, const void *w, int64_t groups,
                                    int64_t gstride);
 sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, void *out);

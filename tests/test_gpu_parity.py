@@ -211,3 +211,40 @@ def test_tiny_and_huge_scales_bit_exact():
     ow = oracle.quantize_weight(w, 0)
     qw = sq.quantize_weight(cuda16(w), 0)
     assert_weight_matches(sq.weight_export(qw), ow)
+
+
+RMS_CASES = [
+    # (m_tok, k, fmt, n, m, weight): warp-per-row statistics (k <= 8192) and
+    # CTA-per-row statistics (few rows of k = 14336)
+    (37, 256, 0, 2, 4, False),
+    (300, 1024, 1, 2, 4, True),
+    (129, 768, 0, 4, 8, True),
+    (5, 14336, 0, 2, 4, False),
+    (3, 14336, 1, 2, 4, True),
+]
+
+
+@pytest.mark.parametrize("m_tok,k,fmt,n,m,weight", RMS_CASES)
+def test_prepare_rms_bit_exact(m_tok, k, fmt, n, m, weight):
+    import sparsity_gemm_b200 as sq
+    x = synth.activations_student(500 + m_tok + k, m_tok, k)
+    g = synth.ln_params(501, k)[0] if weight else None
+    op = oracle.prepare(x, g, None, 1e-5, n, m, fmt, norm="rms")
+    p = sq.prepare(cuda16(x), None if g is None else cuda16(g), None, 1e-5, n, m, fmt, norm="rms")
+    assert_prep_matches(sq.prep_export(p), op)
+    assert sq.get_last_error() == sq.OK
+
+
+def test_linear_on_rms_prepared_input():
+    import sparsity_gemm_b200 as sq
+    m_tok, k, n_out = 200, 1024, 544
+    x = synth.activations_student(510, m_tok, k)
+    g = synth.ln_params(511, k)[0]
+    w = synth.weights(512, n_out, k)
+    op = oracle.prepare(x, g, None, 1e-5, 2, 4, 0, norm="rms")
+    ow = oracle.quantize_weight(w, 0)
+    p = sq.prepare(cuda16(x), cuda16(g), None, 1e-5, 2, 4, 0, norm="rms")
+    out = sq.linear(p, sq.quantize_weight(cuda16(w), 0)).cpu().numpy()
+    want, bound = oracle.linear_prepared(op, ow)
+    assert_linear_close(out, want, bound)
+    assert sq.get_last_error() == sq.OK
