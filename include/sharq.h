@@ -248,7 +248,8 @@ sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, int64_t k,
  *   with the block-scaled code values; products are exact, accumulation is
  *   fp32 in tensor memory (both paths into one accumulator).
  * Preconditions: prep and wq from this library, prep->fmt == wq->fmt,
- * prep->k == wq->k, out_dev non-NULL (may be NULL only if m_tok == 0).
+ * prep->k == wq->k, out_dev non-NULL (may be NULL only if m_tok == 0) and at
+ * least 32-byte aligned (the epilogue writes whole 32-byte sectors).
  */
 sharq_status sharq_linear(const sharq_prep *prep, const sharq_wq *wq, void *out_dev,
                           void *stream);

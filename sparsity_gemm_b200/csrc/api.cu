@@ -182,7 +182,7 @@ sharq_status sharq_linear(const sharq_prep *prep, const sharq_wq *wq, void *out_
         prep->sf_rows % sq::kActRowPad != 0)
         return SHARQ_ERR_INVALID_ARG;
     if (prep->m_tok == 0) return SHARQ_OK;
-    if (!out_dev || !aligned(out_dev, 16) || !prep->s_codes || !prep->r_codes || !wq->codes ||
+    if (!out_dev || !aligned(out_dev, 32) || !prep->s_codes || !prep->r_codes || !wq->codes ||
         wq->scales_backbone != wq->scales_residual)
         return SHARQ_ERR_INVALID_ARG;
     if (prep->m_tok > (1ll << 31) - 256) return SHARQ_ERR_UNSUPPORTED;
@@ -269,7 +269,7 @@ sharq_status sharq_linear_grouped(const sharq_prep *prep, const int32_t *offsets
         return SHARQ_ERR_INVALID_ARG;
     if (!prep->s_codes || !prep->r_codes || !wq->codes || wq->scales_backbone != wq->scales_residual)
         return SHARQ_ERR_INVALID_ARG;
-    if (rows > 0 && (!out_dev || !aligned(out_dev, 16))) return SHARQ_ERR_INVALID_ARG;
+    if (rows > 0 && (!out_dev || !aligned(out_dev, 32))) return SHARQ_ERR_INVALID_ARG;
     if (prep->m_tok > (1ll << 31) - 256) return SHARQ_ERR_UNSUPPORTED;
     sq::LaunchCtx ctx;
     sharq_status st = make_ctx(stream, ctx);

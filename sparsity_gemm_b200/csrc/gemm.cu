@@ -40,6 +40,11 @@ namespace sq {
 #ifndef SQ_GEMM_BKB
 #define SQ_GEMM_BKB 128
 #endif
+// Pause between the epilogue's 32-column store chunks, per K step of the
+// main loop (the stores of a tile are spread over the next tile's loop).
+#ifndef SQ_STORE_PAUSE_NS_PER_KSTEP
+#define SQ_STORE_PAUSE_NS_PER_KSTEP 60
+#endif
 constexpr int kBM = 128, kBN = 256, kBKBytes = SQ_GEMM_BKB;
 constexpr int kABytes = kBM * kBKBytes;
 constexpr int kBBytes = kBN * kBKBytes;
@@ -363,7 +368,9 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
         const float s_t = *p.s_t;
         float alpha = __fmul_rn(s_t, *p.s_tw);
-        const unsigned store_pause_ns = (unsigned)min(60 * kt_n, 1000);
+        // (short loops, fewer than 8 K steps, store at once: the next drain
+        // comes too soon for pacing to pay)
+        const unsigned store_pause_ns = kt_n >= 8 ? (unsigned)min(SQ_STORE_PAUSE_NS_PER_KSTEP * kt_n, 1000) : 0u;
         uint32_t tile_iter = 0;
         for (int tile = tile_begin; tile < num_tiles; tile += tile_step, ++tile_iter) {
             const int nb = tile % n_tiles, mb = tile / n_tiles;
@@ -434,10 +441,12 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             for (int cc = 0; cc < kBN / 32; ++cc) {
                 const int col0 = nb * kBN + cc * 32;
                 if (row < row_end && col0 < p.n_out) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.out + row * p.n_out + col0);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(h[cc][4 * i], h[cc][4 * i + 1], h[cc][4 * i + 2], h[cc][4 * i + 3]);
+                    // two full 32-byte sectors (the output base is 32-byte aligned,
+                    // rows are multiples of 64 bytes)
+                    __half *dst = p.out + row * p.n_out + col0;
+                    stg256(dst, h[cc][0], h[cc][1], h[cc][2], h[cc][3], h[cc][4], h[cc][5], h[cc][6], h[cc][7]);
+                    stg256(dst + 16, h[cc][8], h[cc][9], h[cc][10], h[cc][11], h[cc][12], h[cc][13], h[cc][14],
+                           h[cc][15]);
                 }
                 if (cc + 1 < kBN / 32 && pause_ns) __nanosleep(pause_ns);
             }

@@ -135,6 +135,11 @@ def test_linear_rejects_mismatched_handles_without_cuda(sq):
     w.scales_residual = 1 << 25  # the two scale views must hold the same values
     assert L.sharq_linear(C.byref(p), C.byref(w), out, None) == sq.ERR_INVALID_ARG
     w.scales_residual = 1 << 23
+    # the epilogue writes whole 32-byte sectors: a 16-byte aligned output is refused
+    assert L.sharq_linear(C.byref(p), C.byref(w), C.c_void_p((1 << 24) + 16), None) == sq.ERR_INVALID_ARG
+    w.groups = 3  # stacked weights go to sharq_linear_grouped
+    assert L.sharq_linear(C.byref(p), C.byref(w), out, None) == sq.ERR_INVALID_ARG
+    w.groups = 1
     assert L.sharq_linear(None, C.byref(w), out, None) == sq.ERR_INVALID_ARG
     p.m_tok = 0  # empty activations: nothing to do
     assert L.sharq_linear(C.byref(p), C.byref(w), None, None) == sq.OK
