@@ -12,7 +12,7 @@
 // One CTA per 128-row destination tile. Warp 0 builds the groups' tile
 // table from the device offsets (and checks them); the CTA then finds its
 // group, reads the 128 source row indices, and copies codes (16-byte
-// chunks, one warp per row), mask metadata, LayerNorm statistics and the
+// chunks over all threads), mask metadata, LayerNorm statistics and the
 // scale atoms (4-byte words: one row's 4 scales of one atom are 4
 // consecutive bytes in both layouts). Tile rows past the group's end are
 // zero.
@@ -24,6 +24,23 @@
 namespace sq {
 
 constexpr int kGatherThreads = 256;
+constexpr int kCopyUnroll = 4;  // 16-byte code chunks per operand in flight per thread
+
+// (row, column) of a flat index over rows of `width` items, stepped by a
+// fixed stride without dividing again.
+struct RowCol {
+    int32_t r, c, width, step_r, step_c;
+    __device__ RowCol(int32_t i, int32_t w, int32_t stride)
+        : r(i / w), c(i % w), width(w), step_r(stride / w), step_c(stride % w) {}
+    __device__ void advance() {
+        r += step_r;
+        c += step_c;
+        if (c >= width) {
+            c -= width;
+            ++r;
+        }
+    }
+};
 
 struct GatherParams {
     const uint8_t *s_codes, *r_codes, *s_scales, *r_scales, *meta;
@@ -77,30 +94,85 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherPara
     __syncthreads();
 
     const int64_t d0 = (int64_t)tile * 128;  // first destination row
-    const int64_t row_bytes = p.k / 2, chunks = p.k / 32;
+    const int64_t row_bytes = p.k / 2, chunks = p.k / 32;  // 16-byte chunks per row
+    // Codes: (row, chunk) pairs of the tile over all threads, consecutive
+    // threads on consecutive chunks of a row; kCopyUnroll loads per operand
+    // in flight before the stores (the copy is latency-bound).
+    const int64_t items = 128 * chunks;  // < 2^18
     const uint4 zero4 = make_uint4(0, 0, 0, 0);
-    for (int r = warp; r < 128; r += kGatherThreads / 32) {
-        const int64_t src = src_row[r];
-        const int64_t sp = src >= 0 ? src : 0;  // pointers stay inside the source for zero rows
-        const int64_t dst = d0 + r;
-        const uint4 *ss = reinterpret_cast<const uint4 *>(p.s_codes + sp * row_bytes);
-        const uint4 *sr = reinterpret_cast<const uint4 *>(p.r_codes + sp * row_bytes);
-        uint4 *ds = reinterpret_cast<uint4 *>(p.d_s_codes + dst * row_bytes);
-        uint4 *dr = reinterpret_cast<uint4 *>(p.d_r_codes + dst * row_bytes);
-        for (int64_t c = lane; c < chunks; c += 32) {
-            ds[c] = src >= 0 ? __ldg(ss + c) : zero4;
-            dr[c] = src >= 0 ? __ldg(sr + c) : zero4;
+    RowCol rc(threadIdx.x, (int32_t)chunks, kGatherThreads);
+    for (int64_t i0 = threadIdx.x; i0 < items; i0 += kCopyUnroll * kGatherThreads) {
+        uint4 vs[kCopyUnroll], vr[kCopyUnroll];
+        int64_t dst[kCopyUnroll];
+#pragma unroll
+        for (int j = 0; j < kCopyUnroll; ++j) {
+            const int64_t i = i0 + (int64_t)j * kGatherThreads;
+            vs[j] = zero4;
+            vr[j] = zero4;
+            dst[j] = -1;
+            if (i < items) {
+                const int64_t r = rc.r, c = rc.c;
+                const int64_t src = src_row[r];
+                dst[j] = (d0 + r) * chunks + c;
+                if (src >= 0) {
+                    vs[j] = __ldg(reinterpret_cast<const uint4 *>(p.s_codes) + src * chunks + c);
+                    vr[j] = __ldg(reinterpret_cast<const uint4 *>(p.r_codes) + src * chunks + c);
+                }
+            }
+            rc.advance();
         }
-        if ((p.meta_row & 3) == 0) {
-            const uint32_t *sm = reinterpret_cast<const uint32_t *>(p.meta + sp * p.meta_row);
-            uint32_t *dm = reinterpret_cast<uint32_t *>(p.d_meta + dst * p.meta_row);
-            for (int64_t b = lane; b < p.meta_row / 4; b += 32) dm[b] = src >= 0 ? sm[b] : 0u;
-        } else {
-            const uint8_t *sm = p.meta + sp * p.meta_row;
-            uint8_t *dm = p.d_meta + dst * p.meta_row;
-            for (int64_t b = lane; b < p.meta_row; b += 32) dm[b] = src >= 0 ? sm[b] : (uint8_t)0;
+#pragma unroll
+        for (int j = 0; j < kCopyUnroll; ++j)
+            if (dst[j] >= 0) {
+                reinterpret_cast<uint4 *>(p.d_s_codes)[dst[j]] = vs[j];
+                reinterpret_cast<uint4 *>(p.d_r_codes)[dst[j]] = vr[j];
+            }
+    }
+    // Metadata: 16-byte chunks when the rows allow (four loads in flight),
+    // else 4-byte words, else bytes; then the statistics.
+    if ((p.meta_row & 15) == 0) {
+        const int64_t cpr = p.meta_row / 16, mitems = 128 * cpr;
+        RowCol mc(threadIdx.x, (int32_t)cpr, kGatherThreads);
+        for (int64_t i0 = threadIdx.x; i0 < mitems; i0 += 4 * kGatherThreads) {
+            uint4 v[4];
+            int64_t dst[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t i = i0 + (int64_t)j * kGatherThreads;
+                v[j] = zero4;
+                dst[j] = -1;
+                if (i < mitems) {
+                    const int64_t src = src_row[mc.r];
+                    dst[j] = (d0 + mc.r) * cpr + mc.c;
+                    if (src >= 0) v[j] = __ldg(reinterpret_cast<const uint4 *>(p.meta) + src * cpr + mc.c);
+                }
+                mc.advance();
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                if (dst[j] >= 0) reinterpret_cast<uint4 *>(p.d_meta)[dst[j]] = v[j];
         }
-        if (lane == 0) p.d_stats[dst] = src >= 0 ? p.stats[src] : make_float2(0.0f, 0.0f);
+    } else if ((p.meta_row & 3) == 0) {
+        const int64_t wpr = p.meta_row / 4, mitems = 128 * wpr;
+        RowCol mc(threadIdx.x, (int32_t)wpr, kGatherThreads);
+        for (int64_t i = threadIdx.x; i < mitems; i += kGatherThreads, mc.advance()) {
+            const int64_t r = mc.r, c = mc.c;
+            const int64_t src = src_row[r];
+            reinterpret_cast<uint32_t *>(p.d_meta)[(d0 + r) * wpr + c] =
+                src >= 0 ? reinterpret_cast<const uint32_t *>(p.meta)[src * wpr + c] : 0u;
+        }
+    } else {
+        const int64_t mitems = 128 * p.meta_row;
+        RowCol mc(threadIdx.x, (int32_t)p.meta_row, kGatherThreads);
+        for (int64_t i = threadIdx.x; i < mitems; i += kGatherThreads, mc.advance()) {
+            const int64_t r = mc.r, c = mc.c;
+            const int64_t src = src_row[r];
+            p.d_meta[(d0 + r) * p.meta_row + c] = src >= 0 ? p.meta[src * p.meta_row + c] : (uint8_t)0;
+        }
+    }
+    if (threadIdx.x < 128) {
+        const int64_t src = src_row[threadIdx.x];
+        p.d_stats[d0 + threadIdx.x] = src >= 0 ? p.stats[src] : make_float2(0.0f, 0.0f);
     }
 
     // Scale atoms of this tile: (nblk / 4) atoms of 128 words per operand.
@@ -110,17 +182,31 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherPara
     const uint32_t *swr = reinterpret_cast<const uint32_t *>(p.r_scales);
     uint32_t *dws = reinterpret_cast<uint32_t *>(p.d_s_scales) + (int64_t)tile * words;
     uint32_t *dwr = reinterpret_cast<uint32_t *>(p.d_r_scales) + (int64_t)tile * words;
-    for (int64_t w = threadIdx.x; w < words; w += kGatherThreads) {
-        const int64_t a = w >> 7, o = w & 127;
-        const int64_t src = src_row[(o >> 2) + 32 * (o & 3)];
-        uint32_t vs = 0, vr = 0;
-        if (src >= 0) {
-            const int64_t sw = ((src >> 7) * atoms + a) * 128 + (src & 31) * 4 + ((src >> 5) & 3);
-            vs = __ldg(sws + sw);
-            vr = __ldg(swr + sw);
+    for (int64_t w0 = threadIdx.x; w0 < words; w0 += 4 * kGatherThreads) {  // four loads per operand in flight
+        uint32_t vs[4], vr[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t w = w0 + (int64_t)j * kGatherThreads;
+            vs[j] = 0;
+            vr[j] = 0;
+            if (w < words) {
+                const int64_t a = w >> 7, o = w & 127;
+                const int64_t src = src_row[(o >> 2) + 32 * (o & 3)];
+                if (src >= 0) {
+                    const int64_t sw = ((src >> 7) * atoms + a) * 128 + (src & 31) * 4 + ((src >> 5) & 3);
+                    vs[j] = __ldg(sws + sw);
+                    vr[j] = __ldg(swr + sw);
+                }
+            }
         }
-        dws[w] = vs;
-        dwr[w] = vr;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int64_t w = w0 + (int64_t)j * kGatherThreads;
+            if (w < words) {
+                dws[w] = vs[j];
+                dwr[w] = vr[j];
+            }
+        }
     }
 }
 
