@@ -401,36 +401,77 @@ def quality_report(sq, dev, xs, preps, prep_bufs, outs, ls, prep_index):
 
 def e2e_sharq(args, sq, dev, stream, xs_host, preps, prep_bufs, qws, outs, ls, prep_index, world):
     """Same metric through the public API with host buffers: every step copies
-    its activations from pinned host memory and reads every output back."""
+    its activations from pinned host memory and reads every output back. The
+    steps are pipelined as a serving loop would run them: inputs go in on a
+    copy stream one step ahead (two device input buffers), each linear's
+    output goes back on a second copy stream as soon as it is computed (two
+    device output sets), so host-to-device copies, compute and
+    device-to-host copies overlap; events order every buffer reuse. The
+    timed region runs from the first input copy to the completion of the
+    last output copy."""
     M = args.tokens
-    pinned_in = [t.pin_memory() for t in xs_host]
-    pinned_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
-    dev_in = [torch.empty_like(t, device=dev) for t in xs_host]
     steps = max(3, min(args.steps, 20))
+    pinned_in = [t.pin_memory() for t in xs_host]
+    dev_in = [[torch.empty_like(t, device=dev) for t in xs_host] for _ in range(2)]
+    dev_out = [outs, [torch.empty_like(o) for o in outs]]
+    pinned_out = [[torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs] for _ in range(2)]
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev = lambda: torch.cuda.Event()
 
-    def one():
-        for i in range(len(preps)):
-            dev_in[i].copy_(pinned_in[i], non_blocking=True)
-        for i in range(len(preps)):
-            prep_bufs[i] = sq.prepare(dev_in[i], None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4, out=prep_bufs[i])
-        for j, lin in enumerate(ls.linears):
-            sq.linear(prep_bufs[prep_index[lin.prep]], qws[j], out=outs[j])
-        for j in range(len(outs)):
-            pinned_out[j].copy_(outs[j], non_blocking=True)
+    def run(n_steps, e_start=None):
+        in_ready = [ev() for _ in range(n_steps)]
+        in_free = [ev() for _ in range(n_steps)]      # compute of step s no longer reads dev_in[s % 2]
+        lin_done = [[ev() for _ in outs] for _ in range(n_steps)]
+        out_free = [ev() for _ in range(n_steps)]     # outputs of step s copied back
+        if e_start is not None:
+            e_start.record(s_in)
 
-    one()
+        def load(t):
+            with torch.cuda.stream(s_in):
+                if t >= 2:
+                    s_in.wait_event(in_free[t - 2])
+                for i, x in enumerate(pinned_in):
+                    dev_in[t % 2][i].copy_(x, non_blocking=True)
+                in_ready[t].record(s_in)
+
+        load(0)
+        for t in range(n_steps):
+            if t + 1 < n_steps:
+                load(t + 1)
+            b = t % 2
+            stream.wait_event(in_ready[t])
+            if t >= 2:
+                stream.wait_event(out_free[t - 2])
+            for i in range(len(preps)):
+                prep_bufs[i] = sq.prepare(dev_in[b][i], None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4,
+                                          out=prep_bufs[i], stream=stream)
+            in_free[t].record(stream)
+            for j, lin in enumerate(ls.linears):
+                sq.linear(prep_bufs[prep_index[lin.prep]], qws[j], out=dev_out[b][j], stream=stream)
+                lin_done[t][j].record(stream)
+            with torch.cuda.stream(s_out):
+                for j in range(len(outs)):
+                    s_out.wait_event(lin_done[t][j])
+                    pinned_out[b][j].copy_(dev_out[b][j], non_blocking=True)
+                out_free[t].record(s_out)
+        return out_free[n_steps - 1]
+
+    run(2)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        one()
-    e1.record(stream)
+    last = run(steps, e_start=e0)
+    s_out.wait_event(last)
+    e1.record(s_out)
     torch.cuda.synchronize()
+    st = sq.get_last_error()
+    if st != sq.OK:
+        raise RuntimeError(f"device status after the end-to-end run: {sq.status_name(st)}")
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     return {"value": world * M * steps / (ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": int(sum(t.numel() * 2 for t in xs_host)),
-            "d2h_bytes_per_step": int(sum(o.numel() * 2 for o in outs)), "steps": steps}
+            "d2h_bytes_per_step": int(sum(o.numel() * 2 for o in outs)), "steps": steps,
+            "pipelined": "inputs one step ahead and outputs back on separate copy streams"}
 
 
 # ---------------------------------------------------------------------------
