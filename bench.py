@@ -566,6 +566,8 @@ def run_case(args, world, rank, local):
         return run_moe(args, nums[0] if nums else 4096)
     if kind == "sweep":
         return run_sweep(args)
+    if kind == "vendor_fp4":
+        return run_vendor_fp4(args)
     if kind == "prep":
         M, K = nums[:2]
         fmt, n, m = (nums[2:5] + [0, N_KEEP, M_GROUP][len(nums[2:5]):])
@@ -671,6 +673,43 @@ def run_sweep(args):
     return {"case": "sweep", "workload": "Llama-3.1-8B down projection 14336 -> 4096, NVFP4 2:4, M = 1 .. 16384",
             "outlier_frac": args.outlier_frac, "crossover_M": cross,
             "peaks": {"fp4_tflops": fp4 / 1e12, "hbm_gbs": hbm / 1e9, "source": peak_src},
+            "l2": "flushed (256 MB write) before every call", "steps": args.steps, "rows": rows}
+
+
+def run_vendor_fp4(args):
+    """Context only, outside the library: the vendor's NVFP4 GEMM (cuBLASLt
+    through torch._scaled_mm, random FP4 codes, unit scales) on the layer
+    set's GEMM shapes, timed with CUDA events (L2 flushed before each call).
+    One dense FP4 GEMM per call; the dual-path linear runs two such
+    contractions (backbone and residual) per call."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rows = []
+
+    def ones_blocked(r, c):
+        return torch.ones(((r + 127) // 128 * 128) * ((c + 3) // 4 * 4), device=dev).to(torch.float8_e4m3fn)
+
+    for (M, N, K) in [(8192, 4096, 14336), (8192, 14336, 4096), (8192, 4096, 4096), (8192, 1024, 4096)]:
+        g = torch.Generator(device=dev).manual_seed(0)
+        a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev, generator=g).view(torch.float4_e2m1fn_x2)
+        b = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev, generator=g).view(torch.float4_e2m1fn_x2)
+        sa, sb = ones_blocked(M, K // 16), ones_blocked(N, K // 16)
+        f = lambda: torch._scaled_mm(a, b.t(), sa, sb, out_dtype=torch.bfloat16)
+        for _ in range(args.warmup):
+            flush.zero_()
+            f()
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            e1.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        t = statistics.median(ms) / 1e3
+        rows.append({"M": M, "N": N, "K": K, "us": t * 1e6, "tflops": 2.0 * M * N * K / t / 1e12})
+    return {"case": "vendor_fp4", "what": "cuBLASLt NVFP4 GEMM via torch._scaled_mm, one dense contraction per call",
             "l2": "flushed (256 MB write) before every call", "steps": args.steps, "rows": rows}
 
 
