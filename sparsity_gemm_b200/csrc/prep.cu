@@ -26,40 +26,75 @@
 
 namespace sq {
 
+// Resident encode CTAs per SM the register allocation must allow.
+#ifndef SQ_ENCODE_MIN_CTAS
+#define SQ_ENCODE_MIN_CTAS 3
+#endif
 constexpr int kStatsThreads = 256;
 constexpr int kEncodeThreads = 256;
 constexpr int kUnit = 16;  // elements per encode thread
 
 // ---------------------------------------------------------------------------
 // Exact statistics. With a = x * 2^24 (an integer, |a| < 2^40), write
-// t = x * 2^4 = hi + lo * 2^-20 with hi = floor(t) (|hi| <= 2^20, signed) and
-// 0 <= lo < 2^20, so that a = hi * 2^20 + lo and
+// x = hi * 2^-4 + lo * 2^-24 with hi = floor(x * 2^4) (|hi| <= 1048064,
+// signed) and 0 <= lo < 2^20, so that a = hi * 2^20 + lo and
 //   S1 = 2^20 sum hi + sum lo,
 //   S2 = 2^40 sum hi^2 + 2^21 sum hi*lo + sum lo^2.
-// hi and lo come out of the binary32 pipeline exactly: t + 1.5*2^23 rounded
-// toward -inf holds floor(t) in its low mantissa bits, and (t - floor(t)) *
-// 2^20 + 2^23 holds lo in its low mantissa bits (every step is exact).
+// hi and lo come out of the binary32 pipeline exactly: x + 1.5*2^19 rounded
+// toward -inf lies in [2^19, 2^20), where the spacing of binary32 is 2^-4,
+// so it is 1.5*2^19 + hi * 2^-4 and its bit pattern exceeds that of 1.5*2^19
+// by hi; (x - hi * 2^-4) * 2^24 + 2^23 holds lo in its low mantissa bits
+// (every step is exact).
 struct ExactSums {
     int64_t hi, lo;  // sum hi, sum lo
     int64_t hh, hl;  // sum hi^2, sum hi*lo
     uint64_t ll;     // sum lo^2
 };
 
-__device__ __forceinline__ void accum_pair(uint32_t w, ExactSums &e) {
-    // The product x * 2^4 is exact, so fusing it into the following add is harmless.
-    const uint64_t t = mul2(h2_to_f2(w), pk2(16.0f, 16.0f));             // x * 2^4, exact
-    const uint64_t hm = add2_rm(t, pk2(12582912.0f, 12582912.0f));      // 1.5*2^23 + floor(t)
-    const uint64_t hf = sub2(hm, pk2(12582912.0f, 12582912.0f));        // floor(t), exact
-    const uint64_t lm = fma2(sub2(t, hf), pk2(1048576.0f, 1048576.0f),  // frac * 2^20 + 2^23, exact
+// One lane's sums: hi and lo in 32 bits, the three products in binary64.
+// A lane adds at most SHARQ_K_MAX / 32 values (one warp per row is the
+// narrowest split of a row): 2048 * 1048064 < 2^31 and 2048 * (2^20 - 1) <
+// 2^31; every product is an integer below 2^40, so each binary64 FMA adds
+// an exact product to an integer sum below 2048 * 2^40 = 2^51 < 2^53 and
+// rounds nothing. (On B200 the products on the FP64 pipe cost less than the
+// 64-bit integer multiplies on the FMA pipe, which saturated it.)
+struct LaneSums {
+    int32_t hi, lo;
+    double hh, hl, ll;
+};
+static_assert((int64_t)SHARQ_K_MAX / 32 * 1048064 < (1ll << 31), "lane sums of hi fit in 32 bits");
+static_assert((int64_t)SHARQ_K_MAX / 32 * ((1 << 20) - 1) < (1ll << 31), "lane sums of lo fit in 32 bits");
+static_assert((double)(SHARQ_K_MAX / 32) * 1099511627776.0 < 9007199254740992.0, "lane product sums exact in binary64");
+
+__device__ __forceinline__ ExactSums widen(const LaneSums &l) {
+    return ExactSums{l.hi, l.lo, __double2ll_rn(l.hh), __double2ll_rn(l.hl), (uint64_t)__double2ll_rn(l.ll)};
+}
+
+// Integer h (|h| < 2^31) as a binary64, exactly: the bit pattern of
+// 1.5 * 2^52 plus h (sign-extended) is the value 1.5 * 2^52 + h.
+__device__ __forceinline__ double i32_to_f64_exact(int32_t h) {
+    return __dsub_rn(__hiloint2double(0x43380000 + (h >> 31), h), 6755399441055744.0);
+}
+
+__device__ __forceinline__ void accum_pair(uint32_t w, LaneSums &e) {
+    const uint64_t f = h2_to_f2(w);                                    // x, exact
+    const uint64_t hm = add2_rm(f, pk2(786432.0f, 786432.0f));         // 1.5*2^19 + hi * 2^-4
+    const uint64_t hf = sub2(hm, pk2(786432.0f, 786432.0f));           // hi * 2^-4, exact
+    const uint64_t lm = fma2(sub2(f, hf), pk2(16777216.0f, 16777216.0f),  // lo + 2^23, exact
                              pk2(8388608.0f, 8388608.0f));
     const float2 hmf = up2(hm), lmf = up2(lm);
-    const int32_t h0 = (int32_t)__float_as_uint(hmf.x) - 0x4B400000, h1 = (int32_t)__float_as_uint(hmf.y) - 0x4B400000;
+    const int32_t h0 = (int32_t)__float_as_uint(hmf.x) - 0x49400000, h1 = (int32_t)__float_as_uint(hmf.y) - 0x49400000;
     const int32_t l0 = (int32_t)(__float_as_uint(lmf.x) & 0x7FFFFFu), l1 = (int32_t)(__float_as_uint(lmf.y) & 0x7FFFFFu);
     e.hi += h0 + h1;
     e.lo += l0 + l1;
-    e.hh += (int64_t)h0 * h0 + (int64_t)h1 * h1;
-    e.hl += (int64_t)h0 * l0 + (int64_t)h1 * l1;
-    e.ll += (uint64_t)(uint32_t)l0 * (uint32_t)l0 + (uint64_t)(uint32_t)l1 * (uint32_t)l1;
+    const double hd0 = i32_to_f64_exact(h0), hd1 = i32_to_f64_exact(h1);
+    const double ld0 = i32_to_f64_exact(l0), ld1 = i32_to_f64_exact(l1);
+    e.hh = __fma_rn(hd0, hd0, e.hh);
+    e.hh = __fma_rn(hd1, hd1, e.hh);
+    e.hl = __fma_rn(hd0, ld0, e.hl);
+    e.hl = __fma_rn(hd1, ld1, e.hl);
+    e.ll = __fma_rn(ld0, ld0, e.ll);
+    e.ll = __fma_rn(ld1, ld1, e.ll);
 }
 
 // Round-to-nearest-even binary64 value of a non-negative 128-bit integer.
@@ -112,14 +147,14 @@ ln_stats_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gam
     const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * k);
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-    ExactSums e = {0, 0, 0, 0, 0};
+    LaneSums l = {0, 0, 0.0, 0.0, 0.0};
     uint32_t mx = 0xFC00FC00u, mn = 0x7C007C00u;  // (-inf, -inf), (+inf, +inf) as half2
     auto consume = [&](const uint4 &v, int c) {
         if (AFFINE) row_cache[c] = v;
-        accum_pair(v.x, e);
-        accum_pair(v.y, e);
-        accum_pair(v.z, e);
-        accum_pair(v.w, e);
+        accum_pair(v.x, l);
+        accum_pair(v.y, l);
+        accum_pair(v.z, l);
+        accum_pair(v.w, l);
         if (!AFFINE) {
             asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(v.x));
             asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(v.y));
@@ -140,6 +175,7 @@ ln_stats_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gam
         consume(v1, c + kStatsThreads);
     }
     if (c < nvec) consume(xr[c], c);
+    ExactSums e = widen(l);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         e.hi += __shfl_xor_sync(0xFFFFFFFFu, e.hi, o);
@@ -215,32 +251,53 @@ ln_stats_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gam
 }
 
 // Warp per row (rows of at most kWarpRowMaxK elements, or any row length
-// when the rows fill the GPU): eight rows per CTA, the statistics reduced with shuffles only, and one atomic per CTA for
-// the tensor's amax (one CTA per row leaves most threads idle on short rows
-// and puts one atomic per row on a single word). Same exact sums, so the
-// results equal those of ln_stats_kernel bit for bit. With gamma/beta the
-// row is read a second time (from L2) for amax|X_ln|.
+// when the rows fill the GPU): eight rows per CTA, the statistics reduced with
+// shuffles only, and one atomic per CTA for the tensor's amax (one CTA per row
+// leaves most threads idle on short rows and puts one atomic per row on a
+// single word). Same exact sums, so the results equal those of
+// ln_stats_kernel bit for bit. The row streams through a ring of
+// kStatsStages slots per lane (four 16-byte vectors each) filled by
+// asynchronous copies issued two iterations ahead, so that loads stay in
+// flight while the lane computes. With gamma/beta the row is read a second
+// time (from L2) for amax|X_ln|.
 constexpr int64_t kWarpRowMaxK = 8192;
+constexpr int kStatsStages = 3;
+constexpr int kStatsRingBytes = (kStatsThreads / 32) * kStatsStages * 4 * 32 * 16;  // 48 KB
 
 template <bool AFFINE, bool RMS>
 __global__ void __launch_bounds__(kStatsThreads)
 ln_stats_warp_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gamma,
                      const uint16_t *__restrict__ beta, float eps, int64_t k, int64_t m_tok,
                      float2 *__restrict__ stats, unsigned *__restrict__ amax_word) {
+    extern __shared__ uint4 ring[];  // [warp][stage][vector j][lane]
     __shared__ float red_max[kStatsThreads / 32];
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int64_t row = (int64_t)blockIdx.x * (kStatsThreads / 32) + warp;
     float amax = 0.0f;
     if (row < m_tok) {
         const int nvec = (int)(k / 8);
+        const int nvl = nvec / 32;           // vectors per lane (k is a multiple of 256)
+        const int iters = (nvl + 3) / 4;     // four vectors per lane per iteration
         const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * k);
-        ExactSums e = {0, 0, 0, 0, 0};
+        uint4 *wring = ring + (size_t)warp * kStatsStages * 4 * 32;
+        const uint32_t wbase = smem_u32(wring);
+        auto issue = [&](int it) {
+            if (it < iters) {
+                const int st = it % kStatsStages;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (4 * it + j < nvl)
+                        cp_async16(wbase + (uint32_t)(((st * 4 + j) * 32 + lane) * 16), xr + lane + 32 * (4 * it + j));
+            }
+            cp_async_commit();  // possibly empty: one group per iteration keeps the count uniform
+        };
+        LaneSums l = {0, 0, 0.0, 0.0, 0.0};
         uint32_t mx = 0xFC00FC00u, mn = 0x7C007C00u;  // (-inf, -inf), (+inf, +inf) as half2
         auto consume = [&](const uint4 &v) {
-            accum_pair(v.x, e);
-            accum_pair(v.y, e);
-            accum_pair(v.z, e);
-            accum_pair(v.w, e);
+            accum_pair(v.x, l);
+            accum_pair(v.y, l);
+            accum_pair(v.z, l);
+            accum_pair(v.w, l);
             if (!AFFINE) {
                 const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -250,15 +307,25 @@ ln_stats_warp_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
                 }
             }
         };
-        int c = lane;
-        for (; c + 96 < nvec; c += 128) {  // four loads in flight per lane
-            const uint4 v0 = xr[c], v1 = xr[c + 32], v2 = xr[c + 64], v3 = xr[c + 96];
-            consume(v0);
-            consume(v1);
-            consume(v2);
-            consume(v3);
+        issue(0);
+        issue(1);
+        for (int it = 0; it < iters; ++it) {
+            cp_async_wait<1>();  // this lane's copies of iteration `it` have landed
+            const int st = it % kStatsStages;
+            if (4 * it + 3 < nvl) {
+                const uint4 v0 = wring[(st * 4 + 0) * 32 + lane], v1 = wring[(st * 4 + 1) * 32 + lane];
+                const uint4 v2 = wring[(st * 4 + 2) * 32 + lane], v3 = wring[(st * 4 + 3) * 32 + lane];
+                consume(v0);
+                consume(v1);
+                consume(v2);
+                consume(v3);
+            } else {
+                for (int j = 0; 4 * it + j < nvl; ++j) consume(wring[(st * 4 + j) * 32 + lane]);
+            }
+            issue(it + 2);  // refills the slot consumed in the previous iteration
         }
-        for (; c < nvec; c += 32) consume(xr[c]);
+        cp_async_wait<0>();
+        ExactSums e = widen(l);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             e.hi += __shfl_xor_sync(0xFFFFFFFFu, e.hi, o);
@@ -423,42 +490,93 @@ __device__ __forceinline__ uint32_t keep_mask<2>(const float (&v)[kUnit], int n)
     return keep;
 }
 
+// m = 4, n = 2 with n fixed at compile time: an element survives iff it
+// beats at least two of the other three (a before b beats b iff |a| >= |b|).
+// Each comparison is one predicate, each verdict a majority of three (one
+// predicate logic operation), each backbone value one select; returns the
+// keep mask and writes the backbone values to s.
+__device__ __forceinline__ uint32_t select_42(const float (&v)[kUnit], float (&s)[kUnit]) {
+    uint32_t keep = 0;
+#pragma unroll
+    for (int g = 0; g < kUnit / 4; ++g) {
+        const float a0 = v[4 * g], a1 = v[4 * g + 1], a2 = v[4 * g + 2], a3 = v[4 * g + 3];
+        const bool c01 = fabsf(a0) >= fabsf(a1), c02 = fabsf(a0) >= fabsf(a2), c03 = fabsf(a0) >= fabsf(a3);
+        const bool c12 = fabsf(a1) >= fabsf(a2), c13 = fabsf(a1) >= fabsf(a3), c23 = fabsf(a2) >= fabsf(a3);
+        const bool k0 = (c01 & c02) | (c01 & c03) | (c02 & c03);
+        const bool k1 = (!c01 & c12) | (!c01 & c13) | (c12 & c13);
+        const bool k2 = (!c02 & !c12) | (!c02 & c23) | (!c12 & c23);
+        const bool k3 = (!c03 & !c13) | (!c03 & !c23) | (!c13 & !c23);
+        s[4 * g] = k0 ? a0 : 0.0f;
+        s[4 * g + 1] = k1 ? a1 : 0.0f;
+        s[4 * g + 2] = k2 ? a2 : 0.0f;
+        s[4 * g + 3] = k3 ? a3 : 0.0f;
+        keep |= ((uint32_t)k0 | (uint32_t)k1 << 1 | (uint32_t)k2 << 2 | (uint32_t)k3 << 3) << (4 * g);
+    }
+    return keep;
+}
+
+// Step d and scale code of an NVFP4 block as block_step does, with the
+// division a / c6 by the reciprocal method when y6 = RN(1/c6) != 0 (the
+// caller sets y6 = 0 unless c6 is in [2^-90, 2^90]): exact for quotients
+// >= 2^-11, and every smaller quotient has UE4M3 code 0 either way (the
+// code's smallest rounding boundary is 2^-10). MXFP4 takes block_step.
 template <int FMT>
-__device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, float c6, uint32_t &scale_code,
-                                            uint32_t &codes_lo, uint32_t &codes_hi) {
+__device__ __forceinline__ float block_step_rcp(float a, float s_t, float c6, float y6, uint32_t &code) {
+    if (FMT == kFmtNV) {
+        const float u = y6 != 0.0f ? div1(a, c6, y6) : __fdiv_rn(a, c6);
+        code = ue4m3_code(u);
+        return __fmul_rn(ue4m3_value(code), s_t);
+    }
+    return block_step<FMT>(a, s_t, c6, code);
+}
+
+template <int FMT>
+__device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, float c6, float y6,
+                                            uint32_t &scale_code, uint32_t &codes_lo, uint32_t &codes_hi) {
     float a = 0.0f;
 #pragma unroll
     for (int i = 0; i < kUnit; ++i) a = fmaxf(a, fabsf(v[i]));
     if (FMT == kFmtMX) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
-    const float d = block_step<FMT>(a, s_t, c6, scale_code);
-    uint32_t c[2] = {0u, 0u};
+    const float d = block_step_rcp<FMT>(a, s_t, c6, y6, scale_code);
+    codes_lo = 0u;
+    codes_hi = 0u;
     if (d != 0.0f) {
+        // Two halves of eight values each, so that only four quotient pairs
+        // are live at a time.
+        uint32_t c[2];
         if (FMT == kFmtMX) {
             const float inv = pow2f(-mx_exponent(a));  // division by 2^e is this exact product
             const uint64_t y2 = pk2(inv, inv);
 #pragma unroll
-            for (int i = 0; i < kUnit; i += 2) {
-                const uint64_t q = mul2(pk2(v[i], v[i + 1]), y2);
-                c[i / 8] |= e2m1_pair(q, __float_as_uint(v[i]), __float_as_uint(v[i + 1])) << (4 * (i % 8));
+            for (int h = 0; h < 2; ++h) {
+                uint64_t q[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) q[p] = mul2(pk2(v[8 * h + 2 * p], v[8 * h + 2 * p + 1]), y2);
+                c[h] = e2m1x8(q, v + 8 * h);
             }
         } else if (d >= 0x1p-90f && d <= 0x1p90f) {
             const float y = __frcp_rn(d);
             const uint64_t y2 = pk2(y, y), nd2 = pk2(-d, -d), d2 = pk2(d, d);
 #pragma unroll
-            for (int i = 0; i < kUnit; i += 2) {
-                const uint64_t q = div2(pk2(v[i], v[i + 1]), d2, nd2, y2);
-                c[i / 8] |= e2m1_pair(q, __float_as_uint(v[i]), __float_as_uint(v[i + 1])) << (4 * (i % 8));
+            for (int h = 0; h < 2; ++h) {
+                uint64_t q[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) q[p] = div2(pk2(v[8 * h + 2 * p], v[8 * h + 2 * p + 1]), d2, nd2, y2);
+                c[h] = e2m1x8(q, v + 8 * h);
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < kUnit; i += 2) {
-                const uint64_t q = pk2(__fdiv_rn(v[i], d), __fdiv_rn(v[i + 1], d));
-                c[i / 8] |= e2m1_pair(q, __float_as_uint(v[i]), __float_as_uint(v[i + 1])) << (4 * (i % 8));
+            for (int h = 0; h < 2; ++h) {
+                uint64_t q[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+                    q[p] = pk2(__fdiv_rn(v[8 * h + 2 * p], d), __fdiv_rn(v[8 * h + 2 * p + 1], d));
+                c[h] = e2m1x8(q, v + 8 * h);
             }
         }
+        codes_lo = c[0];
+        codes_hi = c[1];
     }
-    codes_lo = c[0];
-    codes_hi = c[1];
     return d;
 }
 
@@ -474,9 +592,10 @@ struct EncodeArgs {
 // Encode step of unit u of row `row`: LayerNorm apply, mask, Q(S), R, Q(R),
 // stores. `active` lanes with row >= m_tok are scale-layout padding (zero
 // scales); inactive lanes only take part in the MXFP4 lane-pair exchanges.
-template <int FMT, int M>
+// NK > 0: n fixed at compile time (the 2:4 default takes its own mask).
+template <int FMT, int M, int NK>
 __device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t *lut, int64_t row, int64_t u,
-                                            bool active, float s_t, float c6) {
+                                            bool active, float s_t, float c6, float y6) {
     constexpr int IB = M <= 2 ? 1 : M <= 4 ? 2 : M <= 8 ? 3 : 4;
     constexpr int G = kUnit / M;  // mask groups per unit
     const uint16_t *__restrict__ x = a.x;
@@ -484,7 +603,7 @@ __device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t 
     const uint16_t *__restrict__ beta = a.beta;
     const float2 *__restrict__ stats = a.stats;
     const int64_t m_tok = a.m_tok, k = a.k, meta_row = a.meta_row, nblk = a.nblk;
-    const int n = a.n;
+    const int n = NK > 0 ? NK : a.n;
     uint8_t *__restrict__ s_codes = a.s_codes;
     uint8_t *__restrict__ r_codes = a.r_codes;
     uint8_t *__restrict__ s_sf = a.s_sf;
@@ -540,14 +659,18 @@ __device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t 
         }
     }
 
-    const uint32_t keep = keep_mask<M>(v, n);
-
-    // Backbone S = X_ln on the mask, +0 elsewhere.
+    // Mask, and the backbone S = X_ln on the mask, +0 elsewhere.
+    uint32_t keep;
     float s[kUnit];
+    if constexpr (M == 4 && NK == 2) {
+        keep = select_42(v, s);
+    } else {
+        keep = keep_mask<M>(v, n);
 #pragma unroll
-    for (int i = 0; i < kUnit; ++i) s[i] = ((keep >> i) & 1u) ? v[i] : 0.0f;
+        for (int i = 0; i < kUnit; ++i) s[i] = ((keep >> i) & 1u) ? v[i] : 0.0f;
+    }
     uint32_t s_scale, s_lo, s_hi;
-    const float ds = quantize16<FMT>(s, s_t, c6, s_scale, s_lo, s_hi);
+    const float ds = quantize16<FMT>(s, s_t, c6, y6, s_scale, s_lo, s_hi);
 
     // Residual against the quantized backbone: R = RN32(X_ln - RN32(value * d)).
     // Scalar intrinsics: the product must be rounded before the subtraction.
@@ -560,7 +683,7 @@ __device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t 
         r[i + 1] = __fsub_rn(v[i + 1], __fmul_rn(cv.y, ds));
     }
     uint32_t r_scale, r_lo, r_hi;
-    quantize16<FMT>(r, s_t, c6, r_scale, r_lo, r_hi);
+    quantize16<FMT>(r, s_t, c6, y6, r_scale, r_lo, r_hi);
 
     // Mask metadata: each group holds exactly n kept positions, so its
     // field sits at a fixed offset of the unit's bit range.
@@ -604,8 +727,8 @@ __device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t 
     }
 }
 
-template <int FMT, int M>
-__global__ void __launch_bounds__(kEncodeThreads)
+template <int FMT, int M, int NK>
+__global__ void __launch_bounds__(kEncodeThreads, SQ_ENCODE_MIN_CTAS)
 prep_encode_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gamma,
                    const uint16_t *__restrict__ beta, const float2 *__restrict__ stats,
                    const unsigned *__restrict__ amax_word, float *__restrict__ s_t_out, int64_t m_tok,
@@ -613,7 +736,6 @@ prep_encode_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ 
                    uint8_t *__restrict__ s_sf, uint8_t *__restrict__ r_sf, uint8_t *__restrict__ meta,
                    int64_t meta_row) {
     constexpr int IB = M <= 2 ? 1 : M <= 4 ? 2 : M <= 8 ? 3 : 4;
-    constexpr int G = kUnit / M;  // mask groups per unit
     __shared__ uint32_t lut[M <= 8 ? (1 << M) : 1];  // keep bits of a group -> kept positions, ascending
     if (M <= 8) {
         for (int msk = threadIdx.x; msk < (1 << M); msk += kEncodeThreads) {
@@ -632,6 +754,7 @@ prep_encode_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ 
     const float amax = __uint_as_float(*amax_word);
     const float s_t = (FMT == kFmtNV && amax != 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
     const float c6 = __fmul_rn(6.0f, s_t);
+    const float y6 = (FMT == kFmtNV && c6 >= 0x1p-90f && c6 <= 0x1p90f) ? __frcp_rn(c6) : 0.0f;
     if (blockIdx.x == 0 && threadIdx.x == 0) *s_t_out = s_t;
 
     const int64_t upr = k / kUnit;                 // units per row
@@ -644,6 +767,7 @@ prep_encode_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ 
     const int64_t t0 = (int64_t)blockIdx.x * kEncodeThreads + threadIdx.x;
     int64_t row_i = t0 / upr, u_i = t0 - (t0 / upr) * upr;
     const int64_t step_rows = stride / upr, step_units = stride - (stride / upr) * upr;
+    EncodeArgs ea{x, gamma, beta, stats, m_tok, k, meta_row, nblk, n, s_codes, r_codes, s_sf, r_sf, meta};
     for (int64_t base = (int64_t)blockIdx.x * kEncodeThreads; base < total; base += stride) {
         const int64_t t = base + threadIdx.x;
         const bool active = t < total;
@@ -654,8 +778,7 @@ prep_encode_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ 
             u_i -= upr;
             ++row_i;
         }
-        EncodeArgs ea{x, gamma, beta, stats, m_tok, k, meta_row, nblk, n, s_codes, r_codes, s_sf, r_sf, meta};
-        encode_unit<FMT, M>(ea, lut, row, u, active, s_t, c6);
+        encode_unit<FMT, M, NK>(ea, lut, row, u, active, s_t, c6, y6);
     }
 }
 
@@ -703,7 +826,7 @@ prep_small_kernel(const EncodeArgs a, float eps, int64_t sf_rows, float *__restr
     const bool affine = a.gamma != nullptr || a.beta != nullptr;
     for (int64_t row = rank; row < m_tok; row += kSmallCtas) {
         const uint4 *xr = reinterpret_cast<const uint4 *>(a.x + row * k);
-        ExactSums e = {0, 0, 0, 0, 0};
+        LaneSums l = {0, 0, 0.0, 0.0, 0.0};
         uint32_t mx = 0xFC00FC00u, mn = 0x7C007C00u;
         // Four loads in flight per thread before any is consumed: one
         // memory round trip per 4 x 512 vectors of the row.
@@ -717,10 +840,10 @@ prep_small_kernel(const EncodeArgs a, float eps, int64_t sf_rows, float *__restr
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 if (c0 + j * kSmallThreads >= nvec) break;
-                accum_pair(v[j].x, e);
-                accum_pair(v[j].y, e);
-                accum_pair(v[j].z, e);
-                accum_pair(v[j].w, e);
+                accum_pair(v[j].x, l);
+                accum_pair(v[j].y, l);
+                accum_pair(v[j].z, l);
+                accum_pair(v[j].w, l);
                 const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -729,6 +852,7 @@ prep_small_kernel(const EncodeArgs a, float eps, int64_t sf_rows, float *__restr
                 }
             }
         }
+        ExactSums e = widen(l);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             e.hi += __shfl_xor_sync(0xFFFFFFFFu, e.hi, o);
@@ -818,6 +942,7 @@ prep_small_kernel(const EncodeArgs a, float eps, int64_t sf_rows, float *__restr
                                                                      (uint32_t)(row % kSmallCtas)))));
     const float s_t = (FMT == kFmtNV && amax != 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
     const float c6 = __fmul_rn(6.0f, s_t);
+    const float y6 = (FMT == kFmtNV && c6 >= 0x1p-90f && c6 <= 0x1p90f) ? __frcp_rn(c6) : 0.0f;
     if (rank == 0 && tid == 0) {
         words[0] = amax;
         words[1] = s_t;
@@ -827,20 +952,21 @@ prep_small_kernel(const EncodeArgs a, float eps, int64_t sf_rows, float *__restr
         const int64_t t = base + tid;
         const bool active = t < total;
         const int64_t row = active ? t / upr : m_tok, u = active ? t - (t / upr) * upr : 0;
-        encode_unit<FMT, M>(a, lut, row, u, active, s_t, c6);
+        encode_unit<FMT, M, 0>(a, lut, row, u, active, s_t, c6, y6);
     }
     cluster_sync();  // no CTA leaves while its row amax may still be read
 }
 
 // ---------------------------------------------------------------------------
-// Division self-test: the packed correction division against the correctly
-// rounded hardware division, on operands drawn from a counter-based hash:
-// random quotients in [2^-4, 2^4], quotients within a few ulps of the E2M1
-// rounding boundaries, and quotients of exponent -30 .. 30; divisors span
-// [2^-90, 2^90]. A mismatch is a quotient of magnitude >= 2^-4 whose bits
-// differ, or any quotient whose E2M1 code differs. (Below 2^-4 the remainder
-// of the method can leave the normal range; such quotients only ever give a
-// zero code, whose sign comes from the dividend.)
+// Division self-test: the packed correction division (and its scalar form)
+// against the correctly rounded hardware division, on operands drawn from a
+// counter-based hash: random quotients in [2^-4, 2^4] and in [2^-11, 2^-4],
+// quotients within a few ulps of the E2M1 and UE4M3 rounding boundaries, and
+// quotients of exponent -30 .. 30; divisors span [2^-90, 2^90]. A mismatch
+// is a quotient of magnitude >= 2^-11 whose bits differ, or any quotient
+// whose E2M1 code (or UE4M3 code of its magnitude) differs. (Far below 2^-11
+// the remainder of the method can leave the normal range; such quotients
+// only ever give a zero code, whose sign comes from the dividend.)
 __device__ unsigned long long g_div_mismatch;
 __device__ float g_div_examples[16][4];  // first mismatches: v, d, quotient, reference
 
@@ -857,7 +983,7 @@ __global__ void div_check_kernel(uint64_t count, uint64_t seed) {
         const int de = (int)(h % 181) - 90;                       // divisor exponent in [-90, 90]
         const float d = __uint_as_float((uint32_t)(de + 127) << 23 | (uint32_t)(g & 0x7FFFFF));
         float v;
-        const int kind = (int)((h >> 40) & 3);
+        const int kind = (int)((h >> 40) % 5);
         if (kind == 0) {  // near an E2M1 rounding boundary
             const float t = ties[(g >> 23) % 7];
             const int ulps = (int)((g >> 30) % 9) - 4;
@@ -865,18 +991,29 @@ __global__ void div_check_kernel(uint64_t count, uint64_t seed) {
         } else if (kind == 1) {  // quotient exponent in [-30, 30]
             const int qe = (int)((g >> 24) % 61) - 30;
             v = __fmul_rn(__uint_as_float((uint32_t)(qe + 127) << 23 | (uint32_t)(h & 0x7FFFFF)), d);
-        } else {  // quotient in [2^-4, 2^4]
+        } else if (kind == 2) {  // quotient in [2^-4, 2^4]
             const int qe = (int)((g >> 24) % 9) - 4;
             v = __fmul_rn(__uint_as_float((uint32_t)(qe + 127) << 23 | (uint32_t)(h & 0x7FFFFF)), d);
+        } else if (kind == 3) {  // quotient in [2^-11, 2^-4]
+            const int qe = (int)((g >> 24) % 7) - 11;
+            v = __fmul_rn(__uint_as_float((uint32_t)(qe + 127) << 23 | (uint32_t)(h & 0x7FFFFF)), d);
+        } else {  // near a UE4M3 rounding boundary (the midpoint of two neighbouring codes)
+            const uint32_t c = (uint32_t)((g >> 23) % 126);
+            const float t = __fmul_rn(__fadd_rn(ue4m3_value(c), ue4m3_value(c + 1)), 0.5f);
+            const int ulps = (int)((g >> 30) % 9) - 4;
+            v = __fmul_rn(__uint_as_float(__float_as_uint(t) + ulps), d);
         }
         if ((g >> 63) & 1) v = -v;
         const float y = __frcp_rn(d);
         const float2 q = up2(div2(pk2(v, v), pk2(d, d), pk2(-d, -d), pk2(y, y)));
         const float ref = __fdiv_rn(v, d);
+        const float q1 = div1(v, d, y);
         const uint32_t sv = __float_as_uint(v);
-        const bool bits_differ = (__float_as_uint(q.x) & 0x7FFFFFFFu) != (__float_as_uint(ref) & 0x7FFFFFFFu);
-        const bool code_differs = (e2m1_pair(pk2(q.x, q.x), sv, sv) & 0xFu) != (e2m1_pair(pk2(ref, ref), sv, sv) & 0xFu);
-        if (ref == ref && ((bits_differ && fabsf(ref) >= 0x1p-4f) || code_differs)) {
+        const bool bits_differ = (__float_as_uint(q.x) & 0x7FFFFFFFu) != (__float_as_uint(ref) & 0x7FFFFFFFu) ||
+                                 (__float_as_uint(q1) & 0x7FFFFFFFu) != (__float_as_uint(ref) & 0x7FFFFFFFu);
+        const bool code_differs = (e2m1_pair(pk2(q.x, q.x), sv, sv) & 0xFu) != (e2m1_pair(pk2(ref, ref), sv, sv) & 0xFu) ||
+                                  ue4m3_code(fabsf(q1)) != ue4m3_code(fabsf(ref));
+        if (ref == ref && ((bits_differ && fabsf(ref) >= 0x1p-11f) || code_differs)) {
             const unsigned long long slot = atomicAdd(&g_div_mismatch, 1ull);
             if (slot < 16) {
                 g_div_examples[slot][0] = v;
@@ -904,13 +1041,38 @@ sharq_status launch_div_check(LaunchCtx &ctx, uint64_t count, uint64_t seed, uin
     return SHARQ_OK;
 }
 
+// Encode grid: every CTA resident at once (SMs x resident CTAs per SM, as
+// the occupancy calculator gives it for the kernel), each looping over units
+// with the grid stride, so that no partial last wave is left.
+static int64_t encode_grid(void *fn, int num_sms, int64_t total_units) {
+    struct Entry {
+        void *fn;
+        int dev, occ;
+    };
+    static Entry cache[64];
+    static int used = 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    int occ = 0;
+    for (int i = 0; i < used; ++i)
+        if (cache[i].fn == fn && cache[i].dev == dev) occ = cache[i].occ;
+    if (occ == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kEncodeThreads, 0) != cudaSuccess || occ < 1)
+            occ = 1;
+        if (used < 64) cache[used++] = Entry{fn, dev, occ};
+    }
+    const int64_t blocks = (total_units + kEncodeThreads - 1) / kEncodeThreads;
+    const int64_t cap = (int64_t)num_sms * occ;
+    return blocks < cap ? blocks : cap;
+}
+
 template <int FMT>
-static void *encode_fn(int m) {
+static void *encode_fn(int m, int n) {
     switch (m) {
-        case 2: return (void *)prep_encode_kernel<FMT, 2>;
-        case 4: return (void *)prep_encode_kernel<FMT, 4>;
-        case 8: return (void *)prep_encode_kernel<FMT, 8>;
-        default: return (void *)prep_encode_kernel<FMT, 16>;
+        case 2: return (void *)prep_encode_kernel<FMT, 2, 0>;
+        case 4: return n == 2 ? (void *)prep_encode_kernel<FMT, 4, 2> : (void *)prep_encode_kernel<FMT, 4, 0>;
+        case 8: return (void *)prep_encode_kernel<FMT, 8, 0>;
+        default: return (void *)prep_encode_kernel<FMT, 16, 0>;
     }
 }
 
@@ -1058,9 +1220,8 @@ extern "C" sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, 
                                                                            eps, k, stats, amax_word);
     }
     const int64_t total = P.sf_rows * (k / kUnit);
-    int64_t blocks = (total + kEncodeThreads - 1) / kEncodeThreads;
-    if (blocks > (int64_t)sms[dev] * 16) blocks = (int64_t)sms[dev] * 16;
-    void *fn = fmt == kFmtNV ? encode_fn<kFmtNV>(m) : encode_fn<kFmtMX>(m);
+    void *fn = fmt == kFmtNV ? encode_fn<kFmtNV>(m, n) : encode_fn<kFmtMX>(m, n);
+    const int64_t blocks = encode_grid(fn, sms[dev], total);
     const uint16_t *xx = (const uint16_t *)x_dev, *gg = (const uint16_t *)ln_w_dev, *bb = (const uint16_t *)ln_b_dev;
     const float2 *cst = stats;
     const unsigned *aw = amax_word;
@@ -1092,6 +1253,10 @@ static sharq_status launch_stats(LaunchCtx &ctx, const sharq_prep &P, const void
     if (!attr_done[dev]) {
         SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_kernel<true, RMS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)(2 * SHARQ_K_MAX)));
+        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<true, RMS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kStatsRingBytes));
+        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<false, RMS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
         attr_done[dev] = true;
     }
     if (P.m_tok == 0) return SHARQ_OK;
@@ -1100,10 +1265,10 @@ static sharq_status launch_stats(LaunchCtx &ctx, const sharq_prep &P, const void
     if (warp_rows) {
         const unsigned grid = (unsigned)((P.m_tok + kStatsThreads / 32 - 1) / (kStatsThreads / 32));
         if (gamma || beta)
-            ln_stats_warp_kernel<true, RMS><<<grid, kStatsThreads, 0, ctx.stream>>>(xx, gg, bb, eps, P.k, P.m_tok,
+            ln_stats_warp_kernel<true, RMS><<<grid, kStatsThreads, kStatsRingBytes, ctx.stream>>>(xx, gg, bb, eps, P.k, P.m_tok,
                                                                                    stats, words);
         else
-            ln_stats_warp_kernel<false, RMS><<<grid, kStatsThreads, 0, ctx.stream>>>(xx, nullptr, nullptr, eps, P.k,
+            ln_stats_warp_kernel<false, RMS><<<grid, kStatsThreads, kStatsRingBytes, ctx.stream>>>(xx, nullptr, nullptr, eps, P.k,
                                                                                     P.m_tok, stats, words);
     } else {
         if (gamma || beta)
@@ -1135,10 +1300,8 @@ sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, 
                                   : launch_stats<false>(ctx, P, x, gamma, beta, eps, stats, words);
     if (sst != SHARQ_OK) return sst;
     const int64_t total = P.sf_rows * (P.k / kUnit);
-    int64_t blocks = (total + kEncodeThreads - 1) / kEncodeThreads;
-    const int64_t cap = (int64_t)ctx.num_sms * 16;
-    if (blocks > cap) blocks = cap;
-    void *fn = P.fmt == kFmtNV ? encode_fn<kFmtNV>(P.m) : encode_fn<kFmtMX>(P.m);
+    void *fn = P.fmt == kFmtNV ? encode_fn<kFmtNV>(P.m, P.n) : encode_fn<kFmtMX>(P.m, P.n);
+    const int64_t blocks = encode_grid(fn, ctx.num_sms, total);
     const uint16_t *xx = (const uint16_t *)x, *gg = (const uint16_t *)gamma, *bb = (const uint16_t *)beta;
     const float2 *cst = stats;
     const unsigned *aw = words;

@@ -163,8 +163,8 @@ __device__ __forceinline__ uint64_t h2_to_f2(uint32_t w) {
 }
 
 // Correctly rounded quotients v / d of a packed pair, for d in [2^-90, 2^90]
-// with y = RN(1/d) and |v / d| >= 2^-4 (smaller quotients come out within an
-// ulp, which is all E2M1 encoding needs there). Markstein's correction (P. Markstein, "Computation of
+// with y = RN(1/d) and |v / d| >= 2^-11 (smaller quotients come out within
+// an ulp, which is all E2M1 and UE4M3 encoding need there). Markstein's correction (P. Markstein, "Computation of
 // elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
 // Dev. 34(1), 1990): q0 = RN(v y); one FMA residual step makes the quotient
 // faithful; with the remainder r = v - d q1 then exact, RN(q1 + r y) is the
@@ -176,6 +176,42 @@ __device__ __forceinline__ uint64_t div2(uint64_t v, uint64_t d2, uint64_t nd2, 
     q = fma2(r, y2, q);
     r = fma2(q, nd2, v);
     return fma2(r, y2, q);
+}
+
+// The same correctly rounded quotient for one value (v / d, y = RN(1/d),
+// d in [2^-90, 2^90], |v / d| >= 2^-11). The remainder v - d q1 is then a
+// multiple of ulp(q1) ulp(d) >= 2^-147, hence exact even below the normal
+// range.
+__device__ __forceinline__ float div1(float v, float d, float y) {
+    float q = __fmul_rn(v, y);
+    float r = __fmaf_rn(q, -d, v);
+    q = __fmaf_rn(r, y, q);
+    r = __fmaf_rn(q, -d, v);
+    return __fmaf_rn(r, y, q);
+}
+
+// E2M1 codes of eight quotients (four packed pairs) as one word, lowest
+// nibble first, rounded to nearest even with saturation to 6. Each quotient
+// first takes the sign bit of its dividend (sv: bit patterns), as in
+// e2m1_pair below.
+__device__ __forceinline__ uint32_t e2m1x8(const uint64_t *q, const float *sv) {
+    float f[8];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float2 t = up2(q[p]);
+        f[2 * p] = __uint_as_float(__float_as_uint(t.x) | (__float_as_uint(sv[2 * p]) & 0x80000000u));
+        f[2 * p + 1] = __uint_as_float(__float_as_uint(t.y) | (__float_as_uint(sv[2 * p + 1]) & 0x80000000u));
+    }
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(f[0]), "f"(f[1]), "f"(f[2]), "f"(f[3]), "f"(f[4]), "f"(f[5]), "f"(f[6]), "f"(f[7]));
+    return r;
 }
 
 // E2M1 byte of two quotients (lo nibble = q.x), rounded to nearest even with
@@ -198,6 +234,18 @@ __device__ __forceinline__ uint32_t e2m1_pair(uint64_t q, uint32_t sign_lo, uint
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// Per-thread asynchronous 16-byte copies global -> shared (L2 only), grouped
+// by commit; wait_group<N> returns once at most N of this thread's groups are
+// still in flight, after which the thread may read what it copied.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
