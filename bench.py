@@ -568,6 +568,8 @@ def run_case(args, world, rank, local):
         return run_sweep(args)
     if kind == "vendor_fp4":
         return run_vendor_fp4(args)
+    if kind == "fused":
+        return run_fused(args, nums[0] if nums else 8192)
     if kind == "prep":
         M, K = nums[:2]
         fmt, n, m = (nums[2:5] + [0, N_KEEP, M_GROUP][len(nums[2:5]):])
@@ -613,6 +615,75 @@ def run_case(args, world, rank, local):
     return {"case": args.case, "ms_median": t * 1e3, "ms_min": min(ms), "achieved": achieved, "unit": unit,
             "peak": peak, "frac": achieved / peak, "bound": bound, "steps": args.steps,
             "outlier_frac": args.outlier_frac, "peak_source": peak_src}
+
+
+def fused_linears(ls):
+    """The layer set's linears grouped by the activation they read (q/k/v,
+    o, gate/up, down): one fused linear per group, in order."""
+    groups = []
+    for lin in ls.linears:
+        if groups and groups[-1][0].prep == lin.prep:
+            groups[-1].append(lin)
+        else:
+            groups.append([lin])
+    return groups
+
+
+def run_fused(args, M):
+    """The layer-set step with the linears that share an input fused (q/k/v
+    into one weight, gate/up into one; each segment keeps its own tensor
+    scale, so the outputs equal the separate linears'): 4 preps + 4 linears,
+    timed like the default step. Per-linear event times included."""
+    import sparsity_gemm_b200 as sq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ls, preps = layer_set()
+    prep_index = {name: i for i, (name, _) in enumerate(preps)}
+    groups = fused_linears(ls)
+    xs = [torch.from_numpy(synth.activations_student(i, M, k).view(np.float16)).to(dev)
+          for i, (_, k) in enumerate(preps)]
+    lin_index = {lin.name: j for j, lin in enumerate(ls.linears)}
+    qws = []
+    for g in groups:
+        ws = [torch.from_numpy(synth.weights(1000 + lin_index[l.name], l.n_out, l.k).view(np.float16)).to(dev)
+              for l in g]
+        qws.append(sq.quantize_weight_fused(ws, sq.NVFP4) if len(ws) > 1 else sq.quantize_weight(ws[0], sq.NVFP4))
+        del ws
+    bufs = [sq.prepare(xs[i], None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4) for i in range(len(preps))]
+    outs = [torch.empty((M, q.n_out), dtype=torch.float16, device=dev) for q in qws]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    n_ev = 1 + len(preps) + len(groups)
+
+    def step(ev=None):
+        for i in range(len(preps)):
+            bufs[i] = sq.prepare(xs[i], None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4, out=bufs[i])
+            if ev is not None:
+                ev[1 + i].record(stream)
+        for j, g in enumerate(groups):
+            sq.linear(bufs[prep_index[g[0].prep]], qws[j], out=outs[j])
+            if ev is not None:
+                ev[1 + len(preps) + j].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    for s in range(args.steps):
+        flush.zero_()
+        events[s][0].record(stream)
+        step(events[s])
+    torch.cuda.synchronize()
+    st = sq.get_last_error()
+    if st != sq.OK:
+        raise RuntimeError(sq.status_name(st))
+    prep_ms = sum(ev[i].elapsed_time(ev[i + 1]) for ev in events for i in range(len(preps))) / args.steps
+    each = [sum(ev[len(preps) + j].elapsed_time(ev[len(preps) + j + 1]) for ev in events) / args.steps
+            for j in range(len(groups))]
+    total = prep_ms + sum(each)
+    return {"case": args.case, "tokens_per_s": M / (total / 1e3), "ms_per_step": total, "prep_ms": prep_ms,
+            "gemm_ms": sum(each), "gemm_each": {"+".join(l.name for l in g): each[j] for j, g in enumerate(groups)},
+            "steps": args.steps}
 
 
 def run_sweep(args):

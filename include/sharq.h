@@ -63,6 +63,8 @@ typedef enum sharq_status {
 #define SHARQ_K_ALIGN 256
 #define SHARQ_K_MAX 65536
 #define SHARQ_N_ALIGN 32
+/* Most segments of a fused weight (sharq_quantize_weight_fused). */
+#define SHARQ_SEGMENTS_MAX 8
 
 /*
  * Block-scale layout ("MMA scale view"). Scales of a [rows][k/blk] matrix
@@ -103,8 +105,12 @@ typedef struct sharq_wq {
     void *codes;         /* device, [n_out][k/2] bytes */
     void *scales_backbone; /* device, MMA scale view for the backbone path */
     void *scales_residual; /* device, MMA scale view for the residual path */
-    float *tensor_scale; /* device, 1 float: s_tW = amax(W)/2688 (NVFP4) or 1 */
+    float *tensor_scale; /* device, 1 float: s_tW = amax(W)/2688 (NVFP4) or 1;
+                            one float per segment for a fused weight */
     void *scratch;       /* device, library-internal words */
+    int32_t segments;    /* fused weights: stacked segments along n_out, 1 (0
+                            reads as 1) otherwise */
+    int32_t seg_end[SHARQ_SEGMENTS_MAX]; /* exclusive end row of each segment */
 } sharq_wq;
 
 /* Prepared activation: outputs of the preparation operator. */
@@ -253,6 +259,45 @@ sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, int64_t k,
  */
 sharq_status sharq_linear(const sharq_prep *prep, const sharq_wq *wq, void *out_dev,
                           void *stream);
+
+/*
+ * Fused projections: weights that read the same prepared activation (q, k
+ * and v of attention; gate and up of a gated MLP), stacked along n_out into
+ * one payload so that one linear computes all of them. An interface
+ * addition: the SharQ abstract describes one linear at a time. Each segment
+ * is quantized on its own (its own tensor scale s_tW[g], block scales and
+ * codes exactly as sharq_quantize_weight gives for that weight alone), so
+ * every output column of the fused linear equals the column of the separate
+ * linear bit for bit.
+ *   w_dev     fp16 [sum seg_rows][k], the segments' rows one after another.
+ *   seg_rows  host array of n_segs row counts, each >= 1 and a multiple of
+ *             SHARQ_N_ALIGN; 1 <= n_segs <= SHARQ_SEGMENTS_MAX.
+ *   wq_dev    device buffer of at least sharq_weight_bytes_fused(...) bytes
+ *             (the same as sharq_weight_bytes of the stacked shape).
+ * wq_out describes one weight of n_out = sum seg_rows rows with
+ * segments = n_segs, seg_end[g] = rows of segments 0..g, and tensor_scale
+ * pointing at n_segs floats.
+ */
+size_t sharq_weight_bytes_fused(const int64_t *seg_rows, int n_segs, int64_t k, int fmt);
+sharq_status sharq_quantize_weight_fused(const void *w_dev, const int64_t *seg_rows, int n_segs, int64_t k,
+                                         int fmt, void *wq_dev, size_t wq_bytes, sharq_wq *wq_out,
+                                         void *stream);
+
+/*
+ * The dual-path linear with a bias (Qwen2.5's q, k and v projections have
+ * one): column j of segment g is
+ *     out = RN16( RN32( RN32(acc * RN32(s_t * s_tW[g])) + bias[j] ) )
+ * with acc the fp32 accumulator of sharq_linear. bias_dev: fp16 [n_out],
+ * 16-byte aligned, or NULL (then the result equals sharq_linear's).
+ * sharq_linear accepts fused weights too (no bias). Preconditions as
+ * sharq_linear.
+ */
+sharq_status sharq_linear_bias(const sharq_prep *prep, const sharq_wq *wq, const void *bias_dev, void *out_dev,
+                               void *stream);
+
+/* The tensor scales of a weight's segments (one float each) to the host.
+ * Synchronizes `stream`. s_tw_host holds at least wq->segments floats. */
+sharq_status sharq_weight_tensor_scales(const sharq_wq *wq, float *s_tw_host, void *stream);
 
 /*
  * Mixture-of-experts grouped variant.

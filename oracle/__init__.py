@@ -316,3 +316,33 @@ def linear_grouped(p: Prepared, row_idx, offsets, qws: list, sel=None, cols=None
                       p.s_t, qw.codes[cols], qw.scales[cols], qw.s_tw, p.fmt)
         out[j], bound[j] = o[0], b[0]
     return out, bound
+
+
+# --------------------------------------------------------------------------
+# Fused projections and bias. An interface addition: the SharQ abstract
+# describes one linear at a time. Reading: a fused weight is its segments
+# (q, k, v or gate, up), each quantized on its own with its own tensor
+# scale, and the fused output is the segments' outputs side by side. The
+# bias (Qwen2.5's q/k/v projections have one) is added after the scaled
+# accumulator: out = RN16(RN32(RN32(acc * s_t * s_tW) + b)); here the exact
+# fp64 dual-path value plus b.
+
+
+def quantize_weight_fused(ws, fmt: int) -> list:
+    """One QWeight per segment of a fused weight."""
+    return [quantize_weight(w, fmt) for w in ws]
+
+
+def linear_fused(p: Prepared, qws: list, bias=None, rows=None):
+    """fp64 output of a fused linear (segments side by side) plus the bias
+    (fp16 [n_out] or None), and the tolerance scale: the dual-path bound
+    plus |bias|, which bounds |output| and so the final fp16 rounding."""
+    parts = [linear_prepared(p, q, rows) for q in qws]
+    out = np.concatenate([o for o, _ in parts], axis=1)
+    bound = np.concatenate([b for _, b in parts], axis=1)
+    if bias is not None:
+        b = np.asarray(bias, np.float16).astype(np.float64)
+        assert b.shape == (out.shape[1],)
+        out = out + b[None, :]
+        bound = bound + np.abs(b)[None, :]
+    return out, bound

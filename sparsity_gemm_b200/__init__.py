@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libsharq.so")
 NVFP4, MXFP4 = 0, 1
 BLOCK = {NVFP4: 16, MXFP4: 32}
 K_ALIGN, K_MAX, N_ALIGN = 256, 65536, 32
+SEGMENTS_MAX = 8
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
 
@@ -36,7 +37,8 @@ class SharqError(RuntimeError):
 class SharqWQ(C.Structure):
     _fields_ = [("n_out", C.c_int64), ("k", C.c_int64), ("fmt", C.c_int32), ("groups", C.c_int32),
                 ("sf_rows", C.c_int64), ("codes", C.c_void_p), ("scales_backbone", C.c_void_p),
-                ("scales_residual", C.c_void_p), ("tensor_scale", C.c_void_p), ("scratch", C.c_void_p)]
+                ("scales_residual", C.c_void_p), ("tensor_scale", C.c_void_p), ("scratch", C.c_void_p),
+                ("segments", C.c_int32), ("seg_end", C.c_int32 * SEGMENTS_MAX)]
 
 
 class SharqPrep(C.Structure):
@@ -85,12 +87,19 @@ def lib():
         L.sharq_gather_bytes.restype = sz
         L.sharq_gather_rows.argtypes = [C.POINTER(SharqPrep), vp, vp, i64, i64, vp, sz, C.POINTER(SharqPrep), vp]
         L.sharq_linear_grouped.argtypes = [C.POINTER(SharqPrep), vp, i64, i64, C.POINTER(SharqWQ), vp, vp]
+        L.sharq_weight_bytes_fused.argtypes = [C.POINTER(C.c_int64), i32, i64, i32]
+        L.sharq_weight_bytes_fused.restype = sz
+        L.sharq_quantize_weight_fused.argtypes = [vp, C.POINTER(C.c_int64), i32, i64, i32, vp, sz,
+                                                  C.POINTER(SharqWQ), vp]
+        L.sharq_linear_bias.argtypes = [C.POINTER(SharqPrep), C.POINTER(SharqWQ), vp, vp, vp]
+        L.sharq_weight_tensor_scales.argtypes = [C.POINTER(SharqWQ), vp, vp]
         L.sharq_status_string.argtypes = [i32]
         L.sharq_status_string.restype = C.c_char_p
         L.sharq_last_launch_count.restype = i32
         for name in ("sharq_quantize_weight", "sharq_prepare", "sharq_linear", "sharq_prep_export",
                      "sharq_weight_export", "sharq_get_last_error", "sharq_quantize_weight_grouped",
-                     "sharq_gather_rows", "sharq_linear_grouped", "sharq_prepare_rms"):
+                     "sharq_gather_rows", "sharq_linear_grouped", "sharq_prepare_rms",
+                     "sharq_quantize_weight_fused", "sharq_linear_bias", "sharq_weight_tensor_scales"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -194,13 +203,53 @@ def prepare(x: torch.Tensor, ln_w=None, ln_b=None, eps: float = 1e-5, n: int = 2
     return Prepared(buf, desc)
 
 
-def linear(prep: Prepared, qw: QuantizedWeight, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Dual-path FP4 linear: fp16 [m_tok, n_out] = (Q(S) + Q(R)) Q(W)^T, scaled."""
+def linear(prep: Prepared, qw: QuantizedWeight, out: torch.Tensor | None = None, stream=None,
+           bias: torch.Tensor | None = None) -> torch.Tensor:
+    """Dual-path FP4 linear: fp16 [m_tok, n_out] = (Q(S) + Q(R)) Q(W)^T, scaled,
+    plus an optional fp16 bias [n_out]. A fused weight (quantize_weight_fused)
+    gives its segments' outputs side by side."""
     if out is None:
         out = torch.empty((prep.m_tok, qw.n_out), dtype=torch.float16, device=prep.buf.device)
     assert out.dtype == torch.float16 and out.is_contiguous() and tuple(out.shape) == (prep.m_tok, qw.n_out)
     optr = _ptr(out) if out.numel() else None
-    _check(lib().sharq_linear(C.byref(prep.desc), C.byref(qw.desc), optr, _stream(stream)), "sharq_linear")
+    if bias is None:
+        _check(lib().sharq_linear(C.byref(prep.desc), C.byref(qw.desc), optr, _stream(stream)), "sharq_linear")
+    else:
+        assert bias.dtype == torch.float16 and bias.is_cuda and bias.is_contiguous() and bias.numel() == qw.n_out
+        _check(lib().sharq_linear_bias(C.byref(prep.desc), C.byref(qw.desc), _ptr(bias), optr, _stream(stream)),
+               "sharq_linear_bias")
+    return out
+
+
+def quantize_weight_fused(ws, fmt: int = NVFP4, stream=None) -> QuantizedWeight:
+    """Offline FP4 quantization of several weights that read the same input
+    (q/k/v, gate/up), stacked along n_out into one payload; each keeps its own
+    tensor scale, so the fused linear's columns equal the separate linears'.
+    ws: list of fp16 CUDA tensors [n_g, k]."""
+    ws = list(ws)
+    assert ws and all(w.dtype == torch.float16 and w.is_cuda and w.dim() == 2 for w in ws)
+    k = ws[0].shape[1]
+    assert all(w.shape[1] == k for w in ws)
+    rows = (C.c_int64 * len(ws))(*[w.shape[0] for w in ws])
+    nbytes = int(lib().sharq_weight_bytes_fused(rows, len(ws), k, fmt))
+    if nbytes == 0:
+        raise SharqError(ERR_INVALID_ARG, f"fused weight segments {[tuple(w.shape) for w in ws]} fmt {fmt}")
+    w = torch.cat([t.contiguous() for t in ws], 0)
+    buf = _device_buffer(nbytes, w.device)
+    desc = SharqWQ()
+    _check(lib().sharq_quantize_weight_fused(_ptr(w), rows, len(ws), k, fmt, _ptr(buf), nbytes, C.byref(desc),
+                                             _stream(stream)), "sharq_quantize_weight_fused")
+    qw = QuantizedWeight(buf, desc)
+    qw._src = w  # the stacked copy stays alive until the quantizer has read it
+    return qw
+
+
+def weight_tensor_scales(qw: QuantizedWeight, stream=None) -> np.ndarray:
+    """The tensor scale s_tW of each segment of a weight (one for a plain weight)."""
+    segs = max(1, qw.desc.segments)
+    out = np.zeros(segs, np.float32)
+    _check(lib().sharq_weight_tensor_scales(C.byref(qw.desc), out.ctypes.data_as(C.c_void_p), _stream(stream)),
+           "sharq_weight_tensor_scales")
     return out
 
 

@@ -20,6 +20,7 @@ FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "-O3", "-std=c++17", "-fmad=false",
     "-Xcompiler", "-fPIC", "-shared",
+    "-Xcompiler", "-Werror=return-type", "--diag-error=940",  # a missing return is an error
     "-cudart", "shared",
     "-Xlinker", "-rpath=/usr/local/cuda/lib64",
 ]

@@ -76,6 +76,23 @@ void fill_wq(sharq_wq *W, void *buf, int64_t n_out, int64_t k, int fmt) {
     W->scales_residual = b + L.scales;  // same values in the same MMA layout
     W->scratch = b + L.words;
     W->tensor_scale = reinterpret_cast<float *>(b + L.words) + 1;
+    W->segments = 1;
+    W->seg_end[0] = (int32_t)n_out;
+}
+
+// Segments of a weight descriptor: 1..SHARQ_SEGMENTS_MAX, ends increasing,
+// multiples of SHARQ_N_ALIGN, the last one n_out.
+static bool segments_ok(const sharq_wq *wq) {
+    const int s = wq->segments > 1 ? wq->segments : 1;
+    if (s > SHARQ_SEGMENTS_MAX) return false;
+    if (s == 1) return true;
+    int64_t prev = 0;
+    for (int g = 0; g < s; ++g) {
+        const int64_t e = wq->seg_end[g];
+        if (e <= prev || e % SHARQ_N_ALIGN != 0) return false;
+        prev = e;
+    }
+    return prev == wq->n_out && wq->groups <= 1;
 }
 
 void unpack_codes(const std::vector<uint8_t> &packed, int64_t count, uint8_t *dst) {
@@ -173,8 +190,14 @@ sharq_status sharq_prepare_rms(const void *x_dev, int64_t m_tok, int64_t k, cons
 }
 
 sharq_status sharq_linear(const sharq_prep *prep, const sharq_wq *wq, void *out_dev, void *stream) {
+    return sharq_linear_bias(prep, wq, nullptr, out_dev, stream);
+}
+
+sharq_status sharq_linear_bias(const sharq_prep *prep, const sharq_wq *wq, const void *bias_dev, void *out_dev,
+                               void *stream) {
     g_last_launches = 0;
     if (!prep || !wq) return SHARQ_ERR_INVALID_ARG;
+    if (!segments_ok(wq) || (bias_dev && !aligned(bias_dev, 16))) return SHARQ_ERR_INVALID_ARG;
     if (!fmt_ok(prep->fmt) || prep->fmt != wq->fmt || prep->k != wq->k || !k_ok(prep->k)) return SHARQ_ERR_INVALID_ARG;
     if (wq->n_out < 1 || wq->n_out % SHARQ_N_ALIGN != 0 || prep->m_tok < 0) return SHARQ_ERR_INVALID_ARG;
     if (wq->groups > 1) return SHARQ_ERR_INVALID_ARG;  // stacked weights: sharq_linear_grouped
@@ -189,9 +212,56 @@ sharq_status sharq_linear(const sharq_prep *prep, const sharq_wq *wq, void *out_
     sq::LaunchCtx ctx;
     sharq_status st = make_ctx(stream, ctx);
     if (st != SHARQ_OK) return st;
-    st = sq::launch_linear(ctx, *prep, *wq, out_dev);
+    st = sq::launch_linear(ctx, *prep, *wq, bias_dev, out_dev);
     g_last_launches = ctx.launches;
     return st;
+}
+
+static int64_t fused_rows(const int64_t *seg_rows, int n_segs) {
+    if (!seg_rows || n_segs < 1 || n_segs > SHARQ_SEGMENTS_MAX) return -1;
+    int64_t total = 0;
+    for (int g = 0; g < n_segs; ++g) {
+        if (seg_rows[g] < 1 || seg_rows[g] % SHARQ_N_ALIGN != 0 || seg_rows[g] > (1ll << 30)) return -1;
+        total += seg_rows[g];
+    }
+    return total <= (1ll << 30) ? total : -1;
+}
+
+size_t sharq_weight_bytes_fused(const int64_t *seg_rows, int n_segs, int64_t k, int fmt) {
+    const int64_t total = fused_rows(seg_rows, n_segs);
+    return total < 0 ? 0 : sharq_weight_bytes(total, k, fmt);
+}
+
+sharq_status sharq_quantize_weight_fused(const void *w_dev, const int64_t *seg_rows, int n_segs, int64_t k, int fmt,
+                                         void *wq_dev, size_t wq_bytes, sharq_wq *wq_out, void *stream) {
+    g_last_launches = 0;
+    const size_t need = sharq_weight_bytes_fused(seg_rows, n_segs, k, fmt);
+    if (!need || !w_dev || !wq_dev || !wq_out || wq_bytes < need) return SHARQ_ERR_INVALID_ARG;
+    if (!aligned(w_dev, 16) || !aligned(wq_dev, sq::kAlign)) return SHARQ_ERR_INVALID_ARG;
+    sq::LaunchCtx ctx;
+    sharq_status st = make_ctx(stream, ctx);
+    if (st != SHARQ_OK) return st;
+    const int64_t total = fused_rows(seg_rows, n_segs);
+    fill_wq(wq_out, wq_dev, total, k, fmt);
+    wq_out->segments = n_segs;
+    int64_t end = 0;
+    for (int g = 0; g < n_segs; ++g) {
+        end += seg_rows[g];
+        wq_out->seg_end[g] = (int32_t)end;
+    }
+    st = sq::launch_quantize_weight_fused(ctx, *wq_out, w_dev, seg_rows, n_segs);
+    g_last_launches = ctx.launches;
+    return st;
+}
+
+sharq_status sharq_weight_tensor_scales(const sharq_wq *wq, float *s_tw_host, void *stream) {
+    if (!wq || !s_tw_host || !wq->tensor_scale || !segments_ok(wq)) return SHARQ_ERR_INVALID_ARG;
+    const int segs = wq->segments > 1 ? wq->segments : 1;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SHARQ_ERR_CUDA;
+    if (cudaMemcpy(s_tw_host, wq->tensor_scale, sizeof(float) * (size_t)segs, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SHARQ_ERR_CUDA;
+    return SHARQ_OK;
 }
 
 size_t sharq_weight_bytes_grouped(int64_t n_groups, int64_t n_out, int64_t k, int fmt) {
@@ -260,7 +330,8 @@ sharq_status sharq_linear_grouped(const sharq_prep *prep, const int32_t *offsets
     g_last_launches = 0;
     if (!prep || !wq || !offsets_dev || !aligned(offsets_dev, 4)) return SHARQ_ERR_INVALID_ARG;
     if (!fmt_ok(prep->fmt) || prep->fmt != wq->fmt || prep->k != wq->k || !k_ok(prep->k)) return SHARQ_ERR_INVALID_ARG;
-    if (n_groups < 1 || n_groups > sq::kGroupsMax || prep->groups != n_groups || wq->groups != n_groups)
+    if (n_groups < 1 || n_groups > sq::kGroupsMax || prep->groups != n_groups || wq->groups != n_groups ||
+        wq->segments > 1)
         return SHARQ_ERR_INVALID_ARG;
     if (wq->n_out < 1 || wq->n_out % SHARQ_N_ALIGN != 0 || rows < 0 || rows > prep->m_tok)
         return SHARQ_ERR_INVALID_ARG;

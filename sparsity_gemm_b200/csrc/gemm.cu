@@ -114,7 +114,22 @@ struct GemmParams {
     // tile, each over a K range, and reduce through distributed shared
     // memory; 1 = no split.
     int32_t split;
+    // dense launches only: fused weights (segs > 1: column j of segment g,
+    // seg_end[g-1] <= j < seg_end[g], takes s_tw[g]; boundaries are
+    // multiples of 32 columns) and an optional fp16 bias per column
+    int32_t segs;
+    int32_t seg_end[SHARQ_SEGMENTS_MAX];
+    const __half *bias;
 };
+
+// alpha = RN32(s_t * s_tW[g]) of the segment holding column `col`.
+__device__ __forceinline__ float alpha_of_col(const GemmParams &p, float s_t, float alpha0, int col) {
+    if (p.segs <= 1) return alpha0;
+    int g = 0;
+#pragma unroll 1
+    for (int i = 0; i + 1 < p.segs; ++i) g += col >= p.seg_end[i] ? 1 : 0;
+    return __fmul_rn(s_t, p.s_tw[g]);
+}
 
 // Instruction descriptor of the block-scaled MMA (M = 128, N = 256, E2M1 x
 // E2M1, K-major A and B): A/B format E2M1 at bits 7-9 / 10-12, N >> 3 at
@@ -144,7 +159,9 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 // rows; tile table in shared memory), W is a stack of `groups` weights read
 // through a 3-D tensor map (K bytes, n_out, group), each group with its own
 // tensor scale, and output rows are remapped to grouped-row order.
-template <int FMT, bool GROUPED>
+// EXT (dense only): fused-weight segments and/or a bias in the epilogue; the
+// plain instantiation keeps the epilogue without them.
+template <int FMT, bool GROUPED, bool EXT>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constant__ CUtensorMap tm_ar,
                  const __grid_constant__ CUtensorMap tm_b, const GemmParams p) {
@@ -404,19 +421,44 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                 break;  // one tile per CTA
             }
             // out = RN16(RN32(acc * alpha)) (packed multiplies round each
-            // product to fp32 before the conversion).
+            // product to fp32 before the conversion); with a bias,
+            // RN16(RN32(RN32(acc * alpha) + bias)) in scalar operations, so
+            // that no multiply is fused into the add. Fused weights: alpha
+            // per 32-column chunk (a chunk never spans two segments).
             uint32_t h[kBN / 32][16];
-            const uint64_t alpha2 = pk2(alpha, alpha);
 #pragma unroll
             for (int cc = 0; cc < kBN / 32; ++cc) {
+                const int col0 = nb * kBN + cc * 32;
+                float a_cc = alpha;
+                if constexpr (EXT) a_cc = alpha_of_col(p, s_t, alpha, col0);
                 uint32_t r[32];
                 tmem_ld32(tmem + lane_base + (uint32_t)(cc * 32), r);
                 tmem_ld_wait();
+                if (EXT && p.bias != nullptr && col0 < p.n_out) {
+                    const uint4 *bp = reinterpret_cast<const uint4 *>(p.bias + col0);  // same for every lane
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float2 f = up2(mul2(pk2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), alpha2));
-                    __half2 v = __floats2half2_rn(f.x, f.y);
-                    h[cc][i] = *reinterpret_cast<uint32_t *>(&v);
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        const uint4 bw = __ldg(bp + v4);
+                        const uint32_t bb[4] = {bw.x, bw.y, bw.z, bw.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const int i = 4 * v4 + j;
+                            const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&bb[j]));
+                            const float y0 = __fadd_rn(__fmul_rn(__uint_as_float(r[2 * i]), a_cc), b.x);
+                            const float y1 = __fadd_rn(__fmul_rn(__uint_as_float(r[2 * i + 1]), a_cc), b.y);
+                            __half2 v = __floats2half2_rn(y0, y1);
+                            h[cc][i] = *reinterpret_cast<uint32_t *>(&v);
+                        }
+                    }
+                } else {
+                    const uint64_t alpha2 = pk2(a_cc, a_cc);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 f =
+                            up2(mul2(pk2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), alpha2));
+                        __half2 v = __floats2half2_rn(f.x, f.y);
+                        h[cc][i] = *reinterpret_cast<uint32_t *>(&v);
+                    }
                 }
             }
             tc_fence_before();
@@ -464,10 +506,12 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             const int mb = tile_begin / n_tiles, nb = tile_begin % n_tiles;
             const int S = p.split, cols = kBN / S, groups4 = cols / 4;
             const int valid = (int)min((int64_t)kBM, (int64_t)p.m_tok - (int64_t)mb * kBM);
-            const float alpha = __fmul_rn(*p.s_t, *p.s_tw);
+            const float s_t = *p.s_t;
+            const float alpha0 = __fmul_rn(s_t, *p.s_tw);
             for (int item = (warp - 2) * 32 + lane; item < valid * groups4; item += 128) {
                 const int r = item / groups4, col = rank * cols + (item % groups4) * 4;
                 if (nb * kBN + col >= p.n_out) continue;
+                const float alpha = EXT ? alpha_of_col(p, s_t, alpha0, nb * kBN + col) : alpha0;
                 const uint32_t off = sbase + (uint32_t)r * kPartStride + (uint32_t)col * 4u;
                 float4 acc = ld_cluster_f4(mapa_shared(off, 0));
                 for (int c = 1; c < S; ++c) {
@@ -477,8 +521,17 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                     acc.z = __fadd_rn(acc.z, v.z);
                     acc.w = __fadd_rn(acc.w, v.w);
                 }
-                __half2 h0 = __floats2half2_rn(__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha));
-                __half2 h1 = __floats2half2_rn(__fmul_rn(acc.z, alpha), __fmul_rn(acc.w, alpha));
+                float4 y = make_float4(__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha), __fmul_rn(acc.z, alpha),
+                                       __fmul_rn(acc.w, alpha));
+                if (EXT && p.bias != nullptr) {
+                    const uint2 bw = *reinterpret_cast<const uint2 *>(p.bias + nb * kBN + col);
+                    const float2 b01 = __half22float2(*reinterpret_cast<const __half2 *>(&bw.x));
+                    const float2 b23 = __half22float2(*reinterpret_cast<const __half2 *>(&bw.y));
+                    y = make_float4(__fadd_rn(y.x, b01.x), __fadd_rn(y.y, b01.y), __fadd_rn(y.z, b23.x),
+                                    __fadd_rn(y.w, b23.y));
+                }
+                __half2 h0 = __floats2half2_rn(y.x, y.y);
+                __half2 h1 = __floats2half2_rn(y.z, y.w);
                 *reinterpret_cast<uint2 *>(p.out + ((int64_t)mb * kBM + r) * p.n_out + nb * kBN + col) =
                     make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
             }
@@ -565,37 +618,37 @@ static bool make_grouped_code_map(CUtensorMap *tm, const void *base, uint64_t ro
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, bool GROUPED>
+template <int FMT, bool GROUPED, bool EXT>
 static sharq_status set_gemm_attrs() {
     static bool attr_done[64] = {};
     int dev = 0;
     SQ_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
     if (!attr_done[dev]) {
-        SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<FMT, GROUPED>,
+        SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<FMT, GROUPED, EXT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes));
         attr_done[dev] = true;
     }
     return SHARQ_OK;
 }
 
-template <int FMT, bool GROUPED>
+template <int FMT, bool GROUPED, bool EXT>
 static sharq_status launch_gemm(LaunchCtx &ctx, const CUtensorMap &tm_as, const CUtensorMap &tm_ar,
                                 const CUtensorMap &tm_b, const GemmParams &gp, int64_t max_tiles) {
-    sharq_status st = set_gemm_attrs<FMT, GROUPED>();
+    sharq_status st = set_gemm_attrs<FMT, GROUPED, EXT>();
     if (st != SHARQ_OK) return st;
     const unsigned grid = (unsigned)(max_tiles < ctx.num_sms ? max_tiles : ctx.num_sms);
-    dual_gemm_kernel<FMT, GROUPED><<<grid, kGemmThreads, kSmemBytes, ctx.stream>>>(tm_as, tm_ar, tm_b, gp);
+    dual_gemm_kernel<FMT, GROUPED, EXT><<<grid, kGemmThreads, kSmemBytes, ctx.stream>>>(tm_as, tm_ar, tm_b, gp);
     ctx.launches++;
     SQ_CUDA_TRY(cudaGetLastError());
     return SHARQ_OK;
 }
 
 // Split-K launch: `tiles` clusters of gp.split CTAs, one tile per cluster.
-template <int FMT>
+template <int FMT, bool EXT>
 static sharq_status launch_gemm_split(LaunchCtx &ctx, const CUtensorMap &tm_as, const CUtensorMap &tm_ar,
                                       const CUtensorMap &tm_b, const GemmParams &gp, int64_t tiles) {
-    sharq_status st = set_gemm_attrs<FMT, false>();
+    sharq_status st = set_gemm_attrs<FMT, false, EXT>();
     if (st != SHARQ_OK) return st;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
@@ -610,7 +663,7 @@ static sharq_status launch_gemm_split(LaunchCtx &ctx, const CUtensorMap &tm_as, 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    SQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, dual_gemm_kernel<FMT, false>, tm_as, tm_ar, tm_b, gp));
+    SQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, dual_gemm_kernel<FMT, false, EXT>, tm_as, tm_ar, tm_b, gp));
     ctx.launches++;
     SQ_CUDA_TRY(cudaGetLastError());
     return SHARQ_OK;
@@ -625,7 +678,7 @@ static int active_clusters(int split) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || split > kMaxSplit) return 0;
     if (!known[dev][split]) {
-        if (set_gemm_attrs<FMT, false>() != SHARQ_OK) return 0;
+        if (set_gemm_attrs<FMT, false, false>() != SHARQ_OK) return 0;
         cudaLaunchConfig_t cfg;
         memset(&cfg, 0, sizeof(cfg));
         cfg.gridDim = dim3((unsigned)split, 1, 1);
@@ -639,7 +692,7 @@ static int active_clusters(int split) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, dual_gemm_kernel<FMT, false>, &cfg) != cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&n, dual_gemm_kernel<FMT, false, false>, &cfg) != cudaSuccess) {
             cudaGetLastError();
             n = 0;
         }
@@ -675,10 +728,13 @@ static GemmParams gemm_params(LaunchCtx &ctx, const sharq_prep &P, const sharq_w
     gp.status = ctx.status;
     gp.wait_ns = ctx.wait_ns;
     gp.split = 1;
+    gp.segs = W.segments > 1 ? W.segments : 1;
+    for (int g = 0; g < gp.segs && g < SHARQ_SEGMENTS_MAX; ++g) gp.seg_end[g] = W.seg_end[g];
+    gp.bias = nullptr;
     return gp;
 }
 
-sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, void *out) {
+sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, const void *bias, void *out) {
     if (P.m_tok == 0) return SHARQ_OK;
     CUtensorMap tm_as, tm_ar, tm_b;
     if (!make_code_map(&tm_as, P.s_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
@@ -686,14 +742,24 @@ sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &
         !make_code_map(&tm_b, W.codes, (uint64_t)(W.k / 2), (uint64_t)W.n_out, kBN))
         return SHARQ_ERR_CUDA;
     GemmParams gp = gemm_params(ctx, P, W, out);
+    gp.bias = (const __half *)bias;
     const int64_t tiles = ((P.m_tok + kBM - 1) / kBM) * ((W.n_out + kBN - 1) / kBN);
     const int kt_count = (int)(P.k / (2 * kBKBytes));
     gp.split = P.fmt == kFmtNV ? choose_split<kFmtNV>(ctx, tiles, kt_count) : choose_split<kFmtMX>(ctx, tiles, kt_count);
-    if (gp.split > 1)
-        return P.fmt == kFmtNV ? launch_gemm_split<kFmtNV>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
-                               : launch_gemm_split<kFmtMX>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
-    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
-                           : launch_gemm<kFmtMX, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
+    // the extended epilogue (fused segments, bias) only where needed
+    const bool ext = gp.bias != nullptr || gp.segs > 1;
+    if (gp.split > 1) {
+        if (ext)
+            return P.fmt == kFmtNV ? launch_gemm_split<kFmtNV, true>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
+                                   : launch_gemm_split<kFmtMX, true>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
+        return P.fmt == kFmtNV ? launch_gemm_split<kFmtNV, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
+                               : launch_gemm_split<kFmtMX, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
+    }
+    if (ext)
+        return P.fmt == kFmtNV ? launch_gemm<kFmtNV, false, true>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
+                               : launch_gemm<kFmtMX, false, true>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
+    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, false, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
+                           : launch_gemm<kFmtMX, false, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
 }
 
 sharq_status launch_linear_grouped(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, const int32_t *offsets,
@@ -705,6 +771,7 @@ sharq_status launch_linear_grouped(LaunchCtx &ctx, const sharq_prep &P, const sh
                                (uint64_t)w_gstride, kBN))
         return SHARQ_ERR_CUDA;
     GemmParams gp = gemm_params(ctx, P, W, out);
+    gp.segs = 1;  // stacked experts, never fused segments
     gp.offsets = offsets;
     gp.groups = groups;
     gp.rows = rows;
@@ -712,8 +779,8 @@ sharq_status launch_linear_grouped(LaunchCtx &ctx, const sharq_prep &P, const sh
     // at most P.m_tok / 128 m tiles (the device checks the offsets against it)
     const int64_t tiles = (P.m_tok / kBM) * ((W.n_out + kBN - 1) / kBN);
     if (tiles == 0) return SHARQ_OK;
-    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, true>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
-                           : launch_gemm<kFmtMX, true>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
+    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, true, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
+                           : launch_gemm<kFmtMX, true, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
 }
 
 }  // namespace sq

@@ -20,7 +20,10 @@ sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, 
                             const void *beta, float eps, int norm);
 sharq_status launch_quantize_weight(LaunchCtx &ctx, const sharq_wq &W, const void *w, int64_t groups,
                                    int64_t gstride);
-sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, void *out);
+sharq_status launch_quantize_weight_fused(LaunchCtx &ctx, const sharq_wq &W, const void *w, const int64_t *seg_rows,
+                                         int n_segs);
+// bias: fp16 [n_out] or NULL
+sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, const void *bias, void *out);
 sharq_status launch_linear_grouped(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, const int32_t *offsets,
                                    int32_t groups, int64_t rows, int64_t w_gstride, void *out);
 sharq_status launch_gather(LaunchCtx &ctx, const sharq_prep &S, const int32_t *row_idx, const int32_t *offsets,

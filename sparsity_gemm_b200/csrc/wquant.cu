@@ -51,11 +51,14 @@ __global__ void __launch_bounds__(kWThreads) absmax_kernel(const uint16_t *__res
     }
 }
 
+// Rows [0, sf_rows) of one weight (rows >= n_out are scale-layout padding),
+// written at rows row0 + r of the code and scale layouts (row0 > 0: a
+// segment of a fused weight).
 template <int FMT>
 __global__ void __launch_bounds__(kWThreads)
 wq_encode_kernel(const uint16_t *__restrict__ w, int64_t n_out, int64_t sf_rows, int64_t k,
                  const unsigned *__restrict__ amax_word, float *__restrict__ s_tw_out, uint8_t *__restrict__ codes,
-                 uint8_t *__restrict__ sf, int64_t gstride) {
+                 uint8_t *__restrict__ sf, int64_t gstride, int64_t row0) {
     constexpr int BLK = FMT == kFmtNV ? 16 : 32;
     {
         const int64_t gofs = (int64_t)blockIdx.y * gstride;
@@ -72,10 +75,10 @@ wq_encode_kernel(const uint16_t *__restrict__ w, int64_t n_out, int64_t sf_rows,
     if (blockIdx.x == 0 && threadIdx.x == 0) *s_tw_out = s_t;
     const int64_t cpr = k / 32, nblk = k / BLK, total = sf_rows * cpr;
     for (int64_t t = (int64_t)blockIdx.x * kWThreads + threadIdx.x; t < total; t += (int64_t)gridDim.x * kWThreads) {
-        const int64_t row = t / cpr, c = t - row * cpr;
+        const int64_t row = t / cpr, c = t - row * cpr, orow = row0 + row;
         if (row >= n_out) {  // scale-layout padding rows
-            if (FMT == kFmtNV) *reinterpret_cast<uint16_t *>(sf + sf_offset(row, 2 * c, nblk)) = 0;
-            else sf[sf_offset(row, c, nblk)] = 0;
+            if (FMT == kFmtNV) *reinterpret_cast<uint16_t *>(sf + sf_offset(orow, 2 * c, nblk)) = 0;
+            else sf[sf_offset(orow, c, nblk)] = 0;
             continue;
         }
         const uint4 *wp = reinterpret_cast<const uint4 *>(w + row * k + c * 32);
@@ -102,9 +105,9 @@ wq_encode_kernel(const uint16_t *__restrict__ w, int64_t n_out, int64_t sf_rows,
                     pk[i / 8] |= e2m1x2(__fdiv_rn(v[i], d), __fdiv_rn(v[i + 1], d)) << (4 * (i % 8));
             }
         }
-        *reinterpret_cast<uint4 *>(codes + row * (k / 2) + c * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        if (FMT == kFmtNV) *reinterpret_cast<uint16_t *>(sf + sf_offset(row, 2 * c, nblk)) = (uint16_t)(sc[0] | (sc[NB - 1] << 8));
-        else sf[sf_offset(row, c, nblk)] = (uint8_t)sc[0];
+        *reinterpret_cast<uint4 *>(codes + orow * (k / 2) + c * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        if (FMT == kFmtNV) *reinterpret_cast<uint16_t *>(sf + sf_offset(orow, 2 * c, nblk)) = (uint16_t)(sc[0] | (sc[NB - 1] << 8));
+        else sf[sf_offset(orow, c, nblk)] = (uint8_t)sc[0];
     }
 }
 
@@ -128,12 +131,48 @@ sharq_status launch_quantize_weight(LaunchCtx &ctx, const sharq_wq &W, const voi
     if (W.fmt == kFmtNV)
         wq_encode_kernel<kFmtNV><<<ge, kWThreads, 0, ctx.stream>>>(
             (const uint16_t *)w, W.n_out, W.sf_rows, W.k, words, W.tensor_scale, (uint8_t *)W.codes,
-            (uint8_t *)W.scales_backbone, gstride);
+            (uint8_t *)W.scales_backbone, gstride, 0);
     else
         wq_encode_kernel<kFmtMX><<<ge, kWThreads, 0, ctx.stream>>>(
             (const uint16_t *)w, W.n_out, W.sf_rows, W.k, words, W.tensor_scale, (uint8_t *)W.codes,
-            (uint8_t *)W.scales_backbone, gstride);
+            (uint8_t *)W.scales_backbone, gstride, 0);
     ctx.launches++;
+    SQ_CUDA_TRY(cudaGetLastError());
+    return SHARQ_OK;
+}
+
+// Fused weight: segment g (rows seg_rows[g], after the earlier segments'
+// rows) is quantized on its own, with its amax in word 0 (g = 0) or 8 + g of
+// the weight's words and its tensor scale in tensor_scale[g] (words 1 + g);
+// the last segment also zeroes the scale-layout padding rows.
+sharq_status launch_quantize_weight_fused(LaunchCtx &ctx, const sharq_wq &W, const void *w, const int64_t *seg_rows,
+                                         int n_segs) {
+    unsigned *words = reinterpret_cast<unsigned *>(W.tensor_scale) - 1;
+    SQ_CUDA_TRY(cudaMemsetAsync(words, 0, 16 * sizeof(unsigned), ctx.stream));
+    int64_t off = 0;
+    for (int g = 0; g < n_segs; ++g) {
+        const int64_t rows = seg_rows[g];
+        unsigned *aw = g == 0 ? words : words + 8 + g;
+        const uint16_t *wg = (const uint16_t *)w + off * W.k;
+        const int64_t count = rows * W.k;
+        int64_t blocks = (count / 8 + kWThreads - 1) / kWThreads;
+        if (blocks > (int64_t)ctx.num_sms * 4) blocks = (int64_t)ctx.num_sms * 4;
+        absmax_kernel<<<(unsigned)blocks, kWThreads, 0, ctx.stream>>>(wg, count, aw, 0);
+        ctx.launches++;
+        const int64_t iter_rows = g + 1 == n_segs ? W.sf_rows - off : rows;
+        int64_t eb = (iter_rows * (W.k / 32) + kWThreads - 1) / kWThreads;
+        if (eb > (int64_t)ctx.num_sms * 8) eb = (int64_t)ctx.num_sms * 8;
+        if (W.fmt == kFmtNV)
+            wq_encode_kernel<kFmtNV><<<(unsigned)eb, kWThreads, 0, ctx.stream>>>(
+                wg, rows, iter_rows, W.k, aw, W.tensor_scale + g, (uint8_t *)W.codes, (uint8_t *)W.scales_backbone, 0,
+                off);
+        else
+            wq_encode_kernel<kFmtMX><<<(unsigned)eb, kWThreads, 0, ctx.stream>>>(
+                wg, rows, iter_rows, W.k, aw, W.tensor_scale + g, (uint8_t *)W.codes, (uint8_t *)W.scales_backbone, 0,
+                off);
+        ctx.launches++;
+        off += rows;
+    }
     SQ_CUDA_TRY(cudaGetLastError());
     return SHARQ_OK;
 }

@@ -145,6 +145,40 @@ def test_linear_rejects_mismatched_handles_without_cuda(sq):
     assert L.sharq_linear(C.byref(p), C.byref(w), None, None) == sq.OK
 
 
+def test_fused_weights_and_bias_validation_without_cuda(sq):
+    L = sq.lib()
+    rows = lambda *r: (C.c_int64 * len(r))(*r)
+    assert L.sharq_weight_bytes_fused(rows(4096, 1024, 1024), 3, 4096, 0) == sq.weight_bytes(6144, 4096, 0)
+    assert L.sharq_weight_bytes_fused(rows(64, 48), 2, 256, 0) == 0          # 48 is not a multiple of 32
+    assert L.sharq_weight_bytes_fused(rows(64, 0), 2, 256, 0) == 0
+    assert L.sharq_weight_bytes_fused(rows(*([32] * 9)), 9, 256, 0) == 0     # more than SHARQ_SEGMENTS_MAX
+    assert L.sharq_weight_bytes_fused(None, 1, 256, 0) == 0
+    desc = sq.SharqWQ()
+    assert L.sharq_quantize_weight_fused(C.c_void_p(1 << 20), rows(64, 48), 2, 256, 0, C.c_void_p(1 << 21),
+                                         1 << 20, C.byref(desc), None) == sq.ERR_INVALID_ARG
+    p = sq.SharqPrep(m_tok=16, k=256, n=2, m=4, fmt=0, sf_rows=128, meta_row_bytes=32,
+                     s_codes=1 << 20, r_codes=1 << 21)
+    w = sq.SharqWQ(n_out=256, k=256, fmt=0, sf_rows=256, codes=1 << 22, scales_backbone=1 << 23,
+                   scales_residual=1 << 23)
+    out = C.c_void_p(1 << 24)
+    w.segments = 2
+    w.seg_end[0], w.seg_end[1] = 128, 200   # the last segment must end at n_out
+    assert L.sharq_linear(C.byref(p), C.byref(w), out, None) == sq.ERR_INVALID_ARG
+    w.seg_end[0], w.seg_end[1] = 100, 256   # boundaries are multiples of 32
+    assert L.sharq_linear(C.byref(p), C.byref(w), out, None) == sq.ERR_INVALID_ARG
+    w.seg_end[0], w.seg_end[1] = 256, 256   # strictly increasing
+    assert L.sharq_linear(C.byref(p), C.byref(w), out, None) == sq.ERR_INVALID_ARG
+    w.segments = 9
+    assert L.sharq_linear(C.byref(p), C.byref(w), out, None) == sq.ERR_INVALID_ARG
+    w.segments = 1
+    # the bias must be 16-byte aligned
+    assert L.sharq_linear_bias(C.byref(p), C.byref(w), C.c_void_p((1 << 25) + 8), out, None) == sq.ERR_INVALID_ARG
+    w.segments, w.groups = 2, 2
+    w.seg_end[0], w.seg_end[1] = 128, 256   # stacked experts cannot also be fused
+    assert L.sharq_linear_grouped(C.byref(p), C.c_void_p(1 << 26), 2, 16, C.byref(w), out,
+                                  None) == sq.ERR_INVALID_ARG
+
+
 def test_status_strings(sq):
     assert sq.status_name(0) == "SHARQ_OK"
     assert sq.status_name(4) == "SHARQ_ERR_TIMEOUT"
