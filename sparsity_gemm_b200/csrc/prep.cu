@@ -251,36 +251,50 @@ ln_stats_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gam
 }
 
 // Warp per row (rows of at most kWarpRowMaxK elements, or any row length
-// when the rows fill the GPU): eight rows per CTA, the statistics reduced with
-// shuffles only, and one atomic per CTA for the tensor's amax (one CTA per row
-// leaves most threads idle on short rows and puts one atomic per row on a
-// single word). Same exact sums, so the results equal those of
+// when the rows fill the GPU): eight warps per CTA, the statistics reduced
+// with shuffles only, and one atomic per CTA for the tensor's amax (one CTA
+// per row leaves most threads idle on short rows and puts one atomic per row
+// on a single word). Same exact sums, so the results equal those of
 // ln_stats_kernel bit for bit. The row streams through a ring of
 // kStatsStages slots per lane (four 16-byte vectors each) filled by
 // asynchronous copies issued two iterations ahead, so that loads stay in
-// flight while the lane computes. With gamma/beta the row is read a second
-// time (from L2) for amax|X_ln|.
+// flight while the lane computes.
+// Without gamma/beta, each warp takes `rpw` consecutive rows and leaves
+// each row's reduced sums in shared memory; once all warps are done, one
+// thread per row finishes the statistics (the binary64 divisions and the
+// 128-bit products run on 8 * rpw threads at once instead of one lane per
+// warp and row, which dominated on short rows). With gamma/beta (rpw = 1)
+// lane 0 finishes each row at once and the warp reads the row a second time
+// (from L2) for amax|X_ln|.
 constexpr int64_t kWarpRowMaxK = 8192;
 constexpr int kStatsStages = 3;
 constexpr int kStatsRingBytes = (kStatsThreads / 32) * kStatsStages * 4 * 32 * 16;  // 48 KB
+constexpr int kStatsMaxRpw = 4;  // rows per warp, short rows
 
 template <bool AFFINE, bool RMS>
 __global__ void __launch_bounds__(kStatsThreads)
 ln_stats_warp_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gamma,
-                     const uint16_t *__restrict__ beta, float eps, int64_t k, int64_t m_tok,
+                     const uint16_t *__restrict__ beta, float eps, int64_t k, int64_t m_tok, int rpw,
                      float2 *__restrict__ stats, unsigned *__restrict__ amax_word) {
+    constexpr int W = kStatsThreads / 32;
     extern __shared__ uint4 ring[];  // [warp][stage][vector j][lane]
-    __shared__ float red_max[kStatsThreads / 32];
+    __shared__ float red_max[W];
+    __shared__ ExactSums rsum[AFFINE ? 1 : W * kStatsMaxRpw];
+    __shared__ uint32_t rmx[AFFINE ? 1 : W * kStatsMaxRpw], rmn[AFFINE ? 1 : W * kStatsMaxRpw];
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int64_t row = (int64_t)blockIdx.x * (kStatsThreads / 32) + warp;
+    if (AFFINE) rpw = 1;
+    const int64_t cta_row0 = (int64_t)blockIdx.x * W * rpw;
+    const int nvec = (int)(k / 8);
+    const int nvl = nvec / 32;        // vectors per lane (k is a multiple of 256)
+    const int iters = (nvl + 3) / 4;  // four vectors per lane per iteration
+    uint4 *wring = ring + (size_t)warp * kStatsStages * 4 * 32;
+    const uint32_t wbase = smem_u32(wring);
     float amax = 0.0f;
-    if (row < m_tok) {
-        const int nvec = (int)(k / 8);
-        const int nvl = nvec / 32;           // vectors per lane (k is a multiple of 256)
-        const int iters = (nvl + 3) / 4;     // four vectors per lane per iteration
+    for (int i = 0; i < rpw; ++i) {
+        const int slot = warp * rpw + i;
+        const int64_t row = cta_row0 + slot;
+        if (row >= m_tok) break;  // warp-uniform
         const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * k);
-        uint4 *wring = ring + (size_t)warp * kStatsStages * 4 * 32;
-        const uint32_t wbase = smem_u32(wring);
         auto issue = [&](int it) {
             if (it < iters) {
                 const int st = it % kStatsStages;
@@ -339,6 +353,14 @@ ln_stats_warp_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
                 asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(omn));
             }
         }
+        if (!AFFINE) {
+            if (lane == 0) {
+                rsum[slot] = e;
+                rmx[slot] = mx;
+                rmn[slot] = mn;
+            }
+            continue;
+        }
         float2 st = make_float2(0.0f, 0.0f);
         if (lane == 0) {
             st = RMS ? finish_stats_rms(e, k, eps) : finish_stats(e, k, eps);
@@ -346,38 +368,45 @@ ln_stats_warp_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
         }
         st.x = __shfl_sync(0xFFFFFFFFu, st.x, 0);
         st.y = __shfl_sync(0xFFFFFFFFu, st.y, 0);
-        if (!AFFINE) {
+        const bool has_g = gamma != nullptr, has_b = beta != nullptr;
+        for (int cc = lane; cc < nvec; cc += 32) {
+            const uint4 v = xr[cc];
+            const uint4 g = has_g ? __ldg(reinterpret_cast<const uint4 *>(gamma) + cc) : make_uint4(0, 0, 0, 0);
+            const uint4 bb = has_b ? __ldg(reinterpret_cast<const uint4 *>(beta) + cc) : make_uint4(0, 0, 0, 0);
+            const uint32_t xv[4] = {v.x, v.y, v.z, v.w}, gv[4] = {g.x, g.y, g.z, g.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float xl = ln_apply(h2f((uint16_t)(xv[q] >> (16 * h))), st.x, st.y, has_g,
+                                              h2f((uint16_t)(gv[q] >> (16 * h))), has_b,
+                                              h2f((uint16_t)(bv[q] >> (16 * h))));
+                    amax = fmaxf(amax, fabsf(xl));
+                }
+        }
+    }
+    if (!AFFINE) {
+        __syncthreads();  // every row's sums are in shared memory
+        const int slot = threadIdx.x;
+        const int64_t row = cta_row0 + slot;
+        if (slot < W * rpw && row < m_tok) {
+            const float2 st = RMS ? finish_stats_rms(rsum[slot], k, eps) : finish_stats(rsum[slot], k, eps);
+            stats[row] = st;
             // X_ln = RN(RN(x - mu) * rstd) is non-decreasing in x: the row's
             // amax|X_ln| is reached at its smallest or largest x.
+            const uint32_t mx = rmx[slot], mn = rmn[slot];
             const float xmax = fmaxf(h2f((uint16_t)mx), h2f((uint16_t)(mx >> 16)));
             const float xmin = fminf(h2f((uint16_t)mn), h2f((uint16_t)(mn >> 16)));
             amax = fmaxf(fabsf(__fmul_rn(__fsub_rn(xmax, st.x), st.y)), fabsf(__fmul_rn(__fsub_rn(xmin, st.x), st.y)));
-        } else {
-            const bool has_g = gamma != nullptr, has_b = beta != nullptr;
-            for (int cc = lane; cc < nvec; cc += 32) {
-                const uint4 v = xr[cc];
-                const uint4 g = has_g ? __ldg(reinterpret_cast<const uint4 *>(gamma) + cc) : make_uint4(0, 0, 0, 0);
-                const uint4 bb = has_b ? __ldg(reinterpret_cast<const uint4 *>(beta) + cc) : make_uint4(0, 0, 0, 0);
-                const uint32_t xv[4] = {v.x, v.y, v.z, v.w}, gv[4] = {g.x, g.y, g.z, g.w}, bv[4] = {bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const float xl = ln_apply(h2f((uint16_t)(xv[q] >> (16 * h))), st.x, st.y, has_g,
-                                                  h2f((uint16_t)(gv[q] >> (16 * h))), has_b,
-                                                  h2f((uint16_t)(bv[q] >> (16 * h))));
-                        amax = fmaxf(amax, fabsf(xl));
-                    }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
         }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
     if (lane == 0) red_max[warp] = amax;
     __syncthreads();
     if (threadIdx.x == 0) {
         float a = 0.0f;
-        for (int w = 0; w < kStatsThreads / 32; ++w) a = fmaxf(a, red_max[w]);
+        for (int w = 0; w < W; ++w) a = fmaxf(a, red_max[w]);
         atomicMax(amax_word, __float_as_uint(a));  // non-negative floats order like their bits
     }
 }
@@ -491,26 +520,24 @@ __device__ __forceinline__ uint32_t keep_mask<2>(const float (&v)[kUnit], int n)
 }
 
 // m = 4, n = 2 with n fixed at compile time: an element survives iff it
-// beats at least two of the other three (a before b beats b iff |a| >= |b|).
-// Each comparison is one predicate, each verdict a majority of three (one
-// predicate logic operation), each backbone value one select; returns the
-// keep mask and writes the backbone values to s.
-__device__ __forceinline__ uint32_t select_42(const float (&v)[kUnit], float (&s)[kUnit]) {
+// beats at least two of the other three. For a before b in the group, the
+// sign of RN(|a| - |b|) is set iff |a| < |b| (equal magnitudes give +0),
+// i.e. iff b beats a; each verdict is a majority of three such signs, one
+// three-input logic operation on the bit patterns. (Measured on B200: fewer
+// instructions than comparisons into predicates and predicate logic.)
+__device__ __forceinline__ uint32_t keep_mask_42(const float (&v)[kUnit]) {
     uint32_t keep = 0;
 #pragma unroll
     for (int g = 0; g < kUnit / 4; ++g) {
-        const float a0 = v[4 * g], a1 = v[4 * g + 1], a2 = v[4 * g + 2], a3 = v[4 * g + 3];
-        const bool c01 = fabsf(a0) >= fabsf(a1), c02 = fabsf(a0) >= fabsf(a2), c03 = fabsf(a0) >= fabsf(a3);
-        const bool c12 = fabsf(a1) >= fabsf(a2), c13 = fabsf(a1) >= fabsf(a3), c23 = fabsf(a2) >= fabsf(a3);
-        const bool k0 = (c01 & c02) | (c01 & c03) | (c02 & c03);
-        const bool k1 = (!c01 & c12) | (!c01 & c13) | (c12 & c13);
-        const bool k2 = (!c02 & !c12) | (!c02 & c23) | (!c12 & c23);
-        const bool k3 = (!c03 & !c13) | (!c03 & !c23) | (!c13 & !c23);
-        s[4 * g] = k0 ? a0 : 0.0f;
-        s[4 * g + 1] = k1 ? a1 : 0.0f;
-        s[4 * g + 2] = k2 ? a2 : 0.0f;
-        s[4 * g + 3] = k3 ? a3 : 0.0f;
-        keep |= ((uint32_t)k0 | (uint32_t)k1 << 1 | (uint32_t)k2 << 2 | (uint32_t)k3 << 3) << (4 * g);
+        const float a0 = fabsf(v[4 * g]), a1 = fabsf(v[4 * g + 1]), a2 = fabsf(v[4 * g + 2]), a3 = fabsf(v[4 * g + 3]);
+        const uint32_t s01 = __float_as_uint(__fsub_rn(a0, a1)), s02 = __float_as_uint(__fsub_rn(a0, a2));
+        const uint32_t s03 = __float_as_uint(__fsub_rn(a0, a3)), s12 = __float_as_uint(__fsub_rn(a1, a2));
+        const uint32_t s13 = __float_as_uint(__fsub_rn(a1, a3)), s23 = __float_as_uint(__fsub_rn(a2, a3));
+        const uint32_t k0 = ~((s01 & s02) | (s01 & s03) | (s02 & s03));
+        const uint32_t k1 = (s01 & ~s12) | (s01 & ~s13) | (~s12 & ~s13);
+        const uint32_t k2 = (s02 & s12) | (s02 & ~s23) | (s12 & ~s23);
+        const uint32_t k3 = (s03 & s13) | (s03 & s23) | (s13 & s23);
+        keep |= ((k0 >> 31) | (k1 >> 31) << 1 | (k2 >> 31) << 2 | (k3 >> 31) << 3) << (4 * g);
     }
     return keep;
 }
@@ -662,13 +689,12 @@ __device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t 
     // Mask, and the backbone S = X_ln on the mask, +0 elsewhere.
     uint32_t keep;
     float s[kUnit];
-    if constexpr (M == 4 && NK == 2) {
-        keep = select_42(v, s);
-    } else {
+    if constexpr (M == 4 && NK == 2)
+        keep = keep_mask_42(v);
+    else
         keep = keep_mask<M>(v, n);
 #pragma unroll
-        for (int i = 0; i < kUnit; ++i) s[i] = ((keep >> i) & 1u) ? v[i] : 0.0f;
-    }
+    for (int i = 0; i < kUnit; ++i) s[i] = ((keep >> i) & 1u) ? v[i] : 0.0f;
     uint32_t s_scale, s_lo, s_hi;
     const float ds = quantize16<FMT>(s, s_t, c6, y6, s_scale, s_lo, s_hi);
 
@@ -1263,13 +1289,21 @@ static sharq_status launch_stats(LaunchCtx &ctx, const sharq_prep &P, const void
     const bool warp_rows = P.m_tok >= (int64_t)ctx.num_sms * (kStatsThreads / 32) || P.k <= kWarpRowMaxK;
     const uint16_t *xx = (const uint16_t *)x, *gg = (const uint16_t *)gamma, *bb = (const uint16_t *)beta;
     if (warp_rows) {
-        const unsigned grid = (unsigned)((P.m_tok + kStatsThreads / 32 - 1) / (kStatsThreads / 32));
+        // Short rows and rows enough for 16 warps per SM: several rows per
+        // warp, so that the per-row finish runs on many threads at once.
+        int rpw = 1;
+        if (!(gamma || beta) && P.k <= 2048) {
+            const int64_t r = P.m_tok / ((int64_t)ctx.num_sms * 16);
+            rpw = (int)(r < 1 ? 1 : (r > kStatsMaxRpw ? kStatsMaxRpw : r));
+        }
+        const int64_t per_cta = (int64_t)(kStatsThreads / 32) * rpw;
+        const unsigned grid = (unsigned)((P.m_tok + per_cta - 1) / per_cta);
         if (gamma || beta)
-            ln_stats_warp_kernel<true, RMS><<<grid, kStatsThreads, kStatsRingBytes, ctx.stream>>>(xx, gg, bb, eps, P.k, P.m_tok,
-                                                                                   stats, words);
+            ln_stats_warp_kernel<true, RMS><<<grid, kStatsThreads, kStatsRingBytes, ctx.stream>>>(
+                xx, gg, bb, eps, P.k, P.m_tok, 1, stats, words);
         else
-            ln_stats_warp_kernel<false, RMS><<<grid, kStatsThreads, kStatsRingBytes, ctx.stream>>>(xx, nullptr, nullptr, eps, P.k,
-                                                                                    P.m_tok, stats, words);
+            ln_stats_warp_kernel<false, RMS><<<grid, kStatsThreads, kStatsRingBytes, ctx.stream>>>(
+                xx, nullptr, nullptr, eps, P.k, P.m_tok, rpw, stats, words);
     } else {
         if (gamma || beta)
             ln_stats_kernel<true, RMS><<<(unsigned)P.m_tok, kStatsThreads, (size_t)(2 * P.k), ctx.stream>>>(

@@ -68,6 +68,19 @@ def test_prepare_bit_exact(m_tok, k, fmt, n, m, affine):
     assert_prep_matches(ex, op)
 
 
+@pytest.mark.parametrize("m_tok,k,fmt,norm", [(5000, 256, 0, "layer"), (10007, 512, 1, "layer"),
+                                               (9500, 768, 0, "rms")])
+def test_prepare_many_short_rows_bit_exact(m_tok, k, fmt, norm):
+    """Rows enough for several rows per statistics warp (their sums finished
+    together after all warps are done), with a ragged last CTA: every row's
+    statistics and every code and scale bit-exact."""
+    import sparsity_gemm_b200 as sq
+    x = synth.activations_student(700 + m_tok, m_tok, k)
+    op = oracle.prepare(x, None, None, 1e-5, 2, 4, fmt, norm=norm)
+    p = sq.prepare(cuda16(x), None, None, 1e-5, 2, 4, fmt, norm=norm)
+    assert_prep_matches(sq.prep_export(p), op)
+
+
 @pytest.mark.parametrize("n_out,k,fmt", [(32, 256, 0), (544, 512, 0), (544, 512, 1), (256, 1024, 1)])
 def test_weight_quantization_bit_exact(n_out, k, fmt):
     import sparsity_gemm_b200 as sq
