@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # one ncu capture of the current dual_gemm_kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum of the layer-set launch list). Set to None whenever
 # the kernel changes until it is captured again.
-GEMM_TRAFFIC_BYTES_PER_STEP_M8192 = 1039.5e6
+GEMM_TRAFFIC_BYTES_PER_STEP_M8192 = 1019.0e6
 
 
 def parse_args():
@@ -570,6 +570,8 @@ def run_case(args, world, rank, local):
         return run_vendor_fp4(args)
     if kind == "fused":
         return run_fused(args, nums[0] if nums else 8192)
+    if kind == "decode":
+        return run_decode(args, nums[0] if nums else 1)
     if kind == "prep":
         M, K = nums[:2]
         fmt, n, m = (nums[2:5] + [0, N_KEEP, M_GROUP][len(nums[2:5]):])
@@ -684,6 +686,77 @@ def run_fused(args, M):
     return {"case": args.case, "tokens_per_s": M / (total / 1e3), "ms_per_step": total, "prep_ms": prep_ms,
             "gemm_ms": sum(each), "gemm_each": {"+".join(l.name for l in g): each[j] for j, g in enumerate(groups)},
             "steps": args.steps}
+
+
+def run_decode(args, M):
+    """The layer-set step at decode sizes (M tokens, default 1): 4 preps + 7
+    linears launched eagerly from Python, and the same step captured once in
+    a CUDA graph and replayed. L2 is flushed before every step (outside the
+    graph), so the weights stream from HBM as they do when a model's layers
+    take turns; the roofline is that weight stream (codes + scales of the 7
+    weights) at the measured HBM bandwidth."""
+    import sparsity_gemm_b200 as sq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ls, preps = layer_set()
+    prep_index = {name: i for i, (name, _) in enumerate(preps)}
+    xs = [torch.from_numpy(synth.activations_student(i, M, k).view(np.float16)).to(dev)
+          for i, (_, k) in enumerate(preps)]
+    qws = []
+    for j, lin in enumerate(ls.linears):
+        w = torch.from_numpy(synth.weights(1000 + j, lin.n_out, lin.k).view(np.float16)).to(dev)
+        qws.append(sq.quantize_weight(w, sq.NVFP4))
+        del w
+    bufs = [sq.prepare(xs[i], None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4) for i in range(len(preps))]
+    outs = [torch.empty((M, lin.n_out), dtype=torch.float16, device=dev) for lin in ls.linears]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peaks, peak_src = load_peaks()
+
+    def step():
+        for i in range(len(preps)):
+            sq.prepare(xs[i], None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4, out=bufs[i])
+        for j, lin in enumerate(ls.linears):
+            sq.linear(bufs[prep_index[lin.prep]], qws[j], out=outs[j])
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for _ in range(max(args.warmup, 1)):
+            step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    eager_out = [o.clone() for o in outs]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    stream = torch.cuda.current_stream()
+
+    def timed(run):
+        for _ in range(args.warmup):
+            flush.zero_()
+            run()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            run()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return statistics.median([a.elapsed_time(b) for a, b in ev])
+
+    eager_ms = timed(step)
+    graph_ms = timed(graph.replay)
+    same = all(torch.equal(o.view(torch.int16), e.view(torch.int16)) for o, e in zip(outs, eager_out))
+    st = sq.get_last_error()
+    if st != sq.OK:
+        raise RuntimeError(sq.status_name(st))
+    w_bytes = sum(l.n_out * l.k / 2 + l.n_out * l.k / 16 for l in ls.linears)  # E2M1 codes + UE4M3 scales
+    x_bytes = sum(M * k * 2 for _, k in preps)
+    floor_ms = (w_bytes + x_bytes) / (peaks["hbm_gbs"] * 1e9) * 1e3
+    return {"case": args.case, "tokens": M, "eager_ms_per_step": eager_ms, "graph_ms_per_step": graph_ms,
+            "graph_tokens_per_s": M / (graph_ms / 1e3), "kernels_per_step": 4 * 2 + 7,
+            "weight_stream_floor_ms": floor_ms, "graph_frac_of_floor": floor_ms / graph_ms,
+            "graph_equals_eager": same, "peak_source": f"{peak_src} hbm {peaks['hbm_gbs']} GB/s",
+            "l2": "flushed (256 MB write) before every step", "steps": args.steps}
 
 
 def run_sweep(args):

@@ -126,8 +126,9 @@ struct GemmParams {
 __device__ __forceinline__ float alpha_of_col(const GemmParams &p, float s_t, float alpha0, int col) {
     if (p.segs <= 1) return alpha0;
     int g = 0;
-#pragma unroll 1
-    for (int i = 0; i + 1 < p.segs; ++i) g += col >= p.seg_end[i] ? 1 : 0;
+#pragma unroll
+    for (int i = 0; i + 1 < SHARQ_SEGMENTS_MAX; ++i)  // constant indices: no local copy of the parameters
+        g += (i + 1 < p.segs && col >= p.seg_end[i]) ? 1 : 0;
     return __fmul_rn(s_t, p.s_tw[g]);
 }
 
