@@ -572,6 +572,10 @@ def run_case(args, world, rank, local):
         return run_fused(args, nums[0] if nums else 8192)
     if kind == "decode":
         return run_decode(args, nums[0] if nums else 1)
+    if kind == "qwen25":
+        return run_qwen25(args, nums[0] if nums else 4096)
+    if kind == "layerset":
+        return run_layerset_tokens(args, nums or [1, 16, 128, 2048, 8192])
     if kind == "prep":
         M, K = nums[:2]
         fmt, n, m = (nums[2:5] + [0, N_KEEP, M_GROUP][len(nums[2:5]):])
@@ -686,6 +690,106 @@ def run_fused(args, M):
     return {"case": args.case, "tokens_per_s": M / (total / 1e3), "ms_per_step": total, "prep_ms": prep_ms,
             "gemm_ms": sum(each), "gemm_each": {"+".join(l.name for l in g): each[j] for j, g in enumerate(groups)},
             "steps": args.steps}
+
+
+def prep_bytes_per_elem(fmt, n, m):
+    """Algorithmic bytes per activation element of one preparation: x read
+    (2), S and R codes (0.5 each, S kept dense with zeros), the mask metadata
+    and two scale arrays (one byte per block of 16 or 32)."""
+    meta = n * max(1, (m - 1).bit_length()) / m / 8.0
+    return 2 + 0.5 + 0.5 + meta + 2.0 / (16 if fmt == 0 else 32)
+
+
+def time_layer_set(ls, M, fmt, n, m, steps, warmup):
+    """Event timing of one layer set's step (its preps, then its linears) at
+    M tokens with L2 flushed before every step: medians of the per-step prep
+    and GEMM milliseconds."""
+    import sparsity_gemm_b200 as sq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    preps = list(ls.preps)
+    prep_index = {name: i for i, (name, _) in enumerate(preps)}
+    xs = [torch.from_numpy(synth.activations_student(i, M, k).view(np.float16)).to(dev)
+          for i, (_, k) in enumerate(preps)]
+    qws = []
+    for j, lin in enumerate(ls.linears):
+        w = torch.from_numpy(synth.weights(1000 + j, lin.n_out, lin.k).view(np.float16)).to(dev)
+        qws.append(sq.quantize_weight(w, fmt))
+        del w
+    bufs = [sq.prepare(xs[i], None, None, EPS, n, m, fmt) for i in range(len(preps))]
+    outs = [torch.empty((M, lin.n_out), dtype=torch.float16, device=dev) for lin in ls.linears]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    np_ = len(preps)
+
+    def step(ev=None):
+        for i in range(np_):
+            sq.prepare(xs[i], None, None, EPS, n, m, fmt, out=bufs[i])
+        if ev is not None:
+            ev[1].record(stream)
+        for j, lin in enumerate(ls.linears):
+            sq.linear(bufs[prep_index[lin.prep]], qws[j], out=outs[j])
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for ev in evs:
+        flush.zero_()
+        ev[0].record(stream)
+        step(ev)
+        ev[2].record(stream)
+    torch.cuda.synchronize()
+    st = sq.get_last_error()
+    if st != sq.OK:
+        raise RuntimeError(sq.status_name(st))
+    prep_ms = statistics.median([e[0].elapsed_time(e[1]) for e in evs])
+    gemm_ms = statistics.median([e[1].elapsed_time(e[2]) for e in evs])
+    del xs, qws, bufs, outs, flush
+    torch.cuda.empty_cache()
+    return prep_ms, gemm_ms
+
+
+def layer_set_report(ls, M, fmt, n, m, prep_ms, gemm_ms, peaks):
+    flops = sum(2.0 * M * l.n_out * l.k * (1.0 + n / m) for l in ls.linears)
+    pbytes = sum(prep_bytes_per_elem(fmt, n, m) * M * k for _, k in ls.preps)
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    gemm_tf = flops / (gemm_ms / 1e3) / 1e12
+    prep_gbs = pbytes / (prep_ms / 1e3) / 1e9
+    return {"tokens": M, "fmt": "nvfp4" if fmt == 0 else "mxfp4", "nm": f"{n}:{m}",
+            "tokens_per_s": M / ((prep_ms + gemm_ms) / 1e3), "ms_per_step": prep_ms + gemm_ms,
+            "prep_ms": prep_ms, "gemm_ms": gemm_ms, "gemm_tflops": gemm_tf, "gemm_frac": gemm_tf / fp4_peak,
+            "prep_gbs": prep_gbs, "prep_frac": prep_gbs / peaks["hbm_gbs"]}
+
+
+def run_qwen25(args, M):
+    """The Qwen2.5-7B layer set (hidden 3584, GQA kv 512, intermediate 18944)
+    at M tokens (prefill, 4096 by default) for each format and N:M ratio:
+    {NVFP4, MXFP4} x {2:4, 4:8}."""
+    peaks, peak_src = load_peaks()
+    rows = []
+    for fmt in (0, 1):
+        for n, m in ((2, 4), (4, 8)):
+            prep_ms, gemm_ms = time_layer_set(synth.QWEN25_7B, M, fmt, n, m, args.steps, args.warmup)
+            rows.append(layer_set_report(synth.QWEN25_7B, M, fmt, n, m, prep_ms, gemm_ms, peaks))
+    return {"case": args.case, "workload": "Qwen2.5-7B layer set (q/k/v 3584->3584/512/512, o 3584->3584, "
+            "gate/up 3584->18944, down 18944->3584): 4 preps + 7 dual-path linears", "tokens": M, "rows": rows,
+            "peak_source": f"{peak_src}: FP4 = bf16 {peaks['bf16_tflops']} TF/s x {FP4_OVER_BF16}, "
+            f"HBM {peaks['hbm_gbs']} GB/s", "l2": "flushed (256 MB write) before every step", "steps": args.steps}
+
+
+def run_layerset_tokens(args, tokens):
+    """The Llama-3.1-8B layer set (NVFP4, 2:4) at each token count (decode to
+    prefill: 1, 16, 128, 2048, 8192 by default)."""
+    peaks, peak_src = load_peaks()
+    rows = []
+    for M in tokens:
+        prep_ms, gemm_ms = time_layer_set(synth.LLAMA31_8B, M, 0, N_KEEP, M_GROUP, args.steps, args.warmup)
+        rows.append(layer_set_report(synth.LLAMA31_8B, M, 0, N_KEEP, M_GROUP, prep_ms, gemm_ms, peaks))
+    return {"case": args.case, "workload": workload_desc("M"), "rows": rows,
+            "peak_source": f"{peak_src}: FP4 = bf16 {peaks['bf16_tflops']} TF/s x {FP4_OVER_BF16}, "
+            f"HBM {peaks['hbm_gbs']} GB/s", "l2": "flushed (256 MB write) before every step",
+            "launch": "eager from Python (see --case decode:M for CUDA-graph replay)", "steps": args.steps}
 
 
 def run_decode(args, M):

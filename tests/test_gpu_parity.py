@@ -9,8 +9,8 @@ import torch
 
 import oracle
 import synth
-from gpu_common import (assert_linear_close, assert_prep_matches, assert_weight_matches, cuda16,
-                        gpu_prepare)
+from gpu_common import (assert_bits_equal, assert_linear_close, assert_prep_matches, assert_weight_matches,
+                        cuda16, gpu_prepare)
 
 pytestmark = pytest.mark.gpu
 
@@ -79,6 +79,43 @@ def test_prepare_many_short_rows_bit_exact(m_tok, k, fmt, norm):
     op = oracle.prepare(x, None, None, 1e-5, 2, 4, fmt, norm=norm)
     p = sq.prepare(cuda16(x), None, None, 1e-5, 2, 4, fmt, norm=norm)
     assert_prep_matches(sq.prep_export(p), op)
+
+
+def test_maximum_k_statistics_at_the_lane_sum_bound():
+    """K = SHARQ_K_MAX with rows enough for one warp per row: each lane adds
+    2048 values, the bound of its 32-bit sums; rows of fp16 extremes (all
+    +65504, alternating +-65504, all -65504) and Student-t rows. Statistics
+    bit-exact for every row, LayerNorm and RMSNorm."""
+    import sparsity_gemm_b200 as sq
+    m_tok, k = 1200, sq.K_MAX
+    x = synth.activations_student(910, m_tok, k)
+    x[0] = np.float16(65504.0)
+    x[1, ::2] = np.float16(65504.0)
+    x[1, 1::2] = np.float16(-65504.0)
+    x[2] = np.float16(-65504.0)
+    x[3, : k // 2] = np.float16(65504.0)
+    xd = cuda16(x)
+    for norm, stats in (("layer", oracle.ln_stats), ("rms", oracle.rms_stats)):
+        mu, rstd = stats(x, 1e-5)
+        ex = sq.prep_export(sq.prepare(xd, None, None, 1e-5, 2, 4, sq.NVFP4, norm=norm))
+        assert_bits_equal("mu", ex["mu"], mu)
+        assert_bits_equal("rstd", ex["rstd"], rstd)
+
+
+def test_maximum_k_linear():
+    """A linear at K = SHARQ_K_MAX (256 K steps, split over a cluster at 9
+    rows): prep bit-exact, output within tolerance."""
+    import sparsity_gemm_b200 as sq
+    m_tok, n_out, k = 9, 256, sq.K_MAX
+    x = synth.activations_student(911, m_tok, k)
+    w = synth.weights(912, n_out, k)
+    op = oracle.prepare(x, None, None, 1e-5, 2, 4, 0)
+    p, ex = gpu_prepare(x, None, None, 1e-5, 2, 4, 0)
+    assert_prep_matches(ex, op)
+    out = sq.linear(p, sq.quantize_weight(cuda16(w), 0)).cpu().numpy()
+    want, bound = oracle.linear_prepared(op, oracle.quantize_weight(w, 0))
+    assert_linear_close(out, want, bound)
+    assert sq.get_last_error() == sq.OK
 
 
 @pytest.mark.parametrize("n_out,k,fmt", [(32, 256, 0), (544, 512, 0), (544, 512, 1), (256, 1024, 1)])
