@@ -965,8 +965,8 @@ def run_moe(args, tokens):
     """The Qwen3-30B-A3B-shaped MoE FFN (hidden 2048, 128 experts of
     intermediate 768, top-8 routing from N(0,1) gate logits) as one step:
     prep of the token activation, expert-grouped gather, gate and up
-    grouped linears, prep of the down projection's grouped-order input,
-    its gather (identity rows), down grouped linear. L2 flushed before every
+    grouped linears, prep of the down projection's grouped-order input
+    straight into the grouped layout, down grouped linear. L2 flushed before every
     step; every launch timed with CUDA events on the launching stream."""
     import sparsity_gemm_b200 as sq
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -988,8 +988,7 @@ def run_moe(args, tokens):
         del w
     p_tok = sq.prepare(x, None, None, EPS, n, m, fmt)
     g_tok = sq.gather_rows(p_tok, ri, off, rows)
-    p_d = sq.prepare(xd, None, None, EPS, n, m, fmt)
-    g_d = sq.gather_rows(p_d, None, off, rows)
+    g_d = sq.prepare_grouped(xd, off, None, None, EPS, n, m, fmt)
     o_gate = torch.empty((rows, inter), dtype=torch.float16, device=dev)
     o_up = torch.empty_like(o_gate)
     o_down = torch.empty((rows, hidden), dtype=torch.float16, device=dev)
@@ -998,8 +997,7 @@ def run_moe(args, tokens):
         ("gather", lambda: sq.gather_rows(p_tok, ri, off, rows, out=g_tok)),
         ("gate", lambda: sq.linear_grouped(g_tok, off, qws["gate"], rows, out=o_gate)),
         ("up", lambda: sq.linear_grouped(g_tok, off, qws["up"], rows, out=o_up)),
-        ("prep_down", lambda: sq.prepare(xd, None, None, EPS, n, m, fmt, out=p_d)),
-        ("gather_down", lambda: sq.gather_rows(p_d, None, off, rows, out=g_d)),
+        ("prep_down", lambda: sq.prepare_grouped(xd, off, None, None, EPS, n, m, fmt, out=g_d)),
         ("down", lambda: sq.linear_grouped(g_d, off, qws["down"], rows, out=o_down)),
     ]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)

@@ -381,6 +381,32 @@ sharq_status sharq_gather_rows(const sharq_prep *src, const int32_t *row_idx_dev
  * n_groups and rows <= prep->m_tok. Device-side checks: the offsets, and
  * that the rows they pad to fit in prep->m_tok.
  */
+/*
+ * Preparation straight into the grouped layout, for an activation whose rows
+ * are already in grouped order (the input of a mixture-of-experts down
+ * projection: the output of the grouped gate/up linears and the activation
+ * function). An interface addition. Equal, in codes, scales, mask metadata
+ * and tensor scale, to sharq_gather_rows(prepare(x), NULL, offsets) bit for
+ * bit, in one preparation pass instead of a preparation and a gather.
+ *   x_dev        fp16 [rows][k], rows in grouped order (group g's rows are
+ *                offsets[g] .. offsets[g+1] - 1).
+ *   offsets_dev  int32 [n_groups + 1], device: offsets[0] = 0, ascending,
+ *                offsets[n_groups] = rows; checked on the device (invalid
+ *                offsets leave the output untouched and set the status that
+ *                sharq_get_last_error reports).
+ *   norm         0: LayerNorm (ln_w, ln_b as sharq_prepare); 1: RMSNorm
+ *                (ln_w as sharq_prepare_rms, ln_b must be NULL).
+ *   prep_dev     at least sharq_gather_bytes(rows, n_groups, k, n, m, fmt)
+ *                bytes.
+ * prep_out describes a grouped prep of sharq_grouped_rows(rows, n_groups)
+ * rows (groups = n_groups) for sharq_linear_grouped; its per-row statistics
+ * are indexed by source row. Other preconditions as sharq_prepare.
+ */
+sharq_status sharq_prepare_grouped(const void *x_dev, int64_t rows, int64_t k, const int32_t *offsets_dev,
+                                   int64_t n_groups, const void *ln_w_dev, const void *ln_b_dev, float eps, int norm,
+                                   int n, int m, int fmt, void *prep_dev, size_t prep_bytes, sharq_prep *prep_out,
+                                   void *stream);
+
 sharq_status sharq_linear_grouped(const sharq_prep *prep, const int32_t *offsets_dev, int64_t n_groups,
                                   int64_t rows, const sharq_wq *wq, void *out_dev, void *stream);
 

@@ -93,13 +93,16 @@ def lib():
                                                   C.POINTER(SharqWQ), vp]
         L.sharq_linear_bias.argtypes = [C.POINTER(SharqPrep), C.POINTER(SharqWQ), vp, vp, vp]
         L.sharq_weight_tensor_scales.argtypes = [C.POINTER(SharqWQ), vp, vp]
+        L.sharq_prepare_grouped.argtypes = [vp, i64, i64, vp, i64, vp, vp, f32, i32, i32, i32, i32, vp, sz,
+                                            C.POINTER(SharqPrep), vp]
         L.sharq_status_string.argtypes = [i32]
         L.sharq_status_string.restype = C.c_char_p
         L.sharq_last_launch_count.restype = i32
         for name in ("sharq_quantize_weight", "sharq_prepare", "sharq_linear", "sharq_prep_export",
                      "sharq_weight_export", "sharq_get_last_error", "sharq_quantize_weight_grouped",
                      "sharq_gather_rows", "sharq_linear_grouped", "sharq_prepare_rms",
-                     "sharq_quantize_weight_fused", "sharq_linear_bias", "sharq_weight_tensor_scales"):
+                     "sharq_quantize_weight_fused", "sharq_linear_bias", "sharq_weight_tensor_scales",
+                     "sharq_prepare_grouped"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -335,6 +338,29 @@ def gather_rows(prep: Prepared, row_idx, offsets: torch.Tensor, rows: int, out: 
     desc = SharqPrep()
     _check(lib().sharq_gather_rows(C.byref(d), _ptr(row_idx), _ptr(offsets), groups, rows, _ptr(buf), buf.numel(),
                                    C.byref(desc), _stream(stream)), "sharq_gather_rows")
+    return Prepared(buf, desc)
+
+
+def prepare_grouped(x: torch.Tensor, offsets: torch.Tensor, ln_w=None, ln_b=None, eps: float = 1e-5, n: int = 2,
+                    m: int = 4, fmt: int = NVFP4, norm: str = "layer", out: Prepared | None = None,
+                    stream=None) -> Prepared:
+    """Preparation of x [rows, k] (fp16, CUDA; rows in grouped order, group g
+    = rows offsets[g] .. offsets[g+1]-1) straight into the grouped layout that
+    gather_rows writes (equal to gather_rows(prepare(x), None, offsets) in
+    codes, scales, metadata and tensor scale). offsets: int32 CUDA tensor."""
+    assert norm in ("layer", "rms") and (norm == "layer" or ln_b is None)
+    assert x.dtype == torch.float16 and x.is_cuda and x.dim() == 2 and x.is_contiguous()
+    assert offsets.dtype == torch.int32 and offsets.is_cuda and offsets.is_contiguous()
+    rows, k = x.shape
+    groups = offsets.numel() - 1
+    nbytes = int(lib().sharq_gather_bytes(rows, groups, k, n, m, fmt))
+    if nbytes == 0:
+        raise SharqError(ERR_INVALID_ARG, f"grouped prep rows {rows} groups {groups} k {k}")
+    buf = out.buf if out is not None and out.buf.numel() >= nbytes else _device_buffer(nbytes, x.device)
+    desc = SharqPrep()
+    _check(lib().sharq_prepare_grouped(_ptr(x) if rows > 0 else None, rows, k, _ptr(offsets), groups, _ptr(ln_w),
+                                       _ptr(ln_b), float(eps), 1 if norm == "rms" else 0, n, m, fmt, _ptr(buf),
+                                       buf.numel(), C.byref(desc), _stream(stream)), "sharq_prepare_grouped")
     return Prepared(buf, desc)
 
 

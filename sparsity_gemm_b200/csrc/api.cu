@@ -325,6 +325,34 @@ sharq_status sharq_gather_rows(const sharq_prep *src, const int32_t *row_idx_dev
     return st;
 }
 
+sharq_status sharq_prepare_grouped(const void *x_dev, int64_t rows, int64_t k, const int32_t *offsets_dev,
+                                   int64_t n_groups, const void *ln_w_dev, const void *ln_b_dev, float eps, int norm,
+                                   int n, int m, int fmt, void *prep_dev, size_t prep_bytes, sharq_prep *prep_out,
+                                   void *stream) {
+    g_last_launches = 0;
+    if (!offsets_dev || !prep_dev || !prep_out || !aligned(offsets_dev, 4) || !aligned(prep_dev, sq::kAlign))
+        return SHARQ_ERR_INVALID_ARG;
+    if (!fmt_ok(fmt) || !nm_ok(n, m) || !k_ok(k) || rows < 0 || rows > (1ll << 30) || n_groups < 1 ||
+        n_groups > sq::kGroupsMax)
+        return SHARQ_ERR_INVALID_ARG;
+    if ((norm != 0 && norm != 1) || (norm == 1 && ln_b_dev)) return SHARQ_ERR_INVALID_ARG;
+    if (!(eps > 0.0f) || eps != eps || eps > 3.0e38f) return SHARQ_ERR_INVALID_ARG;
+    if (rows > 0 && (!x_dev || !aligned(x_dev, 16))) return SHARQ_ERR_INVALID_ARG;
+    if ((ln_w_dev && !aligned(ln_w_dev, 16)) || (ln_b_dev && !aligned(ln_b_dev, 16))) return SHARQ_ERR_INVALID_ARG;
+    const size_t need = sharq_gather_bytes(rows, n_groups, k, n, m, fmt);
+    if (!need || prep_bytes < need) return SHARQ_ERR_INVALID_ARG;
+    sq::LaunchCtx ctx;
+    sharq_status st = make_ctx(stream, ctx);
+    if (st != SHARQ_OK) return st;
+    fill_prep(prep_out, prep_dev, sq::grouped_rows(rows, n_groups), k, n, m, fmt);
+    prep_out->groups = (int32_t)n_groups;
+    st = sq::launch_prepare_grouped(ctx, *prep_out, x_dev, rows, offsets_dev, (int32_t)n_groups, ln_w_dev, ln_b_dev,
+                                    eps, norm);
+    if (st == SHARQ_OK && cudaGetLastError() != cudaSuccess) st = SHARQ_ERR_CUDA;
+    g_last_launches = ctx.launches;
+    return st;
+}
+
 sharq_status sharq_linear_grouped(const sharq_prep *prep, const int32_t *offsets_dev, int64_t n_groups, int64_t rows,
                                   const sharq_wq *wq, void *out_dev, void *stream) {
     g_last_launches = 0;

@@ -392,9 +392,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         uint32_t tile_iter = 0;
         for (int tile = tile_begin; tile < num_tiles; tile += tile_step, ++tile_iter) {
             const int nb = tile % n_tiles, mb = tile / n_tiles;
-            int grp = 0;
             if constexpr (GROUPED) {
-                grp = group_of_tile(tiles, p.groups, mb);
+                const int grp = group_of_tile(tiles, p.groups, mb);
                 alpha = __fmul_rn(s_t, *reinterpret_cast<const float *>(
                                            reinterpret_cast<const uint8_t *>(p.s_tw) + (int64_t)grp * p.w_gstride));
             }
@@ -466,8 +465,10 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             mbar_arrive(acc_empty);
             int64_t row, row_end;  // output row of this lane; end of the tile's valid rows
             if constexpr (GROUPED) {
-                const int32_t first = p.offsets[grp], last = p.offsets[grp + 1];
-                row = (int64_t)first + (int64_t)(mb - tiles[grp]) * kBM + q * 32 + lane;
+                // looked up again rather than kept live across the drain (register pressure)
+                const int g2 = group_of_tile(tiles, p.groups, mb);
+                const int32_t first = p.offsets[g2], last = p.offsets[g2 + 1];
+                row = (int64_t)first + (int64_t)(mb - tiles[g2]) * kBM + q * 32 + lane;
                 row_end = last;
             } else {
                 row = mb * kBM + q * 32 + lane;

@@ -617,12 +617,15 @@ struct EncodeArgs {
 };
 
 // Encode step of unit u of row `row`: LayerNorm apply, mask, Q(S), R, Q(R),
-// stores. `active` lanes with row >= m_tok are scale-layout padding (zero
-// scales); inactive lanes only take part in the MXFP4 lane-pair exchanges.
+// stores. `active` lanes with row >= m_tok (or row < 0) are padding: zero
+// scales, and with pad_codes also zero codes and metadata; inactive lanes
+// only take part in the MXFP4 lane-pair exchanges. The outputs go to row
+// `dst` (-1: the same row).
 // NK > 0: n fixed at compile time (the 2:4 default takes its own mask).
 template <int FMT, int M, int NK>
 __device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t *lut, int64_t row, int64_t u,
-                                            bool active, float s_t, float c6, float y6) {
+                                            bool active, float s_t, float c6, float y6, int64_t dst = -1,
+                                            bool pad_codes = false) {
     constexpr int IB = M <= 2 ? 1 : M <= 4 ? 2 : M <= 8 ? 3 : 4;
     constexpr int G = kUnit / M;  // mask groups per unit
     const uint16_t *__restrict__ x = a.x;
@@ -640,7 +643,8 @@ __device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t 
     const int B = G * gbits;   // metadata bits per unit
     const bool byte_aligned = (B & 7) == 0;
     const bool has_g = gamma != nullptr, has_b = beta != nullptr;
-    const bool real = active && row < m_tok;
+    const bool real = active && row >= 0 && row < m_tok;
+    const int64_t orow = dst >= 0 ? dst : row;  // output row
 
     // LayerNorm apply on the unit's 16 values (zeros on idle lanes, which
     // still take part in the MXFP4 lane-pair exchanges).
@@ -729,26 +733,32 @@ __device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t 
     }
 
     if (real) {
-        *reinterpret_cast<uint2 *>(s_codes + row * (k / 2) + u * 8) = make_uint2(s_lo, s_hi);
-        *reinterpret_cast<uint2 *>(r_codes + row * (k / 2) + u * 8) = make_uint2(r_lo, r_hi);
+        *reinterpret_cast<uint2 *>(s_codes + orow * (k / 2) + u * 8) = make_uint2(s_lo, s_hi);
+        *reinterpret_cast<uint2 *>(r_codes + orow * (k / 2) + u * 8) = make_uint2(r_lo, r_hi);
         if (FMT == kFmtNV) {
-            s_sf[sf_offset(row, u, nblk)] = (uint8_t)s_scale;
-            r_sf[sf_offset(row, u, nblk)] = (uint8_t)r_scale;
+            s_sf[sf_offset(orow, u, nblk)] = (uint8_t)s_scale;
+            r_sf[sf_offset(orow, u, nblk)] = (uint8_t)r_scale;
         } else if ((u & 1) == 0) {
-            s_sf[sf_offset(row, u >> 1, nblk)] = (uint8_t)s_scale;
-            r_sf[sf_offset(row, u >> 1, nblk)] = (uint8_t)r_scale;
+            s_sf[sf_offset(orow, u >> 1, nblk)] = (uint8_t)s_scale;
+            r_sf[sf_offset(orow, u >> 1, nblk)] = (uint8_t)r_scale;
         }
         if (byte_aligned)
-            store_bytes(meta + row * meta_row + u * (B / 8), mbits, B / 8);
+            store_bytes(meta + orow * meta_row + u * (B / 8), mbits, B / 8);
         else
-            or_bits(reinterpret_cast<uint32_t *>(meta), (uint64_t)row * meta_row * 8 + (uint64_t)u * B, mbits, B);
-    } else if (active) {  // scale-layout padding rows: zero scales
+            or_bits(reinterpret_cast<uint32_t *>(meta), (uint64_t)orow * meta_row * 8 + (uint64_t)u * B, mbits, B);
+    } else if (active) {  // padding rows: zero scales (and codes and metadata where asked)
         if (FMT == kFmtNV) {
-            s_sf[sf_offset(row, u, nblk)] = 0;
-            r_sf[sf_offset(row, u, nblk)] = 0;
+            s_sf[sf_offset(orow, u, nblk)] = 0;
+            r_sf[sf_offset(orow, u, nblk)] = 0;
         } else if ((u & 1) == 0) {
-            s_sf[sf_offset(row, u >> 1, nblk)] = 0;
-            r_sf[sf_offset(row, u >> 1, nblk)] = 0;
+            s_sf[sf_offset(orow, u >> 1, nblk)] = 0;
+            r_sf[sf_offset(orow, u >> 1, nblk)] = 0;
+        }
+        if (pad_codes) {
+            *reinterpret_cast<uint2 *>(s_codes + orow * (k / 2) + u * 8) = make_uint2(0u, 0u);
+            *reinterpret_cast<uint2 *>(r_codes + orow * (k / 2) + u * 8) = make_uint2(0u, 0u);
+            if (byte_aligned) store_bytes(meta + orow * meta_row + u * (B / 8), 0ull, B / 8);
+            // (unaligned metadata fields are OR-ed into a stream zeroed beforehand)
         }
     }
 }
@@ -805,6 +815,99 @@ prep_encode_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ 
             ++row_i;
         }
         encode_unit<FMT, M, NK>(ea, lut, row, u, active, s_t, c6, y6);
+    }
+}
+
+constexpr int kGroupedTileTable = 4096;  // tiles whose group the grouped encode tabulates in shared memory
+
+// Encode pass straight into the expert-grouped layout (the layout of
+// sharq_gather_rows): source rows in grouped order, group g's rows placed
+// from row 128 T_g on (T_g: 128-row tiles of the groups before g), every
+// other row zero. Warp 0 builds the groups' tile table from the device
+// offsets; invalid offsets record the status and leave the outputs alone.
+template <int FMT, int M, int NK>
+__global__ void __launch_bounds__(kEncodeThreads, SQ_ENCODE_MIN_CTAS)
+prep_encode_grouped_kernel(const EncodeArgs ea, const unsigned *__restrict__ amax_word, float *__restrict__ s_t_out,
+                           int64_t cap_rows, const int32_t *__restrict__ offsets, int32_t groups, int64_t rows,
+                           unsigned *status) {
+    constexpr int IB = M <= 2 ? 1 : M <= 4 ? 2 : M <= 8 ? 3 : 4;
+    __shared__ uint32_t lut[M <= 8 ? (1 << M) : 1];  // keep bits of a group -> kept positions, ascending
+    __shared__ int32_t tiles[kGroupsMax + 1];
+    __shared__ int16_t tile_group[kGroupedTileTable];  // group of each 128-row tile (small launches)
+    __shared__ int table_ok;
+    if (M <= 8) {
+        for (int msk = threadIdx.x; msk < (1 << M); msk += kEncodeThreads) {
+            uint32_t packed = 0;
+            int pos = 0;
+            for (int i = 0; i < M; ++i)
+                if ((msk >> i) & 1) {
+                    packed |= (uint32_t)i << pos;
+                    pos += IB;
+                }
+            lut[msk] = packed;
+        }
+    }
+    if (threadIdx.x / 32 == 0) {
+        const bool ok = build_tile_table(offsets, groups, rows, cap_rows, tiles);
+        if (threadIdx.x == 0) table_ok = ok ? 1 : 0;
+    }
+    __syncthreads();
+    if (!table_ok) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) record_status(status, kSiteBadOffsets);
+        return;
+    }
+    // Group of every used tile, once per CTA, when the tiles are few enough.
+    const int32_t used_tiles = tiles[groups];
+    const bool small_table = used_tiles <= kGroupedTileTable;
+    if (small_table)
+        for (int32_t t = threadIdx.x; t < used_tiles; t += kEncodeThreads)
+            tile_group[t] = (int16_t)group_of_tile(tiles, groups, t);
+    __syncthreads();
+    const float amax = __uint_as_float(*amax_word);
+    const float s_t = (FMT == kFmtNV && amax != 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+    const float c6 = __fmul_rn(6.0f, s_t);
+    const float y6 = (FMT == kFmtNV && c6 >= 0x1p-90f && c6 <= 0x1p90f) ? __frcp_rn(c6) : 0.0f;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *s_t_out = s_t;
+    constexpr int IBm = M <= 2 ? 1 : M <= 4 ? 2 : M <= 8 ? 3 : 4;
+    const int unit_meta_bits = (kUnit / M) * ea.n * IBm;
+
+    const int64_t upr = ea.k / kUnit;  // units per row
+    const int64_t total = cap_rows * upr;
+    const int64_t stride = (int64_t)gridDim.x * kEncodeThreads;
+    const int64_t t0 = (int64_t)blockIdx.x * kEncodeThreads + threadIdx.x;
+    int64_t row_i = t0 / upr, u_i = t0 - (t0 / upr) * upr;
+    const int64_t step_rows = stride / upr, step_units = stride - (stride / upr) * upr;
+    for (int64_t base = (int64_t)blockIdx.x * kEncodeThreads; base < total; base += stride) {
+        const int64_t t = base + threadIdx.x;
+        const bool active = t < total;
+        const int64_t d = row_i, u = u_i;
+        row_i += step_rows;
+        u_i += step_units;
+        if (u_i >= upr) {
+            u_i -= upr;
+            ++row_i;
+        }
+        int64_t src = -1;
+        if (active) {
+            const int32_t tile = (int32_t)(d >> 7);
+            if (tile < used_tiles) {
+                const int g = small_table ? (int)tile_group[tile] : group_of_tile(tiles, groups, tile);
+                const int64_t local = d - 128 * (int64_t)tiles[g];
+                if (local < (int64_t)offsets[g + 1] - offsets[g]) src = offsets[g] + local;
+            }
+        }
+        if (FMT == kFmtNV && active && src < 0) {
+            // A padding row: zeros, without the arithmetic (NVFP4 encodes
+            // have no lane exchanges, so this lane may skip the unit).
+            *reinterpret_cast<uint2 *>(ea.s_codes + d * (ea.k / 2) + u * 8) = make_uint2(0u, 0u);
+            *reinterpret_cast<uint2 *>(ea.r_codes + d * (ea.k / 2) + u * 8) = make_uint2(0u, 0u);
+            ea.s_sf[sf_offset(d, u, ea.nblk)] = 0;
+            ea.r_sf[sf_offset(d, u, ea.nblk)] = 0;
+            if ((unit_meta_bits & 7) == 0) store_bytes(ea.meta + d * ea.meta_row + u * (unit_meta_bits / 8), 0ull,
+                                                       unit_meta_bits / 8);
+            continue;
+        }
+        encode_unit<FMT, M, NK>(ea, lut, src, u, active, s_t, c6, y6, d, true);
     }
 }
 
@@ -1102,6 +1205,16 @@ static void *encode_fn(int m, int n) {
     }
 }
 
+template <int FMT>
+static void *encode_grouped_fn(int m, int n) {
+    switch (m) {
+        case 2: return (void *)prep_encode_grouped_kernel<FMT, 2, 0>;
+        case 4: return n == 2 ? (void *)prep_encode_grouped_kernel<FMT, 4, 2> : (void *)prep_encode_grouped_kernel<FMT, 4, 0>;
+        case 8: return (void *)prep_encode_grouped_kernel<FMT, 8, 0>;
+        default: return (void *)prep_encode_grouped_kernel<FMT, 16, 0>;
+    }
+}
+
 template <int FMT, bool RMS>
 static void *small_fn(int m) {
     switch (m) {
@@ -1345,6 +1458,40 @@ sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, 
     uint8_t *sc = (uint8_t *)P.s_codes, *rc = (uint8_t *)P.r_codes, *ss = (uint8_t *)P.s_scales,
             *rs = (uint8_t *)P.r_scales, *mt = (uint8_t *)P.meta;
     void *args[] = {&xx, &gg, &bb, &cst, &aw, &st, &m_tok, &sf_rows, &k, &n, &sc, &rc, &ss, &rs, &mt, &meta_row};
+    SQ_CUDA_TRY(cudaLaunchKernel(fn, dim3((unsigned)blocks), dim3(kEncodeThreads), args, 0, ctx.stream));
+    ctx.launches++;
+    return SHARQ_OK;
+}
+
+// Preparation of `rows` rows in grouped order straight into a grouped prep P
+// (P.m_tok = P.sf_rows = the grouped capacity): statistics over the source
+// rows (kept in P's statistics area, indexed by source row), then the
+// grouped encode pass.
+sharq_status launch_prepare_grouped(LaunchCtx &ctx, const sharq_prep &P, const void *x, int64_t rows,
+                                    const int32_t *offsets, int32_t groups, const void *gamma, const void *beta,
+                                    float eps, int norm) {
+    unsigned *words = reinterpret_cast<unsigned *>(P.tensor_scale) - 1;  // [0] amax bits, [1] s_t
+    SQ_CUDA_TRY(cudaMemsetAsync(words, 0, sizeof(unsigned), ctx.stream));
+    const bool meta_atomic = ((kUnit / P.m) * P.n * idx_bits(P.m)) % 8 != 0;
+    if (meta_atomic && P.m_tok > 0)
+        SQ_CUDA_TRY(cudaMemsetAsync(P.meta, 0, (size_t)(P.m_tok * P.meta_row_bytes), ctx.stream));
+    float2 *stats = reinterpret_cast<float2 *>(P.scratch);
+    sharq_prep src = P;  // the statistics pass sees the source rows
+    src.m_tok = rows;
+    const sharq_status sst = norm ? launch_stats<true>(ctx, src, x, gamma, beta, eps, stats, words)
+                                  : launch_stats<false>(ctx, src, x, gamma, beta, eps, stats, words);
+    if (sst != SHARQ_OK) return sst;
+    void *fn = P.fmt == kFmtNV ? encode_grouped_fn<kFmtNV>(P.m, P.n) : encode_grouped_fn<kFmtMX>(P.m, P.n);
+    const int64_t blocks = encode_grid(fn, ctx.num_sms, P.m_tok * (P.k / kUnit));
+    EncodeArgs ea{(const uint16_t *)x, (const uint16_t *)gamma, (const uint16_t *)beta, stats, rows, P.k,
+                  P.meta_row_bytes, P.k / (P.fmt == kFmtNV ? 16 : 32), P.n, (uint8_t *)P.s_codes,
+                  (uint8_t *)P.r_codes, (uint8_t *)P.s_scales, (uint8_t *)P.r_scales, (uint8_t *)P.meta};
+    const unsigned *aw = words;
+    float *sto = P.tensor_scale;
+    int64_t cap = P.m_tok, nrows = rows;
+    int32_t ng = groups;
+    unsigned *status = ctx.status;
+    void *args[] = {&ea, &aw, &sto, &cap, &offsets, &ng, &nrows, &status};
     SQ_CUDA_TRY(cudaLaunchKernel(fn, dim3((unsigned)blocks), dim3(kEncodeThreads), args, 0, ctx.stream));
     ctx.launches++;
     return SHARQ_OK;

@@ -18,6 +18,9 @@ struct LaunchCtx {
 // norm: 0 = LayerNorm, 1 = RMSNorm (beta must be NULL).
 sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, const void *gamma,
                             const void *beta, float eps, int norm);
+sharq_status launch_prepare_grouped(LaunchCtx &ctx, const sharq_prep &P, const void *x, int64_t rows,
+                                    const int32_t *offsets, int32_t groups, const void *gamma, const void *beta,
+                                    float eps, int norm);
 sharq_status launch_quantize_weight(LaunchCtx &ctx, const sharq_wq &W, const void *w, int64_t groups,
                                    int64_t gstride);
 sharq_status launch_quantize_weight_fused(LaunchCtx &ctx, const sharq_wq &W, const void *w, const int64_t *seg_rows,

@@ -100,6 +100,55 @@ def test_gather_rows_bit_exact(sq, fmt, n, m):
     assert sq.get_last_error() == sq.OK
 
 
+@pytest.mark.parametrize("fmt,n,m,norm", [(0, 2, 4, "layer"), (1, 2, 4, "layer"), (0, 3, 8, "layer"),
+                                          (0, 2, 4, "rms")])
+def test_prepare_grouped_equals_prepare_then_gather(sq, fmt, n, m, norm):
+    """Rows in grouped order prepared straight into the grouped layout: the
+    codes, scales, mask metadata and tensor scale equal a preparation
+    followed by the identity gather bit for bit (over the groups' tiles),
+    the statistics equal the plain preparation's (indexed by source row),
+    and a grouped linear on either gives the same output bit for bit."""
+    k = 512
+    rows = int(sum(COUNTS))
+    offsets = np.concatenate([[0], np.cumsum(COUNTS)]).astype(np.int32)
+    x = cuda16(synth.activations_student(270, rows, k))
+    off = _i32(offsets)
+    gp = sq.prepare_grouped(x, off, None, None, EPS, n, m, fmt, norm=norm)
+    p = sq.prepare(x, None, None, EPS, n, m, fmt, norm=norm)
+    gg = sq.gather_rows(p, None, off, rows)
+    assert gp.m_tok == gg.m_tok and gp.desc.groups == gg.desc.groups
+    eg, ed, ep = sq.prep_export(gp), sq.prep_export(gg), sq.prep_export(p)
+    used = padded_rows(offsets)[1]
+    for key in ("idx", "s_codes", "s_scales", "r_codes", "r_scales"):
+        assert_bits_equal(key, eg[key][:used], ed[key][:used])
+    assert_bits_equal("s_t", np.float32([eg["s_t"]]), np.float32([ed["s_t"]]))
+    assert_bits_equal("mu", eg["mu"][:rows], ep["mu"])
+    assert_bits_equal("rstd", eg["rstd"][:rows], ep["rstd"])
+    qw = sq.quantize_weight_grouped(cuda16(np.stack([synth.weights(271 + g, 96, k) for g in range(len(COUNTS))])), fmt)
+    a = sq.linear_grouped(gp, off, qw, rows).cpu().numpy()
+    b = sq.linear_grouped(gg, off, qw, rows).cpu().numpy()
+    assert_bits_equal("grouped linear", a.view(np.uint16), b.view(np.uint16))
+    assert sq.get_last_error() == sq.OK
+
+
+def test_prepare_grouped_edge_cases(sq):
+    """No rows (every tile row zero, tensor scale 1), and invalid offsets
+    (recorded on the device, output untouched)."""
+    k = 256
+    empty = sq.prepare_grouped(torch.zeros((0, k), dtype=torch.float16, device="cuda"), _i32([0, 0, 0]))
+    assert sq.prep_export(empty)["s_t"] == 1.0
+    assert sq.get_last_error() == sq.OK
+    x = cuda16(synth.activations_student(280, 40, k))
+    good = sq.prepare_grouped(x, _i32([0, 20, 40]))
+    sentinel = torch.full_like(good.buf, 0xA5)
+    sq.prepare_grouped(x, _i32([0, 30, 20]), out=sq.Prepared(sentinel, None))
+    assert sq.get_last_error() == sq.ERR_INVALID_ARG
+    assert sq.last_timeout_site() == 0x201
+    # the encode pass wrote nothing; only the statistics area and words may change
+    n_codes = good.desc.m_tok * (k // 2)
+    assert bool((sentinel[:n_codes] == 0xA5).all())
+
+
 @pytest.mark.parametrize("fmt,n_out", [(0, 544), (1, 256), (0, 96)])
 def test_linear_grouped_matches_oracle(sq, fmt, n_out):
     tokens, k = 300, 512
