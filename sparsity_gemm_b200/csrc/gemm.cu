@@ -45,43 +45,70 @@ namespace sq {
 #ifndef SQ_STORE_PAUSE_NS_PER_KSTEP
 #define SQ_STORE_PAUSE_NS_PER_KSTEP 60
 #endif
-constexpr int kBM = 128, kBN = 256, kBKBytes = SQ_GEMM_BKB;
+constexpr int kBM = 128, kBKBytes = SQ_GEMM_BKB;
 constexpr int kABytes = kBM * kBKBytes;
-constexpr int kBBytes = kBN * kBKBytes;
-constexpr int kSfaMax = 512 * (kBKBytes / 32), kSfbMax = 2 * kSfaMax;  // NVFP4 sizes (MXFP4 uses half)
+constexpr int kSfaMax = 512 * (kBKBytes / 32);  // scale bytes of 128 rows per stage, NVFP4 (MXFP4 uses half)
 constexpr int kOffAS = 0, kOffAR = kABytes, kOffB = 2 * kABytes;
-constexpr int kOffSFAS = kOffB + kBBytes, kOffSFAR = kOffSFAS + kSfaMax, kOffSFB = kOffSFAR + kSfaMax;
-constexpr int kStageBytes = kOffSFB + kSfbMax;                     // a multiple of 1024
-constexpr int kStages = (232448 - 2048) / kStageBytes;
-constexpr int kBarOff = kStages * kStageBytes;
-// Scale buffers in tensor memory after the accumulator (columns 0..255):
-// per buffer, the backbone A scales, the residual A scales and the W scales
-// of one stage (NVFP4: kBKBytes / 32 atoms per 128 rows; MXFP4 uses half).
+// Scale buffers in tensor memory after the accumulators: per buffer, the
+// backbone A scales, the residual A scales and the W scales of one stage
+// (NVFP4: kBKBytes / 32 atoms per 128 rows; MXFP4 uses half).
 constexpr uint32_t kNvAtoms = kBKBytes / 32;
-constexpr uint32_t kColSf0 = 256, kSfBufCols = 16 * kNvAtoms;
 constexpr uint32_t kSfaS = 0, kSfaR = 4 * kNvAtoms, kSfb = 8 * kNvAtoms;
-constexpr int kSfBufs = (int)(256 / kSfBufCols);
-// mbarriers: full[s], empty[s], sf_loaded[s], acc_full, acc_empty, drain,
-// sf_full[b], sf_empty[b]; the tensor-memory slot follows.
-constexpr int kBarBytes = 8 * (3 * kStages + 3 + 2 * kSfBufs);
-constexpr int kBarArea = (kBarBytes + 4 + 127) / 128 * 128;
 // Grouped launches: the tile table (kGroupsMax + 1 ints) and its valid flag.
-constexpr int kTableOff = kBarOff + kBarArea, kTableBytes = 4 * (int)(kGroupsMax + 1) + 12;
-constexpr int kSmemBytes = kTableOff + kTableBytes + 1024;        // barriers, table, alignment slack
+constexpr int kTableBytes = 4 * (int)(kGroupsMax + 1) + 12;
 constexpr int kMmaPerStage = kBKBytes / 32;                        // MMAs of K = 64 per path per stage
 constexpr uint32_t kSwizzleLayout = kBKBytes == 128 ? 2u : 4u;     // descriptor layout: 128B / 64B swizzle
 constexpr uint32_t kTmemCols = 512;
 constexpr int kGemmThreads = 320;
-static_assert(kStageBytes % 1024 == 0, "stage buffers must stay 1024-byte aligned");
-static_assert(kSmemBytes <= 232448, "shared memory budget");
-static_assert(kBarBytes + 4 <= kBarArea, "barrier area");
-static_assert(kColSf0 + kSfBufs * kSfBufCols <= kTmemCols, "tensor memory columns");
-static_assert(kTableBytes % 4 == 0, "table alignment");
-// Split-K partial tile in the stage memory: 128 rows of 256 fp32, rows
-// padded by 16 bytes so that a warp's 32 rows hit different banks.
-constexpr uint32_t kPartStride = kBN * 4 + 16;
 constexpr int kMaxSplit = 8;
-static_assert(kBM * kPartStride <= (uint32_t)(kStages * kStageBytes), "split-K partial fits the stages");
+static_assert(kTableBytes % 4 == 0, "table alignment");
+
+// Tile width N. 256: one accumulator (columns 0..255), four scale buffers
+// after it. 128: two accumulators used in turn (columns 0..127 and
+// 128..255), so that the next tile's MMAs run while the epilogue drains the
+// previous tile, and a fourth pipeline stage in the smaller stage memory.
+// Both widths give identical results. 256 is the default for dense and
+// grouped launches alike: with two A operands (backbone and residual) per
+// B tile, halving N raises the operand bytes per FLOP by half, which cost
+// more than the hidden drain saved on the short-K expert GEMMs (Qwen3 MoE
+// shapes, K = 2048 and 768: 22% slower at 128). SQ_GROUPED_BN=128 builds
+// the other width for grouped launches.
+template <int BN>
+struct TileCfg {
+    static constexpr int kBN = BN;
+    static constexpr int kBlk = BN / 128;            // 128-row W blocks (scale atoms) per tile
+    static constexpr int kNacc = BN == 256 ? 1 : 2;  // accumulators in tensor memory
+    static constexpr int kBBytes = BN * kBKBytes;
+    static constexpr int kSfbMax = kBlk * kSfaMax;
+    static constexpr int kOffSFAS = kOffB + kBBytes, kOffSFAR = kOffSFAS + kSfaMax, kOffSFB = kOffSFAR + kSfaMax;
+    static constexpr int kStageBytes = kOffSFB + kSfbMax;  // a multiple of 1024
+    static constexpr int kStages = (232448 - 2048) / kStageBytes;
+    static constexpr int kBarOff = kStages * kStageBytes;
+    static constexpr uint32_t kColSf0 = kNacc * BN;
+    static constexpr uint32_t kSfBufCols = (8 + 4 * kBlk) * kNvAtoms;  // A_S, A_R, then kBlk W blocks
+    static constexpr int kSfBufs = (int)((kTmemCols - kColSf0) / kSfBufCols) < 4 ? (int)((kTmemCols - kColSf0) / kSfBufCols) : 4;
+    // mbarriers: full[s], empty[s], sf_loaded[s], acc_full[a], acc_empty[a],
+    // drain, sf_full[b], sf_empty[b]; the tensor-memory slot follows.
+    static constexpr int kBarBytes = 8 * (3 * kStages + 2 * kNacc + 1 + 2 * kSfBufs);
+    static constexpr int kBarArea = (kBarBytes + 4 + 127) / 128 * 128;
+    static constexpr int kTableOff = kBarOff + kBarArea;
+    static constexpr int kSmemBytes = kTableOff + kTableBytes + 1024;  // barriers, table, alignment slack
+    // Split-K partial tile in the stage memory: 128 rows of BN fp32, rows
+    // padded by 16 bytes so that a warp's 32 rows hit different banks.
+    static constexpr uint32_t kPartStride = BN * 4 + 16;
+    static_assert(BN == 128 || BN == 256, "tile width");
+    static_assert(kStageBytes % 1024 == 0, "stage buffers must stay 1024-byte aligned");
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kBarBytes + 4 <= kBarArea, "barrier area");
+    static_assert(kSfBufs >= 2, "scale buffers");
+    static_assert(kColSf0 + kSfBufs * kSfBufCols <= kTmemCols, "tensor memory columns");
+    static_assert(kBM * kPartStride <= (uint32_t)(kStages * kStageBytes), "split-K partial fits the stages");
+};
+
+#ifndef SQ_GROUPED_BN
+#define SQ_GROUPED_BN 256
+#endif
+constexpr int kDenseBN = 256, kGroupedBN = SQ_GROUPED_BN;
 
 enum : unsigned {
     kSiteProducer = 0x101,
@@ -132,13 +159,13 @@ __device__ __forceinline__ float alpha_of_col(const GemmParams &p, float s_t, fl
     return __fmul_rn(s_t, p.s_tw[g]);
 }
 
-// Instruction descriptor of the block-scaled MMA (M = 128, N = 256, E2M1 x
+// Instruction descriptor of the block-scaled MMA (M = 128, N = BN, E2M1 x
 // E2M1, K-major A and B): A/B format E2M1 at bits 7-9 / 10-12, N >> 3 at
 // bits 17-22, scale format (0 = UE4M3, 1 = E8M0) at bit 23, M >> 4 at bits
 // 24-28; scale-factor byte selectors at bits 29-30 (A) and 4-5 (B).
-template <int FMT>
+template <int FMT, int BN>
 __device__ __forceinline__ uint32_t idesc_of(uint32_t sf_id) {
-    return (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((FMT == kFmtMX ? 1u : 0u) << 23) |
+    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((FMT == kFmtMX ? 1u : 0u) << 23) |
            ((uint32_t)(kBM >> 4) << 24) | (sf_id << 29) | (sf_id << 4);
 }
 
@@ -162,27 +189,28 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 // tensor scale, and output rows are remapped to grouped-row order.
 // EXT (dense only): fused-weight segments and/or a bias in the epilogue; the
 // plain instantiation keeps the epilogue without them.
-template <int FMT, bool GROUPED, bool EXT>
+template <int FMT, bool GROUPED, bool EXT, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constant__ CUtensorMap tm_ar,
                  const __grid_constant__ CUtensorMap tm_b, const GemmParams p) {
+    using C = TileCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
     const uint32_t sbase = smem_u32(smem);
     // barriers: full[s] (operands), empty[s], sf_loaded[s] (scale atoms),
-    // acc_full, acc_empty, drain, sf_full[b], sf_empty[b]
-    const uint32_t bar0 = sbase + kBarOff;
+    // acc_full[a], acc_empty[a], drain, sf_full[b], sf_empty[b]
+    const uint32_t bar0 = sbase + C::kBarOff;
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
-    auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-    auto sf_loaded_bar = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
-    const uint32_t acc_full = bar0 + 8u * (3 * kStages);
-    const uint32_t acc_empty = acc_full + 8u;
-    const uint32_t drain_bar = acc_full + 16u;
-    auto sf_full_bar = [&](int b) { return acc_full + 24u + 8u * b; };
-    auto sf_empty_bar = [&](int b) { return acc_full + 24u + 8u * (kSfBufs + b); };
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kBarOff + kBarBytes);
-    int32_t *tiles = reinterpret_cast<int32_t *>(smem + kTableOff);
+    auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
+    auto sf_loaded_bar = [&](int s) { return bar0 + 8u * (2 * C::kStages + s); };
+    auto acc_full_bar = [&](int a) { return bar0 + 8u * (3 * C::kStages + a); };
+    auto acc_empty_bar = [&](int a) { return bar0 + 8u * (3 * C::kStages + C::kNacc + a); };
+    const uint32_t drain_bar = bar0 + 8u * (3 * C::kStages + 2 * C::kNacc);
+    auto sf_full_bar = [&](int b) { return drain_bar + 8u + 8u * b; };
+    auto sf_empty_bar = [&](int b) { return drain_bar + 8u + 8u * (C::kSfBufs + b); };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kBarOff + C::kBarBytes);
+    int32_t *tiles = reinterpret_cast<int32_t *>(smem + C::kTableOff);
     int32_t *table_ok = tiles + (kGroupsMax + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -198,15 +226,17 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     constexpr uint32_t kSfBytes = 512u * kAtomsPerTile;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < C::kStages; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
             mbar_init(sf_loaded_bar(s), 1);
         }
-        mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 128);
+        for (int a = 0; a < C::kNacc; ++a) {
+            mbar_init(acc_full_bar(a), 1);
+            mbar_init(acc_empty_bar(a), 128);
+        }
         mbar_init(drain_bar, 1);
-        for (int b = 0; b < kSfBufs; ++b) {
+        for (int b = 0; b < C::kSfBufs; ++b) {
             mbar_init(sf_full_bar(b), 128);
             mbar_init(sf_empty_bar(b), 1);
         }
@@ -226,7 +256,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     // m tiles: 128-row tiles of the prep (grouped: of all groups; none if the
     // offsets are invalid)
     const int m_tiles = GROUPED ? (*table_ok ? tiles[p.groups] : 0) : (p.m_tok + kBM - 1) / kBM;
-    const int n_tiles = (p.n_out + kBN - 1) / kBN;
+    const int n_tiles = (p.n_out + C::kBN - 1) / C::kBN;
     const int num_tiles = m_tiles * n_tiles, kt_count = p.k / (2 * kBKBytes);
     // Tiles of this CTA: tile_begin, tile_begin + tile_step, ...; K steps
     // kt_begin .. kt_end - 1 of each. Split-K: one tile per cluster, one K
@@ -245,8 +275,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
 
     if (warp == 0) {
         if (lane == 0) {
-            int32_t last[kStages];
-            for (int s = 0; s < kStages; ++s) last[s] = -1;
+            int32_t last[C::kStages];
+            for (int s = 0; s < C::kStages; ++s) last[s] = -1;
             uint32_t it = 0;
             bool ok = true;
             for (int tile = tile_begin; ok && tile < num_tiles; tile += tile_step) {
@@ -254,38 +284,40 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                 const int grp = GROUPED ? group_of_tile(tiles, p.groups, mb) : 0;
                 const uint8_t *sfb = p.sfb + (GROUPED ? (int64_t)grp * p.w_gstride : 0);
                 for (int kt = kt_begin; kt < kt_end; ++kt, ++it) {
-                    const int s = (int)(it % kStages);
-                    const uint32_t ph = (it / kStages) & 1u;
+                    const int s = (int)(it % C::kStages);
+                    const uint32_t ph = (it / C::kStages) & 1u;
                     if (!mbar_wait(empty_bar(s), ph ^ 1u, p.status, kSiteProducer, p.wait_ns)) {
                         ok = false;
                         break;
                     }
                     const uint32_t fb = full_bar(s), lb = sf_loaded_bar(s);
-                    const uint32_t st = sbase + (uint32_t)(s * kStageBytes);
+                    const uint32_t st = sbase + (uint32_t)(s * C::kStageBytes);
                     // Scale atoms first, on their own barrier: the scale
                     // writers move them to tensor memory while the operand
                     // tiles are still in flight.
                     const int64_t a_off = ((int64_t)mb * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
-                    const int64_t b0 = ((int64_t)(2 * nb) * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
-                    const int64_t b1 = b0 + atoms_per_row_blk * 512;
-                    mbar_arrive_expect_tx(lb, 4 * kSfBytes);
-                    bulk_load(st + kOffSFAS, p.sfa_s + a_off, kSfBytes, lb);
-                    bulk_load(st + kOffSFAR, p.sfa_r + a_off, kSfBytes, lb);
-                    bulk_load(st + kOffSFB, sfb + b0, kSfBytes, lb);
-                    bulk_load(st + kOffSFB + kSfBytes, sfb + b1, kSfBytes, lb);
-                    mbar_arrive_expect_tx(fb, 2 * kABytes + kBBytes);
+                    const int64_t b0 =
+                        ((int64_t)(C::kBlk * nb) * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
+                    mbar_arrive_expect_tx(lb, (2 + C::kBlk) * kSfBytes);
+                    bulk_load(st + C::kOffSFAS, p.sfa_s + a_off, kSfBytes, lb);
+                    bulk_load(st + C::kOffSFAR, p.sfa_r + a_off, kSfBytes, lb);
+#pragma unroll
+                    for (int bk = 0; bk < C::kBlk; ++bk)  // the tile's 128-row W blocks
+                        bulk_load(st + C::kOffSFB + bk * kSfBytes, sfb + b0 + bk * atoms_per_row_blk * 512, kSfBytes,
+                                  lb);
+                    mbar_arrive_expect_tx(fb, 2 * kABytes + C::kBBytes);
                     tma_load_2d(st + kOffAS, &tm_as, kt * kBKBytes, mb * kBM, fb);
                     tma_load_2d(st + kOffAR, &tm_ar, kt * kBKBytes, mb * kBM, fb);
-                    if (GROUPED) tma_load_3d(st + kOffB, &tm_b, kt * kBKBytes, nb * kBN, grp, fb);
-                    else tma_load_2d(st + kOffB, &tm_b, kt * kBKBytes, nb * kBN, fb);
+                    if (GROUPED) tma_load_3d(st + kOffB, &tm_b, kt * kBKBytes, nb * C::kBN, grp, fb);
+                    else tma_load_2d(st + kOffB, &tm_b, kt * kBKBytes, nb * C::kBN, fb);
                     last[s] = (int32_t)it;
                 }
             }
             // Never leave the CTA with copies in flight.
-            for (int s = 0; s < kStages; ++s)
+            for (int s = 0; s < C::kStages; ++s)
                 if (last[s] >= 0) {
-                    drain_wait(full_bar(s), ((uint32_t)last[s] / kStages) & 1u, kDrainNs);
-                    drain_wait(sf_loaded_bar(s), ((uint32_t)last[s] / kStages) & 1u, kDrainNs);
+                    drain_wait(full_bar(s), ((uint32_t)last[s] / C::kStages) & 1u, kDrainNs);
+                    drain_wait(sf_loaded_bar(s), ((uint32_t)last[s] / C::kStages) & 1u, kDrainNs);
                 }
         }
         __syncwarp();
@@ -293,41 +325,48 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         if (lane == 0) {
             uint32_t it = 0, tile_iter = 0;
             for (int tile = tile_begin; tile < num_tiles; tile += tile_step, ++tile_iter) {
-                if (!mbar_wait(acc_empty, (tile_iter & 1u) ^ 1u, p.status, kSiteMmaAcc, p.wait_ns)) break;
+                // accumulator of this tile (two in turn at BN = 128)
+                const int ab = (int)(tile_iter % C::kNacc);
+                const uint32_t acc_par = ((tile_iter / C::kNacc) & 1u) ^ 1u;
+                if (!mbar_wait(acc_empty_bar(ab), acc_par, p.status, kSiteMmaAcc, p.wait_ns)) break;
                 tc_fence_after();
+                const uint32_t dacc = tmem + (uint32_t)(ab * BN);
                 bool ok = true;
                 for (int kt = kt_begin; kt < kt_end; ++kt, ++it) {
-                    const int s = (int)(it % kStages);
-                    const uint32_t ph = (it / kStages) & 1u;
+                    const int s = (int)(it % C::kStages);
+                    const uint32_t ph = (it / C::kStages) & 1u;
                     if (!mbar_wait(full_bar(s), ph, p.status, kSiteMmaFull, p.wait_ns)) {
                         ok = false;
                         break;
                     }
-                    const int sb = (int)(it % kSfBufs);  // scale buffer of this stage
-                    if (!mbar_wait(sf_full_bar(sb), (it / kSfBufs) & 1u, p.status, kSiteMmaScales, p.wait_ns)) {
+                    const int sb = (int)(it % C::kSfBufs);  // scale buffer of this stage
+                    if (!mbar_wait(sf_full_bar(sb), (it / C::kSfBufs) & 1u, p.status, kSiteMmaScales, p.wait_ns)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t st = sbase + (uint32_t)(s * kStageBytes);
-                    const uint32_t sf = tmem + kColSf0 + kSfBufCols * (uint32_t)sb;
+                    const uint32_t st = sbase + (uint32_t)(s * C::kStageBytes);
+                    const uint32_t sf = tmem + C::kColSf0 + C::kSfBufCols * (uint32_t)sb;
                     const uint64_t da_s = desc_operand(st + kOffAS);
                     const uint64_t da_r = desc_operand(st + kOffAR);
                     const uint64_t db = desc_operand(st + kOffB);
 #pragma unroll
                     for (int j = 0; j < kMmaPerStage; ++j) {  // MMAs of K = 64 (32 bytes) per K tile
                         const uint32_t acc = (kt != kt_begin || j != 0) ? 1u : 0u;
+                        // W scales: 4 columns per 128-row block per atom, the
+                        // tile's blocks side by side
                         if (FMT == kFmtNV) {
-                            const uint32_t idesc = idesc_of<FMT>(0);
-                            tc_mma_nvf4(tmem, da_s + 2 * j, db + 2 * j, idesc, sf + kSfaS + 4 * j, sf + kSfb + 8 * j, acc);
-                            tc_mma_nvf4(tmem, da_r + 2 * j, db + 2 * j, idesc, sf + kSfaR + 4 * j, sf + kSfb + 8 * j, 1u);
+                            const uint32_t idesc = idesc_of<FMT, BN>(0);
+                            const uint32_t b_col = 4 * C::kBlk * j;
+                            tc_mma_nvf4(dacc, da_s + 2 * j, db + 2 * j, idesc, sf + kSfaS + 4 * j, sf + kSfb + b_col, acc);
+                            tc_mma_nvf4(dacc, da_r + 2 * j, db + 2 * j, idesc, sf + kSfaR + 4 * j, sf + kSfb + b_col, 1u);
                         } else {
                             const uint32_t sf_id = (uint32_t)(j & 1) * 2u;  // 2 scales per row per MMA
-                            const uint32_t idesc = idesc_of<FMT>(sf_id);
-                            const uint32_t a_col = 4 * (j >> 1), b_col = 8 * (j >> 1);
-                            tc_mma_mxf4(tmem, da_s + 2 * j, db + 2 * j, idesc, (sf + kSfaS + a_col) | (sf_id << 30),
+                            const uint32_t idesc = idesc_of<FMT, BN>(sf_id);
+                            const uint32_t a_col = 4 * (j >> 1), b_col = 4 * C::kBlk * (j >> 1);
+                            tc_mma_mxf4(dacc, da_s + 2 * j, db + 2 * j, idesc, (sf + kSfaS + a_col) | (sf_id << 30),
                                         (sf + kSfb + b_col) | (sf_id << 30), acc);
-                            tc_mma_mxf4(tmem, da_r + 2 * j, db + 2 * j, idesc, (sf + kSfaR + a_col) | (sf_id << 30),
+                            tc_mma_mxf4(dacc, da_r + 2 * j, db + 2 * j, idesc, (sf + kSfaR + a_col) | (sf_id << 30),
                                         (sf + kSfb + b_col) | (sf_id << 30), 1u);
                         }
                     }
@@ -335,7 +374,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                     tc_commit(sf_empty_bar(sb));  // and the scale buffer
                 }
                 if (!ok) break;
-                tc_commit(acc_full);
+                tc_commit(acc_full_bar(ab));
             }
             tc_commit(drain_bar);  // every MMA of this thread done before exit
             drain_wait(drain_bar, 0, kDrainNs);
@@ -357,21 +396,22 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         const int my_tiles = tile_begin < num_tiles ? (num_tiles - 1 - tile_begin) / tile_step + 1 : 0;
         const uint32_t total_stages = (uint32_t)my_tiles * (uint32_t)kt_n;
         for (uint32_t it = 0; it < total_stages; ++it) {
-            const int s = (int)(it % kStages);
-            const int b = (int)(it % kSfBufs);
-            const bool w1 = mbar_wait(sf_loaded_bar(s), (it / kStages) & 1u, p.status, kSiteScaleFull, p.wait_ns);
-            const bool w2 = w1 && mbar_wait(sf_empty_bar(b), ((it / kSfBufs) & 1u) ^ 1u, p.status, kSiteScaleEmpty,
+            const int s = (int)(it % C::kStages);
+            const int b = (int)(it % C::kSfBufs);
+            const bool w1 = mbar_wait(sf_loaded_bar(s), (it / C::kStages) & 1u, p.status, kSiteScaleFull, p.wait_ns);
+            const bool w2 = w1 && mbar_wait(sf_empty_bar(b), ((it / C::kSfBufs) & 1u) ^ 1u, p.status, kSiteScaleEmpty,
                                             p.wait_ns);
             if (!__all_sync(0xFFFFFFFFu, w2)) break;  // warp-uniform: tcgen05.st is .aligned
             tc_fence_after();
-            const uint32_t st = sbase + (uint32_t)(s * kStageBytes) + (uint32_t)lane * 16u;
-            const uint32_t sf = tmem + lane_base + kColSf0 + kSfBufCols * (uint32_t)b;
+            const uint32_t st = sbase + (uint32_t)(s * C::kStageBytes) + (uint32_t)lane * 16u;
+            const uint32_t sf = tmem + lane_base + C::kColSf0 + C::kSfBufCols * (uint32_t)b;
 #pragma unroll
             for (int a = 0; a < kAtomsPerTile; ++a) {
-                tmem_st4(sf + kSfaS + 4 * a, lds128(st + kOffSFAS + 512 * a));
-                tmem_st4(sf + kSfaR + 4 * a, lds128(st + kOffSFAR + 512 * a));
-                tmem_st4(sf + kSfb + 8 * a, lds128(st + kOffSFB + 512 * a));
-                tmem_st4(sf + kSfb + 8 * a + 4, lds128(st + kOffSFB + kSfBytes + 512 * a));
+                tmem_st4(sf + kSfaS + 4 * a, lds128(st + C::kOffSFAS + 512 * a));
+                tmem_st4(sf + kSfaR + 4 * a, lds128(st + C::kOffSFAR + 512 * a));
+#pragma unroll
+                for (int bk = 0; bk < C::kBlk; ++bk)
+                    tmem_st4(sf + kSfb + 4 * C::kBlk * a + 4 * bk, lds128(st + C::kOffSFB + bk * kSfBytes + 512 * a));
             }
             tmem_st_wait();
             tc_fence_before();
@@ -397,20 +437,23 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                 alpha = __fmul_rn(s_t, *reinterpret_cast<const float *>(
                                            reinterpret_cast<const uint8_t *>(p.s_tw) + (int64_t)grp * p.w_gstride));
             }
-            const bool got = mbar_wait(acc_full, tile_iter & 1u, p.status, kSiteEpilogue, p.wait_ns);
+            const int ab = (int)(tile_iter % C::kNacc);  // the accumulator this tile used
+            const bool got =
+                mbar_wait(acc_full_bar(ab), (tile_iter / C::kNacc) & 1u, p.status, kSiteEpilogue, p.wait_ns);
             if (!__all_sync(0xFFFFFFFFu, got)) break;  // warp-uniform: tcgen05.ld is .aligned
             tc_fence_after();
+            const uint32_t acc_base = tmem + lane_base + (uint32_t)(ab * BN);
             if (split) {
                 // Split-K: the fp32 partial tile (rows below m_tok) goes to
                 // this CTA's stage memory, which no copy or MMA uses any
                 // more; the cluster reduces it at the end of the kernel.
                 const int row_local = q * 32 + lane;
                 const bool keep = (int64_t)mb * kBM + row_local < p.m_tok;
-                const uint32_t dst = sbase + (uint32_t)row_local * kPartStride;
+                const uint32_t dst = sbase + (uint32_t)row_local * C::kPartStride;
 #pragma unroll
-                for (int cc = 0; cc < kBN / 32; ++cc) {
+                for (int cc = 0; cc < C::kBN / 32; ++cc) {
                     uint32_t r[32];
-                    tmem_ld32(tmem + lane_base + (uint32_t)(cc * 32), r);
+                    tmem_ld32(acc_base + (uint32_t)(cc * 32), r);
                     tmem_ld_wait();
                     if (keep) {
 #pragma unroll
@@ -425,14 +468,14 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             // RN16(RN32(RN32(acc * alpha) + bias)) in scalar operations, so
             // that no multiply is fused into the add. Fused weights: alpha
             // per 32-column chunk (a chunk never spans two segments).
-            uint32_t h[kBN / 32][16];
+            uint32_t h[C::kBN / 32][16];
 #pragma unroll
-            for (int cc = 0; cc < kBN / 32; ++cc) {
-                const int col0 = nb * kBN + cc * 32;
+            for (int cc = 0; cc < C::kBN / 32; ++cc) {
+                const int col0 = nb * C::kBN + cc * 32;
                 float a_cc = alpha;
                 if constexpr (EXT) a_cc = alpha_of_col(p, s_t, alpha, col0);
                 uint32_t r[32];
-                tmem_ld32(tmem + lane_base + (uint32_t)(cc * 32), r);
+                tmem_ld32(acc_base + (uint32_t)(cc * 32), r);
                 tmem_ld_wait();
                 if (EXT && p.bias != nullptr && col0 < p.n_out) {
                     const uint4 *bp = reinterpret_cast<const uint4 *>(p.bias + col0);  // same for every lane
@@ -462,7 +505,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                 }
             }
             tc_fence_before();
-            mbar_arrive(acc_empty);
+            mbar_arrive(acc_empty_bar(ab));
             int64_t row, row_end;  // output row of this lane; end of the tile's valid rows
             if constexpr (GROUPED) {
                 // looked up again rather than kept live across the drain (register pressure)
@@ -482,8 +525,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             // main loop's length (about 60 ns per K step, at most 1 us); the
             // CTA's last tile stores at once.
 #pragma unroll
-            for (int cc = 0; cc < kBN / 32; ++cc) {
-                const int col0 = nb * kBN + cc * 32;
+            for (int cc = 0; cc < C::kBN / 32; ++cc) {
+                const int col0 = nb * C::kBN + cc * 32;
                 if (row < row_end && col0 < p.n_out) {
                     // two full 32-byte sectors (the output base is 32-byte aligned,
                     // rows are multiples of 64 bytes)
@@ -492,7 +535,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                     stg256(dst + 16, h[cc][8], h[cc][9], h[cc][10], h[cc][11], h[cc][12], h[cc][13], h[cc][14],
                            h[cc][15]);
                 }
-                if (cc + 1 < kBN / 32 && pause_ns) __nanosleep(pause_ns);
+                if (cc + 1 < C::kBN / 32 && pause_ns) __nanosleep(pause_ns);
             }
         }
     }
@@ -506,15 +549,15 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         cluster_sync();  // every partial is in its CTA's shared memory
         if (warp >= 2 && warp <= 5 && tile_begin < num_tiles) {
             const int mb = tile_begin / n_tiles, nb = tile_begin % n_tiles;
-            const int S = p.split, cols = kBN / S, groups4 = cols / 4;
+            const int S = p.split, cols = C::kBN / S, groups4 = cols / 4;
             const int valid = (int)min((int64_t)kBM, (int64_t)p.m_tok - (int64_t)mb * kBM);
             const float s_t = *p.s_t;
             const float alpha0 = __fmul_rn(s_t, *p.s_tw);
             for (int item = (warp - 2) * 32 + lane; item < valid * groups4; item += 128) {
                 const int r = item / groups4, col = rank * cols + (item % groups4) * 4;
-                if (nb * kBN + col >= p.n_out) continue;
-                const float alpha = EXT ? alpha_of_col(p, s_t, alpha0, nb * kBN + col) : alpha0;
-                const uint32_t off = sbase + (uint32_t)r * kPartStride + (uint32_t)col * 4u;
+                if (nb * C::kBN + col >= p.n_out) continue;
+                const float alpha = EXT ? alpha_of_col(p, s_t, alpha0, nb * C::kBN + col) : alpha0;
+                const uint32_t off = sbase + (uint32_t)r * C::kPartStride + (uint32_t)col * 4u;
                 float4 acc = ld_cluster_f4(mapa_shared(off, 0));
                 for (int c = 1; c < S; ++c) {
                     const float4 v = ld_cluster_f4(mapa_shared(off, (uint32_t)c));
@@ -526,7 +569,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                 float4 y = make_float4(__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha), __fmul_rn(acc.z, alpha),
                                        __fmul_rn(acc.w, alpha));
                 if (EXT && p.bias != nullptr) {
-                    const uint2 bw = *reinterpret_cast<const uint2 *>(p.bias + nb * kBN + col);
+                    const uint2 bw = *reinterpret_cast<const uint2 *>(p.bias + nb * C::kBN + col);
                     const float2 b01 = __half22float2(*reinterpret_cast<const __half2 *>(&bw.x));
                     const float2 b23 = __half22float2(*reinterpret_cast<const __half2 *>(&bw.y));
                     y = make_float4(__fadd_rn(y.x, b01.x), __fadd_rn(y.y, b01.y), __fadd_rn(y.z, b23.x),
@@ -534,7 +577,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                 }
                 __half2 h0 = __floats2half2_rn(y.x, y.y);
                 __half2 h1 = __floats2half2_rn(y.z, y.w);
-                *reinterpret_cast<uint2 *>(p.out + ((int64_t)mb * kBM + r) * p.n_out + nb * kBN + col) =
+                *reinterpret_cast<uint2 *>(p.out + ((int64_t)mb * kBM + r) * p.n_out + nb * C::kBN + col) =
                     make_uint2(*reinterpret_cast<uint32_t *>(&h0), *reinterpret_cast<uint32_t *>(&h1));
             }
         }
@@ -620,27 +663,28 @@ static bool make_grouped_code_map(CUtensorMap *tm, const void *base, uint64_t ro
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, bool GROUPED, bool EXT>
+template <int FMT, bool GROUPED, bool EXT, int BN>
 static sharq_status set_gemm_attrs() {
     static bool attr_done[64] = {};
     int dev = 0;
     SQ_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
     if (!attr_done[dev]) {
-        SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<FMT, GROUPED, EXT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes));
+        SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<FMT, GROUPED, EXT, BN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TileCfg<BN>::kSmemBytes));
         attr_done[dev] = true;
     }
     return SHARQ_OK;
 }
 
-template <int FMT, bool GROUPED, bool EXT>
+template <int FMT, bool GROUPED, bool EXT, int BN>
 static sharq_status launch_gemm(LaunchCtx &ctx, const CUtensorMap &tm_as, const CUtensorMap &tm_ar,
                                 const CUtensorMap &tm_b, const GemmParams &gp, int64_t max_tiles) {
-    sharq_status st = set_gemm_attrs<FMT, GROUPED, EXT>();
+    sharq_status st = set_gemm_attrs<FMT, GROUPED, EXT, BN>();
     if (st != SHARQ_OK) return st;
     const unsigned grid = (unsigned)(max_tiles < ctx.num_sms ? max_tiles : ctx.num_sms);
-    dual_gemm_kernel<FMT, GROUPED, EXT><<<grid, kGemmThreads, kSmemBytes, ctx.stream>>>(tm_as, tm_ar, tm_b, gp);
+    dual_gemm_kernel<FMT, GROUPED, EXT, BN>
+        <<<grid, kGemmThreads, TileCfg<BN>::kSmemBytes, ctx.stream>>>(tm_as, tm_ar, tm_b, gp);
     ctx.launches++;
     SQ_CUDA_TRY(cudaGetLastError());
     return SHARQ_OK;
@@ -650,13 +694,13 @@ static sharq_status launch_gemm(LaunchCtx &ctx, const CUtensorMap &tm_as, const 
 template <int FMT, bool EXT>
 static sharq_status launch_gemm_split(LaunchCtx &ctx, const CUtensorMap &tm_as, const CUtensorMap &tm_ar,
                                       const CUtensorMap &tm_b, const GemmParams &gp, int64_t tiles) {
-    sharq_status st = set_gemm_attrs<FMT, false, EXT>();
+    sharq_status st = set_gemm_attrs<FMT, false, EXT, kDenseBN>();
     if (st != SHARQ_OK) return st;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3((unsigned)(tiles * gp.split), 1, 1);
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
-    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.dynamicSmemBytes = TileCfg<kDenseBN>::kSmemBytes;
     cfg.stream = ctx.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -665,7 +709,7 @@ static sharq_status launch_gemm_split(LaunchCtx &ctx, const CUtensorMap &tm_as, 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    SQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, dual_gemm_kernel<FMT, false, EXT>, tm_as, tm_ar, tm_b, gp));
+    SQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, dual_gemm_kernel<FMT, false, EXT, kDenseBN>, tm_as, tm_ar, tm_b, gp));
     ctx.launches++;
     SQ_CUDA_TRY(cudaGetLastError());
     return SHARQ_OK;
@@ -680,12 +724,12 @@ static int active_clusters(int split) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || split > kMaxSplit) return 0;
     if (!known[dev][split]) {
-        if (set_gemm_attrs<FMT, false, false>() != SHARQ_OK) return 0;
+        if (set_gemm_attrs<FMT, false, false, kDenseBN>() != SHARQ_OK) return 0;
         cudaLaunchConfig_t cfg;
         memset(&cfg, 0, sizeof(cfg));
         cfg.gridDim = dim3((unsigned)split, 1, 1);
         cfg.blockDim = dim3(kGemmThreads, 1, 1);
-        cfg.dynamicSmemBytes = kSmemBytes;
+        cfg.dynamicSmemBytes = TileCfg<kDenseBN>::kSmemBytes;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = (unsigned)split;
@@ -694,7 +738,7 @@ static int active_clusters(int split) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, dual_gemm_kernel<FMT, false, false>, &cfg) != cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&n, dual_gemm_kernel<FMT, false, false, kDenseBN>, &cfg) != cudaSuccess) {
             cudaGetLastError();
             n = 0;
         }
@@ -741,11 +785,11 @@ sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &
     CUtensorMap tm_as, tm_ar, tm_b;
     if (!make_code_map(&tm_as, P.s_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
         !make_code_map(&tm_ar, P.r_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
-        !make_code_map(&tm_b, W.codes, (uint64_t)(W.k / 2), (uint64_t)W.n_out, kBN))
+        !make_code_map(&tm_b, W.codes, (uint64_t)(W.k / 2), (uint64_t)W.n_out, kDenseBN))
         return SHARQ_ERR_CUDA;
     GemmParams gp = gemm_params(ctx, P, W, out);
     gp.bias = (const __half *)bias;
-    const int64_t tiles = ((P.m_tok + kBM - 1) / kBM) * ((W.n_out + kBN - 1) / kBN);
+    const int64_t tiles = ((P.m_tok + kBM - 1) / kBM) * ((W.n_out + kDenseBN - 1) / kDenseBN);
     const int kt_count = (int)(P.k / (2 * kBKBytes));
     gp.split = P.fmt == kFmtNV ? choose_split<kFmtNV>(ctx, tiles, kt_count) : choose_split<kFmtMX>(ctx, tiles, kt_count);
     // the extended epilogue (fused segments, bias) only where needed
@@ -758,10 +802,10 @@ sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &
                                : launch_gemm_split<kFmtMX, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
     }
     if (ext)
-        return P.fmt == kFmtNV ? launch_gemm<kFmtNV, false, true>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
-                               : launch_gemm<kFmtMX, false, true>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
-    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, false, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
-                           : launch_gemm<kFmtMX, false, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
+        return P.fmt == kFmtNV ? launch_gemm<kFmtNV, false, true, kDenseBN>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
+                               : launch_gemm<kFmtMX, false, true, kDenseBN>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
+    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, false, false, kDenseBN>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
+                           : launch_gemm<kFmtMX, false, false, kDenseBN>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
 }
 
 sharq_status launch_linear_grouped(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, const int32_t *offsets,
@@ -770,7 +814,7 @@ sharq_status launch_linear_grouped(LaunchCtx &ctx, const sharq_prep &P, const sh
     if (!make_code_map(&tm_as, P.s_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
         !make_code_map(&tm_ar, P.r_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
         !make_grouped_code_map(&tm_b, W.codes, (uint64_t)(W.k / 2), (uint64_t)W.n_out, (uint64_t)groups,
-                               (uint64_t)w_gstride, kBN))
+                               (uint64_t)w_gstride, kGroupedBN))
         return SHARQ_ERR_CUDA;
     GemmParams gp = gemm_params(ctx, P, W, out);
     gp.segs = 1;  // stacked experts, never fused segments
@@ -779,10 +823,10 @@ sharq_status launch_linear_grouped(LaunchCtx &ctx, const sharq_prep &P, const sh
     gp.rows = rows;
     gp.w_gstride = w_gstride;
     // at most P.m_tok / 128 m tiles (the device checks the offsets against it)
-    const int64_t tiles = (P.m_tok / kBM) * ((W.n_out + kBN - 1) / kBN);
+    const int64_t tiles = (P.m_tok / kBM) * ((W.n_out + kGroupedBN - 1) / kGroupedBN);
     if (tiles == 0) return SHARQ_OK;
-    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, true, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
-                           : launch_gemm<kFmtMX, true, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
+    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, true, false, kGroupedBN>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
+                           : launch_gemm<kFmtMX, true, false, kGroupedBN>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
 }
 
 }  // namespace sq

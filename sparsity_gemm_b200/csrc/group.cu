@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kGatherThreads) gather_kernel(const GatherPara
     __syncthreads();
 
     const int64_t d0 = (int64_t)tile * 128;  // first destination row
-    const int64_t row_bytes = p.k / 2, chunks = p.k / 32;  // 16-byte chunks per row
+    const int64_t chunks = p.k / 32;  // 16-byte chunks per row (p.k / 2 bytes)
     // Codes: (row, chunk) pairs of the tile over all threads, consecutive
     // threads on consecutive chunks of a row; kCopyUnroll loads per operand
     // in flight before the stores (the copy is latency-bound).
