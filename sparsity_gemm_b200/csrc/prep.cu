@@ -542,29 +542,42 @@ __device__ __forceinline__ uint32_t keep_mask_42(const float (&v)[kUnit]) {
     return keep;
 }
 
-// Step d and scale code of an NVFP4 block as block_step does, with the
-// division a / c6 by the reciprocal method when y6 = RN(1/c6) != 0 (the
-// caller sets y6 = 0 unless c6 is in [2^-90, 2^90]): exact for quotients
-// >= 2^-11, and every smaller quotient has UE4M3 code 0 either way (the
-// code's smallest rounding boundary is 2^-10). MXFP4 takes block_step.
+// Step d = RN32(value(code) s_t) and, for d in [2^-90, 2^90], y = RN(1/d)
+// (else 0) of every UE4M3 scale code: one table per CTA, so that a block's
+// step and reciprocal are one shared-memory load instead of a conversion, a
+// product and a correctly rounded reciprocal per block.
 template <int FMT>
-__device__ __forceinline__ float block_step_rcp(float a, float s_t, float c6, float y6, uint32_t &code) {
-    if (FMT == kFmtNV) {
-        const float u = y6 != 0.0f ? div1(a, c6, y6) : __fdiv_rn(a, c6);
-        code = ue4m3_code(u);
-        return __fmul_rn(ue4m3_value(code), s_t);
-    }
-    return block_step<FMT>(a, s_t, c6, code);
+__device__ __forceinline__ void build_step_table(float2 *tab, float s_t) {
+    if constexpr (FMT == kFmtNV)
+        for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+            const float d = __fmul_rn(ue4m3_value((uint32_t)c), s_t);
+            tab[c] = make_float2(d, (d >= 0x1p-90f && d <= 0x1p90f) ? __frcp_rn(d) : 0.0f);
+        }
 }
 
 template <int FMT>
-__device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, float c6, float y6,
+__device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, float c6, float y6, const float2 *tab,
                                             uint32_t &scale_code, uint32_t &codes_lo, uint32_t &codes_hi) {
     float a = 0.0f;
 #pragma unroll
     for (int i = 0; i < kUnit; ++i) a = fmaxf(a, fabsf(v[i]));
     if (FMT == kFmtMX) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
-    const float d = block_step_rcp<FMT>(a, s_t, c6, y6, scale_code);
+    // Step d and scale code as block_step gives them. NVFP4: the division
+    // a / c6 by the reciprocal method when y6 = RN(1/c6) != 0 (the caller
+    // sets y6 = 0 unless c6 is in [2^-90, 2^90]), exact for quotients >=
+    // 2^-11, and every smaller quotient has UE4M3 code 0 either way (the
+    // code's smallest rounding boundary is 2^-10); d and y = RN(1/d) from
+    // the step table.
+    float d, y = 0.0f;
+    if (FMT == kFmtNV) {
+        const float u = y6 != 0.0f ? div1(a, c6, y6) : __fdiv_rn(a, c6);
+        scale_code = ue4m3_code(u);
+        const float2 dy = tab[scale_code];
+        d = dy.x;
+        y = dy.y;
+    } else {
+        d = block_step<FMT>(a, s_t, c6, scale_code);
+    }
     codes_lo = 0u;
     codes_hi = 0u;
     if (d != 0.0f) {
@@ -581,8 +594,7 @@ __device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, 
                 for (int p = 0; p < 4; ++p) q[p] = mul2(pk2(v[8 * h + 2 * p], v[8 * h + 2 * p + 1]), y2);
                 c[h] = e2m1x8(q, v + 8 * h);
             }
-        } else if (d >= 0x1p-90f && d <= 0x1p90f) {
-            const float y = __frcp_rn(d);
+        } else if (y != 0.0f) {
             const uint64_t y2 = pk2(y, y), nd2 = pk2(-d, -d), d2 = pk2(d, d);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -623,8 +635,8 @@ struct EncodeArgs {
 // `dst` (-1: the same row).
 // NK > 0: n fixed at compile time (the 2:4 default takes its own mask).
 template <int FMT, int M, int NK>
-__device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t *lut, int64_t row, int64_t u,
-                                            bool active, float s_t, float c6, float y6, int64_t dst = -1,
+__device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t *lut, const float2 *tab, int64_t row,
+                                            int64_t u, bool active, float s_t, float c6, float y6, int64_t dst = -1,
                                             bool pad_codes = false) {
     constexpr int IB = M <= 2 ? 1 : M <= 4 ? 2 : M <= 8 ? 3 : 4;
     constexpr int G = kUnit / M;  // mask groups per unit
@@ -700,7 +712,7 @@ __device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t 
 #pragma unroll
     for (int i = 0; i < kUnit; ++i) s[i] = ((keep >> i) & 1u) ? v[i] : 0.0f;
     uint32_t s_scale, s_lo, s_hi;
-    const float ds = quantize16<FMT>(s, s_t, c6, y6, s_scale, s_lo, s_hi);
+    const float ds = quantize16<FMT>(s, s_t, c6, y6, tab, s_scale, s_lo, s_hi);
 
     // Residual against the quantized backbone: R = RN32(X_ln - RN32(value * d)).
     // Scalar intrinsics: the product must be rounded before the subtraction.
@@ -713,7 +725,7 @@ __device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t 
         r[i + 1] = __fsub_rn(v[i + 1], __fmul_rn(cv.y, ds));
     }
     uint32_t r_scale, r_lo, r_hi;
-    quantize16<FMT>(r, s_t, c6, y6, r_scale, r_lo, r_hi);
+    quantize16<FMT>(r, s_t, c6, y6, tab, r_scale, r_lo, r_hi);
 
     // Mask metadata: each group holds exactly n kept positions, so its
     // field sits at a fixed offset of the unit's bit range.
@@ -792,6 +804,9 @@ prep_encode_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ 
     const float c6 = __fmul_rn(6.0f, s_t);
     const float y6 = (FMT == kFmtNV && c6 >= 0x1p-90f && c6 <= 0x1p90f) ? __frcp_rn(c6) : 0.0f;
     if (blockIdx.x == 0 && threadIdx.x == 0) *s_t_out = s_t;
+    __shared__ float2 tab[128];  // NVFP4 steps and reciprocals by scale code
+    build_step_table<FMT>(tab, s_t);
+    __syncthreads();
 
     const int64_t upr = k / kUnit;                 // units per row
     const int64_t nblk = k / (FMT == kFmtNV ? 16 : 32);
@@ -814,7 +829,7 @@ prep_encode_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ 
             u_i -= upr;
             ++row_i;
         }
-        encode_unit<FMT, M, NK>(ea, lut, row, u, active, s_t, c6, y6);
+        encode_unit<FMT, M, NK>(ea, lut, tab, row, u, active, s_t, c6, y6);
     }
 }
 
@@ -868,6 +883,9 @@ prep_encode_grouped_kernel(const EncodeArgs ea, const unsigned *__restrict__ ama
     const float c6 = __fmul_rn(6.0f, s_t);
     const float y6 = (FMT == kFmtNV && c6 >= 0x1p-90f && c6 <= 0x1p90f) ? __frcp_rn(c6) : 0.0f;
     if (blockIdx.x == 0 && threadIdx.x == 0) *s_t_out = s_t;
+    __shared__ float2 tab[128];  // NVFP4 steps and reciprocals by scale code
+    build_step_table<FMT>(tab, s_t);
+    __syncthreads();
     constexpr int IBm = M <= 2 ? 1 : M <= 4 ? 2 : M <= 8 ? 3 : 4;
     const int unit_meta_bits = (kUnit / M) * ea.n * IBm;
 
@@ -907,7 +925,7 @@ prep_encode_grouped_kernel(const EncodeArgs ea, const unsigned *__restrict__ ama
                                                        unit_meta_bits / 8);
             continue;
         }
-        encode_unit<FMT, M, NK>(ea, lut, src, u, active, s_t, c6, y6, d, true);
+        encode_unit<FMT, M, NK>(ea, lut, tab, src, u, active, s_t, c6, y6, d, true);
     }
 }
 
@@ -1076,12 +1094,15 @@ prep_small_kernel(const EncodeArgs a, float eps, int64_t sf_rows, float *__restr
         words[0] = amax;
         words[1] = s_t;
     }
+    __shared__ float2 tab[128];  // NVFP4 steps and reciprocals by scale code
+    build_step_table<FMT>(tab, s_t);
+    __syncthreads();
     const int64_t upr = k / kUnit, total = m_tok * upr;
     for (int64_t base = (int64_t)rank * kSmallThreads; base < total; base += gstride) {
         const int64_t t = base + tid;
         const bool active = t < total;
         const int64_t row = active ? t / upr : m_tok, u = active ? t - (t / upr) * upr : 0;
-        encode_unit<FMT, M, 0>(a, lut, row, u, active, s_t, c6, y6);
+        encode_unit<FMT, M, 0>(a, lut, tab, row, u, active, s_t, c6, y6);
     }
     cluster_sync();  // no CTA leaves while its row amax may still be read
 }
