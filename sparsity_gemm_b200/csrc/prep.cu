@@ -543,20 +543,32 @@ __device__ __forceinline__ uint32_t keep_mask_42(const float (&v)[kUnit]) {
 }
 
 // Step d = RN32(value(code) s_t) and, for d in [2^-90, 2^90], y = RN(1/d)
-// (else 0) of every UE4M3 scale code: one table per CTA, so that a block's
-// step and reciprocal are one shared-memory load instead of a conversion, a
-// product and a correctly rounded reciprocal per block.
+// and the bracketing factors RN(y (1 -/+ 2^-21)) of e2m1x8_div (else all
+// three 0) of every UE4M3 scale code: one table per CTA, so that a block's
+// step and reciprocals are one shared-memory load instead of a conversion,
+// a product and a correctly rounded reciprocal per block.
 template <int FMT>
-__device__ __forceinline__ void build_step_table(float2 *tab, float s_t) {
+__device__ __forceinline__ void build_step_table(float4 *tab, float s_t) {
     if constexpr (FMT == kFmtNV)
         for (int c = threadIdx.x; c < 128; c += blockDim.x) {
             const float d = __fmul_rn(ue4m3_value((uint32_t)c), s_t);
-            tab[c] = make_float2(d, (d >= 0x1p-90f && d <= 0x1p90f) ? __frcp_rn(d) : 0.0f);
+            const float y = (d >= 0x1p-90f && d <= 0x1p90f) ? __frcp_rn(d) : 0.0f;
+            tab[c] = make_float4(d, y, __fmul_rn(y, 1.0f - 0x1p-21f), __fmul_rn(y, 1.0f + 0x1p-21f));
         }
 }
 
+// Nibble mask of eight keep bits (bit i of k sets nibble i to 0xF): three
+// spreading steps whose shifted copies never overlap, so each multiply is
+// an OR of shifts.
+__device__ __forceinline__ uint32_t nibble_mask8(uint32_t k) {
+    uint32_t x = ((k & 0xFFu) * 0x1001u) & 0x000F000Fu;  // bits 0-3 at 0-3, bits 4-7 at 16-19
+    x = (x * 0x41u) & 0x03030303u;                        // two bits per byte
+    x = (x * 0x9u) & 0x11111111u;                         // one bit per nibble
+    return x * 0xFu;
+}
+
 template <int FMT>
-__device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, float c6, float y6, const float2 *tab,
+__device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, float c6, float y6, const float4 *tab,
                                             uint32_t &scale_code, uint32_t &codes_lo, uint32_t &codes_hi) {
     float a = 0.0f;
 #pragma unroll
@@ -566,15 +578,17 @@ __device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, 
     // a / c6 by the reciprocal method when y6 = RN(1/c6) != 0 (the caller
     // sets y6 = 0 unless c6 is in [2^-90, 2^90]), exact for quotients >=
     // 2^-11, and every smaller quotient has UE4M3 code 0 either way (the
-    // code's smallest rounding boundary is 2^-10); d and y = RN(1/d) from
-    // the step table.
-    float d, y = 0.0f;
+    // code's smallest rounding boundary is 2^-10); d, y = RN(1/d) and the
+    // bracketing factors from the step table.
+    float d, y = 0.0f, ylo = 0.0f, yhi = 0.0f;
     if (FMT == kFmtNV) {
         const float u = y6 != 0.0f ? div1(a, c6, y6) : __fdiv_rn(a, c6);
         scale_code = ue4m3_code(u);
-        const float2 dy = tab[scale_code];
+        const float4 dy = tab[scale_code];
         d = dy.x;
         y = dy.y;
+        ylo = dy.z;
+        yhi = dy.w;
     } else {
         d = block_step<FMT>(a, s_t, c6, scale_code);
     }
@@ -597,12 +611,7 @@ __device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, 
         } else if (y != 0.0f) {
             const uint64_t y2 = pk2(y, y), nd2 = pk2(-d, -d), d2 = pk2(d, d);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint64_t q[4];
-#pragma unroll
-                for (int p = 0; p < 4; ++p) q[p] = div2(pk2(v[8 * h + 2 * p], v[8 * h + 2 * p + 1]), d2, nd2, y2);
-                c[h] = e2m1x8(q, v + 8 * h);
-            }
+            for (int h = 0; h < 2; ++h) c[h] = e2m1x8_div(v + 8 * h, pk2(ylo, ylo), pk2(yhi, yhi), d2, nd2, y2);
         } else {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -635,7 +644,7 @@ struct EncodeArgs {
 // `dst` (-1: the same row).
 // NK > 0: n fixed at compile time (the 2:4 default takes its own mask).
 template <int FMT, int M, int NK>
-__device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t *lut, const float2 *tab, int64_t row,
+__device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t *lut, const float4 *tab, int64_t row,
                                             int64_t u, bool active, float s_t, float c6, float y6, int64_t dst = -1,
                                             bool pad_codes = false) {
     constexpr int IB = M <= 2 ? 1 : M <= 4 ? 2 : M <= 8 ? 3 : 4;
@@ -702,17 +711,20 @@ __device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t 
         }
     }
 
-    // Mask, and the backbone S = X_ln on the mask, +0 elsewhere.
+    // Mask, and Q(S) for the backbone S = X_ln on the mask, +0 elsewhere.
+    // Every group keeps its largest magnitude (n >= 1), so the block amax
+    // of S is that of X_ln (over the lane pair too, for MXFP4) and so are
+    // the step and the codes on the mask: Q(S) is the encoding of X_ln with
+    // the dropped positions' nibbles cleared to the +0 code of S's zeros.
     uint32_t keep;
-    float s[kUnit];
     if constexpr (M == 4 && NK == 2)
         keep = keep_mask_42(v);
     else
         keep = keep_mask<M>(v, n);
-#pragma unroll
-    for (int i = 0; i < kUnit; ++i) s[i] = ((keep >> i) & 1u) ? v[i] : 0.0f;
     uint32_t s_scale, s_lo, s_hi;
-    const float ds = quantize16<FMT>(s, s_t, c6, y6, tab, s_scale, s_lo, s_hi);
+    const float ds = quantize16<FMT>(v, s_t, c6, y6, tab, s_scale, s_lo, s_hi);
+    s_lo &= nibble_mask8(keep);
+    s_hi &= nibble_mask8(keep >> 8);
 
     // Residual against the quantized backbone: R = RN32(X_ln - RN32(value * d)).
     // Scalar intrinsics: the product must be rounded before the subtraction.
@@ -804,7 +816,7 @@ prep_encode_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ 
     const float c6 = __fmul_rn(6.0f, s_t);
     const float y6 = (FMT == kFmtNV && c6 >= 0x1p-90f && c6 <= 0x1p90f) ? __frcp_rn(c6) : 0.0f;
     if (blockIdx.x == 0 && threadIdx.x == 0) *s_t_out = s_t;
-    __shared__ float2 tab[128];  // NVFP4 steps and reciprocals by scale code
+    __shared__ float4 tab[128];  // NVFP4 steps and reciprocals by scale code
     build_step_table<FMT>(tab, s_t);
     __syncthreads();
 
@@ -883,7 +895,7 @@ prep_encode_grouped_kernel(const EncodeArgs ea, const unsigned *__restrict__ ama
     const float c6 = __fmul_rn(6.0f, s_t);
     const float y6 = (FMT == kFmtNV && c6 >= 0x1p-90f && c6 <= 0x1p90f) ? __frcp_rn(c6) : 0.0f;
     if (blockIdx.x == 0 && threadIdx.x == 0) *s_t_out = s_t;
-    __shared__ float2 tab[128];  // NVFP4 steps and reciprocals by scale code
+    __shared__ float4 tab[128];  // NVFP4 steps and reciprocals by scale code
     build_step_table<FMT>(tab, s_t);
     __syncthreads();
     constexpr int IBm = M <= 2 ? 1 : M <= 4 ? 2 : M <= 8 ? 3 : 4;
@@ -1094,7 +1106,7 @@ prep_small_kernel(const EncodeArgs a, float eps, int64_t sf_rows, float *__restr
         words[0] = amax;
         words[1] = s_t;
     }
-    __shared__ float2 tab[128];  // NVFP4 steps and reciprocals by scale code
+    __shared__ float4 tab[128];  // NVFP4 steps and reciprocals by scale code
     build_step_table<FMT>(tab, s_t);
     __syncthreads();
     const int64_t upr = k / kUnit, total = m_tok * upr;
@@ -1114,7 +1126,9 @@ prep_small_kernel(const EncodeArgs a, float eps, int64_t sf_rows, float *__restr
 // quotients within a few ulps of the E2M1 and UE4M3 rounding boundaries, and
 // quotients of exponent -30 .. 30; divisors span [2^-90, 2^90]. A mismatch
 // is a quotient of magnitude >= 2^-11 whose bits differ, or any quotient
-// whose E2M1 code (or UE4M3 code of its magnitude) differs. (Far below 2^-11
+// whose E2M1 code (or UE4M3 code of its magnitude) differs, or a code of
+// the bracketed eight-value encoding (e2m1x8_div) that differs from the
+// code of the correctly rounded quotient. (Far below 2^-11
 // the remainder of the method can leave the normal range; such quotients
 // only ever give a zero code, whose sign comes from the dividend.)
 __device__ unsigned long long g_div_mismatch;
@@ -1163,7 +1177,25 @@ __global__ void div_check_kernel(uint64_t count, uint64_t seed) {
                                  (__float_as_uint(q1) & 0x7FFFFFFFu) != (__float_as_uint(ref) & 0x7FFFFFFFu);
         const bool code_differs = (e2m1_pair(pk2(q.x, q.x), sv, sv) & 0xFu) != (e2m1_pair(pk2(ref, ref), sv, sv) & 0xFu) ||
                                   ue4m3_code(fabsf(q1)) != ue4m3_code(fabsf(ref));
-        if (ref == ref && ((bits_differ && fabsf(ref) >= 0x1p-11f) || code_differs)) {
+        // The bracketed encoding of eight dividends around v (magnitudes
+        // 20 ulps below to 15 ulps above |v|, signs alternating), so that
+        // near a rounding boundary some quotients are decided by the
+        // bracketing products and some by the fallback.
+        float vs[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            vs[j] = __uint_as_float(((sv & 0x7FFFFFFFu) + 5 * j - 20) | ((sv ^ (uint32_t)j << 31) & 0x80000000u));
+        const uint32_t word = e2m1x8_div(vs, pk2(__fmul_rn(y, 1.0f - 0x1p-21f), __fmul_rn(y, 1.0f - 0x1p-21f)),
+                                         pk2(__fmul_rn(y, 1.0f + 0x1p-21f), __fmul_rn(y, 1.0f + 0x1p-21f)), pk2(d, d),
+                                         pk2(-d, -d), pk2(y, y));
+        bool word_differs = false;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float rj = __fdiv_rn(vs[j], d);
+            const uint32_t sj = __float_as_uint(vs[j]);
+            word_differs |= ((word >> (4 * j)) & 0xFu) != (e2m1_pair(pk2(rj, rj), sj, sj) & 0xFu);
+        }
+        if (ref == ref && ((bits_differ && fabsf(ref) >= 0x1p-11f) || code_differs || word_differs)) {
             const unsigned long long slot = atomicAdd(&g_div_mismatch, 1ull);
             if (slot < 16) {
                 g_div_examples[slot][0] = v;

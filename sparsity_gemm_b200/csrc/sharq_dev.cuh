@@ -214,6 +214,61 @@ __device__ __forceinline__ uint32_t e2m1x8(const uint64_t *q, const float *sv) {
     return r;
 }
 
+// E2M1 codes of eight quotients (four packed pairs) as one word, lowest
+// nibble first, each with the sign of its quotient as it stands (the
+// conversion keeps the sign of zeros and of values rounding to zero).
+__device__ __forceinline__ uint32_t e2m1x8_as_is(const uint64_t *q) {
+    float f[8];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float2 t = up2(q[p]);
+        f[2 * p] = t.x;
+        f[2 * p + 1] = t.y;
+    }
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(f[0]), "f"(f[1]), "f"(f[2]), "f"(f[3]), "f"(f[4]), "f"(f[5]), "f"(f[6]), "f"(f[7]));
+    return r;
+}
+
+// E2M1 codes of RN32(v_i / d) for eight values, lowest nibble first, for
+// d in [2^-90, 2^90] with y = RN(1/d), ylo = RN(y (1 - 2^-21)) and
+// yhi = RN(y (1 + 2^-21)) (packed pairs yl2, yh2, y2; d2 = (d, d),
+// nd2 = (-d, -d)). Each relative error below is at most 2^-24 (RN of a
+// normal number), so for v > 0
+//   RN(v ylo) <= (v / d)(1 + 2^-24)^3 (1 - 2^-21) < v / d,
+//   RN(v yhi) >= (v / d)(1 - 2^-24)^3 (1 + 2^-21) > v / d
+// (mirrored for v < 0): the two products bracket the exact quotient, hence
+// also RN32(v / d). Rounding to binary32 and encoding to E2M1 are both
+// monotone, so when the two products give the same code word, every value
+// between them has that code, RN32(v / d) included; where a product falls
+// below the normal range, both it and the quotient are far below 1/4 and
+// all of them give the zero code of v's sign. Products keep the sign of a
+// zero dividend. Otherwise (a quotient within about 2^-21 of a rounding
+// boundary) the correctly rounded quotients of div2 decide.
+__device__ __forceinline__ uint32_t e2m1x8_div(const float *v, uint64_t yl2, uint64_t yh2, uint64_t d2, uint64_t nd2,
+                                               uint64_t y2) {
+    uint64_t ql[4], qh[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const uint64_t vv = pk2(v[2 * p], v[2 * p + 1]);
+        ql[p] = mul2(vv, yl2);
+        qh[p] = mul2(vv, yh2);
+    }
+    const uint32_t c = e2m1x8_as_is(ql);
+    if (c == e2m1x8_as_is(qh)) return c;
+    uint64_t q[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) q[p] = div2(pk2(v[2 * p], v[2 * p + 1]), d2, nd2, y2);
+    return e2m1x8(q, v);
+}
+
 // E2M1 byte of two quotients (lo nibble = q.x), rounded to nearest even with
 // saturation to 6 by the hardware conversion, which keeps the sign of zeros.
 // The quotients first take the sign bits of their dividends (sign_lo,
