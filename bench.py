@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # one ncu capture of the current dual_gemm_kernel (dram__bytes_read.sum +
 # dram__bytes_write.sum of the layer-set launch list). Set to None whenever
 # the kernel changes until it is captured again.
-GEMM_TRAFFIC_BYTES_PER_STEP_M8192 = 1019.0e6
+GEMM_TRAFFIC_BYTES_PER_STEP_M8192 = 1033.9e6
 
 
 def parse_args():
