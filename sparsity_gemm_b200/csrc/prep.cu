@@ -16,7 +16,7 @@
 //   2. prep_encode_kernel (one thread per 16 consecutive elements; an MXFP4
 //      block of 32 spans a lane pair): LayerNorm apply, top-n-of-m selection,
 //      Q(S), R = X_ln - deq(Q(S)), Q(R), and packed code / scale / metadata
-//      stores. The second read of x mostly hits L2.
+//      stores. The second read of x hits L2 when x fits in it (126 MB).
 #include <cuda_fp16.h>
 
 #include <string.h>
