@@ -111,23 +111,125 @@ __device__ double u128_to_f64(unsigned __int128 v) {
     return __dmul_rn(__ull2double_rn((uint64_t)q), scale);
 }
 
-// mu = RN32(RN64(S1) / (K 2^24)); rstd = RN32(1 / sqrt(RN64(D) / (K^2 2^48) + eps)).
-__device__ float2 finish_stats(const ExactSums &e, int64_t k, float eps) {
-    const __int128 s1 = (__int128)e.hi * 1048576 + e.lo;
-    const __int128 s2 = ((__int128)e.hh << 40) + ((__int128)e.hl << 21) + (__int128)e.ll;
-    const __int128 d = (__int128)k * s2 - s1 * s1;
+// mu = RN32(RN64(S1) / (K 2^24)); rstd = RN32(1 / sqrt(RN64(D) / (K^2 2^48) + eps))
+// from S1 = sum a and D = K S2 - S1^2 >= 0 (integers, a = x 2^24).
+__device__ float2 finish_ld(int64_t s1, unsigned __int128 d, int64_t k, float eps) {
     const double kd = (double)k;
     const double mean64 = __ddiv_rn(__ll2double_rn((long long)s1), __dmul_rn(kd, 16777216.0));
-    const double var64 = __ddiv_rn(u128_to_f64((unsigned __int128)d), __dmul_rn(__dmul_rn(kd, kd), 281474976710656.0));
+    const double var64 = __ddiv_rn(u128_to_f64(d), __dmul_rn(__dmul_rn(kd, kd), 281474976710656.0));
     return make_float2(__double2float_rn(mean64),
                        __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(var64, (double)eps)))));
 }
 
+__device__ float2 finish_stats(const ExactSums &e, int64_t k, float eps) {
+    const __int128 s1 = (__int128)e.hi * 1048576 + e.lo;
+    const __int128 s2 = ((__int128)e.hh << 40) + ((__int128)e.hl << 21) + (__int128)e.ll;
+    const __int128 d = (__int128)k * s2 - s1 * s1;
+    return finish_ld((int64_t)s1, (unsigned __int128)d, k, eps);
+}
+
 // RMSNorm: ms = RN64(S2) / (K 2^48); rstd = RN32(1 / sqrt(ms + eps)); mu = 0.
+__device__ float finish_rms_rstd(unsigned __int128 s2, int64_t k, float eps) {
+    const double ms64 = __ddiv_rn(u128_to_f64(s2), __dmul_rn((double)k, 281474976710656.0));
+    return __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms64, (double)eps))));
+}
+
 __device__ float2 finish_stats_rms(const ExactSums &e, int64_t k, float eps) {
     const __int128 s2 = ((__int128)e.hh << 40) + ((__int128)e.hl << 21) + (__int128)e.ll;
-    const double ms64 = __ddiv_rn(u128_to_f64((unsigned __int128)s2), __dmul_rn((double)k, 281474976710656.0));
-    return make_float2(0.0f, __double2float_rn(__ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(ms64, (double)eps)))));
+    return make_float2(0.0f, finish_rms_rstd((unsigned __int128)s2, k, eps));
+}
+
+// ---------------------------------------------------------------------------
+// Certified statistics (long rows, one warp per row). Each lane sums x in
+// binary64, exactly: every x is a multiple of 2^-24 below 2^16 and a lane
+// adds at most SHARQ_K_MAX / 32 = 2048 of them, so every partial sum is a
+// multiple of 2^-24 below 2^27 (52 significant bits). Each lane also sums
+// x^2 in binary64 (each square exact, 22 significant bits) in two
+// accumulators, one rounding per addition; with the join of the two and the
+// five butterfly levels, no square passes through more than K/64 + 6
+// roundings, so (Higham, Accuracy and Stability of Numerical Algorithms,
+// 2nd ed., section 4.2, for non-negative terms) the computed sum s2 is
+// within gamma_h S2 <= 2 h u s2 of S2 (h = K/64 + 6, u = 2^-53). The bound
+// used below, (K/32 + 8) 2^-51 s2, is larger still. Every step from D (or
+// S2, for RMSNorm) to rstd is a monotone rounding or a monotone function,
+// so if rstd is the same binary32 value at both ends of the interval that
+// holds the exact sum, it is the value at the exact sum: the statistics of
+// the exact method, bit for bit. Otherwise the warp sums the row again with
+// the exact integer method.
+struct FastLane {
+    double s1;        // sum x, exact
+    double s2a, s2b;  // sum x^2 over alternate elements, rounded
+};
+
+__device__ __forceinline__ void fast_pair(uint32_t w, FastLane &f) {
+    double d0, d1;
+    asm("{\n\t.reg .f16 h0, h1;\n\tmov.b32 {h0, h1}, %2;\n\tcvt.f64.f16 %0, h0;\n\tcvt.f64.f16 %1, h1;\n\t}"
+        : "=d"(d0), "=d"(d1) : "r"(w));
+    f.s1 = __dadd_rn(f.s1, __dadd_rn(d0, d1));  // both sums exact (multiples of 2^-24 below 2^28)
+    f.s2a = __fma_rn(d0, d0, f.s2a);
+    f.s2b = __fma_rn(d1, d1, f.s2b);
+}
+
+// Floor (up = false) or ceiling (up = true) of a non-negative binary64 value
+// below 2^127, as a 128-bit integer.
+__device__ unsigned __int128 f64_to_u128(double v, bool up) {
+    if (!(v > 0.0)) return 0;
+    const uint64_t b = (uint64_t)__double_as_longlong(v);
+    const int ex = (int)(b >> 52);
+    if (ex == 0) return up ? 1 : 0;  // subnormal: 0 < v < 1
+    const uint64_t m = (b & 0xFFFFFFFFFFFFFull) | (1ull << 52);
+    const int e = ex - 1075;  // v = m 2^e
+    if (e >= 0) return (unsigned __int128)m << e;
+    if (e <= -53) return up ? 1 : 0;  // 0 < v < 1
+    const uint64_t q = m >> -e;
+    const bool frac = (m & ((1ull << -e) - 1ull)) != 0;
+    return (unsigned __int128)(q + ((up && frac) ? 1ull : 0ull));
+}
+
+// Statistics from the warp's certified sums (s1 = sum a exactly, s2 the
+// rounded sum of x^2), or false where the error bound leaves the binary32
+// rstd undecided.
+__device__ bool certified_stats(int64_t s1, double s2, int64_t k, float eps, bool rms, float2 &out) {
+    const double err = __dmul_ru(s2, __dmul_ru((double)(k / 32 + 8), 0x1p-51));
+    const unsigned __int128 lo = f64_to_u128(__dmul_rd(__dsub_rd(s2, err), 0x1p48), false);
+    const unsigned __int128 hi = f64_to_u128(__dmul_ru(__dadd_ru(s2, err), 0x1p48), true);
+    float r_lo, r_hi;
+    if (rms) {
+        out = make_float2(0.0f, finish_rms_rstd(lo, k, eps));
+        r_lo = out.y;
+        r_hi = finish_rms_rstd(hi, k, eps);
+    } else {
+        const __int128 sq = (__int128)s1 * s1;
+        const __int128 dlo = (__int128)k * (__int128)lo - sq, dhi = (__int128)k * (__int128)hi - sq;
+        out = finish_ld(s1, dlo < 0 ? (unsigned __int128)0 : (unsigned __int128)dlo, k, eps);
+        r_lo = out.y;
+        r_hi = finish_ld(s1, dhi < 0 ? (unsigned __int128)0 : (unsigned __int128)dhi, k, eps).y;
+    }
+    return __float_as_uint(r_lo) == __float_as_uint(r_hi);
+}
+
+// The exact statistics of one row, summed by a whole warp from global memory
+// (every lane returns them).
+template <bool RMS>
+__device__ float2 exact_row_stats(const uint4 *xr, int nvec, int lane, int64_t k, float eps) {
+    LaneSums l = {};
+    for (int c = lane; c < nvec; c += 32) {
+        const uint4 v = xr[c];
+        accum_pair(v.x, l);
+        accum_pair(v.y, l);
+        accum_pair(v.z, l);
+        accum_pair(v.w, l);
+    }
+    ExactSums e = widen(l);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        e.hi += __shfl_xor_sync(0xFFFFFFFFu, e.hi, o);
+        e.lo += __shfl_xor_sync(0xFFFFFFFFu, e.lo, o);
+        e.hh += __shfl_xor_sync(0xFFFFFFFFu, e.hh, o);
+        e.hl += __shfl_xor_sync(0xFFFFFFFFu, e.hl, o);
+        e.ll += __shfl_xor_sync(0xFFFFFFFFu, e.ll, o);
+    }
+    return RMS ? finish_stats_rms(e, k, eps) : finish_stats(e, k, eps);
 }
 
 // RMS: RMSNorm statistics (no centring) instead of LayerNorm's.
@@ -271,16 +373,22 @@ constexpr int kStatsStages = 3;
 constexpr int kStatsRingBytes = (kStatsThreads / 32) * kStatsStages * 4 * 32 * 16;  // 48 KB
 constexpr int kStatsMaxRpw = 4;  // rows per warp, short rows
 
-template <bool AFFINE, bool RMS>
+// FAST: certified binary64 sums with the exact method as the fallback (rows
+// longer than 2048 elements).
+template <bool AFFINE, bool RMS, bool FAST>
 __global__ void __launch_bounds__(kStatsThreads)
 ln_stats_warp_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gamma,
                      const uint16_t *__restrict__ beta, float eps, int64_t k, int64_t m_tok, int rpw,
                      float2 *__restrict__ stats, unsigned *__restrict__ amax_word) {
     constexpr int W = kStatsThreads / 32;
+    constexpr int NS = (AFFINE || !FAST) ? 1 : W * kStatsMaxRpw;
     extern __shared__ uint4 ring[];  // [warp][stage][vector j][lane]
     __shared__ float red_max[W];
-    __shared__ ExactSums rsum[AFFINE ? 1 : W * kStatsMaxRpw];
+    __shared__ ExactSums rsum[(AFFINE || FAST) ? 1 : W * kStatsMaxRpw];
     __shared__ uint32_t rmx[AFFINE ? 1 : W * kStatsMaxRpw], rmn[AFFINE ? 1 : W * kStatsMaxRpw];
+    __shared__ int64_t fs1[NS];
+    __shared__ double fs2[NS];
+    __shared__ int redo[NS];
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (AFFINE) rpw = 1;
     const int64_t cta_row0 = (int64_t)blockIdx.x * W * rpw;
@@ -305,13 +413,21 @@ ln_stats_warp_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
             }
             cp_async_commit();  // possibly empty: one group per iteration keeps the count uniform
         };
-        LaneSums l = {0, 0, 0.0, 0.0, 0.0};
+        LaneSums l = {};
+        FastLane f = {0.0, 0.0, 0.0};
         uint32_t mx = 0xFC00FC00u, mn = 0x7C007C00u;  // (-inf, -inf), (+inf, +inf) as half2
         auto consume = [&](const uint4 &v) {
-            accum_pair(v.x, l);
-            accum_pair(v.y, l);
-            accum_pair(v.z, l);
-            accum_pair(v.w, l);
+            if (FAST) {
+                fast_pair(v.x, f);
+                fast_pair(v.y, f);
+                fast_pair(v.z, f);
+                fast_pair(v.w, f);
+            } else {
+                accum_pair(v.x, l);
+                accum_pair(v.y, l);
+                accum_pair(v.z, l);
+                accum_pair(v.w, l);
+            }
             if (!AFFINE) {
                 const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -339,35 +455,64 @@ ln_stats_warp_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
             issue(it + 2);  // refills the slot consumed in the previous iteration
         }
         cp_async_wait<0>();
-        ExactSums e = widen(l);
+        if (!AFFINE) {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            e.hi += __shfl_xor_sync(0xFFFFFFFFu, e.hi, o);
-            e.lo += __shfl_xor_sync(0xFFFFFFFFu, e.lo, o);
-            e.hh += __shfl_xor_sync(0xFFFFFFFFu, e.hh, o);
-            e.hl += __shfl_xor_sync(0xFFFFFFFFu, e.hl, o);
-            e.ll += __shfl_xor_sync(0xFFFFFFFFu, e.ll, o);
-            if (!AFFINE) {
+            for (int o = 16; o > 0; o >>= 1) {
                 const uint32_t omx = __shfl_xor_sync(0xFFFFFFFFu, mx, o), omn = __shfl_xor_sync(0xFFFFFFFFu, mn, o);
                 asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(omx));
                 asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(omn));
             }
         }
+        // Butterfly reductions: every lane ends with the same totals (each
+        // step adds the same two operands on both lanes of a pair).
+        ExactSums e = {};
+        int64_t s1 = 0;
+        double s2 = 0.0;
+        if (FAST) {
+            s1 = __double2ll_rn(__dmul_rn(f.s1, 16777216.0));  // sum a over the lane, an integer below 2^51
+            s2 = __dadd_rn(f.s2a, f.s2b);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
+                s2 = __dadd_rn(s2, __shfl_xor_sync(0xFFFFFFFFu, s2, o));
+            }
+        } else {
+            e = widen(l);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                e.hi += __shfl_xor_sync(0xFFFFFFFFu, e.hi, o);
+                e.lo += __shfl_xor_sync(0xFFFFFFFFu, e.lo, o);
+                e.hh += __shfl_xor_sync(0xFFFFFFFFu, e.hh, o);
+                e.hl += __shfl_xor_sync(0xFFFFFFFFu, e.hl, o);
+                e.ll += __shfl_xor_sync(0xFFFFFFFFu, e.ll, o);
+            }
+        }
         if (!AFFINE) {
             if (lane == 0) {
-                rsum[slot] = e;
+                if (FAST) {
+                    fs1[slot] = s1;
+                    fs2[slot] = s2;
+                } else {
+                    rsum[slot] = e;
+                }
                 rmx[slot] = mx;
                 rmn[slot] = mn;
             }
             continue;
         }
         float2 st = make_float2(0.0f, 0.0f);
-        if (lane == 0) {
-            st = RMS ? finish_stats_rms(e, k, eps) : finish_stats(e, k, eps);
-            stats[row] = st;
+        if (FAST) {
+            const bool ok = certified_stats(s1, s2, k, eps, RMS, st);  // the same on every lane
+            if (!ok) st = exact_row_stats<RMS>(xr, nvec, lane, k, eps);
+            if (lane == 0) stats[row] = st;
+        } else {
+            if (lane == 0) {
+                st = RMS ? finish_stats_rms(e, k, eps) : finish_stats(e, k, eps);
+                stats[row] = st;
+            }
+            st.x = __shfl_sync(0xFFFFFFFFu, st.x, 0);
+            st.y = __shfl_sync(0xFFFFFFFFu, st.y, 0);
         }
-        st.x = __shfl_sync(0xFFFFFFFFu, st.x, 0);
-        st.y = __shfl_sync(0xFFFFFFFFu, st.y, 0);
         const bool has_g = gamma != nullptr, has_b = beta != nullptr;
         for (int cc = lane; cc < nvec; cc += 32) {
             const uint4 v = xr[cc];
@@ -386,18 +531,44 @@ ln_stats_warp_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
         }
     }
     if (!AFFINE) {
+        // X_ln = RN(RN(x - mu) * rstd) is non-decreasing in x: the row's
+        // amax|X_ln| is reached at its smallest or largest x.
+        auto row_amax = [&](const float2 &st, int slot) {
+            const uint32_t mx = rmx[slot], mn = rmn[slot];
+            const float xmax = fmaxf(h2f((uint16_t)mx), h2f((uint16_t)(mx >> 16)));
+            const float xmin = fminf(h2f((uint16_t)mn), h2f((uint16_t)(mn >> 16)));
+            return fmaxf(fabsf(__fmul_rn(__fsub_rn(xmax, st.x), st.y)), fabsf(__fmul_rn(__fsub_rn(xmin, st.x), st.y)));
+        };
         __syncthreads();  // every row's sums are in shared memory
         const int slot = threadIdx.x;
         const int64_t row = cta_row0 + slot;
         if (slot < W * rpw && row < m_tok) {
-            const float2 st = RMS ? finish_stats_rms(rsum[slot], k, eps) : finish_stats(rsum[slot], k, eps);
-            stats[row] = st;
-            // X_ln = RN(RN(x - mu) * rstd) is non-decreasing in x: the row's
-            // amax|X_ln| is reached at its smallest or largest x.
-            const uint32_t mx = rmx[slot], mn = rmn[slot];
-            const float xmax = fmaxf(h2f((uint16_t)mx), h2f((uint16_t)(mx >> 16)));
-            const float xmin = fminf(h2f((uint16_t)mn), h2f((uint16_t)(mn >> 16)));
-            amax = fmaxf(fabsf(__fmul_rn(__fsub_rn(xmax, st.x), st.y)), fabsf(__fmul_rn(__fsub_rn(xmin, st.x), st.y)));
+            float2 st;
+            bool ok = true;
+            if (FAST) {
+                ok = certified_stats(fs1[slot], fs2[slot], k, eps, RMS, st);
+                redo[slot] = ok ? 0 : 1;
+            } else {
+                st = RMS ? finish_stats_rms(rsum[slot], k, eps) : finish_stats(rsum[slot], k, eps);
+            }
+            if (ok) {
+                stats[row] = st;
+                amax = row_amax(st, slot);
+            }
+        }
+        if (FAST) {
+            __syncthreads();  // the undecided rows are marked
+            for (int i = 0; i < rpw; ++i) {
+                const int rs = warp * rpw + i;
+                const int64_t rrow = cta_row0 + rs;
+                if (rrow >= m_tok) break;  // warp-uniform
+                if (!redo[rs]) continue;   // warp-uniform
+                const float2 st = exact_row_stats<RMS>(reinterpret_cast<const uint4 *>(x + rrow * k), nvec, lane, k, eps);
+                if (lane == 0) {
+                    stats[rrow] = st;
+                    amax = fmaxf(amax, row_amax(st, rs));
+                }
+            }
         }
     }
 #pragma unroll
@@ -1445,9 +1616,13 @@ static sharq_status launch_stats(LaunchCtx &ctx, const sharq_prep &P, const void
     if (!attr_done[dev]) {
         SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_kernel<true, RMS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)(2 * SHARQ_K_MAX)));
-        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<true, RMS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kStatsRingBytes));
-        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<false, RMS>,
+        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<true, RMS, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
+        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<false, RMS, false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
+        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<true, RMS, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
+        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<false, RMS, true>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
         attr_done[dev] = true;
     }
@@ -1464,12 +1639,17 @@ static sharq_status launch_stats(LaunchCtx &ctx, const sharq_prep &P, const void
         }
         const int64_t per_cta = (int64_t)(kStatsThreads / 32) * rpw;
         const unsigned grid = (unsigned)((P.m_tok + per_cta - 1) / per_cta);
-        if (gamma || beta)
-            ln_stats_warp_kernel<true, RMS><<<grid, kStatsThreads, kStatsRingBytes, ctx.stream>>>(
-                xx, gg, bb, eps, P.k, P.m_tok, 1, stats, words);
-        else
-            ln_stats_warp_kernel<false, RMS><<<grid, kStatsThreads, kStatsRingBytes, ctx.stream>>>(
-                xx, nullptr, nullptr, eps, P.k, P.m_tok, rpw, stats, words);
+        // Rows longer than 2048 elements take the certified sums (two finishes
+        // per row, which short rows would feel).
+        const bool fast = P.k > 2048;
+        if (gamma || beta) {
+            auto fn = fast ? ln_stats_warp_kernel<true, RMS, true> : ln_stats_warp_kernel<true, RMS, false>;
+            fn<<<grid, kStatsThreads, kStatsRingBytes, ctx.stream>>>(xx, gg, bb, eps, P.k, P.m_tok, 1, stats, words);
+        } else {
+            auto fn = fast ? ln_stats_warp_kernel<false, RMS, true> : ln_stats_warp_kernel<false, RMS, false>;
+            fn<<<grid, kStatsThreads, kStatsRingBytes, ctx.stream>>>(xx, nullptr, nullptr, eps, P.k, P.m_tok, rpw,
+                                                                   stats, words);
+        }
     } else {
         if (gamma || beta)
             ln_stats_kernel<true, RMS><<<(unsigned)P.m_tok, kStatsThreads, (size_t)(2 * P.k), ctx.stream>>>(

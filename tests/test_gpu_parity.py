@@ -102,6 +102,35 @@ def test_maximum_k_statistics_at_the_lane_sum_bound():
         assert_bits_equal("rstd", ex["rstd"], rstd)
 
 
+@pytest.mark.parametrize("norm", ["layer", "rms"])
+@pytest.mark.parametrize("affine", [False, True])
+def test_certified_statistics_and_exact_fallback(norm, affine):
+    """Rows longer than 2048 elements (one warp per row) take binary64 sums
+    whose error bound must decide the binary32 rstd; rows where it does not
+    (a constant row, fp16 extremes of both signs, a large mean over a small
+    spread) are summed again by the exact method. Every row bit-exact, with
+    and without the affine parameters."""
+    import sparsity_gemm_b200 as sq
+    m_tok, k = 48, 4096
+    x = synth.activations_student(920 + affine, m_tok, k)
+    x[0] = np.float16(3.5)
+    x[1, ::2] = np.float16(65504.0)
+    x[1, 1::2] = np.float16(-65504.0)
+    x[2] = np.float16(1000.0)
+    x[2, ::7] = np.float16(1000.5)
+    x[3] = 0
+    x[4].view(np.uint16)[:] = np.arange(k, dtype=np.uint16) % 64 + 1  # fp16 subnormals
+    x[5, : k // 2] = np.float16(65504.0)
+    g, b = synth.ln_params(921, k) if affine else (None, None)
+    if norm == "rms":
+        b = None
+    op = oracle.prepare(x, g, b, 1e-5, 2, 4, 0, norm=norm)
+    p = sq.prepare(cuda16(x), None if g is None else cuda16(g), None if b is None else cuda16(b), 1e-5, 2, 4, 0,
+                   norm=norm)
+    assert_prep_matches(sq.prep_export(p), op)
+    assert sq.get_last_error() == sq.OK
+
+
 def test_maximum_k_linear():
     """A linear at K = SHARQ_K_MAX (256 K steps, split over a cluster at 9
     rows): prep bit-exact, output within tolerance."""
