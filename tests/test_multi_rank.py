@@ -40,7 +40,7 @@ def _worker(rank, world, port, out):
 def test_max_over_ranks_and_barrier_with_gloo():
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:  # no fork of a multi-threaded test process
         out = m.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         assert dict(out) == {0: 3.5, 1: 3.5}
