@@ -46,6 +46,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_write.sum of the layer-set launch list). Set to None whenever
 # the kernel changes until it is captured again.
 GEMM_TRAFFIC_BYTES_PER_STEP_M8192 = 1033.9e6
+# The only performance and accuracy figures of the method's own evaluation
+# (abstract of "SharQ: Bridging Activation Sparsity and FP4 Quantization for
+# LLM Inference"): other hardware and end-to-end serving, reported for
+# context next to the measured line, never as its baseline.
+PAGES_CONTEXT = {
+    "hardware": "RTX 5090 (sm_120)",
+    "latency_vs_fp16": "2.2-2.4x lower",
+    "throughput_vs_fp8": "1.2-1.4x higher",
+    "accuracy_gap_recovered": "43-63% of the NVFP4-to-FP16 gap",
+    "comparable": "no: other GPU, whole-model serving; see quality for this path's output error",
+}
 
 
 def parse_args():
@@ -318,6 +329,7 @@ def run_sharq(args, world, rank, local):
                               "gemm_each": {lin.name: float(gemm_each[j] / steps) for j, lin in enumerate(ls.linears)}},
         "gpu_launches": gpu_launches,
         "wall_s_timed": t1 - t0,
+        "pages_context": PAGES_CONTEXT,
     }
     cs = clocks.summary(t0, t1)
     result["clocks"] = {"sm_mhz": cs.get("sm_mhz"), "sm_max_mhz": cs.get("sm_max_mhz"), "reasons": cs.get("reasons"),
