@@ -126,6 +126,33 @@ def _ptr(t):
     return None if t is None else C.c_void_p(t.data_ptr())
 
 
+def _require(cond: bool, what: str):
+    """Argument check that survives python -O (raises ValueError)."""
+    if not cond:
+        raise ValueError(what)
+
+
+def _cuda_here(t: torch.Tensor, name: str):
+    """t must live on the current CUDA device: the library launches on the
+    current device, and a host or other-device pointer would reach a kernel."""
+    _require(isinstance(t, torch.Tensor) and t.is_cuda, f"{name} must be a CUDA tensor")
+    cur = torch.cuda.current_device()
+    _require(t.device.index == cur,
+             f"{name} is on {t.device} but the current device is cuda:{cur} (call torch.cuda.set_device first)")
+
+
+def _fp16_matrix(t: torch.Tensor, name: str, dims: int = 2):
+    _require(isinstance(t, torch.Tensor) and t.dtype == torch.float16 and t.dim() == dims and t.is_contiguous(),
+             f"{name} must be a contiguous fp16 tensor with {dims} dimensions")
+    _cuda_here(t, name)
+
+
+def _int32_vector(t: torch.Tensor, name: str):
+    _require(isinstance(t, torch.Tensor) and t.dtype == torch.int32 and t.dim() == 1 and t.is_contiguous(),
+             f"{name} must be a contiguous int32 vector")
+    _cuda_here(t, name)
+
+
 def weight_bytes(n_out: int, k: int, fmt: int) -> int:
     return int(lib().sharq_weight_bytes(n_out, k, fmt))
 
@@ -166,7 +193,7 @@ def _device_buffer(nbytes: int, device) -> torch.Tensor:
 
 def quantize_weight(w: torch.Tensor, fmt: int = NVFP4, stream=None) -> QuantizedWeight:
     """Offline FP4 quantization of W [n_out, k] (fp16, CUDA)."""
-    assert w.dtype == torch.float16 and w.is_cuda and w.dim() == 2 and w.is_contiguous()
+    _fp16_matrix(w, "w")
     n_out, k = w.shape
     nbytes = weight_bytes(n_out, k, fmt)
     if nbytes == 0:
@@ -183,10 +210,13 @@ def prepare(x: torch.Tensor, ln_w=None, ln_b=None, eps: float = 1e-5, n: int = 2
     """Fused preparation operator on x [m_tok, k] (fp16, CUDA). norm:
     "layer" (LayerNorm with ln_w, ln_b) or "rms" (RMSNorm with weight ln_w;
     ln_b must be None)."""
-    assert norm in ("layer", "rms") and (norm == "layer" or ln_b is None)
-    assert x.dtype == torch.float16 and x.is_cuda and x.dim() == 2 and x.is_contiguous()
-    for t in (ln_w, ln_b):
-        assert t is None or (t.dtype == torch.float16 and t.is_cuda and t.numel() == x.shape[1] and t.is_contiguous())
+    _require(norm in ("layer", "rms") and (norm == "layer" or ln_b is None),
+             'norm must be "layer" or "rms" (RMSNorm takes no ln_b)')
+    _fp16_matrix(x, "x")
+    for t, name in ((ln_w, "ln_w"), (ln_b, "ln_b")):
+        if t is not None:
+            _fp16_matrix(t.view(-1) if t.is_contiguous() else t, name, 1)
+            _require(t.numel() == x.shape[1], f"{name} must have {x.shape[1]} elements")
     m_tok, k = x.shape
     nbytes = prep_bytes(m_tok, k, n, m, fmt)
     if nbytes == 0:
@@ -195,6 +225,7 @@ def prepare(x: torch.Tensor, ln_w=None, ln_b=None, eps: float = 1e-5, n: int = 2
         buf = _device_buffer(nbytes, x.device)
     else:
         buf = out.buf
+        _cuda_here(buf, "out.buf")
     desc = SharqPrep()
     xp = _ptr(x) if m_tok > 0 else None
     if norm == "rms":
@@ -211,14 +242,20 @@ def linear(prep: Prepared, qw: QuantizedWeight, out: torch.Tensor | None = None,
     """Dual-path FP4 linear: fp16 [m_tok, n_out] = (Q(S) + Q(R)) Q(W)^T, scaled,
     plus an optional fp16 bias [n_out]. A fused weight (quantize_weight_fused)
     gives its segments' outputs side by side."""
+    _cuda_here(prep.buf, "prep.buf")
+    _cuda_here(qw.buf, "qw.buf")
     if out is None:
         out = torch.empty((prep.m_tok, qw.n_out), dtype=torch.float16, device=prep.buf.device)
-    assert out.dtype == torch.float16 and out.is_contiguous() and tuple(out.shape) == (prep.m_tok, qw.n_out)
+    _require(out.dtype == torch.float16 and out.is_contiguous() and tuple(out.shape) == (prep.m_tok, qw.n_out),
+             f"out must be a contiguous fp16 tensor of shape {(prep.m_tok, qw.n_out)}")
+    _cuda_here(out, "out")
     optr = _ptr(out) if out.numel() else None
     if bias is None:
         _check(lib().sharq_linear(C.byref(prep.desc), C.byref(qw.desc), optr, _stream(stream)), "sharq_linear")
     else:
-        assert bias.dtype == torch.float16 and bias.is_cuda and bias.is_contiguous() and bias.numel() == qw.n_out
+        _require(bias.dtype == torch.float16 and bias.is_contiguous() and bias.numel() == qw.n_out,
+                 f"bias must be a contiguous fp16 tensor of {qw.n_out} elements")
+        _cuda_here(bias, "bias")
         _check(lib().sharq_linear_bias(C.byref(prep.desc), C.byref(qw.desc), _ptr(bias), optr, _stream(stream)),
                "sharq_linear_bias")
     return out
@@ -230,9 +267,13 @@ def quantize_weight_fused(ws, fmt: int = NVFP4, stream=None) -> QuantizedWeight:
     tensor scale, so the fused linear's columns equal the separate linears'.
     ws: list of fp16 CUDA tensors [n_g, k]."""
     ws = list(ws)
-    assert ws and all(w.dtype == torch.float16 and w.is_cuda and w.dim() == 2 for w in ws)
+    _require(len(ws) > 0, "ws must hold at least one weight")
+    for i, w in enumerate(ws):
+        _require(isinstance(w, torch.Tensor) and w.dtype == torch.float16 and w.dim() == 2,
+                 f"ws[{i}] must be an fp16 matrix")
+        _cuda_here(w, f"ws[{i}]")
     k = ws[0].shape[1]
-    assert all(w.shape[1] == k for w in ws)
+    _require(all(w.shape[1] == k for w in ws), "every weight of a fused payload must have the same k")
     rows = (C.c_int64 * len(ws))(*[w.shape[0] for w in ws])
     nbytes = int(lib().sharq_weight_bytes_fused(rows, len(ws), k, fmt))
     if nbytes == 0:
@@ -292,7 +333,7 @@ def weight_export(qw: QuantizedWeight, stream=None) -> dict:
 def quantize_weight_grouped(w: torch.Tensor, fmt: int = NVFP4, stream=None) -> QuantizedWeight:
     """Offline FP4 quantization of a stack of weights w [groups, n_out, k]
     (fp16, CUDA), each with its own tensor scale."""
-    assert w.dtype == torch.float16 and w.is_cuda and w.dim() == 3 and w.is_contiguous()
+    _fp16_matrix(w, "w", 3)
     groups, n_out, k = w.shape
     nbytes = int(lib().sharq_weight_bytes_grouped(groups, n_out, k, fmt))
     if nbytes == 0:
@@ -308,7 +349,7 @@ def group_view(qw: QuantizedWeight, g: int) -> QuantizedWeight:
     """A plain (one-group) descriptor of group g of a stacked weight; it
     shares qw's buffer."""
     d = qw.desc
-    assert 0 <= g < max(1, d.groups)
+    _require(0 <= g < max(1, d.groups), f"group {g} out of range (groups = {max(1, d.groups)})")
     stride = weight_bytes(d.n_out, d.k, d.fmt) * g
     v = SharqWQ()
     C.pointer(v)[0] = d
@@ -327,14 +368,17 @@ def gather_rows(prep: Prepared, row_idx, offsets: torch.Tensor, rows: int, out: 
     """Expert-grouped copy of prepared rows: grouped row i of group g (offsets
     [g] <= i < offsets[g+1]) is prepared row row_idx[i] (row_idx None: i).
     row_idx and offsets are int32 CUDA tensors."""
-    for t in (row_idx, offsets):
-        assert t is None or (t.dtype == torch.int32 and t.is_cuda and t.is_contiguous())
+    _int32_vector(offsets, "offsets")
+    if row_idx is not None:
+        _int32_vector(row_idx, "row_idx")
+    _cuda_here(prep.buf, "prep.buf")
     groups = offsets.numel() - 1
     d = prep.desc
     nbytes = int(lib().sharq_gather_bytes(rows, groups, d.k, d.n, d.m, d.fmt))
     if nbytes == 0:
         raise SharqError(ERR_INVALID_ARG, f"gather rows {rows} groups {groups}")
     buf = out.buf if out is not None and out.buf.numel() >= nbytes else _device_buffer(nbytes, prep.buf.device)
+    _cuda_here(buf, "out.buf")
     desc = SharqPrep()
     _check(lib().sharq_gather_rows(C.byref(d), _ptr(row_idx), _ptr(offsets), groups, rows, _ptr(buf), buf.numel(),
                                    C.byref(desc), _stream(stream)), "sharq_gather_rows")
@@ -348,15 +392,21 @@ def prepare_grouped(x: torch.Tensor, offsets: torch.Tensor, ln_w=None, ln_b=None
     = rows offsets[g] .. offsets[g+1]-1) straight into the grouped layout that
     gather_rows writes (equal to gather_rows(prepare(x), None, offsets) in
     codes, scales, metadata and tensor scale). offsets: int32 CUDA tensor."""
-    assert norm in ("layer", "rms") and (norm == "layer" or ln_b is None)
-    assert x.dtype == torch.float16 and x.is_cuda and x.dim() == 2 and x.is_contiguous()
-    assert offsets.dtype == torch.int32 and offsets.is_cuda and offsets.is_contiguous()
+    _require(norm in ("layer", "rms") and (norm == "layer" or ln_b is None),
+             'norm must be "layer" or "rms" (RMSNorm takes no ln_b)')
+    _fp16_matrix(x, "x")
+    _int32_vector(offsets, "offsets")
+    for t, name in ((ln_w, "ln_w"), (ln_b, "ln_b")):
+        if t is not None:
+            _fp16_matrix(t.view(-1) if t.is_contiguous() else t, name, 1)
+            _require(t.numel() == x.shape[1], f"{name} must have {x.shape[1]} elements")
     rows, k = x.shape
     groups = offsets.numel() - 1
     nbytes = int(lib().sharq_gather_bytes(rows, groups, k, n, m, fmt))
     if nbytes == 0:
         raise SharqError(ERR_INVALID_ARG, f"grouped prep rows {rows} groups {groups} k {k}")
     buf = out.buf if out is not None and out.buf.numel() >= nbytes else _device_buffer(nbytes, x.device)
+    _cuda_here(buf, "out.buf")
     desc = SharqPrep()
     _check(lib().sharq_prepare_grouped(_ptr(x) if rows > 0 else None, rows, k, _ptr(offsets), groups, _ptr(ln_w),
                                        _ptr(ln_b), float(eps), 1 if norm == "rms" else 0, n, m, fmt, _ptr(buf),
@@ -368,10 +418,14 @@ def linear_grouped(prep: Prepared, offsets: torch.Tensor, qw: QuantizedWeight, r
                    out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
     """Grouped dual-path FP4 linear: fp16 [rows, n_out] in grouped order,
     group g's rows through group g's weight."""
-    assert offsets.dtype == torch.int32 and offsets.is_cuda and offsets.is_contiguous()
+    _int32_vector(offsets, "offsets")
+    _cuda_here(prep.buf, "prep.buf")
+    _cuda_here(qw.buf, "qw.buf")
     if out is None:
         out = torch.empty((rows, qw.n_out), dtype=torch.float16, device=prep.buf.device)
-    assert out.dtype == torch.float16 and out.is_contiguous() and tuple(out.shape) == (rows, qw.n_out)
+    _require(out.dtype == torch.float16 and out.is_contiguous() and tuple(out.shape) == (rows, qw.n_out),
+             f"out must be a contiguous fp16 tensor of shape {(rows, qw.n_out)}")
+    _cuda_here(out, "out")
     optr = _ptr(out) if out.numel() else None
     _check(lib().sharq_linear_grouped(C.byref(prep.desc), _ptr(offsets), offsets.numel() - 1, rows, C.byref(qw.desc),
                                       optr, _stream(stream)), "sharq_linear_grouped")
