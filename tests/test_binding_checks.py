@@ -63,3 +63,55 @@ def test_group_view_range():
     qw = sq.QuantizedWeight(torch.zeros(16, dtype=torch.uint8), d)
     with pytest.raises(ValueError, match="out of range"):
         sq.group_view(qw, 2)
+
+
+class _AsCuda(torch.Tensor):
+    """A host tensor that reports itself as living on cuda:0, so that the
+    binding's checks can be driven on a machine without a GPU."""
+
+    @property
+    def is_cuda(self):
+        return True
+
+    @property
+    def device(self):
+        return torch.device("cuda", 0)
+
+
+def _as_cuda(t):
+    return t.as_subclass(_AsCuda)
+
+
+def test_valid_arguments_pass_the_checks_and_reach_the_library(monkeypatch):
+    from unittest import mock
+    fake = mock.MagicMock()
+    for name in ("sharq_weight_bytes", "sharq_prep_bytes", "sharq_weight_bytes_grouped", "sharq_gather_bytes",
+                 "sharq_weight_bytes_fused"):
+        getattr(fake, name).return_value = 4096
+    monkeypatch.setattr(sq, "lib", lambda: fake)
+    monkeypatch.setattr(sq, "_device_buffer", lambda n, dev: _as_cuda(torch.zeros(max(n, 1), dtype=torch.uint8)))
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a: mock.Mock(cuda_stream=0))
+    for name in ("sharq_quantize_weight", "sharq_prepare", "sharq_prepare_rms", "sharq_linear", "sharq_linear_bias",
+                 "sharq_quantize_weight_fused", "sharq_quantize_weight_grouped", "sharq_gather_rows",
+                 "sharq_prepare_grouped", "sharq_linear_grouped"):
+        getattr(fake, name).return_value = sq.OK
+
+    x = _as_cuda(_cpu16(16, 256))
+    g = _as_cuda(_cpu16(256))
+    p = sq.prepare(x, g, g)
+    sq.prepare(x, g, None, norm="rms", out=p)
+    qw = sq.quantize_weight(_as_cuda(_cpu16(64, 256)))
+    p.desc.m_tok, qw.desc.n_out = 16, 64  # what the library would have filled in
+    sq.linear(p, qw, out=_as_cuda(_cpu16(16, 64)), bias=_as_cuda(_cpu16(64)))
+    sq.quantize_weight_fused([_as_cuda(_cpu16(64, 256)), _as_cuda(_cpu16(32, 256))])
+    qg = sq.quantize_weight_grouped(_as_cuda(_cpu16(2, 64, 256)))
+    off = _as_cuda(torch.zeros(3, dtype=torch.int32))
+    gp = sq.gather_rows(p, _as_cuda(torch.zeros(4, dtype=torch.int32)), off, 4)
+    sq.prepare_grouped(x, off, g, None, norm="rms", out=gp)
+    qg.desc.n_out = 64
+    sq.linear_grouped(gp, off, qg, 4, out=_as_cuda(_cpu16(4, 64)))
+    for name in ("sharq_prepare", "sharq_prepare_rms", "sharq_quantize_weight", "sharq_linear_bias",
+                 "sharq_quantize_weight_fused", "sharq_quantize_weight_grouped", "sharq_gather_rows",
+                 "sharq_prepare_grouped", "sharq_linear_grouped"):
+        assert getattr(fake, name).called, name
