@@ -34,6 +34,11 @@
  *  - Kernels that wait on the hardware bound every wait; a wait that runs
  *    out records a status that sharq_get_last_error reports as
  *    SHARQ_ERR_TIMEOUT.
+ *  - Host threads may call the library concurrently (each with its own
+ *    buffers and streams): its per-device caches are filled once under a
+ *    lock. sharq_last_launch_count and sharq_last_timeout_site report the
+ *    most recent call of any thread; the device status word and the
+ *    no-allocation entry point's array are shared by all callers.
  */
 #ifndef SHARQ_H
 #define SHARQ_H

@@ -5,6 +5,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
+#include <mutex>
 #include <vector>
 
 #include "layout.h"
@@ -14,9 +16,11 @@ namespace {
 
 __device__ unsigned g_status;  // first timeout site since the last sharq_get_last_error
 
-uint64_t g_wait_ns = 2000000000ull;
-uint32_t g_last_site = 0;
-int g_last_launches = 0;
+// Process-wide settings and last-call diagnostics; atomics, so that callers on
+// several host threads read and write them without a data race.
+std::atomic<uint64_t> g_wait_ns{2000000000ull};
+std::atomic<uint32_t> g_last_site{0};
+std::atomic<int> g_last_launches{0};
 
 bool fmt_ok(int fmt) { return fmt == sq::kFmtNV || fmt == sq::kFmtMX; }
 bool nm_ok(int n, int m) { return (m == 2 || m == 4 || m == 8 || m == 16) && n >= 1 && n <= m; }
@@ -27,10 +31,12 @@ sharq_status make_ctx(void *stream, sq::LaunchCtx &ctx) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SHARQ_ERR_CUDA;
     static int sms[64] = {0};
+    static unsigned *status_ptr[64] = {nullptr};
+    static std::mutex mu;  // first calls from several host threads fill the caches once
+    std::lock_guard<std::mutex> lock(mu);
     if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
     if (!sms[dev] && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return SHARQ_ERR_CUDA;
-    static unsigned *status_ptr[64] = {nullptr};
     if (!status_ptr[dev] && cudaGetSymbolAddress((void **)&status_ptr[dev], g_status) != cudaSuccess)
         return SHARQ_ERR_CUDA;
     ctx.stream = reinterpret_cast<cudaStream_t>(stream);
@@ -125,8 +131,7 @@ const char *sharq_status_string(sharq_status s) {
 int sharq_last_launch_count(void) { return g_last_launches; }
 
 uint64_t sharq_set_wait_limit_ns(uint64_t ns) {
-    uint64_t old = g_wait_ns;
-    g_wait_ns = ns ? ns : 2000000000ull;
+    const uint64_t old = g_wait_ns.exchange(ns ? ns : 2000000000ull);
     return old;
 }
 

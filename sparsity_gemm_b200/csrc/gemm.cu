@@ -28,6 +28,8 @@
 #include <cuda_fp16.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "sharq_dev.cuh"
 #include "sq_internal.h"
 
@@ -666,9 +668,11 @@ static bool make_grouped_code_map(CUtensorMap *tm, const void *base, uint64_t ro
 template <int FMT, bool GROUPED, bool EXT, int BN>
 static sharq_status set_gemm_attrs() {
     static bool attr_done[64] = {};
+    static std::mutex mu;  // one setter per device, also under concurrent first calls
     int dev = 0;
     SQ_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
     if (!attr_done[dev]) {
         SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<FMT, GROUPED, EXT, BN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, TileCfg<BN>::kSmemBytes));
@@ -721,8 +725,10 @@ template <int FMT>
 static int active_clusters(int split) {
     static int cache[64][kMaxSplit + 1];
     static bool known[64][kMaxSplit + 1] = {};
+    static std::mutex mu;  // set_gemm_attrs below takes its own lock (never this one)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || split > kMaxSplit) return 0;
+    std::lock_guard<std::mutex> lock(mu);
     if (!known[dev][split]) {
         if (set_gemm_attrs<FMT, false, false, kDenseBN>() != SHARQ_OK) return 0;
         cudaLaunchConfig_t cfg;

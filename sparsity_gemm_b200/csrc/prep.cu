@@ -21,6 +21,8 @@
 
 #include <string.h>
 
+#include <mutex>
+
 #include "sharq_dev.cuh"
 #include "sq_internal.h"
 
@@ -1404,8 +1406,10 @@ static int64_t encode_grid(void *fn, int num_sms, int64_t total_units) {
     };
     static Entry cache[64];
     static int used = 0;
+    static std::mutex mu;  // lookups and appends from concurrent host threads
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    std::lock_guard<std::mutex> lock(mu);
     int occ = 0;
     for (int i = 0; i < used; ++i)
         if (cache[i].fn == fn && cache[i].dev == dev) occ = cache[i].occ;
@@ -1494,7 +1498,9 @@ static __device__ __align__(256) unsigned char g_prep_scratch[kStaticScratchByte
 // device (in host code the array's name is only a stand-in for the symbol).
 static sharq_status static_scratch(int dev, unsigned char **out) {
     static unsigned char *addr[64] = {nullptr};
+    static std::mutex mu;
     if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
     if (!addr[dev]) {
         unsigned char *p = nullptr;
         if (cudaGetSymbolAddress((void **)&p, g_prep_scratch) != cudaSuccess || !p) return SHARQ_ERR_CUDA;
@@ -1538,14 +1544,18 @@ extern "C" sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, 
     sharq_status st = static_scratch(dev, &scratch);
     if (st != SHARQ_OK) return st;
     static int sms[64] = {0};
-    if (!sms[dev] && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return SHARQ_ERR_CUDA;
     static bool attr_done[64] = {false};
-    if (!attr_done[dev]) {
-        if (cudaFuncSetAttribute(ln_stats_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)(2 * SHARQ_K_MAX)) != cudaSuccess)
+    {
+        static std::mutex mu;
+        std::lock_guard<std::mutex> lock(mu);
+        if (!sms[dev] && cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return SHARQ_ERR_CUDA;
-        attr_done[dev] = true;
+        if (!attr_done[dev]) {
+            if (cudaFuncSetAttribute(ln_stats_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)(2 * SHARQ_K_MAX)) != cudaSuccess)
+                return SHARQ_ERR_CUDA;
+            attr_done[dev] = true;
+        }
     }
 
     const PrepLayout L = prep_layout(m_tok, k, n, m, fmt);
@@ -1610,21 +1620,25 @@ template <bool RMS>
 static sharq_status launch_stats(LaunchCtx &ctx, const sharq_prep &P, const void *x, const void *gamma,
                                  const void *beta, float eps, float2 *stats, unsigned *words) {
     static bool attr_done[64] = {false};
+    static std::mutex mu;
     int dev = 0;
     SQ_CUDA_TRY(cudaGetDevice(&dev));
     if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
-    if (!attr_done[dev]) {
-        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_kernel<true, RMS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(2 * SHARQ_K_MAX)));
-        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<true, RMS, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
-        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<false, RMS, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
-        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<true, RMS, true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
-        SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<false, RMS, true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
-        attr_done[dev] = true;
+    {
+        std::lock_guard<std::mutex> lock(mu);  // held for the attribute set-up only
+        if (!attr_done[dev]) {
+            SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_kernel<true, RMS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)(2 * SHARQ_K_MAX)));
+            SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<true, RMS, false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
+            SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<false, RMS, false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
+            SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<true, RMS, true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
+            SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<false, RMS, true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
+            attr_done[dev] = true;
+        }
     }
     if (P.m_tok == 0) return SHARQ_OK;
     const bool warp_rows = P.m_tok >= (int64_t)ctx.num_sms * (kStatsThreads / 32) || P.k <= kWarpRowMaxK;
