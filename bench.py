@@ -322,7 +322,7 @@ def run_sharq(args, world, rank, local):
                      "peak_source": f"{peak_src} bf16 {peaks['bf16_tflops']} TF/s x {FP4_OVER_BF16} (FP4/BF16 nominal)",
                      "flops_per_step": flops_algorithmic(M), "flop_count": "2*M*N*K*(1+n/m)",
                      "executed_tflops": gemm_exec_tflops, "executed_frac": gemm_exec_tflops / fp4_peak},
-        "prep_roofline": {"bound": "hbm", "kernel": "ln_stats_kernel + prep_encode_kernel (4 preps)",
+        "prep_roofline": {"bound": "hbm", "kernel": "ln_stats_warp_kernel + prep_encode_kernel (4 preps)",
                           "achieved": prep_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                           "frac": prep_gbs / peaks["hbm_gbs"], "bytes_per_elem": PREP_BYTES_PER_ELEM},
         "split_ms_per_step": {"prep": prep_ms / steps, "gemm": gemm_ms / steps,
