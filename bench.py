@@ -24,6 +24,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -39,7 +40,23 @@ UNIT = "tokens/s"
 EPS = 1e-5
 N_KEEP, M_GROUP = 2, 4
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
-PREP_BYTES_PER_ELEM = 3.25  # x 2 + S codes 0.5 + mask metadata 0.125 + S scales 0.0625 + R codes 0.5 + R scales 0.0625
+
+
+def prep_bytes_per_elem(fmt, n, m, dense_s=False):
+    """Algorithmic bytes per activation element of one preparation: x read
+    (2), the backbone's codes compressed to its n of every m values
+    (0.5 n / m), the mask metadata (n indices of ceil(log2 m) bits per m),
+    one scale byte per block for S and for R (1/16 NVFP4, 1/32 MXFP4) and
+    the residual's codes (0.5). NVFP4 2:4: 3.0 B. dense_s=True counts the
+    backbone's codes as stored by the dense-backbone layout (0.5, zeros off
+    the mask): NVFP4 2:4 3.25 B."""
+    meta = n * max(1, (m - 1).bit_length()) / m / 8.0
+    s_codes = 0.5 if dense_s else 0.5 * n / m
+    return 2 + s_codes + meta + 2.0 / (16 if fmt == 0 else 32) + 0.5
+
+
+PREP_BYTES_PER_ELEM = prep_bytes_per_elem(0, N_KEEP, M_GROUP)  # 3.0
+PREP_BYTES_PER_ELEM_DENSE_S = prep_bytes_per_elem(0, N_KEEP, M_GROUP, dense_s=True)  # 3.25
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of the 7 GEMM launches of one M = 8192 step, from
 # one ncu capture of the current dual_gemm_kernel (dram__bytes_read.sum +
@@ -122,8 +139,7 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.proc = None
         self.gpu_index = gpu_index
-        self.path = os.path.join(ROOT, "gpurun_out" if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ".",
-                                 f".clocks_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"sharq_clocks_{os.getpid()}.csv")
 
     def __enter__(self):
         q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -324,7 +340,14 @@ def run_sharq(args, world, rank, local):
                      "executed_tflops": gemm_exec_tflops, "executed_frac": gemm_exec_tflops / fp4_peak},
         "prep_roofline": {"bound": "hbm", "kernel": "ln_stats_warp_kernel + prep_encode_kernel (4 preps)",
                           "achieved": prep_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                          "frac": prep_gbs / peaks["hbm_gbs"], "bytes_per_elem": PREP_BYTES_PER_ELEM},
+                          "frac": prep_gbs / peaks["hbm_gbs"], "bytes_per_elem": PREP_BYTES_PER_ELEM,
+                          "bytes_count": "algorithmic: x 2 + S codes 0.25 (n/m of 0.5) + metadata 0.125 + "
+                                         "S scales 0.0625 + R codes 0.5 + R scales 0.0625",
+                          "dense_s": {"bytes_per_elem": PREP_BYTES_PER_ELEM_DENSE_S,
+                                      "achieved": prep_gbs * PREP_BYTES_PER_ELEM_DENSE_S / PREP_BYTES_PER_ELEM,
+                                      "frac": prep_gbs * PREP_BYTES_PER_ELEM_DENSE_S / PREP_BYTES_PER_ELEM
+                                      / peaks["hbm_gbs"],
+                                      "note": "S codes as the dense-backbone layout stores them (0.5 B)"}},
         "split_ms_per_step": {"prep": prep_ms / steps, "gemm": gemm_ms / steps,
                               "gemm_each": {lin.name: float(gemm_each[j] / steps) for j, lin in enumerate(ls.linears)}},
         "gpu_launches": gpu_launches,
@@ -594,8 +617,7 @@ def run_case(args, world, rank, local):
         x = torch.from_numpy(synth.activations_student(0, M, K, outlier_frac=args.outlier_frac).view(np.float16)).to(dev)
         buf = sq.prepare(x, None, None, EPS, n, m, fmt)
         op = lambda: sq.prepare(x, None, None, EPS, n, m, fmt, out=buf)
-        meta = (K // m) * n * max(1, (m - 1).bit_length()) / 8.0 / K
-        per_elem = 2 + 0.5 + meta + 2.0 / (16 if fmt == 0 else 32) + 0.5
+        per_elem = prep_bytes_per_elem(fmt, n, m)
         work, unit, peak, bound = per_elem * M * K, "GB/s", peaks["hbm_gbs"], "hbm"
     elif kind == "linear":
         M, N, K = nums[:3]
@@ -702,14 +724,6 @@ def run_fused(args, M):
     return {"case": args.case, "tokens_per_s": M / (total / 1e3), "ms_per_step": total, "prep_ms": prep_ms,
             "gemm_ms": sum(each), "gemm_each": {"+".join(l.name for l in g): each[j] for j, g in enumerate(groups)},
             "steps": args.steps}
-
-
-def prep_bytes_per_elem(fmt, n, m):
-    """Algorithmic bytes per activation element of one preparation: x read
-    (2), S and R codes (0.5 each, S kept dense with zeros), the mask metadata
-    and two scale arrays (one byte per block of 16 or 32)."""
-    meta = n * max(1, (m - 1).bit_length()) / m / 8.0
-    return 2 + 0.5 + 0.5 + meta + 2.0 / (16 if fmt == 0 else 32)
 
 
 def time_layer_set(ls, M, fmt, n, m, steps, warmup):

@@ -216,8 +216,10 @@ sharq_status sharq_prepare_rms(const void *x_dev, int64_t m_tok, int64_t k, cons
  * allocator; code on a latency-critical path must not call cudaMalloc,
  * which waits for the device to go idle; and deployments that plan all
  * device memory ahead of time have no room for a per-call scratch region.
- * This entry point computes exactly what sharq_prepare computes (same
- * kernels, same results bit for bit) but keeps that working memory in one
+ * This entry point computes exactly what sharq_prepare computes (the same
+ * results bit for bit; its statistics always come from the one-CTA-per-row
+ * kernel, whose exact sums sharq_prepare's other statistics kernels equal)
+ * but keeps that working memory in one
  * fixed array compiled into the library: 256 + 8 * SHARQ_NOALLOC_MAX_ROWS
  * bytes (about 128 KB) on every GPU that loads the library, held until the
  * process exits. It calls no allocator.

@@ -22,6 +22,15 @@ std::atomic<uint64_t> g_wait_ns{2000000000ull};
 std::atomic<uint32_t> g_last_site{0};
 std::atomic<int> g_last_launches{0};
 
+}  // namespace
+
+namespace sq {
+// Last-call launch count for entry points outside this file.
+void note_launches(int n) { g_last_launches = n; }
+}  // namespace sq
+
+namespace {
+
 bool fmt_ok(int fmt) { return fmt == sq::kFmtNV || fmt == sq::kFmtMX; }
 bool nm_ok(int n, int m) { return (m == 2 || m == 4 || m == 8 || m == 16) && n >= 1 && n <= m; }
 bool k_ok(int64_t k) { return k > 0 && k <= SHARQ_K_MAX && k % SHARQ_K_ALIGN == 0; }

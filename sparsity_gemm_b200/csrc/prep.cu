@@ -1520,6 +1520,7 @@ extern "C" sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, 
                                               void *r_scales_dev, void *meta_dev, float *s_t_dev,
                                               sharq_prep *prep_out, void *stream) {
     using namespace sq;
+    note_launches(0);
     const bool fmt_ok = fmt == kFmtNV || fmt == kFmtMX;
     const bool nm_ok = (m == 2 || m == 4 || m == 8 || m == 16) && n >= 1 && n <= m;
     if (!fmt_ok || !nm_ok || k <= 0 || k > SHARQ_K_MAX || k % SHARQ_K_ALIGN != 0 || m_tok < 0 || !prep_out ||
@@ -1607,6 +1608,7 @@ extern "C" sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, 
     if (cudaLaunchKernel(fn, dim3((unsigned)blocks), dim3(kEncodeThreads), args, 0, s) != cudaSuccess)
         return SHARQ_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return SHARQ_ERR_CUDA;
+    note_launches(m_tok > 0 ? 2 : 1);  // statistics (rows only) and encode
     *prep_out = P;
     return SHARQ_OK;
 }

@@ -32,6 +32,8 @@ sharq_status launch_linear_grouped(LaunchCtx &ctx, const sharq_prep &P, const sh
 sharq_status launch_gather(LaunchCtx &ctx, const sharq_prep &S, const int32_t *row_idx, const int32_t *offsets,
                            int32_t groups, int64_t rows, const sharq_prep &D);
 sharq_status launch_wait_probe(LaunchCtx &ctx, uint64_t limit_ns);
+// Records the kernel count that sharq_last_launch_count reports.
+void note_launches(int n);
 sharq_status launch_div_check(LaunchCtx &ctx, uint64_t count, uint64_t seed, uint64_t *mismatches, float *examples);
 
 }  // namespace sq
