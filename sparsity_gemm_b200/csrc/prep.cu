@@ -584,6 +584,134 @@ ln_stats_warp_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
     }
 }
 
+// Statistics of rows longer than 2048 elements: one warp per row, the
+// warps of a persistent grid (every CTA resident) taking rows in increasing
+// order with the grid stride, so that no partial last wave is left. Certified
+// binary64 sums as in ln_stats_warp_kernel's FAST form, each warp finishing
+// its own rows (all lanes compute the same finish; undecided rows are summed
+// again exactly). Without gamma/beta the row's amax|X_ln| comes from its
+// min and max of x; with them the warp reads the row again (from L2). One
+// amax atomic per CTA. The kernel lets the encode pass launch at once: its
+// CTAs take an SM's slots only as this kernel's CTAs leave, and wait for
+// this kernel's completion before reading anything it writes.
+template <bool AFFINE, bool RMS>
+__global__ void __launch_bounds__(kStatsThreads)
+ln_stats_long_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ gamma,
+                     const uint16_t *__restrict__ beta, float eps, int64_t k, int64_t m_tok,
+                     float2 *__restrict__ stats, unsigned *__restrict__ amax_word) {
+    constexpr int W = kStatsThreads / 32;
+    extern __shared__ uint4 ring[];  // [warp][stage][vector j][lane]
+    __shared__ float red_max[W];
+    griddep_launch();
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nvec = (int)(k / 8);
+    const int nvl = nvec / 32;        // vectors per lane (k is a multiple of 256)
+    const int iters = (nvl + 3) / 4;  // four vectors per lane per iteration
+    uint4 *wring = ring + (size_t)warp * kStatsStages * 4 * 32;
+    const uint32_t wbase = smem_u32(wring);
+    const int64_t nwarps = (int64_t)gridDim.x * W;
+    float amax = 0.0f;
+    for (int64_t row = (int64_t)blockIdx.x * W + warp; row < m_tok; row += nwarps) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(x + row * k);
+        auto issue = [&](int it) {
+            if (it < iters) {
+                const int stg = it % kStatsStages;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    if (4 * it + j < nvl)
+                        cp_async16(wbase + (uint32_t)(((stg * 4 + j) * 32 + lane) * 16), xr + lane + 32 * (4 * it + j));
+            }
+            cp_async_commit();  // possibly empty: one group per iteration keeps the count uniform
+        };
+        FastLane f = {0.0, 0.0, 0.0};
+        uint32_t mx = 0xFC00FC00u, mn = 0x7C007C00u;  // (-inf, -inf), (+inf, +inf) as half2
+        auto consume = [&](const uint4 &v) {
+            fast_pair(v.x, f);
+            fast_pair(v.y, f);
+            fast_pair(v.z, f);
+            fast_pair(v.w, f);
+            if (!AFFINE) {
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(w4[q]));
+                    asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(w4[q]));
+                }
+            }
+        };
+        issue(0);
+        issue(1);
+        for (int it = 0; it < iters; ++it) {
+            cp_async_wait<1>();  // this lane's copies of iteration `it` have landed
+            const int stg = it % kStatsStages;
+            if (4 * it + 3 < nvl) {
+                const uint4 v0 = wring[(stg * 4 + 0) * 32 + lane], v1 = wring[(stg * 4 + 1) * 32 + lane];
+                const uint4 v2 = wring[(stg * 4 + 2) * 32 + lane], v3 = wring[(stg * 4 + 3) * 32 + lane];
+                consume(v0);
+                consume(v1);
+                consume(v2);
+                consume(v3);
+            } else {
+                for (int j = 0; 4 * it + j < nvl; ++j) consume(wring[(stg * 4 + j) * 32 + lane]);
+            }
+            issue(it + 2);  // refills the slot consumed in the previous iteration
+        }
+        cp_async_wait<0>();
+        // Butterfly reductions: every lane ends with the same totals.
+        int64_t s1 = __double2ll_rn(__dmul_rn(f.s1, 16777216.0));  // sum a over the lane, an integer below 2^51
+        double s2 = __dadd_rn(f.s2a, f.s2b);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
+            s2 = __dadd_rn(s2, __shfl_xor_sync(0xFFFFFFFFu, s2, o));
+            if (!AFFINE) {
+                const uint32_t omx = __shfl_xor_sync(0xFFFFFFFFu, mx, o), omn = __shfl_xor_sync(0xFFFFFFFFu, mn, o);
+                asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(omx));
+                asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(omn));
+            }
+        }
+        float2 st;
+        const bool ok = certified_stats(s1, s2, k, eps, RMS, st);  // the same on every lane
+        if (!ok) st = exact_row_stats<RMS>(xr, nvec, lane, k, eps);
+        if (lane == 0) stats[row] = st;
+        if (!AFFINE) {
+            // X_ln = RN(RN(x - mu) * rstd) is non-decreasing in x: the row's
+            // amax|X_ln| is reached at its smallest or largest x.
+            const float xmax = fmaxf(h2f((uint16_t)mx), h2f((uint16_t)(mx >> 16)));
+            const float xmin = fminf(h2f((uint16_t)mn), h2f((uint16_t)(mn >> 16)));
+            amax = fmaxf(amax, fmaxf(fabsf(__fmul_rn(__fsub_rn(xmax, st.x), st.y)),
+                                     fabsf(__fmul_rn(__fsub_rn(xmin, st.x), st.y))));
+        } else {
+            const bool has_g = gamma != nullptr, has_b = beta != nullptr;
+            for (int cc = lane; cc < nvec; cc += 32) {
+                const uint4 v = xr[cc];
+                const uint4 g = has_g ? __ldg(reinterpret_cast<const uint4 *>(gamma) + cc) : make_uint4(0, 0, 0, 0);
+                const uint4 bb = has_b ? __ldg(reinterpret_cast<const uint4 *>(beta) + cc) : make_uint4(0, 0, 0, 0);
+                const uint32_t xv[4] = {v.x, v.y, v.z, v.w}, gv[4] = {g.x, g.y, g.z, g.w},
+                               bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const float xl = ln_apply(h2f((uint16_t)(xv[q] >> (16 * h))), st.x, st.y, has_g,
+                                                  h2f((uint16_t)(gv[q] >> (16 * h))), has_b,
+                                                  h2f((uint16_t)(bv[q] >> (16 * h))));
+                        amax = fmaxf(amax, fabsf(xl));
+                    }
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    if (lane == 0) red_max[warp] = amax;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float a = 0.0f;
+        for (int w = 0; w < W; ++w) a = fmaxf(a, red_max[w]);
+        atomicMax(amax_word, __float_as_uint(a));  // non-negative floats order like their bits
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Encode pass.
 
@@ -801,6 +929,66 @@ __device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, 
     return d;
 }
 
+// The encode arithmetic of one unit of 16 LayerNorm outputs v: mask, Q(S),
+// R = X_ln - deq(Q(S)), Q(R) and the mask metadata bits of the unit's
+// groups (n kept positions per group, ascending, LSB-first).
+struct UnitCodes {
+    uint32_t s_lo, s_hi, r_lo, r_hi;  // E2M1 codes of S and R, eight per word
+    uint32_t s_scale, r_scale;        // block scale codes
+    uint64_t mbits;                   // metadata bits of the unit
+};
+
+template <int FMT, int M, int NK>
+__device__ __forceinline__ void encode_core(const float (&v)[kUnit], int n, const uint32_t *lut, const float4 *tab,
+                                            float s_t, float c6, float y6, UnitCodes &o) {
+    constexpr int IB = M <= 2 ? 1 : M <= 4 ? 2 : M <= 8 ? 3 : 4;
+    constexpr int G = kUnit / M;  // mask groups per unit
+    const int gbits = n * IB;     // metadata bits per group
+    // Mask, and Q(S) for the backbone S = X_ln on the mask, +0 elsewhere.
+    // Every group keeps its largest magnitude (n >= 1), so the block amax
+    // of S is that of X_ln (over the lane pair too, for MXFP4) and so are
+    // the step and the codes on the mask: Q(S) is the encoding of X_ln with
+    // the dropped positions' nibbles cleared to the +0 code of S's zeros.
+    uint32_t keep;
+    if constexpr (M == 4 && NK == 2)
+        keep = keep_mask_42(v);
+    else
+        keep = keep_mask<M>(v, n);
+    const float ds = quantize16<FMT>(v, s_t, c6, y6, tab, o.s_scale, o.s_lo, o.s_hi);
+    o.s_lo &= nibble_mask8(keep);
+    o.s_hi &= nibble_mask8(keep >> 8);
+
+    // Residual against the quantized backbone: R = RN32(X_ln - RN32(value * d)).
+    // Scalar intrinsics: the product must be rounded before the subtraction.
+    float r[kUnit];
+#pragma unroll
+    for (int i = 0; i < kUnit; i += 2) {
+        const uint32_t byte = ((i < 8 ? o.s_lo : o.s_hi) >> (4 * (i % 8))) & 0xFFu;
+        const float2 cv = e2m1x2_value(byte);
+        r[i] = __fsub_rn(v[i], __fmul_rn(cv.x, ds));
+        r[i + 1] = __fsub_rn(v[i + 1], __fmul_rn(cv.y, ds));
+    }
+    quantize16<FMT>(r, s_t, c6, y6, tab, o.r_scale, o.r_lo, o.r_hi);
+
+    // Mask metadata: each group holds exactly n kept positions, so its
+    // field sits at a fixed offset of the unit's bit range.
+    uint64_t mbits = 0;
+    if (M <= 8) {
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            mbits |= (uint64_t)lut[(keep >> (g * M)) & ((1u << M) - 1u)] << (g * gbits);
+    } else {
+        int pos = 0;
+#pragma unroll
+        for (int i = 0; i < M; ++i)
+            if ((keep >> i) & 1u) {
+                mbits |= (uint64_t)i << pos;
+                pos += IB;
+            }
+    }
+    o.mbits = mbits;
+}
+
 // Arguments of the encode step (one unit = 16 consecutive elements of a row).
 struct EncodeArgs {
     const uint16_t *x, *gamma, *beta;
@@ -884,50 +1072,11 @@ __device__ __forceinline__ void encode_unit(const EncodeArgs &a, const uint32_t 
         }
     }
 
-    // Mask, and Q(S) for the backbone S = X_ln on the mask, +0 elsewhere.
-    // Every group keeps its largest magnitude (n >= 1), so the block amax
-    // of S is that of X_ln (over the lane pair too, for MXFP4) and so are
-    // the step and the codes on the mask: Q(S) is the encoding of X_ln with
-    // the dropped positions' nibbles cleared to the +0 code of S's zeros.
-    uint32_t keep;
-    if constexpr (M == 4 && NK == 2)
-        keep = keep_mask_42(v);
-    else
-        keep = keep_mask<M>(v, n);
-    uint32_t s_scale, s_lo, s_hi;
-    const float ds = quantize16<FMT>(v, s_t, c6, y6, tab, s_scale, s_lo, s_hi);
-    s_lo &= nibble_mask8(keep);
-    s_hi &= nibble_mask8(keep >> 8);
-
-    // Residual against the quantized backbone: R = RN32(X_ln - RN32(value * d)).
-    // Scalar intrinsics: the product must be rounded before the subtraction.
-    float r[kUnit];
-#pragma unroll
-    for (int i = 0; i < kUnit; i += 2) {
-        const uint32_t byte = ((i < 8 ? s_lo : s_hi) >> (4 * (i % 8))) & 0xFFu;
-        const float2 cv = e2m1x2_value(byte);
-        r[i] = __fsub_rn(v[i], __fmul_rn(cv.x, ds));
-        r[i + 1] = __fsub_rn(v[i + 1], __fmul_rn(cv.y, ds));
-    }
-    uint32_t r_scale, r_lo, r_hi;
-    quantize16<FMT>(r, s_t, c6, y6, tab, r_scale, r_lo, r_hi);
-
-    // Mask metadata: each group holds exactly n kept positions, so its
-    // field sits at a fixed offset of the unit's bit range.
-    uint64_t mbits = 0;
-    if (M <= 8) {
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-            mbits |= (uint64_t)lut[(keep >> (g * M)) & ((1u << M) - 1u)] << (g * gbits);
-    } else {
-        int pos = 0;
-#pragma unroll
-        for (int i = 0; i < M; ++i)
-            if ((keep >> i) & 1u) {
-                mbits |= (uint64_t)i << pos;
-                pos += IB;
-            }
-    }
+    UnitCodes o;
+    encode_core<FMT, M, NK>(v, n, lut, tab, s_t, c6, y6, o);
+    const uint32_t s_lo = o.s_lo, s_hi = o.s_hi, r_lo = o.r_lo, r_hi = o.r_hi;
+    const uint32_t s_scale = o.s_scale, r_scale = o.r_scale;
+    const uint64_t mbits = o.mbits;
 
     if (real) {
         *reinterpret_cast<uint2 *>(s_codes + orow * (k / 2) + u * 8) = make_uint2(s_lo, s_hi);
@@ -1015,6 +1164,171 @@ prep_encode_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ 
             ++row_i;
         }
         encode_unit<FMT, M, NK>(ea, lut, tab, row, u, active, s_t, c6, y6);
+    }
+}
+
+// Encode pass over the rows of one activation: one warp per 512-element
+// chunk of a row (a lane per 16-element unit), the chunks of the persistent
+// grid's warps taken in reverse row order. The statistics pass reads the rows
+// in increasing order, so the rows it read last (still in L2 when x is
+// larger than L2) are the ones this pass reads first. Per chunk: one 32-byte
+// load per lane, the row's statistics once, and addresses from per-row bases.
+// The next chunk's loads are issued before the current chunk is encoded.
+// Padding rows of the scale layouts (m_tok .. sf_rows - 1) are zeroed after
+// the main loop. Launched with programmatic stream serialization: the look-up
+// tables are built before griddep_wait, everything the statistics pass wrote
+// is read after it.
+template <int FMT, int M, int NK, bool AFFINE>
+__global__ void __launch_bounds__(kEncodeThreads, SQ_ENCODE_MIN_CTAS)
+prep_encode_rows_kernel(const EncodeArgs a, const unsigned *amax_word, float *__restrict__ s_t_out,
+                        int64_t sf_rows) {
+    constexpr int IB = M <= 2 ? 1 : M <= 4 ? 2 : M <= 8 ? 3 : 4;
+    __shared__ uint32_t lut[M <= 8 ? (1 << M) : 1];  // keep bits of a group -> kept positions, ascending
+    __shared__ float4 tab[128];                       // NVFP4 steps and reciprocals by scale code
+    if (M <= 8)
+        for (int msk = threadIdx.x; msk < (1 << M); msk += kEncodeThreads) {
+            uint32_t packed = 0;
+            int pos = 0;
+            for (int i = 0; i < M; ++i)
+                if ((msk >> i) & 1) {
+                    packed |= (uint32_t)i << pos;
+                    pos += IB;
+                }
+            lut[msk] = packed;
+        }
+    griddep_wait();  // the statistics and the amax word are complete
+    // What the statistics kernel wrote is read with L2 loads through pointers
+    // without __restrict__, so that no load can move above the wait.
+    const float amax = __uint_as_float(__ldcg(amax_word));
+    const float s_t = (FMT == kFmtNV && amax != 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+    const float c6 = __fmul_rn(6.0f, s_t);
+    const float y6 = (FMT == kFmtNV && c6 >= 0x1p-90f && c6 <= 0x1p90f) ? __frcp_rn(c6) : 0.0f;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *s_t_out = s_t;
+    build_step_table<FMT>(tab, s_t);
+    __syncthreads();
+
+    const uint16_t *__restrict__ x = a.x;
+    const float2 *stats = a.stats;
+    uint8_t *__restrict__ s_codes = a.s_codes;
+    uint8_t *__restrict__ r_codes = a.r_codes;
+    uint8_t *__restrict__ s_sf = a.s_sf;
+    uint8_t *__restrict__ r_sf = a.r_sf;
+    uint8_t *__restrict__ meta = a.meta;
+    const int64_t k = a.k, m_tok = a.m_tok, nblk = a.nblk, meta_row = a.meta_row;
+    const int n = NK > 0 ? NK : a.n;
+    const int B = (kUnit / M) * n * IB;  // metadata bits per unit
+    const bool byte_aligned = (B & 7) == 0;
+    const int lane = threadIdx.x & 31;
+    const int upr = (int)(k / kUnit);         // units per row
+    const int chunks = (upr + 31) >> 5;       // 32-unit chunks per row
+    const int64_t nwarps = (int64_t)gridDim.x * (kEncodeThreads / 32);
+    const int64_t gw = (int64_t)blockIdx.x * (kEncodeThreads / 32) + threadIdx.x / 32;
+    const int64_t items = m_tok * chunks;
+    const int64_t step_r = nwarps / chunks;
+    const int step_c = (int)(nwarps - step_r * chunks);
+
+    // Item `it` is chunk it % chunks of row m_tok - 1 - it / chunks.
+    int64_t ri = gw / chunks;
+    int ci = (int)(gw - ri * chunks);
+    uint32_t xw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    float2 st = make_float2(0.0f, 1.0f);
+    // one 32-byte load where x is 32-byte aligned (every unit then is), else two
+    const bool x32 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0;
+    auto fetch = [&](int64_t r, int c, uint32_t (&w)[8], float2 &sv) {
+        const int u = c * 32 + lane;
+        if (u < upr) {
+            const uint16_t *p = x + r * k + (int64_t)u * kUnit;
+            if (x32) {
+                ldg256_cs(p, w);
+            } else {
+                const uint4 va = __ldcs(reinterpret_cast<const uint4 *>(p)), vb = __ldcs(reinterpret_cast<const uint4 *>(p) + 1);
+                w[0] = va.x, w[1] = va.y, w[2] = va.z, w[3] = va.w, w[4] = vb.x, w[5] = vb.y, w[6] = vb.z, w[7] = vb.w;
+            }
+        }
+        sv = __ldcg(stats + r);
+    };
+    if (gw < items) fetch(m_tok - 1 - ri, ci, xw, st);
+    for (int64_t it = gw; it < items; it += nwarps) {
+        const int64_t row = m_tok - 1 - ri;
+        const int u = ci * 32 + lane;
+        const bool act = u < upr;
+        ri += step_r;
+        ci += step_c;
+        if (ci >= chunks) {
+            ci -= chunks;
+            ++ri;
+        }
+        // the next chunk's loads go out before this chunk is encoded
+        uint32_t nw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        float2 nst = make_float2(0.0f, 1.0f);
+        if (it + nwarps < items) fetch(m_tok - 1 - ri, ci, nw, nst);
+
+        float v[kUnit];
+        {
+            // (x - mu) * rstd in packed pairs (no multiply feeds an add here);
+            // gamma and beta with scalar intrinsics, which are never fused.
+            const uint64_t mu2 = pk2(st.x, st.x), rs2 = pk2(st.y, st.y);
+            uint4 ga = make_uint4(0, 0, 0, 0), gb = ga, ba = ga, bb = ga;
+            if (AFFINE && act) {
+                if (a.gamma) {
+                    ga = __ldg(reinterpret_cast<const uint4 *>(a.gamma + (int64_t)u * kUnit));
+                    gb = __ldg(reinterpret_cast<const uint4 *>(a.gamma + (int64_t)u * kUnit) + 1);
+                }
+                if (a.beta) {
+                    ba = __ldg(reinterpret_cast<const uint4 *>(a.beta + (int64_t)u * kUnit));
+                    bb = __ldg(reinterpret_cast<const uint4 *>(a.beta + (int64_t)u * kUnit) + 1);
+                }
+            }
+            const uint32_t gw8[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+            const uint32_t bw8[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                float2 f = up2(mul2(sub2(h2_to_f2(xw[p]), mu2), rs2));
+                if (AFFINE) {
+                    if (a.gamma) {
+                        f.x = __fmul_rn(f.x, h2f((uint16_t)gw8[p]));
+                        f.y = __fmul_rn(f.y, h2f((uint16_t)(gw8[p] >> 16)));
+                    }
+                    if (a.beta) {
+                        f.x = __fadd_rn(f.x, h2f((uint16_t)bw8[p]));
+                        f.y = __fadd_rn(f.y, h2f((uint16_t)(bw8[p] >> 16)));
+                    }
+                }
+                v[2 * p] = f.x;
+                v[2 * p + 1] = f.y;
+            }
+        }
+        UnitCodes o;
+        encode_core<FMT, M, NK>(v, n, lut, tab, s_t, c6, y6, o);
+        if (act) {
+            const int64_t cofs = row * (k / 2) + (int64_t)u * 8;
+            *reinterpret_cast<uint2 *>(s_codes + cofs) = make_uint2(o.s_lo, o.s_hi);
+            *reinterpret_cast<uint2 *>(r_codes + cofs) = make_uint2(o.r_lo, o.r_hi);
+            if (FMT == kFmtNV) {
+                const int64_t so = sf_offset(row, u, nblk);
+                s_sf[so] = (uint8_t)o.s_scale;
+                r_sf[so] = (uint8_t)o.r_scale;
+            } else if ((u & 1) == 0) {
+                const int64_t so = sf_offset(row, u >> 1, nblk);
+                s_sf[so] = (uint8_t)o.s_scale;
+                r_sf[so] = (uint8_t)o.r_scale;
+            }
+            if (byte_aligned)
+                store_bytes(meta + row * meta_row + (int64_t)u * (B / 8), o.mbits, B / 8);
+            else
+                or_bits(reinterpret_cast<uint32_t *>(meta), (uint64_t)row * meta_row * 8 + (uint64_t)u * B, o.mbits, B);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xw[i] = nw[i];
+        st = nst;
+    }
+    // Zero scales of the padding rows of the last 128-row scale atoms.
+    const int64_t pad = (sf_rows - m_tok) * nblk;
+    const int64_t gthreads = (int64_t)gridDim.x * kEncodeThreads;
+    for (int64_t i = (int64_t)blockIdx.x * kEncodeThreads + threadIdx.x; i < pad; i += gthreads) {
+        const int64_t r = m_tok + i / nblk, j = i - (i / nblk) * nblk;
+        s_sf[sf_offset(r, j, nblk)] = 0;
+        r_sf[sf_offset(r, j, nblk)] = 0;
     }
 }
 
@@ -1433,6 +1747,45 @@ static void *encode_fn(int m, int n) {
     }
 }
 
+template <int FMT, bool AFFINE>
+static void *encode_rows_fn(int m, int n) {
+    switch (m) {
+        case 2: return (void *)prep_encode_rows_kernel<FMT, 2, 0, AFFINE>;
+        case 4: return n == 2 ? (void *)prep_encode_rows_kernel<FMT, 4, 2, AFFINE>
+                              : (void *)prep_encode_rows_kernel<FMT, 4, 0, AFFINE>;
+        case 8: return (void *)prep_encode_rows_kernel<FMT, 8, 0, AFFINE>;
+        default: return (void *)prep_encode_rows_kernel<FMT, 16, 0, AFFINE>;
+    }
+}
+
+// Grid of a persistent kernel: every CTA resident at once (SMs x resident
+// CTAs per SM for `threads` threads and `smem` dynamic shared memory), at
+// most `blocks`.
+static int64_t resident_grid(void *fn, int num_sms, int threads, size_t smem, int64_t blocks) {
+    struct Entry {
+        void *fn;
+        int dev, occ;
+    };
+    static Entry cache[64];
+    static int used = 0;
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    int occ = 0;
+    for (int i = 0; i < used; ++i)
+        if (cache[i].fn == fn && cache[i].dev == dev) occ = cache[i].occ;
+    if (occ == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, threads, smem) != cudaSuccess || occ < 1) {
+            cudaGetLastError();
+            occ = 1;
+        }
+        if (used < 64) cache[used++] = Entry{fn, dev, occ};
+    }
+    const int64_t cap = (int64_t)num_sms * occ;
+    return blocks < cap ? blocks : cap;
+}
+
 template <int FMT>
 static void *encode_grouped_fn(int m, int n) {
     switch (m) {
@@ -1639,6 +1992,10 @@ static sharq_status launch_stats(LaunchCtx &ctx, const sharq_prep &P, const void
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
             SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_warp_kernel<false, RMS, true>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
+            SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_long_kernel<true, RMS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
+            SQ_CUDA_TRY(cudaFuncSetAttribute(ln_stats_long_kernel<false, RMS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kStatsRingBytes));
             attr_done[dev] = true;
         }
     }
@@ -1656,9 +2013,17 @@ static sharq_status launch_stats(LaunchCtx &ctx, const sharq_prep &P, const void
         const int64_t per_cta = (int64_t)(kStatsThreads / 32) * rpw;
         const unsigned grid = (unsigned)((P.m_tok + per_cta - 1) / per_cta);
         // Rows longer than 2048 elements take the certified sums (two finishes
-        // per row, which short rows would feel).
+        // per row, which short rows would feel), in the persistent kernel.
         const bool fast = P.k > 2048;
-        if (gamma || beta) {
+        if (fast) {
+            void *fn = (gamma || beta) ? (void *)ln_stats_long_kernel<true, RMS> : (void *)ln_stats_long_kernel<false, RMS>;
+            const int64_t need = (P.m_tok + (kStatsThreads / 32) - 1) / (kStatsThreads / 32);
+            const unsigned lgrid = (unsigned)resident_grid(fn, ctx.num_sms, kStatsThreads, kStatsRingBytes, need);
+            float e = eps;
+            int64_t kk = P.k, mt = P.m_tok;
+            void *args[] = {&xx, &gg, &bb, &e, &kk, &mt, &stats, &words};
+            SQ_CUDA_TRY(cudaLaunchKernel(fn, dim3(lgrid), dim3(kStatsThreads), args, kStatsRingBytes, ctx.stream));
+        } else if (gamma || beta) {
             auto fn = fast ? ln_stats_warp_kernel<true, RMS, true> : ln_stats_warp_kernel<true, RMS, false>;
             fn<<<grid, kStatsThreads, kStatsRingBytes, ctx.stream>>>(xx, gg, bb, eps, P.k, P.m_tok, 1, stats, words);
         } else {
@@ -1695,19 +2060,32 @@ sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, 
     const sharq_status sst = norm ? launch_stats<true>(ctx, P, x, gamma, beta, eps, stats, words)
                                   : launch_stats<false>(ctx, P, x, gamma, beta, eps, stats, words);
     if (sst != SHARQ_OK) return sst;
-    const int64_t total = P.sf_rows * (P.k / kUnit);
-    void *fn = P.fmt == kFmtNV ? encode_fn<kFmtNV>(P.m, P.n) : encode_fn<kFmtMX>(P.m, P.n);
-    const int64_t blocks = encode_grid(fn, ctx.num_sms, total);
-    const uint16_t *xx = (const uint16_t *)x, *gg = (const uint16_t *)gamma, *bb = (const uint16_t *)beta;
-    const float2 *cst = stats;
+    const bool affine = gamma != nullptr || beta != nullptr;
+    void *fn = P.fmt == kFmtNV ? (affine ? encode_rows_fn<kFmtNV, true>(P.m, P.n) : encode_rows_fn<kFmtNV, false>(P.m, P.n))
+                               : (affine ? encode_rows_fn<kFmtMX, true>(P.m, P.n) : encode_rows_fn<kFmtMX, false>(P.m, P.n));
+    const int64_t chunks = (P.k / kUnit + 31) / 32;
+    const int64_t warps = P.m_tok * chunks > 0 ? P.m_tok * chunks : 1;
+    const int64_t blocks = encode_grid(fn, ctx.num_sms, warps * 32);
+    EncodeArgs ea{(const uint16_t *)x, (const uint16_t *)gamma, (const uint16_t *)beta, stats, P.m_tok, P.k,
+                  P.meta_row_bytes, P.k / (P.fmt == kFmtNV ? 16 : 32), P.n, (uint8_t *)P.s_codes,
+                  (uint8_t *)P.r_codes, (uint8_t *)P.s_scales, (uint8_t *)P.r_scales, (uint8_t *)P.meta};
     const unsigned *aw = words;
-    float *st = P.tensor_scale;
-    int64_t m_tok = P.m_tok, sf_rows = P.sf_rows, k = P.k, meta_row = P.meta_row_bytes;
-    int n = P.n;
-    uint8_t *sc = (uint8_t *)P.s_codes, *rc = (uint8_t *)P.r_codes, *ss = (uint8_t *)P.s_scales,
-            *rs = (uint8_t *)P.r_scales, *mt = (uint8_t *)P.meta;
-    void *args[] = {&xx, &gg, &bb, &cst, &aw, &st, &m_tok, &sf_rows, &k, &n, &sc, &rc, &ss, &rs, &mt, &meta_row};
-    SQ_CUDA_TRY(cudaLaunchKernel(fn, dim3((unsigned)blocks), dim3(kEncodeThreads), args, 0, ctx.stream));
+    float *sto = P.tensor_scale;
+    int64_t sf_rows = P.sf_rows;
+    void *args[] = {&ea, &aw, &sto, &sf_rows};
+    // Programmatic dependent launch: the encode may start while the
+    // statistics kernel finishes (it waits for it before reading).
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)blocks, 1, 1);
+    cfg.blockDim = dim3(kEncodeThreads, 1, 1);
+    cfg.stream = ctx.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = P.m_tok > 0 ? 1 : 0;  // no statistics kernel before it otherwise
+    SQ_CUDA_TRY(cudaLaunchKernelExC(&cfg, fn, args));
     ctx.launches++;
     return SHARQ_OK;
 }

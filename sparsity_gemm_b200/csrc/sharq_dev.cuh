@@ -285,6 +285,23 @@ __device__ __forceinline__ uint32_t e2m1_pair(uint64_t q, uint32_t sign_lo, uint
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization may start while the kernel before it in the stream is still
+// running; griddep_wait blocks until that kernel has completed and its memory
+// is visible, so everything before it must not read what the previous kernel
+// writes. griddep_launch lets the next kernel (if launched that way) start
+// its own launch and set-up early.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// 32 bytes of global memory (p 32-byte aligned), streaming: read once.
+__device__ __forceinline__ void ldg256_cs(const void *p, uint32_t (&r)[8]) {
+    asm volatile("ld.global.cs.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "l"(p));
+}
+
+// ---------------------------------------------------------------------------
 // Shared-memory and barrier primitives
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
