@@ -60,6 +60,11 @@ def _declare(L):
     L.oracle_prepare_norm.argtypes = [vp, i64, i64, vp, vp, f32, i32, i32, i32, i32] + [vp] * 14
     L.oracle_quantize_weight.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp]
     L.oracle_linear.argtypes = [vp, vp, vp, vp, f32, vp, vp, f32, i64, i64, i64, i32, vp, vp]
+    L.oracle_mask_pairs48.argtypes = [vp, i64, i64, vp, vp]
+    L.oracle_quantize_blk.argtypes = [vp, i64, i64, i32, i32, f32, vp, vp]
+    L.oracle_prepare_sparse.argtypes = [vp, i64, i64, vp, vp, f32, i32, i32] + [vp] * 14
+    L.oracle_quantize_weight_blk.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, vp]
+    L.oracle_linear_blk.argtypes = [vp, vp, i32, vp, vp, i32, f32, vp, vp, i32, f32, i64, i64, i64, i32, vp, vp]
 
 
 def _u16(a):
@@ -346,3 +351,94 @@ def linear_fused(p: Prepared, qws: list, bias=None, rows=None):
         out = out + b[None, :]
         bound = bound + np.abs(b)[None, :]
     return out, bound
+
+
+# --------------------------------------------------------------------------
+# Pair-wise 4:8 sparse-backbone mode (the pattern the sparse block-scaled FP4
+# tensor-core instructions accept). In every aligned group of 8 along K the
+# two of the four adjacent pairs with the largest max(|a|, |b|) are kept
+# (equal: the lower pair); the backbone and the weights use blocks twice the
+# format's length (NVFP4 32, MXFP4 64); the residual keeps the format's own.
+
+SPARSE_BLOCK = {NVFP4: 32, MXFP4: 64}
+
+
+def mask_pairs48(x_ln: np.ndarray):
+    x_ln = np.ascontiguousarray(x_ln, np.float32)
+    rows, k = x_ln.shape
+    idx = np.empty((rows, k // 8, 4), np.uint8)
+    keep = np.empty((rows, k), np.uint8)
+    lib().oracle_mask_pairs48(_p(x_ln), rows, k, _p(idx), _p(keep))
+    return idx, keep
+
+
+def quantize_blk(v: np.ndarray, fmt: int, blk: int, s_t: float):
+    v = np.ascontiguousarray(v, np.float32)
+    rows, k = v.shape
+    codes = np.empty((rows, k), np.uint8)
+    scales = np.empty((rows, k // blk), np.uint8)
+    lib().oracle_quantize_blk(_p(v), rows, k, fmt, blk, float(s_t), _p(codes), _p(scales))
+    return codes, scales
+
+
+def prepare_sparse(x, gamma, beta, eps: float, fmt: int, s_t=None, norm: str = "layer") -> Prepared:
+    """The preparation operator in the pair-wise 4:8 mode (n = 4, m = 8 in
+    the result; s_scales has one scale per SPARSE_BLOCK[fmt] values)."""
+    assert norm in NORMS and (norm == "layer" or beta is None)
+    x = _u16(x)
+    rows, k = x.shape
+    g = None if gamma is None else _u16(gamma)
+    b = None if beta is None else _u16(beta)
+    f = lambda: np.empty((rows, k), np.float32)
+    mu, rstd = np.empty(rows, np.float32), np.empty(rows, np.float32)
+    x_ln, s, deq_s, r = f(), f(), f(), f()
+    idx = np.empty((rows, k // 8, 4), np.uint8)
+    keep = np.empty((rows, k), np.uint8)
+    s_codes, r_codes = np.empty((rows, k), np.uint8), np.empty((rows, k), np.uint8)
+    s_scales = np.empty((rows, k // SPARSE_BLOCK[fmt]), np.uint8)
+    r_scales = np.empty((rows, k // BLOCK[fmt]), np.uint8)
+    s_t_arr = np.empty(1, np.float32)
+    s_t_in = None if s_t is None else np.array([s_t], np.float32)
+    lib().oracle_prepare_sparse(_p(x), rows, k, _p(g), _p(b), eps, fmt, NORMS[norm],
+                                _p(mu), _p(rstd), _p(x_ln), _p(s), _p(deq_s), _p(r),
+                                _p(idx), _p(keep), _p(s_codes), _p(s_scales),
+                                _p(r_codes), _p(r_scales), _p(s_t_arr), _p(s_t_in))
+    return Prepared(mu, rstd, x_ln, s, deq_s, r, idx, keep, s_codes, s_scales,
+                    r_codes, r_scales, s_t_arr[0], fmt, 4, 8)
+
+
+def quantize_weight_sparse(w, fmt: int) -> QWeight:
+    """Weights for the pair-wise mode: blocks of SPARSE_BLOCK[fmt]."""
+    w = _u16(w)
+    n_out, k = w.shape
+    blk = SPARSE_BLOCK[fmt]
+    w_f32 = np.empty((n_out, k), np.float32)
+    codes = np.empty((n_out, k), np.uint8)
+    scales = np.empty((n_out, k // blk), np.uint8)
+    s_tw = np.empty(1, np.float32)
+    lib().oracle_quantize_weight_blk(_p(w), n_out, k, fmt, blk, _p(w_f32), _p(codes), _p(scales), _p(s_tw))
+    return QWeight(w_f32, codes, scales, s_tw[0], fmt)
+
+
+def linear_blk(s_codes, s_scales, blk_s, r_codes, r_scales, blk_r, s_t, w_codes, w_scales, blk_w, s_tw, fmt,
+               want_bound: bool = True):
+    """fp64 dual-path output and its tolerance scale with explicit block
+    lengths of the three scale arrays."""
+    arr = lambda a: np.ascontiguousarray(a, np.uint8)
+    s_codes, r_codes, w_codes = arr(s_codes), arr(r_codes), arr(w_codes)
+    s_scales, r_scales, w_scales = arr(s_scales), arr(r_scales), arr(w_scales)
+    rows, k = s_codes.shape
+    n_out = w_codes.shape[0]
+    out = np.empty((rows, n_out), np.float64)
+    bound = np.empty((rows, n_out), np.float64) if want_bound else None
+    lib().oracle_linear_blk(_p(s_codes), _p(s_scales), blk_s, _p(r_codes), _p(r_scales), blk_r, float(s_t),
+                            _p(w_codes), _p(w_scales), blk_w, float(s_tw), rows, n_out, k, fmt,
+                            _p(out), _p(bound))
+    return out, bound
+
+
+def linear_sparse(p: Prepared, qw: QWeight, rows=None):
+    """Dual-path output for a pair-wise-mode activation and weight."""
+    sel = slice(None) if rows is None else rows
+    return linear_blk(p.s_codes[sel], p.s_scales[sel], SPARSE_BLOCK[p.fmt], p.r_codes[sel], p.r_scales[sel],
+                      BLOCK[p.fmt], p.s_t, qw.codes, qw.scales, SPARSE_BLOCK[p.fmt], qw.s_tw, p.fmt)

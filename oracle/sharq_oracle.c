@@ -240,10 +240,12 @@ int oracle_mx_exponent(float a)
 /* The per-value division (not a multiply by a reciprocal) is the reading */
 /* of "quantizes it to FP4"; d doubles as the dequantization step.        */
 
-static void quantize_row(const float *v, int64_t k, int fmt, float s_t,
-                         uint8_t *codes, uint8_t *scales)
+/* blk: the block length; the format's own (16 or 32) everywhere except in
+ * the pair-wise sparse mode below, whose backbone and weight blocks are
+ * twice as long. */
+static void quantize_row_blk(const float *v, int64_t k, int fmt, int blk, float s_t,
+                             uint8_t *codes, uint8_t *scales)
 {
-    int blk = fmt == FMT_NVFP4 ? 16 : 32;
     for (int64_t b = 0; b < k / blk; ++b) {
         const float *vb = v + b * blk;
         float a = 0.0f;
@@ -270,6 +272,12 @@ static void quantize_row(const float *v, int64_t k, int fmt, float s_t,
         for (int i = 0; i < blk; ++i)
             codes[b * blk + i] = d == 0.0f ? 0 : (uint8_t)oracle_e2m1_encode(vb[i] / d);
     }
+}
+
+static void quantize_row(const float *v, int64_t k, int fmt, float s_t,
+                         uint8_t *codes, uint8_t *scales)
+{
+    quantize_row_blk(v, k, fmt, fmt == FMT_NVFP4 ? 16 : 32, s_t, codes, scales);
 }
 
 /* Dequantized value of one code with step d (RN32 product). */
@@ -411,13 +419,18 @@ void oracle_quantize_weight(const uint16_t *w, int64_t n_out, int64_t k, int fmt
 
 /* Dequantized value of element (row, i) in the factored form the GEMM uses:
  * value(code) * value(scale), without the tensor scale. Exact in binary64. */
-static double block_value(int fmt, const uint8_t *codes, const uint8_t *scales,
-                          int64_t k, int64_t row, int64_t i)
+static double block_value_blk(int fmt, int blk, const uint8_t *codes, const uint8_t *scales,
+                              int64_t k, int64_t row, int64_t i)
 {
-    int blk = fmt == FMT_NVFP4 ? 16 : 32;
     int sc = scales[row * (k / blk) + i / blk];
     double sv = fmt == FMT_NVFP4 ? oracle_ue4m3_value(sc) : ldexp(1.0, sc - 127);
     return oracle_e2m1_value(codes[row * k + i]) * sv;
+}
+
+static double block_value(int fmt, const uint8_t *codes, const uint8_t *scales,
+                          int64_t k, int64_t row, int64_t i)
+{
+    return block_value_blk(fmt, fmt == FMT_NVFP4 ? 16 : 32, codes, scales, k, row, i);
 }
 
 /* Dual-path linear: the backbone GEMM on Q(S) and the residual GEMM on    */
@@ -441,6 +454,134 @@ void oracle_linear(const uint8_t *s_codes, const uint8_t *s_scales,
                 double a_s = block_value(fmt, s_codes, s_scales, k, i, q);
                 double a_r = block_value(fmt, r_codes, r_scales, k, i, q);
                 double w = block_value(fmt, w_codes, w_scales, k, j, q);
+                acc += a_s * w + a_r * w;
+                mag += fabs(a_s) * fabs(w) + fabs(a_r) * fabs(w);
+            }
+            if (out)
+                out[i * n_out + j] = ts * acc;
+            if (bound)
+                bound[i * n_out + j] = ts * mag;
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* Pair-wise 4:8 sparse-backbone mode.                                  */
+/*                                                                      */
+/* The abstract's backbone GEMM is "sparse". The block-scaled FP4        */
+/* tensor-core instructions with structured sparsity accept one pattern:  */
+/* in every aligned group of 8 values along K, two of the four adjacent   */
+/* pairs (2j, 2j+1) are kept, and the hardware then applies one scale     */
+/* per 32 logical values along K (NVFP4) or per 64 (MXFP4), on both       */
+/* operands. Reading for this opt-in mode:                                */
+/*   mask: in every aligned group of 8, the two pairs with the largest    */
+/*         pair magnitude max(|x_2j|, |x_2j+1|) are kept, equal pair      */
+/*         magnitudes going to the lower pair; exactly 4 survivors;       */
+/*   Q(S): blocks of 32 values along K (NVFP4; 64 for MXFP4), i.e. the    */
+/*         16 (32) kept values of the block, with the rules above;       */
+/*   R = X_ln - deq(Q(S)) and Q(R) exactly as in the default mode;       */
+/*   W:    one code payload quantized with blocks of 32 (64): the         */
+/*         backbone path reads one scale per 32 (64) values, the residual */
+/*         path the same values once per 16 (32) (its scale view repeats  */
+/*         each one), so deq(W) is the same on both paths.                */
+
+/* Kept positions (ascending, 4 per group of 8) and the 0/1 keep map. */
+void oracle_mask_pairs48(const float *x_ln, int64_t rows, int64_t k, uint8_t *idx, uint8_t *keep)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t g = 0; g < k / 8; ++g) {
+            const float *v = x_ln + r * k + g * 8;
+            float key[4];
+            for (int j = 0; j < 4; ++j)
+                key[j] = fabsf(v[2 * j]) > fabsf(v[2 * j + 1]) ? fabsf(v[2 * j]) : fabsf(v[2 * j + 1]);
+            uint8_t taken[4] = {0, 0, 0, 0};
+            for (int t = 0; t < 2; ++t) { /* pick the t-th largest pair */
+                int best = -1;
+                for (int j = 0; j < 4; ++j)
+                    if (!taken[j] && (best < 0 || key[j] > key[best]))
+                        best = j;
+                taken[best] = 1;
+            }
+            int w = 0;
+            for (int j = 0; j < 4; ++j) {
+                if (taken[j]) {
+                    idx[(r * (k / 8) + g) * 4 + w++] = (uint8_t)(2 * j);
+                    idx[(r * (k / 8) + g) * 4 + w++] = (uint8_t)(2 * j + 1);
+                }
+                if (keep) {
+                    keep[r * k + g * 8 + 2 * j] = taken[j];
+                    keep[r * k + g * 8 + 2 * j + 1] = taken[j];
+                }
+            }
+        }
+}
+
+/* Block quantization with an explicit block length (canonical layout:
+ * scales [rows][k / blk]). */
+void oracle_quantize_blk(const float *v, int64_t rows, int64_t k, int fmt, int blk, float s_t,
+                         uint8_t *codes, uint8_t *scales)
+{
+    for (int64_t r = 0; r < rows; ++r)
+        quantize_row_blk(v + r * k, k, fmt, blk, s_t, codes + r * k, scales + r * (k / blk));
+}
+
+/* The preparation operator in the pair-wise mode, in the abstract's order.
+ * Outputs as oracle_prepare_norm (s_scales: [rows][k / (2 blk)]). */
+void oracle_prepare_sparse(const uint16_t *x, int64_t rows, int64_t k,
+                           const uint16_t *gamma, const uint16_t *beta, float eps, int fmt, int norm,
+                           float *mu, float *rstd, float *x_ln, float *s, float *deq_s, float *r,
+                           uint8_t *idx, uint8_t *keep,
+                           uint8_t *s_codes, uint8_t *s_scales,
+                           uint8_t *r_codes, uint8_t *r_scales, float *s_t_out, const float *s_t_in)
+{
+    int blk = fmt == FMT_NVFP4 ? 16 : 32, sblk = 2 * blk;
+    if (norm)
+        oracle_rms_stats(x, rows, k, eps, mu, rstd);
+    else
+        oracle_ln_stats(x, rows, k, eps, mu, rstd);
+    oracle_ln_apply(x, rows, k, gamma, beta, mu, rstd, x_ln);
+    float s_t = s_t_in ? *s_t_in : oracle_tensor_scale(x_ln, rows * k, fmt);
+    *s_t_out = s_t;
+    oracle_mask_pairs48(x_ln, rows, k, idx, keep);
+    for (int64_t i = 0; i < rows * k; ++i)
+        s[i] = keep[i] ? x_ln[i] : 0.0f;
+    oracle_quantize_blk(s, rows, k, fmt, sblk, s_t, s_codes, s_scales);
+    for (int64_t row = 0; row < rows; ++row)
+        for (int64_t i = 0; i < k; ++i) {
+            int64_t e = row * k + i;
+            float d = block_step(fmt, s_scales[row * (k / sblk) + i / sblk], s_t);
+            deq_s[e] = keep[e] ? deq(s_codes[e], d) : 0.0f;
+            r[e] = x_ln[e] - deq_s[e];
+        }
+    oracle_quantize(r, rows, k, fmt, s_t, r_codes, r_scales);
+}
+
+/* Weight quantization with an explicit block length (the pair-wise mode's
+ * weights: 32 for NVFP4, 64 for MXFP4); s_tW as oracle_quantize_weight. */
+void oracle_quantize_weight_blk(const uint16_t *w, int64_t n_out, int64_t k, int fmt, int blk,
+                                float *w_f32, uint8_t *codes, uint8_t *scales, float *s_tw)
+{
+    for (int64_t i = 0; i < n_out * k; ++i)
+        w_f32[i] = (float)oracle_half_to_double(w[i]);
+    *s_tw = oracle_tensor_scale(w_f32, n_out * k, fmt);
+    oracle_quantize_blk(w_f32, n_out, k, fmt, blk, *s_tw, codes, scales);
+}
+
+/* Dual-path linear with explicit block lengths of the backbone, residual
+ * and weight scales (the formula of oracle_linear). */
+void oracle_linear_blk(const uint8_t *s_codes, const uint8_t *s_scales, int blk_s,
+                       const uint8_t *r_codes, const uint8_t *r_scales, int blk_r, float s_t,
+                       const uint8_t *w_codes, const uint8_t *w_scales, int blk_w, float s_tw,
+                       int64_t rows, int64_t n_out, int64_t k, int fmt,
+                       double *out, double *bound)
+{
+    double ts = (double)s_t * (double)s_tw;
+    for (int64_t i = 0; i < rows; ++i)
+        for (int64_t j = 0; j < n_out; ++j) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t q = 0; q < k; ++q) {
+                double a_s = block_value_blk(fmt, blk_s, s_codes, s_scales, k, i, q);
+                double a_r = block_value_blk(fmt, blk_r, r_codes, r_scales, k, i, q);
+                double w = block_value_blk(fmt, blk_w, w_codes, w_scales, k, j, q);
                 acc += a_s * w + a_r * w;
                 mag += fabs(a_s) * fabs(w) + fabs(a_r) * fabs(w);
             }

@@ -973,7 +973,16 @@ __device__ __forceinline__ void encode_core(const float (&v)[kUnit], int n, cons
     // Mask metadata: each group holds exactly n kept positions, so its
     // field sits at a fixed offset of the unit's bit range.
     uint64_t mbits = 0;
-    if (M <= 8) {
+    if constexpr (M == 4 && NK == 2) {
+        // 2:4: a group's keep nibble has two bits set, so nibble >> 1 is one
+        // of 1..6 and selects the group's field (first | second << 2) from
+        // a byte table; one byte permute does all four groups, then the
+        // four fields are packed into 16 bits.
+        const uint32_t sel = (keep >> 1) & 0x7777u;
+        const uint32_t w = __byte_perm(0x09080400u, 0x000E0D0Cu, sel);  // table: -, 4, 8, 9, 12, 13, 14, -
+        const uint32_t t = w | (w >> 4);                                  // bytes 0 and 2 hold two fields each
+        mbits = __byte_perm(t, 0u, 0x4420u);
+    } else if (M <= 8) {
 #pragma unroll
         for (int g = 0; g < G; ++g)
             mbits |= (uint64_t)lut[(keep >> (g * M)) & ((1u << M) - 1u)] << (g * gbits);
@@ -1313,7 +1322,9 @@ prep_encode_rows_kernel(const EncodeArgs a, const unsigned *amax_word, float *__
                 s_sf[so] = (uint8_t)o.s_scale;
                 r_sf[so] = (uint8_t)o.r_scale;
             }
-            if (byte_aligned)
+            if constexpr (M == 4 && NK == 2)  // 16 bits per unit; rows are k / 8 bytes, so 2-byte aligned
+                *reinterpret_cast<uint16_t *>(meta + row * meta_row + (int64_t)u * 2) = (uint16_t)o.mbits;
+            else if (byte_aligned)
                 store_bytes(meta + row * meta_row + (int64_t)u * (B / 8), o.mbits, B / 8);
             else
                 or_bits(reinterpret_cast<uint32_t *>(meta), (uint64_t)row * meta_row * 8 + (uint64_t)u * B, o.mbits, B);
