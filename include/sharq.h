@@ -116,6 +116,9 @@ typedef struct sharq_wq {
     int32_t segments;    /* fused weights: stacked segments along n_out, 1 (0
                             reads as 1) otherwise */
     int32_t seg_end[SHARQ_SEGMENTS_MAX]; /* exclusive end row of each segment */
+    int32_t sparse;      /* 0: one scale per blk values; 1: the pair-wise
+                            sparse mode's weight (sharq_quantize_weight_sparse):
+                            one scale per 2 blk values */
 } sharq_wq;
 
 /* Prepared activation: outputs of the preparation operator. */
@@ -135,6 +138,8 @@ typedef struct sharq_prep {
     void *meta;          /* device, mask metadata [m_tok][meta_row_bytes] */
     float *tensor_scale; /* device, 1 float: s_t = amax(X_ln)/2688 (NVFP4) or 1 */
     void *scratch;       /* device, per-row statistics and reduction words */
+    int32_t sparse;      /* 0: element-wise n:m mask, backbone codes stored
+                            dense; 1: pair-wise 4:8 mode (sharq_prepare_sparse) */
 } sharq_prep;
 
 /* Bytes of the device buffer sharq_quantize_weight needs. 0 if the shape or
@@ -253,6 +258,57 @@ sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, int64_t k,
                                    sharq_prep *prep_out, void *stream);
 
 /*
+ * Pair-wise 4:8 sparse-backbone mode. SharQ, Abstract: "A sparse FP4 GEMM
+ * processes the backbone". The tensor cores' structured-sparse block-scaled
+ * FP4 MMA (tcgen05.mma.sp, kind::mxf4nvf4 / kind::mxf4) accepts one
+ * pattern: in every aligned group of 8 values along k, two of the four
+ * adjacent pairs (2j, 2j+1) hold the non-zeros; and it applies one scale per
+ * 32 logical values (NVFP4) or 64 (MXFP4) along k to both operands. This
+ * opt-in mode makes the backbone match that pattern, so that the backbone
+ * GEMM runs at the sparse tensor-core rate on half of K:
+ *   mask   in every aligned group of 8, the two pairs with the largest
+ *          max(|x_2j|, |x_2j+1|) of X_ln (equal: the lower pair);
+ *   Q(S)   blocks of 32 (NVFP4) / 64 (MXFP4) values: the 16 / 32 kept
+ *          values of a block quantized exactly like a block of the format;
+ *   R, Q(R) as sharq_prepare (blocks of 16 / 32);
+ *   W      one code payload with blocks of 32 / 64 (sharq_quantize_weight_
+ *          sparse): the backbone path reads one scale per 32 / 64 values,
+ *          the residual path the same scale for each half block, so deq(W)
+ *          is the same on both paths.
+ * The element-wise n:m mask of sharq_prepare is a different mask (it is not
+ * pair-wise in general), so the two modes give different results.
+ *
+ * Layouts in the prep buffer (sparse = 1, n = 4, m = 8):
+ *   s_codes  [m_tok][k/4] bytes: per group of 8, the four kept codes in
+ *            order (first pair's two, then the second's), two per byte.
+ *   s_scales MMA scale view with one scale per 32 (64) values.
+ *   meta     [m_tok][k/16] bytes: per group g of a row, bits 4g .. 4g+3 hold
+ *            first | second << 2 (the kept pairs' indices, ascending); the
+ *            layout the sparse MMA reads.
+ *   r_codes, r_scales as sharq_prepare.
+ * sharq_prep_export returns the canonical forms: idx [m_tok][k/8][4] kept
+ * positions, s_codes [m_tok][k] (+0 off the mask), s_scales
+ * [m_tok][k/32] (NVFP4) or [m_tok][k/64] (MXFP4).
+ */
+size_t sharq_prep_bytes_sparse(int64_t m_tok, int64_t k, int fmt);
+
+/*   norm  0: LayerNorm (ln_w, ln_b as sharq_prepare); 1: RMSNorm (ln_w as
+ *         sharq_prepare_rms, ln_b must be NULL).
+ * Other arguments, preconditions and the statistics as sharq_prepare;
+ * prep_bytes >= sharq_prep_bytes_sparse(m_tok, k, fmt). */
+sharq_status sharq_prepare_sparse(const void *x_dev, int64_t m_tok, int64_t k, const void *ln_w_dev,
+                                  const void *ln_b_dev, float eps, int norm, int fmt, void *prep_dev,
+                                  size_t prep_bytes, sharq_prep *prep_out, void *stream);
+
+/* The weight of the pair-wise mode: as sharq_quantize_weight with blocks of
+ * 32 (NVFP4) or 64 (MXFP4) values; wq_out->sparse = 1. sharq_weight_export
+ * returns the backbone view as [n_out][k/32] ([n_out][k/64]) and the
+ * residual view as [n_out][k/16] ([n_out][k/32]), every scale twice. */
+size_t sharq_weight_bytes_sparse(int64_t n_out, int64_t k, int fmt);
+sharq_status sharq_quantize_weight_sparse(const void *w_dev, int64_t n_out, int64_t k, int fmt, void *wq_dev,
+                                          size_t wq_bytes, sharq_wq *wq_out, void *stream);
+
+/*
  * Dual-path FP4 linear layer. SharQ, Abstract: the backbone goes through a
  * sparse FP4 GEMM, and a dense FP4 GEMM on the residual makes up both for
  * what the mask dropped and for the backbone's quantization error.
@@ -263,6 +319,11 @@ sharq_status sharq_prepare_noalloc(const void *x_dev, int64_t m_tok, int64_t k,
  * Preconditions: prep and wq from this library, prep->fmt == wq->fmt,
  * prep->k == wq->k, out_dev non-NULL (may be NULL only if m_tok == 0) and at
  * least 32-byte aligned (the epilogue writes whole 32-byte sectors).
+ * A pair-wise-mode prep (sharq_prepare_sparse) needs a pair-wise-mode weight
+ * (sharq_quantize_weight_sparse) and the reverse (SHARQ_ERR_INVALID_ARG
+ * otherwise); its backbone then runs through the structured-sparse MMA on
+ * the K-compacted codes. That mode takes no bias and no fused or grouped
+ * weights (SHARQ_ERR_UNSUPPORTED).
  */
 sharq_status sharq_linear(const sharq_prep *prep, const sharq_wq *wq, void *out_dev,
                           void *stream);

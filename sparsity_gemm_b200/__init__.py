@@ -38,7 +38,7 @@ class SharqWQ(C.Structure):
     _fields_ = [("n_out", C.c_int64), ("k", C.c_int64), ("fmt", C.c_int32), ("groups", C.c_int32),
                 ("sf_rows", C.c_int64), ("codes", C.c_void_p), ("scales_backbone", C.c_void_p),
                 ("scales_residual", C.c_void_p), ("tensor_scale", C.c_void_p), ("scratch", C.c_void_p),
-                ("segments", C.c_int32), ("seg_end", C.c_int32 * SEGMENTS_MAX)]
+                ("segments", C.c_int32), ("seg_end", C.c_int32 * SEGMENTS_MAX), ("sparse", C.c_int32)]
 
 
 class SharqPrep(C.Structure):
@@ -46,7 +46,7 @@ class SharqPrep(C.Structure):
                 ("fmt", C.c_int32), ("groups", C.c_int32), ("sf_rows", C.c_int64),
                 ("meta_row_bytes", C.c_int64), ("s_codes", C.c_void_p), ("r_codes", C.c_void_p),
                 ("s_scales", C.c_void_p), ("r_scales", C.c_void_p), ("meta", C.c_void_p),
-                ("tensor_scale", C.c_void_p), ("scratch", C.c_void_p)]
+                ("tensor_scale", C.c_void_p), ("scratch", C.c_void_p), ("sparse", C.c_int32)]
 
 
 _lib = None
@@ -95,6 +95,12 @@ def lib():
         L.sharq_weight_tensor_scales.argtypes = [C.POINTER(SharqWQ), vp, vp]
         L.sharq_prepare_grouped.argtypes = [vp, i64, i64, vp, i64, vp, vp, f32, i32, i32, i32, i32, vp, sz,
                                             C.POINTER(SharqPrep), vp]
+        L.sharq_prep_bytes_sparse.argtypes = [i64, i64, i32]
+        L.sharq_prep_bytes_sparse.restype = sz
+        L.sharq_prepare_sparse.argtypes = [vp, i64, i64, vp, vp, f32, i32, i32, vp, sz, C.POINTER(SharqPrep), vp]
+        L.sharq_weight_bytes_sparse.argtypes = [i64, i64, i32]
+        L.sharq_weight_bytes_sparse.restype = sz
+        L.sharq_quantize_weight_sparse.argtypes = [vp, i64, i64, i32, vp, sz, C.POINTER(SharqWQ), vp]
         L.sharq_status_string.argtypes = [i32]
         L.sharq_status_string.restype = C.c_char_p
         L.sharq_last_launch_count.restype = i32
@@ -102,7 +108,7 @@ def lib():
                      "sharq_weight_export", "sharq_get_last_error", "sharq_quantize_weight_grouped",
                      "sharq_gather_rows", "sharq_linear_grouped", "sharq_prepare_rms",
                      "sharq_quantize_weight_fused", "sharq_linear_bias", "sharq_weight_tensor_scales",
-                     "sharq_prepare_grouped"):
+                     "sharq_prepare_grouped", "sharq_prepare_sparse", "sharq_quantize_weight_sparse"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -297,13 +303,60 @@ def weight_tensor_scales(qw: QuantizedWeight, stream=None) -> np.ndarray:
     return out
 
 
+def prepare_sparse(x: torch.Tensor, ln_w=None, ln_b=None, eps: float = 1e-5, fmt: int = NVFP4,
+                   out: Prepared | None = None, stream=None, norm: str = "layer") -> Prepared:
+    """The preparation operator in the pair-wise 4:8 mode (the pattern of the
+    structured-sparse FP4 tensor-core MMA): x [m_tok, k] (fp16, CUDA); the
+    backbone is stored K-compacted and feeds tcgen05.mma.sp in linear(), with
+    a weight from quantize_weight_sparse."""
+    _require(norm in ("layer", "rms") and (norm == "layer" or ln_b is None),
+             'norm must be "layer" or "rms" (RMSNorm takes no ln_b)')
+    _fp16_matrix(x, "x")
+    for t, name in ((ln_w, "ln_w"), (ln_b, "ln_b")):
+        if t is not None:
+            _fp16_matrix(t.view(-1) if t.is_contiguous() else t, name, 1)
+            _require(t.numel() == x.shape[1], f"{name} must have {x.shape[1]} elements")
+    m_tok, k = x.shape
+    nbytes = int(lib().sharq_prep_bytes_sparse(m_tok, k, fmt))
+    if nbytes == 0:
+        raise SharqError(ERR_INVALID_ARG, f"sparse prep shape {tuple(x.shape)} fmt {fmt}")
+    if out is None or out.buf.numel() < nbytes:
+        buf = _device_buffer(nbytes, x.device)
+    else:
+        buf = out.buf
+        _cuda_here(buf, "out.buf")
+    desc = SharqPrep()
+    _check(lib().sharq_prepare_sparse(_ptr(x) if m_tok > 0 else None, m_tok, k, _ptr(ln_w), _ptr(ln_b), float(eps),
+                                      1 if norm == "rms" else 0, fmt, _ptr(buf), buf.numel(), C.byref(desc),
+                                      _stream(stream)), "sharq_prepare_sparse")
+    return Prepared(buf, desc)
+
+
+def quantize_weight_sparse(w: torch.Tensor, fmt: int = NVFP4, stream=None) -> QuantizedWeight:
+    """Offline FP4 quantization of W [n_out, k] (fp16, CUDA) for the pair-wise
+    4:8 mode: one scale per 32 (NVFP4) or 64 (MXFP4) values, which the
+    backbone path reads as is and the residual path once per half block."""
+    _fp16_matrix(w, "w")
+    n_out, k = w.shape
+    nbytes = int(lib().sharq_weight_bytes_sparse(n_out, k, fmt))
+    if nbytes == 0:
+        raise SharqError(ERR_INVALID_ARG, f"sparse weight shape {tuple(w.shape)} fmt {fmt}")
+    buf = _device_buffer(nbytes, w.device)
+    desc = SharqWQ()
+    _check(lib().sharq_quantize_weight_sparse(_ptr(w), n_out, k, fmt, _ptr(buf), nbytes, C.byref(desc),
+                                              _stream(stream)), "sharq_quantize_weight_sparse")
+    return QuantizedWeight(buf, desc)
+
+
 def prep_export(prep: Prepared, stream=None) -> dict:
-    """Canonical host copies (numpy) of a prepared activation."""
+    """Canonical host copies (numpy) of a prepared activation (pair-wise mode:
+    backbone codes decompressed, one backbone scale per 2 blocks)."""
     d = prep.desc
     m_tok, k, blk = d.m_tok, d.k, BLOCK[d.fmt]
+    sblk = 2 * blk if d.sparse else blk
     out = dict(
         idx=np.zeros((m_tok, k // d.m, d.n), np.uint8),
-        s_codes=np.zeros((m_tok, k), np.uint8), s_scales=np.zeros((m_tok, k // blk), np.uint8),
+        s_codes=np.zeros((m_tok, k), np.uint8), s_scales=np.zeros((m_tok, k // sblk), np.uint8),
         r_codes=np.zeros((m_tok, k), np.uint8), r_scales=np.zeros((m_tok, k // blk), np.uint8),
         mu=np.zeros(m_tok, np.float32), rstd=np.zeros(m_tok, np.float32), s_t=np.zeros(1, np.float32))
     p = lambda a: a.ctypes.data_as(C.c_void_p)
@@ -317,7 +370,8 @@ def prep_export(prep: Prepared, stream=None) -> dict:
 def weight_export(qw: QuantizedWeight, stream=None) -> dict:
     d = qw.desc
     blk = BLOCK[d.fmt]
-    out = dict(codes=np.zeros((d.n_out, d.k), np.uint8), scales=np.zeros((d.n_out, d.k // blk), np.uint8),
+    sblk = 2 * blk if d.sparse else blk
+    out = dict(codes=np.zeros((d.n_out, d.k), np.uint8), scales=np.zeros((d.n_out, d.k // sblk), np.uint8),
                scales_residual=np.zeros((d.n_out, d.k // blk), np.uint8), s_tw=np.zeros(1, np.float32))
     p = lambda a: a.ctypes.data_as(C.c_void_p)
     _check(lib().sharq_weight_export(C.byref(d), p(out["codes"]), p(out["scales"]), p(out["scales_residual"]),

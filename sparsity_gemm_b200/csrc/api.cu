@@ -77,14 +77,37 @@ void fill_prep(sharq_prep *P, void *buf, int64_t m_tok, int64_t k, int n, int m,
     P->tensor_scale = reinterpret_cast<float *>(b + L.words) + 1;
 }
 
-void fill_wq(sharq_wq *W, void *buf, int64_t n_out, int64_t k, int fmt) {
-    sq::WLayout L = sq::w_layout(n_out, k, fmt);
+void fill_prep_sparse(sharq_prep *P, void *buf, int64_t m_tok, int64_t k, int fmt) {
+    sq::PrepLayout L = sq::prep_layout_sparse(m_tok, k, fmt);
+    uint8_t *b = static_cast<uint8_t *>(buf);
+    memset(P, 0, sizeof(*P));
+    P->m_tok = m_tok;
+    P->groups = 1;
+    P->k = k;
+    P->n = 4;
+    P->m = 8;
+    P->fmt = fmt;
+    P->sparse = 1;
+    P->sf_rows = L.sf_rows;
+    P->meta_row_bytes = L.meta_row;
+    P->s_codes = b + L.s_codes;
+    P->r_codes = b + L.r_codes;
+    P->s_scales = b + L.s_scales;
+    P->r_scales = b + L.r_scales;
+    P->meta = b + L.meta;
+    P->scratch = b + L.stats;
+    P->tensor_scale = reinterpret_cast<float *>(b + L.words) + 1;
+}
+
+void fill_wq(sharq_wq *W, void *buf, int64_t n_out, int64_t k, int fmt, bool sparse = false) {
+    sq::WLayout L = sq::w_layout(n_out, k, fmt, sparse);
     uint8_t *b = static_cast<uint8_t *>(buf);
     memset(W, 0, sizeof(*W));
     W->n_out = n_out;
     W->groups = 1;
     W->k = k;
     W->fmt = fmt;
+    W->sparse = sparse ? 1 : 0;
     W->sf_rows = L.sf_rows;
     W->codes = b + L.codes;
     W->scales_backbone = b + L.scales;
@@ -120,6 +143,70 @@ void unpack_codes(const std::vector<uint8_t> &packed, int64_t count, uint8_t *ds
 void unpack_scales(const std::vector<uint8_t> &sf, int64_t rows, int64_t nblk, uint8_t *dst) {
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t j = 0; j < nblk; ++j) dst[r * nblk + j] = sf[sq::sf_offset(r, j, nblk)];
+}
+
+// Canonical export of a pair-wise-mode prep: kept positions [m_tok][k/8][4]
+// (the two kept pairs' elements, ascending), backbone codes decompressed to
+// [m_tok][k] (+0 off the mask), backbone scales [m_tok][k / (2 blk)].
+sharq_status export_sparse(const sharq_prep *prep, uint8_t *idx_host, uint8_t *s_codes_host, uint8_t *s_scales_host,
+                           uint8_t *r_codes_host, uint8_t *r_scales_host, float *mu_host, float *rstd_host,
+                           float *s_t_host) {
+    const int64_t m_tok = prep->m_tok, k = prep->k, blk = sq::blk_of(prep->fmt);
+    const int64_t nblk_r = k / blk, nblk_s = k / (2 * blk);
+    std::vector<uint8_t> buf, meta;
+    auto fetch = [&](std::vector<uint8_t> &dst, const void *src, int64_t bytes) -> bool {
+        dst.resize((size_t)(bytes > 0 ? bytes : 1));
+        return bytes == 0 || cudaMemcpy(dst.data(), src, (size_t)bytes, cudaMemcpyDeviceToHost) == cudaSuccess;
+    };
+    if ((idx_host || s_codes_host) && !fetch(meta, prep->meta, m_tok * (k / 16))) return SHARQ_ERR_CUDA;
+    auto pairs = [&](int64_t r, int64_t g, int &p0, int &p1) {
+        const uint32_t f = (meta[(size_t)(r * (k / 16) + g / 2)] >> (4 * (g & 1))) & 0xFu;
+        p0 = (int)(f & 3u);
+        p1 = (int)(f >> 2);
+    };
+    if (idx_host)
+        for (int64_t r = 0; r < m_tok; ++r)
+            for (int64_t g = 0; g < k / 8; ++g) {
+                int p0, p1;
+                pairs(r, g, p0, p1);
+                uint8_t *d = idx_host + (r * (k / 8) + g) * 4;
+                d[0] = (uint8_t)(2 * p0), d[1] = (uint8_t)(2 * p0 + 1), d[2] = (uint8_t)(2 * p1), d[3] = (uint8_t)(2 * p1 + 1);
+            }
+    if (s_codes_host) {
+        if (!fetch(buf, prep->s_codes, m_tok * (k / 4))) return SHARQ_ERR_CUDA;
+        for (int64_t r = 0; r < m_tok; ++r)
+            for (int64_t g = 0; g < k / 8; ++g) {
+                int p0, p1;
+                pairs(r, g, p0, p1);
+                uint8_t *d = s_codes_host + r * k + g * 8;
+                memset(d, 0, 8);
+                const uint8_t b0 = buf[(size_t)(r * (k / 4) + g * 2)], b1 = buf[(size_t)(r * (k / 4) + g * 2 + 1)];
+                d[2 * p0] = b0 & 0xF, d[2 * p0 + 1] = b0 >> 4, d[2 * p1] = b1 & 0xF, d[2 * p1 + 1] = b1 >> 4;
+            }
+    }
+    if (r_codes_host) {
+        if (!fetch(buf, prep->r_codes, m_tok * (k / 2))) return SHARQ_ERR_CUDA;
+        unpack_codes(buf, m_tok * k, r_codes_host);
+    }
+    if (s_scales_host) {
+        if (!fetch(buf, prep->s_scales, prep->sf_rows * nblk_s)) return SHARQ_ERR_CUDA;
+        unpack_scales(buf, m_tok, nblk_s, s_scales_host);
+    }
+    if (r_scales_host) {
+        if (!fetch(buf, prep->r_scales, prep->sf_rows * nblk_r)) return SHARQ_ERR_CUDA;
+        unpack_scales(buf, m_tok, nblk_r, r_scales_host);
+    }
+    if (mu_host || rstd_host) {
+        if (!fetch(buf, prep->scratch, m_tok * 8)) return SHARQ_ERR_CUDA;
+        const float *st = reinterpret_cast<const float *>(buf.data());
+        for (int64_t r = 0; r < m_tok; ++r) {
+            if (mu_host) mu_host[r] = st[2 * r];
+            if (rstd_host) rstd_host[r] = st[2 * r + 1];
+        }
+    }
+    if (s_t_host && cudaMemcpy(s_t_host, prep->tensor_scale, sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SHARQ_ERR_CUDA;
+    return SHARQ_OK;
 }
 
 }  // namespace
@@ -203,6 +290,53 @@ sharq_status sharq_prepare_rms(const void *x_dev, int64_t m_tok, int64_t k, cons
     return prepare_norm(x_dev, m_tok, k, w_dev, nullptr, eps, n, m, fmt, prep_dev, prep_bytes, prep_out, stream, 1);
 }
 
+size_t sharq_prep_bytes_sparse(int64_t m_tok, int64_t k, int fmt) {
+    if (m_tok < 0 || m_tok > (1ll << 30) || !k_ok(k) || !fmt_ok(fmt)) return 0;
+    return (size_t)sq::prep_layout_sparse(m_tok, k, fmt).total;
+}
+
+sharq_status sharq_prepare_sparse(const void *x_dev, int64_t m_tok, int64_t k, const void *ln_w_dev,
+                                  const void *ln_b_dev, float eps, int norm, int fmt, void *prep_dev,
+                                  size_t prep_bytes, sharq_prep *prep_out, void *stream) {
+    g_last_launches = 0;
+    const size_t need = sharq_prep_bytes_sparse(m_tok, k, fmt);
+    if (!need || !prep_dev || !prep_out || prep_bytes < need) return SHARQ_ERR_INVALID_ARG;
+    if ((norm != 0 && norm != 1) || (norm == 1 && ln_b_dev)) return SHARQ_ERR_INVALID_ARG;
+    if (m_tok > 0 && !x_dev) return SHARQ_ERR_INVALID_ARG;
+    if (!(eps > 0.0f) || eps != eps || eps > 3.0e38f) return SHARQ_ERR_INVALID_ARG;
+    if ((x_dev && !aligned(x_dev, 16)) || !aligned(prep_dev, sq::kAlign) || (ln_w_dev && !aligned(ln_w_dev, 16)) ||
+        (ln_b_dev && !aligned(ln_b_dev, 16)))
+        return SHARQ_ERR_INVALID_ARG;
+    sq::LaunchCtx ctx;
+    sharq_status st = make_ctx(stream, ctx);
+    if (st != SHARQ_OK) return st;
+    fill_prep_sparse(prep_out, prep_dev, m_tok, k, fmt);
+    st = sq::launch_prepare_sparse(ctx, *prep_out, x_dev, ln_w_dev, ln_b_dev, eps, norm);
+    if (st == SHARQ_OK && cudaGetLastError() != cudaSuccess) st = SHARQ_ERR_CUDA;
+    g_last_launches = ctx.launches;
+    return st;
+}
+
+size_t sharq_weight_bytes_sparse(int64_t n_out, int64_t k, int fmt) {
+    if (n_out < 1 || n_out % SHARQ_N_ALIGN != 0 || n_out > (1ll << 30) || !k_ok(k) || !fmt_ok(fmt)) return 0;
+    return (size_t)sq::w_layout(n_out, k, fmt, true).total;
+}
+
+sharq_status sharq_quantize_weight_sparse(const void *w_dev, int64_t n_out, int64_t k, int fmt, void *wq_dev,
+                                          size_t wq_bytes, sharq_wq *wq_out, void *stream) {
+    g_last_launches = 0;
+    const size_t need = sharq_weight_bytes_sparse(n_out, k, fmt);
+    if (!need || !w_dev || !wq_dev || !wq_out || wq_bytes < need) return SHARQ_ERR_INVALID_ARG;
+    if (!aligned(w_dev, 16) || !aligned(wq_dev, sq::kAlign)) return SHARQ_ERR_INVALID_ARG;
+    sq::LaunchCtx ctx;
+    sharq_status st = make_ctx(stream, ctx);
+    if (st != SHARQ_OK) return st;
+    fill_wq(wq_out, wq_dev, n_out, k, fmt, true);
+    st = sq::launch_quantize_weight(ctx, *wq_out, w_dev, 1, (int64_t)need);
+    g_last_launches = ctx.launches;
+    return st;
+}
+
 sharq_status sharq_linear(const sharq_prep *prep, const sharq_wq *wq, void *out_dev, void *stream) {
     return sharq_linear_bias(prep, wq, nullptr, out_dev, stream);
 }
@@ -213,6 +347,10 @@ sharq_status sharq_linear_bias(const sharq_prep *prep, const sharq_wq *wq, const
     if (!prep || !wq) return SHARQ_ERR_INVALID_ARG;
     if (!segments_ok(wq) || (bias_dev && !aligned(bias_dev, 16))) return SHARQ_ERR_INVALID_ARG;
     if (!fmt_ok(prep->fmt) || prep->fmt != wq->fmt || prep->k != wq->k || !k_ok(prep->k)) return SHARQ_ERR_INVALID_ARG;
+    // the pair-wise mode's activation and weight go together (the weight's
+    // scale blocks are the backbone's)
+    if ((prep->sparse != 0) != (wq->sparse != 0)) return SHARQ_ERR_INVALID_ARG;
+    if (prep->sparse && (bias_dev || wq->segments > 1 || wq->groups > 1)) return SHARQ_ERR_UNSUPPORTED;
     if (wq->n_out < 1 || wq->n_out % SHARQ_N_ALIGN != 0 || prep->m_tok < 0) return SHARQ_ERR_INVALID_ARG;
     if (wq->groups > 1) return SHARQ_ERR_INVALID_ARG;  // stacked weights: sharq_linear_grouped
     if (prep->sf_rows < prep->m_tok || wq->sf_rows < wq->n_out || wq->sf_rows % sq::kWRowPad != 0 ||
@@ -315,6 +453,7 @@ sharq_status sharq_gather_rows(const sharq_prep *src, const int32_t *row_idx_dev
                                void *stream) {
     g_last_launches = 0;
     if (!src || !offsets_dev || !dst_dev || !dst_out) return SHARQ_ERR_INVALID_ARG;
+    if (src->sparse) return SHARQ_ERR_UNSUPPORTED;  // grouped launches take the default mode
     if (!fmt_ok(src->fmt) || !nm_ok(src->n, src->m) || !k_ok(src->k) || src->m_tok < 0 || src->m_tok > (1ll << 30))
         return SHARQ_ERR_INVALID_ARG;
     if (src->meta_row_bytes != sq::meta_row_bytes(src->k, src->n, src->m) || src->sf_rows < src->m_tok ||
@@ -372,6 +511,7 @@ sharq_status sharq_linear_grouped(const sharq_prep *prep, const int32_t *offsets
     g_last_launches = 0;
     if (!prep || !wq || !offsets_dev || !aligned(offsets_dev, 4)) return SHARQ_ERR_INVALID_ARG;
     if (!fmt_ok(prep->fmt) || prep->fmt != wq->fmt || prep->k != wq->k || !k_ok(prep->k)) return SHARQ_ERR_INVALID_ARG;
+    if (prep->sparse || wq->sparse) return SHARQ_ERR_UNSUPPORTED;  // grouped launches take the default mode
     if (n_groups < 1 || n_groups > sq::kGroupsMax || prep->groups != n_groups || wq->groups != n_groups ||
         wq->segments > 1)
         return SHARQ_ERR_INVALID_ARG;
@@ -399,6 +539,9 @@ sharq_status sharq_prep_export(const sharq_prep *prep, uint8_t *idx_host, uint8_
     if (!prep || !fmt_ok(prep->fmt) || !nm_ok(prep->n, prep->m) || prep->m_tok < 0) return SHARQ_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return SHARQ_ERR_CUDA;
+    if (prep->sparse)
+        return export_sparse(prep, idx_host, s_codes_host, s_scales_host, r_codes_host, r_scales_host, mu_host,
+                             rstd_host, s_t_host);
     const int64_t m_tok = prep->m_tok, k = prep->k, nblk = k / sq::blk_of(prep->fmt);
     const int64_t codes = m_tok * (k / 2), sf = prep->sf_rows * nblk;
     std::vector<uint8_t> buf;
@@ -454,7 +597,9 @@ sharq_status sharq_weight_export(const sharq_wq *wq, uint8_t *codes_host, uint8_
                                  uint8_t *scales_residual_host, float *s_tw_host, void *stream) {
     if (!wq || !fmt_ok(wq->fmt)) return SHARQ_ERR_INVALID_ARG;
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SHARQ_ERR_CUDA;
-    const int64_t nblk = wq->k / sq::blk_of(wq->fmt);
+    // the pair-wise mode's weight: one scale per 2 blk values in the
+    // backbone view; the residual view repeats each of them
+    const int64_t nblk = wq->k / (sq::blk_of(wq->fmt) * (wq->sparse ? 2 : 1));
     std::vector<uint8_t> buf;
     if (codes_host) {
         buf.resize((size_t)(wq->n_out * (wq->k / 2)));
@@ -467,7 +612,14 @@ sharq_status sharq_weight_export(const sharq_wq *wq, uint8_t *codes_host, uint8_
         if (!dsts[v]) continue;
         buf.resize((size_t)(wq->sf_rows * nblk));
         if (cudaMemcpy(buf.data(), views[v], buf.size(), cudaMemcpyDeviceToHost) != cudaSuccess) return SHARQ_ERR_CUDA;
-        unpack_scales(buf, wq->n_out, nblk, dsts[v]);
+        if (wq->sparse && v == 1) {  // [n_out][k / blk]: every scale twice
+            std::vector<uint8_t> once((size_t)(wq->n_out * nblk));
+            unpack_scales(buf, wq->n_out, nblk, once.data());
+            for (int64_t r = 0; r < wq->n_out; ++r)
+                for (int64_t j = 0; j < 2 * nblk; ++j) dsts[v][r * 2 * nblk + j] = once[(size_t)(r * nblk + j / 2)];
+        } else {
+            unpack_scales(buf, wq->n_out, nblk, dsts[v]);
+        }
     }
     if (s_tw_host && cudaMemcpy(s_tw_host, wq->tensor_scale, sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess)
         return SHARQ_ERR_CUDA;

@@ -50,7 +50,7 @@ namespace sq {
 constexpr int kBM = 128, kBKBytes = SQ_GEMM_BKB;
 constexpr int kABytes = kBM * kBKBytes;
 constexpr int kSfaMax = 512 * (kBKBytes / 32);  // scale bytes of 128 rows per stage, NVFP4 (MXFP4 uses half)
-constexpr int kOffAS = 0, kOffAR = kABytes, kOffB = 2 * kABytes;
+constexpr int kOffAS = 0;
 // Scale buffers in tensor memory after the accumulators: per buffer, the
 // backbone A scales, the residual A scales and the W scales of one stage
 // (NVFP4: kBKBytes / 32 atoms per 128 rows; MXFP4 uses half).
@@ -75,19 +75,35 @@ static_assert(kTableBytes % 4 == 0, "table alignment");
 // more than the hidden drain saved on the short-K expert GEMMs (Qwen3 MoE
 // shapes, K = 2048 and 768: 22% slower at 128). SQ_GROUPED_BN=128 builds
 // the other width for grouped launches.
-template <int BN>
+// SP: the pair-wise 4:8 backbone (sharq_prepare_sparse): per stage the
+// backbone tile holds the kept half of K (64-byte rows), its scales and the
+// W view the sparse MMA reads hold one scale per 32 values (half the
+// atoms), and the mask metadata rides with the scales (16 bytes per row).
+template <int BN, bool SP = false>
 struct TileCfg {
     static constexpr int kBN = BN;
     static constexpr int kBlk = BN / 128;            // 128-row W blocks (scale atoms) per tile
     static constexpr int kNacc = BN == 256 ? 1 : 2;  // accumulators in tensor memory
+    static constexpr int kASBytes = SP ? kABytes / 2 : kABytes;
+    static constexpr int kOffAR = kASBytes, kOffB = kASBytes + kABytes;
     static constexpr int kBBytes = BN * kBKBytes;
-    static constexpr int kSfbMax = kBlk * kSfaMax;
-    static constexpr int kOffSFAS = kOffB + kBBytes, kOffSFAR = kOffSFAS + kSfaMax, kOffSFB = kOffSFAR + kSfaMax;
-    static constexpr int kStageBytes = kOffSFB + kSfbMax;  // a multiple of 1024
+    static constexpr int kSfaSMax = SP ? kSfaMax / 2 : kSfaMax;  // backbone scale bytes per stage
+    static constexpr int kSfbMax = kBlk * kSfaSMax;              // W scale view of the backbone path
+    static constexpr int kMetaBytes = SP ? kBM * 16 : 0;
+    static constexpr int kOffSFAS = kOffB + kBBytes, kOffSFAR = kOffSFAS + kSfaSMax, kOffSFB = kOffSFAR + kSfaMax;
+    static constexpr int kOffMeta = kOffSFB + kSfbMax;
+    static constexpr int kStageBytes = kOffMeta + kMetaBytes;  // a multiple of 1024
     static constexpr int kStages = (232448 - 2048) / kStageBytes;
     static constexpr int kBarOff = kStages * kStageBytes;
     static constexpr uint32_t kColSf0 = kNacc * BN;
-    static constexpr uint32_t kSfBufCols = (8 + 4 * kBlk) * kNvAtoms;  // A_S, A_R, then kBlk W blocks
+    // Columns of one scale buffer. Dense: A_S, A_R, then kBlk W blocks.
+    // SP (NVFP4 counts; MXFP4 uses half): backbone scales (2 atoms), the W
+    // backbone view (2 atoms x kBlk), residual scales (4 atoms), the W
+    // residual view (4 atoms x kBlk, written from the backbone view's values),
+    // then the metadata (4 columns per MMA, two used).
+    static constexpr uint32_t kSpS = 0, kSpWb = 8, kSpR = kSpWb + 8 * kBlk, kSpWr = kSpR + 16,
+                              kSpMeta = kSpWr + 16 * kBlk;
+    static constexpr uint32_t kSfBufCols = SP ? kSpMeta + 8 : (8 + 4 * kBlk) * kNvAtoms;
     static constexpr int kSfBufs = (int)((kTmemCols - kColSf0) / kSfBufCols) < 4 ? (int)((kTmemCols - kColSf0) / kSfBufCols) : 4;
     // mbarriers: full[s], empty[s], sf_loaded[s], acc_full[a], acc_empty[a],
     // drain, sf_full[b], sf_empty[b]; the tensor-memory slot follows.
@@ -99,6 +115,7 @@ struct TileCfg {
     // padded by 16 bytes so that a warp's 32 rows hit different banks.
     static constexpr uint32_t kPartStride = BN * 4 + 16;
     static_assert(BN == 128 || BN == 256, "tile width");
+    static_assert(!SP || (BN == 256 && kBKBytes == 128), "the sparse mode uses the 256-column, 128-byte K tile");
     static_assert(kStageBytes % 1024 == 0, "stage buffers must stay 1024-byte aligned");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kBarBytes + 4 <= kBarArea, "barrier area");
@@ -178,6 +195,12 @@ __device__ __forceinline__ uint64_t desc_operand(uint32_t addr) {
 }
 
 
+// The sparse mode's compacted backbone tile: rows of kBKBytes / 2 bytes,
+// 64-byte swizzle; 8-row groups 8 * kBKBytes / 2 bytes apart.
+__device__ __forceinline__ uint64_t desc_operand_half(uint32_t addr) {
+    return smem_desc(addr, 16, 8 * (kBKBytes / 2), 4u);
+}
+
 // Wait bounded only by time (used to drain in-flight copies on exit).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     uint64_t t0 = globaltimer_ns();
@@ -191,11 +214,16 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 // tensor scale, and output rows are remapped to grouped-row order.
 // EXT (dense only): fused-weight segments and/or a bias in the epilogue; the
 // plain instantiation keeps the epilogue without them.
-template <int FMT, bool GROUPED, bool EXT, int BN>
+// SP (dense only): the pair-wise 4:8 backbone through tcgen05.mma.sp on a
+// K-compacted tile (tm_as rows of k/4 bytes), its metadata tile tm_meta
+// ([m_tok][k/16] bytes) moved to tensor memory by the scale writers.
+template <int FMT, bool GROUPED, bool EXT, int BN, bool SP = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constant__ CUtensorMap tm_ar,
-                 const __grid_constant__ CUtensorMap tm_b, const GemmParams p) {
-    using C = TileCfg<BN>;
+                 const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_meta,
+                 const GemmParams p) {
+    using C = TileCfg<BN, SP>;
+    static_assert(!SP || !GROUPED, "the sparse mode runs dense launches");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
@@ -226,6 +254,9 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     // 512-byte scale atoms (128 rows x 4 scales) per 128 rows per K tile
     constexpr int kAtomsPerTile = FMT == kFmtNV ? kBKBytes / 32 : kBKBytes / 64;
     constexpr uint32_t kSfBytes = 512u * kAtomsPerTile;
+    // the backbone's (and the W backbone view's) atoms in the sparse mode
+    constexpr int kAtomsS = SP ? kAtomsPerTile / 2 : kAtomsPerTile;
+    constexpr uint32_t kSfBytesS = 512u * kAtomsS;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) {
@@ -246,6 +277,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         prefetch_tmap(&tm_as);
         prefetch_tmap(&tm_ar);
         prefetch_tmap(&tm_b);
+        if (SP) prefetch_tmap(&tm_meta);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), kTmemCols);
@@ -274,6 +306,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     }
     const int kt_n = kt_end - kt_begin;
     const int64_t atoms_per_row_blk = (int64_t)(p.k / (FMT == kFmtNV ? 16 : 32)) / 4;
+    const int64_t atoms_per_row_blk_s = SP ? atoms_per_row_blk / 2 : atoms_per_row_blk;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -298,20 +331,22 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                     // writers move them to tensor memory while the operand
                     // tiles are still in flight.
                     const int64_t a_off = ((int64_t)mb * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
+                    const int64_t a_off_s = ((int64_t)mb * atoms_per_row_blk_s + (int64_t)kt * kAtomsS) * 512;
                     const int64_t b0 =
-                        ((int64_t)(C::kBlk * nb) * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
-                    mbar_arrive_expect_tx(lb, (2 + C::kBlk) * kSfBytes);
-                    bulk_load(st + C::kOffSFAS, p.sfa_s + a_off, kSfBytes, lb);
+                        ((int64_t)(C::kBlk * nb) * atoms_per_row_blk_s + (int64_t)kt * kAtomsS) * 512;
+                    mbar_arrive_expect_tx(lb, (1 + C::kBlk) * kSfBytesS + kSfBytes + C::kMetaBytes);
+                    bulk_load(st + C::kOffSFAS, p.sfa_s + a_off_s, kSfBytesS, lb);
                     bulk_load(st + C::kOffSFAR, p.sfa_r + a_off, kSfBytes, lb);
 #pragma unroll
                     for (int bk = 0; bk < C::kBlk; ++bk)  // the tile's 128-row W blocks
-                        bulk_load(st + C::kOffSFB + bk * kSfBytes, sfb + b0 + bk * atoms_per_row_blk * 512, kSfBytes,
-                                  lb);
-                    mbar_arrive_expect_tx(fb, 2 * kABytes + C::kBBytes);
-                    tma_load_2d(st + kOffAS, &tm_as, kt * kBKBytes, mb * kBM, fb);
-                    tma_load_2d(st + kOffAR, &tm_ar, kt * kBKBytes, mb * kBM, fb);
-                    if (GROUPED) tma_load_3d(st + kOffB, &tm_b, kt * kBKBytes, nb * C::kBN, grp, fb);
-                    else tma_load_2d(st + kOffB, &tm_b, kt * kBKBytes, nb * C::kBN, fb);
+                        bulk_load(st + C::kOffSFB + bk * kSfBytesS, sfb + b0 + bk * atoms_per_row_blk_s * 512,
+                                  kSfBytesS, lb);
+                    if (SP) tma_load_2d(st + C::kOffMeta, &tm_meta, kt * 16, mb * kBM, lb);
+                    mbar_arrive_expect_tx(fb, C::kASBytes + kABytes + C::kBBytes);
+                    tma_load_2d(st + kOffAS, &tm_as, kt * (SP ? kBKBytes / 2 : kBKBytes), mb * kBM, fb);
+                    tma_load_2d(st + C::kOffAR, &tm_ar, kt * kBKBytes, mb * kBM, fb);
+                    if (GROUPED) tma_load_3d(st + C::kOffB, &tm_b, kt * kBKBytes, nb * C::kBN, grp, fb);
+                    else tma_load_2d(st + C::kOffB, &tm_b, kt * kBKBytes, nb * C::kBN, fb);
                     last[s] = (int32_t)it;
                 }
             }
@@ -349,11 +384,43 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                     tc_fence_after();
                     const uint32_t st = sbase + (uint32_t)(s * C::kStageBytes);
                     const uint32_t sf = tmem + C::kColSf0 + C::kSfBufCols * (uint32_t)sb;
-                    const uint64_t da_s = desc_operand(st + kOffAS);
-                    const uint64_t da_r = desc_operand(st + kOffAR);
-                    const uint64_t db = desc_operand(st + kOffB);
+                    const uint64_t da_s = SP ? desc_operand_half(st + kOffAS) : desc_operand(st + kOffAS);
+                    const uint64_t da_r = desc_operand(st + C::kOffAR);
+                    const uint64_t db = desc_operand(st + C::kOffB);
+                    if constexpr (SP) {
+                        // backbone: two sparse MMAs of 128 logical K (32 bytes of
+                        // the compacted tile, 64 of the W tile) each
 #pragma unroll
-                    for (int j = 0; j < kMmaPerStage; ++j) {  // MMAs of K = 64 (32 bytes) per K tile
+                        for (int j = 0; j < 2; ++j) {
+                            const uint32_t acc = (kt != kt_begin || j != 0) ? 1u : 0u;
+                            const uint32_t e = sf + C::kSpMeta + 4 * j;
+                            if (FMT == kFmtNV) {
+                                tc_mma_sp_nvf4(dacc, da_s + 2 * j, db + 4 * j, idesc_of<FMT, BN>(0) | (1u << 2),
+                                               sf + C::kSpS + 4 * j, sf + C::kSpWb + 4 * C::kBlk * j, e, acc);
+                            } else {
+                                const uint32_t sf_id = (uint32_t)j * 2u;  // 2 scales per row per MMA
+                                tc_mma_sp_mxf4(dacc, da_s + 2 * j, db + 4 * j, idesc_of<FMT, BN>(sf_id) | (1u << 2),
+                                               (sf + C::kSpS) | (sf_id << 30), (sf + C::kSpWb) | (sf_id << 30), e,
+                                               acc);
+                            }
+                        }
+                        // residual: the dense MMAs of K = 64 on the W residual view
+#pragma unroll
+                        for (int j = 0; j < kMmaPerStage; ++j) {
+                            if (FMT == kFmtNV) {
+                                tc_mma_nvf4(dacc, da_r + 2 * j, db + 2 * j, idesc_of<FMT, BN>(0), sf + C::kSpR + 4 * j,
+                                            sf + C::kSpWr + 4 * C::kBlk * j, 1u);
+                            } else {
+                                const uint32_t sf_id = (uint32_t)(j & 1) * 2u;
+                                const uint32_t a_col = 4 * (j >> 1), b_col = 4 * C::kBlk * (j >> 1);
+                                tc_mma_mxf4(dacc, da_r + 2 * j, db + 2 * j, idesc_of<FMT, BN>(sf_id),
+                                            (sf + C::kSpR + a_col) | (sf_id << 30),
+                                            (sf + C::kSpWr + b_col) | (sf_id << 30), 1u);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < (SP ? 0 : kMmaPerStage); ++j) {  // MMAs of K = 64 (32 bytes) per K tile
                         const uint32_t acc = (kt != kt_begin || j != 0) ? 1u : 0u;
                         // W scales: 4 columns per 128-row block per atom, the
                         // tile's blocks side by side
@@ -407,8 +474,36 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             tc_fence_after();
             const uint32_t st = sbase + (uint32_t)(s * C::kStageBytes) + (uint32_t)lane * 16u;
             const uint32_t sf = tmem + lane_base + C::kColSf0 + C::kSfBufCols * (uint32_t)b;
+            if constexpr (SP) {
 #pragma unroll
-            for (int a = 0; a < kAtomsPerTile; ++a) {
+                for (int a = 0; a < kAtomsS; ++a) {
+                    tmem_st4(sf + C::kSpS + 4 * a, lds128(st + C::kOffSFAS + 512 * a));
+#pragma unroll
+                    for (int bk = 0; bk < C::kBlk; ++bk) {
+                        const uint4 w = lds128(st + C::kOffSFB + bk * kSfBytesS + 512 * a);
+                        tmem_st4(sf + C::kSpWb + 4 * C::kBlk * a + 4 * bk, w);
+                        // the residual view: each scale of a 32 (64) value block
+                        // for both of its 16 (32) value halves
+                        const uint4 lo = make_uint4(__byte_perm(w.x, 0u, 0x1100u), __byte_perm(w.y, 0u, 0x1100u),
+                                                    __byte_perm(w.z, 0u, 0x1100u), __byte_perm(w.w, 0u, 0x1100u));
+                        const uint4 hi = make_uint4(__byte_perm(w.x, 0u, 0x3322u), __byte_perm(w.y, 0u, 0x3322u),
+                                                    __byte_perm(w.z, 0u, 0x3322u), __byte_perm(w.w, 0u, 0x3322u));
+                        tmem_st4(sf + C::kSpWr + 4 * C::kBlk * (2 * a) + 4 * bk, lo);
+                        tmem_st4(sf + C::kSpWr + 4 * C::kBlk * (2 * a + 1) + 4 * bk, hi);
+                    }
+                }
+#pragma unroll
+                for (int a = 0; a < kAtomsPerTile; ++a)
+                    tmem_st4(sf + C::kSpR + 4 * a, lds128(st + C::kOffSFAR + 512 * a));
+                // metadata of this lane's row (lane quadrant q holds rows 32q ..):
+                // the first 64 bits for the first sparse MMA, the rest for the second
+                const uint4 mt = lds128(sbase + (uint32_t)(s * C::kStageBytes) + C::kOffMeta +
+                                        (uint32_t)(q * 32 + lane) * 16u);
+                tmem_st2(sf + C::kSpMeta, mt.x, mt.y);
+                tmem_st2(sf + C::kSpMeta + 4, mt.z, mt.w);
+            }
+#pragma unroll
+            for (int a = 0; a < (SP ? 0 : kAtomsPerTile); ++a) {
                 tmem_st4(sf + kSfaS + 4 * a, lds128(st + C::kOffSFAS + 512 * a));
                 tmem_st4(sf + kSfaR + 4 * a, lds128(st + C::kOffSFAR + 512 * a));
 #pragma unroll
@@ -632,19 +727,22 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 2-D byte tensor [rows][row_bytes], box = kBKBytes x box_rows, swizzled in
-// kBKBytes-wide atoms.
-static bool make_code_map(CUtensorMap *tm, const void *base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows) {
+// 2-D byte tensor [rows][row_bytes], box = box_bytes x box_rows (default: the
+// K tile, swizzled in kBKBytes-wide atoms; 64 bytes: the sparse mode's
+// compacted backbone, 64-byte swizzle; 16 bytes: its metadata, unswizzled).
+static bool make_code_map(CUtensorMap *tm, const void *base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows,
+                          uint32_t box_bytes = kBKBytes) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {row_bytes, rows};
     cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {(cuuint32_t)kBKBytes, box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)box_bytes, box_rows};
     cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle sw = box_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : box_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                    : CU_TENSOR_MAP_SWIZZLE_NONE;
     CUresult r = enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     kBKBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -667,7 +765,7 @@ static bool make_grouped_code_map(CUtensorMap *tm, const void *base, uint64_t ro
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, bool GROUPED, bool EXT, int BN>
+template <int FMT, bool GROUPED, bool EXT, int BN, bool SP = false>
 static sharq_status set_gemm_attrs() {
     static bool attr_done[64] = {};
     static std::mutex mu;  // one setter per device, also under concurrent first calls
@@ -676,37 +774,39 @@ static sharq_status set_gemm_attrs() {
     if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(mu);
     if (!attr_done[dev]) {
-        SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<FMT, GROUPED, EXT, BN>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TileCfg<BN>::kSmemBytes));
+        SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<FMT, GROUPED, EXT, BN, SP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TileCfg<BN, SP>::kSmemBytes));
         attr_done[dev] = true;
     }
     return SHARQ_OK;
 }
 
-template <int FMT, bool GROUPED, bool EXT, int BN>
+template <int FMT, bool GROUPED, bool EXT, int BN, bool SP = false>
 static sharq_status launch_gemm(LaunchCtx &ctx, const CUtensorMap &tm_as, const CUtensorMap &tm_ar,
-                                const CUtensorMap &tm_b, const GemmParams &gp, int64_t max_tiles) {
-    sharq_status st = set_gemm_attrs<FMT, GROUPED, EXT, BN>();
+                                const CUtensorMap &tm_b, const CUtensorMap &tm_meta, const GemmParams &gp,
+                                int64_t max_tiles) {
+    sharq_status st = set_gemm_attrs<FMT, GROUPED, EXT, BN, SP>();
     if (st != SHARQ_OK) return st;
     const unsigned grid = (unsigned)(max_tiles < ctx.num_sms ? max_tiles : ctx.num_sms);
-    dual_gemm_kernel<FMT, GROUPED, EXT, BN>
-        <<<grid, kGemmThreads, TileCfg<BN>::kSmemBytes, ctx.stream>>>(tm_as, tm_ar, tm_b, gp);
+    dual_gemm_kernel<FMT, GROUPED, EXT, BN, SP>
+        <<<grid, kGemmThreads, TileCfg<BN, SP>::kSmemBytes, ctx.stream>>>(tm_as, tm_ar, tm_b, tm_meta, gp);
     ctx.launches++;
     SQ_CUDA_TRY(cudaGetLastError());
     return SHARQ_OK;
 }
 
 // Split-K launch: `tiles` clusters of gp.split CTAs, one tile per cluster.
-template <int FMT, bool EXT>
+template <int FMT, bool EXT, bool SP = false>
 static sharq_status launch_gemm_split(LaunchCtx &ctx, const CUtensorMap &tm_as, const CUtensorMap &tm_ar,
-                                      const CUtensorMap &tm_b, const GemmParams &gp, int64_t tiles) {
-    sharq_status st = set_gemm_attrs<FMT, false, EXT, kDenseBN>();
+                                      const CUtensorMap &tm_b, const CUtensorMap &tm_meta, const GemmParams &gp,
+                                      int64_t tiles) {
+    sharq_status st = set_gemm_attrs<FMT, false, EXT, kDenseBN, SP>();
     if (st != SHARQ_OK) return st;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3((unsigned)(tiles * gp.split), 1, 1);
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
-    cfg.dynamicSmemBytes = TileCfg<kDenseBN>::kSmemBytes;
+    cfg.dynamicSmemBytes = TileCfg<kDenseBN, SP>::kSmemBytes;
     cfg.stream = ctx.stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -715,7 +815,8 @@ static sharq_status launch_gemm_split(LaunchCtx &ctx, const CUtensorMap &tm_as, 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    SQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, dual_gemm_kernel<FMT, false, EXT, kDenseBN>, tm_as, tm_ar, tm_b, gp));
+    SQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, dual_gemm_kernel<FMT, false, EXT, kDenseBN, SP>, tm_as, tm_ar, tm_b, tm_meta,
+                                   gp));
     ctx.launches++;
     SQ_CUDA_TRY(cudaGetLastError());
     return SHARQ_OK;
@@ -790,30 +891,45 @@ static GemmParams gemm_params(LaunchCtx &ctx, const sharq_prep &P, const sharq_w
 
 sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, const void *bias, void *out) {
     if (P.m_tok == 0) return SHARQ_OK;
-    CUtensorMap tm_as, tm_ar, tm_b;
-    if (!make_code_map(&tm_as, P.s_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
+    const bool sp = P.sparse != 0;
+    CUtensorMap tm_as, tm_ar, tm_b, tm_meta;
+    if (!make_code_map(&tm_as, P.s_codes, (uint64_t)(P.k / (sp ? 4 : 2)), (uint64_t)P.m_tok, kBM,
+                       sp ? kBKBytes / 2 : kBKBytes) ||
         !make_code_map(&tm_ar, P.r_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kBM) ||
         !make_code_map(&tm_b, W.codes, (uint64_t)(W.k / 2), (uint64_t)W.n_out, kDenseBN))
         return SHARQ_ERR_CUDA;
+    if (sp) {
+        if (!make_code_map(&tm_meta, P.meta, (uint64_t)(P.k / 16), (uint64_t)P.m_tok, kBM, 16)) return SHARQ_ERR_CUDA;
+    } else {
+        tm_meta = tm_b;  // unused
+    }
     GemmParams gp = gemm_params(ctx, P, W, out);
     gp.bias = (const __half *)bias;
     const int64_t tiles = ((P.m_tok + kBM - 1) / kBM) * ((W.n_out + kDenseBN - 1) / kDenseBN);
     const int kt_count = (int)(P.k / (2 * kBKBytes));
     gp.split = P.fmt == kFmtNV ? choose_split<kFmtNV>(ctx, tiles, kt_count) : choose_split<kFmtMX>(ctx, tiles, kt_count);
+    if (sp) {  // no bias or fused segments in this mode (checked by the caller)
+        if (gp.split > 1)
+            return P.fmt == kFmtNV ? launch_gemm_split<kFmtNV, false, true>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles)
+                                   : launch_gemm_split<kFmtMX, false, true>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles);
+        return P.fmt == kFmtNV
+                   ? launch_gemm<kFmtNV, false, false, kDenseBN, true>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles)
+                   : launch_gemm<kFmtMX, false, false, kDenseBN, true>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles);
+    }
     // the extended epilogue (fused segments, bias) only where needed
     const bool ext = gp.bias != nullptr || gp.segs > 1;
     if (gp.split > 1) {
         if (ext)
-            return P.fmt == kFmtNV ? launch_gemm_split<kFmtNV, true>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
-                                   : launch_gemm_split<kFmtMX, true>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
-        return P.fmt == kFmtNV ? launch_gemm_split<kFmtNV, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
-                               : launch_gemm_split<kFmtMX, false>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
+            return P.fmt == kFmtNV ? launch_gemm_split<kFmtNV, true>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles)
+                                   : launch_gemm_split<kFmtMX, true>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles);
+        return P.fmt == kFmtNV ? launch_gemm_split<kFmtNV, false>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles)
+                               : launch_gemm_split<kFmtMX, false>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles);
     }
     if (ext)
-        return P.fmt == kFmtNV ? launch_gemm<kFmtNV, false, true, kDenseBN>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
-                               : launch_gemm<kFmtMX, false, true, kDenseBN>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
-    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, false, false, kDenseBN>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
-                           : launch_gemm<kFmtMX, false, false, kDenseBN>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
+        return P.fmt == kFmtNV ? launch_gemm<kFmtNV, false, true, kDenseBN>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles)
+                               : launch_gemm<kFmtMX, false, true, kDenseBN>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles);
+    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, false, false, kDenseBN>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles)
+                           : launch_gemm<kFmtMX, false, false, kDenseBN>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles);
 }
 
 sharq_status launch_linear_grouped(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, const int32_t *offsets,
@@ -833,8 +949,8 @@ sharq_status launch_linear_grouped(LaunchCtx &ctx, const sharq_prep &P, const sh
     // at most P.m_tok / 128 m tiles (the device checks the offsets against it)
     const int64_t tiles = (P.m_tok / kBM) * ((W.n_out + kGroupedBN - 1) / kGroupedBN);
     if (tiles == 0) return SHARQ_OK;
-    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, true, false, kGroupedBN>(ctx, tm_as, tm_ar, tm_b, gp, tiles)
-                           : launch_gemm<kFmtMX, true, false, kGroupedBN>(ctx, tm_as, tm_ar, tm_b, gp, tiles);
+    return P.fmt == kFmtNV ? launch_gemm<kFmtNV, true, false, kGroupedBN>(ctx, tm_as, tm_ar, tm_b, tm_b, gp, tiles)
+                           : launch_gemm<kFmtMX, true, false, kGroupedBN>(ctx, tm_as, tm_ar, tm_b, tm_b, gp, tiles);
 }
 
 }  // namespace sq

@@ -61,14 +61,38 @@ SQ_HD PrepLayout prep_layout(int64_t m_tok, int64_t k, int n, int m, int fmt) {
     return L;
 }
 
+// Sections of a prep buffer in the pair-wise 4:8 mode: backbone codes
+// K-compacted to the kept half ([rows][k/4] bytes), backbone scales one per
+// 2 blk values, metadata 4 bits per group of 8 ([rows][k/16] bytes, the
+// layout the sparse MMA reads: group g of a row in bits 4g .. 4g+3, the
+// lower kept pair's index in the low two bits); residual as in prep_layout.
+SQ_HD PrepLayout prep_layout_sparse(int64_t m_tok, int64_t k, int fmt) {
+    PrepLayout L;
+    L.sf_rows = round_up(m_tok > 0 ? m_tok : 1, kActRowPad);
+    L.sf_bytes = L.sf_rows * (k / blk_of(fmt));  // residual scales
+    L.meta_row = k / 16;
+    const int64_t s_sf = L.sf_rows * (k / (2 * blk_of(fmt)));
+    int64_t off = 0;
+    L.s_codes = off; off = round_up(off + m_tok * (k / 4), kAlign);
+    L.r_codes = off; off = round_up(off + m_tok * (k / 2), kAlign);
+    L.s_scales = off; off = round_up(off + s_sf, kAlign);
+    L.r_scales = off; off = round_up(off + L.sf_bytes, kAlign);
+    L.meta = off; off = round_up(off + m_tok * L.meta_row, kAlign);
+    L.stats = off; off = round_up(off + m_tok * 8, kAlign);
+    L.words = off; off = round_up(off + 64, kAlign);
+    L.total = off;
+    return L;
+}
+
 struct WLayout {
     int64_t codes, scales, words, total, sf_rows, sf_bytes;
 };
 
-SQ_HD WLayout w_layout(int64_t n_out, int64_t k, int fmt) {
+// sparse: the pair-wise mode's weights, one scale per 2 blk values.
+SQ_HD WLayout w_layout(int64_t n_out, int64_t k, int fmt, bool sparse = false) {
     WLayout L;
     L.sf_rows = round_up(n_out, kWRowPad);
-    L.sf_bytes = L.sf_rows * (k / blk_of(fmt));
+    L.sf_bytes = L.sf_rows * (k / (blk_of(fmt) * (sparse ? 2 : 1)));
     int64_t off = 0;
     L.codes = off; off = round_up(off + n_out * (k / 2), kAlign);
     L.scales = off; off = round_up(off + L.sf_bytes, kAlign);

@@ -868,6 +868,14 @@ __device__ __forceinline__ uint32_t nibble_mask8(uint32_t k) {
     return x * 0xFu;
 }
 
+// Block quantization of one thread's 16 values given the amax `a` of the
+// whole block they belong to (this unit's 16, or the 32 / 64 values of a
+// lane pair / quad).
+template <int FMT>
+__device__ __forceinline__ float quantize16_amax(const float (&v)[kUnit], float a, float s_t, float c6, float y6,
+                                                 const float4 *tab, uint32_t &scale_code, uint32_t &codes_lo,
+                                                 uint32_t &codes_hi);
+
 template <int FMT>
 __device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, float c6, float y6, const float4 *tab,
                                             uint32_t &scale_code, uint32_t &codes_lo, uint32_t &codes_hi) {
@@ -875,6 +883,13 @@ __device__ __forceinline__ float quantize16(const float (&v)[kUnit], float s_t, 
 #pragma unroll
     for (int i = 0; i < kUnit; ++i) a = fmaxf(a, fabsf(v[i]));
     if (FMT == kFmtMX) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
+    return quantize16_amax<FMT>(v, a, s_t, c6, y6, tab, scale_code, codes_lo, codes_hi);
+}
+
+template <int FMT>
+__device__ __forceinline__ float quantize16_amax(const float (&v)[kUnit], float a, float s_t, float c6, float y6,
+                                                 const float4 *tab, uint32_t &scale_code, uint32_t &codes_lo,
+                                                 uint32_t &codes_hi) {
     // Step d and scale code as block_step gives them. NVFP4: the division
     // a / c6 by the reciprocal method when y6 = RN(1/c6) != 0 (the caller
     // sets y6 = 0 unless c6 is in [2^-90, 2^90]), exact for quotients >=
@@ -996,6 +1011,86 @@ __device__ __forceinline__ void encode_core(const float (&v)[kUnit], int n, cons
             }
     }
     o.mbits = mbits;
+}
+
+// ---------------------------------------------------------------------------
+// Pair-wise 4:8 sparse-backbone mode. In every aligned group of 8 values
+// along K (four adjacent pairs) the two pairs with the largest pair
+// magnitude max(|a|, |b|) are kept, equal magnitudes going to the lower
+// pair; the backbone's blocks are 32 values (NVFP4, a lane pair of units) or
+// 64 (MXFP4, a lane quad), the blocks the structured-sparse block-scaled MMA
+// applies; its kept codes are stored K-compacted (2 bytes per group) beside
+// 4 metadata bits per group (first kept pair | second << 2). The residual is
+// as in the default mode.
+
+// Bit j set: pair j is among the two largest keys (equal keys: lower pair
+// first). The majority logic of keep_mask_42 on four non-negative keys.
+__device__ __forceinline__ uint32_t keep_pairs(float a0, float a1, float a2, float a3) {
+    const uint32_t s01 = __float_as_uint(__fsub_rn(a0, a1)), s02 = __float_as_uint(__fsub_rn(a0, a2));
+    const uint32_t s03 = __float_as_uint(__fsub_rn(a0, a3)), s12 = __float_as_uint(__fsub_rn(a1, a2));
+    const uint32_t s13 = __float_as_uint(__fsub_rn(a1, a3)), s23 = __float_as_uint(__fsub_rn(a2, a3));
+    const uint32_t k0 = ~((s01 & s02) | (s01 & s03) | (s02 & s03));
+    const uint32_t k1 = (s01 & ~s12) | (s01 & ~s13) | (~s12 & ~s13);
+    const uint32_t k2 = (s02 & s12) | (s02 & ~s23) | (s12 & ~s23);
+    const uint32_t k3 = (s03 & s13) | (s03 & s23) | (s13 & s23);
+    return (k0 >> 31) | (k1 >> 31) << 1 | (k2 >> 31) << 2 | (k3 >> 31) << 3;
+}
+
+// 0xFF in byte j for every set bit j of a 4-bit mask (the four shifted
+// copies never overlap).
+__device__ __forceinline__ uint32_t pair_bytes(uint32_t n4) {
+    return ((n4 * 0x00204081u) & 0x01010101u) * 0xFFu;
+}
+
+struct SparseUnitCodes {
+    uint32_t s_comp;        // kept backbone codes, K-compacted (8 codes)
+    uint32_t s_scale;       // backbone block scale code (of the lane pair / quad)
+    uint32_t r_lo, r_hi;    // residual codes
+    uint32_t r_scale;       // residual block scale code
+    uint32_t meta;          // metadata byte: group 0 in bits 0-3, group 1 in bits 4-7
+};
+
+template <int FMT>
+__device__ __forceinline__ void encode_core_sparse(const float (&v)[kUnit], const float4 *tab, float s_t, float c6,
+                                                   float y6, SparseUnitCodes &o) {
+    uint32_t pk = 0;  // kept pairs: 4 bits per group
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        float key[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) key[j] = fmaxf(fabsf(v[8 * g + 2 * j]), fabsf(v[8 * g + 2 * j + 1]));
+        pk |= keep_pairs(key[0], key[1], key[2], key[3]) << (4 * g);
+    }
+    // Every group keeps its largest magnitude, so the backbone block's amax
+    // is that of X_ln over the block's units, and so are the step and the
+    // kept codes: the codes of X_ln itself, the dropped pairs cleared.
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kUnit; ++i) a = fmaxf(a, fabsf(v[i]));
+    a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
+    if (FMT == kFmtMX) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
+    uint32_t c0, c1;
+    const float ds = quantize16_amax<FMT>(v, a, s_t, c6, y6, tab, o.s_scale, c0, c1);
+    // A group's kept-pair nibble has two bits set, so nibble >> 1 (1..6)
+    // indexes byte tables: the metadata field (first | second << 2) and the
+    // byte selector (first | second << 4) of the group's kept code bytes.
+    const uint32_t sel2 = (pk >> 1) & 0x77u;
+    const uint32_t mt = __byte_perm(0x09080400u, 0x000E0D0Cu, sel2);  // -, 4, 8, 9, 12, 13, 14, -
+    o.meta = (mt & 0xFu) | ((mt >> 4) & 0xF0u);
+    const uint32_t ct = __byte_perm(0x21201000u, 0x00323130u, sel2);  // -, 10, 20, 21, 30, 31, 32, - (hex)
+    o.s_comp = __byte_perm(c0, c1, ct + 0x4400u);                      // group 1's bytes are 4..7
+    c0 &= pair_bytes(pk & 0xFu);
+    c1 &= pair_bytes(pk >> 4);
+    // Residual against the quantized backbone, as in the default mode.
+    float r[kUnit];
+#pragma unroll
+    for (int i = 0; i < kUnit; i += 2) {
+        const uint32_t byte = ((i < 8 ? c0 : c1) >> (4 * (i % 8))) & 0xFFu;
+        const float2 cv = e2m1x2_value(byte);
+        r[i] = __fsub_rn(v[i], __fmul_rn(cv.x, ds));
+        r[i + 1] = __fsub_rn(v[i + 1], __fmul_rn(cv.y, ds));
+    }
+    quantize16<FMT>(r, s_t, c6, y6, tab, o.r_scale, o.r_lo, o.r_hi);
 }
 
 // Arguments of the encode step (one unit = 16 consecutive elements of a row).
@@ -1176,6 +1271,45 @@ prep_encode_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ 
     }
 }
 
+// LayerNorm apply on one unit's 16 values (x as eight fp16 pairs): (x - mu)
+// * rstd in packed pairs (no multiply feeds an add there), then gamma and
+// beta (AFFINE; either may be NULL) with scalar intrinsics, which are never
+// fused into a multiply-add.
+template <bool AFFINE>
+__device__ __forceinline__ void ln_apply16(const uint32_t (&xw)[8], float2 st, const uint16_t *gamma,
+                                           const uint16_t *beta, int u, bool act, float (&v)[kUnit]) {
+    const uint64_t mu2 = pk2(st.x, st.x), rs2 = pk2(st.y, st.y);
+    uint4 ga = make_uint4(0, 0, 0, 0), gb = ga, ba = ga, bb = ga;
+    if (AFFINE && act) {
+        if (gamma) {
+            ga = __ldg(reinterpret_cast<const uint4 *>(gamma + (int64_t)u * kUnit));
+            gb = __ldg(reinterpret_cast<const uint4 *>(gamma + (int64_t)u * kUnit) + 1);
+        }
+        if (beta) {
+            ba = __ldg(reinterpret_cast<const uint4 *>(beta + (int64_t)u * kUnit));
+            bb = __ldg(reinterpret_cast<const uint4 *>(beta + (int64_t)u * kUnit) + 1);
+        }
+    }
+    const uint32_t gw8[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+    const uint32_t bw8[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+        float2 f = up2(mul2(sub2(h2_to_f2(xw[p]), mu2), rs2));
+        if (AFFINE) {
+            if (gamma) {
+                f.x = __fmul_rn(f.x, h2f((uint16_t)gw8[p]));
+                f.y = __fmul_rn(f.y, h2f((uint16_t)(gw8[p] >> 16)));
+            }
+            if (beta) {
+                f.x = __fadd_rn(f.x, h2f((uint16_t)bw8[p]));
+                f.y = __fadd_rn(f.y, h2f((uint16_t)(bw8[p] >> 16)));
+            }
+        }
+        v[2 * p] = f.x;
+        v[2 * p + 1] = f.y;
+    }
+}
+
 // Encode pass over the rows of one activation: one warp per 512-element
 // chunk of a row (a lane per 16-element unit), the chunks of the persistent
 // grid's warps taken in reverse row order. The statistics pass reads the rows
@@ -1273,40 +1407,7 @@ prep_encode_rows_kernel(const EncodeArgs a, const unsigned *amax_word, float *__
         if (it + nwarps < items) fetch(m_tok - 1 - ri, ci, nw, nst);
 
         float v[kUnit];
-        {
-            // (x - mu) * rstd in packed pairs (no multiply feeds an add here);
-            // gamma and beta with scalar intrinsics, which are never fused.
-            const uint64_t mu2 = pk2(st.x, st.x), rs2 = pk2(st.y, st.y);
-            uint4 ga = make_uint4(0, 0, 0, 0), gb = ga, ba = ga, bb = ga;
-            if (AFFINE && act) {
-                if (a.gamma) {
-                    ga = __ldg(reinterpret_cast<const uint4 *>(a.gamma + (int64_t)u * kUnit));
-                    gb = __ldg(reinterpret_cast<const uint4 *>(a.gamma + (int64_t)u * kUnit) + 1);
-                }
-                if (a.beta) {
-                    ba = __ldg(reinterpret_cast<const uint4 *>(a.beta + (int64_t)u * kUnit));
-                    bb = __ldg(reinterpret_cast<const uint4 *>(a.beta + (int64_t)u * kUnit) + 1);
-                }
-            }
-            const uint32_t gw8[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
-            const uint32_t bw8[8] = {ba.x, ba.y, ba.z, ba.w, bb.x, bb.y, bb.z, bb.w};
-#pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                float2 f = up2(mul2(sub2(h2_to_f2(xw[p]), mu2), rs2));
-                if (AFFINE) {
-                    if (a.gamma) {
-                        f.x = __fmul_rn(f.x, h2f((uint16_t)gw8[p]));
-                        f.y = __fmul_rn(f.y, h2f((uint16_t)(gw8[p] >> 16)));
-                    }
-                    if (a.beta) {
-                        f.x = __fadd_rn(f.x, h2f((uint16_t)bw8[p]));
-                        f.y = __fadd_rn(f.y, h2f((uint16_t)(bw8[p] >> 16)));
-                    }
-                }
-                v[2 * p] = f.x;
-                v[2 * p + 1] = f.y;
-            }
-        }
+        ln_apply16<AFFINE>(xw, st, a.gamma, a.beta, u, act, v);
         UnitCodes o;
         encode_core<FMT, M, NK>(v, n, lut, tab, s_t, c6, y6, o);
         if (act) {
@@ -1341,6 +1442,107 @@ prep_encode_rows_kernel(const EncodeArgs a, const unsigned *amax_word, float *__
         s_sf[sf_offset(r, j, nblk)] = 0;
         r_sf[sf_offset(r, j, nblk)] = 0;
     }
+}
+
+// Encode pass of the pair-wise 4:8 mode: the walk of prep_encode_rows_kernel
+// (a warp per 512-element row chunk, reverse row order, next chunk
+// prefetched, launched as a programmatic dependent of the statistics pass),
+// with the backbone stored K-compacted (4 bytes per unit), its block scale
+// once per lane pair (NVFP4, 32 values) or quad (MXFP4, 64 values) and one
+// metadata byte per unit.
+template <int FMT, bool AFFINE>
+__global__ void __launch_bounds__(kEncodeThreads, SQ_ENCODE_MIN_CTAS)
+prep_encode_sparse_kernel(const EncodeArgs a, const unsigned *amax_word, float *__restrict__ s_t_out,
+                          int64_t sf_rows) {
+    __shared__ float4 tab[128];  // NVFP4 steps and reciprocals by scale code
+    griddep_wait();  // the statistics and the amax word are complete
+    // (read with L2 loads through pointers without __restrict__, so that no
+    // load can move above the wait)
+    const float amax = __uint_as_float(__ldcg(amax_word));
+    const float s_t = (FMT == kFmtNV && amax != 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
+    const float c6 = __fmul_rn(6.0f, s_t);
+    const float y6 = (FMT == kFmtNV && c6 >= 0x1p-90f && c6 <= 0x1p90f) ? __frcp_rn(c6) : 0.0f;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *s_t_out = s_t;
+    build_step_table<FMT>(tab, s_t);
+    __syncthreads();
+
+    const uint16_t *__restrict__ x = a.x;
+    const float2 *stats = a.stats;
+    uint8_t *__restrict__ s_codes = a.s_codes;
+    uint8_t *__restrict__ r_codes = a.r_codes;
+    uint8_t *__restrict__ s_sf = a.s_sf;
+    uint8_t *__restrict__ r_sf = a.r_sf;
+    uint8_t *__restrict__ meta = a.meta;
+    const int64_t k = a.k, m_tok = a.m_tok;
+    const int64_t nblk_r = k / (FMT == kFmtNV ? 16 : 32), nblk_s = nblk_r / 2;
+    const int lane = threadIdx.x & 31;
+    const int upr = (int)(k / kUnit);
+    const int chunks = (upr + 31) >> 5;
+    const int64_t nwarps = (int64_t)gridDim.x * (kEncodeThreads / 32);
+    const int64_t gw = (int64_t)blockIdx.x * (kEncodeThreads / 32) + threadIdx.x / 32;
+    const int64_t items = m_tok * chunks;
+    const int64_t step_r = nwarps / chunks;
+    const int step_c = (int)(nwarps - step_r * chunks);
+    int64_t ri = gw / chunks;
+    int ci = (int)(gw - ri * chunks);
+    uint32_t xw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    float2 st = make_float2(0.0f, 1.0f);
+    const bool x32 = (reinterpret_cast<uintptr_t>(x) & 31u) == 0;
+    auto fetch = [&](int64_t r, int c, uint32_t (&w)[8], float2 &sv) {
+        const int u = c * 32 + lane;
+        if (u < upr) {
+            const uint16_t *p = x + r * k + (int64_t)u * kUnit;
+            if (x32) {
+                ldg256_cs(p, w);
+            } else {
+                const uint4 va = __ldcs(reinterpret_cast<const uint4 *>(p)), vb = __ldcs(reinterpret_cast<const uint4 *>(p) + 1);
+                w[0] = va.x, w[1] = va.y, w[2] = va.z, w[3] = va.w, w[4] = vb.x, w[5] = vb.y, w[6] = vb.z, w[7] = vb.w;
+            }
+        }
+        sv = __ldcg(stats + r);
+    };
+    if (gw < items) fetch(m_tok - 1 - ri, ci, xw, st);
+    for (int64_t it = gw; it < items; it += nwarps) {
+        const int64_t row = m_tok - 1 - ri;
+        const int u = ci * 32 + lane;
+        const bool act = u < upr;
+        ri += step_r;
+        ci += step_c;
+        if (ci >= chunks) {
+            ci -= chunks;
+            ++ri;
+        }
+        uint32_t nw[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        float2 nst = make_float2(0.0f, 1.0f);
+        if (it + nwarps < items) fetch(m_tok - 1 - ri, ci, nw, nst);
+
+        float v[kUnit];
+        ln_apply16<AFFINE>(xw, st, a.gamma, a.beta, u, act, v);
+        SparseUnitCodes o;
+        encode_core_sparse<FMT>(v, tab, s_t, c6, y6, o);
+        if (act) {
+            *reinterpret_cast<uint32_t *>(s_codes + row * (k / 4) + (int64_t)u * 4) = o.s_comp;
+            *reinterpret_cast<uint2 *>(r_codes + row * (k / 2) + (int64_t)u * 8) = make_uint2(o.r_lo, o.r_hi);
+            meta[row * (k / 16) + u] = (uint8_t)o.meta;
+            if (FMT == kFmtNV) {
+                r_sf[sf_offset(row, u, nblk_r)] = (uint8_t)o.r_scale;
+                if ((u & 1) == 0) s_sf[sf_offset(row, u >> 1, nblk_s)] = (uint8_t)o.s_scale;
+            } else {
+                if ((u & 1) == 0) r_sf[sf_offset(row, u >> 1, nblk_r)] = (uint8_t)o.r_scale;
+                if ((u & 3) == 0) s_sf[sf_offset(row, u >> 2, nblk_s)] = (uint8_t)o.s_scale;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) xw[i] = nw[i];
+        st = nst;
+    }
+    // Zero scales of the padding rows of the last 128-row scale atoms.
+    const int64_t gthreads = (int64_t)gridDim.x * kEncodeThreads;
+    const int64_t t0 = (int64_t)blockIdx.x * kEncodeThreads + threadIdx.x;
+    for (int64_t i = t0; i < (sf_rows - m_tok) * nblk_r; i += gthreads)
+        r_sf[sf_offset(m_tok + i / nblk_r, i % nblk_r, nblk_r)] = 0;
+    for (int64_t i = t0; i < (sf_rows - m_tok) * nblk_s; i += gthreads)
+        s_sf[sf_offset(m_tok + i / nblk_s, i % nblk_s, nblk_s)] = 0;
 }
 
 constexpr int kGroupedTileTable = 4096;  // tiles whose group the grouped encode tabulates in shared memory
@@ -2096,6 +2298,45 @@ sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = P.m_tok > 0 ? 1 : 0;  // no statistics kernel before it otherwise
+    SQ_CUDA_TRY(cudaLaunchKernelExC(&cfg, fn, args));
+    ctx.launches++;
+    return SHARQ_OK;
+}
+
+// Pair-wise 4:8 mode: the statistics pass, then the sparse encode pass
+// (a programmatic dependent of it).
+sharq_status launch_prepare_sparse(LaunchCtx &ctx, const sharq_prep &P, const void *x, const void *gamma,
+                                   const void *beta, float eps, int norm) {
+    unsigned *words = reinterpret_cast<unsigned *>(P.tensor_scale) - 1;  // [0] amax bits, [1] s_t
+    SQ_CUDA_TRY(cudaMemsetAsync(words, 0, sizeof(unsigned), ctx.stream));
+    float2 *stats = reinterpret_cast<float2 *>(P.scratch);
+    const sharq_status sst = norm ? launch_stats<true>(ctx, P, x, gamma, beta, eps, stats, words)
+                                  : launch_stats<false>(ctx, P, x, gamma, beta, eps, stats, words);
+    if (sst != SHARQ_OK) return sst;
+    const bool affine = gamma != nullptr || beta != nullptr;
+    void *fn = P.fmt == kFmtNV
+                   ? (affine ? (void *)prep_encode_sparse_kernel<kFmtNV, true> : (void *)prep_encode_sparse_kernel<kFmtNV, false>)
+                   : (affine ? (void *)prep_encode_sparse_kernel<kFmtMX, true> : (void *)prep_encode_sparse_kernel<kFmtMX, false>);
+    const int64_t chunks = (P.k / kUnit + 31) / 32;
+    const int64_t warps = P.m_tok * chunks > 0 ? P.m_tok * chunks : 1;
+    const int64_t blocks = encode_grid(fn, ctx.num_sms, warps * 32);
+    EncodeArgs ea{(const uint16_t *)x, (const uint16_t *)gamma, (const uint16_t *)beta, stats, P.m_tok, P.k,
+                  P.meta_row_bytes, P.k / (P.fmt == kFmtNV ? 16 : 32), P.n, (uint8_t *)P.s_codes,
+                  (uint8_t *)P.r_codes, (uint8_t *)P.s_scales, (uint8_t *)P.r_scales, (uint8_t *)P.meta};
+    const unsigned *aw = words;
+    float *sto = P.tensor_scale;
+    int64_t sf_rows = P.sf_rows;
+    void *args[] = {&ea, &aw, &sto, &sf_rows};
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)blocks, 1, 1);
+    cfg.blockDim = dim3(kEncodeThreads, 1, 1);
+    cfg.stream = ctx.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = P.m_tok > 0 ? 1 : 0;
     SQ_CUDA_TRY(cudaLaunchKernelExC(&cfg, fn, args));
     ctx.launches++;
     return SHARQ_OK;

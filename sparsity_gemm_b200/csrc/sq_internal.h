@@ -18,6 +18,9 @@ struct LaunchCtx {
 // norm: 0 = LayerNorm, 1 = RMSNorm (beta must be NULL).
 sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, const void *gamma,
                             const void *beta, float eps, int norm);
+// The pair-wise 4:8 mode (P from prep_layout_sparse).
+sharq_status launch_prepare_sparse(LaunchCtx &ctx, const sharq_prep &P, const void *x, const void *gamma,
+                                   const void *beta, float eps, int norm);
 sharq_status launch_prepare_grouped(LaunchCtx &ctx, const sharq_prep &P, const void *x, int64_t rows,
                                     const int32_t *offsets, int32_t groups, const void *gamma, const void *beta,
                                     float eps, int norm);

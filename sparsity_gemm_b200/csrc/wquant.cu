@@ -53,13 +53,16 @@ __global__ void __launch_bounds__(kWThreads) absmax_kernel(const uint16_t *__res
 
 // Rows [0, sf_rows) of one weight (rows >= n_out are scale-layout padding),
 // written at rows row0 + r of the code and scale layouts (row0 > 0: a
-// segment of a fused weight).
-template <int FMT>
+// segment of a fused weight). BLK: the block length (the format's own, or
+// twice it for the pair-wise sparse mode's weights); each thread takes a
+// chunk of max(BLK, 32) values of a row.
+template <int FMT, int BLK>
 __global__ void __launch_bounds__(kWThreads)
 wq_encode_kernel(const uint16_t *__restrict__ w, int64_t n_out, int64_t sf_rows, int64_t k,
                  const unsigned *__restrict__ amax_word, float *__restrict__ s_tw_out, uint8_t *__restrict__ codes,
                  uint8_t *__restrict__ sf, int64_t gstride, int64_t row0) {
-    constexpr int BLK = FMT == kFmtNV ? 16 : 32;
+    constexpr int CH = BLK > 32 ? BLK : 32;  // values per thread
+    constexpr int NB = CH / BLK;             // blocks per chunk (1 or 2)
     {
         const int64_t gofs = (int64_t)blockIdx.y * gstride;
         w += (int64_t)blockIdx.y * n_out * k;
@@ -68,29 +71,30 @@ wq_encode_kernel(const uint16_t *__restrict__ w, int64_t n_out, int64_t sf_rows,
         codes += gofs;
         sf += gofs;
     }
-    constexpr int NB = 32 / BLK;
     const float amax = __uint_as_float(*amax_word);
     const float s_t = (FMT == kFmtNV && amax != 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
     const float c6 = __fmul_rn(6.0f, s_t);
     if (blockIdx.x == 0 && threadIdx.x == 0) *s_tw_out = s_t;
-    const int64_t cpr = k / 32, nblk = k / BLK, total = sf_rows * cpr;
+    const int64_t cpr = k / CH, nblk = k / BLK, total = sf_rows * cpr;
     for (int64_t t = (int64_t)blockIdx.x * kWThreads + threadIdx.x; t < total; t += (int64_t)gridDim.x * kWThreads) {
         const int64_t row = t / cpr, c = t - row * cpr, orow = row0 + row;
         if (row >= n_out) {  // scale-layout padding rows
-            if (FMT == kFmtNV) *reinterpret_cast<uint16_t *>(sf + sf_offset(orow, 2 * c, nblk)) = 0;
+            if (NB == 2) *reinterpret_cast<uint16_t *>(sf + sf_offset(orow, 2 * c, nblk)) = 0;
             else sf[sf_offset(orow, c, nblk)] = 0;
             continue;
         }
-        const uint4 *wp = reinterpret_cast<const uint4 *>(w + row * k + c * 32);
-        float v[32];
+        const uint4 *wp = reinterpret_cast<const uint4 *>(w + row * k + c * CH);
+        float v[CH];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < CH / 8; ++q) {
             uint4 u = __ldcs(wp + q);
             const uint32_t ws[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[8 * q + i] = h2f((uint16_t)(ws[i / 2] >> (16 * (i % 2))));
         }
-        uint32_t pk[4] = {0, 0, 0, 0}, sc[NB];
+        uint32_t pk[CH / 8], sc[NB];
+#pragma unroll
+        for (int i = 0; i < CH / 8; ++i) pk[i] = 0;
 #pragma unroll
         for (int bk = 0; bk < NB; ++bk) {
             float a = 0.0f;
@@ -105,10 +109,26 @@ wq_encode_kernel(const uint16_t *__restrict__ w, int64_t n_out, int64_t sf_rows,
                     pk[i / 8] |= e2m1x2(__fdiv_rn(v[i], d), __fdiv_rn(v[i + 1], d)) << (4 * (i % 8));
             }
         }
-        *reinterpret_cast<uint4 *>(codes + orow * (k / 2) + c * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        if (FMT == kFmtNV) *reinterpret_cast<uint16_t *>(sf + sf_offset(orow, 2 * c, nblk)) = (uint16_t)(sc[0] | (sc[NB - 1] << 8));
+#pragma unroll
+        for (int q = 0; q < CH / 32; ++q)
+            *reinterpret_cast<uint4 *>(codes + orow * (k / 2) + c * (CH / 2) + 16 * q) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        if (NB == 2) *reinterpret_cast<uint16_t *>(sf + sf_offset(orow, 2 * c, nblk)) = (uint16_t)(sc[0] | (sc[NB - 1] << 8));
         else sf[sf_offset(orow, c, nblk)] = (uint8_t)sc[0];
     }
+}
+
+// The encode launch of one weight payload's rows.
+template <int FMT>
+static void launch_wq_encode(dim3 grid, cudaStream_t stream, bool sparse, const uint16_t *w, int64_t n_out,
+                             int64_t sf_rows, int64_t k, const unsigned *aw, float *s_tw, uint8_t *codes, uint8_t *sf,
+                             int64_t gstride, int64_t row0) {
+    if (sparse)
+        wq_encode_kernel<FMT, FMT == kFmtNV ? 32 : 64><<<grid, kWThreads, 0, stream>>>(w, n_out, sf_rows, k, aw, s_tw,
+                                                                                     codes, sf, gstride, row0);
+    else
+        wq_encode_kernel<FMT, FMT == kFmtNV ? 16 : 32><<<grid, kWThreads, 0, stream>>>(w, n_out, sf_rows, k, aw, s_tw,
+                                                                                     codes, sf, gstride, row0);
 }
 
 sharq_status launch_quantize_weight(LaunchCtx &ctx, const sharq_wq &W, const void *w, int64_t groups,
@@ -124,18 +144,18 @@ sharq_status launch_quantize_weight(LaunchCtx &ctx, const sharq_wq &W, const voi
     const dim3 ga((unsigned)blocks, (unsigned)groups);
     absmax_kernel<<<ga, kWThreads, 0, ctx.stream>>>((const uint16_t *)w, count, words, gstride);
     ctx.launches++;
-    const int64_t total = W.sf_rows * (W.k / 32);
+    const bool sparse = W.sparse != 0;
+    const int64_t ch = (sparse && W.fmt == kFmtMX) ? 64 : 32;  // values per encode thread
+    const int64_t total = W.sf_rows * (W.k / ch);
     int64_t eb = (total + kWThreads - 1) / kWThreads;
     if (eb > 2 * per_group_cap) eb = 2 * per_group_cap;
     const dim3 ge((unsigned)eb, (unsigned)groups);
     if (W.fmt == kFmtNV)
-        wq_encode_kernel<kFmtNV><<<ge, kWThreads, 0, ctx.stream>>>(
-            (const uint16_t *)w, W.n_out, W.sf_rows, W.k, words, W.tensor_scale, (uint8_t *)W.codes,
-            (uint8_t *)W.scales_backbone, gstride, 0);
+        launch_wq_encode<kFmtNV>(ge, ctx.stream, sparse, (const uint16_t *)w, W.n_out, W.sf_rows, W.k, words,
+                                 W.tensor_scale, (uint8_t *)W.codes, (uint8_t *)W.scales_backbone, gstride, 0);
     else
-        wq_encode_kernel<kFmtMX><<<ge, kWThreads, 0, ctx.stream>>>(
-            (const uint16_t *)w, W.n_out, W.sf_rows, W.k, words, W.tensor_scale, (uint8_t *)W.codes,
-            (uint8_t *)W.scales_backbone, gstride, 0);
+        launch_wq_encode<kFmtMX>(ge, ctx.stream, sparse, (const uint16_t *)w, W.n_out, W.sf_rows, W.k, words,
+                                 W.tensor_scale, (uint8_t *)W.codes, (uint8_t *)W.scales_backbone, gstride, 0);
     ctx.launches++;
     SQ_CUDA_TRY(cudaGetLastError());
     return SHARQ_OK;
@@ -163,13 +183,11 @@ sharq_status launch_quantize_weight_fused(LaunchCtx &ctx, const sharq_wq &W, con
         int64_t eb = (iter_rows * (W.k / 32) + kWThreads - 1) / kWThreads;
         if (eb > (int64_t)ctx.num_sms * 8) eb = (int64_t)ctx.num_sms * 8;
         if (W.fmt == kFmtNV)
-            wq_encode_kernel<kFmtNV><<<(unsigned)eb, kWThreads, 0, ctx.stream>>>(
-                wg, rows, iter_rows, W.k, aw, W.tensor_scale + g, (uint8_t *)W.codes, (uint8_t *)W.scales_backbone, 0,
-                off);
+            launch_wq_encode<kFmtNV>(dim3((unsigned)eb), ctx.stream, false, wg, rows, iter_rows, W.k, aw,
+                                     W.tensor_scale + g, (uint8_t *)W.codes, (uint8_t *)W.scales_backbone, 0, off);
         else
-            wq_encode_kernel<kFmtMX><<<(unsigned)eb, kWThreads, 0, ctx.stream>>>(
-                wg, rows, iter_rows, W.k, aw, W.tensor_scale + g, (uint8_t *)W.codes, (uint8_t *)W.scales_backbone, 0,
-                off);
+            launch_wq_encode<kFmtMX>(dim3((unsigned)eb), ctx.stream, false, wg, rows, iter_rows, W.k, aw,
+                                     W.tensor_scale + g, (uint8_t *)W.codes, (uint8_t *)W.scales_backbone, 0, off);
         ctx.launches++;
         off += rows;
     }
