@@ -87,8 +87,11 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-quality", action="store_true", help="skip the output-error report")
     ap.add_argument("--cpu-sample-tokens", type=int, default=1)
-    ap.add_argument("--cpu-sample-cols", type=int, default=512,
+    ap.add_argument("--cpu-sample-cols", type=int, default=8192,
                     help="output columns of each linear in the CPU sample (cost is linear in columns)")
+    ap.add_argument("--ref-sample-cols", type=int, default=1024,
+                    help="output columns of each linear in each step of the reference arm's sample")
+    ap.add_argument("--no-extras", action="store_true", help="skip the other workloads' summary numbers")
     ap.add_argument("--case", default=None,
                     help="time one op instead of the layer set: prep:M:K[:fmt:n:m] or linear:M:N:K[:fmt:n:m] "
                          "(fmt 0 = NVFP4, 1 = MXFP4); used for profiling and shape sweeps")
@@ -362,6 +365,8 @@ def run_sharq(args, world, rank, local):
         result["quality"] = quality_report(sq, dev, xs, preps, prep_bufs, outs, ls, prep_index)
     if not args.no_e2e:
         result["e2e"] = e2e_sharq(args, sq, dev, stream, xs_host, preps, prep_bufs, qws, outs, ls, prep_index, world)
+    if rank == 0 and world == 1 and not args.no_extras:
+        result["configs"] = config_summaries(args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args)
     return result
@@ -527,12 +532,12 @@ def oracle_sample(tokens: int, cols: int):
 
 
 def oracle_step(sample):
+    """One pass of the oracle over the sample; returns the linears' outputs."""
     import oracle
     ls, preps, xs, ws = sample
     prepared = [oracle.prepare(x, None, None, EPS, N_KEEP, M_GROUP, oracle.NVFP4) for x in xs]
     pidx = {name: i for i, (name, _) in enumerate(preps)}
-    for j, lin in enumerate(ls.linears):
-        oracle.linear_prepared(prepared[pidx[lin.prep]], ws[j])
+    return [oracle.linear_prepared(prepared[pidx[lin.prep]], ws[j])[0] for j, lin in enumerate(ls.linears)]
 
 
 def token_fraction(sample, tokens):
@@ -545,22 +550,90 @@ def token_fraction(sample, tokens):
     return tokens * macs_sample / macs_full
 
 
+def _host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
 def cpu_baseline(args):
+    """The oracle on the host cores, on a bounded sample of the step: the
+    single-threaded build on one core, then the OpenMP build of the same
+    source on all cores (independent rows and output elements split across
+    threads), whose outputs are checked equal to the single-threaded ones."""
+    import oracle
     sample = oracle_sample(args.cpu_sample_tokens, args.cpu_sample_cols)
+    oracle.use_openmp(False)
     t0 = time.perf_counter()
-    oracle_step(sample)
-    dt = time.perf_counter() - t0
+    out1 = oracle_step(sample)
+    dt1 = time.perf_counter() - t0
     tok = token_fraction(sample, args.cpu_sample_tokens)
-    return {"value": tok / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{args.cpu_sample_tokens} token(s): full prep of each activation row, and the first "
-                      f"{args.cpu_sample_cols} output columns of each linear (cost linear in columns; value = "
-                      f"{tok:.4f} token-equivalents / {dt:.2f} s), single-threaded C oracle"}
+    oracle.use_openmp(True)
+    threads = oracle.threads()
+    t0 = time.perf_counter()
+    out_n = oracle_step(sample)
+    dtn = time.perf_counter() - t0
+    oracle.use_openmp(False)
+    same = all(np.array_equal(a, b) for a, b in zip(out1, out_n))
+    desc = (f"{args.cpu_sample_tokens} token(s): full prep of each activation row, and the first "
+            f"{args.cpu_sample_cols} output columns of each linear (cost linear in columns; value = "
+            f"{tok:.4f} token-equivalents / time)")
+    return {"value": tok / dt1, "unit": UNIT, "cores": 1, "kind": "oracle", "nproc": _host_cores(),
+            "sample": desc + f", single-threaded C oracle: {dt1:.2f} s",
+            "all_cores": {"value": tok / dtn, "unit": UNIT, "cores": threads, "seconds": dtn,
+                          "build": "same source with OpenMP over independent rows and output elements",
+                          "outputs_identical": bool(same)}}
+
+
+def config_summaries(args):
+    """Summary numbers of the other workloads, measured after the timed step
+    (each on its own, L2 flushed before every step): the preparation with the
+    normalization's parameters (LayerNorm gamma/beta, RMSNorm weight; the
+    timed step takes none), the pair-wise 4:8 sparse-backbone mode on the
+    same layer set, the Qwen2.5-7B layer set (NVFP4/MXFP4 x 2:4/4:8, M =
+    4096), the Qwen3-30B-A3B MoE FFN (M = 4096) and the decode-vs-prefill
+    sweep of the down projection (1% outliers)."""
+    peaks, _ = load_peaks()
+    st, wu = 5, 2
+    M = args.tokens
+    ls = synth.LLAMA31_8B
+    out = {"steps": st, "warmup": wu, "timing": "median per step, CUDA events, L2 flushed before every step"}
+    keep = ("tokens_per_s", "ms_per_step", "prep_ms", "gemm_ms", "gemm_tflops", "gemm_frac", "gemm_executed_frac",
+            "prep_gbs", "prep_frac", "prep_bytes_per_elem")
+    pick = lambda r: {k: r[k] for k in ("fmt", "nm") + keep}
+    aff = {}
+    for name, a in (("layernorm_gamma_beta", "layer"), ("rmsnorm_weight", "rms")):
+        prep_ms, gemm_ms = time_layer_set(ls, M, 0, N_KEEP, M_GROUP, st, wu, affine=a)
+        aff[name] = pick(layer_set_report(ls, M, 0, N_KEEP, M_GROUP, prep_ms, gemm_ms, peaks))
+    out["llama31_8b_prep_with_norm_params"] = aff
+    prep_ms, gemm_ms = time_layer_set(ls, M, 0, N_KEEP, M_GROUP, st, wu, sparse=True)
+    out["llama31_8b_pairwise_sparse_backbone"] = layer_set_report(ls, M, 0, N_KEEP, M_GROUP, prep_ms, gemm_ms,
+                                                                  peaks, sparse=True)
+    q = []
+    for fmt in (0, 1):
+        for n, m in ((2, 4), (4, 8)):
+            prep_ms, gemm_ms = time_layer_set(synth.QWEN25_7B, 4096, fmt, n, m, st, wu)
+            q.append(pick(layer_set_report(synth.QWEN25_7B, 4096, fmt, n, m, prep_ms, gemm_ms, peaks)))
+    out["qwen25_7b_m4096"] = q
+    a = argparse.Namespace(**vars(args))
+    a.steps, a.warmup, a.outlier_frac = 10, 3, 0.01
+    moe = run_moe(a, 4096)
+    out["qwen3_30b_a3b_moe_m4096"] = {k: moe[k] for k in ("tokens_per_s", "ms_per_step", "rows", "padded_rows", "ms")}
+    out["qwen3_30b_a3b_moe_m4096"]["grouped_gemm_frac"] = moe["gemm_roofline"]["frac"]
+    sw = run_sweep(a, [1, 16, 256, 2048, 16384])
+    out["down_proj_decode_prefill_sweep"] = {
+        "crossover_M": sw["crossover_M"],
+        "rows": [{k: r[k] for k in ("M", "prep_us", "gemm_us", "gemm_tflops", "gemm_bound", "gemm_roofline_frac")}
+                 for r in sw["rows"]]}
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return None
-    sample = oracle_sample(args.cpu_sample_tokens, args.cpu_sample_cols)
+    sample = oracle_sample(args.cpu_sample_tokens, args.ref_sample_cols)
     for _ in range(args.warmup):
         oracle_step(sample)
     times = []
@@ -572,14 +645,15 @@ def run_reference(args, world, rank):
     total = sum(times)
     value = tok * len(times) / total
     desc = (f"{args.cpu_sample_tokens} token(s) per step: full prep of each activation row and the first "
-            f"{args.cpu_sample_cols} output columns of each linear ({tok:.4f} token-equivalents per step)")
+            f"{args.ref_sample_cols} output columns of each linear ({tok:.4f} token-equivalents per step)")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32 prep, f64 GEMM",
             "data": "synthetic (same seeded generator)",
             "config": {"workload": workload_desc(args.tokens), "tokens": args.tokens, "fmt": "nvfp4",
                        "nm": f"{N_KEEP}:{M_GROUP}"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+                             "nproc": _host_cores()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
 
@@ -607,6 +681,8 @@ def run_case(args, world, rank, local):
         return run_fused(args, nums[0] if nums else 8192)
     if kind == "decode":
         return run_decode(args, nums[0] if nums else 1)
+    if kind == "sparse":
+        return run_sparse(args, nums[0] if nums else 8192)
     if kind == "qwen25":
         return run_qwen25(args, nums[0] if nums else 4096)
     if kind == "layerset":
@@ -726,10 +802,20 @@ def run_fused(args, M):
             "steps": args.steps}
 
 
-def time_layer_set(ls, M, fmt, n, m, steps, warmup):
+def prep_bytes_per_elem_sparse(fmt):
+    """Algorithmic bytes per element of the pair-wise 4:8 mode's preparation:
+    x (2), the kept half of the backbone codes (0.25), 4 metadata bits per 8
+    values (0.0625), one backbone scale per 32 (64) values, the residual's
+    codes (0.5) and one residual scale per 16 (32) values. NVFP4: 2.90625 B."""
+    blk = 16 if fmt == 0 else 32
+    return 2 + 0.25 + 0.0625 + 1.0 / (2 * blk) + 0.5 + 1.0 / blk
+
+
+def time_layer_set(ls, M, fmt, n, m, steps, warmup, sparse=False, affine=None):
     """Event timing of one layer set's step (its preps, then its linears) at
     M tokens with L2 flushed before every step: medians of the per-step prep
-    and GEMM milliseconds."""
+    and GEMM milliseconds. sparse: the pair-wise 4:8 mode (n, m ignored).
+    affine: None, "layer" (LayerNorm gamma/beta) or "rms" (RMSNorm weight)."""
     import sparsity_gemm_b200 as sq
     dev = torch.device("cuda", torch.cuda.current_device())
     preps = list(ls.preps)
@@ -739,9 +825,25 @@ def time_layer_set(ls, M, fmt, n, m, steps, warmup):
     qws = []
     for j, lin in enumerate(ls.linears):
         w = torch.from_numpy(synth.weights(1000 + j, lin.n_out, lin.k).view(np.float16)).to(dev)
-        qws.append(sq.quantize_weight(w, fmt))
+        qws.append(sq.quantize_weight_sparse(w, fmt) if sparse else sq.quantize_weight(w, fmt))
         del w
-    bufs = [sq.prepare(xs[i], None, None, EPS, n, m, fmt) for i in range(len(preps))]
+    lnp = []
+    for i, (_, k) in enumerate(preps):
+        g = b = None
+        if affine is not None:
+            g16, b16 = synth.ln_params(50 + i, k)
+            g = torch.from_numpy(g16.view(np.float16)).to(dev)
+            b = torch.from_numpy(b16.view(np.float16)).to(dev) if affine == "layer" else None
+        lnp.append((g, b))
+    norm = "rms" if affine == "rms" else "layer"
+
+    def prep_one(i, out=None):
+        g, b = lnp[i]
+        if sparse:
+            return sq.prepare_sparse(xs[i], g, b, EPS, fmt, out=out, norm=norm)
+        return sq.prepare(xs[i], g, b, EPS, n, m, fmt, out=out, norm=norm)
+
+    bufs = [prep_one(i) for i in range(len(preps))]
     outs = [torch.empty((M, lin.n_out), dtype=torch.float16, device=dev) for lin in ls.linears]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -749,7 +851,7 @@ def time_layer_set(ls, M, fmt, n, m, steps, warmup):
 
     def step(ev=None):
         for i in range(np_):
-            sq.prepare(xs[i], None, None, EPS, n, m, fmt, out=bufs[i])
+            prep_one(i, bufs[i])
         if ev is not None:
             ev[1].record(stream)
         for j, lin in enumerate(ls.linears):
@@ -776,16 +878,43 @@ def time_layer_set(ls, M, fmt, n, m, steps, warmup):
     return prep_ms, gemm_ms
 
 
-def layer_set_report(ls, M, fmt, n, m, prep_ms, gemm_ms, peaks):
+def layer_set_report(ls, M, fmt, n, m, prep_ms, gemm_ms, peaks, sparse=False):
+    """Throughput and roofline figures of one layer-set timing. The GEMM's
+    algorithmic FLOPs are 2 M N K (1 + n/m); executed FLOPs count what the
+    tensor cores run in dense-MMA units: both paths dense (4 M N K) in the
+    default mode, half of K on the backbone in the pair-wise mode (3 M N K,
+    equal to the algorithmic count)."""
+    if sparse:
+        n, m = 4, 8
     flops = sum(2.0 * M * l.n_out * l.k * (1.0 + n / m) for l in ls.linears)
-    pbytes = sum(prep_bytes_per_elem(fmt, n, m) * M * k for _, k in ls.preps)
+    executed = sum((3.0 if sparse else 4.0) * M * l.n_out * l.k for l in ls.linears)
+    per_elem = prep_bytes_per_elem_sparse(fmt) if sparse else prep_bytes_per_elem(fmt, n, m)
+    pbytes = sum(per_elem * M * k for _, k in ls.preps)
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     gemm_tf = flops / (gemm_ms / 1e3) / 1e12
+    exec_tf = executed / (gemm_ms / 1e3) / 1e12
     prep_gbs = pbytes / (prep_ms / 1e3) / 1e9
-    return {"tokens": M, "fmt": "nvfp4" if fmt == 0 else "mxfp4", "nm": f"{n}:{m}",
+    return {"tokens": M, "fmt": "nvfp4" if fmt == 0 else "mxfp4", "nm": "pair-wise 4:8" if sparse else f"{n}:{m}",
+            "backbone_mma": "tcgen05.mma.sp on the K-compacted backbone" if sparse else "dense MMA, zeros off the mask",
             "tokens_per_s": M / ((prep_ms + gemm_ms) / 1e3), "ms_per_step": prep_ms + gemm_ms,
             "prep_ms": prep_ms, "gemm_ms": gemm_ms, "gemm_tflops": gemm_tf, "gemm_frac": gemm_tf / fp4_peak,
-            "prep_gbs": prep_gbs, "prep_frac": prep_gbs / peaks["hbm_gbs"]}
+            "gemm_executed_tflops": exec_tf, "gemm_executed_frac": exec_tf / fp4_peak,
+            "prep_gbs": prep_gbs, "prep_frac": prep_gbs / peaks["hbm_gbs"], "prep_bytes_per_elem": per_elem}
+
+
+def run_sparse(args, M):
+    """The Llama-3.1-8B layer set at M tokens (8192 by default), NVFP4, in the
+    default mode (element-wise 2:4, dense backbone MMA) and the pair-wise 4:8
+    mode (structured-sparse backbone MMA), and MXFP4 in the pair-wise mode."""
+    peaks, peak_src = load_peaks()
+    rows = []
+    for fmt, sparse in ((0, False), (0, True), (1, True)):
+        prep_ms, gemm_ms = time_layer_set(synth.LLAMA31_8B, M, fmt, N_KEEP, M_GROUP, args.steps, args.warmup,
+                                          sparse=sparse)
+        rows.append(layer_set_report(synth.LLAMA31_8B, M, fmt, N_KEEP, M_GROUP, prep_ms, gemm_ms, peaks, sparse))
+    return {"case": args.case, "workload": workload_desc(M), "rows": rows,
+            "peak_source": f"{peak_src}: FP4 = bf16 {peaks['bf16_tflops']} TF/s x {FP4_OVER_BF16}, "
+            f"HBM {peaks['hbm_gbs']} GB/s", "l2": "flushed (256 MB write) before every step", "steps": args.steps}
 
 
 def run_qwen25(args, M):
@@ -889,7 +1018,7 @@ def run_decode(args, M):
             "l2": "flushed (256 MB write) before every step", "steps": args.steps}
 
 
-def run_sweep(args):
+def run_sweep(args, ms=None):
     """Decode-vs-prefill sweep on the Llama-3.1-8B down projection (14336 ->
     4096), NVFP4 2:4: for M = 1, 2, 4, ..., 16384 the prep and the dual GEMM
     are timed separately (CUDA events, L2 flushed before every call, median
@@ -910,8 +1039,7 @@ def run_sweep(args):
     stream = torch.cuda.current_stream()
     w_bytes = N * K * (0.5 + 1.0 / 16)
     rows = []
-    for lg in range(15):
-        M = 1 << lg
+    for M in (ms or [1 << lg for lg in range(15)]):
         x = torch.from_numpy(synth.activations_student(6, M, K, outlier_frac=args.outlier_frac).view(np.float16)).to(dev)
         p = sq.prepare(x, None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4)
         out = torch.empty((M, N), dtype=torch.float16, device=dev)

@@ -19,12 +19,28 @@ NVFP4, MXFP4 = 0, 1
 BLOCK = {NVFP4: 16, MXFP4: 32}
 
 _lib = None
+_omp = False
+
+
+def use_openmp(on: bool) -> None:
+    """Selects the OpenMP build of the same oracle source (independent rows
+    and output elements split across threads; identical results) for the
+    calls that follow. Default: the single-threaded build."""
+    global _lib, _omp
+    if bool(on) != _omp:
+        _omp = bool(on)
+        _lib = None
+
+
+def threads() -> int:
+    """Threads the current build's parallel loops use (1: the plain build)."""
+    return int(lib().oracle_threads())
 
 
 def lib():
     global _lib
     if _lib is None:
-        _lib = C.CDLL(_build.build())
+        _lib = C.CDLL(_build.build(omp=_omp))
         _declare(_lib)
     return _lib
 
@@ -35,6 +51,7 @@ def _p(a):
 
 def _declare(L):
     vp, i64, f32, i32 = C.c_void_p, C.c_int64, C.c_float, C.c_int
+    L.oracle_threads.restype = i32
     L.oracle_half_to_double.argtypes = [C.c_uint16]
     L.oracle_half_to_double.restype = C.c_double
     L.oracle_u128_to_double.argtypes = [C.c_uint64, C.c_uint64]

@@ -33,12 +33,25 @@
 #include <math.h>
 #include <stdint.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 typedef unsigned __int128 u128;
 typedef __int128 i128;
 
 #define FMT_NVFP4 0
 #define FMT_MXFP4 1
+
+/* Threads the row and output-element loops use: 1 in the plain build. */
+int oracle_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
 
 /* ------------------------------------------------------------------ */
 /* fp16 decode (IEEE-754 binary16), exact in binary64.                 */
@@ -99,6 +112,7 @@ double oracle_u128_to_double(uint64_t hi, uint64_t lo)
 void oracle_ln_stats(const uint16_t *x, int64_t rows, int64_t k, float eps,
                      float *mu, float *rstd)
 {
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
         int64_t s1 = 0;
         u128 s2 = 0;
@@ -298,6 +312,7 @@ void oracle_quantize(const float *v, int64_t rows, int64_t k, int fmt, float s_t
                      uint8_t *codes, uint8_t *scales)
 {
     int blk = fmt == FMT_NVFP4 ? 16 : 32;
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r)
         quantize_row(v + r * k, k, fmt, s_t, codes + r * k, scales + r * (k / blk));
 }
@@ -447,6 +462,10 @@ void oracle_linear(const uint8_t *s_codes, const uint8_t *s_scales,
                    double *out, double *bound)
 {
     double ts = (double)s_t * (double)s_tw;
+    /* Output elements are independent: built with OpenMP (the all-cores
+     * baseline build), they are split across threads; each is still the
+     * same sequential sum, so the results are identical. */
+#pragma omp parallel for collapse(2) schedule(static)
     for (int64_t i = 0; i < rows; ++i)
         for (int64_t j = 0; j < n_out; ++j) {
             double acc = 0.0, mag = 0.0;
@@ -575,6 +594,7 @@ void oracle_linear_blk(const uint8_t *s_codes, const uint8_t *s_scales, int blk_
                        double *out, double *bound)
 {
     double ts = (double)s_t * (double)s_tw;
+#pragma omp parallel for collapse(2) schedule(static)
     for (int64_t i = 0; i < rows; ++i)
         for (int64_t j = 0; j < n_out; ++j) {
             double acc = 0.0, mag = 0.0;
