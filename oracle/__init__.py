@@ -78,6 +78,9 @@ def _declare(L):
     L.oracle_quantize_weight.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp]
     L.oracle_linear.argtypes = [vp, vp, vp, vp, f32, vp, vp, f32, i64, i64, i64, i32, vp, vp]
     L.oracle_mask_pairs48.argtypes = [vp, i64, i64, vp, vp]
+    L.oracle_double_to_half_rn.argtypes = [C.c_double]
+    L.oracle_double_to_half_rn.restype = C.c_uint16
+    L.oracle_add_fp16.argtypes = [vp, vp, i64, vp]
     L.oracle_quantize_blk.argtypes = [vp, i64, i64, i32, i32, f32, vp, vp]
     L.oracle_prepare_sparse.argtypes = [vp, i64, i64, vp, vp, f32, i32, i32] + [vp] * 14
     L.oracle_quantize_weight_blk.argtypes = [vp, i64, i64, i32, i32, vp, vp, vp, vp]
@@ -459,3 +462,22 @@ def linear_sparse(p: Prepared, qw: QWeight, rows=None):
     sel = slice(None) if rows is None else rows
     return linear_blk(p.s_codes[sel], p.s_scales[sel], SPARSE_BLOCK[p.fmt], p.r_codes[sel], p.r_scales[sel],
                       BLOCK[p.fmt], p.s_t, qw.codes, qw.scales, SPARSE_BLOCK[p.fmt], qw.s_tw, p.fmt)
+
+
+# --------------------------------------------------------------------------
+# Residual add feeding the preparation operator: x = RN16(h + d) (IEEE
+# binary16 addition; in pre-norm transformers the normalization's input is
+# the residual stream after this add).
+
+
+def double_to_half(v: float) -> int:
+    """Nearest binary16 (ties to even) of a binary64 value, as bits."""
+    return int(lib().oracle_double_to_half_rn(float(v)))
+
+
+def add_fp16(h, d) -> np.ndarray:
+    h, d = _u16(h), _u16(d)
+    assert h.shape == d.shape
+    x = np.empty(h.shape, np.uint16)
+    lib().oracle_add_fp16(_p(h), _p(d), h.size, _p(x))
+    return x

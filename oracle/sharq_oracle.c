@@ -611,3 +611,47 @@ void oracle_linear_blk(const uint8_t *s_codes, const uint8_t *s_scales, int blk_
                 bound[i * n_out + j] = ts * mag;
         }
 }
+
+/* ------------------------------------------------------------------ */
+/* Residual add feeding the preparation operator (reading: in pre-norm  */
+/* transformers the normalization's input is the residual stream after  */
+/* the add x = h + d; the abstract's fused operator starts from x. The  */
+/* add is IEEE binary16 addition: x = RN16(h + d), the exact sum         */
+/* (exact in binary64) rounded to nearest even binary16, overflowing to  */
+/* +-inf).                                                               */
+
+/* Nearest binary16 (ties to even) of a binary64 value, as bits. */
+uint16_t oracle_double_to_half_rn(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0)
+        return sign;
+    /* a = q * 2^-24 in the subnormal range and below: the grid 2^-24 */
+    int e;
+    frexp(a, &e); /* a in [2^(e-1), 2^e) */
+    int ulp_exp = e - 1 - 10; /* spacing of binary16 at this binade */
+    if (ulp_exp < -24)
+        ulp_exp = -24;
+    double q = ldexp(a, -ulp_exp); /* a in units of the spacing */
+    double f = floor(q);
+    double rem = q - f;
+    if (rem > 0.5 || (rem == 0.5 && fmod(f, 2.0) != 0.0))
+        f += 1.0;
+    double r = ldexp(f, ulp_exp);
+    if (r > 65504.0)
+        return sign | 0x7C00; /* overflow: infinity */
+    /* encode r exactly */
+    if (r < ldexp(1.0, -14))
+        return sign | (uint16_t)ldexp(r, 24); /* subnormal (or the smallest normal reached by rounding) */
+    frexp(r, &e);
+    int be = e - 1 + 15;
+    uint16_t mant = (uint16_t)(ldexp(r, -(e - 1)) * 1024.0 - 1024.0);
+    return sign | (uint16_t)(be << 10) | mant;
+}
+
+void oracle_add_fp16(const uint16_t *h, const uint16_t *d, int64_t count, uint16_t *x)
+{
+    for (int64_t i = 0; i < count; ++i)
+        x[i] = oracle_double_to_half_rn(oracle_half_to_double(h[i]) + oracle_half_to_double(d[i]));
+}
