@@ -681,6 +681,8 @@ def run_case(args, world, rank, local):
         return run_fused(args, nums[0] if nums else 8192)
     if kind == "decode":
         return run_decode(args, nums[0] if nums else 1)
+    if kind == "add_prep":
+        return run_add_prep(args, *(nums[:2] if len(nums) >= 2 else [8192, 4096]))
     if kind == "sparse":
         return run_sparse(args, nums[0] if nums else 8192)
     if kind == "qwen25":
@@ -900,6 +902,57 @@ def layer_set_report(ls, M, fmt, n, m, prep_ms, gemm_ms, peaks, sparse=False):
             "prep_ms": prep_ms, "gemm_ms": gemm_ms, "gemm_tflops": gemm_tf, "gemm_frac": gemm_tf / fp4_peak,
             "gemm_executed_tflops": exec_tf, "gemm_executed_frac": exec_tf / fp4_peak,
             "prep_gbs": prep_gbs, "prep_frac": prep_gbs / peaks["hbm_gbs"], "prep_bytes_per_elem": per_elem}
+
+
+def run_add_prep(args, M, K):
+    """The residual add x = h + d followed by the preparation of x, fused
+    (sharq_prepare_add: x's statistics taken in the add's pass, so the encode
+    pass is the only other read of x) and unfused (the add, then
+    sharq_prepare, which reads x twice). The unfused add is torch's fp16 add
+    (context for the comparison only; the library has no standalone add).
+    Bytes: the add moves 6 B per element (h, d in, x out); the preparation's
+    algorithmic 3.0 B per element counts its own read of x."""
+    import sparsity_gemm_b200 as sq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks, peak_src = load_peaks()
+    h = torch.from_numpy(synth.activations_student(0, M, K).view(np.float16)).to(dev)
+    d = torch.from_numpy(synth.activations_student(1, M, K, outlier_frac=0.0).view(np.float16)).to(dev)
+    x = torch.empty_like(h)
+    buf = sq.prepare(h, None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fused():
+        sq.prepare_add(h, d, None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4, x_out=x, out=buf)
+
+    def unfused():
+        torch.add(h, d, out=x)
+        sq.prepare(x, None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4, out=buf)
+
+    res = {}
+    for name, op in (("fused", fused), ("unfused", unfused)):
+        for _ in range(args.warmup):
+            flush.zero_()
+            op()
+        ms = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            op()
+            b.record(stream)
+            b.synchronize()
+            ms.append(a.elapsed_time(b))
+        t = statistics.median(ms) / 1e3
+        nbytes = (6.0 + PREP_BYTES_PER_ELEM - 2.0) * M * K  # add (6) + prep without its own read of x
+        res[name] = {"us": t * 1e6, "algorithmic_gbs": nbytes / t / 1e9, "frac": nbytes / t / 1e9 / peaks["hbm_gbs"]}
+    st = sq.get_last_error()
+    if st != sq.OK:
+        raise RuntimeError(sq.status_name(st))
+    return {"case": args.case, "M": M, "K": K, "fmt": "nvfp4", "nm": f"{N_KEEP}:{M_GROUP}", **res,
+            "bytes_per_elem": 6.0 + PREP_BYTES_PER_ELEM - 2.0,
+            "bytes_count": "add: h, d read and x written (6); preparation outputs (1.0): 7.0 B per element",
+            "peak_source": peak_src, "l2": "flushed (256 MB write) before every call", "steps": args.steps}
 
 
 def run_sparse(args, M):

@@ -211,6 +211,31 @@ sharq_status sharq_prepare_rms(const void *x_dev, int64_t m_tok, int64_t k, cons
                                void *stream);
 
 /*
+ * The preparation operator fused with the operation that produces its input.
+ * SharQ, Abstract: one fused operator absorbs the layer normalization; in a
+ * pre-norm transformer the normalization's input is the residual stream
+ * right after the add x = h + d (h the residual stream, d the output of the
+ * previous attention or MLP block). This call performs that add and takes
+ * x's normalization statistics and tensor amax in the same pass, so that
+ * the encode pass is the only other read of x (sharq_prepare on a stored x
+ * reads it twice):
+ *   x_out[i] = RN16(h[i] + d[i])   (binary16 addition, round to nearest even;
+ *                                   a sum beyond 65504 gives +-inf, which the
+ *                                   preparation's finiteness precondition
+ *                                   then excludes)
+ * then exactly what sharq_prepare (norm = 0) or sharq_prepare_rms (norm = 1,
+ * ln_b NULL) computes on x_out, bit for bit.
+ *   h_dev, d_dev  fp16 [m_tok][k], 16-byte aligned.
+ *   x_out_dev     fp16 [m_tok][k]: may be h_dev itself (the residual stream
+ *                 updated in place); must not otherwise overlap h or d.
+ * Other arguments and preconditions as sharq_prepare; prep_bytes >=
+ * sharq_prep_bytes(m_tok, k, n, m, fmt).
+ */
+sharq_status sharq_prepare_add(const void *h_dev, const void *d_dev, void *x_out_dev, int64_t m_tok, int64_t k,
+                               const void *ln_w_dev, const void *ln_b_dev, float eps, int norm, int n, int m, int fmt,
+                               void *prep_dev, size_t prep_bytes, sharq_prep *prep_out, void *stream);
+
+/*
  * Preparation operator for callers that cannot allocate device memory.
  * (An interface addition: the SharQ paper has no counterpart.)
  *

@@ -95,6 +95,8 @@ def lib():
         L.sharq_weight_tensor_scales.argtypes = [C.POINTER(SharqWQ), vp, vp]
         L.sharq_prepare_grouped.argtypes = [vp, i64, i64, vp, i64, vp, vp, f32, i32, i32, i32, i32, vp, sz,
                                             C.POINTER(SharqPrep), vp]
+        L.sharq_prepare_add.argtypes = [vp, vp, vp, i64, i64, vp, vp, f32, i32, i32, i32, i32, vp, sz,
+                                        C.POINTER(SharqPrep), vp]
         L.sharq_prep_bytes_sparse.argtypes = [i64, i64, i32]
         L.sharq_prep_bytes_sparse.restype = sz
         L.sharq_prepare_sparse.argtypes = [vp, i64, i64, vp, vp, f32, i32, i32, vp, sz, C.POINTER(SharqPrep), vp]
@@ -108,7 +110,7 @@ def lib():
                      "sharq_weight_export", "sharq_get_last_error", "sharq_quantize_weight_grouped",
                      "sharq_gather_rows", "sharq_linear_grouped", "sharq_prepare_rms",
                      "sharq_quantize_weight_fused", "sharq_linear_bias", "sharq_weight_tensor_scales",
-                     "sharq_prepare_grouped", "sharq_prepare_sparse", "sharq_quantize_weight_sparse"):
+                     "sharq_prepare_grouped", "sharq_prepare_sparse", "sharq_quantize_weight_sparse", "sharq_prepare_add"):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -301,6 +303,43 @@ def weight_tensor_scales(qw: QuantizedWeight, stream=None) -> np.ndarray:
     _check(lib().sharq_weight_tensor_scales(C.byref(qw.desc), out.ctypes.data_as(C.c_void_p), _stream(stream)),
            "sharq_weight_tensor_scales")
     return out
+
+
+def prepare_add(h: torch.Tensor, d: torch.Tensor, ln_w=None, ln_b=None, eps: float = 1e-5, n: int = 2, m: int = 4,
+                fmt: int = NVFP4, x_out: torch.Tensor | None = None, out: Prepared | None = None, stream=None,
+                norm: str = "layer"):
+    """Residual add fused with the preparation: x = RN16(h + d) (fp16 [m_tok,
+    k], CUDA) is written to x_out (a new tensor if None; may be h itself) and
+    prepared as prepare(x) would, with x's statistics taken in the add's pass.
+    Returns (x_out, Prepared)."""
+    _require(norm in ("layer", "rms") and (norm == "layer" or ln_b is None),
+             'norm must be "layer" or "rms" (RMSNorm takes no ln_b)')
+    _fp16_matrix(h, "h")
+    _fp16_matrix(d, "d")
+    _require(h.shape == d.shape, "h and d must have the same shape")
+    if x_out is None:
+        x_out = torch.empty_like(h)
+    _fp16_matrix(x_out, "x_out")
+    _require(x_out.shape == h.shape, "x_out must have the shape of h")
+    for t, name in ((ln_w, "ln_w"), (ln_b, "ln_b")):
+        if t is not None:
+            _fp16_matrix(t.view(-1) if t.is_contiguous() else t, name, 1)
+            _require(t.numel() == h.shape[1], f"{name} must have {h.shape[1]} elements")
+    m_tok, k = h.shape
+    nbytes = prep_bytes(m_tok, k, n, m, fmt)
+    if nbytes == 0:
+        raise SharqError(ERR_INVALID_ARG, f"prep shape {tuple(h.shape)} {n}:{m} fmt {fmt}")
+    if out is None or out.buf.numel() < nbytes:
+        buf = _device_buffer(nbytes, h.device)
+    else:
+        buf = out.buf
+        _cuda_here(buf, "out.buf")
+    desc = SharqPrep()
+    p = (lambda t: _ptr(t) if m_tok > 0 else None)
+    _check(lib().sharq_prepare_add(p(h), p(d), p(x_out), m_tok, k, _ptr(ln_w), _ptr(ln_b), float(eps),
+                                   1 if norm == "rms" else 0, n, m, fmt, _ptr(buf), buf.numel(), C.byref(desc),
+                                   _stream(stream)), "sharq_prepare_add")
+    return x_out, Prepared(buf, desc)
 
 
 def prepare_sparse(x: torch.Tensor, ln_w=None, ln_b=None, eps: float = 1e-5, fmt: int = NVFP4,

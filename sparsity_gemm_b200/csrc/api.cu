@@ -290,6 +290,37 @@ sharq_status sharq_prepare_rms(const void *x_dev, int64_t m_tok, int64_t k, cons
     return prepare_norm(x_dev, m_tok, k, w_dev, nullptr, eps, n, m, fmt, prep_dev, prep_bytes, prep_out, stream, 1);
 }
 
+sharq_status sharq_prepare_add(const void *h_dev, const void *d_dev, void *x_out_dev, int64_t m_tok, int64_t k,
+                               const void *ln_w_dev, const void *ln_b_dev, float eps, int norm, int n, int m, int fmt,
+                               void *prep_dev, size_t prep_bytes, sharq_prep *prep_out, void *stream) {
+    g_last_launches = 0;
+    const size_t need = sharq_prep_bytes(m_tok, k, n, m, fmt);
+    if (!need || !prep_dev || !prep_out || prep_bytes < need) return SHARQ_ERR_INVALID_ARG;
+    if ((norm != 0 && norm != 1) || (norm == 1 && ln_b_dev)) return SHARQ_ERR_INVALID_ARG;
+    if (m_tok > 0 && (!h_dev || !d_dev || !x_out_dev)) return SHARQ_ERR_INVALID_ARG;
+    if (!(eps > 0.0f) || eps != eps || eps > 3.0e38f) return SHARQ_ERR_INVALID_ARG;
+    if ((h_dev && !aligned(h_dev, 16)) || (d_dev && !aligned(d_dev, 16)) || (x_out_dev && !aligned(x_out_dev, 16)) ||
+        !aligned(prep_dev, sq::kAlign) || (ln_w_dev && !aligned(ln_w_dev, 16)) || (ln_b_dev && !aligned(ln_b_dev, 16)))
+        return SHARQ_ERR_INVALID_ARG;
+    // x_out may be h itself (the residual stream updated in place), but must
+    // not overlap d or h partly
+    const uintptr_t bytes = (uintptr_t)(m_tok * k * 2);
+    auto overlap = [bytes](const void *a, const void *b) {
+        const uintptr_t pa = reinterpret_cast<uintptr_t>(a), pb = reinterpret_cast<uintptr_t>(b);
+        return pa < pb + bytes && pb < pa + bytes;
+    };
+    if (m_tok > 0 && (overlap(x_out_dev, d_dev) || (x_out_dev != h_dev && overlap(x_out_dev, h_dev))))
+        return SHARQ_ERR_INVALID_ARG;
+    sq::LaunchCtx ctx;
+    sharq_status st = make_ctx(stream, ctx);
+    if (st != SHARQ_OK) return st;
+    fill_prep(prep_out, prep_dev, m_tok, k, n, m, fmt);
+    st = sq::launch_prepare_add(ctx, *prep_out, h_dev, d_dev, x_out_dev, ln_w_dev, ln_b_dev, eps, norm);
+    if (st == SHARQ_OK && cudaGetLastError() != cudaSuccess) st = SHARQ_ERR_CUDA;
+    g_last_launches = ctx.launches;
+    return st;
+}
+
 size_t sharq_prep_bytes_sparse(int64_t m_tok, int64_t k, int fmt) {
     if (m_tok < 0 || m_tok > (1ll << 30) || !k_ok(k) || !fmt_ok(fmt)) return 0;
     return (size_t)sq::prep_layout_sparse(m_tok, k, fmt).total;

@@ -712,6 +712,131 @@ ln_stats_long_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict_
     }
 }
 
+// Residual add fused with the statistics pass: x = RN16(h + d) (binary16
+// addition, the residual stream update of a pre-norm layer) is written out
+// and, in the same pass, x's exact LayerNorm / RMSNorm statistics and the
+// row's amax|X_ln| are taken as in ln_stats_long_kernel (FAST: certified
+// binary64 sums with the exact fallback, for rows longer than 2048
+// elements; otherwise the exact integer sums). One warp per row, the warps
+// of a persistent grid taking rows with the grid stride; each lane adds and
+// stores the 16-byte vectors lane, lane + 32, ... of its row, so the
+// fallback and the affine amax sweep re-read only what the same lane wrote.
+// The encode pass then reads x once more (the only other read of x).
+template <bool AFFINE, bool RMS, bool FAST>
+__global__ void __launch_bounds__(kStatsThreads)
+add_stats_kernel(const uint16_t *h, const uint16_t *d, uint16_t *x_out,
+                 const uint16_t *__restrict__ gamma, const uint16_t *__restrict__ beta, float eps, int64_t k,
+                 int64_t m_tok, float2 *__restrict__ stats, unsigned *__restrict__ amax_word) {
+    constexpr int W = kStatsThreads / 32;
+    constexpr int V = 4;  // vectors per lane in flight
+    __shared__ float red_max[W];
+    griddep_launch();
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nvec = (int)(k / 8);
+    const int64_t nwarps = (int64_t)gridDim.x * W;
+    float amax = 0.0f;
+    for (int64_t row = (int64_t)blockIdx.x * W + warp; row < m_tok; row += nwarps) {
+        const uint4 *hr = reinterpret_cast<const uint4 *>(h + row * k);
+        const uint4 *dr = reinterpret_cast<const uint4 *>(d + row * k);
+        uint4 *xr = reinterpret_cast<uint4 *>(x_out + row * k);
+        LaneSums l = {};
+        FastLane f = {0.0, 0.0, 0.0};
+        uint32_t mx = 0xFC00FC00u, mn = 0x7C007C00u;  // (-inf, -inf), (+inf, +inf) as half2
+        for (int c0 = lane; c0 < nvec; c0 += 32 * V) {
+            uint4 hv[V], dv[V];
+#pragma unroll
+            for (int j = 0; j < V; ++j)
+                if (c0 + 32 * j < nvec) {
+                    hv[j] = __ldcs(hr + c0 + 32 * j);
+                    dv[j] = __ldcs(dr + c0 + 32 * j);
+                }
+#pragma unroll
+            for (int j = 0; j < V; ++j) {
+                if (c0 + 32 * j >= nvec) break;
+                uint4 xv;
+                asm("add.rn.f16x2 %0, %1, %2;" : "=r"(xv.x) : "r"(hv[j].x), "r"(dv[j].x));
+                asm("add.rn.f16x2 %0, %1, %2;" : "=r"(xv.y) : "r"(hv[j].y), "r"(dv[j].y));
+                asm("add.rn.f16x2 %0, %1, %2;" : "=r"(xv.z) : "r"(hv[j].z), "r"(dv[j].z));
+                asm("add.rn.f16x2 %0, %1, %2;" : "=r"(xv.w) : "r"(hv[j].w), "r"(dv[j].w));
+                xr[c0 + 32 * j] = xv;
+                const uint32_t w4[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (FAST) fast_pair(w4[q], f);
+                    else accum_pair(w4[q], l);
+                    if (!AFFINE) {
+                        asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(w4[q]));
+                        asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(w4[q]));
+                    }
+                }
+            }
+        }
+        if (!AFFINE) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const uint32_t omx = __shfl_xor_sync(0xFFFFFFFFu, mx, o), omn = __shfl_xor_sync(0xFFFFFFFFu, mn, o);
+                asm("max.f16x2 %0, %0, %1;" : "+r"(mx) : "r"(omx));
+                asm("min.f16x2 %0, %0, %1;" : "+r"(mn) : "r"(omn));
+            }
+        }
+        float2 st;
+        if (FAST) {
+            int64_t s1 = __double2ll_rn(__dmul_rn(f.s1, 16777216.0));
+            double s2 = __dadd_rn(f.s2a, f.s2b);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
+                s2 = __dadd_rn(s2, __shfl_xor_sync(0xFFFFFFFFu, s2, o));
+            }
+            if (!certified_stats(s1, s2, k, eps, RMS, st))  // the same on every lane
+                st = exact_row_stats<RMS>(xr, nvec, lane, k, eps);
+        } else {
+            ExactSums e = widen(l);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                e.hi += __shfl_xor_sync(0xFFFFFFFFu, e.hi, o);
+                e.lo += __shfl_xor_sync(0xFFFFFFFFu, e.lo, o);
+                e.hh += __shfl_xor_sync(0xFFFFFFFFu, e.hh, o);
+                e.hl += __shfl_xor_sync(0xFFFFFFFFu, e.hl, o);
+                e.ll += __shfl_xor_sync(0xFFFFFFFFu, e.ll, o);
+            }
+            st = RMS ? finish_stats_rms(e, k, eps) : finish_stats(e, k, eps);
+        }
+        if (lane == 0) stats[row] = st;
+        if (!AFFINE) {
+            const float xmax = fmaxf(h2f((uint16_t)mx), h2f((uint16_t)(mx >> 16)));
+            const float xmin = fminf(h2f((uint16_t)mn), h2f((uint16_t)(mn >> 16)));
+            amax = fmaxf(amax, fmaxf(fabsf(__fmul_rn(__fsub_rn(xmax, st.x), st.y)),
+                                     fabsf(__fmul_rn(__fsub_rn(xmin, st.x), st.y))));
+        } else {
+            const bool has_g = gamma != nullptr, has_b = beta != nullptr;
+            for (int cc = lane; cc < nvec; cc += 32) {
+                const uint4 v = xr[cc];
+                const uint4 g = has_g ? __ldg(reinterpret_cast<const uint4 *>(gamma) + cc) : make_uint4(0, 0, 0, 0);
+                const uint4 bb = has_b ? __ldg(reinterpret_cast<const uint4 *>(beta) + cc) : make_uint4(0, 0, 0, 0);
+                const uint32_t xv[4] = {v.x, v.y, v.z, v.w}, gv[4] = {g.x, g.y, g.z, g.w},
+                               bv[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+                        amax = fmaxf(amax, fabsf(ln_apply(h2f((uint16_t)(xv[q] >> (16 * hh))), st.x, st.y, has_g,
+                                                          h2f((uint16_t)(gv[q] >> (16 * hh))), has_b,
+                                                          h2f((uint16_t)(bv[q] >> (16 * hh))))));
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    if (lane == 0) red_max[warp] = amax;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float a = 0.0f;
+        for (int w = 0; w < W; ++w) a = fmaxf(a, red_max[w]);
+        atomicMax(amax_word, __float_as_uint(a));
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Encode pass.
 
@@ -2321,6 +2446,64 @@ sharq_status launch_prepare_sparse(LaunchCtx &ctx, const sharq_prep &P, const vo
     const int64_t warps = P.m_tok * chunks > 0 ? P.m_tok * chunks : 1;
     const int64_t blocks = encode_grid(fn, ctx.num_sms, warps * 32);
     EncodeArgs ea{(const uint16_t *)x, (const uint16_t *)gamma, (const uint16_t *)beta, stats, P.m_tok, P.k,
+                  P.meta_row_bytes, P.k / (P.fmt == kFmtNV ? 16 : 32), P.n, (uint8_t *)P.s_codes,
+                  (uint8_t *)P.r_codes, (uint8_t *)P.s_scales, (uint8_t *)P.r_scales, (uint8_t *)P.meta};
+    const unsigned *aw = words;
+    float *sto = P.tensor_scale;
+    int64_t sf_rows = P.sf_rows;
+    void *args[] = {&ea, &aw, &sto, &sf_rows};
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)blocks, 1, 1);
+    cfg.blockDim = dim3(kEncodeThreads, 1, 1);
+    cfg.stream = ctx.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = P.m_tok > 0 ? 1 : 0;
+    SQ_CUDA_TRY(cudaLaunchKernelExC(&cfg, fn, args));
+    ctx.launches++;
+    return SHARQ_OK;
+}
+
+// Residual add and preparation: x_out = RN16(h + d) with its statistics in
+// one pass, then the encode pass over x_out (a programmatic dependent).
+sharq_status launch_prepare_add(LaunchCtx &ctx, const sharq_prep &P, const void *h, const void *d, void *x_out,
+                                const void *gamma, const void *beta, float eps, int norm) {
+    unsigned *words = reinterpret_cast<unsigned *>(P.tensor_scale) - 1;  // [0] amax bits, [1] s_t
+    SQ_CUDA_TRY(cudaMemsetAsync(words, 0, sizeof(unsigned), ctx.stream));
+    const bool meta_atomic = ((kUnit / P.m) * P.n * idx_bits(P.m)) % 8 != 0;
+    if (meta_atomic && P.m_tok > 0)
+        SQ_CUDA_TRY(cudaMemsetAsync(P.meta, 0, (size_t)(P.m_tok * P.meta_row_bytes), ctx.stream));
+    float2 *stats = reinterpret_cast<float2 *>(P.scratch);
+    const bool affine = gamma != nullptr || beta != nullptr;
+    if (P.m_tok > 0) {
+        const bool fast = P.k > 2048;
+        void *fn;
+        if (norm)
+            fn = affine ? (fast ? (void *)add_stats_kernel<true, true, true> : (void *)add_stats_kernel<true, true, false>)
+                        : (fast ? (void *)add_stats_kernel<false, true, true> : (void *)add_stats_kernel<false, true, false>);
+        else
+            fn = affine ? (fast ? (void *)add_stats_kernel<true, false, true> : (void *)add_stats_kernel<true, false, false>)
+                        : (fast ? (void *)add_stats_kernel<false, false, true> : (void *)add_stats_kernel<false, false, false>);
+        const int64_t need = (P.m_tok + (kStatsThreads / 32) - 1) / (kStatsThreads / 32);
+        const unsigned grid = (unsigned)resident_grid(fn, ctx.num_sms, kStatsThreads, 0, need);
+        const uint16_t *hh = (const uint16_t *)h, *dd = (const uint16_t *)d, *gg = (const uint16_t *)gamma,
+                       *bb = (const uint16_t *)beta;
+        uint16_t *xo = (uint16_t *)x_out;
+        float e = eps;
+        int64_t kk = P.k, mt = P.m_tok;
+        void *args[] = {&hh, &dd, &xo, &gg, &bb, &e, &kk, &mt, &stats, &words};
+        SQ_CUDA_TRY(cudaLaunchKernel(fn, dim3(grid), dim3(kStatsThreads), args, 0, ctx.stream));
+        ctx.launches++;
+    }
+    void *fn = P.fmt == kFmtNV ? (affine ? encode_rows_fn<kFmtNV, true>(P.m, P.n) : encode_rows_fn<kFmtNV, false>(P.m, P.n))
+                               : (affine ? encode_rows_fn<kFmtMX, true>(P.m, P.n) : encode_rows_fn<kFmtMX, false>(P.m, P.n));
+    const int64_t chunks = (P.k / kUnit + 31) / 32;
+    const int64_t warps = P.m_tok * chunks > 0 ? P.m_tok * chunks : 1;
+    const int64_t blocks = encode_grid(fn, ctx.num_sms, warps * 32);
+    EncodeArgs ea{(const uint16_t *)x_out, (const uint16_t *)gamma, (const uint16_t *)beta, stats, P.m_tok, P.k,
                   P.meta_row_bytes, P.k / (P.fmt == kFmtNV ? 16 : 32), P.n, (uint8_t *)P.s_codes,
                   (uint8_t *)P.r_codes, (uint8_t *)P.s_scales, (uint8_t *)P.r_scales, (uint8_t *)P.meta};
     const unsigned *aw = words;

@@ -21,6 +21,9 @@ sharq_status launch_prepare(LaunchCtx &ctx, const sharq_prep &P, const void *x, 
 // The pair-wise 4:8 mode (P from prep_layout_sparse).
 sharq_status launch_prepare_sparse(LaunchCtx &ctx, const sharq_prep &P, const void *x, const void *gamma,
                                    const void *beta, float eps, int norm);
+// x_out = RN16(h + d), then the preparation of x_out (P from prep_layout).
+sharq_status launch_prepare_add(LaunchCtx &ctx, const sharq_prep &P, const void *h, const void *d, void *x_out,
+                                const void *gamma, const void *beta, float eps, int norm);
 sharq_status launch_prepare_grouped(LaunchCtx &ctx, const sharq_prep &P, const void *x, int64_t rows,
                                     const int32_t *offsets, int32_t groups, const void *gamma, const void *beta,
                                     float eps, int norm);
