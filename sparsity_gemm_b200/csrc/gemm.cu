@@ -244,6 +244,11 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     int32_t *table_ok = tiles + (kGroupsMax + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    // Launched as a programmatic dependent (dense launches): the set-up
+    // below (barriers, tensor memory) overlaps the previous kernel's tail,
+    // and nothing reads or writes global memory before griddep_wait. The
+    // grouped table reads device offsets, so grouped launches wait first.
+    if constexpr (GROUPED) griddep_wait();
     if (GROUPED && warp == 2) {
         const bool ok = build_tile_table(p.offsets, p.groups, p.rows, p.m_tok, tiles);
         if (lane == 0) {
@@ -286,6 +291,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if constexpr (!GROUPED) griddep_wait();
+    griddep_launch();  // the next kernel may start its own set-up
     const uint32_t tmem = *tmem_slot;
     // m tiles: 128-row tiles of the prep (grouped: of all groups; none if the
     // offsets are invalid)
@@ -788,8 +795,18 @@ static sharq_status launch_gemm(LaunchCtx &ctx, const CUtensorMap &tm_as, const 
     sharq_status st = set_gemm_attrs<FMT, GROUPED, EXT, BN, SP>();
     if (st != SHARQ_OK) return st;
     const unsigned grid = (unsigned)(max_tiles < ctx.num_sms ? max_tiles : ctx.num_sms);
-    dual_gemm_kernel<FMT, GROUPED, EXT, BN, SP>
-        <<<grid, kGemmThreads, TileCfg<BN, SP>::kSmemBytes, ctx.stream>>>(tm_as, tm_ar, tm_b, tm_meta, gp);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = TileCfg<BN, SP>::kSmemBytes;
+    cfg.stream = ctx.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = GROUPED ? 0 : 1;  // dense launches: a programmatic dependent of the previous kernel
+    SQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, dual_gemm_kernel<FMT, GROUPED, EXT, BN, SP>, tm_as, tm_ar, tm_b, tm_meta, gp));
     ctx.launches++;
     SQ_CUDA_TRY(cudaGetLastError());
     return SHARQ_OK;
@@ -808,13 +825,15 @@ static sharq_status launch_gemm_split(LaunchCtx &ctx, const CUtensorMap &tm_as, 
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
     cfg.dynamicSmemBytes = TileCfg<kDenseBN, SP>::kSmemBytes;
     cfg.stream = ctx.stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)gp.split;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     SQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, dual_gemm_kernel<FMT, false, EXT, kDenseBN, SP>, tm_as, tm_ar, tm_b, tm_meta,
                                    gp));
     ctx.launches++;

@@ -1465,6 +1465,7 @@ prep_encode_rows_kernel(const EncodeArgs a, const unsigned *amax_word, float *__
             lut[msk] = packed;
         }
     griddep_wait();  // the statistics and the amax word are complete
+    griddep_launch();
     // What the statistics kernel wrote is read with L2 loads through pointers
     // without __restrict__, so that no load can move above the wait.
     const float amax = __uint_as_float(__ldcg(amax_word));
@@ -1581,6 +1582,7 @@ prep_encode_sparse_kernel(const EncodeArgs a, const unsigned *amax_word, float *
                           int64_t sf_rows) {
     __shared__ float4 tab[128];  // NVFP4 steps and reciprocals by scale code
     griddep_wait();  // the statistics and the amax word are complete
+    griddep_launch();
     // (read with L2 loads through pointers without __restrict__, so that no
     // load can move above the wait)
     const float amax = __uint_as_float(__ldcg(amax_word));
@@ -1803,6 +1805,10 @@ prep_small_kernel(const EncodeArgs a, float eps, int64_t sf_rows, float *__restr
         }
     if (tid < kSmallMaxRows) row_amax[tid] = 0.0f;
     __syncthreads();
+    // Launched as a programmatic dependent: everything above overlaps the
+    // previous kernel's tail; global memory only after the wait.
+    griddep_wait();
+    griddep_launch();
 
     // Phase 1a: statistics (same sums, finish and amax rule as ln_stats_kernel).
     const int64_t k = a.k, m_tok = a.m_tok;
@@ -2162,13 +2168,15 @@ static sharq_status launch_prepare_small(LaunchCtx &ctx, const sharq_prep &P, co
     cfg.gridDim = dim3(kSmallCtas, 1, 1);
     cfg.blockDim = dim3(kSmallThreads, 1, 1);
     cfg.stream = ctx.stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = kSmallCtas;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     SQ_CUDA_TRY(cudaLaunchKernelExC(&cfg, fn, args));
     ctx.launches++;
     SQ_CUDA_TRY(cudaGetLastError());
