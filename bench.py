@@ -58,11 +58,13 @@ def prep_bytes_per_elem(fmt, n, m, dense_s=False):
 PREP_BYTES_PER_ELEM = prep_bytes_per_elem(0, N_KEEP, M_GROUP)  # 3.0
 PREP_BYTES_PER_ELEM_DENSE_S = prep_bytes_per_elem(0, N_KEEP, M_GROUP, dense_s=True)  # 3.25
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) of the 7 GEMM launches of one M = 8192 step, from
-# one ncu capture of the current dual_gemm_kernel (dram__bytes_read.sum +
-# dram__bytes_write.sum of the layer-set launch list). Set to None whenever
-# the kernel changes until it is captured again.
-GEMM_TRAFFIC_BYTES_PER_STEP_M8192 = 1033.9e6
+# DRAM bytes (read + write) of the 7 GEMM launches of one M = 8192 step:
+# the sum over the step's linears of dram__bytes_read.sum +
+# dram__bytes_write.sum of one ncu capture per shape (one launch each, caches
+# flushed before it: q and o 70.9 MB, k and v 40.7 MB, gate and up 277.8 MB,
+# down 248.5 MB) of the current dual_gemm_kernel. Set to None whenever the
+# kernel changes until it is captured again.
+GEMM_TRAFFIC_BYTES_PER_STEP_M8192 = 1027.6e6
 # The only performance and accuracy figures of the method's own evaluation
 # (abstract of "SharQ: Bridging Activation Sparsity and FP4 Quantization for
 # LLM Inference"): other hardware and end-to-end serving, reported for
@@ -337,7 +339,7 @@ def run_sharq(args, world, rank, local):
                      "achieved": gemm_alg_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": gemm_alg_tflops / fp4_peak,
                      "traffic": GEMM_TRAFFIC_BYTES_PER_STEP_M8192 if M == 8192 else None,
-                     "traffic_scope": "DRAM bytes of the 7 GEMM launches of one step (ncu capture)",
+                     "traffic_scope": "DRAM bytes of the 7 GEMM launches of one step (sum of per-launch ncu captures)",
                      "peak_source": f"{peak_src} bf16 {peaks['bf16_tflops']} TF/s x {FP4_OVER_BF16} (FP4/BF16 nominal)",
                      "flops_per_step": flops_algorithmic(M), "flop_count": "2*M*N*K*(1+n/m)",
                      "executed_tflops": gemm_exec_tflops, "executed_frac": gemm_exec_tflops / fp4_peak},
@@ -697,6 +699,24 @@ def run_case(args, world, rank, local):
         op = lambda: sq.prepare(x, None, None, EPS, n, m, fmt, out=buf)
         per_elem = prep_bytes_per_elem(fmt, n, m)
         work, unit, peak, bound = per_elem * M * K, "GB/s", peaks["hbm_gbs"], "hbm"
+    elif kind == "prep_sparse":
+        M, K = nums[:2]
+        fmt = nums[2] if len(nums) > 2 else 0
+        x = torch.from_numpy(synth.activations_student(0, M, K, outlier_frac=args.outlier_frac).view(np.float16)).to(dev)
+        buf = sq.prepare_sparse(x, None, None, EPS, fmt)
+        op = lambda: sq.prepare_sparse(x, None, None, EPS, fmt, out=buf)
+        work, unit, peak, bound = prep_bytes_per_elem_sparse(fmt) * M * K, "GB/s", peaks["hbm_gbs"], "hbm"
+    elif kind == "linear_sparse":
+        M, N, K = nums[:3]
+        fmt = nums[3] if len(nums) > 3 else 0
+        x = torch.from_numpy(synth.activations_student(0, M, K, outlier_frac=args.outlier_frac).view(np.float16)).to(dev)
+        w = torch.from_numpy(synth.weights(1000, N, K).view(np.float16)).to(dev)
+        qw = sq.quantize_weight_sparse(w, fmt)
+        prep = sq.prepare_sparse(x, None, None, EPS, fmt)
+        out = torch.empty((M, N), dtype=torch.float16, device=dev)
+        op = lambda: sq.linear(prep, qw, out=out)
+        work, unit, bound = 3.0 * M * N * K, "TFLOP/s", "tensor"
+        peak = peaks["bf16_tflops"] * FP4_OVER_BF16 * 1e3  # in GFLOP/s, scaled below
     elif kind == "linear":
         M, N, K = nums[:3]
         fmt, n, m = (nums[3:6] + [0, N_KEEP, M_GROUP][len(nums[3:6]):])
