@@ -201,6 +201,32 @@ __device__ __forceinline__ uint64_t desc_operand_half(uint32_t addr) {
     return smem_desc(addr, 16, 8 * (kBKBytes / 2), 4u);
 }
 
+// Output tile of linear tile index `tile`. Dense launches walk the tiles in
+// groups of kRasterRows 128-row blocks, M fastest inside a group: the CTAs
+// running at one time share a few W tiles across many M blocks, and a W
+// tile is streamed once per group instead of once per M block (the
+// difference matters when W does not stay in L2 next to the outputs, as for
+// a fused gate/up weight). Grouped launches keep N fastest (an expert's
+// tiles stay together).
+#ifndef SQ_RASTER_ROWS
+#define SQ_RASTER_ROWS 16
+#endif
+constexpr int kRasterRows = SQ_RASTER_ROWS;
+
+template <bool GROUPED>
+__device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int &mb, int &nb) {
+    if (GROUPED || kRasterRows <= 1) {
+        mb = tile / n_tiles;
+        nb = tile % n_tiles;
+        return;
+    }
+    const int per_group = kRasterRows * n_tiles;
+    const int g = tile / per_group, in = tile - g * per_group;
+    const int rows = min(kRasterRows, m_tiles - g * kRasterRows);  // the last group may be shorter
+    nb = in / rows;
+    mb = g * kRasterRows + (in - nb * rows);
+}
+
 // Wait bounded only by time (used to drain in-flight copies on exit).
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
     uint64_t t0 = globaltimer_ns();
@@ -322,7 +348,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             uint32_t it = 0;
             bool ok = true;
             for (int tile = tile_begin; ok && tile < num_tiles; tile += tile_step) {
-                const int nb = tile % n_tiles, mb = tile / n_tiles;
+                int nb, mb;
+                tile_coords<GROUPED>(tile, m_tiles, n_tiles, mb, nb);
                 const int grp = GROUPED ? group_of_tile(tiles, p.groups, mb) : 0;
                 const uint8_t *sfb = p.sfb + (GROUPED ? (int64_t)grp * p.w_gstride : 0);
                 for (int kt = kt_begin; kt < kt_end; ++kt, ++it) {
@@ -535,7 +562,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         const unsigned store_pause_ns = kt_n >= 8 ? (unsigned)min(SQ_STORE_PAUSE_NS_PER_KSTEP * kt_n, 1000) : 0u;
         uint32_t tile_iter = 0;
         for (int tile = tile_begin; tile < num_tiles; tile += tile_step, ++tile_iter) {
-            const int nb = tile % n_tiles, mb = tile / n_tiles;
+            int nb, mb;
+            tile_coords<GROUPED>(tile, m_tiles, n_tiles, mb, nb);
             if constexpr (GROUPED) {
                 const int grp = group_of_tile(tiles, p.groups, mb);
                 alpha = __fmul_rn(s_t, *reinterpret_cast<const float *>(
@@ -652,7 +680,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         // threads of all CTAs pass both cluster barriers.
         cluster_sync();  // every partial is in its CTA's shared memory
         if (warp >= 2 && warp <= 5 && tile_begin < num_tiles) {
-            const int mb = tile_begin / n_tiles, nb = tile_begin % n_tiles;
+            int mb, nb;
+            tile_coords<GROUPED>(tile_begin, m_tiles, n_tiles, mb, nb);
             const int S = p.split, cols = C::kBN / S, groups4 = cols / 4;
             const int valid = (int)min((int64_t)kBM, (int64_t)p.m_tok - (int64_t)mb * kBM);
             const float s_t = *p.s_t;

@@ -968,6 +968,43 @@ __device__ __forceinline__ uint32_t keep_mask_42(const float (&v)[kUnit]) {
     return keep;
 }
 
+// m = 8, n = 4 with n fixed at compile time: the fourth largest magnitude t
+// of a group comes from sorting each half with a four-input network and
+// merging (for halves sorted descending, the four largest of the group are
+// max(a_i, b_{3-i}), so t is the smallest of those); an element survives iff
+// its magnitude is >= t. Where exactly four do, nothing ties at t and that
+// is the top-4 set whatever the tie rule; otherwise (a tie at t) the
+// rank-based selection decides the unit.
+__device__ __forceinline__ uint32_t keep_mask_84(const float (&v)[kUnit]) {
+    uint32_t keep = 0;
+    bool exact = true;
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+        float a[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = fabsf(v[8 * g + i]);
+        float srt[2][4];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const float p = fmaxf(a[4 * h], a[4 * h + 1]), q = fminf(a[4 * h], a[4 * h + 1]);
+            const float r = fmaxf(a[4 * h + 2], a[4 * h + 3]), s = fminf(a[4 * h + 2], a[4 * h + 3]);
+            const float x = fminf(p, r), y = fmaxf(q, s);
+            srt[h][0] = fmaxf(p, r);
+            srt[h][1] = fmaxf(x, y);
+            srt[h][2] = fminf(x, y);
+            srt[h][3] = fminf(q, s);
+        }
+        const float t = fminf(fminf(fmaxf(srt[0][0], srt[1][3]), fmaxf(srt[0][1], srt[1][2])),
+                              fminf(fmaxf(srt[0][2], srt[1][1]), fmaxf(srt[0][3], srt[1][0])));
+        uint32_t kg = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) kg |= ((~__float_as_uint(__fsub_rn(a[i], t))) >> 31) << i;  // a_i >= t
+        exact = exact && __popc(kg) == 4;
+        keep |= kg << (8 * g);
+    }
+    return exact ? keep : keep_mask<8>(v, 4);
+}
+
 // Step d = RN32(value(code) s_t) and, for d in [2^-90, 2^90], y = RN(1/d)
 // and the bracketing factors RN(y (1 -/+ 2^-21)) of e2m1x8_div (else all
 // three 0) of every UE4M3 scale code: one table per CTA, so that a block's
@@ -1092,6 +1129,8 @@ __device__ __forceinline__ void encode_core(const float (&v)[kUnit], int n, cons
     uint32_t keep;
     if constexpr (M == 4 && NK == 2)
         keep = keep_mask_42(v);
+    else if constexpr (M == 8 && NK == 4)
+        keep = keep_mask_84(v);
     else
         keep = keep_mask<M>(v, n);
     const float ds = quantize16<FMT>(v, s_t, c6, y6, tab, o.s_scale, o.s_lo, o.s_hi);
@@ -2097,7 +2136,8 @@ static void *encode_rows_fn(int m, int n) {
         case 2: return (void *)prep_encode_rows_kernel<FMT, 2, 0, AFFINE>;
         case 4: return n == 2 ? (void *)prep_encode_rows_kernel<FMT, 4, 2, AFFINE>
                               : (void *)prep_encode_rows_kernel<FMT, 4, 0, AFFINE>;
-        case 8: return (void *)prep_encode_rows_kernel<FMT, 8, 0, AFFINE>;
+        case 8: return n == 4 ? (void *)prep_encode_rows_kernel<FMT, 8, 4, AFFINE>
+                              : (void *)prep_encode_rows_kernel<FMT, 8, 0, AFFINE>;
         default: return (void *)prep_encode_rows_kernel<FMT, 16, 0, AFFINE>;
     }
 }
