@@ -26,6 +26,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -79,20 +80,24 @@ static_assert(kTableBytes % 4 == 0, "table alignment");
 // backbone tile holds the kept half of K (64-byte rows), its scales and the
 // W view the sparse MMA reads hold one scale per 32 values (half the
 // atoms), and the mask metadata rides with the scales (16 bytes per row).
-template <int BN, bool SP = false>
+// PAIR: a CTA pair computes a 256-row tile with cta_group::2 MMAs; each CTA
+// stages its own 128 A rows and half of the tile's W rows (the W scale view
+// for all of them), which leaves room for four stages.
+template <int BN, bool SP = false, bool PAIR = false>
 struct TileCfg {
     static constexpr int kBN = BN;
     static constexpr int kBlk = BN / 128;            // 128-row W blocks (scale atoms) per tile
     static constexpr int kNacc = BN == 256 ? 1 : 2;  // accumulators in tensor memory
     static constexpr int kASBytes = SP ? kABytes / 2 : kABytes;
     static constexpr int kOffAR = kASBytes, kOffB = kASBytes + kABytes;
-    static constexpr int kBBytes = BN * kBKBytes;
+    static constexpr int kBBytes = (PAIR ? BN / 2 : BN) * kBKBytes;
     static constexpr int kSfaSMax = SP ? kSfaMax / 2 : kSfaMax;  // backbone scale bytes per stage
     static constexpr int kSfbMax = kBlk * kSfaSMax;              // W scale view of the backbone path
     static constexpr int kMetaBytes = SP ? kBM * 16 : 0;
     static constexpr int kOffSFAS = kOffB + kBBytes, kOffSFAR = kOffSFAS + kSfaSMax, kOffSFB = kOffSFAR + kSfaMax;
     static constexpr int kOffMeta = kOffSFB + kSfbMax;
     static constexpr int kStageBytes = kOffMeta + kMetaBytes;  // a multiple of 1024
+    static constexpr int kTableArea = PAIR ? 0 : kTableBytes;  // the grouped tile table (not in pair launches)
     static constexpr int kStages = (232448 - 2048) / kStageBytes;
     static constexpr int kBarOff = kStages * kStageBytes;
     static constexpr uint32_t kColSf0 = kNacc * BN;
@@ -110,12 +115,13 @@ struct TileCfg {
     static constexpr int kBarBytes = 8 * (3 * kStages + 2 * kNacc + 1 + 2 * kSfBufs);
     static constexpr int kBarArea = (kBarBytes + 4 + 127) / 128 * 128;
     static constexpr int kTableOff = kBarOff + kBarArea;
-    static constexpr int kSmemBytes = kTableOff + kTableBytes + 1024;  // barriers, table, alignment slack
+    static constexpr int kSmemBytes = kTableOff + kTableArea + 1024;  // barriers, table, alignment slack
     // Split-K partial tile in the stage memory: 128 rows of BN fp32, rows
     // padded by 16 bytes so that a warp's 32 rows hit different banks.
     static constexpr uint32_t kPartStride = BN * 4 + 16;
     static_assert(BN == 128 || BN == 256, "tile width");
     static_assert(!SP || (BN == 256 && kBKBytes == 128), "the sparse mode uses the 256-column, 128-byte K tile");
+    static_assert(!PAIR || (BN == 256 && !SP), "pair launches: dense mode, 256 columns");
     static_assert(kStageBytes % 1024 == 0, "stage buffers must stay 1024-byte aligned");
     static_assert(kSmemBytes <= 232448, "shared memory budget");
     static_assert(kBarBytes + 4 <= kBarArea, "barrier area");
@@ -182,10 +188,10 @@ __device__ __forceinline__ float alpha_of_col(const GemmParams &p, float s_t, fl
 // E2M1, K-major A and B): A/B format E2M1 at bits 7-9 / 10-12, N >> 3 at
 // bits 17-22, scale format (0 = UE4M3, 1 = E8M0) at bit 23, M >> 4 at bits
 // 24-28; scale-factor byte selectors at bits 29-30 (A) and 4-5 (B).
-template <int FMT, int BN>
+template <int FMT, int BN, int MM = kBM>
 __device__ __forceinline__ uint32_t idesc_of(uint32_t sf_id) {
     return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((FMT == kFmtMX ? 1u : 0u) << 23) |
-           ((uint32_t)(kBM >> 4) << 24) | (sf_id << 29) | (sf_id << 4);
+           ((uint32_t)(MM >> 4) << 24) | (sf_id << 29) | (sf_id << 4);
 }
 
 // K-major operand tile, rows of kBKBytes bytes swizzled in kBKBytes-wide
@@ -212,19 +218,26 @@ __device__ __forceinline__ uint64_t desc_operand_half(uint32_t addr) {
 #define SQ_RASTER_ROWS 16
 #endif
 constexpr int kRasterRows = SQ_RASTER_ROWS;
+// Pair launches: groups of this many 256-row tiles (the same rows per group
+// as kRasterRows single tiles).
+#ifndef SQ_RASTER_PAIR_ROWS
+#define SQ_RASTER_PAIR_ROWS 8
+#endif
+constexpr int kRasterPairRows = SQ_RASTER_PAIR_ROWS;
 
-template <bool GROUPED>
+template <bool GROUPED, bool PAIR = false>
 __device__ __forceinline__ void tile_coords(int tile, int m_tiles, int n_tiles, int &mb, int &nb) {
-    if (GROUPED || kRasterRows <= 1) {
+    constexpr int R = PAIR ? kRasterPairRows : kRasterRows;
+    if (GROUPED || R <= 1) {
         mb = tile / n_tiles;
         nb = tile % n_tiles;
         return;
     }
-    const int per_group = kRasterRows * n_tiles;
+    const int per_group = R * n_tiles;
     const int g = tile / per_group, in = tile - g * per_group;
-    const int rows = min(kRasterRows, m_tiles - g * kRasterRows);  // the last group may be shorter
+    const int rows = min(R, m_tiles - g * R);  // the last group may be shorter
     nb = in / rows;
-    mb = g * kRasterRows + (in - nb * rows);
+    mb = g * R + (in - nb * rows);
 }
 
 // Wait bounded only by time (used to drain in-flight copies on exit).
@@ -243,13 +256,21 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 // SP (dense only): the pair-wise 4:8 backbone through tcgen05.mma.sp on a
 // K-compacted tile (tm_as rows of k/4 bytes), its metadata tile tm_meta
 // ([m_tok][k/16] bytes) moved to tensor memory by the scale writers.
-template <int FMT, bool GROUPED, bool EXT, int BN, bool SP = false>
+// PAIR (dense only, default mode): clusters of two CTAs; the pair computes
+// 256 x BN tiles with cta_group::2 MMAs issued by the even CTA (the leader).
+// Each CTA loads its own 128 A rows (both paths), its half of the W rows
+// (tm_b with 128-row boxes) and the W scales of all BN rows; the leader's
+// full and scale barriers count both CTAs' bytes and scale writes, the MMA
+// commits arrive on both CTAs' barriers, and the peer's epilogue releases
+// the accumulator on the leader's barrier.
+template <int FMT, bool GROUPED, bool EXT, int BN, bool SP = false, bool PAIR = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constant__ CUtensorMap tm_ar,
                  const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_meta,
                  const GemmParams p) {
-    using C = TileCfg<BN, SP>;
+    using C = TileCfg<BN, SP, PAIR>;
     static_assert(!SP || !GROUPED, "the sparse mode runs dense launches");
+    static_assert(!PAIR || (!GROUPED && !SP), "pair launches: dense, default mode");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_s = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
@@ -270,6 +291,11 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     int32_t *table_ok = tiles + (kGroupsMax + 1);
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    // pair launches: this CTA's place in the pair (0: leader) and the
+    // leader's address of a barrier
+    const uint32_t prank = PAIR ? (cluster_ctarank() & 1u) : 0u;
+    const bool leader = prank == 0;
+    auto at_leader = [&](uint32_t bar) { return PAIR ? mapa_shared(bar, cluster_ctarank() & ~1u) : bar; };
     // Launched as a programmatic dependent (dense launches): the set-up
     // below (barriers, tensor memory) overlaps the previous kernel's tail,
     // and nothing reads or writes global memory before griddep_wait. The
@@ -297,11 +323,11 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         }
         for (int a = 0; a < C::kNacc; ++a) {
             mbar_init(acc_full_bar(a), 1);
-            mbar_init(acc_empty_bar(a), 128);
+            mbar_init(acc_empty_bar(a), PAIR ? 256 : 128);  // pair: both CTAs' epilogue threads
         }
         mbar_init(drain_bar, 1);
         for (int b = 0; b < C::kSfBufs; ++b) {
-            mbar_init(sf_full_bar(b), 128);
+            mbar_init(sf_full_bar(b), PAIR ? 256 : 128);  // pair: both CTAs' scale writers
             mbar_init(sf_empty_bar(b), 1);
         }
         mbar_fence_init();
@@ -311,25 +337,33 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         if (SP) prefetch_tmap(&tm_meta);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
-        tmem_relinquish();
+        if (PAIR) {
+            tmem_alloc_pair(smem_u32(tmem_slot), kTmemCols);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    __syncthreads();
+    if (PAIR) cluster_sync();  // the peer's barriers exist before any remote arrival
+    else __syncthreads();
     tc_fence_after();
     if constexpr (!GROUPED) griddep_wait();
     griddep_launch();  // the next kernel may start its own set-up
     const uint32_t tmem = *tmem_slot;
     // m tiles: 128-row tiles of the prep (grouped: of all groups; none if the
     // offsets are invalid)
-    const int m_tiles = GROUPED ? (*table_ok ? tiles[p.groups] : 0) : (p.m_tok + kBM - 1) / kBM;
+    const int m_tiles = GROUPED ? (*table_ok ? tiles[p.groups] : 0)
+                                : (p.m_tok + (PAIR ? 2 * kBM : kBM) - 1) / (PAIR ? 2 * kBM : kBM);
     const int n_tiles = (p.n_out + C::kBN - 1) / C::kBN;
     const int num_tiles = m_tiles * n_tiles, kt_count = p.k / (2 * kBKBytes);
     // Tiles of this CTA: tile_begin, tile_begin + tile_step, ...; K steps
     // kt_begin .. kt_end - 1 of each. Split-K: one tile per cluster, one K
     // range per CTA of the cluster.
     const bool split = !GROUPED && p.split > 1;
-    int tile_begin = blockIdx.x, tile_step = gridDim.x, kt_begin = 0, kt_end = kt_count, rank = 0;
+    int tile_begin = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x, tile_step = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    int kt_begin = 0, kt_end = kt_count, rank = 0;
     if (split) {
         rank = (int)cluster_ctarank();
         tile_begin = blockIdx.x / p.split;
@@ -349,7 +383,13 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             bool ok = true;
             for (int tile = tile_begin; ok && tile < num_tiles; tile += tile_step) {
                 int nb, mb;
-                tile_coords<GROUPED>(tile, m_tiles, n_tiles, mb, nb);
+                tile_coords<GROUPED, PAIR>(tile, m_tiles, n_tiles, mb, nb);
+                const int rb = PAIR ? 2 * mb + (int)prank : mb;  // this CTA's 128-row block
+                // its scale atoms: a pair's second block past the last one (odd
+                // block counts) is all padding (A zero-filled by the tile load);
+                // it takes block 0's atoms, so that no copy reads past the scale
+                // arrays, and its rows are never stored
+                const int rb_sf = (PAIR && rb * kBM >= p.m_tok) ? 0 : rb;
                 const int grp = GROUPED ? group_of_tile(tiles, p.groups, mb) : 0;
                 const uint8_t *sfb = p.sfb + (GROUPED ? (int64_t)grp * p.w_gstride : 0);
                 for (int kt = kt_begin; kt < kt_end; ++kt, ++it) {
@@ -364,8 +404,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                     // Scale atoms first, on their own barrier: the scale
                     // writers move them to tensor memory while the operand
                     // tiles are still in flight.
-                    const int64_t a_off = ((int64_t)mb * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
-                    const int64_t a_off_s = ((int64_t)mb * atoms_per_row_blk_s + (int64_t)kt * kAtomsS) * 512;
+                    const int64_t a_off = ((int64_t)rb_sf * atoms_per_row_blk + (int64_t)kt * kAtomsPerTile) * 512;
+                    const int64_t a_off_s = ((int64_t)rb_sf * atoms_per_row_blk_s + (int64_t)kt * kAtomsS) * 512;
                     const int64_t b0 =
                         ((int64_t)(C::kBlk * nb) * atoms_per_row_blk_s + (int64_t)kt * kAtomsS) * 512;
                     mbar_arrive_expect_tx(lb, (1 + C::kBlk) * kSfBytesS + kSfBytes + C::kMetaBytes);
@@ -376,24 +416,35 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                         bulk_load(st + C::kOffSFB + bk * kSfBytesS, sfb + b0 + bk * atoms_per_row_blk_s * 512,
                                   kSfBytesS, lb);
                     if (SP) tma_load_2d(st + C::kOffMeta, &tm_meta, kt * 16, mb * kBM, lb);
-                    mbar_arrive_expect_tx(fb, C::kASBytes + kABytes + C::kBBytes);
-                    tma_load_2d(st + kOffAS, &tm_as, kt * (SP ? kBKBytes / 2 : kBKBytes), mb * kBM, fb);
-                    tma_load_2d(st + C::kOffAR, &tm_ar, kt * kBKBytes, mb * kBM, fb);
-                    if (GROUPED) tma_load_3d(st + C::kOffB, &tm_b, kt * kBKBytes, nb * C::kBN, grp, fb);
-                    else tma_load_2d(st + C::kOffB, &tm_b, kt * kBKBytes, nb * C::kBN, fb);
+                    if constexpr (PAIR) {
+                        // both CTAs' tiles complete on the leader's barrier
+                        if (leader) mbar_arrive_expect_tx(fb, 2 * (C::kASBytes + kABytes + C::kBBytes));
+                        const uint32_t lfb = at_leader(fb);
+                        tma_load_2d_pair(st + kOffAS, &tm_as, kt * kBKBytes, rb * kBM, lfb);
+                        tma_load_2d_pair(st + C::kOffAR, &tm_ar, kt * kBKBytes, rb * kBM, lfb);
+                        tma_load_2d_pair(st + C::kOffB, &tm_b, kt * kBKBytes, nb * C::kBN + (int)prank * (C::kBN / 2), lfb);
+                    } else {
+                        mbar_arrive_expect_tx(fb, C::kASBytes + kABytes + C::kBBytes);
+                        tma_load_2d(st + kOffAS, &tm_as, kt * (SP ? kBKBytes / 2 : kBKBytes), mb * kBM, fb);
+                        tma_load_2d(st + C::kOffAR, &tm_ar, kt * kBKBytes, mb * kBM, fb);
+                        if (GROUPED) tma_load_3d(st + C::kOffB, &tm_b, kt * kBKBytes, nb * C::kBN, grp, fb);
+                        else tma_load_2d(st + C::kOffB, &tm_b, kt * kBKBytes, nb * C::kBN, fb);
+                    }
                     last[s] = (int32_t)it;
                 }
             }
             // Never leave the CTA with copies in flight.
+            // (pair: the operand tiles of both CTAs complete on the leader's
+            // barriers, which the leader drains before the final cluster barrier)
             for (int s = 0; s < C::kStages; ++s)
                 if (last[s] >= 0) {
-                    drain_wait(full_bar(s), ((uint32_t)last[s] / C::kStages) & 1u, kDrainNs);
+                    if (!PAIR || leader) drain_wait(full_bar(s), ((uint32_t)last[s] / C::kStages) & 1u, kDrainNs);
                     drain_wait(sf_loaded_bar(s), ((uint32_t)last[s] / C::kStages) & 1u, kDrainNs);
                 }
         }
         __syncwarp();
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && (!PAIR || leader)) {  // pair: the leader issues for both CTAs
             uint32_t it = 0, tile_iter = 0;
             for (int tile = tile_begin; tile < num_tiles; tile += tile_step, ++tile_iter) {
                 // accumulator of this tile (two in turn at BN = 128)
@@ -453,8 +504,35 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                             }
                         }
                     }
+                    if constexpr (PAIR) {
+                        // M = 256 over the pair: each CTA's A rows and W half at
+                        // the same shared-memory offsets, the W scales of all
+                        // BN rows in each CTA's tensor memory
 #pragma unroll
-                    for (int j = 0; j < (SP ? 0 : kMmaPerStage); ++j) {  // MMAs of K = 64 (32 bytes) per K tile
+                        for (int j = 0; j < kMmaPerStage; ++j) {
+                            const uint32_t acc = (kt != kt_begin || j != 0) ? 1u : 0u;
+                            if (FMT == kFmtNV) {
+                                const uint32_t idesc = idesc_of<FMT, BN, 2 * kBM>(0);
+                                const uint32_t b_col = 4 * C::kBlk * j;
+                                tc_mma_nvf4_pair(dacc, da_s + 2 * j, db + 2 * j, idesc, sf + kSfaS + 4 * j,
+                                                 sf + kSfb + b_col, acc);
+                                tc_mma_nvf4_pair(dacc, da_r + 2 * j, db + 2 * j, idesc, sf + kSfaR + 4 * j,
+                                                 sf + kSfb + b_col, 1u);
+                            } else {
+                                const uint32_t sf_id = (uint32_t)(j & 1) * 2u;
+                                const uint32_t idesc = idesc_of<FMT, BN, 2 * kBM>(sf_id);
+                                const uint32_t a_col = 4 * (j >> 1), b_col = 4 * C::kBlk * (j >> 1);
+                                tc_mma_mxf4_pair(dacc, da_s + 2 * j, db + 2 * j, idesc,
+                                                 (sf + kSfaS + a_col) | (sf_id << 30), (sf + kSfb + b_col) | (sf_id << 30),
+                                                 acc);
+                                tc_mma_mxf4_pair(dacc, da_r + 2 * j, db + 2 * j, idesc,
+                                                 (sf + kSfaR + a_col) | (sf_id << 30), (sf + kSfb + b_col) | (sf_id << 30),
+                                                 1u);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < ((SP || PAIR) ? 0 : kMmaPerStage); ++j) {  // MMAs of K = 64 (32 bytes) per K tile
                         const uint32_t acc = (kt != kt_begin || j != 0) ? 1u : 0u;
                         // W scales: 4 columns per 128-row block per atom, the
                         // tile's blocks side by side
@@ -473,13 +551,20 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                                         (sf + kSfb + b_col) | (sf_id << 30), 1u);
                         }
                     }
-                    tc_commit(empty_bar(s));      // frees the stage once these MMAs complete
-                    tc_commit(sf_empty_bar(sb));  // and the scale buffer
+                    if (PAIR) {  // frees the stage and the scale buffer in both CTAs
+                        tc_commit_pair(empty_bar(s), 0x3);
+                        tc_commit_pair(sf_empty_bar(sb), 0x3);
+                    } else {
+                        tc_commit(empty_bar(s));      // frees the stage once these MMAs complete
+                        tc_commit(sf_empty_bar(sb));  // and the scale buffer
+                    }
                 }
                 if (!ok) break;
-                tc_commit(acc_full_bar(ab));
+                if (PAIR) tc_commit_pair(acc_full_bar(ab), 0x3);
+                else tc_commit(acc_full_bar(ab));
             }
-            tc_commit(drain_bar);  // every MMA of this thread done before exit
+            if (PAIR) tc_commit_pair(drain_bar, 0x1);
+            else tc_commit(drain_bar);  // every MMA of this thread done before exit
             drain_wait(drain_bar, 0, kDrainNs);
         }
         __syncwarp();
@@ -546,7 +631,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
             }
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(sf_full_bar(b));
+            if (PAIR) mbar_arrive_cluster(at_leader(sf_full_bar(b)));  // the leader's MMAs wait for both CTAs
+            else mbar_arrive(sf_full_bar(b));
         }
     } else {
         // Warps 2..5, one per tensor-memory lane quadrant q: epilogue. The
@@ -563,7 +649,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         uint32_t tile_iter = 0;
         for (int tile = tile_begin; tile < num_tiles; tile += tile_step, ++tile_iter) {
             int nb, mb;
-            tile_coords<GROUPED>(tile, m_tiles, n_tiles, mb, nb);
+            tile_coords<GROUPED, PAIR>(tile, m_tiles, n_tiles, mb, nb);
             if constexpr (GROUPED) {
                 const int grp = group_of_tile(tiles, p.groups, mb);
                 alpha = __fmul_rn(s_t, *reinterpret_cast<const float *>(
@@ -637,7 +723,8 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                 }
             }
             tc_fence_before();
-            mbar_arrive(acc_empty_bar(ab));
+            if (PAIR) mbar_arrive_cluster(at_leader(acc_empty_bar(ab)));
+            else mbar_arrive(acc_empty_bar(ab));
             int64_t row, row_end;  // output row of this lane; end of the tile's valid rows
             if constexpr (GROUPED) {
                 // looked up again rather than kept live across the drain (register pressure)
@@ -646,7 +733,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                 row = (int64_t)first + (int64_t)(mb - tiles[g2]) * kBM + q * 32 + lane;
                 row_end = last;
             } else {
-                row = mb * kBM + q * 32 + lane;
+                row = (PAIR ? 2 * mb + (int)prank : mb) * kBM + q * 32 + lane;
                 row_end = p.m_tok;
             }
             const unsigned pause_ns = tile + tile_step < num_tiles ? store_pause_ns : 0u;
@@ -681,7 +768,7 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
         cluster_sync();  // every partial is in its CTA's shared memory
         if (warp >= 2 && warp <= 5 && tile_begin < num_tiles) {
             int mb, nb;
-            tile_coords<GROUPED>(tile_begin, m_tiles, n_tiles, mb, nb);
+            tile_coords<GROUPED, PAIR>(tile_begin, m_tiles, n_tiles, mb, nb);
             const int S = p.split, cols = C::kBN / S, groups4 = cols / 4;
             const int valid = (int)min((int64_t)kBM, (int64_t)p.m_tok - (int64_t)mb * kBM);
             const float s_t = *p.s_t;
@@ -718,10 +805,12 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     }
 
     tc_fence_before();
-    __syncthreads();
+    if (PAIR) cluster_sync();  // both CTAs done with the pair's tensor memory and barriers
+    else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        if (PAIR) tmem_dealloc_pair(tmem, kTmemCols);
+        else tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -801,7 +890,7 @@ static bool make_grouped_code_map(CUtensorMap *tm, const void *base, uint64_t ro
     return r == CUDA_SUCCESS;
 }
 
-template <int FMT, bool GROUPED, bool EXT, int BN, bool SP = false>
+template <int FMT, bool GROUPED, bool EXT, int BN, bool SP = false, bool PAIR = false>
 static sharq_status set_gemm_attrs() {
     static bool attr_done[64] = {};
     static std::mutex mu;  // one setter per device, also under concurrent first calls
@@ -810,8 +899,8 @@ static sharq_status set_gemm_attrs() {
     if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> lock(mu);
     if (!attr_done[dev]) {
-        SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<FMT, GROUPED, EXT, BN, SP>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TileCfg<BN, SP>::kSmemBytes));
+        SQ_CUDA_TRY(cudaFuncSetAttribute(dual_gemm_kernel<FMT, GROUPED, EXT, BN, SP, PAIR>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TileCfg<BN, SP, PAIR>::kSmemBytes));
         attr_done[dev] = true;
     }
     return SHARQ_OK;
@@ -839,6 +928,72 @@ static sharq_status launch_gemm(LaunchCtx &ctx, const CUtensorMap &tm_as, const 
     ctx.launches++;
     SQ_CUDA_TRY(cudaGetLastError());
     return SHARQ_OK;
+}
+
+// Pair launch: clusters of two CTAs, each pair walking 256-row tiles
+// (`pair_tiles` of them) with the grid stride; as many pairs as can be
+// resident at once.
+template <int FMT, bool EXT>
+static sharq_status launch_gemm_pair(LaunchCtx &ctx, const CUtensorMap &tm_as, const CUtensorMap &tm_ar,
+                                     const CUtensorMap &tm_b, const GemmParams &gp, int64_t pair_tiles) {
+    sharq_status st = set_gemm_attrs<FMT, false, EXT, kDenseBN, false, true>();
+    if (st != SHARQ_OK) return st;
+    static int cache[64] = {0};
+    static std::mutex mu;
+    int dev = 0;
+    SQ_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.blockDim = dim3(kGemmThreads, 1, 1);
+    cfg.dynamicSmemBytes = TileCfg<kDenseBN, false, true>::kSmemBytes;
+    cfg.stream = ctx.stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    int pairs = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!cache[dev]) {
+            cfg.gridDim = dim3(2, 1, 1);
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, dual_gemm_kernel<FMT, false, EXT, kDenseBN, false, true>, &cfg) !=
+                    cudaSuccess ||
+                n < 1) {
+                cudaGetLastError();
+                n = ctx.num_sms / 2;
+            }
+            cache[dev] = n;
+        }
+        pairs = cache[dev];
+    }
+    if (pair_tiles < pairs) pairs = (int)pair_tiles;
+    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    cfg.numAttrs = 2;
+    SQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, dual_gemm_kernel<FMT, false, EXT, kDenseBN, false, true>, tm_as, tm_ar, tm_b,
+                                   tm_b, gp));
+    ctx.launches++;
+    SQ_CUDA_TRY(cudaGetLastError());
+    return SHARQ_OK;
+}
+
+// Pair launches for the default mode's shapes of two or more 128-row tiles
+// when SHARQ_GEMM_PAIR=1 is set in the environment (read once per process).
+// Off by default: on B200 the pair kernel is correct but slower than the
+// single-CTA kernel (down projection 8192 x 4096 x 14336: 0.43 ms against
+// 0.30 ms), its tensor pipe idle half of the time between stages.
+static bool pair_enabled() {
+    static const bool on = []() {
+        const char *e = getenv("SHARQ_GEMM_PAIR");
+        return e && e[0] == '1';
+    }();
+    return on;
 }
 
 // Split-K launch: `tiles` clusters of gp.split CTAs, one tile per cluster.
@@ -966,6 +1121,18 @@ sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &
     }
     // the extended epilogue (fused segments, bias) only where needed
     const bool ext = gp.bias != nullptr || gp.segs > 1;
+    const int64_t m_tiles = (P.m_tok + kBM - 1) / kBM;
+    if (gp.split == 1 && m_tiles >= 2 && pair_enabled()) {
+        // CTA pairs on 256-row tiles: W staged half per CTA
+        CUtensorMap tm_bh;
+        if (!make_code_map(&tm_bh, W.codes, (uint64_t)(W.k / 2), (uint64_t)W.n_out, kDenseBN / 2)) return SHARQ_ERR_CUDA;
+        const int64_t pair_tiles = ((P.m_tok + 2 * kBM - 1) / (2 * kBM)) * ((W.n_out + kDenseBN - 1) / kDenseBN);
+        if (ext)
+            return P.fmt == kFmtNV ? launch_gemm_pair<kFmtNV, true>(ctx, tm_as, tm_ar, tm_bh, gp, pair_tiles)
+                                   : launch_gemm_pair<kFmtMX, true>(ctx, tm_as, tm_ar, tm_bh, gp, pair_tiles);
+        return P.fmt == kFmtNV ? launch_gemm_pair<kFmtNV, false>(ctx, tm_as, tm_ar, tm_bh, gp, pair_tiles)
+                               : launch_gemm_pair<kFmtMX, false>(ctx, tm_as, tm_ar, tm_bh, gp, pair_tiles);
+    }
     if (gp.split > 1) {
         if (ext)
             return P.fmt == kFmtNV ? launch_gemm_split<kFmtNV, true>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles)
