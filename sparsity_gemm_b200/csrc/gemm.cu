@@ -997,17 +997,17 @@ static bool pair_enabled() {
 }
 
 // Split-K launch: `tiles` clusters of gp.split CTAs, one tile per cluster.
-template <int FMT, bool EXT, bool SP = false>
+template <int FMT, bool EXT, bool SP = false, int BN = kDenseBN>
 static sharq_status launch_gemm_split(LaunchCtx &ctx, const CUtensorMap &tm_as, const CUtensorMap &tm_ar,
                                       const CUtensorMap &tm_b, const CUtensorMap &tm_meta, const GemmParams &gp,
                                       int64_t tiles) {
-    sharq_status st = set_gemm_attrs<FMT, false, EXT, kDenseBN, SP>();
+    sharq_status st = set_gemm_attrs<FMT, false, EXT, BN, SP>();
     if (st != SHARQ_OK) return st;
     cudaLaunchConfig_t cfg;
     memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3((unsigned)(tiles * gp.split), 1, 1);
     cfg.blockDim = dim3(kGemmThreads, 1, 1);
-    cfg.dynamicSmemBytes = TileCfg<kDenseBN, SP>::kSmemBytes;
+    cfg.dynamicSmemBytes = TileCfg<BN, SP>::kSmemBytes;
     cfg.stream = ctx.stream;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1018,8 +1018,7 @@ static sharq_status launch_gemm_split(LaunchCtx &ctx, const CUtensorMap &tm_as, 
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    SQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, dual_gemm_kernel<FMT, false, EXT, kDenseBN, SP>, tm_as, tm_ar, tm_b, tm_meta,
-                                   gp));
+    SQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, dual_gemm_kernel<FMT, false, EXT, BN, SP>, tm_as, tm_ar, tm_b, tm_meta, gp));
     ctx.launches++;
     SQ_CUDA_TRY(cudaGetLastError());
     return SHARQ_OK;
@@ -1027,7 +1026,7 @@ static sharq_status launch_gemm_split(LaunchCtx &ctx, const CUtensorMap &tm_as, 
 
 // Clusters of `split` CTAs of this kernel that can be resident at once (0 if
 // such a cluster does not fit), cached per device, format and size.
-template <int FMT>
+template <int FMT, int BN = kDenseBN>
 static int active_clusters(int split) {
     static int cache[64][kMaxSplit + 1];
     static bool known[64][kMaxSplit + 1] = {};
@@ -1036,12 +1035,12 @@ static int active_clusters(int split) {
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || split > kMaxSplit) return 0;
     std::lock_guard<std::mutex> lock(mu);
     if (!known[dev][split]) {
-        if (set_gemm_attrs<FMT, false, false, kDenseBN>() != SHARQ_OK) return 0;
+        if (set_gemm_attrs<FMT, false, false, BN>() != SHARQ_OK) return 0;
         cudaLaunchConfig_t cfg;
         memset(&cfg, 0, sizeof(cfg));
         cfg.gridDim = dim3((unsigned)split, 1, 1);
         cfg.blockDim = dim3(kGemmThreads, 1, 1);
-        cfg.dynamicSmemBytes = TileCfg<kDenseBN>::kSmemBytes;
+        cfg.dynamicSmemBytes = TileCfg<BN>::kSmemBytes;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = (unsigned)split;
@@ -1050,7 +1049,7 @@ static int active_clusters(int split) {
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, dual_gemm_kernel<FMT, false, false, kDenseBN>, &cfg) != cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&n, dual_gemm_kernel<FMT, false, false, BN>, &cfg) != cudaSuccess) {
             cudaGetLastError();
             n = 0;
         }
@@ -1063,11 +1062,11 @@ static int active_clusters(int split) {
 // Split-K factor for a dense launch: when the tiles fill less than half the
 // SMs, the largest power of two <= 8 with tiles x split <= SMs, split <= K
 // steps, and all the clusters resident at once; 1 otherwise.
-template <int FMT>
+template <int FMT, int BN = kDenseBN>
 static int choose_split(LaunchCtx &ctx, int64_t tiles, int kt_count) {
     if (tiles * 2 > ctx.num_sms) return 1;
     int s = kMaxSplit;
-    while (s > 1 && (tiles * s > ctx.num_sms || s > kt_count || active_clusters<FMT>(s) < tiles)) s >>= 1;
+    while (s > 1 && (tiles * s > ctx.num_sms || s > kt_count || active_clusters<FMT, BN>(s) < tiles)) s >>= 1;
     return s;
 }
 
