@@ -814,6 +814,255 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
     }
 }
 
+// ---------------------------------------------------------------------------
+// Decode GEMM (up to kDecTok tokens): the weight rows are the MMA's M side
+// and the tokens its N side, out^T = W (Q(S) + Q(R))^T. The block-scaled
+// MMA has M = 128 (or 256) rows; with the activation as A, a handful of
+// tokens would pay for 128 rows of tensor work, whereas here the tensor work
+// is 128 x 16 per K slice and the launch streams the weight. One CTA per
+// (128-row weight tile, K range); K ranges of a tile go to the CTAs of a
+// cluster, which reduce their fp32 partials through distributed shared
+// memory as dual_gemm_kernel's split-K does; two CTAs fit on an SM, so that a
+// single wave holds up to 2 x SMs CTAs. Per stage: the W tile (A), the
+// backbone and residual tiles of the tokens (B, 16 rows, zero-filled past
+// m_tok), the W scale atoms (A scales) and the activations' first scale
+// atoms (B scales: the block-scaled MMA reads B scales in the layout of a
+// 128-row operand). 8 warps: warp 0 loads, warp 1 allocates tensor memory
+// and issues the MMAs, warps 4..7 move each stage's scales to tensor memory
+// and, after the K loop, drain the accumulator (lane = weight row, column =
+// token).
+constexpr int kDecTok = 16;                       // token rows of the B tiles (MMA N)
+constexpr int kDecThreads = 256;
+constexpr int kDecW = kBM * kBKBytes;             // W tile bytes (128 rows)
+constexpr int kDecB = kDecTok * kBKBytes;         // one activation tile
+constexpr int kDecSf = 512 * (kBKBytes / 32);     // scale bytes of one 128-row operand per stage (NVFP4)
+constexpr int kDecOffS = kDecW, kDecOffR = kDecW + kDecB, kDecOffSfW = kDecW + 2 * kDecB;
+constexpr int kDecOffSfS = kDecOffSfW + kDecSf, kDecOffSfR = kDecOffSfS + kDecSf;
+constexpr int kDecStage = kDecOffSfR + kDecSf;    // 26 KB, a multiple of 1024
+constexpr int kDecStages = 4;                     // two CTAs per SM: 8 stages in flight per SM
+constexpr int kDecBarOff = kDecStages * kDecStage;
+constexpr int kDecSfBufs = 4;
+constexpr int kDecSfCols = 3 * 4 * (kBKBytes / 32);  // W, S, R atoms per stage, 4 columns each
+constexpr int kDecTmemCols = 256;                    // accumulator (16 columns) + scale buffers
+constexpr int kDecSmem = kDecBarOff + 256 + 1024;
+constexpr uint32_t kDecPartStride = kBM * 4 + 16;    // split-K partial: [token][column] fp32 rows
+static_assert(kDecStage % 1024 == 0, "decode stage alignment");
+static_assert(kDecTok + kDecSfBufs * kDecSfCols <= kDecTmemCols, "decode tensor memory");
+static_assert(2 * (kDecSmem + 1024) <= 233472, "decode shared memory: two CTAs per SM");
+static_assert(kDecTok * kDecPartStride <= (uint32_t)kDecBarOff, "decode split-K partial fits the stages");
+
+template <int FMT, bool EXT>
+__global__ void __launch_bounds__(kDecThreads, 2)
+decode_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_s,
+                   const __grid_constant__ CUtensorMap tm_r, const GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw_s + 1023u) & ~1023u) - raw_s);
+    const uint32_t sbase = smem_u32(smem);
+    const uint32_t bar0 = sbase + kDecBarOff;
+    auto full_bar = [&](int s) { return bar0 + 8u * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (kDecStages + s); };
+    auto sf_loaded_bar = [&](int s) { return bar0 + 8u * (2 * kDecStages + s); };
+    auto sf_full_bar = [&](int b) { return bar0 + 8u * (3 * kDecStages + b); };
+    auto sf_empty_bar = [&](int b) { return bar0 + 8u * (3 * kDecStages + kDecSfBufs + b); };
+    const uint32_t acc_bar = bar0 + 8u * (3 * kDecStages + 2 * kDecSfBufs);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kDecBarOff + 8 * (3 * kDecStages + 2 * kDecSfBufs + 1));
+    constexpr int kAtoms = FMT == kFmtNV ? kBKBytes / 32 : kBKBytes / 64;  // scale atoms per operand per stage
+    constexpr uint32_t kSfBytes = 512u * kAtoms;
+    // columns of a scale buffer: W atoms, then the backbone's, then the residual's
+    constexpr uint32_t kColS = 4 * kAtoms, kColR = 8 * kAtoms;
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int kt_count = p.k / (2 * kBKBytes);
+    const int S = p.split, rank = S > 1 ? (int)cluster_ctarank() : 0;
+    const int nb = (int)blockIdx.x / S;  // weight tile (128 output columns)
+    const int kt_begin = rank * kt_count / S, kt_end = (rank + 1) * kt_count / S, kt_n = kt_end - kt_begin;
+    const int64_t apr = (int64_t)(p.k / (FMT == kFmtNV ? 16 : 32)) / 4;  // scale atoms per 128-row block
+    if (warp == 0) {
+        // This CTA's weight range starts streaming into L2 here, before the
+        // dependency wait, so that it overlaps the previous kernel. Safe even
+        // if that kernel writes the weight: a prefetch only warms L2 (the
+        // point of coherence), and the copies the MMAs read come after the wait.
+        for (int i = lane; i < kt_n; i += 32) tma_prefetch_l2_2d(&tm_w, (kt_begin + i) * kBKBytes, nb * kBM);
+        if (lane == 0)
+            bulk_prefetch_l2(p.sfb + ((int64_t)nb * apr + (int64_t)kt_begin * kAtoms) * 512, (uint32_t)(kt_n * kSfBytes));
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kDecStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+            mbar_init(sf_loaded_bar(s), 1);
+        }
+        for (int b = 0; b < kDecSfBufs; ++b) {
+            mbar_init(sf_full_bar(b), 128);
+            mbar_init(sf_empty_bar(b), 1);
+        }
+        mbar_init(acc_bar, 1);
+        mbar_fence_init();
+        prefetch_tmap(&tm_w);
+        prefetch_tmap(&tm_s);
+        prefetch_tmap(&tm_r);
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), kDecTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    griddep_wait();  // launched as a programmatic dependent: memory only from here
+    griddep_launch();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int32_t last[kDecStages];
+            for (int s = 0; s < kDecStages; ++s) last[s] = -1;
+            for (int i = 0; i < kt_n; ++i) {
+                const int kt = kt_begin + i, s = i % kDecStages;
+                if (!mbar_wait(empty_bar(s), ((i / kDecStages) & 1) ^ 1, p.status, kSiteProducer, p.wait_ns)) break;
+                const uint32_t st = sbase + (uint32_t)(s * kDecStage);
+                const uint32_t lb = sf_loaded_bar(s), fb = full_bar(s);
+                mbar_arrive_expect_tx(lb, 3 * kSfBytes);
+                bulk_load(st + kDecOffSfW, p.sfb + ((int64_t)nb * apr + (int64_t)kt * kAtoms) * 512, kSfBytes, lb);
+                bulk_load(st + kDecOffSfS, p.sfa_s + (int64_t)kt * kAtoms * 512, kSfBytes, lb);
+                bulk_load(st + kDecOffSfR, p.sfa_r + (int64_t)kt * kAtoms * 512, kSfBytes, lb);
+                mbar_arrive_expect_tx(fb, kDecW + 2 * kDecB);
+                tma_load_2d(st, &tm_w, kt * kBKBytes, nb * kBM, fb);
+                tma_load_2d(st + kDecOffS, &tm_s, kt * kBKBytes, 0, fb);
+                tma_load_2d(st + kDecOffR, &tm_r, kt * kBKBytes, 0, fb);
+                last[s] = i;
+            }
+            for (int s = 0; s < kDecStages; ++s)
+                if (last[s] >= 0) {
+                    drain_wait(full_bar(s), ((uint32_t)last[s] / kDecStages) & 1u, kDrainNs);
+                    drain_wait(sf_loaded_bar(s), ((uint32_t)last[s] / kDecStages) & 1u, kDrainNs);
+                }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            bool ok = true;
+            for (int i = 0; i < kt_n && ok; ++i) {
+                const int s = i % kDecStages, sb = i % kDecSfBufs;
+                if (!mbar_wait(full_bar(s), (i / kDecStages) & 1, p.status, kSiteMmaFull, p.wait_ns) ||
+                    !mbar_wait(sf_full_bar(sb), (i / kDecSfBufs) & 1, p.status, kSiteMmaScales, p.wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t st = sbase + (uint32_t)(s * kDecStage);
+                const uint32_t sf = tmem + kDecTok + kDecSfCols * (uint32_t)sb;
+                const uint64_t dw = desc_operand(st), ds = desc_operand(st + kDecOffS), dr = desc_operand(st + kDecOffR);
+#pragma unroll
+                for (int j = 0; j < kMmaPerStage; ++j) {
+                    const uint32_t acc = (i != 0 || j != 0) ? 1u : 0u;
+                    if (FMT == kFmtNV) {
+                        // M = 128 weight rows, N = kDecTok tokens
+                        const uint32_t idesc = idesc_of<FMT, kDecTok>(0);
+                        tc_mma_nvf4(tmem, dw + 2 * j, ds + 2 * j, idesc, sf + 4 * j, sf + kColS + 4 * j, acc);
+                        tc_mma_nvf4(tmem, dw + 2 * j, dr + 2 * j, idesc, sf + 4 * j, sf + kColR + 4 * j, 1u);
+                    } else {
+                        const uint32_t sf_id = (uint32_t)(j & 1) * 2u;
+                        const uint32_t idesc = idesc_of<FMT, kDecTok>(sf_id);
+                        const uint32_t col = 4 * (j >> 1);
+                        tc_mma_mxf4(tmem, dw + 2 * j, ds + 2 * j, idesc, (sf + col) | (sf_id << 30),
+                                    (sf + kColS + col) | (sf_id << 30), acc);
+                        tc_mma_mxf4(tmem, dw + 2 * j, dr + 2 * j, idesc, (sf + col) | (sf_id << 30),
+                                    (sf + kColR + col) | (sf_id << 30), 1u);
+                    }
+                }
+                tc_commit(empty_bar(s));
+                tc_commit(sf_empty_bar(sb));
+            }
+            tc_commit(acc_bar);  // also every MMA done before exit
+            drain_wait(acc_bar, 0, kDrainNs);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // Scale writes (lane quadrant q), then the accumulator drain.
+        const int q = warp & 3;
+        const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        bool ok = true;
+        for (int i = 0; i < kt_n; ++i) {
+            const int s = i % kDecStages, b = i % kDecSfBufs;
+            const bool w1 = mbar_wait(sf_loaded_bar(s), (i / kDecStages) & 1, p.status, kSiteScaleFull, p.wait_ns);
+            const bool w2 = w1 && mbar_wait(sf_empty_bar(b), ((i / kDecSfBufs) & 1) ^ 1, p.status, kSiteScaleEmpty,
+                                            p.wait_ns);
+            if (!__all_sync(0xFFFFFFFFu, w2)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t st = sbase + (uint32_t)(s * kDecStage) + (uint32_t)lane * 16u;
+            const uint32_t sf = tmem + lane_base + kDecTok + kDecSfCols * (uint32_t)b;
+#pragma unroll
+            for (int a = 0; a < kAtoms; ++a) {
+                tmem_st4(sf + 4 * a, lds128(st + kDecOffSfW + 512 * a));
+                tmem_st4(sf + kColS + 4 * a, lds128(st + kDecOffSfS + 512 * a));
+                tmem_st4(sf + kColR + 4 * a, lds128(st + kDecOffSfR + 512 * a));
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(sf_full_bar(b));
+        }
+        const bool got = ok && mbar_wait(acc_bar, 0, p.status, kSiteEpilogue, p.wait_ns);
+        if (__all_sync(0xFFFFFFFFu, got)) {
+            tc_fence_after();
+            uint32_t r[16];
+            tmem_ld16(tmem + lane_base, r);
+            tmem_ld_wait();
+            const int col_local = q * 32 + lane, col = nb * kBM + col_local;  // this lane's output column
+            if (S > 1) {
+                // fp32 partial [token][column] in the stage memory, reduced below
+#pragma unroll
+                for (int t = 0; t < kDecTok; ++t)
+                    if (t < p.m_tok)
+                        *reinterpret_cast<uint32_t *>(smem + (uint32_t)t * kDecPartStride + (uint32_t)col_local * 4u) = r[t];
+            } else if (col < p.n_out) {
+                const float s_t = *p.s_t;
+                const float alpha = EXT ? alpha_of_col(p, s_t, __fmul_rn(s_t, *p.s_tw), col) : __fmul_rn(s_t, *p.s_tw);
+                const float b = (EXT && p.bias != nullptr) ? __half2float(p.bias[col]) : 0.0f;
+#pragma unroll
+                for (int t = 0; t < kDecTok; ++t)
+                    if (t < p.m_tok) {
+                        float y = __fmul_rn(__uint_as_float(r[t]), alpha);
+                        if (EXT && p.bias != nullptr) y = __fadd_rn(y, b);
+                        p.out[(int64_t)t * p.n_out + col] = __float2half_rn(y);
+                    }
+            }
+        }
+    }
+    if (S > 1) {
+        // Split-K: CTA `rank` sums column slice `rank` of the tile over every
+        // CTA's partial in rank order (fixed order: results do not depend on
+        // timing), then scales, rounds and stores.
+        cluster_sync();
+        if (warp >= 4) {
+            const int c0 = rank * kBM / S, cols = (rank + 1) * kBM / S - c0;  // this CTA's column slice
+            const float s_t = *p.s_t;
+            const float alpha0 = __fmul_rn(s_t, *p.s_tw);
+            for (int item = (warp - 4) * 32 + lane; item < p.m_tok * cols; item += 128) {
+                const int t = item / cols, cl = c0 + item % cols, col = nb * kBM + cl;
+                if (col >= p.n_out) continue;
+                const uint32_t off = sbase + (uint32_t)t * kDecPartStride + (uint32_t)cl * 4u;
+                float acc = __uint_as_float(ld_cluster_u32(mapa_shared(off, 0)));
+                for (int c = 1; c < S; ++c) acc = __fadd_rn(acc, __uint_as_float(ld_cluster_u32(mapa_shared(off, (uint32_t)c))));
+                float y = __fmul_rn(acc, EXT ? alpha_of_col(p, s_t, alpha0, col) : alpha0);
+                if (EXT && p.bias != nullptr) y = __fadd_rn(y, __half2float(p.bias[col]));
+                p.out[(int64_t)t * p.n_out + col] = __float2half_rn(y);
+            }
+        }
+        cluster_sync();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kDecTmemCols);
+    }
+}
+
 // Failure-detection probe: one thread waits, with the bounded wait the GEMM
 // uses, on an mbarrier that nothing ever arrives at. The wait runs out and
 // records kSiteProbe; the kernel then returns normally.
@@ -1070,6 +1319,101 @@ static int choose_split(LaunchCtx &ctx, int64_t tiles, int kt_count) {
     return s;
 }
 
+// Decode launches: clusters of gp.split CTAs per 128-row W tile.
+template <int FMT, bool EXT>
+static sharq_status set_decode_attrs() {
+    static bool attr_done[64] = {};
+    static std::mutex mu;
+    int dev = 0;
+    SQ_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return SHARQ_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attr_done[dev]) {
+        SQ_CUDA_TRY(cudaFuncSetAttribute(decode_gemm_kernel<FMT, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kDecSmem));
+        attr_done[dev] = true;
+    }
+    return SHARQ_OK;
+}
+
+// Decode clusters of `split` CTAs that can be resident at once, cached per
+// device and format.
+template <int FMT>
+static int decode_active_clusters(int split) {
+    static int cache[64][kMaxSplit + 1];
+    static bool known[64][kMaxSplit + 1] = {};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || split > kMaxSplit) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!known[dev][split]) {
+        if (set_decode_attrs<FMT, false>() != SHARQ_OK) return 0;
+        cudaLaunchConfig_t cfg;
+        memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3((unsigned)split, 1, 1);
+        cfg.blockDim = dim3(kDecThreads, 1, 1);
+        cfg.dynamicSmemBytes = kDecSmem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)split;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, decode_gemm_kernel<FMT, false>, &cfg) != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        cache[dev][split] = n;
+        known[dev][split] = true;
+    }
+    return cache[dev][split];
+}
+
+// Split-K factor of a decode launch: the largest split <= 8 (any integer)
+// with tiles x split <= SQ_DECODE_WAVE CTAs per SM, split <= K steps and
+// every cluster resident at once. One CTA per SM (the default) leaves each
+// SM room for a CTA of the next launch, whose weight prefetch then overlaps
+// this one.
+#ifndef SQ_DECODE_WAVE
+#define SQ_DECODE_WAVE 1
+#endif
+template <int FMT>
+static int choose_decode_split(LaunchCtx &ctx, int64_t tiles, int kt_count) {
+    int s = kMaxSplit;
+    while (s > 1 && (tiles * s > SQ_DECODE_WAVE * (int64_t)ctx.num_sms || s > kt_count ||
+                     decode_active_clusters<FMT>(s) < tiles))
+        --s;
+    return s;
+}
+
+template <int FMT, bool EXT>
+static sharq_status launch_decode(LaunchCtx &ctx, const CUtensorMap &tm_w, const CUtensorMap &tm_s,
+                                  const CUtensorMap &tm_r, const GemmParams &gp, int64_t tiles) {
+    sharq_status st = set_decode_attrs<FMT, EXT>();
+    if (st != SHARQ_OK) return st;
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(tiles * gp.split), 1, 1);
+    cfg.blockDim = dim3(kDecThreads, 1, 1);
+    cfg.dynamicSmemBytes = kDecSmem;
+    cfg.stream = ctx.stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)gp.split;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = gp.split > 1 ? 2 : 1;
+    SQ_CUDA_TRY(cudaLaunchKernelEx(&cfg, decode_gemm_kernel<FMT, EXT>, tm_w, tm_s, tm_r, gp));
+    ctx.launches++;
+    SQ_CUDA_TRY(cudaGetLastError());
+    return SHARQ_OK;
+}
+
 static GemmParams gemm_params(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, void *out) {
     GemmParams gp;
     memset(&gp, 0, sizeof(gp));
@@ -1094,6 +1438,27 @@ static GemmParams gemm_params(LaunchCtx &ctx, const sharq_prep &P, const sharq_w
 sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &W, const void *bias, void *out) {
     if (P.m_tok == 0) return SHARQ_OK;
     const bool sp = P.sparse != 0;
+    GemmParams gp = gemm_params(ctx, P, W, out);
+    gp.bias = (const __half *)bias;
+    const int kt_count = (int)(P.k / (2 * kBKBytes));
+    // the extended epilogue (fused segments, bias) only where needed
+    const bool ext = gp.bias != nullptr || gp.segs > 1;
+    if (!sp && P.m_tok <= kDecTok) {
+        // decode: W rows on the MMA's M side, the tokens on its N side
+        CUtensorMap tm_w, tm_s, tm_r;
+        if (!make_code_map(&tm_w, W.codes, (uint64_t)(W.k / 2), (uint64_t)W.n_out, kBM) ||
+            !make_code_map(&tm_s, P.s_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kDecTok) ||
+            !make_code_map(&tm_r, P.r_codes, (uint64_t)(P.k / 2), (uint64_t)P.m_tok, kDecTok))
+            return SHARQ_ERR_CUDA;
+        const int64_t w_tiles = (W.n_out + kBM - 1) / kBM;
+        gp.split = P.fmt == kFmtNV ? choose_decode_split<kFmtNV>(ctx, w_tiles, kt_count)
+                                   : choose_decode_split<kFmtMX>(ctx, w_tiles, kt_count);
+        if (ext)
+            return P.fmt == kFmtNV ? launch_decode<kFmtNV, true>(ctx, tm_w, tm_s, tm_r, gp, w_tiles)
+                                   : launch_decode<kFmtMX, true>(ctx, tm_w, tm_s, tm_r, gp, w_tiles);
+        return P.fmt == kFmtNV ? launch_decode<kFmtNV, false>(ctx, tm_w, tm_s, tm_r, gp, w_tiles)
+                               : launch_decode<kFmtMX, false>(ctx, tm_w, tm_s, tm_r, gp, w_tiles);
+    }
     CUtensorMap tm_as, tm_ar, tm_b, tm_meta;
     if (!make_code_map(&tm_as, P.s_codes, (uint64_t)(P.k / (sp ? 4 : 2)), (uint64_t)P.m_tok, kBM,
                        sp ? kBKBytes / 2 : kBKBytes) ||
@@ -1105,10 +1470,7 @@ sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &
     } else {
         tm_meta = tm_b;  // unused
     }
-    GemmParams gp = gemm_params(ctx, P, W, out);
-    gp.bias = (const __half *)bias;
     const int64_t tiles = ((P.m_tok + kBM - 1) / kBM) * ((W.n_out + kDenseBN - 1) / kDenseBN);
-    const int kt_count = (int)(P.k / (2 * kBKBytes));
     gp.split = P.fmt == kFmtNV ? choose_split<kFmtNV>(ctx, tiles, kt_count) : choose_split<kFmtMX>(ctx, tiles, kt_count);
     if (sp) {  // no bias or fused segments in this mode (checked by the caller)
         if (gp.split > 1)
@@ -1118,8 +1480,6 @@ sharq_status launch_linear(LaunchCtx &ctx, const sharq_prep &P, const sharq_wq &
                    ? launch_gemm<kFmtNV, false, false, kDenseBN, true>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles)
                    : launch_gemm<kFmtMX, false, false, kDenseBN, true>(ctx, tm_as, tm_ar, tm_b, tm_meta, gp, tiles);
     }
-    // the extended epilogue (fused segments, bias) only where needed
-    const bool ext = gp.bias != nullptr || gp.segs > 1;
     const int64_t m_tiles = (P.m_tok + kBM - 1) / kBM;
     if (gp.split == 1 && m_tiles >= 2 && pair_enabled()) {
         // CTA pairs on 256-row tiles: W staged half per CTA
