@@ -1026,7 +1026,10 @@ def run_decode(args, M):
     a CUDA graph and replayed. L2 is flushed before every step (outside the
     graph), so the weights stream from HBM as they do when a model's layers
     take turns; the roofline is that weight stream (codes + scales of the 7
-    weights) at the measured HBM bandwidth."""
+    weights) at the measured HBM bandwidth. Also timed (graph only): the
+    fused-projection layout a serving stack uses, q/k/v as one weight and
+    gate/up as one (quantize_weight_fused, each segment with its own tensor
+    scale): 4 preps + 4 linears, the same weight bytes."""
     import sparsity_gemm_b200 as sq
     dev = torch.device("cuda", torch.cuda.current_device())
     ls, preps = layer_set()
@@ -1078,6 +1081,46 @@ def run_decode(args, M):
     eager_ms = timed(step)
     graph_ms = timed(graph.replay)
     same = all(torch.equal(o.view(torch.int16), e.view(torch.int16)) for o, e in zip(outs, eager_out))
+
+    # fused projections: q/k/v and gate/up, each group one weight
+    groups = {}
+    for j, lin in enumerate(ls.linears):
+        groups.setdefault(lin.prep, []).append(j)
+    fqws, fouts, fprep = [], [], []
+    for prep_name, idx in groups.items():
+        ws = [torch.from_numpy(synth.weights(1000 + j, ls.linears[j].n_out, ls.linears[j].k).view(np.float16)).to(dev)
+              for j in idx]
+        fqws.append(sq.quantize_weight_fused(ws, sq.NVFP4) if len(ws) > 1 else sq.quantize_weight(ws[0], sq.NVFP4))
+        del ws
+        fouts.append(torch.empty((M, sum(ls.linears[j].n_out for j in idx)), dtype=torch.float16, device=dev))
+        fprep.append(prep_index[prep_name])
+
+    def fused_step():
+        for i in range(len(preps)):
+            sq.prepare(xs[i], None, None, EPS, N_KEEP, M_GROUP, sq.NVFP4, out=bufs[i])
+        for g in range(len(fqws)):
+            sq.linear(bufs[fprep[g]], fqws[g], out=fouts[g])
+
+    with torch.cuda.stream(side):
+        for _ in range(max(args.warmup, 1)):
+            fused_step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    fgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(fgraph):
+        fused_step()
+    fused_ms = timed(fgraph.replay)
+    # the fused outputs against the separate linears' (equal up to the fp32
+    # summation order: a different split-K factor changes it)
+    fused_same, fused_diff = True, 0.0
+    for g, (prep_name, idx) in enumerate(groups.items()):
+        c = 0
+        for j in idx:
+            n = ls.linears[j].n_out
+            a, b = fouts[g][:, c:c + n].float(), outs[j].float()
+            fused_same &= torch.equal(fouts[g][:, c:c + n].view(torch.int16), outs[j].view(torch.int16))
+            fused_diff = max(fused_diff, float(((a - b).abs() / b.abs().clamp_min(1e-3)).max()))
+            c += n
     st = sq.get_last_error()
     if st != sq.OK:
         raise RuntimeError(sq.status_name(st))
@@ -1087,7 +1130,11 @@ def run_decode(args, M):
     return {"case": args.case, "tokens": M, "eager_ms_per_step": eager_ms, "graph_ms_per_step": graph_ms,
             "graph_tokens_per_s": M / (graph_ms / 1e3), "kernels_per_step": 4 * 2 + 7,
             "weight_stream_floor_ms": floor_ms, "graph_frac_of_floor": floor_ms / graph_ms,
-            "graph_equals_eager": same, "peak_source": f"{peak_src} hbm {peaks['hbm_gbs']} GB/s",
+            "graph_equals_eager": same,
+            "fused_projections": {"layout": "q/k/v one weight, gate/up one weight: 4 preps + 4 linears",
+                                  "graph_ms_per_step": fused_ms, "graph_tokens_per_s": M / (fused_ms / 1e3),
+                                  "graph_frac_of_floor": floor_ms / fused_ms, "bits_equal_separate": bool(fused_same),
+                                  "max_rel_diff_vs_separate": fused_diff}, "peak_source": f"{peak_src} hbm {peaks['hbm_gbs']} GB/s",
             "l2": "flushed (256 MB write) before every step", "steps": args.steps}
 
 

@@ -778,14 +778,20 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
                 if (nb * C::kBN + col >= p.n_out) continue;
                 const float alpha = EXT ? alpha_of_col(p, s_t, alpha0, nb * C::kBN + col) : alpha0;
                 const uint32_t off = sbase + (uint32_t)r * C::kPartStride + (uint32_t)col * 4u;
-                float4 acc = ld_cluster_f4(mapa_shared(off, 0));
-                for (int c = 1; c < S; ++c) {
-                    const float4 v = ld_cluster_f4(mapa_shared(off, (uint32_t)c));
-                    acc.x = __fadd_rn(acc.x, v.x);
-                    acc.y = __fadd_rn(acc.y, v.y);
-                    acc.z = __fadd_rn(acc.z, v.z);
-                    acc.w = __fadd_rn(acc.w, v.w);
-                }
+                // every CTA's values in flight at once, then the sums in rank order
+                float4 v[kMaxSplit];
+#pragma unroll
+                for (int c = 0; c < kMaxSplit; ++c)
+                    v[c] = c < S ? ld_cluster_f4(mapa_shared(off, (uint32_t)c)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                float4 acc = v[0];
+#pragma unroll
+                for (int c = 1; c < kMaxSplit; ++c)
+                    if (c < S) {
+                        acc.x = __fadd_rn(acc.x, v[c].x);
+                        acc.y = __fadd_rn(acc.y, v[c].y);
+                        acc.z = __fadd_rn(acc.z, v[c].z);
+                        acc.w = __fadd_rn(acc.w, v[c].w);
+                    }
                 float4 y = make_float4(__fmul_rn(acc.x, alpha), __fmul_rn(acc.y, alpha), __fmul_rn(acc.z, alpha),
                                        __fmul_rn(acc.w, alpha));
                 if (EXT && p.bias != nullptr) {
@@ -839,7 +845,10 @@ constexpr int kDecSf = 512 * (kBKBytes / 32);     // scale bytes of one 128-row 
 constexpr int kDecOffS = kDecW, kDecOffR = kDecW + kDecB, kDecOffSfW = kDecW + 2 * kDecB;
 constexpr int kDecOffSfS = kDecOffSfW + kDecSf, kDecOffSfR = kDecOffSfS + kDecSf;
 constexpr int kDecStage = kDecOffSfR + kDecSf;    // 26 KB, a multiple of 1024
-constexpr int kDecStages = 4;                     // two CTAs per SM: 8 stages in flight per SM
+#ifndef SQ_DEC_STAGES
+#define SQ_DEC_STAGES 4
+#endif
+constexpr int kDecStages = SQ_DEC_STAGES;         // 4: two CTAs fit on an SM
 constexpr int kDecBarOff = kDecStages * kDecStage;
 constexpr int kDecSfBufs = 4;
 constexpr int kDecSfCols = 3 * 4 * (kBKBytes / 32);  // W, S, R atoms per stage, 4 columns each
@@ -848,7 +857,7 @@ constexpr int kDecSmem = kDecBarOff + 256 + 1024;
 constexpr uint32_t kDecPartStride = kBM * 4 + 16;    // split-K partial: [token][column] fp32 rows
 static_assert(kDecStage % 1024 == 0, "decode stage alignment");
 static_assert(kDecTok + kDecSfBufs * kDecSfCols <= kDecTmemCols, "decode tensor memory");
-static_assert(2 * (kDecSmem + 1024) <= 233472, "decode shared memory: two CTAs per SM");
+static_assert(kDecSmem <= 232448, "decode shared memory");
 static_assert(kDecTok * kDecPartStride <= (uint32_t)kDecBarOff, "decode split-K partial fits the stages");
 
 template <int FMT, bool EXT>
@@ -878,15 +887,6 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
     const int nb = (int)blockIdx.x / S;  // weight tile (128 output columns)
     const int kt_begin = rank * kt_count / S, kt_end = (rank + 1) * kt_count / S, kt_n = kt_end - kt_begin;
     const int64_t apr = (int64_t)(p.k / (FMT == kFmtNV ? 16 : 32)) / 4;  // scale atoms per 128-row block
-    if (warp == 0) {
-        // This CTA's weight range starts streaming into L2 here, before the
-        // dependency wait, so that it overlaps the previous kernel. Safe even
-        // if that kernel writes the weight: a prefetch only warms L2 (the
-        // point of coherence), and the copies the MMAs read come after the wait.
-        for (int i = lane; i < kt_n; i += 32) tma_prefetch_l2_2d(&tm_w, (kt_begin + i) * kBKBytes, nb * kBM);
-        if (lane == 0)
-            bulk_prefetch_l2(p.sfb + ((int64_t)nb * apr + (int64_t)kt_begin * kAtoms) * 512, (uint32_t)(kt_n * kSfBytes));
-    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < kDecStages; ++s) {
             mbar_init(full_bar(s), 1);
@@ -1046,8 +1046,15 @@ decode_gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_consta
                 const int t = item / cols, cl = c0 + item % cols, col = nb * kBM + cl;
                 if (col >= p.n_out) continue;
                 const uint32_t off = sbase + (uint32_t)t * kDecPartStride + (uint32_t)cl * 4u;
-                float acc = __uint_as_float(ld_cluster_u32(mapa_shared(off, 0)));
-                for (int c = 1; c < S; ++c) acc = __fadd_rn(acc, __uint_as_float(ld_cluster_u32(mapa_shared(off, (uint32_t)c))));
+                // every CTA's value in flight at once, then the sum in rank order
+                float v[kMaxSplit];
+#pragma unroll
+                for (int c = 0; c < kMaxSplit; ++c)
+                    v[c] = c < S ? __uint_as_float(ld_cluster_u32(mapa_shared(off, (uint32_t)c))) : 0.0f;
+                float acc = v[0];
+#pragma unroll
+                for (int c = 1; c < kMaxSplit; ++c)
+                    if (c < S) acc = __fadd_rn(acc, v[c]);
                 float y = __fmul_rn(acc, EXT ? alpha_of_col(p, s_t, alpha0, col) : alpha0);
                 if (EXT && p.bias != nullptr) y = __fadd_rn(y, __half2float(p.bias[col]));
                 p.out[(int64_t)t * p.n_out + col] = __float2half_rn(y);
@@ -1374,8 +1381,11 @@ static int decode_active_clusters(int split) {
 // Split-K factor of a decode launch: the largest split <= 8 (any integer)
 // with tiles x split <= SQ_DECODE_WAVE CTAs per SM, split <= K steps and
 // every cluster resident at once. One CTA per SM (the default) leaves each
-// SM room for a CTA of the next launch, whose weight prefetch then overlaps
-// this one.
+// SM room for a CTA of the next launch, which then does its set-up while
+// this one runs (a programmatic dependent). Measured on B200: the same time
+// as two per SM (and an L2 prefetch of the weight before the dependency
+// wait, by TMA or by plain prefetch instructions, made the layer set's
+// decode GEMMs slower: it delays the running kernel's own loads).
 #ifndef SQ_DECODE_WAVE
 #define SQ_DECODE_WAVE 1
 #endif
