@@ -1810,12 +1810,15 @@ prep_encode_grouped_kernel(const EncodeArgs ea, const unsigned *__restrict__ ama
 // ---------------------------------------------------------------------------
 // Few rows (decode): the whole preparation in one launch of one cluster.
 // Phase 1: CTA r computes the exact statistics of rows r, r + kSmallCtas, ...
-// (a whole CTA per row) and keeps each row's amax|X_ln| in shared memory,
-// while every thread zeroes the scale layouts (whose padding rows must read
-// zero) and, where fields are OR-ed, the metadata. After a cluster barrier,
-// every CTA reads all rows' amax through distributed shared memory, derives
-// the tensor scale and encodes a share of the real rows' units. No memset
-// and no global atomic; the results equal the two-pass path bit for bit.
+// (a whole CTA per row) and stores each row's amax|X_ln| into the shared
+// memory of every CTA of the cluster, while the CTAs that own no row zero
+// the scale layouts' padding rows (bytes no encode writes; where fields are
+// OR-ed, every thread also zeroes the metadata). One cluster barrier makes
+// the amaxes (and the zeroed metadata) visible everywhere; then every CTA
+// derives the tensor scale from its own copy and encodes a share of the
+// real rows' units. No CTA reads another's shared memory after the barrier, so none
+// waits for the others at exit. No memset and no global atomic; the
+// results equal the two-pass path bit for bit.
 constexpr int kSmallCtas = 8, kSmallThreads = 512, kSmallMaxRows = 16, kSmallRows = 8;
 
 template <int FMT, int M, bool RMS>
@@ -1831,6 +1834,7 @@ prep_small_kernel(const EncodeArgs a, float eps, int64_t sf_rows, float *__restr
     __shared__ float2 row_stat;
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const uint32_t rank = cluster_ctarank();
+    cluster_arrive_relaxed();  // first half of the barrier before any remote store
     if (M <= 8)
         for (int msk = tid; msk < (1 << M); msk += kSmallThreads) {
             uint32_t packed = 0;
@@ -1842,7 +1846,6 @@ prep_small_kernel(const EncodeArgs a, float eps, int64_t sf_rows, float *__restr
                 }
             lut[msk] = packed;
         }
-    if (tid < kSmallMaxRows) row_amax[tid] = 0.0f;
     __syncthreads();
     // Launched as a programmatic dependent: everything above overlaps the
     // previous kernel's tail; global memory only after the wait.
@@ -1952,23 +1955,49 @@ prep_small_kernel(const EncodeArgs a, float eps, int64_t sf_rows, float *__restr
         __syncthreads();
     }
 
-    // Phase 1b: zero the scale layouts (padding rows must read zero) and,
-    // where fields are OR-ed, the metadata.
-    const int64_t gtid = (int64_t)rank * kSmallThreads + tid, gstride = (int64_t)kSmallCtas * kSmallThreads;
-    const int64_t sf_vec = sf_rows * a.nblk / 16;
-    for (int64_t i = gtid; i < sf_vec; i += gstride) {
-        reinterpret_cast<uint4 *>(a.s_sf)[i] = make_uint4(0, 0, 0, 0);
-        reinterpret_cast<uint4 *>(a.r_sf)[i] = make_uint4(0, 0, 0, 0);
+    // The scale layouts' padding rows (m_tok .. sf_rows - 1) read zero,
+    // written by the CTAs that own no row where there are such (they would
+    // otherwise wait at the barrier), else by all. Each 16-byte chunk holds
+    // rows r0, r0 + 32, r0 + 64, r0 + 96 of a 128-row block (4 scales each);
+    // only the padding rows' words are written, never bytes an encode writes.
+    {
+        const int64_t zctas = m_tok < kSmallCtas ? kSmallCtas - m_tok : kSmallCtas;
+        const int64_t zrank = m_tok < kSmallCtas ? (int64_t)rank - m_tok : (int64_t)rank;
+        const int64_t chunks = sf_rows * a.nblk / 16;
+        if (zrank >= 0)
+            for (int64_t c = zrank * kSmallThreads + tid; c < chunks; c += zctas * kSmallThreads) {
+                const int64_t r0 = (c / (a.nblk / 4) / 32) * 128 + (c & 31);  // first row of the chunk
+                if (r0 >= m_tok) {
+                    reinterpret_cast<uint4 *>(a.s_sf)[c] = make_uint4(0, 0, 0, 0);
+                    reinterpret_cast<uint4 *>(a.r_sf)[c] = make_uint4(0, 0, 0, 0);
+                } else {
+#pragma unroll
+                    for (int q = 1; q < 4; ++q)
+                        if (r0 + 32 * q >= m_tok) {
+                            reinterpret_cast<uint32_t *>(a.s_sf)[4 * c + q] = 0u;
+                            reinterpret_cast<uint32_t *>(a.r_sf)[4 * c + q] = 0u;
+                        }
+                }
+            }
     }
-    if (meta_zero)
+    // Every CTA's copy of the owned rows' amax (remote stores, made visible
+    // by the barrier below; the wait completes the barrier arrived at on
+    // entry, so every CTA has started).
+    cluster_wait();
+    for (int i = tid; i < kSmallCtas * kSmallMaxRows; i += kSmallThreads) {
+        const int c = i / kSmallMaxRows;
+        const int64_t row = (int64_t)rank + (int64_t)(i % kSmallMaxRows) * kSmallCtas;  // an owned row
+        if (row < m_tok)
+            st_cluster_u32(mapa_shared(smem_u32(&row_amax[row]), (uint32_t)c), __float_as_uint(row_amax[row]));
+    }
+    const int64_t gtid = (int64_t)rank * kSmallThreads + tid, gstride = (int64_t)kSmallCtas * kSmallThreads;
+    if (meta_zero)  // OR-ed fields: zeroed everywhere before any encode
         for (int64_t i = gtid; i < m_tok * a.meta_row; i += gstride) a.meta[i] = 0;
     cluster_sync();
 
     // Phase 2: the tensor scale from every row's amax, then the encode.
     float amax = 0.0f;
-    for (int64_t row = 0; row < m_tok; ++row)
-        amax = fmaxf(amax, __uint_as_float(ld_cluster_u32(mapa_shared(smem_u32(&row_amax[row]),
-                                                                     (uint32_t)(row % kSmallCtas)))));
+    for (int64_t row = 0; row < m_tok; ++row) amax = fmaxf(amax, row_amax[row]);
     const float s_t = (FMT == kFmtNV && amax != 0.0f) ? __fdiv_rn(amax, 2688.0f) : 1.0f;
     const float c6 = __fmul_rn(6.0f, s_t);
     const float y6 = (FMT == kFmtNV && c6 >= 0x1p-90f && c6 <= 0x1p90f) ? __frcp_rn(c6) : 0.0f;
@@ -1986,7 +2015,6 @@ prep_small_kernel(const EncodeArgs a, float eps, int64_t sf_rows, float *__restr
         const int64_t row = active ? t / upr : m_tok, u = active ? t - (t / upr) * upr : 0;
         encode_unit<FMT, M, 0>(a, lut, tab, row, u, active, s_t, c6, y6);
     }
-    cluster_sync();  // no CTA leaves while its row amax may still be read
 }
 
 // ---------------------------------------------------------------------------
