@@ -621,7 +621,8 @@ def config_summaries(args):
     a = argparse.Namespace(**vars(args))
     a.steps, a.warmup, a.outlier_frac = 10, 3, 0.01
     moe = run_moe(a, 4096)
-    out["qwen3_30b_a3b_moe_m4096"] = {k: moe[k] for k in ("tokens_per_s", "ms_per_step", "rows", "padded_rows", "ms")}
+    out["qwen3_30b_a3b_moe_m4096"] = {k: moe[k] for k in ("tokens_per_s", "ms_per_step", "rows", "padded_rows", "ms",
+                                                           "fused_gate_up")}
     out["qwen3_30b_a3b_moe_m4096"]["grouped_gemm_frac"] = moe["gemm_roofline"]["frac"]
     sw = run_sweep(a, [1, 16, 256, 2048, 16384])
     out["down_proj_decode_prefill_sweep"] = {
@@ -1296,6 +1297,30 @@ def run_moe(args, tokens):
         raise RuntimeError(sq.status_name(st))
     per = {name: statistics.median([e[i].elapsed_time(e[i + 1]) for e in ev]) for i, (name, _) in enumerate(ops)}
     step_ms = statistics.median([e[0].elapsed_time(e[-1]) for e in ev])
+
+    # gate and up stacked into one grouped weight per expert ([2 * inter,
+    # hidden], one tensor scale per expert): one grouped linear reads each
+    # expert's activation tiles once for both projections
+    w = h16(np.stack([np.concatenate([synth.weights(2000 + g, inter, hidden), synth.weights(3000 + g, inter, hidden)])
+                      for g in range(groups)]))
+    q_gu = sq.quantize_weight_grouped(w, fmt)
+    del w
+    o_gu = torch.empty((rows, 2 * inter), dtype=torch.float16, device=dev)
+    gu = lambda: sq.linear_grouped(g_tok, off, q_gu, rows, out=o_gu)
+    for _ in range(args.warmup):
+        flush.zero_()
+        gu()
+    evg = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for a, b in evg:
+        flush.zero_()
+        a.record(stream)
+        gu()
+        b.record(stream)
+    torch.cuda.synchronize()
+    gu_ms = statistics.median([a.elapsed_time(b) for a, b in evg])
+    st = sq.get_last_error()
+    if st != sq.OK:
+        raise RuntimeError(sq.status_name(st))
     lin = {"gate": (inter, hidden), "up": (inter, hidden), "down": (hidden, inter)}
     flops = {k: 2.0 * rows * no * kk * (1.0 + n / m) for k, (no, kk) in lin.items()}
     counts = np.diff(offsets)
@@ -1310,6 +1335,9 @@ def run_moe(args, tokens):
             "gemm_roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                               "frac": achieved / peak, "flops_algorithmic": sum(flops.values()),
                               "peak_source": peak_src + " (bf16 burst x 4)"},
+            "fused_gate_up": {"ms": gu_ms, "separate_ms": per["gate"] + per["up"],
+                              "frac": (flops["gate"] + flops["up"]) / (gu_ms / 1e3) / 1e12 / peak,
+                              "step_ms_with_fused": step_ms - per["gate"] - per["up"] + gu_ms},
             "gpu_launches_per_step": launches, "steps": args.steps,
             "warmup": args.warmup, "l2": "flushed (256 MB write) before every step"}
 
