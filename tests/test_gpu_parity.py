@@ -81,6 +81,38 @@ def test_prepare_many_short_rows_bit_exact(m_tok, k, fmt, norm):
     assert_prep_matches(sq.prep_export(p), op)
 
 
+@pytest.mark.parametrize("norm", ["layer", "rms"])
+@pytest.mark.parametrize("affine", [False, True])
+def test_certified_short_rows_and_exact_fallback(norm, affine):
+    """Rows of at most 2048 elements, enough of them (>= 8 per SM) that the
+    warp kernel takes its certified form (several rows per warp without the
+    affine parameters); rows the error bound cannot decide (constant rows, fp16
+    extremes, a large mean over a small spread, subnormals) spread over
+    different warps and CTAs are summed again exactly. Every row bit-exact."""
+    import sparsity_gemm_b200 as sq
+    m_tok, k = 3001, 768
+    x = synth.activations_student(940 + affine, m_tok, k)
+    for r in (0, 37, 1500, 2999):
+        x[r] = np.float16(3.5)
+    for r in (5, 1201):
+        x[r, ::2] = np.float16(65504.0)
+        x[r, 1::2] = np.float16(-65504.0)
+    for r in (9, 640, 3000):
+        x[r] = np.float16(1000.0)
+        x[r, ::7] = np.float16(1000.5)
+    x[11] = 0
+    x[13].view(np.uint16)[:] = np.arange(k, dtype=np.uint16) % 64 + 1  # fp16 subnormals
+    x[17, : k // 2] = np.float16(65504.0)
+    g, b = synth.ln_params(941, k) if affine else (None, None)
+    if norm == "rms":
+        b = None
+    op = oracle.prepare(x, g, b, 1e-5, 2, 4, 1, norm=norm)
+    p = sq.prepare(cuda16(x), None if g is None else cuda16(g), None if b is None else cuda16(b), 1e-5, 2, 4, 1,
+                   norm=norm)
+    assert_prep_matches(sq.prep_export(p), op)
+    assert sq.get_last_error() == sq.OK
+
+
 def test_maximum_k_statistics_at_the_lane_sum_bound():
     """K = SHARQ_K_MAX with rows enough for one warp per row: each lane adds
     2048 values, the bound of its 32-bit sums; rows of fp16 extremes (all
