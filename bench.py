@@ -624,6 +624,14 @@ def config_summaries(args):
     out["qwen3_30b_a3b_moe_m4096"] = {k: moe[k] for k in ("tokens_per_s", "ms_per_step", "rows", "padded_rows", "ms",
                                                            "fused_gate_up")}
     out["qwen3_30b_a3b_moe_m4096"]["grouped_gemm_frac"] = moe["gemm_roofline"]["frac"]
+    dec = run_decode(a, 1)
+    out["llama31_8b_decode_m1"] = {
+        "graph_us_per_step": dec["graph_ms_per_step"] * 1e3,
+        "fused_projections_graph_us_per_step": dec["fused_projections"]["graph_ms_per_step"] * 1e3,
+        "weight_stream_floor_us": dec["weight_stream_floor_ms"] * 1e3,
+        "graph_frac_of_floor": dec["graph_frac_of_floor"],
+        "fused_frac_of_floor": dec["fused_projections"]["graph_frac_of_floor"],
+        "launch": "CUDA graph replay, 4 preps + 7 linears (fused: 4 + 4), L2 flushed before every step"}
     sw = run_sweep(a, [1, 16, 256, 2048, 16384])
     out["down_proj_decode_prefill_sweep"] = {
         "crossover_M": sw["crossover_M"],
