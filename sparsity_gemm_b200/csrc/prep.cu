@@ -28,9 +28,12 @@
 
 namespace sq {
 
-// Resident encode CTAs per SM the register allocation must allow.
+// Resident encode CTAs per SM the register allocation must allow. Measured
+// on B200 (K = 14336 / 3584 / 4096 preparations): 2 (80 registers) 202.8 /
+// 36.9 / 69.6 us, 3 (71) 204.8 / 38.8 / 69.7, 4 (64, a few bytes spilled)
+// 204.9 / 38.9 / 69.6: the encode is issue-bound, not short of warps.
 #ifndef SQ_ENCODE_MIN_CTAS
-#define SQ_ENCODE_MIN_CTAS 3
+#define SQ_ENCODE_MIN_CTAS 2
 #endif
 constexpr int kStatsThreads = 256;
 constexpr int kEncodeThreads = 256;
