@@ -828,8 +828,9 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_as, const __grid_constan
 // is 128 x 16 per K slice and the launch streams the weight. One CTA per
 // (128-row weight tile, K range); K ranges of a tile go to the CTAs of a
 // cluster, which reduce their fp32 partials through distributed shared
-// memory as dual_gemm_kernel's split-K does; two CTAs fit on an SM, so that a
-// single wave holds up to 2 x SMs CTAs. Per stage: the W tile (A), the
+// memory as dual_gemm_kernel's split-K does. Two CTAs fit on an SM: one of
+// this launch and one of the next, which does its set-up as a programmatic
+// dependent while this one runs. Per stage: the W tile (A), the
 // backbone and residual tiles of the tokens (B, 16 rows, zero-filled past
 // m_tok), the W scale atoms (A scales) and the activations' first scale
 // atoms (B scales: the block-scaled MMA reads B scales in the layout of a
@@ -848,7 +849,7 @@ constexpr int kDecStage = kDecOffSfR + kDecSf;    // 26 KB, a multiple of 1024
 #ifndef SQ_DEC_STAGES
 #define SQ_DEC_STAGES 4
 #endif
-constexpr int kDecStages = SQ_DEC_STAGES;         // 4: two CTAs fit on an SM
+constexpr int kDecStages = SQ_DEC_STAGES;         // 4: two CTAs fit on an SM (8 measured no faster)
 constexpr int kDecBarOff = kDecStages * kDecStage;
 constexpr int kDecSfBufs = 4;
 constexpr int kDecSfCols = 3 * 4 * (kBKBytes / 32);  // W, S, R atoms per stage, 4 columns each
