@@ -35,6 +35,7 @@ CASES = [  # (m_tok, n_out, k, fmt, n, m)
     (3, 128, 512, 1, 4, 8),
     (9, 14336, 4096, 0, 2, 4),   # 112 tiles: a split of 2
     (12, 992, 2048, 1, 3, 8),
+    (2, 32, 512, 0, 2, 4),       # a weight smaller than one 128-row tile
 ]
 
 
@@ -51,9 +52,11 @@ def test_decode_linear_within_tolerance(sq, m_tok, n_out, k, fmt, n, m):
     assert sq.get_last_error() == sq.OK
 
 
-@pytest.mark.parametrize("fmt", [0, 1])
-def test_decode_fused_segments_with_bias(sq, fmt):
-    rows, k, m_tok = [512, 128, 128], 2048, 4
+@pytest.mark.parametrize("fmt,rows", [(0, [512, 128, 128]), (1, [512, 128, 128]), (0, [96, 160, 32])])
+def test_decode_fused_segments_with_bias(sq, fmt, rows):
+    """Fused segments with a bias; the last case puts segment boundaries
+    inside 128-column W tiles (96, 256)."""
+    k, m_tok = 2048, 4
     ws = [synth.weights(810 + i, r, k) * np.float16(1 + i) for i, r in enumerate(rows)]
     x = synth.activations_student(820, m_tok, k)
     b = synth.to_fp16(synth.normal(821, 0, sum(rows)) * 2.0)
