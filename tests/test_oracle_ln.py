@@ -1,6 +1,7 @@
 """Pins for the oracle's LayerNorm: exact rational statistics, a library
 LayerNorm in fp64, closed-form special rows, and order independence."""
 import decimal
+import math
 from fractions import Fraction
 
 import numpy as np
@@ -51,6 +52,45 @@ def test_stats_match_exact_rationals(orc, eps):
             mean, rs = _exact_stats(x[r], eps32)
             assert abs(float(mu[r]) - float(mean)) <= _ulp32(float(mean)) + 1e-45
             assert abs(float(rstd[r]) - rs) <= 1.5 * _ulp32(rs)
+
+
+def _reading_stats(row16: np.ndarray, eps32: np.float32, norm: str):
+    """The statistics' rounding sequence as the library documents it (exact
+    integer sums of a = x 2^24; then each step one IEEE binary64 operation,
+    as Python floats are, and one rounding to binary32):
+      LayerNorm: mu = RN32(RN64(S1) / (K 2^24)),
+                 rstd = RN32(1 / sqrt(RN64(K S2 - S1^2) / (K^2 2^48) + eps));
+      RMSNorm:   rstd = RN32(1 / sqrt(RN64(S2) / (K 2^48) + eps)), mu = 0."""
+    a = [int(Fraction(float(v)) * 2 ** 24) for v in row16.astype(np.float64)]
+    k = len(a)
+    s1 = sum(a)
+    s2 = sum(v * v for v in a)
+    if norm == "layer":
+        mu = np.float32(float(s1) / float(k * 2 ** 24))
+        var = float(k * s2 - s1 * s1) / float(k * k * 2 ** 48)
+    else:
+        mu = np.float32(0.0)
+        var = float(s2) / float(k * 2 ** 48)
+    return mu, np.float32(1.0 / math.sqrt(var + float(eps32)))
+
+
+@pytest.mark.parametrize("norm", ["layer", "rms"])
+@pytest.mark.parametrize("eps", [1e-5, 1e-6])
+def test_stats_bit_exact_to_the_documented_rounding_sequence(orc, norm, eps):
+    """Bit for bit: the oracle's statistics equal the documented sequence
+    recomputed here with Python integers and IEEE binary64 operations (the
+    rational pin above bounds that sequence against the exact values)."""
+    eps32 = np.float32(eps)
+    rows = list(_rows()) + [synth.activations_student(7, 5, 14336)]
+    big = np.full((1, 16384), np.float16(65504.0))
+    big[0, 1::3] = -65504.0
+    rows.append(big)
+    for x in rows:
+        mu, rstd = (orc.ln_stats if norm == "layer" else orc.rms_stats)(x, eps)
+        for r in range(x.shape[0]):
+            want_mu, want_rstd = _reading_stats(x[r], eps32, norm)
+            assert np.float32(mu[r]).view(np.uint32) == want_mu.view(np.uint32), (norm, r, mu[r], want_mu)
+            assert np.float32(rstd[r]).view(np.uint32) == want_rstd.view(np.uint32), (norm, r, rstd[r], want_rstd)
 
 
 def test_large_row_exercises_wide_sums(orc):
